@@ -1,0 +1,157 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4: NVFP4 block-scaled quantisation and matrix multiplication
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation (reference pages: "The Moment the Zeros Disappeared", section "The Subject
+ * Message"; "The Art of Reading the Manual", section "The Message", the mm_fp4 signature):
+ *
+ *     out[m, n] = bf16( alpha * sum_k deq(A)[m, k] * deq(B)[n, k] )
+ *     deq(X)[r, k] = e2m1(X[r, k]) * e4m3(sfX[r, k / 16])
+ *
+ * Data formats (all row-major, "TN": both operands contiguous along K):
+ *   - packed operand X[rows, K/2] uint8: element k of a row sits in byte k/2, even k in the
+ *     low nibble; a nibble is an e2m1 code (sign, 2-bit exponent, 1-bit mantissa;
+ *     magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6).
+ *   - scales sfX[rows, K/16] uint8: one float8_e4m3fn per 16 consecutive K elements
+ *     (block_size = 16, fixed), linear layout, row stride K/16 bytes.
+ *   - B is stored N x K/2 (the pages' "(K//2, N) column-major" view of the same bytes).
+ *   - alpha: fp32 on the device (a required argument, never implied), out: bf16 [M, N]
+ *     row-major, caller-allocated (also required).
+ *
+ * Conventions shared by every call:
+ *   - The caller owns all memory. Except where a call says otherwise, pointers are device
+ *     pointers and must be 16-byte aligned. The library allocates no device memory; it
+ *     keeps only a per-process cache of TMA descriptors and device attributes.
+ *   - Calls are asynchronous on the given stream (0 = legacy default stream). The returned
+ *     status covers argument checks and launch errors only. A kernel that gives up on a
+ *     bounded internal wait records NVFP4_ERR_TIMEOUT in a device error word that
+ *     nvfp4_last_device_error() reads.
+ *   - No fallback: on a device other than compute capability 10.0 every compute call
+ *     returns NVFP4_ERR_ARCH; there is no CPU or alternative-backend path.
+ *   - Shapes: K % 256 == 0, N % 8 == 0, M >= 0 arbitrary (M == 0 is a no-op), all sizes
+ *     below 2^31 elements per dimension.
+ *   - Thread safety: calls may be made from several host threads.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum value */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 256 != 0, N % 8 != 0, too large, ... */
+    NVFP4_ERR_MISALIGNED = 3,         /* a pointer or leading dimension breaks 16-byte alignment */
+    NVFP4_ERR_ARCH = 4,               /* device is not sm_100 (B200 / B100 class) */
+    NVFP4_ERR_CUDA = 5,               /* a CUDA runtime or driver call failed */
+    NVFP4_ERR_TIMEOUT = 6,            /* a kernel gave up on a bounded wait (device error word) */
+    NVFP4_ERR_WORKSPACE = 7           /* workspace given but smaller than required */
+} nvfp4_status;
+
+typedef enum {
+    NVFP4_IN_F32 = 0,
+    NVFP4_IN_BF16 = 1
+} nvfp4_in_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* nvfp4_status_string(nvfp4_status s);
+
+/*
+ * Per-tensor global scale: gs_out[0] = 2688 / max|x| in fp32 (2688 = 448 * 6, so the
+ * largest block scale of the tensor lands on e4m3's maximum 448), or 1 if x is all zero.
+ * x: device, numel elements of the given dtype, 16-byte aligned. gs_out: device, one
+ * float, used as the reduction accumulator while the call runs (its old value is
+ * ignored). Three stream operations (clear, reduce, finalise). numel == 0 gives 1.
+ */
+nvfp4_status nvfp4_global_scale(const void* x, nvfp4_in_dtype dtype, int64_t numel,
+                                float* gs_out, cudaStream_t stream);
+
+/*
+ * Two-level NVFP4 quantisation of x[rows, K] (row stride ld_x elements) with the global
+ * scale gs (device, one float, normally from nvfp4_global_scale). For every row and every
+ * 16-element block j, in fp32 with round-to-nearest-even and no fused operations:
+ *     amax = max |x|;  s = e4m3_rn_satfinite((amax / 6) * gs);  r = s ? gs / s : 0
+ *     code_k = e2m1_rn_satfinite(x_k * r)    (ties to the even code; sign kept, so a
+ *                                             negative value that rounds to 0 gives 0x8)
+ * Outputs: q[rows, K/2] (device) and sf[rows, K/16] (device, e4m3 bytes), both
+ * caller-allocated. Requires K % 16 == 0 here (the GEMMs require K % 256 == 0),
+ * ld_x * sizeof(dtype) % 16 == 0, x, q 16-byte aligned.
+ */
+nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
+                            int64_t ld_x, const float* gs, uint8_t* q, uint8_t* sf,
+                            cudaStream_t stream);
+
+/*
+ * GEMM scale from the two global scales: alpha[i] = 1 / (gs_a[0] * gs_b[i]) in fp32,
+ * for i < n (n = 1 for a single GEMM, n = experts for the grouped GEMM). All device.
+ */
+nvfp4_status nvfp4_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
+                         cudaStream_t stream);
+
+/*
+ * Workspace bytes nvfp4_gemm uses for split-K on this device for this shape (0 when the
+ * shape runs without split-K). Returns 0 if no CUDA device is usable.
+ */
+size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Block-scaled NVFP4 GEMM: out[M, N] = bf16(alpha[0] * sum_k deq(A)[m, k] deq(B)[n, k]).
+ * A[M, K/2], sfA[M, K/16], B[N, K/2], sfB[N, K/16], alpha[1], out[M, N]: device.
+ * ws / ws_bytes: optional split-K workspace (device). ws == NULL runs without split-K.
+ * A non-NULL ws must be at least nvfp4_gemm_workspace_size(M, N, K) bytes
+ * (NVFP4_ERR_WORKSPACE otherwise), 256-byte aligned, and zero-filled before its first
+ * use; every completed call leaves its tile counters at zero again, so one zero fill
+ * serves any number of calls. Calls that share a workspace must not overlap in time.
+ * Split-K partial sums are reduced in a fixed order, so results are deterministic.
+ */
+nvfp4_status nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                        const uint8_t* sfB, const float* alpha, void* out,
+                        int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
+                        cudaStream_t stream);
+
+/*
+ * Grouped (mixture-of-experts) NVFP4 GEMM ("When a Benchmark Crashes", section "Why This
+ * Message Was Written": 256 experts, 8 active per token). Rows of A are sorted by expert;
+ * expert e owns rows [expert_offsets[e], expert_offsets[e+1]) and computes
+ *     out[r, n] = bf16(alpha[e] * sum_k deq(A)[r, k] deq(B[e])[n, k]).
+ * A[total_rows, K/2], sfA[total_rows, K/16], B[E, N, K/2], sfB[E, N, K/16], alpha[E],
+ * expert_offsets[E + 1] (int32, non-decreasing, offsets[0] == 0, offsets[E] <= total_rows),
+ * out[total_rows, N]: all device. The offsets are read on the device (no host sync);
+ * empty experts are allowed; output rows past offsets[E] are not written.
+ * ws / ws_bytes: reserved, pass NULL / 0 (nvfp4_grouped_gemm_workspace_size returns 0).
+ */
+size_t nvfp4_grouped_gemm_workspace_size(int32_t E, int64_t total_rows, int64_t N, int64_t K);
+
+nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                                const uint8_t* sfB, const float* alpha,
+                                const int32_t* expert_offsets, int32_t E, int64_t total_rows,
+                                int64_t N, int64_t K, void* out, void* ws, size_t ws_bytes,
+                                cudaStream_t stream);
+
+/*
+ * Elementwise conversions used by the quantiser, exposed so that they can be checked
+ * exhaustively: out[i] = e4m3_rn_satfinite(x[i]) (one byte), or e2m1_rn_satfinite(x[i])
+ * (one code 0..15 per byte). x, out: device, n elements, no alignment requirement.
+ */
+nvfp4_status nvfp4_round_e4m3(const float* x, int64_t n, uint8_t* out, cudaStream_t stream);
+nvfp4_status nvfp4_round_e2m1(const float* x, int64_t n, uint8_t* out, cudaStream_t stream);
+
+/*
+ * Reads and clears the current device's error word. Synchronises `stream` first.
+ * Returns NVFP4_OK if no kernel recorded an error since the last call, NVFP4_ERR_TIMEOUT
+ * if one gave up on a bounded wait, NVFP4_ERR_CUDA if the read itself failed.
+ * *where_out (optional, host) receives the raw code: the wait that gave up.
+ */
+nvfp4_status nvfp4_last_device_error(cudaStream_t stream, uint32_t* where_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

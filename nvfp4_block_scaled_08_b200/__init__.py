@@ -1,0 +1,227 @@
+"""nvfp4_block_scaled_08_b200 -- NVFP4 block-scaled matrix multiplication for B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libnvfp4.so`` (``include/nvfp4.h``). Functions take
+torch CUDA tensors for memory and the current CUDA stream, and only marshal pointers and
+sizes: every step of quantisation and matrix multiplication runs in the library's CUDA
+kernels. There is no CPU or alternative-backend path; if the library cannot be built or
+loaded, or the device is not sm_100, calls raise.
+
+    gs  = global_scale(x)                 # 2688 / max|x|  (fp32, device)
+    q, sf = quantize(x, gs)               # packed e2m1 [R, K/2], e4m3 scales [R, K/16]
+    al  = alpha(gs_a, gs_b)               # 1 / (gs_a * gs_b)
+    gemm(Aq, sfA, Bq, sfB, al, out)       # out[M, N] bf16
+    grouped_gemm(Aq, sfA, Bq, sfB, al_e, offsets, out)   # per-expert products
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import _build
+
+__all__ = [
+    "Nvfp4Error", "load", "global_scale", "quantize", "alpha", "gemm", "gemm_workspace_size",
+    "make_workspace", "grouped_gemm", "round_e4m3", "round_e2m1", "last_device_error",
+    "STATUS",
+]
+
+STATUS = {
+    0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_UNSUPPORTED_SHAPE",
+    3: "NVFP4_ERR_MISALIGNED", 4: "NVFP4_ERR_ARCH", 5: "NVFP4_ERR_CUDA",
+    6: "NVFP4_ERR_TIMEOUT", 7: "NVFP4_ERR_WORKSPACE",
+}
+IN_F32, IN_BF16 = 0, 1
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn}: {message}")
+        self.status = status
+
+
+_lib = None
+_lock = threading.Lock()
+
+# exported symbol -> (restype, argtypes)
+_P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+SIGNATURES = {
+    "nvfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "nvfp4_global_scale": (ctypes.c_int, [_P, ctypes.c_int, _I64, _P, _P]),
+    "nvfp4_quantize": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _P, _P]),
+    "nvfp4_alpha": (ctypes.c_int, [_P, _P, _I32, _P, _P]),
+    "nvfp4_gemm_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "nvfp4_grouped_gemm_workspace_size": (_SZ, [_I32, _I64, _I64, _I64]),
+    "nvfp4_grouped_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
+                                          _SZ, _P]),
+    "nvfp4_round_e4m3": (ctypes.c_int, [_P, _I64, _P, _P]),
+    "nvfp4_round_e2m1": (ctypes.c_int, [_P, _I64, _P, _P]),
+    "nvfp4_last_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+}
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def load(build_if_needed: bool = True) -> ctypes.CDLL:
+    """Load libnvfp4.so (compiling it with nvcc first if it is missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if build_if_needed:
+            _build.build()
+        if not os.path.exists(_build.LIB_PATH):
+            raise Nvfp4Error("load", -1, f"CUDA library not found at {_build.LIB_PATH}")
+        lib = ctypes.CDLL(_build.LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        msg = load().nvfp4_status_string(status).decode()
+        raise Nvfp4Error(fn, status, msg)
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _dtype_code(x: torch.Tensor) -> int:
+    if x.dtype == torch.float32:
+        return IN_F32
+    if x.dtype == torch.bfloat16:
+        return IN_BF16
+    raise ValueError("input must be float32 or bfloat16")
+
+
+# ------------------------------------------------------------------ quantisation
+
+def global_scale(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """gs = 2688 / max|x| (or 1 for an all-zero x) as a 1-element fp32 device tensor."""
+    _dev(x, "x")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check("nvfp4_global_scale", load().nvfp4_global_scale(
+        _ptr(x), _dtype_code(x), x.numel(), _ptr(out), _stream(stream)))
+    return out
+
+
+def quantize(x: torch.Tensor, gs: torch.Tensor, q: torch.Tensor | None = None,
+             sf: torch.Tensor | None = None, stream=None):
+    """NVFP4 quantisation of x[rows, K] (fp32 or bf16, unit column stride).
+
+    Returns (q uint8 [rows, K/2], sf uint8 [rows, K/16]) on x's device."""
+    _dev(x, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    rows, K = x.shape
+    if q is None:
+        q = torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(rows, K // 16, dtype=torch.uint8, device=x.device)
+    _check("nvfp4_quantize", load().nvfp4_quantize(
+        _ptr(x), _dtype_code(x), rows, K, x.stride(0), _ptr(gs), _ptr(q), _ptr(sf),
+        _stream(stream)))
+    return q, sf
+
+
+def alpha(gs_a: torch.Tensor, gs_b: torch.Tensor, out: torch.Tensor | None = None,
+          stream=None) -> torch.Tensor:
+    """alpha[i] = 1 / (gs_a[0] * gs_b[i]) (fp32, device)."""
+    n = gs_b.numel()
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=gs_b.device)
+    _check("nvfp4_alpha", load().nvfp4_alpha(_ptr(gs_a), _ptr(gs_b), n, _ptr(out),
+                                             _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ products
+
+def gemm_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load().nvfp4_gemm_workspace_size(M, N, K))
+
+
+def make_workspace(M: int, N: int, K: int, device="cuda") -> torch.Tensor | None:
+    """A zero-filled split-K workspace for this shape (None when none is needed)."""
+    n = gemm_workspace_size(M, N, K)
+    if n == 0:
+        return None
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """out[M, N] = bf16(alpha * sum_k deq(A)[m,k] deq(B)[n,k]).
+
+    Aq [M, K/2] uint8, sfA [M, K/16] uint8, Bq [N, K/2], sfB [N, K/16], alpha_t fp32 [1];
+    out bf16 [M, N] (allocated if None); workspace: zero-filled uint8 tensor of
+    gemm_workspace_size(M, N, K) bytes or None (no split-K)."""
+    M, K = Aq.shape[0], Aq.shape[1] * 2
+    N = Bq.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=Aq.device)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    _check("nvfp4_gemm", load().nvfp4_gemm(
+        _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alpha_t), _ptr(out), M, N, K,
+        ws_ptr, ws_bytes, _stream(stream)))
+    return out
+
+
+def grouped_gemm(Aq, sfA, Bq, sfB, alphas, offsets, out=None, stream=None) -> torch.Tensor:
+    """Per expert e: out[r] = bf16(alpha[e] * deq(A)[r] . deq(B[e])^T) for rows r in
+    [offsets[e], offsets[e+1]). Bq [E, N, K/2], sfB [E, N, K/16], offsets int32 [E+1]."""
+    rows, K = Aq.shape[0], Aq.shape[1] * 2
+    E, N = Bq.shape[0], Bq.shape[1]
+    if out is None:
+        out = torch.empty(rows, N, dtype=torch.bfloat16, device=Aq.device)
+    _check("nvfp4_grouped_gemm", load().nvfp4_grouped_gemm(
+        _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alphas), _ptr(offsets), E, rows, N, K,
+        _ptr(out), None, 0, _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ conversions and errors
+
+def round_e4m3(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    _check("nvfp4_round_e4m3", load().nvfp4_round_e4m3(_ptr(x), x.numel(), _ptr(out),
+                                                       _stream(stream)))
+    return out
+
+
+def round_e2m1(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    _check("nvfp4_round_e2m1", load().nvfp4_round_e2m1(_ptr(x), x.numel(), _ptr(out),
+                                                       _stream(stream)))
+    return out
+
+
+def last_device_error(stream=None) -> tuple[int, int]:
+    """(status, code) of the device error word, which is then cleared; synchronises."""
+    where = ctypes.c_uint32(0)
+    st = load().nvfp4_last_device_error(_stream(stream), ctypes.byref(where))
+    return int(st), int(where.value)

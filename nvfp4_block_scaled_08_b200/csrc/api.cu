@@ -1,0 +1,269 @@
+// api.cu -- the extern "C" boundary of libnvfp4 (declared in include/nvfp4.h): argument
+// checks, device checks, the device error word, and dispatch to the kernels.
+//
+// Interface lessons carried over from the reference pages: alpha and out are explicit,
+// required arguments ("The Moment the Zeros Disappeared", section "What This Means": a
+// call without them failed with a TypeError); block_size is fixed at 16 ("The Art of
+// Reading the Manual", section "Assumptions and Their Consequences"); B is N x K/2
+// ("The Moment the Zeros Disappeared", section "The Subject Message", item 3); bad shapes
+// are rejected with a clear status (the same page's "K dimension mismatch"); and there is
+// no automatic fallback to another backend ("The Moment the Zeros Disappeared", section
+// "What This Means": the auto backend's fallback chain failed).
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/nvfp4.h"
+#include "internal.h"
+
+namespace {
+
+__device__ unsigned g_nvfp4_error_word;
+
+struct DeviceInfo {
+    bool init = false;
+    bool arch_ok = false;
+    int num_sms = 0;
+    unsigned* err_word = nullptr;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+nvfp4_status current_device(DeviceInfo* out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.init) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return NVFP4_ERR_CUDA;
+        }
+        d.arch_ok = (major == 10 && minor == 0);
+        d.num_sms = sms;
+        void* p = nullptr;
+        if (d.arch_ok) {
+            if (cudaGetSymbolAddress(&p, g_nvfp4_error_word) != cudaSuccess) {
+                cudaGetLastError();
+                return NVFP4_ERR_CUDA;
+            }
+        }
+        d.err_word = static_cast<unsigned*>(p);
+        d.init = true;
+    }
+    *out = d;
+    return d.arch_ok ? NVFP4_OK : NVFP4_ERR_ARCH;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+nvfp4_status from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess) return NVFP4_OK;
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+}
+
+// Shape and pointer checks shared by the GEMMs; no CUDA call.
+nvfp4_status check_gemm_common(const void* A, const void* sfA, const void* B, const void* sfB,
+                               const void* alpha, const void* out, int64_t N, int64_t K)
+{
+    if (!A || !sfA || !B || !sfB || !alpha || !out) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 256 != 0 || K > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (N % 8 != 0 || N > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(A) || !aligned16(sfA) || !aligned16(B) || !aligned16(sfB) || !aligned16(out))
+        return NVFP4_ERR_MISALIGNED;
+    if (!aligned4(alpha)) return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_string(nvfp4_status s)
+{
+    switch (s) {
+        case NVFP4_OK: return "NVFP4_OK";
+        case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG: null pointer, negative size or bad enum value";
+        case NVFP4_ERR_UNSUPPORTED_SHAPE: return "NVFP4_ERR_UNSUPPORTED_SHAPE: need K % 256 == 0, N % 8 == 0, dims < 2^31";
+        case NVFP4_ERR_MISALIGNED: return "NVFP4_ERR_MISALIGNED: pointers and row strides must be 16-byte aligned";
+        case NVFP4_ERR_ARCH: return "NVFP4_ERR_ARCH: device is not compute capability 10.0 (sm_100a)";
+        case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA: a CUDA runtime or driver call failed";
+        case NVFP4_ERR_TIMEOUT: return "NVFP4_ERR_TIMEOUT: a kernel gave up on a bounded wait";
+        case NVFP4_ERR_WORKSPACE: return "NVFP4_ERR_WORKSPACE: workspace smaller than nvfp4_gemm_workspace_size()";
+    }
+    return "NVFP4_ERR_UNKNOWN";
+}
+
+nvfp4_status nvfp4_global_scale(const void* x, nvfp4_in_dtype dtype, int64_t numel, float* gs_out,
+                                cudaStream_t stream)
+{
+    if (!gs_out || numel < 0 || (numel > 0 && !x)) return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_F32 && dtype != NVFP4_IN_BF16) return NVFP4_ERR_INVALID_ARG;
+    if ((numel > 0 && !aligned16(x)) || !aligned4(gs_out)) return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_global_scale(x, dtype == NVFP4_IN_BF16, numel, gs_out, stream,
+                                                d.num_sms));
+}
+
+nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
+                            int64_t ld_x, const float* gs, uint8_t* q, uint8_t* sf,
+                            cudaStream_t stream)
+{
+    if (rows < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_F32 && dtype != NVFP4_IN_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0 || K == 0) return NVFP4_OK;
+    if (!x || !gs || !q || !sf) return NVFP4_ERR_INVALID_ARG;
+    if (K % 16 != 0 || K > kMaxDim || rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld_x < K) return NVFP4_ERR_INVALID_ARG;
+    const int64_t esz = dtype == NVFP4_IN_BF16 ? 2 : 4;
+    if (!aligned16(x) || (ld_x * esz) % 16 != 0 || !aligned16(q) || !aligned4(gs))
+        return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_quantize(x, dtype == NVFP4_IN_BF16, rows, K, ld_x, gs, q, sf,
+                                            stream, d.num_sms));
+}
+
+nvfp4_status nvfp4_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
+                         cudaStream_t stream)
+{
+    if (n < 0) return NVFP4_ERR_INVALID_ARG;
+    if (n == 0) return NVFP4_OK;
+    if (!gs_a || !gs_b || !alpha) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned4(gs_a) || !aligned4(gs_b) || !aligned4(alpha)) return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_alpha(gs_a, gs_b, n, alpha, stream));
+}
+
+size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || K % 256 != 0) return 0;
+    DeviceInfo d;
+    if (current_device(&d) != NVFP4_OK) return 0;
+    return nvfp4::plan_gemm(M, N, K, true, d.num_sms).ws_bytes;
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                        const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
+                        size_t ws_bytes, cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (M > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    nvfp4_status st = check_gemm_common(A, sfA, B, sfB, alpha, out, N, K);
+    if (st != NVFP4_OK) return st;
+    if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    nvfp4::GemmPlan plan = nvfp4::plan_gemm(M, N, K, ws != nullptr, d.num_sms);
+    if (plan.splits > 1 && ws_bytes < plan.ws_bytes) return NVFP4_ERR_WORKSPACE;
+    nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0, ws, d.err_word};
+    bool enc_failed = false;
+    cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
+    if (enc_failed) return NVFP4_ERR_CUDA;
+    return from_cuda(e);
+}
+
+size_t nvfp4_grouped_gemm_workspace_size(int32_t E, int64_t total_rows, int64_t N, int64_t K)
+{
+    (void)E; (void)total_rows; (void)N; (void)K;
+    return 0;
+}
+
+nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                                const uint8_t* sfB, const float* alpha,
+                                const int32_t* expert_offsets, int32_t E, int64_t total_rows,
+                                int64_t N, int64_t K, void* out, void* ws, size_t ws_bytes,
+                                cudaStream_t stream)
+{
+    (void)ws; (void)ws_bytes;
+    if (E < 0 || total_rows < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (E == 0 || total_rows == 0 || N == 0) return NVFP4_OK;
+    if (E > nvfp4::kMaxExperts) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (total_rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!expert_offsets) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_gemm_common(A, sfA, B, sfB, alpha, out, N, K);
+    if (st != NVFP4_OK) return st;
+    if (!aligned4(expert_offsets)) return NVFP4_ERR_MISALIGNED;
+    if (static_cast<int64_t>(E) * N > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    DeviceInfo d;
+    st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    nvfp4::GemmPlan plan = nvfp4::plan_grouped(E, total_rows, N, K, d.num_sms);
+    nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, 0, N, K, expert_offsets, E, total_rows,
+                        nullptr, d.err_word};
+    bool enc_failed = false;
+    cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
+    if (enc_failed) return NVFP4_ERR_CUDA;
+    return from_cuda(e);
+}
+
+nvfp4_status nvfp4_round_e4m3(const float* x, int64_t n, uint8_t* out, cudaStream_t stream)
+{
+    if (n < 0) return NVFP4_ERR_INVALID_ARG;
+    if (n == 0) return NVFP4_OK;
+    if (!x || !out) return NVFP4_ERR_INVALID_ARG;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_round(x, n, out, false, stream, d.num_sms));
+}
+
+nvfp4_status nvfp4_round_e2m1(const float* x, int64_t n, uint8_t* out, cudaStream_t stream)
+{
+    if (n < 0) return NVFP4_ERR_INVALID_ARG;
+    if (n == 0) return NVFP4_OK;
+    if (!x || !out) return NVFP4_ERR_INVALID_ARG;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_round(x, n, out, true, stream, d.num_sms));
+}
+
+nvfp4_status nvfp4_last_device_error(cudaStream_t stream, uint32_t* where_out)
+{
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_nvfp4_error_word, sizeof(v)) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    if (where_out) *where_out = v;
+    if (v == 0) return NVFP4_OK;
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_nvfp4_error_word, &zero, sizeof(zero)) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_ERR_TIMEOUT;
+}
+
+}  // extern "C"

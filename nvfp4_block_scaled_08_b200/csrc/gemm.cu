@@ -1,0 +1,262 @@
+// gemm.cu -- host side of the NVFP4 GEMMs: tile planning, TMA descriptor encoding (with a
+// per-process cache) and the launch of the persistent sm_100a kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <array>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+
+#include "gemm_kernel.cuh"
+#include "internal.h"
+
+namespace nvfp4 {
+
+// ------------------------------------------------------------------ planning
+
+static int env_int(const char* name, int dflt)
+{
+    const char* v = std::getenv(name);
+    if (!v || !*v) return dflt;
+    return std::atoi(v);
+}
+
+static int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+// Tiling for out[M, N] = A[M, K] x B[N, K]^T on `num_sms` SMs.
+//  * M <= 64: weights fill the 128-row MMA operand (swap), tokens are an MMA N of 16-64.
+//  * otherwise: 128-row token tiles x 128- or 256-row weight tiles, whichever finishes in
+//    fewer tile-waves (wider tiles cost ~2x per tile but move less data per FLOP).
+//  * split-K when the tiles cannot fill the SMs: K stages are shared out over `splits`
+//    CTAs per output tile, each keeping at least two 256-element K stages.
+// NVFP4_BN and NVFP4_SPLITS override the choice (tuning only).
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_split, int num_sms)
+{
+    GemmPlan p;
+    const int nk = static_cast<int>(K / 256);
+    if (M <= 64) {
+        p.swap = true;
+        p.bn = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+        p.p_tiles = ceil_div(N, 128);
+        p.q_tiles = ceil_div(M, p.bn);
+    } else {
+        p.swap = false;
+        p.p_tiles = ceil_div(M, 128);
+        const int t256 = p.p_tiles * ceil_div(N, 256);
+        const int t128 = p.p_tiles * ceil_div(N, 128);
+        const double c256 = static_cast<double>(ceil_div(t256, num_sms)) * 2.0;
+        const double c128 = static_cast<double>(ceil_div(t128, num_sms)) * 1.15;
+        p.bn = (N > 128 && c256 <= c128) ? 256 : 128;
+        const int force = env_int("NVFP4_BN", 0);
+        if (force == 128 || force == 256) p.bn = force;
+        p.q_tiles = ceil_div(N, p.bn);
+    }
+    const int tiles = p.p_tiles * p.q_tiles;
+    p.splits = 1;
+    if (allow_split && tiles * 4 < num_sms * 3 && nk >= 4) {
+        int s = num_sms / tiles;
+        if (s > nk / 2) s = nk / 2;
+        if (s < 1) s = 1;
+        p.splits = s;
+    }
+    const int force_s = env_int("NVFP4_SPLITS", 0);
+    if (allow_split && force_s > 0) p.splits = force_s < nk ? force_s : nk;
+    p.num_tiles = tiles * p.splits;
+    p.grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    if (p.splits > 1) {
+        p.ws_counter_bytes = ((static_cast<size_t>(tiles) * 4 + 255) / 256) * 256;
+        p.ws_bytes = p.ws_counter_bytes +
+                     static_cast<size_t>(tiles) * p.splits * 128 * p.bn * sizeof(float);
+    }
+    return p;
+}
+
+// Grouped: weights always fill the MMA M; the token tile width follows the mean rows per
+// expert (the actual per-tile MMA N is rounded up from the rows present, on the device).
+GemmPlan plan_grouped(int32_t E, int64_t total_rows, int64_t N, int64_t K, int num_sms)
+{
+    (void)K;
+    GemmPlan p;
+    p.grouped = true;
+    p.swap = true;
+    const int64_t avg = E > 0 ? total_rows / E : 0;
+    p.bn = avg <= 24 ? 32 : avg <= 48 ? 64 : avg <= 96 ? 128 : 256;
+    const int force = env_int("NVFP4_GROUPED_BN", 0);
+    if (force == 32 || force == 64 || force == 128 || force == 256) p.bn = force;
+    p.p_tiles = ceil_div(N, 128);
+    p.splits = 1;
+    p.grid = num_sms;
+    return p;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+struct MapKey {
+    std::array<uint64_t, 11> v;
+    bool operator<(const MapKey& o) const { return v < o.v; }
+};
+
+static std::mutex g_map_mu;
+static std::map<MapKey, CUtensorMap> g_map_cache;
+
+// uint8 tensor of `rank` (2 or 3) dims {inner bytes, rows[, depth]} with row stride
+// `stride1` and depth stride `stride2` (bytes); box {box0, box1[, 1]}.
+static bool get_map(CUtensorMap* out, const void* ptr, int rank, uint64_t d0, uint64_t d1,
+                    uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0, uint32_t box1,
+                    bool swizzle128)
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    MapKey key{{reinterpret_cast<uint64_t>(ptr), static_cast<uint64_t>(rank), d0, d1, d2, stride1,
+                stride2, box0, box1, swizzle128 ? 1ull : 0ull, static_cast<uint64_t>(dev)}};
+    {
+        std::lock_guard<std::mutex> g(g_map_mu);
+        auto it = g_map_cache.find(key);
+        if (it != g_map_cache.end()) {
+            *out = it->second;
+            return true;
+        }
+    }
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1, stride2};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUtensorMap m;
+    std::memset(&m, 0, sizeof(m));
+    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank),
+                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    {
+        std::lock_guard<std::mutex> g(g_map_mu);
+        if (g_map_cache.size() > 8192) g_map_cache.clear();
+        g_map_cache[key] = m;
+    }
+    *out = m;
+    return true;
+}
+
+// ------------------------------------------------------------------ launch
+
+template <int BN, bool SWAP, bool GROUPED>
+static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
+                       bool* encode_failed)
+{
+    using Cfg = GemmCfg<BN, SWAP, GROUPED>;
+    auto kern = nvfp4_gemm_kernel<Cfg>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+
+    const uint64_t kb = static_cast<uint64_t>(L.K / 2);    // packed bytes per row
+    const uint64_t ks = static_cast<uint64_t>(L.K / 16);   // scale bytes per row
+    CUtensorMap tp, tq, tsp, tsq;
+    bool ok = true;
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.M = static_cast<int32_t>(L.M);
+    a.N = static_cast<int32_t>(L.N);
+    a.num_kstages = static_cast<int32_t>(L.K / 256);
+    a.num_p_tiles = plan.p_tiles;
+    a.out = static_cast<__nv_bfloat16*>(L.out);
+    a.alpha = L.alpha;
+    a.err_word = L.err_word;
+    if constexpr (GROUPED) {
+        const uint64_t E = static_cast<uint64_t>(L.E);
+        const uint64_t rows = static_cast<uint64_t>(L.total_rows);
+        ok &= get_map(&tp, L.B, 3, kb, L.N, E, kb, kb * L.N, 128, 128, true);
+        ok &= get_map(&tsp, L.sfB, 3, ks, L.N, E, ks, ks * L.N, 16, 128, false);
+        ok &= get_map(&tq, L.A, 2, kb, rows, 1, kb, 0, 128, BN, true);
+        ok &= get_map(&tsq, L.sfA, 2, ks, rows, 1, ks, 0, 16, BN, false);
+        a.p_rows = a.N;
+        a.q_rows = static_cast<int32_t>(L.total_rows);
+        a.splits = 1;
+        a.expert_offsets = L.offsets;
+        a.num_experts = L.E;
+        a.total_rows = static_cast<int32_t>(L.total_rows);
+    } else {
+        const uint8_t* P = SWAP ? L.B : L.A;
+        const uint8_t* sP = SWAP ? L.sfB : L.sfA;
+        const uint8_t* Q = SWAP ? L.A : L.B;
+        const uint8_t* sQ = SWAP ? L.sfA : L.sfB;
+        const uint64_t p_rows = static_cast<uint64_t>(SWAP ? L.N : L.M);
+        const uint64_t q_rows = static_cast<uint64_t>(SWAP ? L.M : L.N);
+        ok &= get_map(&tp, P, 2, kb, p_rows, 1, kb, 0, 128, 128, true);
+        ok &= get_map(&tsp, sP, 2, ks, p_rows, 1, ks, 0, 16, 128, false);
+        ok &= get_map(&tq, Q, 2, kb, q_rows, 1, kb, 0, 128, BN, true);
+        ok &= get_map(&tsq, sQ, 2, ks, q_rows, 1, ks, 0, 16, BN, false);
+        a.p_rows = static_cast<int32_t>(p_rows);
+        a.q_rows = static_cast<int32_t>(q_rows);
+        a.num_q_tiles = plan.q_tiles;
+        a.splits = plan.splits;
+        a.num_tiles = plan.num_tiles;
+        if (plan.splits > 1) {
+            a.ws_counters = static_cast<uint32_t*>(L.ws);
+            a.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(L.ws) + plan.ws_counter_bytes);
+        }
+    }
+    if (!ok) {
+        *encode_failed = true;
+        return cudaSuccess;
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(plan.grid), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, kern, tp, tq, tsp, tsq, a);
+}
+
+cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
+                        bool* encode_failed)
+{
+    *encode_failed = false;
+    if (plan.grid <= 0) return cudaSuccess;
+    if (plan.grouped) {
+        switch (plan.bn) {
+            case 32: return run<32, true, true>(plan, L, stream, encode_failed);
+            case 64: return run<64, true, true>(plan, L, stream, encode_failed);
+            case 128: return run<128, true, true>(plan, L, stream, encode_failed);
+            case 256: return run<256, true, true>(plan, L, stream, encode_failed);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    if (plan.swap) {
+        switch (plan.bn) {
+            case 16: return run<16, true, false>(plan, L, stream, encode_failed);
+            case 32: return run<32, true, false>(plan, L, stream, encode_failed);
+            case 64: return run<64, true, false>(plan, L, stream, encode_failed);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (plan.bn) {
+        case 128: return run<128, false, false>(plan, L, stream, encode_failed);
+        case 256: return run<256, false, false>(plan, L, stream, encode_failed);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace nvfp4

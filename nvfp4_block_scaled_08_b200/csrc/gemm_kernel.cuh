@@ -1,0 +1,584 @@
+// gemm_kernel.cuh -- persistent, warp-specialised NVFP4 block-scaled GEMM for sm_100a.
+//
+// Computes out[m, n] = bf16(alpha * sum_k deq(A)[m, k] * deq(B)[n, k]) where both operands
+// are packed e2m1 (two per byte, K-contiguous) with one e4m3 scale per 16 K-elements
+// ("The Art of Reading the Manual", section "The Message": mm_fp4 with block_size=16,
+// alpha and out; "When a Benchmark Crashes", section "Input Knowledge Required", item 3).
+//
+// The tensor cores see the problem as D[P, Q] = P x Q^T with a 128-row P tile (the MMA's
+// M) and a BN-row Q tile (the MMA's N):
+//   * SWAP = false: P = A (tokens), Q = B (weights); out[p][q].
+//   * SWAP = true : P = B (weights), Q = A (tokens); out[q][p]. Used when there are few
+//     tokens (decode shapes, MoE experts), so that the 128-row MMA dimension is filled by
+//     weight rows and the tokens become a narrow MMA N.
+//   * GROUPED     : SWAP with per-expert weights B[e] and token rows [off[e], off[e+1]).
+//
+// Roles (256 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer: A/B tiles (128-byte swizzle) and linear scale tiles.
+//   warp 1      TMEM allocator and single-thread MMA issuer (tcgen05.cp of scales, then
+//               four 128 x BN x 64 block-scaled MMAs per 256-element K stage).
+//   warp 2      scale re-layout: turns the TMA'd [rows][16 B] scale tile into the
+//               32-row x 16-byte blocks that tcgen05.cp ... 32x128b.warpx4 replicates into
+//               the TMEM layout the MMA reads (row r at column base + r/32, byte = k-block).
+//   warp 3      (grouped) builds the per-expert tile prefix; otherwise idle.
+//   warps 4-7   epilogue: TMEM -> registers -> alpha -> bf16 -> global; with split-K,
+//               fp32 partials to the workspace and a fixed-order reduction by the last
+//               CTA of each tile (deterministic).
+// Every wait is bounded (kWaitTimeoutNs); on a timeout the CTA records an error code,
+// stops all roles, lets in-flight copies and MMAs land, frees TMEM and exits.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+// Error codes recorded in the device error word (which wait gave up).
+enum : uint32_t {
+    kErrProducerEmpty = 0x101,
+    kErrSfFull = 0x102,
+    kErrMmaAccEmpty = 0x103,
+    kErrMmaFull = 0x104,
+    kErrMmaSf = 0x105,
+    kErrEpiAccFull = 0x106,
+};
+
+struct GemmArgs {
+    int32_t M, N;             // output is out[M][N] (row-major, leading dimension N)
+    int32_t p_rows, q_rows;   // rows of the P and Q operands (non-grouped)
+    int32_t num_kstages;      // K / 256
+    int32_t num_p_tiles;      // ceil(p_rows / 128)
+    int32_t num_q_tiles;      // ceil(q_rows / BN) (non-grouped)
+    int32_t splits;           // split-K factor (non-grouped; 1 = none)
+    int32_t num_tiles;        // non-grouped: p_tiles * q_tiles * splits
+    __nv_bfloat16* out;
+    const float* alpha;       // [1] or [E]
+    float* ws_partial;        // split-K fp32 partial tiles
+    uint32_t* ws_counters;    // split-K per-tile arrival counters
+    unsigned* err_word;
+    const int32_t* expert_offsets;  // grouped: [E + 1]
+    int32_t num_experts;
+    int32_t total_rows;       // grouped: rows of A / out
+};
+
+template <int BN_, bool SWAP_, bool GROUPED_>
+struct GemmCfg {
+    static constexpr int BN = BN_;
+    static constexpr bool SWAP = SWAP_;
+    static constexpr bool GROUPED = GROUPED_;
+    static_assert(!GROUPED || SWAP, "grouped GEMM runs with weights as the MMA M operand");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
+
+    static constexpr int BM = 128;                 // MMA M
+    static constexpr int BK_BYTES = 128;           // 256 fp4 values per K stage
+    static constexpr int P_BYTES = BM * BK_BYTES;  // 16 KB
+    static constexpr int Q_BYTES = BN * BK_BYTES;
+    static constexpr int QG = (BN + 127) / 128;    // 128-row scale groups of the Q tile
+    static constexpr int SFP_BYTES = 2048;         // 128 rows x 16 B (= 4 k-blocks x 512 B)
+    static constexpr int SFQ_BYTES = 2048 * QG;
+    static constexpr int SF_TMA_P = BM * 16;       // bytes the scale TMA writes
+    static constexpr int SF_TMA_Q = BN * 16;
+    static constexpr uint32_t TX_BYTES = P_BYTES + Q_BYTES + SF_TMA_P + SF_TMA_Q;
+    static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
+
+    // TMEM columns: accumulators, then SFA (4 k-blocks x 4 columns), then SFB
+    // (4 k-blocks x 4 columns per 128 Q rows).
+    static constexpr int SF_COLS = 16 + 16 * QG;
+    static constexpr int ACC_STAGES = (2 * BN + SF_COLS <= 512) ? 2 : 1;
+    static constexpr int TMEM_SFA = ACC_STAGES * BN;
+    static constexpr int TMEM_SFB = TMEM_SFA + 16;
+    static constexpr int TMEM_USED = TMEM_SFB + 16 * QG;
+    static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
+                                   : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+    static_assert(TMEM_USED <= 512, "TMEM budget");
+
+    static constexpr int SMEM_LIMIT = 232448;      // max dynamic shared memory per block
+    static constexpr int MISC_BYTES = 1024 + (GROUPED ? 4 * (kMaxExperts + 1) : 0);
+    static constexpr int ALIGN_SLACK = 1024;
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - MISC_BYTES - ALIGN_SLACK) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
+    static_assert(STAGES >= 2, "pipeline depth");
+
+    // Shared memory layout (offsets from a 1024-byte aligned base).
+    static constexpr int OFF_P = 0;
+    static constexpr int OFF_Q = OFF_P + STAGES * P_BYTES;
+    static constexpr int OFF_SFP = OFF_Q + STAGES * Q_BYTES;
+    static constexpr int OFF_SFQ = OFF_SFP + STAGES * SFP_BYTES;
+    static constexpr int OFF_BAR = OFF_SFQ + STAGES * SFQ_BYTES;
+    // barriers: full, sfready, empty [STAGES]; acc_full, acc_empty [2]; mma_done
+    static constexpr int NUM_BARS = 3 * STAGES + 5;
+    static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;     // tmem base, flags
+    static constexpr int OFF_PREFIX = OFF_MISC + 64;
+    static constexpr int SMEM_BYTES = OFF_PREFIX + (GROUPED ? 4 * (kMaxExperts + 1) : 0)
+                                    + ALIGN_SLACK;
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+    static_assert(OFF_Q % 1024 == 0 && OFF_SFP % 1024 == 0, "swizzle atoms need 1 KB alignment");
+};
+
+// One unit of work: a 128-row P tile x a BN-row Q tile over a range of K stages.
+struct Tile {
+    int32_t p0;        // first P row (within the expert for grouped)
+    int32_t q0;        // first Q row (global row of A for grouped)
+    int32_t k0;        // first K stage
+    int32_t kcnt;      // number of K stages
+    int32_t pq;        // index of the output tile (split-K counter slot)
+    int32_t split;     // split index
+    int32_t expert;    // grouped: expert id
+    int32_t q_valid;   // grouped: valid Q rows in this tile (<= BN)
+};
+
+// Row range of expert e, clamped to [0, total_rows] and made non-decreasing, so that
+// malformed offsets can only shrink the work, never index outside A or out.
+__device__ __forceinline__ void expert_rows(const GemmArgs& a, int e, int32_t& r0, int32_t& rows)
+{
+    const int32_t lo = min(max(a.expert_offsets[e], 0), a.total_rows);
+    const int32_t hi = min(max(a.expert_offsets[e + 1], lo), a.total_rows);
+    r0 = lo;
+    rows = hi - lo;
+}
+
+template <class Cfg>
+__device__ __forceinline__ Tile decode_tile(const GemmArgs& a, int32_t t, const int32_t* prefix)
+{
+    Tile ti;
+    if constexpr (Cfg::GROUPED) {
+        // expert e: largest e with prefix[e] <= t (empty experts have prefix[e] == prefix[e+1])
+        int lo = 0, hi = a.num_experts;       // invariant: prefix[lo] <= t < prefix[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (prefix[mid] <= t) lo = mid; else hi = mid;
+        }
+        const int e = lo;
+        int32_t r0, rows;
+        expert_rows(a, e, r0, rows);
+        const int32_t qt_count = (rows + Cfg::BN - 1) / Cfg::BN;
+        const int32_t local = t - prefix[e];
+        const int32_t pt = local / qt_count;
+        const int32_t qt = local - pt * qt_count;
+        ti.p0 = pt * Cfg::BM;
+        ti.q0 = r0 + qt * Cfg::BN;
+        ti.q_valid = min(Cfg::BN, rows - qt * Cfg::BN);
+        ti.k0 = 0;
+        ti.kcnt = a.num_kstages;
+        ti.pq = 0;
+        ti.split = 0;
+        ti.expert = e;
+    } else {
+        const int32_t split = t % a.splits;
+        const int32_t pq = t / a.splits;
+        const int32_t pt = pq % a.num_p_tiles;
+        const int32_t qt = pq / a.num_p_tiles;
+        const int32_t base = a.num_kstages / a.splits;
+        const int32_t rem = a.num_kstages % a.splits;
+        ti.p0 = pt * Cfg::BM;
+        ti.q0 = qt * Cfg::BN;
+        ti.k0 = split * base + min(split, rem);
+        ti.kcnt = base + (split < rem ? 1 : 0);
+        ti.pq = pq;
+        ti.split = split;
+        ti.expert = 0;
+        ti.q_valid = min(Cfg::BN, a.q_rows - ti.q0);
+    }
+    return ti;
+}
+
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(256, 1)
+nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_sfp, const __grid_constant__ CUtensorMap tm_sfq,
+                  const GemmArgs args)
+{
+    constexpr int BN = Cfg::BN;
+    constexpr int STAGES = Cfg::STAGES;
+    constexpr int QG = Cfg::QG;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+    uint64_t* full_bar = bars;
+    uint64_t* sfready_bar = bars + STAGES;
+    uint64_t* empty_bar = bars + 2 * STAGES;
+    uint64_t* acc_full_bar = bars + 3 * STAGES;
+    uint64_t* acc_empty_bar = bars + 3 * STAGES + 2;
+    uint64_t* mma_done_bar = bars + 3 * STAGES + 4;
+    uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+    volatile int* s_is_last = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 8);
+    int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + Cfg::OFF_PREFIX);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const AbortState ab{s_abort, args.err_word};
+
+    // ------------------------------------------------------------------ set-up
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&sfready_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&acc_full_bar[s], 1);
+            mbar_init(&acc_empty_bar[s], 4);
+        }
+        mbar_init(mma_done_bar, 1);
+        *s_abort = 0;
+        *s_is_last = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_p);
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_sfp);
+        prefetch_tensormap(&tm_sfq);
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem_base, Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if constexpr (Cfg::GROUPED) {
+        if (warp == 3) {
+            // Tiles per expert: (N / 128 weight tiles) x ceil(rows_e / BN) token tiles.
+            const int E = args.num_experts;
+            const int per = (E + 31) / 32;
+            const int e0 = lane * per;
+            int local = 0;
+            for (int i = 0; i < per; ++i) {
+                const int e = e0 + i;
+                if (e < E) {
+                    int32_t r0, rows;
+                    expert_rows(args, e, r0, rows);
+                    local += args.num_p_tiles * ((rows + BN - 1) / BN);
+                }
+            }
+            int incl = local;
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += y;
+            }
+            int run = incl - local;
+            for (int i = 0; i < per; ++i) {
+                const int e = e0 + i;
+                if (e < E) {
+                    s_prefix[e] = run;
+                    int32_t r0, rows;
+                    expert_rows(args, e, r0, rows);
+                    run += args.num_p_tiles * ((rows + BN - 1) / BN);
+                }
+            }
+            if (lane == 31) s_prefix[E] = incl;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = *s_tmem_base;
+    const int32_t num_tiles = Cfg::GROUPED ? s_prefix[args.num_experts] : args.num_tiles;
+
+    if (warp == 0) {
+        // -------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            const uint64_t pol_stream = l2_policy_evict_first();  // weights: read once
+            const uint64_t pol_keep = l2_policy_evict_last();     // activations: re-read
+            const uint64_t pol_p = Cfg::SWAP ? pol_stream : pol_keep;
+            const uint64_t pol_q = Cfg::SWAP ? pol_keep : pol_stream;
+            uint32_t stage = 0, phase = 0, issued = 0;
+            bool ok = true;
+            for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
+                for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, ab, kErrProducerEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    uint64_t* fb = &full_bar[stage];
+                    mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
+                    const int32_t kx = (ti.k0 + ks) * Cfg::BK_BYTES;   // byte offset along K
+                    const int32_t sx = (ti.k0 + ks) * 16;              // scale byte offset
+                    uint8_t* pbuf = smem + Cfg::OFF_P + stage * Cfg::P_BYTES;
+                    uint8_t* qbuf = smem + Cfg::OFF_Q + stage * Cfg::Q_BYTES;
+                    uint8_t* sfpb = smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES;
+                    uint8_t* sfqb = smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES;
+                    if constexpr (Cfg::GROUPED) {
+                        tma_load_3d(pbuf, &tm_p, fb, kx, ti.p0, ti.expert, pol_p);
+                        tma_load_3d(sfpb, &tm_sfp, fb, sx, ti.p0, ti.expert, pol_p);
+                    } else {
+                        tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
+                        tma_load_2d(sfpb, &tm_sfp, fb, sx, ti.p0, pol_p);
+                    }
+                    tma_load_2d(qbuf, &tm_q, fb, kx, ti.q0, pol_q);
+                    tma_load_2d(sfqb, &tm_sfq, fb, sx, ti.q0, pol_q);
+                    ++issued;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // Let every copy still in flight land before shared memory can be released.
+            const uint32_t inflight = issued < (uint32_t)STAGES ? issued : (uint32_t)STAGES;
+            for (uint32_t i = 1; i <= inflight; ++i) {
+                const int s = ((int)stage - (int)i + 2 * STAGES) % STAGES;
+                const uint32_t ph = ((int)stage - (int)i < 0) ? (phase ^ 1u) : phase;
+                mbar_wait_drain(&full_bar[s], ph);
+            }
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+            bool ok = true;
+            for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
+                if (!mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, ab, kErrMmaAccEmpty)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t n_mma = BN;
+                if constexpr (Cfg::GROUPED) n_mma = min(BN, (ti.q_valid + 15) & ~15);
+                const uint32_t idesc = idesc_mxf4nvf4(128, n_mma);
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
+                    if (!mbar_wait(&full_bar[stage], phase, ab, kErrMmaFull) ||
+                        !mbar_wait(&sfready_bar[stage], phase, ab, kErrMmaSf)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfp = smem_u32(smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES);
+                    const uint32_t sfq = smem_u32(smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        tmem_cp_32x128b_warpx4(tmem_base + Cfg::TMEM_SFA + 4 * j,
+                                               sdesc_sf_32x16(sfp + 512 * j));
+#pragma unroll
+                        for (int g = 0; g < QG; ++g)
+                            tmem_cp_32x128b_warpx4(tmem_base + Cfg::TMEM_SFB + 4 * QG * j + 4 * g,
+                                                   sdesc_sf_32x16(sfq + 2048 * g + 512 * j));
+                    }
+                    const uint64_t pdesc =
+                        sdesc_kmajor_sw128(smem_u32(smem + Cfg::OFF_P + stage * Cfg::P_BYTES));
+                    const uint64_t qdesc =
+                        sdesc_kmajor_sw128(smem_u32(smem + Cfg::OFF_Q + stage * Cfg::Q_BYTES));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        // advance 32 bytes (64 fp4 values) along K inside the swizzled rows
+                        mma_mxf4nvf4(d_tmem, pdesc + 2u * j, qdesc + 2u * j, idesc,
+                                     tmem_base + Cfg::TMEM_SFA + 4 * j,
+                                     tmem_base + Cfg::TMEM_SFB + 4 * QG * j,
+                                     (ks > 0 || j > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&empty_bar[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit(&acc_full_bar[acc]);
+                if (++acc == Cfg::ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
+            }
+            // Arrives once every tcgen05 operation issued above has completed.
+            mma_commit(mma_done_bar);
+        }
+    } else if (warp == 2) {
+        // -------------------------------------------------------------- scale re-layout
+        // The TMA wrote row r's 16 scale bytes (k-blocks 0..15 of the stage) at r * 16.
+        // The MMA for k-step j (k-blocks 4j..4j+3) needs, per 128-row group, a 512-byte
+        // block whose 16-byte row i holds the 4 scale bytes of rows i, i+32, i+64, i+96.
+        // Each lane owns row i = lane: it reads its 4 rows (16 B each), transposes the
+        // 4 x 4 words in registers and writes 4 blocks (one per k-step), in place.
+        uint32_t stage = 0, phase = 0;
+        for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
+            bool ok = true;
+            for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
+                ok = mbar_wait(&full_bar[stage], phase, ab, kErrSfFull);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                uint8_t* sfpb = smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES;
+                uint8_t* sfqb = smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES;
+#pragma unroll
+                for (int grp = 0; grp < 1 + QG; ++grp) {
+                    uint8_t* base = grp == 0 ? sfpb : sfqb + 2048 * (grp - 1);
+                    const int rows_here = grp == 0 ? 128 : min(128, BN - 128 * (grp - 1));
+                    uint4 v[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int r = 32 * q + lane;
+                        v[q] = (r < rows_here) ? *reinterpret_cast<const uint4*>(base + 16 * r)
+                                               : make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    __syncwarp();
+                    uint4 o0 = make_uint4(v[0].x, v[1].x, v[2].x, v[3].x);
+                    uint4 o1 = make_uint4(v[0].y, v[1].y, v[2].y, v[3].y);
+                    uint4 o2 = make_uint4(v[0].z, v[1].z, v[2].z, v[3].z);
+                    uint4 o3 = make_uint4(v[0].w, v[1].w, v[2].w, v[3].w);
+                    *reinterpret_cast<uint4*>(base + 0 * 512 + 16 * lane) = o0;
+                    *reinterpret_cast<uint4*>(base + 1 * 512 + 16 * lane) = o1;
+                    *reinterpret_cast<uint4*>(base + 2 * 512 + 16 * lane) = o2;
+                    *reinterpret_cast<uint4*>(base + 3 * 512 + 16 * lane) = o3;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfready_bar[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+        }
+    } else if (warp >= 4) {
+        // -------------------------------------------------------------- epilogue
+        const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
+        const int row = 32 * quad + lane;          // accumulator row (P row within the tile)
+        const int epi_tid = threadIdx.x - 128;
+        uint32_t acc = 0, acc_phase = 0;
+        for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
+            bool ok = mbar_wait(&acc_full_bar[acc], acc_phase, ab, kErrEpiAccFull);
+            ok = named_bar_and(1, 128, ok);
+            if (!ok) break;
+            tc_fence_after();
+
+            const float alpha = Cfg::GROUPED ? __ldg(args.alpha + ti.expert) : __ldg(args.alpha);
+            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) + acc * BN;
+            const int p = ti.p0 + row;             // P row this thread owns
+            const bool split_k = !Cfg::GROUPED && args.splits > 1;
+            int n_cols = BN;
+            if constexpr (Cfg::GROUPED) n_cols = min(BN, (ti.q_valid + 15) & ~15);
+            float* part = nullptr;
+            if (split_k)
+                part = args.ws_partial +
+                       (static_cast<size_t>(ti.pq) * args.splits + ti.split) * (128 * BN);
+
+            for (int c = 0; c < n_cols; c += 16) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(tacc + c, r);
+                tmem_ld_wait();
+                if (split_k) {
+                    // fp32 partial, layout [col / 4][row][col % 4]: coalesced 16-byte stores
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float4 f = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                               __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                        __stcg(reinterpret_cast<float4*>(part + (c / 4 + i) * 512 + row * 4), f);
+                    }
+                    continue;
+                }
+                if constexpr (!Cfg::SWAP) {
+                    // thread owns output row m = p, columns n = q0 + c .. + 15
+                    const int n0 = ti.q0 + c;
+                    if (p < args.M) {
+                        __nv_bfloat16* dst = args.out + static_cast<size_t>(p) * args.N + n0;
+                        uint4 w0, w1;
+                        w0.x = pack_bf16x2(alpha * __uint_as_float(r[0]), alpha * __uint_as_float(r[1]));
+                        w0.y = pack_bf16x2(alpha * __uint_as_float(r[2]), alpha * __uint_as_float(r[3]));
+                        w0.z = pack_bf16x2(alpha * __uint_as_float(r[4]), alpha * __uint_as_float(r[5]));
+                        w0.w = pack_bf16x2(alpha * __uint_as_float(r[6]), alpha * __uint_as_float(r[7]));
+                        w1.x = pack_bf16x2(alpha * __uint_as_float(r[8]), alpha * __uint_as_float(r[9]));
+                        w1.y = pack_bf16x2(alpha * __uint_as_float(r[10]), alpha * __uint_as_float(r[11]));
+                        w1.z = pack_bf16x2(alpha * __uint_as_float(r[12]), alpha * __uint_as_float(r[13]));
+                        w1.w = pack_bf16x2(alpha * __uint_as_float(r[14]), alpha * __uint_as_float(r[15]));
+                        if (n0 < args.N) *reinterpret_cast<uint4*>(dst) = w0;
+                        if (n0 + 8 < args.N) *reinterpret_cast<uint4*>(dst + 8) = w1;
+                    }
+                } else {
+                    // thread owns output column n = p; columns of the accumulator are rows m
+                    const int n = p;
+                    if (n < args.N) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int qi = c + j;
+                            bool valid;
+                            if constexpr (Cfg::GROUPED) valid = qi < ti.q_valid;
+                            else valid = ti.q0 + qi < args.M;
+                            if (valid)
+                                args.out[static_cast<size_t>(ti.q0 + qi) * args.N + n] =
+                                    __float2bfloat16_rn(alpha * __uint_as_float(r[j]));
+                        }
+                    }
+                }
+            }
+            // Accumulator drained into registers / workspace: hand it back to the MMA warp.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty_bar[acc]);
+            if (++acc == Cfg::ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
+
+            if (split_k) {
+                // The last of the `splits` CTAs of this output tile sums the partials in
+                // split order (deterministic) and writes bf16.
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (epi_tid == 0) {
+                    const uint32_t prev = atomicAdd(args.ws_counters + ti.pq, 1u);
+                    *s_is_last = (prev == static_cast<uint32_t>(args.splits - 1)) ? 1 : 0;
+                }
+                named_bar_sync(1, 128);
+                if (*s_is_last) {
+                    __threadfence();
+                    const float* tile_base =
+                        args.ws_partial + static_cast<size_t>(ti.pq) * args.splits * (128 * BN);
+                    for (int c4 = 0; c4 < BN / 4; ++c4) {
+                        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int sp = 0; sp < args.splits; ++sp) {
+                            const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                                tile_base + static_cast<size_t>(sp) * (128 * BN) + c4 * 512 + row * 4));
+                            s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+                        }
+                        const float vals[4] = {s.x, s.y, s.z, s.w};
+                        if constexpr (!Cfg::SWAP) {
+                            const int n0 = ti.q0 + 4 * c4;
+                            if (p < args.M && n0 < args.N) {
+                                uint2 w;
+                                w.x = pack_bf16x2(alpha * vals[0], alpha * vals[1]);
+                                w.y = pack_bf16x2(alpha * vals[2], alpha * vals[3]);
+                                *reinterpret_cast<uint2*>(args.out + static_cast<size_t>(p) * args.N + n0) = w;
+                            }
+                        } else {
+                            const int n = p;
+                            if (n < args.N) {
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const int m = ti.q0 + 4 * c4 + j;
+                                    if (m < args.M)
+                                        args.out[static_cast<size_t>(m) * args.N + n] =
+                                            __float2bfloat16_rn(alpha * vals[j]);
+                                }
+                            }
+                        }
+                    }
+                    if (epi_tid == 0) args.ws_counters[ti.pq] = 0u;   // re-arm for the next call
+                }
+            }
+        }
+    }
+
+    // ------------------------------------------------------------------ teardown
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        if (lane == 0) mbar_wait_drain(mma_done_bar, 0);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace nvfp4

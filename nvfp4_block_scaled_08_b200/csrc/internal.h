@@ -1,0 +1,55 @@
+// internal.h -- declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+// Largest expert count the grouped GEMM accepts (its tile prefix lives in shared memory).
+constexpr int kMaxExperts = 1024;
+
+// quantize.cu
+cudaError_t launch_global_scale(const void* x, bool bf16, int64_t numel, float* gs,
+                                cudaStream_t stream, int num_sms);
+cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
+                            const float* gs, uint8_t* q, uint8_t* sf, cudaStream_t stream,
+                            int num_sms);
+cudaError_t launch_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
+                         cudaStream_t stream);
+cudaError_t launch_round(const float* x, int64_t n, uint8_t* out, bool e2m1, cudaStream_t stream,
+                         int num_sms);
+
+// Tiling chosen for one GEMM call.
+struct GemmPlan {
+    int bn = 0;            // Q tile rows (MMA N)
+    bool swap = false;     // weights as the 128-row MMA operand
+    bool grouped = false;
+    int splits = 1;        // split-K factor
+    int p_tiles = 0, q_tiles = 0;
+    int num_tiles = 0;     // work items (non-grouped)
+    int grid = 0;          // persistent CTAs
+    size_t ws_bytes = 0;   // workspace needed (split-K)
+    size_t ws_counter_bytes = 0;
+};
+
+// gemm.cu
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_split, int num_sms);
+GemmPlan plan_grouped(int32_t E, int64_t total_rows, int64_t N, int64_t K, int num_sms);
+
+struct GemmLaunch {
+    const uint8_t* A; const uint8_t* sfA; const uint8_t* B; const uint8_t* sfB;
+    const float* alpha; void* out;
+    int64_t M, N, K;
+    const int32_t* offsets; int32_t E; int64_t total_rows;
+    void* ws;
+    unsigned* err_word;
+};
+
+// Returns cudaSuccess or the first CUDA error; *encode_failed is set if a TMA descriptor
+// could not be encoded.
+cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
+                        bool* encode_failed);
+
+}  // namespace nvfp4

@@ -133,30 +133,41 @@ def routing(T: int, seed: int, num_experts: int = NUM_EXPERTS, top_k: int = TOP_
 
 @dataclass
 class GroupedCase:
+    """One grouped-GEMM workload. Routing and activations are drawn on the CPU; the
+    expert weights (up to 25 GB of fp32 for 256 experts) are drawn per expert by torch's
+    seeded generator on the device that will quantise them. Weight seeds depend only on the
+    projection, so both token counts see the same model weights."""
     name: str
     T: int
     N: int
     K: int
-    seed: int
+    route_seed: int
+    weight_seed: int
     num_experts: int = NUM_EXPERTS
 
     def route(self) -> Routing:
-        return routing(self.T, self.seed, self.num_experts)
+        return routing(self.T, self.route_seed, self.num_experts)
 
     def a(self, rows: int) -> torch.Tensor:
-        """Expert-sorted activations [rows, K] ~ N(0, 1)."""
-        return normal(rows, self.K, 1.0, self.seed + 1)
+        """Expert-sorted activations [rows, K] ~ N(0, 1) (CPU)."""
+        return normal(rows, self.K, 1.0, self.route_seed + 1)
 
-    def b(self, expert: int) -> torch.Tensor:
-        """Expert weights [N, K] ~ N(0, 0.02^2)."""
-        return normal(self.N, self.K, 0.02, self.seed + 1000 + expert)
+    def b(self, expert: int, device="cpu") -> torch.Tensor:
+        """Expert weights [N, K] ~ N(0, 0.02^2), drawn on `device`."""
+        g = torch.Generator(device=device)
+        g.manual_seed(self.weight_seed * 4096 + expert)
+        return torch.randn(self.N, self.K, generator=g, dtype=torch.float32, device=device) * 0.02
+
+    @property
+    def flops_per_row(self) -> int:
+        return 2 * self.N * self.K
 
 
 def grouped_cases() -> list[GroupedCase]:
     out = []
     for i, T in enumerate((512, 4096)):
         out.append(GroupedCase(f"moe_gate_up_T{T}", T, 2 * MOE_INTER, HIDDEN,
-                               SEED_BASE + 3 + 10 * i))
+                               SEED_BASE + 3 + 10 * i, SEED_BASE + 3))
         out.append(GroupedCase(f"moe_down_T{T}", T, HIDDEN, MOE_INTER,
-                               SEED_BASE + 3 + 10 * i))
+                               SEED_BASE + 3 + 10 * i + 5, SEED_BASE + 8))
     return out

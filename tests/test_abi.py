@@ -1,0 +1,117 @@
+"""CPU checks of the C ABI: the library builds and loads without a GPU, exports every
+function include/nvfp4.h declares, and rejects bad arguments on the host with the
+documented status codes before any CUDA call is made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_block_scaled_08_b200 as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return nv.load()
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_functions()
+    for n in ("nvfp4_quantize", "nvfp4_gemm", "nvfp4_grouped_gemm", "nvfp4_global_scale",
+              "nvfp4_last_device_error", "nvfp4_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(nv.SIGNATURES)
+
+
+def test_status_strings(lib):
+    for code, name in nv.STATUS.items():
+        assert lib.nvfp4_status_string(code).decode().startswith(name)
+    assert lib.nvfp4_status_string(99).decode() == "NVFP4_ERR_UNKNOWN"
+
+
+def _gemm(lib, A=0x1000, sfA=0x2000, B=0x3000, sfB=0x4000, alpha=0x5000, out=0x6000,
+          M=16, N=768, K=6144, ws=None, ws_bytes=0):
+    return lib.nvfp4_gemm(A, sfA, B, sfB, alpha, out, M, N, K, ws, ws_bytes, None)
+
+
+def test_gemm_host_validation(lib):
+    # empty problems are a no-op and touch nothing
+    assert _gemm(lib, M=0) == 0
+    assert _gemm(lib, N=0) == 0
+    assert _gemm(lib, M=-1) == 1
+    assert _gemm(lib, A=None) == 1
+    assert _gemm(lib, alpha=None) == 1
+    assert _gemm(lib, out=None) == 1
+    assert _gemm(lib, K=100) == 2          # K % 256
+    assert _gemm(lib, K=0) == 2
+    assert _gemm(lib, N=12) == 2           # N % 8
+    assert _gemm(lib, M=1 << 31) == 2
+    assert _gemm(lib, A=0x1001) == 3       # 16-byte alignment
+    assert _gemm(lib, sfB=0x4008) == 3
+    assert _gemm(lib, out=0x6002) == 3
+    assert _gemm(lib, alpha=0x5002) == 3
+    assert _gemm(lib, ws=0x7010, ws_bytes=1 << 20) == 3   # workspace needs 256-byte alignment
+
+
+def test_grouped_host_validation(lib):
+    f = lib.nvfp4_grouped_gemm
+    args = dict(A=0x1000, sfA=0x2000, B=0x3000, sfB=0x4000, alpha=0x5000, off=0x8000,
+                E=256, rows=4096, N=4096, K=6144, out=0x6000)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(a["A"], a["sfA"], a["B"], a["sfB"], a["alpha"], a["off"], a["E"], a["rows"],
+                 a["N"], a["K"], a["out"], None, 0, None)
+
+    assert call(E=0) == 0
+    assert call(rows=0) == 0
+    assert call(E=-1) == 1
+    assert call(off=None) == 1
+    assert call(E=2048) == 2               # more experts than the kernel supports
+    assert call(K=6000) == 2
+    assert call(off=0x8002) == 3
+    assert call(B=0x3004) == 3
+    assert lib.nvfp4_grouped_gemm_workspace_size(256, 4096, 4096, 6144) == 0
+
+
+def test_quantize_host_validation(lib):
+    q = lib.nvfp4_quantize
+    assert q(0x1000, 0, 0, 6144, 6144, 0x2000, 0x3000, 0x4000, None) == 0   # no rows
+    assert q(0x1000, 7, 4, 64, 64, 0x2000, 0x3000, 0x4000, None) == 1       # bad dtype
+    assert q(None, 0, 4, 64, 64, 0x2000, 0x3000, 0x4000, None) == 1
+    assert q(0x1000, 0, 4, 24, 24, 0x2000, 0x3000, 0x4000, None) == 2       # K % 16
+    assert q(0x1000, 0, 4, 64, 32, 0x2000, 0x3000, 0x4000, None) == 1       # ld < K
+    assert q(0x1008, 0, 4, 64, 64, 0x2000, 0x3000, 0x4000, None) == 3
+    assert q(0x1000, 1, 4, 64, 68, 0x2000, 0x3000, 0x4000, None) == 3       # bf16 row stride 136 B
+    gs = lib.nvfp4_global_scale
+    assert gs(0x1000, 0, -1, 0x2000, None) == 1
+    assert gs(0x1000, 0, 16, None, None) == 1
+    assert gs(0x1004, 0, 16, 0x2000, None) == 3
+
+
+def test_round_and_alpha_host_validation(lib):
+    assert lib.nvfp4_round_e4m3(None, 4, 0x1000, None) == 1
+    assert lib.nvfp4_round_e2m1(0x1000, -1, 0x1000, None) == 1
+    assert lib.nvfp4_round_e2m1(0x1000, 0, 0x1000, None) == 0
+    assert lib.nvfp4_alpha(0x1000, 0x2000, 0, 0x3000, None) == 0
+    assert lib.nvfp4_alpha(None, 0x2000, 1, 0x3000, None) == 1
+
+
+def test_binding_is_argument_marshalling_only():
+    # The binding must not import the oracle or compute anything itself.
+    src = open(os.path.join(ROOT, "nvfp4_block_scaled_08_b200", "__init__.py")).read()
+    assert "oracle" not in src.replace("no CPU or alternative-backend path", "")
+    assert "import numpy" not in src
