@@ -1,0 +1,490 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 block-scaled GEMM hot path on B200.
+
+Metric: NVFP4 GEMM TFLOP/s (whole step) and the fraction of the B200 roofline per
+M x N x K. Workload (default): the attention-projection sweep N=768, K=6144,
+M in {16, 64, 256, 1024}, A ~ N(0,1) fp32 activations, B ~ N(0,0.02) weights quantised
+once to NVFP4 outside the timed region. One step = for every M: per-tensor global scale
+of A, alpha = 1/(gsA gsB), NVFP4 quantisation of A, block-scaled GEMM -> bf16.
+
+Timing: the step is captured once as a CUDA graph (with event-record nodes around every
+GEMM); W warm-up replays, then exactly K timed replays bracketed by a barrier and a
+device synchronise, each replay preceded by an untimed L2 flush (a 512 MB write, larger
+than the 126 MB L2). Step time = sum of the per-replay CUDA-event durations, max over
+ranks. SM clocks and throttle reasons are polled through NVML during the timed bracket.
+
+e2e: the same metric through the public Python API called eagerly per step, with the
+activations copied from pinned host memory and the outputs copied back inside the timed
+region.
+
+--impl reference: the CPU oracle as it stands (test infrastructure), on a bounded sample
+of the same workload per step, on this machine's host cores.
+
+Multi-GPU (torchrun, --gpus N): independent replicas, one per GPU ("weak" scaling); the
+path has no exchange step on one GPU's worth of work, so no collective is used on the
+data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+N_ATTN, K_ATTN, M_SWEEP = 768, 6144, (16, 64, 256, 1024)
+FLUSH_BYTES = 512 << 20
+FP4_PER_BF16 = 4.0     # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PF)
+
+
+# ------------------------------------------------------------------ environment
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML in a background thread."""
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        self._marks = []
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self._physical_index(device_index))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    @staticmethod
+    def _physical_index(i):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            try:
+                return int(vis.split(",")[i])
+            except Exception:
+                return i
+        return i
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def mark(self):
+        self._marks.append(time.perf_counter())
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        nv = self.nv
+        t0, t1 = (self._marks + [0, 0])[:2] if len(self._marks) >= 2 else (0, float("inf"))
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if len(inside) < 3:
+            inside = self.samples
+            window = "timed+warmup"
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+        }
+        seen = set()
+        for _, _, r in inside:
+            for k, bit in names.items():
+                if r & bit:
+                    seen.add(k)
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(seen), "samples": len(inside), "window": window}
+
+
+# ------------------------------------------------------------------ roofline model
+
+def gemm_bytes(M, N, K):
+    """Algorithmic HBM bytes of one GEMM: packed operands + scales once, bf16 out once."""
+    return (M + N) * K * (0.5 + 1.0 / 16.0) + 2.0 * M * N
+
+
+def quant_bytes(M, K):
+    """Algorithmic HBM bytes of quantising an fp32 [M, K]: read once, codes + scales out."""
+    return M * K * (4.0 + 0.5 + 1.0 / 16.0)
+
+
+def roofline_us(flops, nbytes, peaks):
+    p_fp4 = peaks["bf16_tflops"] * FP4_PER_BF16 * 1e12
+    bw = peaks["hbm_gbs"] * 1e9
+    t_tc, t_mem = flops / p_fp4, nbytes / bw
+    return max(t_tc, t_mem) * 1e6, ("tensor" if t_tc >= t_mem else "hbm")
+
+
+# ------------------------------------------------------------------ our implementation
+
+class AttnSweep:
+    """Resident inputs, outputs and workspaces of the attention-projection sweep."""
+
+    def __init__(self, dev, rank):
+        import nvfp4_block_scaled_08_b200 as nv
+        from nvfp4_block_scaled_08_b200 import workloads
+        self.nv = nv
+        self.dev = dev
+        cases = workloads.attn_proj_cases()
+        b = cases[0].b()                     # the same weights for every M
+        bd = b.to(dev)
+        self.gsB = nv.global_scale(bd)
+        self.Bq, self.sfB = nv.quantize(bd, self.gsB)
+        del bd
+        self.items = []
+        for c in cases:
+            a_cpu = c.a()
+            it = {
+                "M": c.M, "a_cpu": a_cpu.pin_memory(),
+                "a": a_cpu.to(dev),
+                "gs": torch.empty(1, dtype=torch.float32, device=dev),
+                "alpha": torch.empty(1, dtype=torch.float32, device=dev),
+                "q": torch.empty(c.M, K_ATTN // 2, dtype=torch.uint8, device=dev),
+                "sf": torch.empty(c.M, K_ATTN // 16, dtype=torch.uint8, device=dev),
+                "out": torch.empty(c.M, N_ATTN, dtype=torch.bfloat16, device=dev),
+                "out_host": torch.empty(c.M, N_ATTN, dtype=torch.bfloat16).pin_memory(),
+                "ws": nv.make_workspace(c.M, N_ATTN, K_ATTN, dev),
+            }
+            self.items.append(it)
+        self.flops = sum(2 * it["M"] * N_ATTN * K_ATTN for it in self.items)
+        self.launches_per_step = 5 * len(self.items)   # amax, finalize, alpha, quantize, gemm
+
+    def run_one(self, it, stream=None):
+        nv = self.nv
+        nv.global_scale(it["a"], out=it["gs"], stream=stream)
+        nv.alpha(it["gs"], self.gsB, out=it["alpha"], stream=stream)
+        nv.quantize(it["a"], it["gs"], q=it["q"], sf=it["sf"], stream=stream)
+
+    def gemm_one(self, it, stream=None):
+        self.nv.gemm(it["q"], it["sf"], self.Bq, self.sfB, it["alpha"], out=it["out"],
+                     workspace=it["ws"], stream=stream)
+
+    def capture(self):
+        """One CUDA graph for the whole step, with event nodes around each kernel group."""
+        self.ev = []
+        for it in self.items:
+            self.ev.append([torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)])
+        # run once eagerly so every lazily-initialised resource exists before capture
+        for it in self.items:
+            self.run_one(it)
+            self.gemm_one(it)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for it, ev in zip(self.items, self.ev):
+                ev[0].record()
+                self.run_one(it)
+                ev[1].record()
+                self.gemm_one(it)
+                ev[2].record()
+        self.graph = g
+        return g
+
+    def e2e_step(self, stream):
+        nv = self.nv
+        for it in self.items:
+            it["a"].copy_(it["a_cpu"], non_blocking=True)
+            self.run_one(it)
+            self.gemm_one(it)
+            it["out_host"].copy_(it["out"], non_blocking=True)
+
+    @property
+    def h2d_bytes(self):
+        return sum(it["a_cpu"].numel() * 4 for it in self.items)
+
+    @property
+    def d2h_bytes(self):
+        return sum(it["out"].numel() * 2 for it in self.items)
+
+
+def run_ours(args, world, rank, local):
+    dev = torch.device("cuda", local)
+    peaks = measured_peaks()
+    sweep = AttnSweep(dev, rank)
+    graph = sweep.capture()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    quant_ms = [0.0] * len(sweep.items)
+    gemm_ms = [0.0] * len(sweep.items)
+    total_ms = 0.0
+    barrier(world)
+    clocks.mark()
+    for _ in range(args.steps):
+        flush.zero_()                      # untimed: evicts the previous step from L2
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+        end.synchronize()                  # read this replay's in-graph event timestamps
+        total_ms += start.elapsed_time(end)
+        for j, ev in enumerate(sweep.ev):
+            quant_ms[j] += ev[0].elapsed_time(ev[1]) / args.steps
+            gemm_ms[j] += ev[1].elapsed_time(ev[2]) / args.steps
+    barrier(world)
+    clocks.mark()
+    clocks.stop()
+    step_ms = total_ms / args.steps
+
+    step_ms = max_over_ranks(step_ms, world)
+    value = sweep.flops * world / (step_ms * 1e-3) / 1e12
+
+    # e2e through the public API with host buffers
+    e2e_start = torch.cuda.Event(enable_timing=True)
+    e2e_end = torch.cuda.Event(enable_timing=True)
+    for _ in range(max(1, min(args.warmup, 3))):
+        sweep.e2e_step(stream)
+    barrier(world)
+    e2e_start.record(stream)
+    for _ in range(args.steps):
+        sweep.e2e_step(stream)
+    e2e_end.record(stream)
+    barrier(world)
+    e2e_ms = max_over_ranks(e2e_start.elapsed_time(e2e_end) / args.steps, world)
+    e2e_value = sweep.flops * world / (e2e_ms * 1e-3) / 1e12
+
+    # roofline: per shape, and for the dominant kernel family
+    per_shape = []
+    tot_gemm_us = tot_quant_us = tot_gemm_bytes = tot_quant_bytes = 0.0
+    for it, qm, gm in zip(sweep.items, quant_ms, gemm_ms):
+        M = it["M"]
+        fl = 2.0 * M * N_ATTN * K_ATTN
+        by = gemm_bytes(M, N_ATTN, K_ATTN)
+        r_us, bound = roofline_us(fl, by, peaks)
+        per_shape.append({
+            "M": M, "N": N_ATTN, "K": K_ATTN, "gemm_us": round(gm * 1e3, 3),
+            "gemm_tflops": round(fl / (gm * 1e-3) / 1e12, 1),
+            "roofline_us": round(r_us, 3), "bound": bound, "frac": round(r_us / (gm * 1e3), 4),
+            "quantize_us": round(qm * 1e3, 3),
+            "quantize_gbs": round(quant_bytes(M, K_ATTN) / (qm * 1e-3) / 1e9, 1),
+        })
+        tot_gemm_us += gm * 1e3
+        tot_quant_us += qm * 1e3
+        tot_gemm_bytes += by
+        tot_quant_bytes += quant_bytes(M, K_ATTN)
+    gemm_dominant = tot_gemm_us >= tot_quant_us
+    if gemm_dominant:
+        achieved = tot_gemm_bytes / (tot_gemm_us * 1e-6) / 1e9
+        kernel = "nvfp4_gemm_kernel (all M of the sweep)"
+        units = f"{tot_gemm_bytes:.0f} algorithmic bytes per sweep of 4 launches"
+    else:
+        achieved = tot_quant_bytes / (tot_quant_us * 1e-6) / 1e9
+        kernel = "global_scale + quantize (all M of the sweep)"
+        units = f"{tot_quant_bytes:.0f} algorithmic bytes per sweep"
+    roof = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": None, "per": units,
+            "peak_source": f"{peaks['source']} hbm_gbs (burst copy)"}
+
+    line = {
+        "metric": "NVFP4 GEMM TFLOPS and % of B200 FP4/HBM roofline per M x N x K",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) -> fp32 acc -> bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
+        "config": {"workload": "attn_proj_sweep N=768 K=6144 M={16,64,256,1024}",
+                   "step": "per M: global_scale + alpha + quantize(A fp32) + gemm; one CUDA graph",
+                   "l2": "flushed (512 MB write) before every timed step",
+                   "parallelism": f"replicas x{world}"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sweep.h2d_bytes, "d2h_bytes_per_step": sweep.d2h_bytes,
+                "ms_per_step": round(e2e_ms, 5),
+                "how": "eager public-API calls per step, pinned host A in, bf16 out back"},
+        "gpu_launches": sweep.launches_per_step * args.steps,
+        "roofline": roof,
+        "per_shape": per_shape,
+        "gemm_only_tflops": round(sweep.flops / (tot_gemm_us * 1e-6) / 1e12, 1),
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    del graph
+    sweep.graph = None
+    return line
+
+
+# ------------------------------------------------------------------ the oracle (CPU)
+
+def oracle_sweep_sample(budget_s: float):
+    """Time the oracle on a bounded sample of the sweep: every M, the first r rows of A
+    (r chosen from a calibration so the sample takes about budget_s)."""
+    import numpy as np
+    import oracle
+    from nvfp4_block_scaled_08_b200 import workloads
+    cases = workloads.attn_proj_cases()
+    b = cases[0].b().numpy()
+    gb = oracle.global_scale(b)
+    qb, sb = oracle.quantize(b, gb)               # weights: once, outside the timing
+    a_all = [c.a().numpy() for c in cases]
+    threads = os.cpu_count() or 1
+    # calibration: 8 rows of the largest case
+    t0 = time.perf_counter()
+    oracle.gemm(*oracle.quantize(a_all[-1][:8], oracle.global_scale(a_all[-1])), qb, sb, 1.0,
+                threads=threads)
+    per_row = (time.perf_counter() - t0) / 8
+    total_rows = sum(c.M for c in cases)
+    frac = min(1.0, budget_s / max(per_row * total_rows, 1e-9))
+    rows = [max(1, int(round(c.M * frac))) for c in cases]
+    t0 = time.perf_counter()
+    flops = 0.0
+    for a, r in zip(a_all, rows):
+        ga = oracle.global_scale(a)
+        qa, sa = oracle.quantize(a[:r], ga)
+        al = oracle.alpha(ga, gb)
+        oracle.gemm(qa, sa, qb, sb, al, threads=threads)
+        flops += 2.0 * r * N_ATTN * K_ATTN
+    dt = time.perf_counter() - t0
+    sample = (f"attn_proj sweep, first {rows} rows of M={list(M_SWEEP)} (global scale over the "
+              f"full A), N=768, K=6144; weights quantised outside timing")
+    return flops, dt, threads, sample
+
+
+def cpu_baseline(budget_s: float):
+    flops, dt, threads, sample = oracle_sweep_sample(budget_s)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    per_step = max(0.2, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sweep_sample(per_step)
+    tot_f = tot_t = 0.0
+    info = None
+    for _ in range(args.steps):
+        f, t, th, sample = oracle_sweep_sample(per_step)
+        tot_f += f
+        tot_t += t
+        info = (th, sample)
+    value = tot_f / tot_t / 1e12
+    return {
+        "impl": "reference",
+        "metric": "NVFP4 GEMM TFLOPS and % of B200 FP4/HBM roofline per M x N x K",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+        "data": "synthetic (seeded)",
+        "config": {"workload": "attn_proj_sweep N=768 K=6144 M={16,64,256,1024}",
+                   "note": "CPU oracle (test infrastructure) on a bounded row sample per step"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": info[0],
+                         "kind": "oracle", "sample": info[1]},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        # CPU only: rank 0 times the oracle, the other ranks exit without work
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        line = run_ours(args, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

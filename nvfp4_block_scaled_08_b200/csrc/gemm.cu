@@ -158,15 +158,27 @@ static bool get_map(CUtensorMap* out, const void* ptr, int rank, uint64_t d0, ui
 
 // ------------------------------------------------------------------ launch
 
+constexpr int kMaxDevicesForAttr = 64;
+
 template <int BN, bool SWAP, bool GROUPED>
 static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
                        bool* encode_failed)
 {
     using Cfg = GemmCfg<BN, SWAP, GROUPED>;
     auto kern = nvfp4_gemm_kernel<Cfg>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg::SMEM_BYTES);
+    // Opt in to the large dynamic shared memory once per device (not a stream operation,
+    // so a later launch may be captured into a CUDA graph).
+    static std::once_flag attr_once[kMaxDevicesForAttr];
+    static cudaError_t attr_err[kMaxDevicesForAttr];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevicesForAttr) return cudaErrorInvalidDevice;
+    std::call_once(attr_once[dev], [&] {
+        attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Cfg::SMEM_BYTES);
+    });
+    if (attr_err[dev] != cudaSuccess) return attr_err[dev];
 
     const uint64_t kb = static_cast<uint64_t>(L.K / 2);    // packed bytes per row
     const uint64_t ks = static_cast<uint64_t>(L.K / 16);   // scale bytes per row

@@ -36,7 +36,7 @@ def run_case(dev, a, b, rows=None, cols=None, use_ws=True, guard=True, what=""):
     al = nv.alpha(gsA, gsB)
     ws = nv.make_workspace(M, N, K, dev) if use_ws else None
     pad = 3 if guard else 0
-    sentinel = -12345.0
+    sentinel = -12352.0   # exactly representable in bf16
     big = torch.full((M + pad, N), sentinel, dtype=torch.bfloat16, device=dev)
     out = big[:M]
     ws_guard = None

@@ -34,7 +34,7 @@ def _small_case(dev, counts, N, K, seed, pad_rows=0):
         nv.global_scale(bd, out=gsB[e:e + 1])
         nv.quantize(bd, gsB[e:e + 1], q=Bq[e], sf=sfB[e])
     al = nv.alpha(gsA, gsB)
-    sentinel = 777.0
+    sentinel = 776.0   # exactly representable in bf16
     out = torch.full((rows, N), sentinel, dtype=torch.bfloat16, device=dev)
     nv.grouped_gemm(Aq, sfA, Bq, sfB, al, torch.from_numpy(off).to(dev), out=out)
     st, code = nv.last_device_error()
