@@ -135,6 +135,31 @@ nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint
                                 cudaStream_t stream);
 
 /*
+ * nvfp4_gemm without a workspace argument and without any device allocation. The reference
+ * pages have no counterpart to this call; it exists for callers that cannot allocate
+ * device memory: code running inside a host framework that has reserved all device memory
+ * for its own pool (a cudaMalloc there fails or fragments memory the framework manages),
+ * plugin-style interfaces whose signature offers no workspace, and latency-critical paths
+ * that cannot afford cudaMalloc / cudaFree because they may synchronise the device.
+ *
+ * Same operation, arguments, layouts and checks as nvfp4_gemm (A, sfA, B, sfB, alpha, out
+ * are caller-owned device memory; the caller still passes inputs and outputs). The split-K
+ * scratch comes from one fixed array inside the library, NVFP4_NOALLOC_SCRATCH_BYTES large,
+ * that every GPU which loads the library holds until the process exits. A shape whose
+ * split-K scratch would exceed that size returns NVFP4_ERR_WORKSPACE (nothing launched).
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress
+ * with that device current); make that first call before any stream capture. All calls on
+ * a device share the array and it keeps the last call's contents: each call clears the part
+ * that must start at zero, and calls whose kernels overlap on the GPU (other streams,
+ * other host threads) race on it, so serialise them. Calls no cudaMalloc / cudaFree.
+ */
+#define NVFP4_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                                const uint8_t* sfB, const float* alpha, void* out,
+                                int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+
+/*
  * Elementwise conversions used by the quantiser, exposed so that they can be checked
  * exhaustively: out[i] = e4m3_rn_satfinite(x[i]) (one byte), or e2m1_rn_satfinite(x[i])
  * (one code 0..15 per byte). x, out: device, n elements, no alignment requirement.

@@ -24,6 +24,7 @@ from . import _build
 
 __all__ = [
     "Nvfp4Error", "load", "global_scale", "quantize", "alpha", "gemm", "gemm_workspace_size",
+    "gemm_noalloc",
     "make_workspace", "grouped_gemm", "round_e4m3", "round_e2m1", "last_device_error",
     "STATUS",
 ]
@@ -54,6 +55,7 @@ SIGNATURES = {
     "nvfp4_alpha": (ctypes.c_int, [_P, _P, _I32, _P, _P]),
     "nvfp4_gemm_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "nvfp4_gemm_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_grouped_gemm_workspace_size": (_SZ, [_I32, _I64, _I64, _I64]),
     "nvfp4_grouped_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
                                           _SZ, _P]),
@@ -186,6 +188,21 @@ def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None) -> to
     _check("nvfp4_gemm", load().nvfp4_gemm(
         _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alpha_t), _ptr(out), M, N, K,
         ws_ptr, ws_bytes, _stream(stream)))
+    return out
+
+
+def gemm_noalloc(Aq, sfA, Bq, sfB, alpha_t, out=None, stream=None) -> torch.Tensor:
+    """Same product as gemm() for callers that cannot allocate device memory: the split-K
+    scratch comes from a fixed array inside the library (no workspace argument). All calls
+    on a device share that array, so calls must not overlap on the GPU. `out` must be given
+    by such callers; allocating it here is a convenience for tests."""
+    M, K = Aq.shape[0], Aq.shape[1] * 2
+    N = Bq.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=Aq.device)
+    _check("nvfp4_gemm_noalloc", load().nvfp4_gemm_noalloc(
+        _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alpha_t), _ptr(out), M, N, K,
+        _stream(stream)))
     return out
 
 

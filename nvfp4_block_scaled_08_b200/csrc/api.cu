@@ -93,6 +93,23 @@ nvfp4_status check_gemm_common(const void* A, const void* sfA, const void* B, co
 
 }  // namespace
 
+namespace nvfp4 {
+
+// Device checks for entry points defined in other translation units: arch, SM count and
+// the device error word of the current device (same rules as every call in this file).
+int query_current_device(int* num_sms, unsigned** err_word)
+{
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st == NVFP4_OK) {
+        *num_sms = d.num_sms;
+        *err_word = d.err_word;
+    }
+    return static_cast<int>(st);
+}
+
+}  // namespace nvfp4
+
 extern "C" {
 
 const char* nvfp4_status_string(nvfp4_status s)

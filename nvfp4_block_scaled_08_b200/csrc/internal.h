@@ -47,6 +47,10 @@ struct GemmLaunch {
     unsigned* err_word;
 };
 
+// api.cu: nvfp4_status of the current device's checks; fills the SM count and the device
+// error word on success.
+int query_current_device(int* num_sms, unsigned** err_word);
+
 // Returns cudaSuccess or the first CUDA error; *encode_failed is set if a TMA descriptor
 // could not be encoded.
 cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
