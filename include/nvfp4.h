@@ -88,6 +88,21 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t rows, i
                             cudaStream_t stream);
 
 /*
+ * Activation quantisation in one launch: computes the global scale of x exactly as
+ * nvfp4_global_scale does, writes it to gs_out[0], quantises x with it exactly as
+ * nvfp4_quantize does, and, for i < n_alpha, writes alpha_out[i] = 1 / (gs_out[0] *
+ * gs_other[i]) exactly as nvfp4_alpha does (n_alpha == 0: gs_other / alpha_out unused).
+ * Same layouts and requirements as nvfp4_quantize; gs_out, gs_other, alpha_out: device.
+ * One cooperative launch (amax, grid barrier, scale, grid barrier, quantise); q is used as
+ * scratch for the per-block maxima before it receives the codes. rows * K must be below
+ * 2^31 * (16 / sizeof(dtype)).
+ */
+nvfp4_status nvfp4_quantize_dynamic(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
+                                    int64_t ld_x, float* gs_out, uint8_t* q, uint8_t* sf,
+                                    const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                    cudaStream_t stream);
+
+/*
  * GEMM scale from the two global scales: alpha[i] = 1 / (gs_a[0] * gs_b[i]) in fp32,
  * for i < n (n = 1 for a single GEMM, n = experts for the grouped GEMM). All device.
  */

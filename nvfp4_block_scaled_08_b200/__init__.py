@@ -23,7 +23,7 @@ import torch
 from . import _build
 
 __all__ = [
-    "Nvfp4Error", "load", "global_scale", "quantize", "alpha", "gemm", "gemm_workspace_size",
+    "Nvfp4Error", "load", "global_scale", "quantize", "quantize_dynamic", "alpha", "gemm", "gemm_workspace_size",
     "gemm_noalloc",
     "make_workspace", "grouped_gemm", "round_e4m3", "round_e2m1", "last_device_error",
     "STATUS",
@@ -53,6 +53,8 @@ SIGNATURES = {
     "nvfp4_global_scale": (ctypes.c_int, [_P, ctypes.c_int, _I64, _P, _P]),
     "nvfp4_quantize": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _P, _P]),
     "nvfp4_alpha": (ctypes.c_int, [_P, _P, _I32, _P, _P]),
+    "nvfp4_quantize_dynamic": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _P, _P,
+                                              _I32, _P, _P]),
     "nvfp4_gemm_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "nvfp4_gemm_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
@@ -147,6 +149,32 @@ def quantize(x: torch.Tensor, gs: torch.Tensor, q: torch.Tensor | None = None,
         _ptr(x), _dtype_code(x), rows, K, x.stride(0), _ptr(gs), _ptr(q), _ptr(sf),
         _stream(stream)))
     return q, sf
+
+
+def quantize_dynamic(x: torch.Tensor, gs_other: torch.Tensor | None = None,
+                     gs: torch.Tensor | None = None, q: torch.Tensor | None = None,
+                     sf: torch.Tensor | None = None, alpha_out: torch.Tensor | None = None,
+                     stream=None):
+    """Global scale + quantisation (+ alpha against gs_other) in one launch.
+
+    Returns (q, sf, gs, alpha) where alpha is None when gs_other is None."""
+    _dev(x, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    rows, K = x.shape
+    if q is None:
+        q = torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(rows, K // 16, dtype=torch.uint8, device=x.device)
+    if gs is None:
+        gs = torch.empty(1, dtype=torch.float32, device=x.device)
+    n = 0 if gs_other is None else gs_other.numel()
+    if n and alpha_out is None:
+        alpha_out = torch.empty(n, dtype=torch.float32, device=x.device)
+    _check("nvfp4_quantize_dynamic", load().nvfp4_quantize_dynamic(
+        _ptr(x), _dtype_code(x), rows, K, x.stride(0), _ptr(gs), _ptr(q), _ptr(sf),
+        _ptr(gs_other), n, _ptr(alpha_out) if n else None, _stream(stream)))
+    return q, sf, gs, (alpha_out if n else None)
 
 
 def alpha(gs_a: torch.Tensor, gs_b: torch.Tensor, out: torch.Tensor | None = None,

@@ -160,6 +160,32 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t rows, i
                                             stream, d.num_sms));
 }
 
+nvfp4_status nvfp4_quantize_dynamic(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
+                                    int64_t ld_x, float* gs_out, uint8_t* q, uint8_t* sf,
+                                    const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                    cudaStream_t stream)
+{
+    if (rows < 0 || K < 0 || n_alpha < 0) return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_F32 && dtype != NVFP4_IN_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (!gs_out) return NVFP4_ERR_INVALID_ARG;
+    if (n_alpha > 0 && (!gs_other || !alpha_out)) return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0 || K == 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;   // no tensor to take a scale of
+    if (!x || !q || !sf) return NVFP4_ERR_INVALID_ARG;
+    if (K % 16 != 0 || K > kMaxDim || rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld_x < K) return NVFP4_ERR_INVALID_ARG;
+    const int64_t esz = dtype == NVFP4_IN_BF16 ? 2 : 4;
+    if (rows * (K * esz / 16) >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || (ld_x * esz) % 16 != 0 || !aligned16(q) || !aligned4(gs_out) ||
+        (n_alpha > 0 && (!aligned4(gs_other) || !aligned4(alpha_out))))
+        return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_quantize_dynamic(x, dtype == NVFP4_IN_BF16, rows, K, ld_x, gs_out,
+                                                    q, sf, gs_other, n_alpha, alpha_out, stream,
+                                                    d.num_sms));
+}
+
 nvfp4_status nvfp4_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
                          cudaStream_t stream)
 {
@@ -195,7 +221,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, 
     st = current_device(&d);
     if (st != NVFP4_OK) return st;
     nvfp4::GemmPlan plan = nvfp4::plan_gemm(M, N, K, ws != nullptr, d.num_sms);
-    if (plan.splits > 1 && ws_bytes < plan.ws_bytes) return NVFP4_ERR_WORKSPACE;
+    if (plan.ws_bytes > 0 && ws_bytes < plan.ws_bytes) return NVFP4_ERR_WORKSPACE;
     nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0, ws, d.err_word};
     bool enc_failed = false;
     cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);

@@ -4,7 +4,9 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <array>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <map>
@@ -26,14 +28,22 @@ static int env_int(const char* name, int dflt)
 
 static int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
+// Largest number of clusters of `cs` CTAs (one CTA per SM, as every GEMM variant here
+// uses over 100 KB of shared memory) that the current device runs at once; cached per
+// device. Clusters are placed inside a GPC, so this is below num_sms / cs.
+static int max_active_clusters(int cs);
+
 // Tiling for out[M, N] = A[M, K] x B[N, K]^T on `num_sms` SMs.
 //  * M <= 64: weights fill the 128-row MMA operand (swap), tokens are an MMA N of 16-64.
 //  * otherwise: 128-row token tiles x 128- or 256-row weight tiles, whichever finishes in
 //    fewer tile-waves (wider tiles cost ~2x per tile but move less data per FLOP).
-//  * split-K when the tiles cannot fill the SMs: K stages are shared out over `splits`
-//    CTAs per output tile, each keeping at least two 256-element K stages.
-// NVFP4_BN and NVFP4_SPLITS override the choice (tuning only).
-GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_split, int num_sms)
+//  * split-K when the tiles cannot fill the SMs: the K stages of a tile are shared out
+//    over the CTAs of one thread-block cluster (up to 8), which reduce their partial tiles
+//    over distributed shared memory; the largest cluster whose clusters all run in one
+//    wave is taken. Layouts with `groups` > 1 clusters per tile, which meet in the
+//    workspace, are available through the overrides (and nvfp4_gemm_noalloc's scratch).
+// NVFP4_BN, NVFP4_CLUSTER and NVFP4_GROUPS override the choice (tuning only).
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int num_sms)
 {
     GemmPlan p;
     const int nk = static_cast<int>(K / 256);
@@ -55,22 +65,38 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_split, int num_sm
         p.q_tiles = ceil_div(N, p.bn);
     }
     const int tiles = p.p_tiles * p.q_tiles;
-    p.splits = 1;
-    if (allow_split && tiles * 4 < num_sms * 3 && nk >= 4) {
-        int s = num_sms / tiles;
-        if (s > nk / 2) s = nk / 2;
-        if (s < 1) s = 1;
-        p.splits = s;
+    int cs = 1, g = 1;
+    if (tiles * 4 < num_sms * 3 && nk >= 2) {
+        // One cluster per output tile, as many K slices per cluster as fit in one wave
+        // (measured: a single cluster reduction beats any workspace round trip).
+        const int s_max = std::min({8, nk, num_sms / tiles});
+        for (int c = s_max; c >= 2; --c) {
+            if (tiles <= max_active_clusters(c)) { cs = c; break; }
+        }
     }
-    const int force_s = env_int("NVFP4_SPLITS", 0);
-    if (allow_split && force_s > 0) p.splits = force_s < nk ? force_s : nk;
+    const int fc = env_int("NVFP4_CLUSTER", 0), fg = env_int("NVFP4_GROUPS", 0);
+    if (fc > 0 || fg > 0) {
+        cs = std::max(1, std::min(fc > 0 ? fc : cs, 8));
+        g = std::max(1, fg > 0 ? fg : g);
+        if (!allow_workspace) g = 1;
+        while (cs * g > nk && g > 1) --g;
+        while (cs * g > nk && cs > 1) --cs;
+    }
+    p.cluster = cs;
+    p.groups = g;
+    p.splits = cs * g;
     p.num_tiles = tiles * p.splits;
-    p.grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-    if (p.splits > 1) {
-        p.ws_counter_bytes = ((static_cast<size_t>(tiles) * 4 + 255) / 256) * 256;
-        p.ws_bytes = p.ws_counter_bytes +
-                     static_cast<size_t>(tiles) * p.splits * 128 * p.bn * sizeof(float);
+    // split-K launches exactly one CTA per work item (the reduction relies on it)
+    p.grid = p.splits > 1 ? p.num_tiles : std::min(p.num_tiles, num_sms);
+    if (g > 1) {
+        p.ws_counter_bytes = ((static_cast<size_t>(tiles) * cs * 4 + 255) / 256) * 256;
+        p.ws_bytes = p.ws_counter_bytes + static_cast<size_t>(tiles) * g * 128 * p.bn * sizeof(float);
     }
+    if (env_int("NVFP4_DEBUG", 0))
+        std::fprintf(stderr, "nvfp4 plan M=%lld N=%lld K=%lld: bn=%d swap=%d tiles=%d cluster=%d groups=%d "
+                     "grid=%d ws=%zu (max active clusters: 2:%d 4:%d 8:%d)\n",
+                     (long long)M, (long long)N, (long long)K, p.bn, (int)p.swap, tiles, cs, g, p.grid,
+                     p.ws_bytes, max_active_clusters(2), max_active_clusters(4), max_active_clusters(8));
     return p;
 }
 
@@ -160,6 +186,43 @@ static bool get_map(CUtensorMap* out, const void* ptr, int rank, uint64_t d0, ui
 
 constexpr int kMaxDevicesForAttr = 64;
 
+static int max_active_clusters(int cs)
+{
+    static std::mutex mu;
+    static int cache[kMaxDevicesForAttr][9];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesForAttr || cs < 1 || cs > 8) {
+        cudaGetLastError();
+        return 0;
+    }
+    std::lock_guard<std::mutex> g(mu);
+    if (cache[dev][cs] == 0) {
+        // any GEMM variant gives the same answer: all use one CTA per SM
+        using Cfg = GemmCfg<128, false, false>;
+        auto kern = nvfp4_gemm_kernel<Cfg>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = cs;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.gridDim = dim3(cs * 64, 1, 1);
+        cfg.blockDim = dim3(256, 1, 1);
+        cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cache[dev][cs] = n > 0 ? n : -1;
+    }
+    return cache[dev][cs] > 0 ? cache[dev][cs] : 0;
+}
+
 template <int BN, bool SWAP, bool GROUPED>
 static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
                        bool* encode_failed)
@@ -186,6 +249,8 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
     bool ok = true;
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
+    a.cluster_size = 1;
+    a.groups = 1;
     a.M = static_cast<int32_t>(L.M);
     a.N = static_cast<int32_t>(L.N);
     a.num_kstages = static_cast<int32_t>(L.K / 256);
@@ -221,8 +286,10 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         a.q_rows = static_cast<int32_t>(q_rows);
         a.num_q_tiles = plan.q_tiles;
         a.splits = plan.splits;
+        a.cluster_size = plan.cluster;
+        a.groups = plan.groups;
         a.num_tiles = plan.num_tiles;
-        if (plan.splits > 1) {
+        if (plan.groups > 1) {
             a.ws_counters = static_cast<uint32_t*>(L.ws);
             a.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(L.ws) + plan.ws_counter_bytes);
         }
@@ -237,8 +304,16 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
     cfg.blockDim = dim3(256, 1, 1);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cfg.stream = stream;
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
+    // programmatic dependent launch: the prologue overlaps the previous kernel's tail
+    cudaLaunchAttribute attrs[2];
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = static_cast<unsigned>(plan.cluster);
+    attrs[1].val.clusterDim.y = 1;
+    attrs[1].val.clusterDim.z = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = (!GROUPED && plan.cluster > 1) ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, kern, tp, tq, tsp, tsq, a);
 }
 

@@ -45,6 +45,7 @@ enum : uint32_t {
     kErrMmaFull = 0x104,
     kErrMmaSf = 0x105,
     kErrEpiAccFull = 0x106,
+    kErrSplitRx = 0x107,
 };
 
 struct GemmArgs {
@@ -53,7 +54,9 @@ struct GemmArgs {
     int32_t num_kstages;      // K / 256
     int32_t num_p_tiles;      // ceil(p_rows / 128)
     int32_t num_q_tiles;      // ceil(q_rows / BN) (non-grouped)
-    int32_t splits;           // split-K factor (non-grouped; 1 = none)
+    int32_t splits;           // split-K factor (non-grouped; 1 = none) = cluster_size * groups
+    int32_t cluster_size;     // split-K CTAs per thread-block cluster (reduced over DSMEM)
+    int32_t groups;           // clusters per output tile (reduced through the workspace)
     int32_t num_tiles;        // non-grouped: p_tiles * q_tiles * splits
     __nv_bfloat16* out;
     const float* alpha;       // [1] or [E]
@@ -109,13 +112,18 @@ struct GemmCfg {
     static constexpr int OFF_SFP = OFF_Q + STAGES * Q_BYTES;
     static constexpr int OFF_SFQ = OFF_SFP + STAGES * SFP_BYTES;
     static constexpr int OFF_BAR = OFF_SFQ + STAGES * SFQ_BYTES;
-    // barriers: full, sfready, empty [STAGES]; acc_full, acc_empty [2]; mma_done
-    static constexpr int NUM_BARS = 3 * STAGES + 5;
+    // barriers: full, sfready, empty [STAGES]; acc_full, acc_empty [2]; mma_done; split-K rx
+    static constexpr int NUM_BARS = 3 * STAGES + 6;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;     // tmem base, flags
     static constexpr int OFF_PREFIX = OFF_MISC + 64;
     static constexpr int SMEM_BYTES = OFF_PREFIX + (GROUPED ? 4 * (kMaxExperts + 1) : 0)
                                     + ALIGN_SLACK;
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+    // split-K partial tile in shared memory: [128 rows][BN + 4 floats]
+    static constexpr int PSTRIDE = BN + 4;
+    // split-K receive buffer: a chunk of ceil(128 / cs) rows from each of cs <= 8 ranks,
+    // cs * ceil(128 / cs) <= 135 rows
+    static_assert(136 * PSTRIDE * 4 <= STAGES * STAGE_BYTES, "split-K receive buffer fits the pipeline buffers");
     static_assert(OFF_Q % 1024 == 0 && OFF_SFP % 1024 == 0, "swizzle atoms need 1 KB alignment");
 };
 
@@ -200,6 +208,166 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
     return r != 0;
 }
 
+// Store 4 consecutive accumulator columns (c4 * 4 .. +3) of P row `row` of a tile.
+template <class Cfg>
+__device__ __forceinline__ void store_out4(const GemmArgs& a, const Tile& ti, int row, int c4,
+                                           float4 v, float alpha)
+{
+    const int p = ti.p0 + row;
+    if constexpr (!Cfg::SWAP) {
+        const int n0 = ti.q0 + 4 * c4;
+        if (p < a.M && n0 < a.N) {
+            uint2 w;
+            w.x = pack_bf16x2(alpha * v.x, alpha * v.y);
+            w.y = pack_bf16x2(alpha * v.z, alpha * v.w);
+            *reinterpret_cast<uint2*>(a.out + static_cast<size_t>(p) * a.N + n0) = w;
+        }
+    } else {
+        if (p < a.N) {
+            const float vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int m = ti.q0 + 4 * c4 + j;
+                if (m < a.M)
+                    a.out[static_cast<size_t>(m) * a.N + p] = __float2bfloat16_rn(alpha * vals[j]);
+            }
+        }
+    }
+}
+
+// Rows [chunk_begin(k), chunk_begin(k + 1)) of a 128-row tile belong to cluster rank k.
+__device__ __forceinline__ int chunk_begin(int k, int cs) { return (k * 128 + cs - 1) / cs; }
+
+// Split-K epilogue of one CTA, run by the 128 epilogue threads (thread = accumulator row);
+// every CTA of a split-K launch owns exactly one tile. The `cluster_size` CTAs of a cluster
+// hold consecutive K slices of the same output tile, and row chunk k is reduced by cluster
+// rank k. After the cluster barrier (every CTA of the cluster has drained its main loop, so
+// its pipeline shared memory is free) each thread sends its accumulator row, straight from
+// TMEM through registers, to the owning rank with st.async; the owner's threads wait on
+// their rx barrier, sum the ranks in order (fixed, deterministic) and write bf16. With
+// `groups` > 1 clusters per tile the owners write their fp32 chunk to the workspace instead,
+// and the last of the `groups` CTAs holding the same chunk (arrival counter) sums the
+// chunks in group order.
+template <class Cfg>
+__device__ __forceinline__ void split_k_epilogue(const GemmArgs& a, const Tile& ti, uint8_t* smem,
+                                                 uint64_t* rx_bar, volatile int* s_is_last,
+                                                 uint32_t tacc, int row, float alpha,
+                                                 const AbortState& ab)
+{
+    constexpr int BN = Cfg::BN;
+    constexpr int PS = Cfg::PSTRIDE;
+    const int cs = a.cluster_size;
+    const int g = a.groups;
+    const int rank = cs > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+    const int owner = (row * cs) / 128;    // == the k with chunk_begin(k) <= row < chunk_begin(k+1)
+    float* rx = reinterpret_cast<float*>(smem + Cfg::OFF_P);
+    if (cs > 1) { cluster_arrive(); cluster_wait(); }
+
+    const int my0 = chunk_begin(rank, cs);
+    const int my_rows = chunk_begin(rank + 1, cs) - my0;
+    const int grp = ti.split / cs;
+    const bool is_owner = owner == rank;
+    // tcgen05.ld is .sync.aligned: every lane of the warp executes every load below, and
+    // only what is done with the values depends on the lane's row.
+
+    // 1. rows owned by another rank go there (TMEM -> registers -> peer shared memory)
+    if (cs > 1) {
+        const int own0 = chunk_begin(owner, cs);
+        const int own_rows = chunk_begin(owner + 1, cs) - own0;
+        const uint32_t dst = mapa_shared(smem_u32(rx + (rank * own_rows + (row - own0)) * PS),
+                                         static_cast<uint32_t>(owner));
+        const uint32_t bar = mapa_shared(smem_u32(rx_bar), static_cast<uint32_t>(owner));
+        for (int c = 0; c < BN; c += 16) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(tacc + c, r);
+            tmem_ld_wait();
+            if (!is_owner) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    st_async_f4(dst + (c + 4 * i) * 4, __uint_as_float(r[4 * i]),
+                                __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
+                                __uint_as_float(r[4 * i + 3]), bar);
+            }
+        }
+    }
+    // 2. wait (all epilogue threads, bounded) for the other ranks' copies of this CTA's rows
+    bool ok = true;
+    if (cs > 1) {
+        if (row == my0)
+            mbar_arrive_expect_tx(rx_bar, static_cast<uint32_t>((cs - 1) * my_rows * BN * 4));
+        ok = mbar_wait(rx_bar, 0, ab, kErrSplitRx);
+        __syncwarp();
+    }
+    // 3. owner rows: own partial (from TMEM) + the received ones, in rank order
+    const int lr = row - my0;
+    float* chunk_ws = nullptr;
+    if (g > 1) chunk_ws = a.ws_partial + (static_cast<size_t>(ti.pq) * g + grp) * (128 * BN);
+    for (int c = 0; c < BN; c += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tacc + c, r);
+        tmem_ld_wait();
+        if (!is_owner) continue;
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+        for (int k = 0; k < cs; ++k) {
+            if (k == rank) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(r[j]);
+            } else if (ok) {
+                const float* src = rx + (k * my_rows + lr) * PS + c;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 f = *reinterpret_cast<const float4*>(src + 4 * i);
+                    v[4 * i] += f.x; v[4 * i + 1] += f.y; v[4 * i + 2] += f.z; v[4 * i + 3] += f.w;
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 f = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            if (g == 1) store_out4<Cfg>(a, ti, row, c / 4 + i, f, alpha);
+            else __stcg(reinterpret_cast<float4*>(chunk_ws + row * BN + c + 4 * i), f);
+        }
+    }
+    __syncwarp();
+    if (g == 1) return;
+
+    // groups > 1: the last of the `groups` CTAs that hold chunk `rank` of this tile sums the
+    // chunks from the workspace in group order
+    __threadfence();
+    __syncwarp();
+    named_bar_sync(1, 128);
+    uint32_t* counter = a.ws_counters + static_cast<size_t>(ti.pq) * cs + rank;
+    if (row == my0) {
+        const uint32_t prev = atomicAdd(counter, 1u);
+        *s_is_last = (prev == static_cast<uint32_t>(g - 1)) ? 1 : 0;
+    }
+    __syncwarp();
+    named_bar_sync(1, 128);
+    if (!*s_is_last) return;
+    __threadfence();
+    if (is_owner) {
+        const float* tile_ws = a.ws_partial + static_cast<size_t>(ti.pq) * g * (128 * BN);
+        for (int c4 = 0; c4 < BN / 4; ++c4) {
+            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j0 = 0; j0 < g; j0 += 4) {
+                float4 v[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (j0 + j < g)
+                        v[j] = __ldcg(reinterpret_cast<const float4*>(
+                            tile_ws + static_cast<size_t>(j0 + j) * (128 * BN) + row * BN + 4 * c4));
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (j0 + j < g) { s.x += v[j].x; s.y += v[j].y; s.z += v[j].z; s.w += v[j].w; }
+            }
+            store_out4<Cfg>(a, ti, row, c4, s, alpha);
+        }
+    }
+    if (row == my0) *counter = 0u;             // re-arm for the next call
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(256, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
@@ -221,6 +389,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     uint64_t* acc_full_bar = bars + 3 * STAGES;
     uint64_t* acc_empty_bar = bars + 3 * STAGES + 2;
     uint64_t* mma_done_bar = bars + 3 * STAGES + 4;
+    uint64_t* rx_bar = bars + 3 * STAGES + 5;       // split-K: partial rows received from peers
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
     volatile int* s_is_last = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 8);
@@ -242,6 +411,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             mbar_init(&acc_empty_bar[s], 4);
         }
         mbar_init(mma_done_bar, 1);
+        mbar_init(rx_bar, 1);
         *s_abort = 0;
         *s_is_last = 0;
         fence_mbarrier_init();
@@ -256,6 +426,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         tmem_alloc(s_tmem_base, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
+    // Everything above touches only this CTA's resources and the kernel parameters; from
+    // here on the kernel reads data that the previous kernel in the stream may have written.
+    grid_dependency_wait();
     if constexpr (Cfg::GROUPED) {
         if (warp == 3) {
             // Tiles per expert: (N / 128 weight tiles) x ceil(rows_e / BN) token tiles.
@@ -298,20 +471,20 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
 
     if (warp == 0) {
         // -------------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            const uint64_t pol_stream = l2_policy_evict_first();  // weights: read once
-            const uint64_t pol_keep = l2_policy_evict_last();     // activations: re-read
-            const uint64_t pol_p = Cfg::SWAP ? pol_stream : pol_keep;
-            const uint64_t pol_q = Cfg::SWAP ? pol_keep : pol_stream;
-            uint32_t stage = 0, phase = 0, issued = 0;
-            bool ok = true;
-            for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
-                for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, ab, kErrProducerEmpty)) {
-                        ok = false;
-                        break;
-                    }
+        // The whole warp walks the loop (uniform control flow and operands); one elected
+        // lane issues the copies.
+        const uint64_t pol_stream = l2_policy_evict_first();  // weights: read once
+        const uint64_t pol_keep = l2_policy_evict_last();     // activations: re-read
+        const uint64_t pol_p = Cfg::SWAP ? pol_stream : pol_keep;
+        const uint64_t pol_q = Cfg::SWAP ? pol_keep : pol_stream;
+        uint32_t stage = 0, phase = 0, issued = 0;
+        bool ok = true;
+        for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
+            for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, ab, kErrProducerEmpty));
+                if (!ok) break;
+                if (elect_one()) {
                     uint64_t* fb = &full_bar[stage];
                     mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
                     const int32_t kx = (ti.k0 + ks) * Cfg::BK_BYTES;   // byte offset along K
@@ -329,41 +502,39 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     }
                     tma_load_2d(qbuf, &tm_q, fb, kx, ti.q0, pol_q);
                     tma_load_2d(sfqb, &tm_sfq, fb, sx, ti.q0, pol_q);
-                    ++issued;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
+                __syncwarp();
+                ++issued;
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-            // Let every copy still in flight land before shared memory can be released.
-            const uint32_t inflight = issued < (uint32_t)STAGES ? issued : (uint32_t)STAGES;
-            for (uint32_t i = 1; i <= inflight; ++i) {
-                const int s = ((int)stage - (int)i + 2 * STAGES) % STAGES;
-                const uint32_t ph = ((int)stage - (int)i < 0) ? (phase ^ 1u) : phase;
-                mbar_wait_drain(&full_bar[s], ph);
-            }
+        }
+        // Let every copy still in flight land before shared memory can be released.
+        const uint32_t inflight = issued < (uint32_t)STAGES ? issued : (uint32_t)STAGES;
+        for (uint32_t i = 1; i <= inflight; ++i) {
+            const int s = ((int)stage - (int)i + 2 * STAGES) % STAGES;
+            const uint32_t ph = ((int)stage - (int)i < 0) ? (phase ^ 1u) : phase;
+            mbar_wait_drain(&full_bar[s], ph);
         }
     } else if (warp == 1) {
         // -------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-            bool ok = true;
-            for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
-                if (!mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, ab, kErrMmaAccEmpty)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                uint32_t n_mma = BN;
-                if constexpr (Cfg::GROUPED) n_mma = min(BN, (ti.q_valid + 15) & ~15);
-                const uint32_t idesc = idesc_mxf4nvf4(128, n_mma);
-                const uint32_t d_tmem = tmem_base + acc * BN;
-                for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
-                    if (!mbar_wait(&full_bar[stage], phase, ab, kErrMmaFull) ||
-                        !mbar_wait(&sfready_bar[stage], phase, ab, kErrMmaSf)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+        // Whole warp in the loop, one elected lane issues tcgen05.cp / tcgen05.mma.
+        uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+        bool ok = true;
+        for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
+            ok = __all_sync(0xffffffffu, mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, ab, kErrMmaAccEmpty));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t n_mma = BN;
+            if constexpr (Cfg::GROUPED) n_mma = min(BN, (ti.q_valid + 15) & ~15);
+            const uint32_t idesc = idesc_mxf4nvf4(128, n_mma);
+            const uint32_t d_tmem = tmem_base + acc * BN;
+            for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
+                bool got = mbar_wait(&full_bar[stage], phase, ab, kErrMmaFull);
+                got = got && mbar_wait(&sfready_bar[stage], phase, ab, kErrMmaSf);
+                ok = __all_sync(0xffffffffu, got);
+                if (!ok) break;
+                if (elect_one()) {
                     const uint32_t sfp = smem_u32(smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES);
                     const uint32_t sfq = smem_u32(smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES);
 #pragma unroll
@@ -388,15 +559,18 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                                      (ks > 0 || j > 0) ? 1u : 0u);
                     }
                     mma_commit(&empty_bar[stage]);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (!ok) break;
-                mma_commit(&acc_full_bar[acc]);
-                if (++acc == Cfg::ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
+                __syncwarp();
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-            // Arrives once every tcgen05 operation issued above has completed.
-            mma_commit(mma_done_bar);
+            if (!ok) break;
+            if (elect_one()) mma_commit(&acc_full_bar[acc]);
+            __syncwarp();
+            if (++acc == Cfg::ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
         }
+        // Arrives once every tcgen05 operation issued above has completed.
+        if (elect_one()) mma_commit(mma_done_bar);
+        __syncwarp();
     } else if (warp == 2) {
         // -------------------------------------------------------------- scale re-layout
         // The TMA wrote row r's 16 scale bytes (k-blocks 0..15 of the stage) at r * 16.
@@ -446,13 +620,18 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         // -------------------------------------------------------------- epilogue
         const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
         const int row = 32 * quad + lane;          // accumulator row (P row within the tile)
-        const int epi_tid = threadIdx.x - 128;
         uint32_t acc = 0, acc_phase = 0;
         for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
             bool ok = mbar_wait(&acc_full_bar[acc], acc_phase, ab, kErrEpiAccFull);
             ok = named_bar_and(1, 128, ok);
-            if (!ok) break;
+            if (!ok) {
+                if constexpr (!Cfg::GROUPED) {
+                    // cluster peers wait for this CTA on the cluster barrier: arrive anyway
+                    if (args.splits > 1 && args.cluster_size > 1) { cluster_arrive(); cluster_wait(); }
+                }
+                break;
+            }
             tc_fence_after();
 
             const float alpha = Cfg::GROUPED ? __ldg(args.alpha + ti.expert) : __ldg(args.alpha);
@@ -461,25 +640,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             const bool split_k = !Cfg::GROUPED && args.splits > 1;
             int n_cols = BN;
             if constexpr (Cfg::GROUPED) n_cols = min(BN, (ti.q_valid + 15) & ~15);
-            float* part = nullptr;
-            if (split_k)
-                part = args.ws_partial +
-                       (static_cast<size_t>(ti.pq) * args.splits + ti.split) * (128 * BN);
+            if constexpr (!Cfg::GROUPED) {
+                if (split_k) split_k_epilogue<Cfg>(args, ti, smem, rx_bar, s_is_last, tacc, row, alpha, ab);
+            }
 
-            for (int c = 0; c < n_cols; c += 16) {
+            for (int c = 0; c < n_cols && !split_k; c += 16) {
                 uint32_t r[16];
                 tmem_ld_32x32b_x16(tacc + c, r);
                 tmem_ld_wait();
-                if (split_k) {
-                    // fp32 partial, layout [col / 4][row][col % 4]: coalesced 16-byte stores
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        float4 f = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                               __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-                        __stcg(reinterpret_cast<float4*>(part + (c / 4 + i) * 512 + row * 4), f);
-                    }
-                    continue;
-                }
                 if constexpr (!Cfg::SWAP) {
                     // thread owns output row m = p, columns n = q0 + c .. + 15
                     const int n0 = ti.q0 + c;
@@ -520,57 +688,18 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             if (lane == 0) mbar_arrive(&acc_empty_bar[acc]);
             if (++acc == Cfg::ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
 
-            if (split_k) {
-                // The last of the `splits` CTAs of this output tile sums the partials in
-                // split order (deterministic) and writes bf16.
-                __threadfence();
-                named_bar_sync(1, 128);
-                if (epi_tid == 0) {
-                    const uint32_t prev = atomicAdd(args.ws_counters + ti.pq, 1u);
-                    *s_is_last = (prev == static_cast<uint32_t>(args.splits - 1)) ? 1 : 0;
-                }
-                named_bar_sync(1, 128);
-                if (*s_is_last) {
-                    __threadfence();
-                    const float* tile_base =
-                        args.ws_partial + static_cast<size_t>(ti.pq) * args.splits * (128 * BN);
-                    for (int c4 = 0; c4 < BN / 4; ++c4) {
-                        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-                        for (int sp = 0; sp < args.splits; ++sp) {
-                            const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                                tile_base + static_cast<size_t>(sp) * (128 * BN) + c4 * 512 + row * 4));
-                            s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-                        }
-                        const float vals[4] = {s.x, s.y, s.z, s.w};
-                        if constexpr (!Cfg::SWAP) {
-                            const int n0 = ti.q0 + 4 * c4;
-                            if (p < args.M && n0 < args.N) {
-                                uint2 w;
-                                w.x = pack_bf16x2(alpha * vals[0], alpha * vals[1]);
-                                w.y = pack_bf16x2(alpha * vals[2], alpha * vals[3]);
-                                *reinterpret_cast<uint2*>(args.out + static_cast<size_t>(p) * args.N + n0) = w;
-                            }
-                        } else {
-                            const int n = p;
-                            if (n < args.N) {
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    const int m = ti.q0 + 4 * c4 + j;
-                                    if (m < args.M)
-                                        args.out[static_cast<size_t>(m) * args.N + n] =
-                                            __float2bfloat16_rn(alpha * vals[j]);
-                                }
-                            }
-                        }
-                    }
-                    if (epi_tid == 0) args.ws_counters[ti.pq] = 0u;   // re-arm for the next call
-                }
-            }
         }
     }
 
     // ------------------------------------------------------------------ teardown
     __syncwarp();
+    grid_launch_dependents();
+    if constexpr (!Cfg::GROUPED) {
+        // split-K: the non-epilogue warps are done with the pipeline; together with the
+        // epilogue's arrival (after its accumulator is complete) this tells the cluster peers
+        // that this CTA's shared memory may receive their partial rows
+        if (warp < 4 && args.splits > 1 && args.cluster_size > 1) { cluster_arrive(); cluster_wait(); }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

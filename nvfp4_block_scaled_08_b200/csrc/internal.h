@@ -16,6 +16,10 @@ cudaError_t launch_global_scale(const void* x, bool bf16, int64_t numel, float* 
 cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
                             const float* gs, uint8_t* q, uint8_t* sf, cudaStream_t stream,
                             int num_sms);
+cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
+                                    float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
+                                    int32_t n_alpha, float* alpha_out, cudaStream_t stream,
+                                    int num_sms);
 cudaError_t launch_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
                          cudaStream_t stream);
 cudaError_t launch_round(const float* x, int64_t n, uint8_t* out, bool e2m1, cudaStream_t stream,
@@ -26,7 +30,9 @@ struct GemmPlan {
     int bn = 0;            // Q tile rows (MMA N)
     bool swap = false;     // weights as the 128-row MMA operand
     bool grouped = false;
-    int splits = 1;        // split-K factor
+    int splits = 1;        // split-K factor = cluster * groups
+    int cluster = 1;       // split-K CTAs per thread-block cluster (DSMEM reduction)
+    int groups = 1;        // clusters per output tile (workspace reduction when > 1)
     int p_tiles = 0, q_tiles = 0;
     int num_tiles = 0;     // work items (non-grouped)
     int grid = 0;          // persistent CTAs
@@ -35,7 +41,9 @@ struct GemmPlan {
 };
 
 // gemm.cu
-GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_split, int num_sms);
+// allow_workspace: a split-K workspace may be used (groups > 1); cluster-only split-K
+// needs none.
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int num_sms);
 GemmPlan plan_grouped(int32_t E, int64_t total_rows, int64_t N, int64_t K, int num_sms);
 
 struct GemmLaunch {

@@ -82,7 +82,7 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint
     // Same tiling as nvfp4_gemm with a workspace available; a plan whose split-K scratch
     // would not fit in the fixed array is rejected, not silently changed.
     nvfp4::GemmPlan plan = nvfp4::plan_gemm(M, N, K, true, num_sms);
-    if (plan.splits > 1) {
+    if (plan.ws_bytes > 0) {
         if (plan.ws_bytes > kNoallocScratchBytes) return NVFP4_ERR_WORKSPACE;
         // The tile counters must start at zero; a previous call may have been cut short.
         if (cudaMemsetAsync(scratch, 0, plan.ws_counter_bytes, stream) != cudaSuccess) {
@@ -91,7 +91,7 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint
         }
     }
     nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0,
-                        plan.splits > 1 ? scratch : nullptr, err_word};
+                        plan.ws_bytes > 0 ? scratch : nullptr, err_word};
     bool enc_failed = false;
     cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
     if (enc_failed) return NVFP4_ERR_CUDA;

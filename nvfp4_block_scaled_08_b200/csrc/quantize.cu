@@ -12,6 +12,10 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <cooperative_groups.h>
+
+#include <algorithm>
+#include <cstring>
 
 #include "internal.h"
 
@@ -70,41 +74,132 @@ template <> struct InTraits<__nv_bfloat16> {
     }
 };
 
-// ------------------------------------------------------------------ global scale
+// ------------------------------------------------------------------ indexing
+
+// A [rows, K] tensor of T (row stride ld) is read as 16-byte vectors, vpr = K / V per row.
+// Grids are 2-D: blockIdx.y strides over rows, blockIdx.x * blockDim.x + threadIdx.x over
+// the vectors of a row, so no index needs a division.
+
+__device__ __forceinline__ float block_max(float m, float* red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.0f;
+    if (threadIdx.x < 32) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (threadIdx.x == 0) red[0] = m;
+    }
+    __syncthreads();
+    m = red[0];
+    __syncthreads();
+    return m;
+}
 
 template <typename T>
-__global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int64_t numel,
-                                                   unsigned* __restrict__ acc_bits)
+__device__ __forceinline__ float amax_partial(const T* x, uint32_t rows, uint32_t vpr, int64_t ld)
 {
     constexpr int V = InTraits<T>::kPerThread;
     float m = 0.0f;
-    const int64_t nvec = numel / V;
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec; i += stride) {
-        float v[V];
-        InTraits<T>::load(x + i * V, v);
+    const uint32_t cstride = gridDim.x * blockDim.x;
+    for (uint32_t r = blockIdx.y; r < rows; r += gridDim.y) {
+        const T* row = x + static_cast<int64_t>(r) * ld;
+        for (uint32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < vpr; c += cstride) {
+            float v[V];
+            InTraits<T>::load(row + static_cast<int64_t>(c) * V, v);
 #pragma unroll
-        for (int k = 0; k < V; ++k) m = fmaxf(m, fabsf(v[k]));
+            for (int k = 0; k < V; ++k) m = fmaxf(m, fabsf(v[k]));
+        }
     }
-    // scalar tail
-    for (int64_t i = nvec * V + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < numel; i += stride) {
-        float f;
-        if constexpr (sizeof(T) == 4) f = x[i];
-        else f = __bfloat162float(x[i]);
-        m = fmaxf(m, fabsf(f));
+    return m;
+}
+
+// Quantise every row. The TPB lanes that share a 16-element block are consecutive lanes of
+// one warp in the same iteration (vpr is a multiple of TPB and the column stride a multiple
+// of 32); the first of them computes the block scale and shares it.
+// Per block, in fp32 with explicit rounding and in this order:
+//   amax -> s = e4m3(amax / 6 * gs) -> r = s ? gs / s : 0 -> codes e2m1(x * r).
+template <typename T>
+__device__ __forceinline__ void quantize_rows(const T* __restrict__ x, uint32_t rows, uint32_t vpr,
+                                              int64_t ld, int64_t K, float gs,
+                                              uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
+{
+    constexpr int V = InTraits<T>::kPerThread;   // elements per thread
+    constexpr int TPB = 16 / V;                  // threads per 16-element block
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t cstride = gridDim.x * blockDim.x;
+    const uint32_t c_first = blockIdx.x * blockDim.x + threadIdx.x;
+    for (uint32_t r = blockIdx.y; r < rows; r += gridDim.y) {
+        const T* row = x + static_cast<int64_t>(r) * ld;
+        uint8_t* qrow = q + static_cast<int64_t>(r) * (K / 2);
+        uint8_t* sfrow = sf + static_cast<int64_t>(r) * (K / 16);
+        for (uint32_t cbase = c_first - lane; cbase < vpr; cbase += cstride) {   // warp-uniform
+            const uint32_t c = cbase + lane;
+            const bool valid = c < vpr;
+            float v[V];
+            if (valid) {
+                InTraits<T>::load(row + static_cast<int64_t>(c) * V, v);
+            } else {
+#pragma unroll
+                for (int k = 0; k < V; ++k) v[k] = 0.0f;
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int k = 0; k < V; ++k) amax = fmaxf(amax, fabsf(v[k]));
+#pragma unroll
+            for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+
+            uint32_t sfq = 0;
+            float rcp = 0.0f;
+            if ((lane & (TPB - 1)) == 0) {
+                const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+                sfq = f32_to_e4m3(sf32);
+                const float sfd = e4m3_to_f32(sfq);
+                rcp = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
+            }
+            const uint32_t leader = lane & ~static_cast<uint32_t>(TPB - 1);
+            rcp = __shfl_sync(0xffffffffu, rcp, leader);
+
+            uint32_t packed = 0;
+#pragma unroll
+            for (int k = 0; k < V; k += 2)
+                packed |= f32x2_to_e2m1x2(__fmul_rn(v[k], rcp), __fmul_rn(v[k + 1], rcp)) << (4 * k);
+            if (valid) {
+                uint8_t* dst = qrow + static_cast<int64_t>(c) * (V / 2);
+                if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+                else *reinterpret_cast<uint32_t*>(dst) = packed;
+                if ((lane & (TPB - 1)) == 0) sfrow[c / TPB] = static_cast<uint8_t>(sfq);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ global scale
+
+template <typename T>
+__global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, uint32_t rows, uint32_t vpr,
+                                                   int64_t ld, unsigned* __restrict__ acc_bits)
+{
+    __shared__ float red[32];
+    float m = amax_partial(x, rows, vpr, ld);
+    m = block_max(m, red);
+    // non-negative floats order like their bit patterns
+    if (threadIdx.x == 0) atomicMax(acc_bits, __float_as_uint(m));
+}
+
+template <typename T>
+__global__ void amax_tail_kernel(const T* __restrict__ x, int n, unsigned* __restrict__ acc_bits)
+{
+    float m = 0.0f;
+    if (static_cast<int>(threadIdx.x) < n) {
+        if constexpr (sizeof(T) == 4) m = fabsf(x[threadIdx.x]);
+        else m = fabsf(__bfloat162float(x[threadIdx.x]));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    __shared__ float warp_max[8];
-    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        m = threadIdx.x < (blockDim.x >> 5) ? warp_max[threadIdx.x] : 0.0f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        // non-negative floats order like their bit patterns
-        if (threadIdx.x == 0) atomicMax(acc_bits, __float_as_uint(m));
-    }
+    if (threadIdx.x == 0) atomicMax(acc_bits, __float_as_uint(m));
 }
 
 // gs = 2688 / amax (448 * 6), or 1 if the tensor is all zero; in place over the amax bits.
@@ -123,56 +218,50 @@ __global__ void alpha_kernel(const float* __restrict__ gs_a, const float* __rest
 
 // ------------------------------------------------------------------ quantisation
 
-// TPB consecutive threads share one 16-element block; each loads 16 bytes of input.
 template <typename T>
-__global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, int64_t rows, int64_t K,
-                                                       int64_t ldx, const float* __restrict__ gs_ptr,
+__global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, uint32_t rows, uint32_t vpr,
+                                                       int64_t ldx, int64_t K, const float* __restrict__ gs_ptr,
                                                        uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
 {
-    constexpr int V = InTraits<T>::kPerThread;   // elements per thread
-    constexpr int TPB = 16 / V;                  // threads per 16-element block
-    const int64_t nblk_row = K / 16;
-    const int64_t total = rows * nblk_row * TPB; // multiple of TPB
-    const float gs = __ldg(gs_ptr);
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    // warp-uniform trip count: lanes past the end compute on zeros and store nothing
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
-         base < total; base += stride) {
-        const int64_t g = base + (threadIdx.x & 31);
-        const bool valid = g < total;
-        const int64_t blk = g / TPB;
-        const int sub = static_cast<int>(g % TPB);
-        const int64_t r = blk / nblk_row;
-        const int64_t j = blk - r * nblk_row;
-        float v[V];
-        if (valid) {
-            InTraits<T>::load(x + r * ldx + j * 16 + sub * V, v);
-        } else {
-#pragma unroll
-            for (int k = 0; k < V; ++k) v[k] = 0.0f;
-        }
-        float amax = 0.0f;
-#pragma unroll
-        for (int k = 0; k < V; ++k) amax = fmaxf(amax, fabsf(v[k]));
-#pragma unroll
-        for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    quantize_rows(x, rows, vpr, ldx, K, __ldg(gs_ptr), q, sf);
+}
 
-        const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
-        const uint32_t sfq = f32_to_e4m3(sf32);
-        const float sfd = e4m3_to_f32(sfq);
-        const float rcp = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
+// One cooperative launch: amax of the whole tensor -> grid barrier -> global scale (and the
+// GEMM alpha against other tensors' global scales) -> grid barrier -> quantisation. The
+// per-block partial maxima are parked in the first bytes of q (overwritten afterwards by
+// the codes); the launcher keeps gridDim.x * 4 <= rows * K / 2.
+template <typename T>
+__global__ void __launch_bounds__(512) quantize_dynamic_kernel(
+    const T* __restrict__ x, uint32_t rows, uint32_t vpr, int64_t ldx, int64_t K,
+    float* __restrict__ gs_out, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+    const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out)
+{
+    namespace cg = cooperative_groups;
+    cg::grid_group grid = cg::this_grid();
+    __shared__ float red[32];
+    float* partial = reinterpret_cast<float*>(q);
+    const uint32_t nblocks = gridDim.x * gridDim.y;
+    const uint32_t bid = blockIdx.y * gridDim.x + blockIdx.x;
 
-        uint32_t packed = 0;
-#pragma unroll
-        for (int k = 0; k < V; k += 2)
-            packed |= f32x2_to_e2m1x2(__fmul_rn(v[k], rcp), __fmul_rn(v[k + 1], rcp)) << (4 * k);
-        if (valid) {
-            uint8_t* dst = q + r * (K / 2) + j * 8 + sub * (V / 2);
-            if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
-            else *reinterpret_cast<uint32_t*>(dst) = packed;
-            if (sub == 0) sf[r * nblk_row + j] = static_cast<uint8_t>(sfq);
-        }
+    float m = amax_partial(x, rows, vpr, ldx);
+    m = block_max(m, red);
+    if (threadIdx.x == 0) partial[bid] = m;
+    grid.sync();
+
+    float a = 0.0f;
+    for (uint32_t i = threadIdx.x; i < nblocks; i += blockDim.x) a = fmaxf(a, __ldcg(partial + i));
+    a = block_max(a, red);
+    const float gs = (a == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, a);
+    if (bid == 0) {
+        if (threadIdx.x == 0) *gs_out = gs;
+        for (int32_t i = threadIdx.x; i < n_alpha; i += blockDim.x)
+            alpha_out[i] = __fdiv_rn(1.0f, __fmul_rn(gs, gs_other[i]));
     }
+    grid.sync();   // every block has read the partial maxima before q is overwritten
+    // a dependent GEMM may start its prologue now (it waits for this grid before reading)
+    cudaTriggerProgrammaticLaunchCompletion();
+
+    quantize_rows(x, rows, vpr, ldx, K, gs, q, sf);
 }
 
 // ------------------------------------------------------------------ elementwise conversions
@@ -193,6 +282,18 @@ __global__ void round_e2m1_kernel(const float* __restrict__ x, int64_t n, uint8_
 
 // ------------------------------------------------------------------ launchers
 
+// 2-D grid for a [rows, vpr-vector] sweep with 512-thread blocks, at most `cap` blocks.
+static dim3 grid_2d(int64_t rows, int64_t vpr, int64_t cap)
+{
+    int64_t gx = (vpr + 511) / 512;
+    if (gx > cap) gx = cap;
+    if (gx < 1) gx = 1;
+    int64_t gy = std::min<int64_t>(rows, std::max<int64_t>(cap / gx, 1));
+    gy = std::min<int64_t>(gy, 65535);
+    if (gy < 1) gy = 1;
+    return dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), 1);
+}
+
 static int grid_for(int64_t threads, int num_sms)
 {
     int64_t blocks = (threads + 255) / 256;
@@ -208,15 +309,36 @@ cudaError_t launch_global_scale(const void* x, bool bf16, int64_t numel, float* 
     cudaError_t e = cudaMemsetAsync(gs, 0, sizeof(float), stream);
     if (e != cudaSuccess) return e;
     if (numel > 0) {
-        const int grid = grid_for(numel / (bf16 ? 8 : 4) + 1, num_sms);
-        if (bf16)
-            amax_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-                static_cast<const __nv_bfloat16*>(x), numel, reinterpret_cast<unsigned*>(gs));
-        else
-            amax_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), numel,
-                                                         reinterpret_cast<unsigned*>(gs));
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+        // numel elements viewed as one row of 16-byte vectors, plus a scalar tail
+        const int V = bf16 ? 8 : 4;
+        const int64_t nvec = numel / V;
+        if (nvec > 0) {
+            if (nvec >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
+            const dim3 grid = grid_2d(1, nvec, static_cast<int64_t>(num_sms) * 4);
+            if (bf16)
+                amax_kernel<__nv_bfloat16><<<grid, 512, 0, stream>>>(
+                    static_cast<const __nv_bfloat16*>(x), 1u, static_cast<uint32_t>(nvec), 0,
+                    reinterpret_cast<unsigned*>(gs));
+            else
+                amax_kernel<float><<<grid, 512, 0, stream>>>(
+                    static_cast<const float*>(x), 1u, static_cast<uint32_t>(nvec), 0,
+                    reinterpret_cast<unsigned*>(gs));
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        const int64_t tail = numel - nvec * V;
+        if (tail > 0) {
+            if (bf16)
+                amax_tail_kernel<__nv_bfloat16><<<1, 32, 0, stream>>>(
+                    static_cast<const __nv_bfloat16*>(x) + nvec * V, static_cast<int>(tail),
+                    reinterpret_cast<unsigned*>(gs));
+            else
+                amax_tail_kernel<float><<<1, 32, 0, stream>>>(
+                    static_cast<const float*>(x) + nvec * V, static_cast<int>(tail),
+                    reinterpret_cast<unsigned*>(gs));
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
     }
     global_scale_finalize_kernel<<<1, 1, 0, stream>>>(gs);
     return cudaGetLastError();
@@ -226,17 +348,63 @@ cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, i
                             const float* gs, uint8_t* q, uint8_t* sf, cudaStream_t stream,
                             int num_sms)
 {
-    const int tpb = bf16 ? 2 : 4;
-    const int64_t threads = rows * (K / 16) * tpb;
-    if (threads == 0) return cudaSuccess;
-    const int grid = grid_for(threads, num_sms);
+    const int V = bf16 ? 8 : 4;
+    const int64_t vpr = K / V;
+    if (rows == 0 || vpr == 0) return cudaSuccess;
+    const dim3 grid = grid_2d(rows, vpr, static_cast<int64_t>(num_sms) * 4);
     if (bf16)
-        quantize_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), rows, K, ldx, gs, q, sf);
+        quantize_kernel<__nv_bfloat16><<<grid, 512, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<uint32_t>(rows),
+            static_cast<uint32_t>(vpr), ldx, K, gs, q, sf);
     else
-        quantize_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), rows, K,
-                                                         ldx, gs, q, sf);
+        quantize_kernel<float><<<grid, 512, 0, stream>>>(static_cast<const float*>(x),
+                                                         static_cast<uint32_t>(rows),
+                                                         static_cast<uint32_t>(vpr), ldx, K, gs, q, sf);
     return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64_t ldx, int64_t K,
+                                    float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
+                                    int32_t n_alpha, float* alpha_out, int64_t q_bytes,
+                                    cudaStream_t stream, int num_sms)
+{
+    auto kern = quantize_dynamic_kernel<T>;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 512, 0);
+    if (e != cudaSuccess) return e;
+    // co-resident blocks only (cooperative), few of them (cheap grid barriers), and room
+    // for one partial maximum per block in q
+    int64_t cap = static_cast<int64_t>(std::min(std::max(per_sm, 1), 2)) * num_sms;
+    cap = std::min<int64_t>(cap, std::max<int64_t>(q_bytes / 4, 1));
+    const dim3 grid = grid_2d(rows, vpr, cap);
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(512, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeCooperative;
+    attr.val.cooperative = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, x, static_cast<uint32_t>(rows), static_cast<uint32_t>(vpr),
+                              ldx, K, gs_out, q, sf, gs_other, n_alpha, alpha_out);
+}
+
+cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
+                                    float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
+                                    int32_t n_alpha, float* alpha_out, cudaStream_t stream,
+                                    int num_sms)
+{
+    const int V = bf16 ? 8 : 4;
+    const int64_t vpr = K / V;
+    const int64_t q_bytes = rows * (K / 2);
+    if (bf16)
+        return launch_dynamic_t(static_cast<const __nv_bfloat16*>(x), rows, vpr, ldx, K, gs_out, q, sf,
+                                gs_other, n_alpha, alpha_out, q_bytes, stream, num_sms);
+    return launch_dynamic_t(static_cast<const float*>(x), rows, vpr, ldx, K, gs_out, q, sf, gs_other,
+                            n_alpha, alpha_out, q_bytes, stream, num_sms);
 }
 
 cudaError_t launch_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,

@@ -102,6 +102,15 @@ def test_quantize_host_validation(lib):
     assert gs(0x1004, 0, 16, 0x2000, None) == 3
 
 
+def test_quantize_dynamic_host_validation(lib):
+    f = lib.nvfp4_quantize_dynamic
+    assert f(0x1000, 0, 4, 64, 64, None, 0x3000, 0x4000, None, 0, None, None) == 1     # gs_out
+    assert f(0x1000, 0, 4, 64, 64, 0x2000, 0x3000, 0x4000, None, 2, 0x5000, None) == 1 # gs_other
+    assert f(0x1000, 0, 0, 64, 64, 0x2000, 0x3000, 0x4000, None, 0, None, None) == 2   # empty
+    assert f(0x1000, 0, 4, 24, 24, 0x2000, 0x3000, 0x4000, None, 0, None, None) == 2   # K % 16
+    assert f(0x1004, 0, 4, 64, 64, 0x2000, 0x3000, 0x4000, None, 0, None, None) == 3
+
+
 def test_round_and_alpha_host_validation(lib):
     assert lib.nvfp4_round_e4m3(None, 4, 0x1000, None) == 1
     assert lib.nvfp4_round_e2m1(0x1000, -1, 0x1000, None) == 1

@@ -144,25 +144,37 @@ def test_one_hot_rows_bit_exact(cuda_device, M, N, K):
         np.testing.assert_array_equal(bf16_bits_of(out), want)
 
 
-def test_split_k_deterministic_and_within_tolerance(cuda_device):
+@pytest.mark.parametrize("cluster,groups", [(1, 1), (8, 1), (2, 6), (1, 12)])
+def test_split_k_deterministic_and_within_tolerance(cuda_device, monkeypatch, cluster, groups):
     c = workloads.attn_proj_cases()[0]          # M = 16: the most split-heavy shape
+    monkeypatch.setenv("NVFP4_CLUSTER", str(cluster))
+    monkeypatch.setenv("NVFP4_GROUPS", str(groups))
     a, b = c.a(), c.b()
     d = cuda_device
     Aq, sfA, gsA = gpu_quantize(a, d)
     Bq, sfB, gsB = gpu_quantize(b, d)
     al = nv.alpha(gsA, gsB)
-    assert nv.gemm_workspace_size(c.M, c.N, c.K) > 0
+    assert (nv.gemm_workspace_size(c.M, c.N, c.K) > 0) == (groups > 1)
     ws = nv.make_workspace(c.M, c.N, c.K, d)
     o1 = nv.gemm(Aq, sfA, Bq, sfB, al, workspace=ws)
     o2 = nv.gemm(Aq, sfA, Bq, sfB, al, workspace=ws)
-    o3 = nv.gemm(Aq, sfA, Bq, sfB, al, workspace=None)
-    o4 = nv.gemm(Aq, sfA, Bq, sfB, al, workspace=None)
     assert torch.equal(bf16_bits_tensor(o1), bf16_bits_tensor(o2))
-    assert torch.equal(bf16_bits_tensor(o3), bf16_bits_tensor(o4))
     qa, sa, qb, sb, alo = _oracle_operands(a, b)
     v, S, _ = oracle.gemm(qa, sa, qb, sb, alo)
-    check_within_tolerance(o1, v, S, alo, "split-K")
-    check_within_tolerance(o3, v, S, alo, "no split")
+    check_within_tolerance(o1, v, S, alo, f"split-K cluster={cluster} groups={groups}")
+
+
+@pytest.mark.parametrize("cluster,groups", [(2, 1), (3, 1), (4, 1), (8, 1), (2, 3), (3, 2), (1, 5)])
+@pytest.mark.parametrize("M,N,K", [(16, 768, 6144), (256, 768, 6144), (130, 776, 2560),
+                                   (40, 264, 4096)])
+def test_split_k_layouts(cuda_device, monkeypatch, cluster, groups, M, N, K):
+    """Every cluster / group layout of split-K (distributed-shared-memory reduction inside
+    a cluster, workspace reduction across clusters) against the oracle."""
+    monkeypatch.setenv("NVFP4_CLUSTER", str(cluster))
+    monkeypatch.setenv("NVFP4_GROUPS", str(groups))
+    a = workloads.normal(M, K, 1.0, M + 3 * N)
+    b = workloads.normal(N, K, 0.02, N + 5 * K)
+    run_case(cuda_device, a, b, use_ws=True)
 
 
 def bf16_bits_tensor(t):
@@ -184,7 +196,9 @@ def test_transposed_product_agrees(cuda_device):
     check_within_tolerance(o2.t().contiguous(), v, S, alo, "(B A^T)^T")
 
 
-def test_workspace_too_small_is_rejected(cuda_device):
+def test_workspace_too_small_is_rejected(cuda_device, monkeypatch):
+    monkeypatch.setenv("NVFP4_CLUSTER", "2")
+    monkeypatch.setenv("NVFP4_GROUPS", "4")
     n = nv.gemm_workspace_size(16, 768, 6144)
     assert n > 0
     d = cuda_device

@@ -107,3 +107,32 @@ def test_rounding_exhaustive_all_finite_fp32(cuda_device, kind):
             raise AssertionError(f"{kind}: {int(mism.sum())} mismatches in chunk {start:#x}, e.g. "
                                  f"{[(float(xh[j]), int(got[j]), int(want[j])) for j in i]}")
         del x
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("rows,K", [(1, 16), (16, 6144), (64, 6144), (1024, 6144), (17, 48),
+                                    (257, 2048), (3, 16)])
+def test_quantize_dynamic_matches_oracle(cuda_device, dtype, rows, K):
+    xc = workloads.normal(rows, K, 1.0, rows * 31 + K)
+    gb = torch.tensor([3.5, 700.25], device=cuda_device)
+    q, sf, gs, al = nv.quantize_dynamic(xc.to(dtype).to(cuda_device), gs_other=gb)
+    qo, sfo, gso = oracle_quantize(xc, dtype)
+    assert np.float32(gs.item()) == gso
+    np.testing.assert_array_equal(sf.cpu().numpy(), sfo)
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    al = al.cpu().numpy()
+    assert al[0] == oracle.alpha(gso, 3.5) and al[1] == oracle.alpha(gso, 700.25)
+
+
+def test_quantize_dynamic_zero_tensor_and_row_stride(cuda_device):
+    q, sf, gs, al = nv.quantize_dynamic(torch.zeros(5, 256, device=cuda_device))
+    assert gs.item() == 1.0 and al is None
+    assert (q == 0).all() and (sf == 0).all()
+    xc = workloads.normal(40, 512, 1.0, 19)
+    big = torch.zeros(40, 640)
+    big[:, :512] = xc
+    q, sf, gs, _ = nv.quantize_dynamic(big.to(cuda_device)[:, :512])
+    qo, sfo, gso = oracle_quantize(xc)
+    assert np.float32(gs.item()) == gso
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(sf.cpu().numpy(), sfo)

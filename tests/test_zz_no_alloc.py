@@ -34,10 +34,15 @@ def _call_noalloc(lib, Aq, sfA, Bq, sfB, al, out, M, N, K):
 
 @pytest.mark.parametrize("case", workloads.attn_proj_cases()[:3] + workloads.moe_expert_cases()[1:2],
                          ids=lambda c: c.name)
-def test_noalloc_matches_gemm_on_two_calls(cuda_device, case):
+@pytest.mark.parametrize("layout", ["planned", "workspace"])
+def test_noalloc_matches_gemm_on_two_calls(cuda_device, case, layout, monkeypatch):
     d = cuda_device
     M, N, K = case.M, case.N, case.K
-    assert nv.gemm_workspace_size(M, N, K) > 0, "shape must exercise the split-K scratch"
+    if layout == "workspace":
+        # split-K across several clusters per tile, so the partials go through the scratch
+        monkeypatch.setenv("NVFP4_CLUSTER", "2")
+        monkeypatch.setenv("NVFP4_GROUPS", "3")
+        assert nv.gemm_workspace_size(M, N, K) > 0, "shape must exercise the split-K scratch"
     a, b = case.a(), case.b()
     Aq, sfA, gsA = gpu_quantize(a, d)
     Bq, sfB, gsB = gpu_quantize(b, d)
@@ -66,8 +71,9 @@ def test_noalloc_matches_gemm_on_two_calls(cuda_device, case):
 
 def test_noalloc_rejects_scratch_beyond_the_fixed_array(cuda_device, monkeypatch):
     d = cuda_device
-    # force 24-way split-K on 1024 x 768 x 6144: 48 tiles x 24 x 64 KB of partials > 16 MiB
-    monkeypatch.setenv("NVFP4_SPLITS", "24")
+    # force 24 cluster groups per tile on 1024 x 768 x 6144: 48 tiles x 24 x 64 KB > 16 MiB
+    monkeypatch.setenv("NVFP4_CLUSTER", "1")
+    monkeypatch.setenv("NVFP4_GROUPS", "24")
     M, N, K = 1024, 768, 6144
     Aq = torch.zeros(M, K // 2, dtype=torch.uint8, device=d)
     sfA = torch.zeros(M, K // 16, dtype=torch.uint8, device=d)
