@@ -7,11 +7,15 @@ M in {16, 64, 256, 1024}, A ~ N(0,1) fp32 activations, B ~ N(0,0.02) weights qua
 once to NVFP4 outside the timed region. One step = for every M: per-tensor global scale
 of A, alpha = 1/(gsA gsB), NVFP4 quantisation of A, block-scaled GEMM -> bf16.
 
-Timing: the step is captured once as a CUDA graph (with event-record nodes around every
-GEMM); W warm-up replays, then exactly K timed replays bracketed by a barrier and a
-device synchronise, each replay preceded by an untimed L2 flush (a 512 MB write, larger
-than the 126 MB L2). Step time = sum of the per-replay CUDA-event durations, max over
-ranks. SM clocks and throttle reasons are polled through NVML during the timed bracket.
+Timing: the step is captured as a CUDA graph (with event-record nodes around every kernel
+group). Inputs are larger than L2: 8 independent input sets of the sweep (activations,
+weights, outputs; about 37 MiB each, 300 MiB in all, "layers" with different seeds) are
+replayed in rotation, so each step's data was last touched 7 steps (about 260 MiB) earlier
+and comes from HBM. --flush instead flushes L2 before every step (a 512 MB write, then a
+256 MB read), which also evicts kernel code and tensor maps. W warm-up replays, then exactly
+K timed replays bracketed by a barrier and a device synchronise; step time = sum of the
+per-replay CUDA-event durations, max over ranks. SM clocks and throttle reasons are polled
+through NVML during the timed bracket.
 
 e2e: the same metric through the public Python API called eagerly per step, with the
 activations copied from pinned host memory and the outputs copied back inside the timed
@@ -75,9 +79,15 @@ def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> float:
+    """TFLOP/s of the whole job: every rank's work over the slowest rank's step time."""
+    return flops_per_rank * world / (step_ms_max * 1e-3) / 1e12
 
 
 def measured_peaks():
@@ -194,20 +204,23 @@ def roofline_us(flops, nbytes, peaks):
 class AttnSweep:
     """Resident inputs, outputs and workspaces of the attention-projection sweep."""
 
-    def __init__(self, dev, rank):
+    def __init__(self, dev, rank, set_index=0):
         import nvfp4_block_scaled_08_b200 as nv
         from nvfp4_block_scaled_08_b200 import workloads
         self.nv = nv
         self.dev = dev
         cases = workloads.attn_proj_cases()
-        b = cases[0].b()                     # the same weights for every M
+        # set 0 is the canonical seeded case; the other sets (other "layers") differ only in
+        # their seeds
+        b = cases[0].b() if set_index == 0 else workloads.normal(
+            N_ATTN, K_ATTN, 0.02, cases[0].seed + 1 + 7919 * set_index)   # same weights for every M
         bd = b.to(dev)
         self.gsB = nv.global_scale(bd)
         self.Bq, self.sfB = nv.quantize(bd, self.gsB)
         del bd
         self.items = []
         for c in cases:
-            a_cpu = c.a()
+            a_cpu = c.a() if set_index == 0 else workloads.normal(c.M, K_ATTN, 1.0, c.seed + 7919 * set_index)
             it = {
                 "M": c.M, "a_cpu": a_cpu.pin_memory(),
                 "a": a_cpu.to(dev),
@@ -273,23 +286,27 @@ class AttnSweep:
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     peaks = measured_peaks()
-    sweep = AttnSweep(dev, rank)
-    graph = sweep.capture()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    clean = torch.ones(CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
+    nsets = 1 if args.flush else args.sets
+    sets = [AttnSweep(dev, rank, i) for i in range(nsets)]
+    graphs = [sw.capture() for sw in sets]
+    sweep = sets[0]
     stream = torch.cuda.current_stream()
+    if args.flush:
+        flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        clean = torch.ones(CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
 
-    def flush_l2():
-        # write a buffer 4x the L2, then read another 2x the L2, so the timed step starts
-        # with none of its data cached and no dirty lines left to write back
-        flush.zero_()
-        torch.sum(clean)
+    def before_step():
+        if args.flush:
+            # write a buffer 4x the L2, then read another 2x the L2: the step starts with
+            # nothing cached (data, kernel code and tensor maps alike) and no dirty lines
+            flush.zero_()
+            torch.sum(clean)
 
     clocks = ClockSampler(local)
     clocks.start()
-    for _ in range(args.warmup):
-        flush_l2()
-        graph.replay()
+    for i in range(args.warmup):
+        before_step()
+        graphs[i % nsets].replay()
     torch.cuda.synchronize()
 
     start = torch.cuda.Event(enable_timing=True)
@@ -299,23 +316,26 @@ def run_ours(args, world, rank, local):
     total_ms = 0.0
     barrier(world)
     clocks.mark()
-    for _ in range(args.steps):
-        flush_l2()                         # untimed: evicts the previous step from L2
+    for i in range(args.steps):
+        k = i % nsets                      # each set was last touched nsets - 1 steps ago
+        before_step()
         start.record(stream)
-        graph.replay()
+        graphs[k].replay()
         end.record(stream)
         end.synchronize()                  # read this replay's in-graph event timestamps
         total_ms += start.elapsed_time(end)
-        for j, ev in enumerate(sweep.ev):
+        for j, ev in enumerate(sets[k].ev):
             quant_ms[j] += ev[0].elapsed_time(ev[1]) / args.steps
             gemm_ms[j] += ev[1].elapsed_time(ev[2]) / args.steps
     barrier(world)
     clocks.mark()
     clocks.stop()
     step_ms = total_ms / args.steps
+    set_bytes = sum(it["a"].numel() * 4 + it["q"].numel() + it["sf"].numel() + it["out"].numel() * 2
+                    for it in sweep.items) + sweep.Bq.numel() + sweep.sfB.numel()
 
     step_ms = max_over_ranks(step_ms, world)
-    value = sweep.flops * world / (step_ms * 1e-3) / 1e12
+    value = whole_job_value(sweep.flops, step_ms, world)
 
     # e2e through the public API with host buffers
     e2e_start = torch.cuda.Event(enable_timing=True)
@@ -329,7 +349,7 @@ def run_ours(args, world, rank, local):
     e2e_end.record(stream)
     barrier(world)
     e2e_ms = max_over_ranks(e2e_start.elapsed_time(e2e_end) / args.steps, world)
-    e2e_value = sweep.flops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = whole_job_value(sweep.flops, e2e_ms, world)
 
     # roofline: per shape, and for the dominant kernel family
     per_shape = []
@@ -372,7 +392,10 @@ def run_ours(args, world, rank, local):
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
         "config": {"workload": "attn_proj_sweep N=768 K=6144 M={16,64,256,1024}",
                    "step": "per M: quantize_dynamic(A fp32: global scale, alpha, codes) + gemm; one CUDA graph",
-                   "l2": "flushed before every timed step (512 MB write, then 256 MB read)",
+                   "l2": ("flushed before every timed step (512 MB write, then 256 MB read)" if args.flush else
+                          f"inputs larger than L2: {nsets} independent input sets of {set_bytes / 2**20:.0f} MiB "
+                          f"(activations, weights, outputs) in rotation, {nsets * set_bytes / 2**20:.0f} MiB "
+                          "in all, so each set was last touched nsets-1 steps ago"),
                    "parallelism": f"replicas x{world}"},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": sweep.h2d_bytes, "d2h_bytes_per_step": sweep.d2h_bytes,
@@ -386,17 +409,18 @@ def run_ours(args, world, rank, local):
     }
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
-    del graph
-    sweep.graph = None
+    for sw in sets:
+        sw.graph = None
+    del graphs
     return line
 
 
 # ------------------------------------------------------------------ the oracle (CPU)
 
 def oracle_sweep_sample(budget_s: float):
-    """Time the oracle on a bounded sample of the sweep: every M, the first r rows of A
-    (r chosen from a calibration so the sample takes about budget_s)."""
-    import numpy as np
+    """Time the oracle on a bounded sample of the sweep: for every M, the first r rows of A
+    (global scale over the full A), repeated until about budget_s has passed. r is the full
+    M when one pass over the whole sweep fits in the budget, else a proportional share."""
     import oracle
     from nvfp4_block_scaled_08_b200 import workloads
     cases = workloads.attn_proj_cases()
@@ -405,25 +429,33 @@ def oracle_sweep_sample(budget_s: float):
     qb, sb = oracle.quantize(b, gb)               # weights: once, outside the timing
     a_all = [c.a().numpy() for c in cases]
     threads = os.cpu_count() or 1
-    # calibration: 8 rows of the largest case
+
+    def one_pass(rows):
+        f = 0.0
+        for a, r in zip(a_all, rows):
+            ga = oracle.global_scale(a)
+            qa, sa = oracle.quantize(a[:r], ga)
+            oracle.gemm(qa, sa, qb, sb, oracle.alpha(ga, gb), threads=threads)
+            f += 2.0 * r * N_ATTN * K_ATTN
+        return f
+
+    # calibration: one pass over 64 rows of every M
     t0 = time.perf_counter()
-    oracle.gemm(*oracle.quantize(a_all[-1][:8], oracle.global_scale(a_all[-1])), qb, sb, 1.0,
-                threads=threads)
-    per_row = (time.perf_counter() - t0) / 8
+    one_pass([min(64, c.M) for c in cases])
+    per_row = (time.perf_counter() - t0) / sum(min(64, c.M) for c in cases)
     total_rows = sum(c.M for c in cases)
     frac = min(1.0, budget_s / max(per_row * total_rows, 1e-9))
     rows = [max(1, int(round(c.M * frac))) for c in cases]
+    flops, passes = 0.0, 0
     t0 = time.perf_counter()
-    flops = 0.0
-    for a, r in zip(a_all, rows):
-        ga = oracle.global_scale(a)
-        qa, sa = oracle.quantize(a[:r], ga)
-        al = oracle.alpha(ga, gb)
-        oracle.gemm(qa, sa, qb, sb, al, threads=threads)
-        flops += 2.0 * r * N_ATTN * K_ATTN
+    while True:
+        flops += one_pass(rows)
+        passes += 1
+        if time.perf_counter() - t0 >= 0.8 * budget_s:
+            break
     dt = time.perf_counter() - t0
     sample = (f"attn_proj sweep, first {rows} rows of M={list(M_SWEEP)} (global scale over the "
-              f"full A), N=768, K=6144; weights quantised outside timing")
+              f"full A), N=768, K=6144, {passes} pass(es); weights quantised outside timing")
     return flops, dt, threads, sample
 
 
@@ -471,6 +503,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sets", type=int, default=8,
+                    help="independent input sets rotated between steps (together larger than L2)")
+    ap.add_argument("--flush", action="store_true",
+                    help="flush L2 before every step instead of rotating input sets")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -235,6 +235,46 @@ __device__ __forceinline__ void store_out4(const GemmArgs& a, const Tile& ti, in
     }
 }
 
+// Store 16 consecutive accumulator columns (c .. c + 15) of P row `p` as bf16(alpha * v).
+template <class Cfg>
+__device__ __forceinline__ void store_out16(const GemmArgs& a, const Tile& ti, int p, int c,
+                                            const uint32_t (&r)[16], float alpha)
+{
+    if constexpr (!Cfg::SWAP) {
+        // thread owns output row m = p, columns n = q0 + c .. + 15 (N % 8 == 0)
+        const int n0 = ti.q0 + c;
+        if (p < a.M) {
+            __nv_bfloat16* dst = a.out + static_cast<size_t>(p) * a.N + n0;
+            uint4 w0, w1;
+            w0.x = pack_bf16x2(alpha * __uint_as_float(r[0]), alpha * __uint_as_float(r[1]));
+            w0.y = pack_bf16x2(alpha * __uint_as_float(r[2]), alpha * __uint_as_float(r[3]));
+            w0.z = pack_bf16x2(alpha * __uint_as_float(r[4]), alpha * __uint_as_float(r[5]));
+            w0.w = pack_bf16x2(alpha * __uint_as_float(r[6]), alpha * __uint_as_float(r[7]));
+            w1.x = pack_bf16x2(alpha * __uint_as_float(r[8]), alpha * __uint_as_float(r[9]));
+            w1.y = pack_bf16x2(alpha * __uint_as_float(r[10]), alpha * __uint_as_float(r[11]));
+            w1.z = pack_bf16x2(alpha * __uint_as_float(r[12]), alpha * __uint_as_float(r[13]));
+            w1.w = pack_bf16x2(alpha * __uint_as_float(r[14]), alpha * __uint_as_float(r[15]));
+            if (n0 < a.N) *reinterpret_cast<uint4*>(dst) = w0;
+            if (n0 + 8 < a.N) *reinterpret_cast<uint4*>(dst + 8) = w1;
+        }
+    } else {
+        // thread owns output column n = p; accumulator columns are output rows
+        const int n = p;
+        if (n < a.N) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int qi = c + j;
+                bool valid;
+                if constexpr (Cfg::GROUPED) valid = qi < ti.q_valid;
+                else valid = ti.q0 + qi < a.M;
+                if (valid)
+                    a.out[static_cast<size_t>(ti.q0 + qi) * a.N + n] =
+                        __float2bfloat16_rn(alpha * __uint_as_float(r[j]));
+            }
+        }
+    }
+}
+
 // Rows [chunk_begin(k), chunk_begin(k + 1)) of a 128-row tile belong to cluster rank k.
 __device__ __forceinline__ int chunk_begin(int k, int cs) { return (k * 128 + cs - 1) / cs; }
 
@@ -426,11 +466,13 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         tmem_alloc(s_tmem_base, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
-    // Everything above touches only this CTA's resources and the kernel parameters; from
-    // here on the kernel reads data that the previous kernel in the stream may have written.
-    grid_dependency_wait();
+    // Everything above touches only this CTA's resources and the kernel parameters. Reads of
+    // data the previous kernel in the stream may write come after grid_dependency_wait():
+    // here for the grouped offsets, in each role below for the rest (the MMA and scale
+    // warps read shared and tensor memory only).
     if constexpr (Cfg::GROUPED) {
         if (warp == 3) {
+            grid_dependency_wait();
             // Tiles per expert: (N / 128 weight tiles) x ceil(rows_e / BN) token tiles.
             const int E = args.num_experts;
             const int per = (E + 31) / 32;
@@ -477,6 +519,21 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         const uint64_t pol_keep = l2_policy_evict_last();     // activations: re-read
         const uint64_t pol_p = Cfg::SWAP ? pol_stream : pol_keep;
         const uint64_t pol_q = Cfg::SWAP ? pol_keep : pol_stream;
+        if constexpr (!Cfg::GROUPED) {
+            // Warm L2 with this CTA's first weight tiles while the previous kernel finishes
+            // (a prefetch only fills L2, the coherence point, so it cannot see stale data).
+            if (blockIdx.x < num_tiles && elect_one()) {
+                const Tile ti = decode_tile<Cfg>(args, blockIdx.x, s_prefix);
+                const int n = ti.kcnt < STAGES ? ti.kcnt : STAGES;
+                for (int ks = 0; ks < n; ++ks) {
+                    const int32_t kx = (ti.k0 + ks) * Cfg::BK_BYTES;
+                    if constexpr (Cfg::SWAP) tma_prefetch_2d(&tm_p, kx, ti.p0);
+                    else tma_prefetch_2d(&tm_q, kx, ti.q0);
+                }
+            }
+            __syncwarp();
+        }
+        grid_dependency_wait();
         uint32_t stage = 0, phase = 0, issued = 0;
         bool ok = true;
         for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -571,18 +628,24 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         // Arrives once every tcgen05 operation issued above has completed.
         if (elect_one()) mma_commit(mma_done_bar);
         __syncwarp();
-    } else if (warp == 2) {
+    } else if (warp == 2 || warp == 3) {
         // -------------------------------------------------------------- scale re-layout
         // The TMA wrote row r's 16 scale bytes (k-blocks 0..15 of the stage) at r * 16.
         // The MMA for k-step j (k-blocks 4j..4j+3) needs, per 128-row group, a 512-byte
         // block whose 16-byte row i holds the 4 scale bytes of rows i, i+32, i+64, i+96.
         // Each lane owns row i = lane: it reads its 4 rows (16 B each), transposes the
         // 4 x 4 words in registers and writes 4 blocks (one per k-step), in place.
-        uint32_t stage = 0, phase = 0;
+        // Warps 2 and 3 take alternate stages.
+        const uint32_t sf_warp = static_cast<uint32_t>(warp - 2);
+        uint32_t stage = 0, phase = 0, seq = 0;
         for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
             bool ok = true;
-            for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
+            for (int32_t ks = 0; ks < ti.kcnt; ++ks, ++seq) {
+                if ((seq & 1u) != sf_warp) {
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    continue;
+                }
                 ok = mbar_wait(&full_bar[stage], phase, ab, kErrSfFull);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
@@ -618,6 +681,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         }
     } else if (warp >= 4) {
         // -------------------------------------------------------------- epilogue
+        grid_dependency_wait();                    // alpha, out and the workspace
         const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
         const int row = 32 * quad + lane;          // accumulator row (P row within the tile)
         uint32_t acc = 0, acc_phase = 0;
@@ -644,42 +708,18 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                 if (split_k) split_k_epilogue<Cfg>(args, ti, smem, rx_bar, s_is_last, tacc, row, alpha, ab);
             }
 
-            for (int c = 0; c < n_cols && !split_k; c += 16) {
-                uint32_t r[16];
-                tmem_ld_32x32b_x16(tacc + c, r);
+            // two 16-column TMEM loads in flight per wait
+            for (int c0 = 0; c0 < n_cols && !split_k; c0 += 32) {
+                uint32_t r[2][16];
+                const bool two = c0 + 16 < n_cols;
+                tmem_ld_32x32b_x16(tacc + c0, r[0]);
+                if (two) tmem_ld_32x32b_x16(tacc + c0 + 16, r[1]);
                 tmem_ld_wait();
-                if constexpr (!Cfg::SWAP) {
-                    // thread owns output row m = p, columns n = q0 + c .. + 15
-                    const int n0 = ti.q0 + c;
-                    if (p < args.M) {
-                        __nv_bfloat16* dst = args.out + static_cast<size_t>(p) * args.N + n0;
-                        uint4 w0, w1;
-                        w0.x = pack_bf16x2(alpha * __uint_as_float(r[0]), alpha * __uint_as_float(r[1]));
-                        w0.y = pack_bf16x2(alpha * __uint_as_float(r[2]), alpha * __uint_as_float(r[3]));
-                        w0.z = pack_bf16x2(alpha * __uint_as_float(r[4]), alpha * __uint_as_float(r[5]));
-                        w0.w = pack_bf16x2(alpha * __uint_as_float(r[6]), alpha * __uint_as_float(r[7]));
-                        w1.x = pack_bf16x2(alpha * __uint_as_float(r[8]), alpha * __uint_as_float(r[9]));
-                        w1.y = pack_bf16x2(alpha * __uint_as_float(r[10]), alpha * __uint_as_float(r[11]));
-                        w1.z = pack_bf16x2(alpha * __uint_as_float(r[12]), alpha * __uint_as_float(r[13]));
-                        w1.w = pack_bf16x2(alpha * __uint_as_float(r[14]), alpha * __uint_as_float(r[15]));
-                        if (n0 < args.N) *reinterpret_cast<uint4*>(dst) = w0;
-                        if (n0 + 8 < args.N) *reinterpret_cast<uint4*>(dst + 8) = w1;
-                    }
-                } else {
-                    // thread owns output column n = p; columns of the accumulator are rows m
-                    const int n = p;
-                    if (n < args.N) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int qi = c + j;
-                            bool valid;
-                            if constexpr (Cfg::GROUPED) valid = qi < ti.q_valid;
-                            else valid = ti.q0 + qi < args.M;
-                            if (valid)
-                                args.out[static_cast<size_t>(ti.q0 + qi) * args.N + n] =
-                                    __float2bfloat16_rn(alpha * __uint_as_float(r[j]));
-                        }
-                    }
+                for (int h = 0; h < 2; ++h) {
+                    if (h == 1 && !two) break;
+                    const int c = c0 + 16 * h;
+                    store_out16<Cfg>(args, ti, p, c, r[h], alpha);
                 }
             }
             // Accumulator drained into registers / workspace: hand it back to the MMA warp.

@@ -16,8 +16,10 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace nvfp4 {
 
@@ -104,13 +106,24 @@ __device__ __forceinline__ float amax_partial(const T* x, uint32_t rows, uint32_
     constexpr int V = InTraits<T>::kPerThread;
     float m = 0.0f;
     const uint32_t cstride = gridDim.x * blockDim.x;
+    constexpr int U = 4;                     // independent loads in flight per thread
     for (uint32_t r = blockIdx.y; r < rows; r += gridDim.y) {
         const T* row = x + static_cast<int64_t>(r) * ld;
-        for (uint32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < vpr; c += cstride) {
-            float v[V];
-            InTraits<T>::load(row + static_cast<int64_t>(c) * V, v);
+        for (uint32_t c0 = blockIdx.x * blockDim.x + threadIdx.x; c0 < vpr; c0 += U * cstride) {
+            float v[U][V];
 #pragma unroll
-            for (int k = 0; k < V; ++k) m = fmaxf(m, fabsf(v[k]));
+            for (int u = 0; u < U; ++u) {
+                const uint32_t c = c0 + u * cstride;
+                if (c < vpr) InTraits<T>::load(row + static_cast<int64_t>(c) * V, v[u]);
+                else {
+#pragma unroll
+                    for (int k = 0; k < V; ++k) v[u][k] = 0.0f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int k = 0; k < V; ++k) m = fmaxf(m, fabsf(v[u][k]));
         }
     }
     return m;
@@ -135,42 +148,52 @@ __device__ __forceinline__ void quantize_rows(const T* __restrict__ x, uint32_t 
         const T* row = x + static_cast<int64_t>(r) * ld;
         uint8_t* qrow = q + static_cast<int64_t>(r) * (K / 2);
         uint8_t* sfrow = sf + static_cast<int64_t>(r) * (K / 16);
-        for (uint32_t cbase = c_first - lane; cbase < vpr; cbase += cstride) {   // warp-uniform
-            const uint32_t c = cbase + lane;
-            const bool valid = c < vpr;
-            float v[V];
-            if (valid) {
-                InTraits<T>::load(row + static_cast<int64_t>(c) * V, v);
-            } else {
+        constexpr int U = 4;                 // independent loads in flight per thread
+        for (uint32_t cb0 = c_first - lane; cb0 < vpr; cb0 += U * cstride) {   // warp-uniform
+            float v[U][V];
 #pragma unroll
-                for (int k = 0; k < V; ++k) v[k] = 0.0f;
+            for (int u = 0; u < U; ++u) {
+                const uint32_t c = cb0 + u * cstride + lane;
+                if (c < vpr) {
+                    InTraits<T>::load(row + static_cast<int64_t>(c) * V, v[u]);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < V; ++k) v[u][k] = 0.0f;
+                }
             }
-            float amax = 0.0f;
 #pragma unroll
-            for (int k = 0; k < V; ++k) amax = fmaxf(amax, fabsf(v[k]));
+            for (int u = 0; u < U; ++u) {
+                const uint32_t cbase = cb0 + u * cstride;
+                if (cbase >= vpr) break;             // warp-uniform
+                const uint32_t c = cbase + lane;
+                const bool valid = c < vpr;
+                float amax = 0.0f;
 #pragma unroll
-            for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                for (int k = 0; k < V; ++k) amax = fmaxf(amax, fabsf(v[u][k]));
+#pragma unroll
+                for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
 
-            uint32_t sfq = 0;
-            float rcp = 0.0f;
-            if ((lane & (TPB - 1)) == 0) {
-                const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
-                sfq = f32_to_e4m3(sf32);
-                const float sfd = e4m3_to_f32(sfq);
-                rcp = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
-            }
-            const uint32_t leader = lane & ~static_cast<uint32_t>(TPB - 1);
-            rcp = __shfl_sync(0xffffffffu, rcp, leader);
+                uint32_t sfq = 0;
+                float rcp = 0.0f;
+                if ((lane & (TPB - 1)) == 0) {
+                    const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+                    sfq = f32_to_e4m3(sf32);
+                    const float sfd = e4m3_to_f32(sfq);
+                    rcp = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
+                }
+                const uint32_t leader = lane & ~static_cast<uint32_t>(TPB - 1);
+                rcp = __shfl_sync(0xffffffffu, rcp, leader);
 
-            uint32_t packed = 0;
+                uint32_t packed = 0;
 #pragma unroll
-            for (int k = 0; k < V; k += 2)
-                packed |= f32x2_to_e2m1x2(__fmul_rn(v[k], rcp), __fmul_rn(v[k + 1], rcp)) << (4 * k);
-            if (valid) {
-                uint8_t* dst = qrow + static_cast<int64_t>(c) * (V / 2);
-                if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
-                else *reinterpret_cast<uint32_t*>(dst) = packed;
-                if ((lane & (TPB - 1)) == 0) sfrow[c / TPB] = static_cast<uint8_t>(sfq);
+                for (int k = 0; k < V; k += 2)
+                    packed |= f32x2_to_e2m1x2(__fmul_rn(v[u][k], rcp), __fmul_rn(v[u][k + 1], rcp)) << (4 * k);
+                if (valid) {
+                    uint8_t* dst = qrow + static_cast<int64_t>(c) * (V / 2);
+                    if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+                    else *reinterpret_cast<uint32_t*>(dst) = packed;
+                    if ((lane & (TPB - 1)) == 0) sfrow[c / TPB] = static_cast<uint8_t>(sfq);
+                }
             }
         }
     }
@@ -262,6 +285,45 @@ __global__ void __launch_bounds__(512) quantize_dynamic_kernel(
     cudaTriggerProgrammaticLaunchCompletion();
 
     quantize_rows(x, rows, vpr, ldx, K, gs, q, sf);
+}
+
+// The same operation for small tensors in one thread-block cluster (no cooperative launch,
+// no grid barrier): blockIdx.y strides over rows, every CTA reduces its rows' maxima, the
+// cluster exchanges the per-CTA maxima through distributed shared memory, and every CTA
+// then quantises its rows. gridDim = (1, cluster size, 1).
+template <typename T>
+__global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
+    const T* __restrict__ x, uint32_t rows, uint32_t vpr, int64_t ldx, int64_t K,
+    float* __restrict__ gs_out, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+    const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out)
+{
+    __shared__ float red[32];
+    __shared__ float cta_max;
+    float m = amax_partial(x, rows, vpr, ldx);
+    m = block_max(m, red);
+    if (threadIdx.x == 0) cta_max = m;
+    cluster_sync();                                   // every CTA's maximum is in place
+    const uint32_t cs = gridDim.y;
+    float a = 0.0f;
+    if (threadIdx.x < 32) {
+        if (threadIdx.x < cs)
+            a = ld_shared_cluster_f32(mapa_shared(smem_u32(&cta_max), threadIdx.x));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if (threadIdx.x == 0) red[0] = a;
+    }
+    cluster_arrive();                                 // done reading the peers' maxima
+    __syncthreads();
+    a = red[0];
+    const float gs = (a == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, a);
+    if (blockIdx.y == 0) {
+        if (threadIdx.x == 0) *gs_out = gs;
+        for (int32_t i = threadIdx.x; i < n_alpha; i += blockDim.x)
+            alpha_out[i] = __fdiv_rn(1.0f, __fmul_rn(gs, gs_other[i]));
+    }
+    cudaTriggerProgrammaticLaunchCompletion();
+    quantize_rows(x, rows, vpr, ldx, K, gs, q, sf);
+    cluster_wait();                                   // no CTA leaves while a peer may read it
 }
 
 // ------------------------------------------------------------------ elementwise conversions
@@ -363,18 +425,78 @@ cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, i
     return cudaGetLastError();
 }
 
+// Largest cluster (16, else 8) of 512-thread quantiser CTAs the device runs; cached.
+template <typename T>
+static int quantize_cluster_size()
+{
+    static int cached[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return 0; }
+    std::lock_guard<std::mutex> g(mu);
+    if (cached[dev] == 0) {
+        auto kern = quantize_dynamic_cluster_kernel<T>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        int best = -1;
+        for (int cs : {16, 8}) {
+            cudaLaunchConfig_t cfg;
+            std::memset(&cfg, 0, sizeof(cfg));
+            cudaLaunchAttribute attr;
+            attr.id = cudaLaunchAttributeClusterDimension;
+            attr.val.clusterDim.x = 1;
+            attr.val.clusterDim.y = cs;
+            attr.val.clusterDim.z = 1;
+            cfg.gridDim = dim3(1, cs, 1);
+            cfg.blockDim = dim3(512, 1, 1);
+            cfg.attrs = &attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) { best = cs; break; }
+            cudaGetLastError();
+        }
+        cached[dev] = best;
+    }
+    return cached[dev] > 0 ? cached[dev] : 0;
+}
+
+// Tensors up to this size are quantised by one cluster; larger ones by a cooperative grid
+// (measured on B200: one 16-CTA cluster wins at 393 KB, loses from 1.5 MB up).
+constexpr int64_t kClusterQuantizeMaxBytes = int64_t(512) << 10;
+
 template <typename T>
 static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64_t ldx, int64_t K,
                                     float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
                                     int32_t n_alpha, float* alpha_out, int64_t q_bytes,
                                     cudaStream_t stream, int num_sms)
 {
+    const int64_t bytes = rows * K * static_cast<int64_t>(sizeof(T));
+    const int ccs = bytes <= kClusterQuantizeMaxBytes ? quantize_cluster_size<T>() : 0;
+    if (ccs > 0) {
+        const int cs = static_cast<int>(std::min<int64_t>(ccs, rows));
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(1, static_cast<unsigned>(cs), 1);
+        cfg.blockDim = dim3(512, 1, 1);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 1;
+        attr.val.clusterDim.y = static_cast<unsigned>(cs);
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, quantize_dynamic_cluster_kernel<T>, x, static_cast<uint32_t>(rows),
+                                  static_cast<uint32_t>(vpr), ldx, K, gs_out, q, sf, gs_other, n_alpha,
+                                  alpha_out);
+    }
     auto kern = quantize_dynamic_kernel<T>;
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 512, 0);
     if (e != cudaSuccess) return e;
     // co-resident blocks only (cooperative), few of them (cheap grid barriers), and room
     // for one partial maximum per block in q
+    // two 512-thread blocks per SM at most: enough warps to hide the arithmetic, few grid
+    // barrier participants
     int64_t cap = static_cast<int64_t>(std::min(std::max(per_sm, 1), 2)) * num_sms;
     cap = std::min<int64_t>(cap, std::max<int64_t>(q_bytes / 4, 1));
     const dim3 grid = grid_2d(rows, vpr, cap);
