@@ -60,8 +60,11 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
         const double c256 = static_cast<double>(ceil_div(t256, num_sms)) * 2.0;
         const double c128 = static_cast<double>(ceil_div(t128, num_sms)) * 1.15;
         p.bn = (N > 128 && c256 <= c128) ? 256 : 128;
+        // too few 256-wide tiles to fill the GPU: split-K follows, and 128-wide tiles halve
+        // the partial tile each CTA hands over (and the splits needed)
+        if (p.bn == 256 && t256 * 4 < num_sms * 3 && nk >= 2) p.bn = 128;
         const int force = env_int("NVFP4_BN", 0);
-        if (force == 128 || force == 256) p.bn = force;
+        if (force == 128 || force == 192 || force == 224 || force == 256) p.bn = force;
         p.q_tiles = ceil_div(N, p.bn);
     }
     const int tiles = p.p_tiles * p.q_tiles;
@@ -81,6 +84,16 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
         if (!allow_workspace) g = 1;
         while (cs * g > nk && g > 1) --g;
         while (cs * g > nk && cs > 1) --cs;
+    }
+    // Rasterisation band. While both packed operands fit in L2 together, P-fastest order
+    // over the whole grid (one band); beyond that, bands of 16 P tiles, so that one wave of
+    // tiles spans similar shares of A rows and B columns (16 P x ~9 Q tiles of 256 on 148
+    // SMs). Measured on B200: 8192^3 runs best in one band, 16384^3 with bands of 16.
+    const double packed_bytes = static_cast<double>(M + N) * static_cast<double>(K) * 0.5;
+    p.band = packed_bytes <= 80e6 ? p.p_tiles : std::max(1, std::min(p.p_tiles, 16));
+    {
+        const int fb = env_int("NVFP4_BAND", 0);
+        if (fb > 0) p.band = std::min(p.p_tiles, fb);
     }
     p.cluster = cs;
     p.groups = g;
@@ -209,7 +222,7 @@ static int max_active_clusters(int cs)
         attr.val.clusterDim.y = 1;
         attr.val.clusterDim.z = 1;
         cfg.gridDim = dim3(cs * 64, 1, 1);
-        cfg.blockDim = dim3(256, 1, 1);
+        cfg.blockDim = dim3(kGemmThreads, 1, 1);
         cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
@@ -289,6 +302,7 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         a.cluster_size = plan.cluster;
         a.groups = plan.groups;
         a.num_tiles = plan.num_tiles;
+        a.band = plan.band;
         if (plan.groups > 1) {
             a.ws_counters = static_cast<uint32_t*>(L.ws);
             a.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(L.ws) + plan.ws_counter_bytes);
@@ -301,7 +315,7 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(plan.grid), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cfg.stream = stream;
     // programmatic dependent launch: the prologue overlaps the previous kernel's tail
@@ -341,6 +355,8 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
     }
     switch (plan.bn) {
         case 128: return run<128, false, false>(plan, L, stream, encode_failed);
+        case 192: return run<192, false, false>(plan, L, stream, encode_failed);
+        case 224: return run<224, false, false>(plan, L, stream, encode_failed);
         case 256: return run<256, false, false>(plan, L, stream, encode_failed);
         default: return cudaErrorInvalidValue;
     }

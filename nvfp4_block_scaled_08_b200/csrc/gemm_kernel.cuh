@@ -13,17 +13,19 @@
 //     weight rows and the tokens become a narrow MMA N.
 //   * GROUPED     : SWAP with per-expert weights B[e] and token rows [off[e], off[e+1]).
 //
-// Roles (256 threads, one CTA per SM, persistent over tiles):
+// Roles (384 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer: A/B tiles (128-byte swizzle) and linear scale tiles.
 //   warp 1      TMEM allocator and single-thread MMA issuer (tcgen05.cp of scales, then
 //               four 128 x BN x 64 block-scaled MMAs per 256-element K stage).
-//   warp 2      scale re-layout: turns the TMA'd [rows][16 B] scale tile into the
-//               32-row x 16-byte blocks that tcgen05.cp ... 32x128b.warpx4 replicates into
-//               the TMEM layout the MMA reads (row r at column base + r/32, byte = k-block).
-//   warp 3      (grouped) builds the per-expert tile prefix; otherwise idle.
-//   warps 4-7   epilogue: TMEM -> registers -> alpha -> bf16 -> global; with split-K,
-//               fp32 partials to the workspace and a fixed-order reduction by the last
-//               CTA of each tile (deterministic).
+//   warps 2-3   scale re-layout, alternate stages: turn the TMA'd [rows][16 B] scale tile
+//               into the 32-row x 16-byte blocks that tcgen05.cp ... 32x128b.warpx4
+//               replicates into the TMEM layout the MMA reads (row r at column base + r/32,
+//               byte = k-block). Warp 3 first builds the per-expert tile prefix (grouped).
+//   warps 4-11  epilogue, two warpgroups (one per half of the tile's columns; warp w reads
+//               TMEM lane quadrant w % 4): TMEM -> registers -> alpha -> bf16 -> global; with split-K,
+//               the cluster's fp32 partials meet in shared memory (st.async over DSMEM)
+//               and are summed in a fixed rank order (deterministic); with several
+//               clusters per tile, through the workspace in a fixed group order.
 // Every wait is bounded (kWaitTimeoutNs); on a timeout the CTA records an error code,
 // stops all roles, lets in-flight copies and MMAs land, frees TMEM and exits.
 #pragma once
@@ -46,7 +48,12 @@ enum : uint32_t {
     kErrMmaSf = 0x105,
     kErrEpiAccFull = 0x106,
     kErrSplitRx = 0x107,
+    kErrMmaSfFree = 0x108,
 };
+
+// Threads per CTA: warps 0-3 (producer, MMA, scale re-layout) and two epilogue warpgroups.
+constexpr int kEpilogueWarps = 8;
+constexpr int kGemmThreads = 32 * (4 + kEpilogueWarps);
 
 struct GemmArgs {
     int32_t M, N;             // output is out[M][N] (row-major, leading dimension N)
@@ -58,6 +65,7 @@ struct GemmArgs {
     int32_t cluster_size;     // split-K CTAs per thread-block cluster (reduced over DSMEM)
     int32_t groups;           // clusters per output tile (reduced through the workspace)
     int32_t num_tiles;        // non-grouped: p_tiles * q_tiles * splits
+    int32_t band;             // non-grouped: P tiles per rasterisation band (>= 1)
     __nv_bfloat16* out;
     const float* alpha;       // [1] or [E]
     float* ws_partial;        // split-K fp32 partial tiles
@@ -88,13 +96,20 @@ struct GemmCfg {
     static constexpr uint32_t TX_BYTES = P_BYTES + Q_BYTES + SF_TMA_P + SF_TMA_Q;
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
 
-    // TMEM columns: accumulators, then SFA (4 k-blocks x 4 columns), then SFB
-    // (4 k-blocks x 4 columns per 128 Q rows).
+    // TMEM columns: two accumulators, then the scale factors: SFA (4 k-blocks x 4 columns),
+    // then SFB (4 k-blocks x 4 columns per 128 Q rows). When two BN = 256 accumulators fill
+    // all 512 columns (SF_IN_ACC), a tile's scale factors live in the top SF_COLS columns of
+    // the other accumulator instead: the epilogue drains those columns of the previous tile
+    // first and signals sf_free, and the MMA warp waits for that before the tile's first
+    // tcgen05.cp (by then the previous tile's MMAs have completed, so the copies cannot
+    // overwrite scales still being read, and the epilogue overlaps the next tile's MMAs).
     static constexpr int SF_COLS = 16 + 16 * QG;
-    static constexpr int ACC_STAGES = (2 * BN + SF_COLS <= 512) ? 2 : 1;
-    static constexpr int TMEM_SFA = ACC_STAGES * BN;
-    static constexpr int TMEM_SFB = TMEM_SFA + 16;
-    static constexpr int TMEM_USED = TMEM_SFB + 16 * QG;
+    static constexpr int ACC_STAGES = 2;
+    static constexpr bool SF_IN_ACC = 2 * BN + SF_COLS > 512;
+    static_assert(!SF_IN_ACC || SF_COLS <= 64, "scale columns fit the last 64-column chunk");
+    // column of SFA: absolute, or (SF_IN_ACC) relative to the other accumulator
+    static constexpr int TMEM_SFA = SF_IN_ACC ? BN - SF_COLS : ACC_STAGES * BN;
+    static constexpr int TMEM_USED = SF_IN_ACC ? ACC_STAGES * BN : ACC_STAGES * BN + SF_COLS;
     static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
                                    : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
     static_assert(TMEM_USED <= 512, "TMEM budget");
@@ -103,7 +118,10 @@ struct GemmCfg {
     static constexpr int MISC_BYTES = 1024 + (GROUPED ? 4 * (kMaxExperts + 1) : 0);
     static constexpr int ALIGN_SLACK = 1024;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - MISC_BYTES - ALIGN_SLACK) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
+    // Few-token (swap, non-grouped) launches split K finely and run a handful of stages per
+    // CTA: four buffers suffice and leave room on the SM for the neighbouring kernels' blocks.
+    static constexpr int STAGE_CAP = (SWAP && !GROUPED) ? 4 : 12;
+    static constexpr int STAGES = STAGES_FIT > STAGE_CAP ? STAGE_CAP : STAGES_FIT;
     static_assert(STAGES >= 2, "pipeline depth");
 
     // Shared memory layout (offsets from a 1024-byte aligned base).
@@ -112,8 +130,9 @@ struct GemmCfg {
     static constexpr int OFF_SFP = OFF_Q + STAGES * Q_BYTES;
     static constexpr int OFF_SFQ = OFF_SFP + STAGES * SFP_BYTES;
     static constexpr int OFF_BAR = OFF_SFQ + STAGES * SFQ_BYTES;
-    // barriers: full, sfready, empty [STAGES]; acc_full, acc_empty [2]; mma_done; split-K rx
-    static constexpr int NUM_BARS = 3 * STAGES + 6;
+    // barriers: full, sfready, empty [STAGES]; acc_full, acc_empty [2]; mma_done; split-K rx;
+    // sf_free [2]
+    static constexpr int NUM_BARS = 3 * STAGES + 8;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;     // tmem base, flags
     static constexpr int OFF_PREFIX = OFF_MISC + 64;
     static constexpr int SMEM_BYTES = OFF_PREFIX + (GROUPED ? 4 * (kMaxExperts + 1) : 0)
@@ -121,9 +140,9 @@ struct GemmCfg {
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     // split-K partial tile in shared memory: [128 rows][BN + 4 floats]
     static constexpr int PSTRIDE = BN + 4;
-    // split-K receive buffer: a chunk of ceil(128 / cs) rows from each of cs <= 8 ranks,
-    // cs * ceil(128 / cs) <= 135 rows
-    static_assert(136 * PSTRIDE * 4 <= STAGES * STAGE_BYTES, "split-K receive buffer fits the pipeline buffers");
+    // split-K receive buffer in the pipeline memory: this rank's chunk (at most
+    // ceil(16 / cs) * 8 rows) from each of cs <= 8 ranks, cs * ceil(16 / cs) * 8 <= 168 rows
+    static_assert(168 * PSTRIDE * 4 <= STAGES * STAGE_BYTES, "split-K receive buffer fits the pipeline buffers");
     static_assert(OFF_Q % 1024 == 0 && OFF_SFP % 1024 == 0, "swizzle atoms need 1 KB alignment");
 };
 
@@ -178,8 +197,14 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, int32_t t, const 
     } else {
         const int32_t split = t % a.splits;
         const int32_t pq = t / a.splits;
-        const int32_t pt = pq % a.num_p_tiles;
-        const int32_t qt = pq / a.num_p_tiles;
+        // Output tiles in bands of `band` P tiles: column by column (Q tile) within a band, P
+        // tile fastest, so that the tiles in flight at once share a few A and B panels in L2.
+        const int32_t per_band = a.band * a.num_q_tiles;
+        const int32_t b = pq / per_band;
+        const int32_t in_band = pq - b * per_band;
+        const int32_t width = min(a.band, a.num_p_tiles - b * a.band);
+        const int32_t qt = in_band / width;
+        const int32_t pt = b * a.band + (in_band - qt * width);
         const int32_t base = a.num_kstages / a.splits;
         const int32_t rem = a.num_kstages % a.splits;
         ti.p0 = pt * Cfg::BM;
@@ -206,33 +231,6 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
         : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
         : "memory");
     return r != 0;
-}
-
-// Store 4 consecutive accumulator columns (c4 * 4 .. +3) of P row `row` of a tile.
-template <class Cfg>
-__device__ __forceinline__ void store_out4(const GemmArgs& a, const Tile& ti, int row, int c4,
-                                           float4 v, float alpha)
-{
-    const int p = ti.p0 + row;
-    if constexpr (!Cfg::SWAP) {
-        const int n0 = ti.q0 + 4 * c4;
-        if (p < a.M && n0 < a.N) {
-            uint2 w;
-            w.x = pack_bf16x2(alpha * v.x, alpha * v.y);
-            w.y = pack_bf16x2(alpha * v.z, alpha * v.w);
-            *reinterpret_cast<uint2*>(a.out + static_cast<size_t>(p) * a.N + n0) = w;
-        }
-    } else {
-        if (p < a.N) {
-            const float vals[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int m = ti.q0 + 4 * c4 + j;
-                if (m < a.M)
-                    a.out[static_cast<size_t>(m) * a.N + p] = __float2bfloat16_rn(alpha * vals[j]);
-            }
-        }
-    }
 }
 
 // Store 16 consecutive accumulator columns (c .. c + 15) of P row `p` as bf16(alpha * v).
@@ -275,17 +273,137 @@ __device__ __forceinline__ void store_out16(const GemmArgs& a, const Tile& ti, i
     }
 }
 
-// Rows [chunk_begin(k), chunk_begin(k + 1)) of a 128-row tile belong to cluster rank k.
-__device__ __forceinline__ int chunk_begin(int k, int cs) { return (k * 128 + cs - 1) / cs; }
+// Stores 64 accumulator columns (c0 .. c0 + 63) of the 32 rows a warp holds (lane = row,
+// non-swap tiles) as bf16(alpha * v), four rows x 128 contiguous bytes per store instruction.
+// A lane's row is eight 16-byte chunks (8 columns each); an 8 x 8 transpose of chunks within
+// each group of 8 lanes (three butterfly stages of shuffles: at stage m the lanes whose bit m
+// differs from the chunk index's swap those chunks) leaves lane 8 g + j holding chunk j of
+// rows 8 g .. 8 g + 7, so that lanes 8 g .. 8 g + 7 write one 128-byte row segment together.
+// (Stores straight from the row-per-lane layout would touch 32 lines per instruction.)
+template <class Cfg>
+__device__ __forceinline__ void store_rows64(const GemmArgs& a, const Tile& ti, int quad, int lane, int c0,
+                                             const uint32_t (&r)[4][16], float alpha)
+{
+    uint32_t w[8][4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[e][k] = pack_bf16x2(alpha * __uint_as_float(r[e >> 1][(e & 1) * 8 + 2 * k]),
+                                  alpha * __uint_as_float(r[e >> 1][(e & 1) * 8 + 2 * k + 1]));
+    const int j = lane & 7;
+#pragma unroll
+    for (int m = 4; m >= 1; m >>= 1) {
+        const bool hi = (j & m) != 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (e & m) continue;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t send = hi ? w[e][k] : w[e ^ m][k];
+                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+                if (hi) w[e][k] = recv;
+                else w[e ^ m][k] = recv;
+            }
+        }
+    }
+    const int n = ti.q0 + c0 + 8 * j;
+    const int m0 = ti.p0 + 32 * quad + (lane & ~7);
+    if (n < a.N) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int m = m0 + t;
+            if (m < a.M)
+                *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(m) * a.N + n) =
+                    make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
+        }
+    }
+}
 
-// Split-K epilogue of one CTA, run by the 128 epilogue threads (thread = accumulator row);
+// Rows [chunk_begin(k), chunk_begin(k + 1)) of a 128-row tile belong to cluster rank k:
+// whole 8-row groups, as evenly as possible (at most ceil(16 / cs) * 8 rows per rank).
+__device__ __forceinline__ int chunk_begin(int k, int cs) { return ((k * 16 + cs - 1) / cs) * 8; }
+// The rank whose chunk holds `row`.
+__device__ __forceinline__ int chunk_owner(int row, int cs) { return ((row >> 3) * cs) >> 4; }
+
+// Writes a reduced chunk of a tile: rows [r0, r0 + rows) of the 128 x BN accumulator tile,
+// each the in-order sum of `nsrc` fp32 copies in shared memory (copy j, chunk row lr, column
+// c at src[(j * rows + lr) * PSTRIDE + c]), times alpha, as bf16. All 128 epilogue threads
+// (tid) take part; every store is 16 bytes (8 bf16) and consecutive threads write
+// consecutive addresses.
+template <class Cfg>
+__device__ __forceinline__ void store_chunk(const GemmArgs& a, const Tile& ti, const float* src, int nsrc,
+                                            int r0, int rows, int tid, float alpha)
+{
+    constexpr int BN = Cfg::BN;
+    constexpr int PS = Cfg::PSTRIDE;
+    if constexpr (!Cfg::SWAP) {
+        // item = (chunk row lr, 8-column group c8); output row p0 + r0 + lr, columns q0 + 8 c8
+        constexpr int G = BN / 8;
+        for (int item = tid; item < rows * G; item += 128) {
+            const int lr = item / G;
+            const int c = (item % G) * 8;
+            float v[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) v[t] = 0.0f;
+            for (int j = 0; j < nsrc; ++j) {
+                const float* s = src + (j * rows + lr) * PS + c;
+                const float4 x0 = *reinterpret_cast<const float4*>(s);
+                const float4 x1 = *reinterpret_cast<const float4*>(s + 4);
+                v[0] += x0.x; v[1] += x0.y; v[2] += x0.z; v[3] += x0.w;
+                v[4] += x1.x; v[5] += x1.y; v[6] += x1.z; v[7] += x1.w;
+            }
+            const int m = ti.p0 + r0 + lr;
+            const int n0 = ti.q0 + c;
+            if (m < a.M && n0 < a.N) {
+                uint4 w;
+                w.x = pack_bf16x2(alpha * v[0], alpha * v[1]);
+                w.y = pack_bf16x2(alpha * v[2], alpha * v[3]);
+                w.z = pack_bf16x2(alpha * v[4], alpha * v[5]);
+                w.w = pack_bf16x2(alpha * v[6], alpha * v[7]);
+                *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(m) * a.N + n0) = w;
+            }
+        }
+    } else {
+        // item = (accumulator column c, 8-row group g); output row q0 + c, columns
+        // p0 + r0 + 8 g .. + 7 (chunk rows are weight rows, i.e. output columns)
+        const int G = rows >> 3;
+        for (int item = tid; item < BN * G; item += 128) {
+            const int c = item / G;
+            const int lr = (item - c * G) * 8;
+            float v[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) v[t] = 0.0f;
+            for (int j = 0; j < nsrc; ++j) {
+                const float* s = src + (j * rows + lr) * PS + c;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) v[t] += s[t * PS];
+            }
+            const int m = ti.q0 + c;
+            const int n0 = ti.p0 + r0 + lr;
+            if (m < a.M && n0 < a.N) {
+                uint4 w;
+                w.x = pack_bf16x2(alpha * v[0], alpha * v[1]);
+                w.y = pack_bf16x2(alpha * v[2], alpha * v[3]);
+                w.z = pack_bf16x2(alpha * v[4], alpha * v[5]);
+                w.w = pack_bf16x2(alpha * v[6], alpha * v[7]);
+                *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(m) * a.N + n0) = w;
+            }
+        }
+    }
+}
+
+// Split-K epilogue of one CTA, run by the 128 threads of the first epilogue warpgroup
+// (thread = accumulator row; named barrier 2);
 // every CTA of a split-K launch owns exactly one tile. The `cluster_size` CTAs of a cluster
 // hold consecutive K slices of the same output tile, and row chunk k is reduced by cluster
 // rank k. After the cluster barrier (every CTA of the cluster has drained its main loop, so
-// its pipeline shared memory is free) each thread sends its accumulator row, straight from
-// TMEM through registers, to the owning rank with st.async; the owner's threads wait on
-// their rx barrier, sum the ranks in order (fixed, deterministic) and write bf16. With
-// `groups` > 1 clusters per tile the owners write their fp32 chunk to the workspace instead,
+// its pipeline shared memory is free) each thread copies its accumulator row, straight from
+// TMEM through registers, into slot `rank` of the owning rank's receive buffer
+// [cs][my_rows][PSTRIDE]: st.async to a peer (completion counted in bytes on the peer's rx
+// barrier), a plain store for its own chunk. Once the peers' bytes have landed all 128
+// threads sum the chunk over the slots in rank order (fixed, deterministic) and write it as
+// bf16. With `groups` > 1 clusters per tile the fp32 chunk goes to the workspace instead,
 // and the last of the `groups` CTAs holding the same chunk (arrival counter) sums the
 // chunks in group order.
 template <class Cfg>
@@ -299,7 +417,7 @@ __device__ __forceinline__ void split_k_epilogue(const GemmArgs& a, const Tile& 
     const int cs = a.cluster_size;
     const int g = a.groups;
     const int rank = cs > 1 ? static_cast<int>(cluster_ctarank()) : 0;
-    const int owner = (row * cs) / 128;    // == the k with chunk_begin(k) <= row < chunk_begin(k+1)
+    const int owner = chunk_owner(row, cs);
     float* rx = reinterpret_cast<float*>(smem + Cfg::OFF_P);
     if (cs > 1) { cluster_arrive(); cluster_wait(); }
 
@@ -307,109 +425,93 @@ __device__ __forceinline__ void split_k_epilogue(const GemmArgs& a, const Tile& 
     const int my_rows = chunk_begin(rank + 1, cs) - my0;
     const int grp = ti.split / cs;
     const bool is_owner = owner == rank;
-    // tcgen05.ld is .sync.aligned: every lane of the warp executes every load below, and
-    // only what is done with the values depends on the lane's row.
+    const int own0 = chunk_begin(owner, cs);
+    const int own_rows = chunk_begin(owner + 1, cs) - own0;
 
-    // 1. rows owned by another rank go there (TMEM -> registers -> peer shared memory)
-    if (cs > 1) {
-        const int own0 = chunk_begin(owner, cs);
-        const int own_rows = chunk_begin(owner + 1, cs) - own0;
-        const uint32_t dst = mapa_shared(smem_u32(rx + (rank * own_rows + (row - own0)) * PS),
-                                         static_cast<uint32_t>(owner));
-        const uint32_t bar = mapa_shared(smem_u32(rx_bar), static_cast<uint32_t>(owner));
+    // 1. every row to slot `rank` of its owner's receive buffer. tcgen05.ld is .sync.aligned:
+    //    every lane of the warp executes every load, only the destination depends on the row.
+    {
+        float* mine = rx + (rank * own_rows + (row - own0)) * PS;        // in the owner's buffer
+        const uint32_t dst = cs > 1 ? mapa_shared(smem_u32(mine), static_cast<uint32_t>(owner)) : 0u;
+        const uint32_t bar = cs > 1 ? mapa_shared(smem_u32(rx_bar), static_cast<uint32_t>(owner)) : 0u;
         for (int c = 0; c < BN; c += 16) {
             uint32_t r[16];
             tmem_ld_32x32b_x16(tacc + c, r);
             tmem_ld_wait();
-            if (!is_owner) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    st_async_f4(dst + (c + 4 * i) * 4, __uint_as_float(r[4 * i]),
-                                __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
-                                __uint_as_float(r[4 * i + 3]), bar);
+            for (int i = 0; i < 4; ++i) {
+                const float4 f = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                             __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                if (is_owner) *reinterpret_cast<float4*>(mine + c + 4 * i) = f;
+                else st_async_f4(dst + (c + 4 * i) * 4, f.x, f.y, f.z, f.w, bar);
             }
         }
     }
-    // 2. wait (all epilogue threads, bounded) for the other ranks' copies of this CTA's rows
+    // 2. wait (all epilogue threads, bounded) for the other ranks' copies of this CTA's rows;
+    //    the named barrier publishes the own-slot rows to all 128 threads
     bool ok = true;
     if (cs > 1) {
         if (row == my0)
             mbar_arrive_expect_tx(rx_bar, static_cast<uint32_t>((cs - 1) * my_rows * BN * 4));
         ok = mbar_wait(rx_bar, 0, ab, kErrSplitRx);
-        __syncwarp();
-    }
-    // 3. owner rows: own partial (from TMEM) + the received ones, in rank order
-    const int lr = row - my0;
-    float* chunk_ws = nullptr;
-    if (g > 1) chunk_ws = a.ws_partial + (static_cast<size_t>(ti.pq) * g + grp) * (128 * BN);
-    for (int c = 0; c < BN; c += 16) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(tacc + c, r);
-        tmem_ld_wait();
-        if (!is_owner) continue;
-        float v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-        for (int k = 0; k < cs; ++k) {
-            if (k == rank) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(r[j]);
-            } else if (ok) {
-                const float* src = rx + (k * my_rows + lr) * PS + c;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 f = *reinterpret_cast<const float4*>(src + 4 * i);
-                    v[4 * i] += f.x; v[4 * i + 1] += f.y; v[4 * i + 2] += f.z; v[4 * i + 3] += f.w;
-                }
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float4 f = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            if (g == 1) store_out4<Cfg>(a, ti, row, c / 4 + i, f, alpha);
-            else __stcg(reinterpret_cast<float4*>(chunk_ws + row * BN + c + 4 * i), f);
-        }
     }
     __syncwarp();
-    if (g == 1) return;
+    ok = named_bar_and(2, 128, ok);
+    if (!ok) return;
+
+    // 3. reduce over the ranks in order
+    if (g == 1) {
+        store_chunk<Cfg>(a, ti, rx, cs, my0, my_rows, row, alpha);
+        return;
+    }
+    float* chunk_ws = a.ws_partial + (static_cast<size_t>(ti.pq) * g + grp) * (128 * BN)
+                    + static_cast<size_t>(my0) * BN;
+    for (int item = row; item < my_rows * (BN / 4); item += 128) {
+        const int lr = item / (BN / 4);
+        const int c = (item % (BN / 4)) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < cs; ++k) {
+            const float4 f = *reinterpret_cast<const float4*>(rx + (k * my_rows + lr) * PS + c);
+            v.x += f.x; v.y += f.y; v.z += f.z; v.w += f.w;
+        }
+        __stcg(reinterpret_cast<float4*>(chunk_ws + lr * BN + c), v);
+    }
 
     // groups > 1: the last of the `groups` CTAs that hold chunk `rank` of this tile sums the
-    // chunks from the workspace in group order
+    // chunks from the workspace in group order (into receive slot 0), then stores them
     __threadfence();
     __syncwarp();
-    named_bar_sync(1, 128);
+    named_bar_sync(2, 128);
     uint32_t* counter = a.ws_counters + static_cast<size_t>(ti.pq) * cs + rank;
-    if (row == my0) {
+    if (row == 0) {
         const uint32_t prev = atomicAdd(counter, 1u);
         *s_is_last = (prev == static_cast<uint32_t>(g - 1)) ? 1 : 0;
     }
     __syncwarp();
-    named_bar_sync(1, 128);
+    named_bar_sync(2, 128);
     if (!*s_is_last) return;
     __threadfence();
-    if (is_owner) {
-        const float* tile_ws = a.ws_partial + static_cast<size_t>(ti.pq) * g * (128 * BN);
-        for (int c4 = 0; c4 < BN / 4; ++c4) {
-            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int j0 = 0; j0 < g; j0 += 4) {
-                float4 v[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (j0 + j < g)
-                        v[j] = __ldcg(reinterpret_cast<const float4*>(
-                            tile_ws + static_cast<size_t>(j0 + j) * (128 * BN) + row * BN + 4 * c4));
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (j0 + j < g) { s.x += v[j].x; s.y += v[j].y; s.z += v[j].z; s.w += v[j].w; }
-            }
-            store_out4<Cfg>(a, ti, row, c4, s, alpha);
+    const float* tile_ws = a.ws_partial + static_cast<size_t>(ti.pq) * g * (128 * BN)
+                         + static_cast<size_t>(my0) * BN;
+    for (int item = row; item < my_rows * (BN / 4); item += 128) {
+        const int lr = item / (BN / 4);
+        const int c = (item % (BN / 4)) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < g; ++j) {
+            const float4 f = __ldcg(reinterpret_cast<const float4*>(
+                tile_ws + static_cast<size_t>(j) * (128 * BN) + lr * BN + c));
+            v.x += f.x; v.y += f.y; v.z += f.z; v.w += f.w;
         }
+        *reinterpret_cast<float4*>(rx + lr * PS + c) = v;
     }
-    if (row == my0) *counter = 0u;             // re-arm for the next call
+    __syncwarp();
+    named_bar_sync(2, 128);
+    store_chunk<Cfg>(a, ti, rx, 1, my0, my_rows, row, alpha);
+    if (row == 0) *counter = 0u;             // re-arm for the next call
 }
 
 template <class Cfg>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_sfp, const __grid_constant__ CUtensorMap tm_sfq,
                   const GemmArgs args)
@@ -430,6 +532,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     uint64_t* acc_empty_bar = bars + 3 * STAGES + 2;
     uint64_t* mma_done_bar = bars + 3 * STAGES + 4;
     uint64_t* rx_bar = bars + 3 * STAGES + 5;       // split-K: partial rows received from peers
+    uint64_t* sf_free_bar = bars + 3 * STAGES + 6;  // SF_IN_ACC: scale columns drained
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
     volatile int* s_is_last = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 8);
@@ -448,7 +551,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full_bar[s], 1);
-            mbar_init(&acc_empty_bar[s], 4);
+            mbar_init(&acc_empty_bar[s], kEpilogueWarps);
+            mbar_init(&sf_free_bar[s], 4);            // the second epilogue warpgroup
         }
         mbar_init(mma_done_bar, 1);
         mbar_init(rx_bar, 1);
@@ -507,6 +611,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Every CTA of this grid is resident: the next kernel in the stream may be scheduled
+    // (it waits for this grid's completion before touching memory).
+    grid_launch_dependents();
 
     const uint32_t tmem_base = *s_tmem_base;
     const int32_t num_tiles = Cfg::GROUPED ? s_prefix[args.num_experts] : args.num_tiles;
@@ -576,12 +683,24 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         // -------------------------------------------------------------- MMA issuer
         // Whole warp in the loop, one elected lane issues tcgen05.cp / tcgen05.mma.
         uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+        uint32_t sf_phases = 0;                    // bit b: parity of the next sf_free[b] wait
         bool ok = true;
         for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
             ok = __all_sync(0xffffffffu, mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, ab, kErrMmaAccEmpty));
             if (!ok) break;
+            if constexpr (Cfg::SF_IN_ACC) {
+                if (t != static_cast<int32_t>(blockIdx.x)) {   // the previous tile's scale columns
+                    const uint32_t o = acc ^ 1u;
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&sf_free_bar[o], (sf_phases >> o) & 1u, ab, kErrMmaSfFree));
+                    if (!ok) break;
+                    sf_phases ^= 1u << o;
+                }
+            }
             tc_fence_after();
+            const uint32_t sf_a = tmem_base + Cfg::TMEM_SFA + (Cfg::SF_IN_ACC ? (acc ^ 1u) * BN : 0u);
+            const uint32_t sf_b = sf_a + 16;
             uint32_t n_mma = BN;
             if constexpr (Cfg::GROUPED) n_mma = min(BN, (ti.q_valid + 15) & ~15);
             const uint32_t idesc = idesc_mxf4nvf4(128, n_mma);
@@ -596,11 +715,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     const uint32_t sfq = smem_u32(smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        tmem_cp_32x128b_warpx4(tmem_base + Cfg::TMEM_SFA + 4 * j,
-                                               sdesc_sf_32x16(sfp + 512 * j));
+                        tmem_cp_32x128b_warpx4(sf_a + 4 * j, sdesc_sf_32x16(sfp + 512 * j));
 #pragma unroll
                         for (int g = 0; g < QG; ++g)
-                            tmem_cp_32x128b_warpx4(tmem_base + Cfg::TMEM_SFB + 4 * QG * j + 4 * g,
+                            tmem_cp_32x128b_warpx4(sf_b + 4 * QG * j + 4 * g,
                                                    sdesc_sf_32x16(sfq + 2048 * g + 512 * j));
                     }
                     const uint64_t pdesc =
@@ -610,10 +728,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         // advance 32 bytes (64 fp4 values) along K inside the swizzled rows
-                        mma_mxf4nvf4(d_tmem, pdesc + 2u * j, qdesc + 2u * j, idesc,
-                                     tmem_base + Cfg::TMEM_SFA + 4 * j,
-                                     tmem_base + Cfg::TMEM_SFB + 4 * QG * j,
-                                     (ks > 0 || j > 0) ? 1u : 0u);
+                        mma_mxf4nvf4(d_tmem, pdesc + 2u * j, qdesc + 2u * j, idesc, sf_a + 4 * j,
+                                     sf_b + 4 * QG * j, (ks > 0 || j > 0) ? 1u : 0u);
                     }
                     mma_commit(&empty_bar[stage]);
                 }
@@ -681,18 +797,22 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         }
     } else if (warp >= 4) {
         // -------------------------------------------------------------- epilogue
+        // Two warpgroups: warps 4 + 4h + q read TMEM lane quadrant q and take half h of the
+        // tile's columns (split-K: the first warpgroup reduces, the second only keeps pace).
         grid_dependency_wait();                    // alpha, out and the workspace
         const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
+        const int half = (warp - 4) >> 2;
         const int row = 32 * quad + lane;          // accumulator row (P row within the tile)
         uint32_t acc = 0, acc_phase = 0;
         for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
             bool ok = mbar_wait(&acc_full_bar[acc], acc_phase, ab, kErrEpiAccFull);
-            ok = named_bar_and(1, 128, ok);
+            ok = named_bar_and(1, 32 * kEpilogueWarps, ok);
             if (!ok) {
                 if constexpr (!Cfg::GROUPED) {
-                    // cluster peers wait for this CTA on the cluster barrier: arrive anyway
-                    if (args.splits > 1 && args.cluster_size > 1) { cluster_arrive(); cluster_wait(); }
+                    // cluster peers wait for this CTA on the cluster barrier: arrive anyway (the
+                    // second warpgroup arrives in the teardown)
+                    if (half == 0 && args.splits > 1 && args.cluster_size > 1) { cluster_arrive(); cluster_wait(); }
                 }
                 break;
             }
@@ -705,21 +825,71 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             int n_cols = BN;
             if constexpr (Cfg::GROUPED) n_cols = min(BN, (ti.q_valid + 15) & ~15);
             if constexpr (!Cfg::GROUPED) {
-                if (split_k) split_k_epilogue<Cfg>(args, ti, smem, rx_bar, s_is_last, tacc, row, alpha, ab);
+                if (split_k && half == 0)
+                    split_k_epilogue<Cfg>(args, ti, smem, rx_bar, s_is_last, tacc, row, alpha, ab);
+            }
+            // this warpgroup's columns [c_lo, c_hi), multiples of 16
+            const int mid = ((n_cols / 2 + 15) / 16) * 16;
+            const int c_lo = half ? mid : 0;
+            int c_hi = split_k ? c_lo : (half ? n_cols : mid);
+            if constexpr (Cfg::SF_IN_ACC) {
+                // the second warpgroup frees the last 64 columns (the next tile's scale
+                // columns) first: into registers, signal, then store them
+                if (half == 1 && !split_k) {
+                    uint32_t r[4][16];
+                    const bool need = n_cols > BN - 64;
+                    if (need) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x16(tacc + BN - 64 + 16 * i, r[i]);
+                        tmem_ld_wait();
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sf_free_bar[acc]);
+                    if (need) {
+                        if constexpr (!Cfg::SWAP && !Cfg::GROUPED) {
+                            store_rows64<Cfg>(args, ti, quad, lane, BN - 64, r, alpha);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                if (BN - 64 + 16 * i < n_cols) store_out16<Cfg>(args, ti, p, BN - 64 + 16 * i, r[i], alpha);
+                        }
+                    }
+                    c_hi = min(c_hi, BN - 64);
+                }
             }
 
-            // two 16-column TMEM loads in flight per wait
-            for (int c0 = 0; c0 < n_cols && !split_k; c0 += 32) {
-                uint32_t r[2][16];
-                const bool two = c0 + 16 < n_cols;
-                tmem_ld_32x32b_x16(tacc + c0, r[0]);
-                if (two) tmem_ld_32x32b_x16(tacc + c0 + 16, r[1]);
-                tmem_ld_wait();
+            if constexpr (!Cfg::SWAP && !Cfg::GROUPED) {
+                // 64-column chunks: four 16-column TMEM loads in flight, coalesced row stores
+                int c0 = c_lo;
+                for (; c0 + 64 <= c_hi; c0 += 64) {
+                    uint32_t r[4][16];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    if (h == 1 && !two) break;
-                    const int c = c0 + 16 * h;
-                    store_out16<Cfg>(args, ti, p, c, r[h], alpha);
+                    for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x16(tacc + c0 + 16 * i, r[i]);
+                    tmem_ld_wait();
+                    store_rows64<Cfg>(args, ti, quad, lane, c0, r, alpha);
+                }
+                // the rest (BN = 224, 192: 48, 32 columns per half) the plain way
+                for (; c0 < c_hi; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(tacc + c0, r);
+                    tmem_ld_wait();
+                    store_out16<Cfg>(args, ti, p, c0, r, alpha);
+                }
+            } else {
+                // two 16-column TMEM loads in flight per wait
+                for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
+                    uint32_t r[2][16];
+                    const bool two = c0 + 16 < c_hi;
+                    tmem_ld_32x32b_x16(tacc + c0, r[0]);
+                    if (two) tmem_ld_32x32b_x16(tacc + c0 + 16, r[1]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (h == 1 && !two) break;
+                        const int c = c0 + 16 * h;
+                        store_out16<Cfg>(args, ti, p, c, r[h], alpha);
+                    }
                 }
             }
             // Accumulator drained into registers / workspace: hand it back to the MMA warp.
@@ -733,12 +903,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
 
     // ------------------------------------------------------------------ teardown
     __syncwarp();
-    grid_launch_dependents();
     if constexpr (!Cfg::GROUPED) {
-        // split-K: the non-epilogue warps are done with the pipeline; together with the
-        // epilogue's arrival (after its accumulator is complete) this tells the cluster peers
-        // that this CTA's shared memory may receive their partial rows
-        if (warp < 4 && args.splits > 1 && args.cluster_size > 1) { cluster_arrive(); cluster_wait(); }
+        // split-K: the non-epilogue warps (and the second epilogue warpgroup) are done with
+        // the pipeline; together with the first epilogue warpgroup's arrival (after its
+        // accumulator is complete) this tells the cluster peers that this CTA's shared memory
+        // may receive their partial rows
+        if ((warp < 4 || warp >= 8) && args.splits > 1 && args.cluster_size > 1) { cluster_arrive(); cluster_wait(); }
     }
     tc_fence_before();
     __syncthreads();

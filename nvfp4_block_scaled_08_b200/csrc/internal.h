@@ -35,6 +35,7 @@ struct GemmPlan {
     int groups = 1;        // clusters per output tile (workspace reduction when > 1)
     int p_tiles = 0, q_tiles = 0;
     int num_tiles = 0;     // work items (non-grouped)
+    int band = 1;          // P tiles per rasterisation band (non-grouped)
     int grid = 0;          // persistent CTAs
     size_t ws_bytes = 0;   // workspace needed (split-K)
     size_t ws_counter_bytes = 0;

@@ -78,9 +78,48 @@ template <> struct InTraits<__nv_bfloat16> {
 
 // ------------------------------------------------------------------ indexing
 
-// A [rows, K] tensor of T (row stride ld) is read as 16-byte vectors, vpr = K / V per row.
-// Grids are 2-D: blockIdx.y strides over rows, blockIdx.x * blockDim.x + threadIdx.x over
-// the vectors of a row, so no index needs a division.
+// A [rows, K] tensor of T (row stride ld elements) is read as nv = rows * vpr 16-byte
+// vectors (V elements each, vpr = K / V per row), numbered row-major: vector i is row
+// i / vpr, column i % vpr. Every launch keeps nv < 2^31, so indices are 32-bit. With
+// contiguous rows (ld == K) vector i sits at x + i * V and no division is needed;
+// otherwise the row comes from a multiply-high by a precomputed reciprocal ("round-up"
+// method of Granlund and Montgomery, PLDI 1994: with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (mulhi(n, m) + n) >> l for every n < 2^32).
+// The codes and scales are written contiguously: vector i's codes at q + i * V / 2, the
+// scale of the 16-element block holding it at sf + i / (16 / V).
+struct VecIndex {
+    uint32_t vpr;      // vectors per row
+    uint32_t mul;      // m above (d = vpr)
+    uint32_t shift;    // l above
+    uint32_t contiguous;
+    int64_t ld;        // row stride in elements
+};
+
+static VecIndex make_vec_index(int64_t vpr, int64_t ld, int64_t K)
+{
+    VecIndex ix;
+    ix.vpr = static_cast<uint32_t>(vpr);
+    uint32_t l = 0;
+    while ((uint64_t(1) << l) < static_cast<uint64_t>(vpr)) ++l;
+    ix.shift = l;
+    ix.mul = static_cast<uint32_t>(((uint64_t(1) << 32) * ((uint64_t(1) << l) - static_cast<uint64_t>(vpr)))
+                                   / static_cast<uint64_t>(vpr) + 1);
+    ix.contiguous = (ld == K) ? 1u : 0u;
+    ix.ld = ld;
+    return ix;
+}
+
+template <int V>
+__device__ __forceinline__ int64_t vec_offset(const VecIndex& ix, uint32_t i)
+{
+    if (ix.contiguous) return static_cast<int64_t>(i) * V;
+    const uint32_t r = static_cast<uint32_t>((static_cast<uint64_t>(__umulhi(i, ix.mul)) + i) >> ix.shift);
+    const uint32_t c = i - r * ix.vpr;
+    return static_cast<int64_t>(r) * ix.ld + static_cast<int64_t>(c) * V;
+}
+
+// Loads in flight per thread in the sweeps below.
+constexpr int kUnroll = 4;
 
 __device__ __forceinline__ float block_max(float m, float* red)
 {
@@ -100,100 +139,93 @@ __device__ __forceinline__ float block_max(float m, float* red)
     return m;
 }
 
+// max |x| over this thread's vectors: block `bid` of `nb` blocks, kUnroll loads in flight.
 template <typename T>
-__device__ __forceinline__ float amax_partial(const T* x, uint32_t rows, uint32_t vpr, int64_t ld)
+__device__ __forceinline__ float amax_partial(const T* x, const VecIndex& ix, uint32_t nv, uint32_t bid,
+                                              uint32_t nb)
 {
     constexpr int V = InTraits<T>::kPerThread;
+    constexpr int U = kUnroll;
+    const uint32_t stride = nb * blockDim.x;
     float m = 0.0f;
-    const uint32_t cstride = gridDim.x * blockDim.x;
-    constexpr int U = 4;                     // independent loads in flight per thread
-    for (uint32_t r = blockIdx.y; r < rows; r += gridDim.y) {
-        const T* row = x + static_cast<int64_t>(r) * ld;
-        for (uint32_t c0 = blockIdx.x * blockDim.x + threadIdx.x; c0 < vpr; c0 += U * cstride) {
-            float v[U][V];
+    for (uint32_t i0 = bid * blockDim.x + threadIdx.x; i0 < nv; i0 += U * stride) {
+        float v[U][V];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const uint32_t c = c0 + u * cstride;
-                if (c < vpr) InTraits<T>::load(row + static_cast<int64_t>(c) * V, v[u]);
-                else {
+        for (int u = 0; u < U; ++u) {
+            const uint32_t i = i0 + u * stride;
+            if (i < nv) InTraits<T>::load(x + vec_offset<V>(ix, i), v[u]);
+            else {
 #pragma unroll
-                    for (int k = 0; k < V; ++k) v[u][k] = 0.0f;
-                }
+                for (int k = 0; k < V; ++k) v[u][k] = 0.0f;
             }
-#pragma unroll
-            for (int u = 0; u < U; ++u)
-#pragma unroll
-                for (int k = 0; k < V; ++k) m = fmaxf(m, fabsf(v[u][k]));
         }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int k = 0; k < V; ++k) m = fmaxf(m, fabsf(v[u][k]));
     }
     return m;
 }
 
-// Quantise every row. The TPB lanes that share a 16-element block are consecutive lanes of
-// one warp in the same iteration (vpr is a multiple of TPB and the column stride a multiple
-// of 32); the first of them computes the block scale and shares it.
+// Quantise this thread's vectors (block `bid` of `nb`). The TPB lanes that share a
+// 16-element block are consecutive lanes of one warp in the same iteration (each warp
+// takes 32 consecutive vectors, and a block never straddles a row since vpr % TPB == 0);
+// the first of them computes the block scale and shares it.
 // Per block, in fp32 with explicit rounding and in this order:
 //   amax -> s = e4m3(amax / 6 * gs) -> r = s ? gs / s : 0 -> codes e2m1(x * r).
 template <typename T>
-__device__ __forceinline__ void quantize_rows(const T* __restrict__ x, uint32_t rows, uint32_t vpr,
-                                              int64_t ld, int64_t K, float gs,
-                                              uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
+__device__ __forceinline__ void quantize_vectors(const T* __restrict__ x, const VecIndex& ix, uint32_t nv,
+                                                 uint32_t bid, uint32_t nb, float gs,
+                                                 uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
 {
     constexpr int V = InTraits<T>::kPerThread;   // elements per thread
     constexpr int TPB = 16 / V;                  // threads per 16-element block
+    constexpr int U = kUnroll;
     const uint32_t lane = threadIdx.x & 31;
-    const uint32_t cstride = gridDim.x * blockDim.x;
-    const uint32_t c_first = blockIdx.x * blockDim.x + threadIdx.x;
-    for (uint32_t r = blockIdx.y; r < rows; r += gridDim.y) {
-        const T* row = x + static_cast<int64_t>(r) * ld;
-        uint8_t* qrow = q + static_cast<int64_t>(r) * (K / 2);
-        uint8_t* sfrow = sf + static_cast<int64_t>(r) * (K / 16);
-        constexpr int U = 4;                 // independent loads in flight per thread
-        for (uint32_t cb0 = c_first - lane; cb0 < vpr; cb0 += U * cstride) {   // warp-uniform
-            float v[U][V];
+    const uint32_t stride = nb * blockDim.x;
+    for (uint32_t w0 = bid * blockDim.x + threadIdx.x - lane; w0 < nv; w0 += U * stride) {   // warp-uniform
+        float v[U][V];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const uint32_t c = cb0 + u * cstride + lane;
-                if (c < vpr) {
-                    InTraits<T>::load(row + static_cast<int64_t>(c) * V, v[u]);
-                } else {
+        for (int u = 0; u < U; ++u) {
+            const uint32_t i = w0 + u * stride + lane;
+            if (i < nv) {
+                InTraits<T>::load(x + vec_offset<V>(ix, i), v[u]);
+            } else {
 #pragma unroll
-                    for (int k = 0; k < V; ++k) v[u][k] = 0.0f;
-                }
+                for (int k = 0; k < V; ++k) v[u][k] = 0.0f;
             }
+        }
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const uint32_t cbase = cb0 + u * cstride;
-                if (cbase >= vpr) break;             // warp-uniform
-                const uint32_t c = cbase + lane;
-                const bool valid = c < vpr;
-                float amax = 0.0f;
+        for (int u = 0; u < U; ++u) {
+            const uint32_t ibase = w0 + u * stride;
+            if (ibase >= nv) break;                  // warp-uniform
+            const uint32_t i = ibase + lane;
+            float amax = 0.0f;
 #pragma unroll
-                for (int k = 0; k < V; ++k) amax = fmaxf(amax, fabsf(v[u][k]));
+            for (int k = 0; k < V; ++k) amax = fmaxf(amax, fabsf(v[u][k]));
 #pragma unroll
-                for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
 
-                uint32_t sfq = 0;
-                float rcp = 0.0f;
-                if ((lane & (TPB - 1)) == 0) {
-                    const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
-                    sfq = f32_to_e4m3(sf32);
-                    const float sfd = e4m3_to_f32(sfq);
-                    rcp = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
-                }
-                const uint32_t leader = lane & ~static_cast<uint32_t>(TPB - 1);
-                rcp = __shfl_sync(0xffffffffu, rcp, leader);
+            uint32_t sfq = 0;
+            float rcp = 0.0f;
+            if ((lane & (TPB - 1)) == 0) {
+                const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+                sfq = f32_to_e4m3(sf32);
+                const float sfd = e4m3_to_f32(sfq);
+                rcp = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
+            }
+            const uint32_t leader = lane & ~static_cast<uint32_t>(TPB - 1);
+            rcp = __shfl_sync(0xffffffffu, rcp, leader);
 
-                uint32_t packed = 0;
+            uint32_t packed = 0;
 #pragma unroll
-                for (int k = 0; k < V; k += 2)
-                    packed |= f32x2_to_e2m1x2(__fmul_rn(v[u][k], rcp), __fmul_rn(v[u][k + 1], rcp)) << (4 * k);
-                if (valid) {
-                    uint8_t* dst = qrow + static_cast<int64_t>(c) * (V / 2);
-                    if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
-                    else *reinterpret_cast<uint32_t*>(dst) = packed;
-                    if ((lane & (TPB - 1)) == 0) sfrow[c / TPB] = static_cast<uint8_t>(sfq);
-                }
+            for (int k = 0; k < V; k += 2)
+                packed |= f32x2_to_e2m1x2(__fmul_rn(v[u][k], rcp), __fmul_rn(v[u][k + 1], rcp)) << (4 * k);
+            if (i < nv) {
+                uint8_t* dst = q + static_cast<int64_t>(i) * (V / 2);
+                if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+                else *reinterpret_cast<uint32_t*>(dst) = packed;
+                if ((lane & (TPB - 1)) == 0) sf[i / TPB] = static_cast<uint8_t>(sfq);
             }
         }
     }
@@ -202,11 +234,11 @@ __device__ __forceinline__ void quantize_rows(const T* __restrict__ x, uint32_t 
 // ------------------------------------------------------------------ global scale
 
 template <typename T>
-__global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, uint32_t rows, uint32_t vpr,
-                                                   int64_t ld, unsigned* __restrict__ acc_bits)
+__global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, const VecIndex ix, uint32_t nv,
+                                                   unsigned* __restrict__ acc_bits)
 {
     __shared__ float red[32];
-    float m = amax_partial(x, rows, vpr, ld);
+    float m = amax_partial(x, ix, nv, blockIdx.x, gridDim.x);
     m = block_max(m, red);
     // non-negative floats order like their bit patterns
     if (threadIdx.x == 0) atomicMax(acc_bits, __float_as_uint(m));
@@ -242,11 +274,11 @@ __global__ void alpha_kernel(const float* __restrict__ gs_a, const float* __rest
 // ------------------------------------------------------------------ quantisation
 
 template <typename T>
-__global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, uint32_t rows, uint32_t vpr,
-                                                       int64_t ldx, int64_t K, const float* __restrict__ gs_ptr,
+__global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, const VecIndex ix, uint32_t nv,
+                                                       const float* __restrict__ gs_ptr,
                                                        uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
 {
-    quantize_rows(x, rows, vpr, ldx, K, __ldg(gs_ptr), q, sf);
+    quantize_vectors(x, ix, nv, blockIdx.x, gridDim.x, __ldg(gs_ptr), q, sf);
 }
 
 // One cooperative launch: amax of the whole tensor -> grid barrier -> global scale (and the
@@ -255,7 +287,7 @@ __global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, 
 // the codes); the launcher keeps gridDim.x * 4 <= rows * K / 2.
 template <typename T>
 __global__ void __launch_bounds__(512) quantize_dynamic_kernel(
-    const T* __restrict__ x, uint32_t rows, uint32_t vpr, int64_t ldx, int64_t K,
+    const T* __restrict__ x, const VecIndex ix, uint32_t nv,
     float* __restrict__ gs_out, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
     const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out)
 {
@@ -263,10 +295,11 @@ __global__ void __launch_bounds__(512) quantize_dynamic_kernel(
     cg::grid_group grid = cg::this_grid();
     __shared__ float red[32];
     float* partial = reinterpret_cast<float*>(q);
-    const uint32_t nblocks = gridDim.x * gridDim.y;
-    const uint32_t bid = blockIdx.y * gridDim.x + blockIdx.x;
+    const uint32_t nblocks = gridDim.x;
+    const uint32_t bid = blockIdx.x;
+    grid_dependency_wait();      // launched early behind the previous kernel: wait for its data
 
-    float m = amax_partial(x, rows, vpr, ldx);
+    float m = amax_partial(x, ix, nv, bid, nblocks);
     m = block_max(m, red);
     if (threadIdx.x == 0) partial[bid] = m;
     grid.sync();
@@ -284,22 +317,23 @@ __global__ void __launch_bounds__(512) quantize_dynamic_kernel(
     // a dependent GEMM may start its prologue now (it waits for this grid before reading)
     cudaTriggerProgrammaticLaunchCompletion();
 
-    quantize_rows(x, rows, vpr, ldx, K, gs, q, sf);
+    quantize_vectors(x, ix, nv, bid, nblocks, gs, q, sf);
 }
 
 // The same operation for small tensors in one thread-block cluster (no cooperative launch,
-// no grid barrier): blockIdx.y strides over rows, every CTA reduces its rows' maxima, the
-// cluster exchanges the per-CTA maxima through distributed shared memory, and every CTA
-// then quantises its rows. gridDim = (1, cluster size, 1).
+// no grid barrier): every CTA reduces the maxima of its share of the vectors, the cluster
+// exchanges the per-CTA maxima through distributed shared memory, and every CTA then
+// quantises its share. gridDim = (1, cluster size, 1).
 template <typename T>
 __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
-    const T* __restrict__ x, uint32_t rows, uint32_t vpr, int64_t ldx, int64_t K,
+    const T* __restrict__ x, const VecIndex ix, uint32_t nv,
     float* __restrict__ gs_out, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
     const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out)
 {
     __shared__ float red[32];
     __shared__ float cta_max;
-    float m = amax_partial(x, rows, vpr, ldx);
+    grid_dependency_wait();      // launched early behind the previous kernel: wait for its data
+    float m = amax_partial(x, ix, nv, blockIdx.y, gridDim.y);
     m = block_max(m, red);
     if (threadIdx.x == 0) cta_max = m;
     cluster_sync();                                   // every CTA's maximum is in place
@@ -322,7 +356,7 @@ __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
             alpha_out[i] = __fdiv_rn(1.0f, __fmul_rn(gs, gs_other[i]));
     }
     cudaTriggerProgrammaticLaunchCompletion();
-    quantize_rows(x, rows, vpr, ldx, K, gs, q, sf);
+    quantize_vectors(x, ix, nv, blockIdx.y, gridDim.y, gs, q, sf);
     cluster_wait();                                   // no CTA leaves while a peer may read it
 }
 
@@ -344,16 +378,14 @@ __global__ void round_e2m1_kernel(const float* __restrict__ x, int64_t n, uint8_
 
 // ------------------------------------------------------------------ launchers
 
-// 2-D grid for a [rows, vpr-vector] sweep with 512-thread blocks, at most `cap` blocks.
-static dim3 grid_2d(int64_t rows, int64_t vpr, int64_t cap)
+// Blocks of 512 threads for a sweep over nv vectors (kUnroll per thread per pass), at most
+// `cap`.
+static int grid_1d(int64_t nv, int64_t cap)
 {
-    int64_t gx = (vpr + 511) / 512;
-    if (gx > cap) gx = cap;
-    if (gx < 1) gx = 1;
-    int64_t gy = std::min<int64_t>(rows, std::max<int64_t>(cap / gx, 1));
-    gy = std::min<int64_t>(gy, 65535);
-    if (gy < 1) gy = 1;
-    return dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), 1);
+    int64_t g = (nv + 512 * kUnroll - 1) / (512 * kUnroll);
+    if (g > cap) g = cap;
+    if (g < 1) g = 1;
+    return static_cast<int>(g);
 }
 
 static int grid_for(int64_t threads, int num_sms)
@@ -375,18 +407,23 @@ cudaError_t launch_global_scale(const void* x, bool bf16, int64_t numel, float* 
         const int V = bf16 ? 8 : 4;
         const int64_t nvec = numel / V;
         if (nvec > 0) {
-            if (nvec >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
-            const dim3 grid = grid_2d(1, nvec, static_cast<int64_t>(num_sms) * 4);
-            if (bf16)
-                amax_kernel<__nv_bfloat16><<<grid, 512, 0, stream>>>(
-                    static_cast<const __nv_bfloat16*>(x), 1u, static_cast<uint32_t>(nvec), 0,
-                    reinterpret_cast<unsigned*>(gs));
-            else
-                amax_kernel<float><<<grid, 512, 0, stream>>>(
-                    static_cast<const float*>(x), 1u, static_cast<uint32_t>(nvec), 0,
-                    reinterpret_cast<unsigned*>(gs));
-            e = cudaGetLastError();
-            if (e != cudaSuccess) return e;
+            // pieces of fewer than 2^31 vectors; the maxima meet in one atomicMax word
+            const int64_t piece = int64_t(1) << 30;
+            for (int64_t v0 = 0; v0 < nvec; v0 += piece) {
+                const int64_t n = std::min(piece, nvec - v0);
+                const VecIndex ix = make_vec_index(n, n * V, n * V);
+                const int grid = grid_1d(n, static_cast<int64_t>(num_sms) * 4);
+                if (bf16)
+                    amax_kernel<__nv_bfloat16><<<grid, 512, 0, stream>>>(
+                        static_cast<const __nv_bfloat16*>(x) + v0 * V, ix, static_cast<uint32_t>(n),
+                        reinterpret_cast<unsigned*>(gs));
+                else
+                    amax_kernel<float><<<grid, 512, 0, stream>>>(
+                        static_cast<const float*>(x) + v0 * V, ix, static_cast<uint32_t>(n),
+                        reinterpret_cast<unsigned*>(gs));
+                e = cudaGetLastError();
+                if (e != cudaSuccess) return e;
+            }
         }
         const int64_t tail = numel - nvec * V;
         if (tail > 0) {
@@ -413,16 +450,27 @@ cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, i
     const int V = bf16 ? 8 : 4;
     const int64_t vpr = K / V;
     if (rows == 0 || vpr == 0) return cudaSuccess;
-    const dim3 grid = grid_2d(rows, vpr, static_cast<int64_t>(num_sms) * 4);
-    if (bf16)
-        quantize_kernel<__nv_bfloat16><<<grid, 512, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), static_cast<uint32_t>(rows),
-            static_cast<uint32_t>(vpr), ldx, K, gs, q, sf);
-    else
-        quantize_kernel<float><<<grid, 512, 0, stream>>>(static_cast<const float*>(x),
-                                                         static_cast<uint32_t>(rows),
-                                                         static_cast<uint32_t>(vpr), ldx, K, gs, q, sf);
-    return cudaGetLastError();
+    const VecIndex ix = make_vec_index(vpr, ldx, K);
+    // row pieces of fewer than 2^31 vectors (rows are independent once gs is known)
+    const int64_t piece_rows = std::max<int64_t>(1, (int64_t(1) << 30) / vpr);
+    const size_t esz = bf16 ? 2 : 4;
+    for (int64_t r0 = 0; r0 < rows; r0 += piece_rows) {
+        const int64_t n_rows = std::min(piece_rows, rows - r0);
+        const int64_t nv = n_rows * vpr;
+        const int grid = grid_1d(nv, static_cast<int64_t>(num_sms) * 4);
+        const void* xp = static_cast<const uint8_t*>(x) + static_cast<size_t>(r0 * ldx) * esz;
+        uint8_t* qp = q + r0 * (K / 2);
+        uint8_t* sp = sf + r0 * (K / 16);
+        if (bf16)
+            quantize_kernel<__nv_bfloat16><<<grid, 512, 0, stream>>>(
+                static_cast<const __nv_bfloat16*>(xp), ix, static_cast<uint32_t>(nv), gs, qp, sp);
+        else
+            quantize_kernel<float><<<grid, 512, 0, stream>>>(
+                static_cast<const float*>(xp), ix, static_cast<uint32_t>(nv), gs, qp, sp);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 // Largest cluster (16, else 8) of 512-thread quantiser CTAs the device runs; cached.
@@ -470,24 +518,27 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
                                     cudaStream_t stream, int num_sms)
 {
     const int64_t bytes = rows * K * static_cast<int64_t>(sizeof(T));
+    const int64_t nv = rows * vpr;                       // < 2^31 (checked by the caller)
+    const VecIndex ix = make_vec_index(vpr, ldx, K);
     const int ccs = bytes <= kClusterQuantizeMaxBytes ? quantize_cluster_size<T>() : 0;
     if (ccs > 0) {
-        const int cs = static_cast<int>(std::min<int64_t>(ccs, rows));
+        const int cs = static_cast<int>(std::min<int64_t>(ccs, (nv + 511) / 512));
         cudaLaunchConfig_t cfg;
         std::memset(&cfg, 0, sizeof(cfg));
         cfg.gridDim = dim3(1, static_cast<unsigned>(cs), 1);
         cfg.blockDim = dim3(512, 1, 1);
         cfg.stream = stream;
-        cudaLaunchAttribute attr;
-        attr.id = cudaLaunchAttributeClusterDimension;
-        attr.val.clusterDim.x = 1;
-        attr.val.clusterDim.y = static_cast<unsigned>(cs);
-        attr.val.clusterDim.z = 1;
-        cfg.attrs = &attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, quantize_dynamic_cluster_kernel<T>, x, static_cast<uint32_t>(rows),
-                                  static_cast<uint32_t>(vpr), ldx, K, gs_out, q, sf, gs_other, n_alpha,
-                                  alpha_out);
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = static_cast<unsigned>(cs);
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        return cudaLaunchKernelEx(&cfg, quantize_dynamic_cluster_kernel<T>, x, ix, static_cast<uint32_t>(nv),
+                                  gs_out, q, sf, gs_other, n_alpha, alpha_out);
     }
     auto kern = quantize_dynamic_kernel<T>;
     int per_sm = 0;
@@ -499,19 +550,28 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
     // barrier participants
     int64_t cap = static_cast<int64_t>(std::min(std::max(per_sm, 1), 2)) * num_sms;
     cap = std::min<int64_t>(cap, std::max<int64_t>(q_bytes / 4, 1));
-    const dim3 grid = grid_2d(rows, vpr, cap);
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = grid;
+    cfg.gridDim = dim3(static_cast<unsigned>(grid_1d(nv, cap)), 1, 1);
     cfg.blockDim = dim3(512, 1, 1);
     cfg.stream = stream;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeCooperative;
-    attr.val.cooperative = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, x, static_cast<uint32_t>(rows), static_cast<uint32_t>(vpr),
-                              ldx, K, gs_out, q, sf, gs_other, n_alpha, alpha_out);
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t le = cudaLaunchKernelEx(&cfg, kern, x, ix, static_cast<uint32_t>(nv), gs_out, q, sf, gs_other,
+                                        n_alpha, alpha_out);
+    if (le == cudaErrorNotSupported || le == cudaErrorInvalidValue) {
+        // a runtime that refuses the early-launch attribute on a cooperative launch: without it
+        cudaGetLastError();
+        cfg.numAttrs = 1;
+        le = cudaLaunchKernelEx(&cfg, kern, x, ix, static_cast<uint32_t>(nv), gs_out, q, sf, gs_other, n_alpha,
+                                alpha_out);
+    }
+    return le;
 }
 
 cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
