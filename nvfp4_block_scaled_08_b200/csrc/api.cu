@@ -182,8 +182,8 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, nvfp4_in_dtype dtype, int64_t
     nvfp4_status st = current_device(&d);
     if (st != NVFP4_OK) return st;
     return from_cuda(nvfp4::launch_quantize_dynamic(x, dtype == NVFP4_IN_BF16, rows, K, ld_x, gs_out,
-                                                    q, sf, gs_other, n_alpha, alpha_out, stream,
-                                                    d.num_sms));
+                                                    q, sf, gs_other, n_alpha, alpha_out, d.err_word,
+                                                    stream, d.num_sms));
 }
 
 nvfp4_status nvfp4_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,

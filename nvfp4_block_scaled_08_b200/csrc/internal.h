@@ -18,8 +18,8 @@ cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, i
                             int num_sms);
 cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
                                     float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
-                                    int32_t n_alpha, float* alpha_out, cudaStream_t stream,
-                                    int num_sms);
+                                    int32_t n_alpha, float* alpha_out, unsigned* err_word,
+                                    cudaStream_t stream, int num_sms);
 cudaError_t launch_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
                          cudaStream_t stream);
 cudaError_t launch_round(const float* x, int64_t n, uint8_t* out, bool e2m1, cudaStream_t stream,

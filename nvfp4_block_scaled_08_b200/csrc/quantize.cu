@@ -56,17 +56,16 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi)
 template <typename T> struct InTraits;
 template <> struct InTraits<float> {
     static constexpr int kPerThread = 4;   // 16 bytes
-    __device__ static void load(const float* p, float (&v)[4])
+    __device__ static void decode(const uint4 u, float (&v)[4])
     {
-        const float4 f = __ldg(reinterpret_cast<const float4*>(p));
-        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+        v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
     }
 };
 template <> struct InTraits<__nv_bfloat16> {
     static constexpr int kPerThread = 8;   // 16 bytes
-    __device__ static void load(const __nv_bfloat16* p, float (&v)[8])
+    __device__ static void decode(const uint4 u, float (&v)[8])
     {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -139,66 +138,77 @@ __device__ __forceinline__ float block_max(float m, float* red)
     return m;
 }
 
-// max |x| over this thread's vectors: block `bid` of `nb` blocks, kUnroll loads in flight.
+// Where a sweep's 16-byte vectors come from: global memory (vector i of the tensor), or this
+// block's shared-memory copy of vectors [v0, v1) (stash[i - v0]).
 template <typename T>
-__device__ __forceinline__ float amax_partial(const T* x, const VecIndex& ix, uint32_t nv, uint32_t bid,
-                                              uint32_t nb)
+struct GlobalVecs {
+    const T* x;
+    VecIndex ix;
+    __device__ uint4 operator()(uint32_t i) const
+    {
+        return __ldg(reinterpret_cast<const uint4*>(x + vec_offset<InTraits<T>::kPerThread>(ix, i)));
+    }
+};
+struct StashVecs {
+    const uint4* stash;
+    uint32_t v0;
+    __device__ uint4 operator()(uint32_t i) const { return stash[i - v0]; }
+};
+
+// max |x| over vectors i0, i0 + step, ... < end of this thread, kUnroll loads in flight. With
+// `keep`, every loaded vector is also copied to stash[i - v0] (the block's own range).
+template <typename T, typename Src>
+__device__ __forceinline__ float amax_sweep(const Src& src, uint32_t i0, uint32_t end, uint32_t step,
+                                            uint4* keep = nullptr, uint32_t v0 = 0)
 {
     constexpr int V = InTraits<T>::kPerThread;
     constexpr int U = kUnroll;
-    const uint32_t stride = nb * blockDim.x;
     float m = 0.0f;
-    for (uint32_t i0 = bid * blockDim.x + threadIdx.x; i0 < nv; i0 += U * stride) {
-        float v[U][V];
+    for (; i0 < end; i0 += U * step) {
+        uint4 w[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const uint32_t i = i0 + u * stride;
-            if (i < nv) InTraits<T>::load(x + vec_offset<V>(ix, i), v[u]);
-            else {
-#pragma unroll
-                for (int k = 0; k < V; ++k) v[u][k] = 0.0f;
-            }
+            const uint32_t i = i0 + u * step;
+            w[u] = i < end ? src(i) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u)
+        for (int u = 0; u < U; ++u) {
+            const uint32_t i = i0 + u * step;
+            if (keep != nullptr && i < end) keep[i - v0] = w[u];
+            float v[V];
+            InTraits<T>::decode(w[u], v);
 #pragma unroll
-            for (int k = 0; k < V; ++k) m = fmaxf(m, fabsf(v[u][k]));
+            for (int k = 0; k < V; ++k) m = fmaxf(m, fabsf(v[k]));
+        }
     }
     return m;
 }
 
-// Quantise this thread's vectors (block `bid` of `nb`). The TPB lanes that share a
-// 16-element block are consecutive lanes of one warp in the same iteration (each warp
-// takes 32 consecutive vectors, and a block never straddles a row since vpr % TPB == 0);
-// the first of them computes the block scale and shares it.
+// Quantise vectors [.., end): this warp takes the 32 consecutive vectors w0 + lane, then
+// w0 + step + lane, ... (w0 warp-uniform and a multiple of 32). The TPB lanes that share a
+// 16-element block are consecutive lanes of the warp (a block never straddles a row since
+// vpr % TPB == 0); the first of them computes the block scale and shares it.
 // Per block, in fp32 with explicit rounding and in this order:
 //   amax -> s = e4m3(amax / 6 * gs) -> r = s ? gs / s : 0 -> codes e2m1(x * r).
-template <typename T>
-__device__ __forceinline__ void quantize_vectors(const T* __restrict__ x, const VecIndex& ix, uint32_t nv,
-                                                 uint32_t bid, uint32_t nb, float gs,
-                                                 uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
+template <typename T, typename Src>
+__device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint32_t end, uint32_t step,
+                                               float gs, uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
 {
     constexpr int V = InTraits<T>::kPerThread;   // elements per thread
     constexpr int TPB = 16 / V;                  // threads per 16-element block
     constexpr int U = kUnroll;
     const uint32_t lane = threadIdx.x & 31;
-    const uint32_t stride = nb * blockDim.x;
-    for (uint32_t w0 = bid * blockDim.x + threadIdx.x - lane; w0 < nv; w0 += U * stride) {   // warp-uniform
+    for (; w0 < end; w0 += U * step) {           // warp-uniform
         float v[U][V];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const uint32_t i = w0 + u * stride + lane;
-            if (i < nv) {
-                InTraits<T>::load(x + vec_offset<V>(ix, i), v[u]);
-            } else {
-#pragma unroll
-                for (int k = 0; k < V; ++k) v[u][k] = 0.0f;
-            }
+            const uint32_t i = w0 + u * step + lane;
+            InTraits<T>::decode(i < end ? src(i) : make_uint4(0u, 0u, 0u, 0u), v[u]);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const uint32_t ibase = w0 + u * stride;
-            if (ibase >= nv) break;                  // warp-uniform
+            const uint32_t ibase = w0 + u * step;
+            if (ibase >= end) break;                 // warp-uniform
             const uint32_t i = ibase + lane;
             float amax = 0.0f;
 #pragma unroll
@@ -221,7 +231,7 @@ __device__ __forceinline__ void quantize_vectors(const T* __restrict__ x, const 
 #pragma unroll
             for (int k = 0; k < V; k += 2)
                 packed |= f32x2_to_e2m1x2(__fmul_rn(v[u][k], rcp), __fmul_rn(v[u][k + 1], rcp)) << (4 * k);
-            if (i < nv) {
+            if (i < end) {
                 uint8_t* dst = q + static_cast<int64_t>(i) * (V / 2);
                 if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
                 else *reinterpret_cast<uint32_t*>(dst) = packed;
@@ -231,6 +241,16 @@ __device__ __forceinline__ void quantize_vectors(const T* __restrict__ x, const 
     }
 }
 
+// This block's contiguous share of nv vectors when they are split into blocks of `chunk`
+// (a multiple of 32): [v0, v1).
+__device__ __forceinline__ void block_range(uint32_t nv, uint32_t chunk, uint32_t bid, uint32_t& v0,
+                                            uint32_t& v1)
+{
+    const uint64_t a = static_cast<uint64_t>(bid) * chunk;
+    v0 = static_cast<uint32_t>(a < nv ? a : nv);
+    v1 = static_cast<uint32_t>(a + chunk < nv ? a + chunk : nv);
+}
+
 // ------------------------------------------------------------------ global scale
 
 template <typename T>
@@ -238,7 +258,8 @@ __global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, cons
                                                    unsigned* __restrict__ acc_bits)
 {
     __shared__ float red[32];
-    float m = amax_partial(x, ix, nv, blockIdx.x, gridDim.x);
+    float m = amax_sweep<T>(GlobalVecs<T>{x, ix}, blockIdx.x * blockDim.x + threadIdx.x, nv,
+                            gridDim.x * blockDim.x);
     m = block_max(m, red);
     // non-negative floats order like their bit patterns
     if (threadIdx.x == 0) atomicMax(acc_bits, __float_as_uint(m));
@@ -278,62 +299,114 @@ __global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, 
                                                        const float* __restrict__ gs_ptr,
                                                        uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
 {
-    quantize_vectors(x, ix, nv, blockIdx.x, gridDim.x, __ldg(gs_ptr), q, sf);
+    quantize_sweep<T>(GlobalVecs<T>{x, ix}, blockIdx.x * blockDim.x + (threadIdx.x & ~31u), nv,
+                      gridDim.x * blockDim.x, __ldg(gs_ptr), q, sf);
 }
 
 // One cooperative launch: amax of the whole tensor -> grid barrier -> global scale (and the
-// GEMM alpha against other tensors' global scales) -> grid barrier -> quantisation. The
-// per-block partial maxima are parked in the first bytes of q (overwritten afterwards by
-// the codes); the launcher keeps gridDim.x * 4 <= rows * K / 2.
-template <typename T>
+// GEMM alpha against other tensors' global scales) -> quantisation.
+// RESIDENT: block b reads its contiguous share [b * chunk, ...) of the vectors once, keeps it
+// in shared memory during the barrier and quantises it from there; otherwise the blocks sweep
+// the tensor grid-strided twice (the second time mostly from L2).
+// The per-block maxima are parked in the first 4 * gridDim.x bytes of q, followed by one
+// "read" flag per block (cleared before the barrier, set once the block has read every
+// maximum). Only the blocks whose codes overwrite that area wait for all flags; the launcher
+// keeps gridDim.x * 8 <= rows * K / 2. The wait is bounded; on a timeout the kernel records
+// kErrQuantFlags in err_word and goes on.
+constexpr uint32_t kFlagRead = 0x52454144u;
+constexpr uint32_t kErrQuantFlags = 0x201;
+
+template <typename T, bool RESIDENT>
 __global__ void __launch_bounds__(512) quantize_dynamic_kernel(
-    const T* __restrict__ x, const VecIndex ix, uint32_t nv,
+    const T* __restrict__ x, const VecIndex ix, uint32_t nv, uint32_t chunk,
     float* __restrict__ gs_out, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
-    const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out)
+    const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out,
+    unsigned* __restrict__ err_word)
 {
     namespace cg = cooperative_groups;
+    constexpr int V = InTraits<T>::kPerThread;
     cg::grid_group grid = cg::this_grid();
+    extern __shared__ uint4 stash[];
     __shared__ float red[32];
     float* partial = reinterpret_cast<float*>(q);
+    volatile uint32_t* read_flag = reinterpret_cast<volatile uint32_t*>(q) + gridDim.x;
     const uint32_t nblocks = gridDim.x;
     const uint32_t bid = blockIdx.x;
     grid_dependency_wait();      // launched early behind the previous kernel: wait for its data
 
-    float m = amax_partial(x, ix, nv, bid, nblocks);
+    uint32_t v0 = 0, v1 = 0;
+    float m;
+    if constexpr (RESIDENT) {
+        block_range(nv, chunk, bid, v0, v1);
+        m = amax_sweep<T>(GlobalVecs<T>{x, ix}, v0 + threadIdx.x, v1, blockDim.x, stash, v0);
+    } else {
+        m = amax_sweep<T>(GlobalVecs<T>{x, ix}, bid * blockDim.x + threadIdx.x, nv, nblocks * blockDim.x);
+    }
     m = block_max(m, red);
-    if (threadIdx.x == 0) partial[bid] = m;
+    if (threadIdx.x == 0) {
+        partial[bid] = m;
+        read_flag[bid] = 0u;
+    }
     grid.sync();
 
     float a = 0.0f;
     for (uint32_t i = threadIdx.x; i < nblocks; i += blockDim.x) a = fmaxf(a, __ldcg(partial + i));
-    a = block_max(a, red);
+    a = block_max(a, red);       // ends with __syncthreads: every read of the maxima is done
     const float gs = (a == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, a);
+    if (threadIdx.x == 0) {
+        __threadfence();
+        read_flag[bid] = kFlagRead;
+    }
     if (bid == 0) {
         if (threadIdx.x == 0) *gs_out = gs;
         for (int32_t i = threadIdx.x; i < n_alpha; i += blockDim.x)
             alpha_out[i] = __fdiv_rn(1.0f, __fmul_rn(gs, gs_other[i]));
     }
-    grid.sync();   // every block has read the partial maxima before q is overwritten
     // a dependent GEMM may start its prologue now (it waits for this grid before reading)
     cudaTriggerProgrammaticLaunchCompletion();
 
-    quantize_vectors(x, ix, nv, bid, nblocks, gs, q, sf);
+    // this block's first code byte; the parked area is q[0, 8 * nblocks)
+    const uint32_t first_vec = RESIDENT ? v0 : bid * blockDim.x;
+    if (static_cast<uint64_t>(first_vec) * (V / 2) < 8ull * nblocks) {
+        // every thread watches its own flags (one L2 round trip, not one per block)
+        const uint64_t t0 = globaltimer_ns();
+        bool late = false;
+        for (uint32_t b = threadIdx.x; b < nblocks && !late; b += blockDim.x) {
+            while (read_flag[b] != kFlagRead) {
+                if (globaltimer_ns() - t0 > kWaitTimeoutNs) { late = true; break; }
+            }
+        }
+        if (late) atomicCAS(err_word, 0u, kErrQuantFlags);
+        __threadfence();
+        __syncthreads();
+    }
+
+    if constexpr (RESIDENT) {
+        quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, q, sf);
+    } else {
+        quantize_sweep<T>(GlobalVecs<T>{x, ix}, bid * blockDim.x + (threadIdx.x & ~31u), nv,
+                          nblocks * blockDim.x, gs, q, sf);
+    }
 }
 
 // The same operation for small tensors in one thread-block cluster (no cooperative launch,
-// no grid barrier): every CTA reduces the maxima of its share of the vectors, the cluster
-// exchanges the per-CTA maxima through distributed shared memory, and every CTA then
-// quantises its share. gridDim = (1, cluster size, 1).
+// no grid barrier): CTA r reads its contiguous share [r * chunk, ...) once into shared
+// memory and reduces its maximum, the cluster exchanges the per-CTA maxima through
+// distributed shared memory, and every CTA quantises its share from shared memory.
+// gridDim = (1, cluster size, 1).
 template <typename T>
 __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
-    const T* __restrict__ x, const VecIndex ix, uint32_t nv,
+    const T* __restrict__ x, const VecIndex ix, uint32_t nv, uint32_t chunk,
     float* __restrict__ gs_out, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
     const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out)
 {
+    extern __shared__ uint4 stash[];
     __shared__ float red[32];
     __shared__ float cta_max;
     grid_dependency_wait();      // launched early behind the previous kernel: wait for its data
-    float m = amax_partial(x, ix, nv, blockIdx.y, gridDim.y);
+    uint32_t v0, v1;
+    block_range(nv, chunk, blockIdx.y, v0, v1);
+    float m = amax_sweep<T>(GlobalVecs<T>{x, ix}, v0 + threadIdx.x, v1, blockDim.x, stash, v0);
     m = block_max(m, red);
     if (threadIdx.x == 0) cta_max = m;
     cluster_sync();                                   // every CTA's maximum is in place
@@ -356,7 +429,7 @@ __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
             alpha_out[i] = __fdiv_rn(1.0f, __fmul_rn(gs, gs_other[i]));
     }
     cudaTriggerProgrammaticLaunchCompletion();
-    quantize_vectors(x, ix, nv, blockIdx.y, gridDim.y, gs, q, sf);
+    quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, q, sf);
     cluster_wait();                                   // no CTA leaves while a peer may read it
 }
 
@@ -510,23 +583,37 @@ static int quantize_cluster_size()
 // Tensors up to this size are quantised by one cluster; larger ones by a cooperative grid
 // (measured on B200: one 16-CTA cluster wins at 393 KB, loses from 1.5 MB up).
 constexpr int64_t kClusterQuantizeMaxBytes = int64_t(512) << 10;
+// Largest shared-memory share per block for the resident cooperative quantiser (two blocks
+// per SM); larger tensors are swept twice instead.
+constexpr int64_t kResidentMaxBytes = int64_t(100) << 10;
+
+static inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 template <typename T>
 static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64_t ldx, int64_t K,
                                     float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
                                     int32_t n_alpha, float* alpha_out, int64_t q_bytes,
-                                    cudaStream_t stream, int num_sms)
+                                    unsigned* err_word, cudaStream_t stream, int num_sms)
 {
     const int64_t bytes = rows * K * static_cast<int64_t>(sizeof(T));
     const int64_t nv = rows * vpr;                       // < 2^31 (checked by the caller)
     const VecIndex ix = make_vec_index(vpr, ldx, K);
     const int ccs = bytes <= kClusterQuantizeMaxBytes ? quantize_cluster_size<T>() : 0;
     if (ccs > 0) {
-        const int cs = static_cast<int>(std::min<int64_t>(ccs, (nv + 511) / 512));
+        const int cs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ccs, (nv + 511) / 512)));
+        const int64_t chunk = round_up((nv + cs - 1) / cs, 32);
+        auto kern = quantize_dynamic_cluster_kernel<T>;
+        static std::once_flag once;
+        std::call_once(once, [&] {
+            // a cluster of >= 8 CTAs: at most 512 KB / 8 of vectors per CTA
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kClusterQuantizeMaxBytes / 8 + 512 * 16));
+        });
         cudaLaunchConfig_t cfg;
         std::memset(&cfg, 0, sizeof(cfg));
         cfg.gridDim = dim3(1, static_cast<unsigned>(cs), 1);
         cfg.blockDim = dim3(512, 1, 1);
+        cfg.dynamicSmemBytes = static_cast<size_t>(chunk) * 16;
         cfg.stream = stream;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -537,23 +624,49 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 2;
-        return cudaLaunchKernelEx(&cfg, quantize_dynamic_cluster_kernel<T>, x, ix, static_cast<uint32_t>(nv),
+        return cudaLaunchKernelEx(&cfg, kern, x, ix, static_cast<uint32_t>(nv), static_cast<uint32_t>(chunk),
                                   gs_out, q, sf, gs_other, n_alpha, alpha_out);
     }
-    auto kern = quantize_dynamic_kernel<T>;
+
+    // Cooperative grid: two 512-thread blocks per SM at most (enough warps to hide the
+    // arithmetic, few grid-barrier participants), at least two vectors per thread, and room
+    // for the parked maxima and flags (8 bytes per block) in q.
+    int64_t blocks = std::min<int64_t>(2 * static_cast<int64_t>(num_sms), (nv + 1023) / 1024);
+    blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, q_bytes / 8));
+    int64_t chunk = round_up((nv + blocks - 1) / blocks, 32);
+    bool resident = chunk * 16 <= kResidentMaxBytes;
+    void (*kern)(const T*, const VecIndex, uint32_t, uint32_t, float*, uint8_t*, uint8_t*, const float*,
+                 int32_t, float*, unsigned*) =
+        resident ? quantize_dynamic_kernel<T, true> : quantize_dynamic_kernel<T, false>;
+    size_t smem = 0;
+    if (resident) {
+        static std::once_flag once;
+        std::call_once(once, [] {
+            cudaFuncSetAttribute(quantize_dynamic_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kResidentMaxBytes));
+        });
+        smem = static_cast<size_t>(chunk) * 16;
+    }
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 512, 0);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 512, smem);
     if (e != cudaSuccess) return e;
-    // co-resident blocks only (cooperative), few of them (cheap grid barriers), and room
-    // for one partial maximum per block in q
-    // two 512-thread blocks per SM at most: enough warps to hide the arithmetic, few grid
-    // barrier participants
-    int64_t cap = static_cast<int64_t>(std::min(std::max(per_sm, 1), 2)) * num_sms;
-    cap = std::min<int64_t>(cap, std::max<int64_t>(q_bytes / 4, 1));
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t fit = static_cast<int64_t>(std::min(per_sm, 2)) * num_sms;   // co-resident blocks
+    if (resident) {
+        if (blocks > fit) {        // fewer blocks than planned: larger shares (same smem bound)
+            blocks = fit;
+            chunk = round_up((nv + blocks - 1) / blocks, 32);
+            if (chunk * 16 > static_cast<int64_t>(smem)) return cudaErrorInvalidConfiguration;
+        }
+        blocks = (nv + chunk - 1) / chunk;       // no empty block
+    } else {
+        blocks = std::min(blocks, fit);
+    }
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>(grid_1d(nv, cap)), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
     cfg.blockDim = dim3(512, 1, 1);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -562,31 +675,32 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaError_t le = cudaLaunchKernelEx(&cfg, kern, x, ix, static_cast<uint32_t>(nv), gs_out, q, sf, gs_other,
-                                        n_alpha, alpha_out);
+    const uint32_t nv32 = static_cast<uint32_t>(nv), chunk32 = static_cast<uint32_t>(chunk);
+    cudaError_t le = cudaLaunchKernelEx(&cfg, kern, x, ix, nv32, chunk32, gs_out, q, sf, gs_other, n_alpha,
+                                        alpha_out, err_word);
     if (le == cudaErrorNotSupported || le == cudaErrorInvalidValue) {
         // a runtime that refuses the early-launch attribute on a cooperative launch: without it
         cudaGetLastError();
         cfg.numAttrs = 1;
-        le = cudaLaunchKernelEx(&cfg, kern, x, ix, static_cast<uint32_t>(nv), gs_out, q, sf, gs_other, n_alpha,
-                                alpha_out);
+        le = cudaLaunchKernelEx(&cfg, kern, x, ix, nv32, chunk32, gs_out, q, sf, gs_other, n_alpha, alpha_out,
+                                err_word);
     }
     return le;
 }
 
 cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
                                     float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
-                                    int32_t n_alpha, float* alpha_out, cudaStream_t stream,
-                                    int num_sms)
+                                    int32_t n_alpha, float* alpha_out, unsigned* err_word,
+                                    cudaStream_t stream, int num_sms)
 {
     const int V = bf16 ? 8 : 4;
     const int64_t vpr = K / V;
     const int64_t q_bytes = rows * (K / 2);
     if (bf16)
         return launch_dynamic_t(static_cast<const __nv_bfloat16*>(x), rows, vpr, ldx, K, gs_out, q, sf,
-                                gs_other, n_alpha, alpha_out, q_bytes, stream, num_sms);
+                                gs_other, n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
     return launch_dynamic_t(static_cast<const float*>(x), rows, vpr, ldx, K, gs_out, q, sf, gs_other,
-                            n_alpha, alpha_out, q_bytes, stream, num_sms);
+                            n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
 }
 
 cudaError_t launch_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
