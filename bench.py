@@ -23,6 +23,9 @@ e2e: the same metric through the public Python API called eagerly per step, with
 activations copied from pinned host memory and the outputs copied back inside the timed
 region.
 
+context (rank 0, after the timed step, --no-context skips it): the compute-bound 8192^3 GEMM
+against the FP4 tensor peak, and 512 x 2048 x 6144 beside a bf16 torch matmul of that shape.
+
 --impl reference: the CPU oracle as it stands (test infrastructure), on a bounded sample
 of the same workload per step, on this machine's host cores.
 
@@ -90,6 +93,26 @@ def max_over_ranks(x: float, world: int) -> float:
 def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> float:
     """TFLOP/s of the whole job: every rank's work over the slowest rank's step time."""
     return flops_per_rank * world / (step_ms_max * 1e-3) / 1e12
+
+
+# DRAM traffic of the GEMM launches of one sweep (M = 16, 64, 256, 1024), from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum, cold L2; the bf16 outputs stay in L2 within a
+# launch): 2763776 + 2935040 + 3601920 + 6256128 bytes; the capture command and its table are
+# in the committed ncu summary of these launches under profiles/. Valid only for the kernel
+# sources it was taken on (hash below); reported as null otherwise.
+GEMM_TRAFFIC_BYTES = 2763776 + 2935040 + 3601920 + 6256128
+GEMM_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "gemm.cu", "ptx.cuh", "internal.h")
+GEMM_TRAFFIC_SHA = "2843df9afe82c1e8"
+
+
+def gemm_traffic():
+    """The captured traffic, or None once the GEMM sources differ from the captured ones."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "nvfp4_block_scaled_08_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return GEMM_TRAFFIC_BYTES if h.hexdigest()[:16] == GEMM_TRAFFIC_SHA else None
 
 
 def measured_peaks():
@@ -292,6 +315,63 @@ class AttnSweep:
         return sum(it["out"].numel() * 2 for it in self.items)
 
 
+def graph_time_us(fn, reps: int, iters: int = 5) -> float:
+    """Median device time of one call, from CUDA graphs of `reps` back-to-back calls."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    ts = []
+    for _ in range(iters):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        g.replay()
+        e.record()
+        e.synchronize()
+        ts.append(s.elapsed_time(e) * 1e3 / reps)
+    del g
+    return statistics.median(ts)
+
+
+def context_gemms(dev, peaks):
+    """Context outside the timed step, from the compute-bound configurations: the 8192^3
+    NVFP4 GEMM (uniform(-1, 1) inputs, quantised on the device) against the FP4 tensor peak,
+    and the 512 x 2048 x 6144 NVFP4 GEMM beside a bf16 torch matmul of the same shape."""
+    import nvfp4_block_scaled_08_b200 as nv
+    from nvfp4_block_scaled_08_b200 import workloads
+    p_fp4 = peaks["bf16_tflops"] * FP4_PER_BF16
+    out = {}
+    for c in workloads.plateau_cases():
+        if c.name not in ("square_8192", "ratio_512x2048x6144"):
+            continue
+        a, b = c.a().to(dev), c.b().to(dev)
+        gsa, gsb = nv.global_scale(a), nv.global_scale(b)
+        qa, sa = nv.quantize(a, gsa)
+        qb, sb = nv.quantize(b, gsb)
+        al = nv.alpha(gsa, gsb)
+        o = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+        ws = nv.make_workspace(c.M, c.N, c.K, dev)
+        us = graph_time_us(lambda: nv.gemm(qa, sa, qb, sb, al, out=o, workspace=ws),
+                           reps=5 if c.M >= 8192 else 20)
+        tf = c.flops / (us * 1e-6) / 1e12
+        item = {"M": c.M, "N": c.N, "K": c.K, "us": round(us, 2), "tflops": round(tf, 1),
+                "frac_of_fp4_peak": round(tf / p_fp4, 4),
+                "fp4_peak_tflops": round(p_fp4, 1), "peak_source": "measured bf16 burst x 4"}
+        if c.name.startswith("ratio"):
+            ab, bb = a.to(torch.bfloat16), b.to(torch.bfloat16)
+            ub = graph_time_us(lambda: torch.matmul(ab, bb.t()), reps=20)
+            item["bf16_torch_us"] = round(ub, 2)
+            item["fp4_over_bf16"] = round(ub / us, 3)
+            del ab, bb
+        out[c.name] = item
+        del a, b, qa, sa, qb, sb, o, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     peaks = measured_peaks()
@@ -398,7 +478,7 @@ def run_ours(args, world, rank, local):
         units = f"{tot_quant_bytes:.0f} algorithmic bytes per sweep"
     roof = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": None, "per": units,
+            "traffic": gemm_traffic() if gemm_dominant else None, "per": units,
             "peak_source": f"{peaks['source']} hbm_gbs (burst copy)"}
 
     line = {
@@ -424,6 +504,8 @@ def run_ours(args, world, rank, local):
         "gemm_only_tflops": round(sweep.flops / (tot_gemm_us * 1e-6) / 1e12, 1),
         "clocks": clocks.summary(),
     }
+    if rank == 0 and not args.no_context:
+        line["context"] = context_gemms(dev, peaks)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     for sw in sets:
@@ -520,6 +602,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-context", action="store_true",
+                    help="skip the compute-bound context GEMMs reported after the timed step")
     ap.add_argument("--sets", type=int, default=8,
                     help="independent input sets rotated between steps (together larger than L2)")
     ap.add_argument("--flush", action="store_true",

@@ -190,9 +190,22 @@ __device__ __forceinline__ float amax_sweep(const Src& src, uint32_t i0, uint32_
 // vpr % TPB == 0); the first of them computes the block scale and shares it.
 // Per block, in fp32 with explicit rounding and in this order:
 //   amax -> s = e4m3(amax / 6 * gs) -> r = s ? gs / s : 0 -> codes e2m1(x * r).
+// rcp_tab[c] = gs / e4m3(c) (0 where e4m3(c) is zero) for all 256 scale codes: every block
+// scale of the tensor shares gs, so the division is done once per code (by the first 256
+// threads), not once per 16-element block. Same operands, same rounding: the same values.
+__device__ __forceinline__ void build_rcp_table(float gs, float* rcp_tab)
+{
+    if (threadIdx.x < 256) {
+        const float sfd = e4m3_to_f32(threadIdx.x);
+        rcp_tab[threadIdx.x] = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
+    }
+    __syncthreads();
+}
+
 template <typename T, typename Src>
 __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint32_t end, uint32_t step,
-                                               float gs, uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
+                                               float gs, const float* rcp_tab, uint8_t* __restrict__ q,
+                                               uint8_t* __restrict__ sf)
 {
     constexpr int V = InTraits<T>::kPerThread;   // elements per thread
     constexpr int TPB = 16 / V;                  // threads per 16-element block
@@ -221,8 +234,7 @@ __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint
             if ((lane & (TPB - 1)) == 0) {
                 const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
                 sfq = f32_to_e4m3(sf32);
-                const float sfd = e4m3_to_f32(sfq);
-                rcp = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
+                rcp = rcp_tab[sfq];
             }
             const uint32_t leader = lane & ~static_cast<uint32_t>(TPB - 1);
             rcp = __shfl_sync(0xffffffffu, rcp, leader);
@@ -299,8 +311,11 @@ __global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, 
                                                        const float* __restrict__ gs_ptr,
                                                        uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
 {
+    __shared__ float rcp_tab[256];
+    const float gs = __ldg(gs_ptr);
+    build_rcp_table(gs, rcp_tab);
     quantize_sweep<T>(GlobalVecs<T>{x, ix}, blockIdx.x * blockDim.x + (threadIdx.x & ~31u), nv,
-                      gridDim.x * blockDim.x, __ldg(gs_ptr), q, sf);
+                      gridDim.x * blockDim.x, gs, rcp_tab, q, sf);
 }
 
 // One cooperative launch: amax of the whole tensor -> grid barrier -> global scale (and the
@@ -381,11 +396,13 @@ __global__ void __launch_bounds__(512) quantize_dynamic_kernel(
         __syncthreads();
     }
 
+    __shared__ float rcp_tab[256];
+    build_rcp_table(gs, rcp_tab);
     if constexpr (RESIDENT) {
-        quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, q, sf);
+        quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sf);
     } else {
         quantize_sweep<T>(GlobalVecs<T>{x, ix}, bid * blockDim.x + (threadIdx.x & ~31u), nv,
-                          nblocks * blockDim.x, gs, q, sf);
+                          nblocks * blockDim.x, gs, rcp_tab, q, sf);
     }
 }
 
@@ -429,7 +446,9 @@ __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
             alpha_out[i] = __fdiv_rn(1.0f, __fmul_rn(gs, gs_other[i]));
     }
     cudaTriggerProgrammaticLaunchCompletion();
-    quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, q, sf);
+    __shared__ float rcp_tab[256];
+    build_rcp_table(gs, rcp_tab);
+    quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sf);
     cluster_wait();                                   // no CTA leaves while a peer may read it
 }
 
