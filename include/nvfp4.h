@@ -93,8 +93,9 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t rows, i
  * nvfp4_quantize does, and, for i < n_alpha, writes alpha_out[i] = 1 / (gs_out[0] *
  * gs_other[i]) exactly as nvfp4_alpha does (n_alpha == 0: gs_other / alpha_out unused).
  * Same layouts and requirements as nvfp4_quantize; gs_out, gs_other, alpha_out: device.
- * One cooperative launch (amax, grid barrier, scale, grid barrier, quantise); q is used as
- * scratch for the per-block maxima before it receives the codes. rows * K must be below
+ * One launch (tensors up to 512 KB: one thread-block cluster; larger: a cooperative grid
+ * with one grid barrier). The first 8 bytes per block of q hold the per-block maxima and
+ * "read" flags before they receive the codes. rows * K must be below
  * 2^31 * (16 / sizeof(dtype)).
  */
 nvfp4_status nvfp4_quantize_dynamic(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,

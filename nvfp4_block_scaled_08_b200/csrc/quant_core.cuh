@@ -1,0 +1,260 @@
+// quant_core.cuh -- the NVFP4 quantisation arithmetic shared by the quantiser kernels and the
+// GEMM's fused activation-quantisation phase: format conversions, the flat vector view of a
+// [rows, K] tensor, the amax and quantisation sweeps and the block reductions.
+//
+// Format: packed e2m1 values two per byte with one float8_e4m3fn scale per 16 K-elements
+// ("When a Benchmark Crashes", section "Input Knowledge Required", item 3; block_size=16
+// from "The Art of Reading the Manual", section "The Message"). The pages give no recipe;
+// this library uses the two-level NVFP4 recipe with the fixed fp32 operation order stated
+// in include/nvfp4.h. Every fp32 operation uses an explicitly rounded intrinsic
+// (__fdiv_rn, __fmul_rn), so no contraction or reassociation can change a result.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+// fp32 -> e4m3fn byte, round to nearest even, finite values saturate to +-448.
+__device__ __forceinline__ uint32_t f32_to_e4m3(float v)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(v), "f"(v));
+    return r & 0xFFu;
+}
+
+// e4m3fn byte -> fp32 (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte)
+{
+    const uint16_t pair = static_cast<uint16_t>(byte | (byte << 8));
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// Two fp32 values -> one byte of e2m1 codes (round to nearest even, saturating at +-6),
+// `lo` in the low nibble.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "mov.b32 %0, {t, 0, 0, 0};\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+template <typename T> struct InTraits;
+template <> struct InTraits<float> {
+    static constexpr int kPerThread = 4;   // 16 bytes
+    __device__ static void decode(const uint4 u, float (&v)[4])
+    {
+        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+        v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+    }
+};
+template <> struct InTraits<__nv_bfloat16> {
+    static constexpr int kPerThread = 8;   // 16 bytes
+    __device__ static void decode(const uint4 u, float (&v)[8])
+    {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+
+// ------------------------------------------------------------------ indexing
+
+// A [rows, K] tensor of T (row stride ld elements) is read as nv = rows * vpr 16-byte
+// vectors (V elements each, vpr = K / V per row), numbered row-major: vector i is row
+// i / vpr, column i % vpr. Every launch keeps nv < 2^31, so indices are 32-bit. With
+// contiguous rows (ld == K) vector i sits at x + i * V and no division is needed;
+// otherwise the row comes from a multiply-high by a precomputed reciprocal ("round-up"
+// method of Granlund and Montgomery, PLDI 1994: with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (mulhi(n, m) + n) >> l for every n < 2^32).
+// The codes and scales are written contiguously: vector i's codes at q + i * V / 2, the
+// scale of the 16-element block holding it at sf + i / (16 / V).
+struct VecIndex {
+    uint32_t vpr;      // vectors per row
+    uint32_t mul;      // m above (d = vpr)
+    uint32_t shift;    // l above
+    uint32_t contiguous;
+    int64_t ld;        // row stride in elements
+};
+
+inline VecIndex make_vec_index(int64_t vpr, int64_t ld, int64_t K)
+{
+    VecIndex ix;
+    ix.vpr = static_cast<uint32_t>(vpr);
+    uint32_t l = 0;
+    while ((uint64_t(1) << l) < static_cast<uint64_t>(vpr)) ++l;
+    ix.shift = l;
+    ix.mul = static_cast<uint32_t>(((uint64_t(1) << 32) * ((uint64_t(1) << l) - static_cast<uint64_t>(vpr)))
+                                   / static_cast<uint64_t>(vpr) + 1);
+    ix.contiguous = (ld == K) ? 1u : 0u;
+    ix.ld = ld;
+    return ix;
+}
+
+template <int V>
+__device__ __forceinline__ int64_t vec_offset(const VecIndex& ix, uint32_t i)
+{
+    if (ix.contiguous) return static_cast<int64_t>(i) * V;
+    const uint32_t r = static_cast<uint32_t>((static_cast<uint64_t>(__umulhi(i, ix.mul)) + i) >> ix.shift);
+    const uint32_t c = i - r * ix.vpr;
+    return static_cast<int64_t>(r) * ix.ld + static_cast<int64_t>(c) * V;
+}
+
+// Loads in flight per thread in the sweeps below.
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ float block_max(float m, float* red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.0f;
+    if (threadIdx.x < 32) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (threadIdx.x == 0) red[0] = m;
+    }
+    __syncthreads();
+    m = red[0];
+    __syncthreads();
+    return m;
+}
+
+// Where a sweep's 16-byte vectors come from: global memory (vector i of the tensor), or this
+// block's shared-memory copy of vectors [v0, v1) (stash[i - v0]).
+template <typename T>
+struct GlobalVecs {
+    const T* x;
+    VecIndex ix;
+    __device__ uint4 operator()(uint32_t i) const
+    {
+        return __ldg(reinterpret_cast<const uint4*>(x + vec_offset<InTraits<T>::kPerThread>(ix, i)));
+    }
+};
+struct StashVecs {
+    const uint4* stash;
+    uint32_t v0;
+    __device__ uint4 operator()(uint32_t i) const { return stash[i - v0]; }
+};
+
+// max |x| over vectors i0, i0 + step, ... < end of this thread, kUnroll loads in flight. With
+// `keep`, every loaded vector is also copied to stash[i - v0] (the block's own range).
+template <typename T, typename Src>
+__device__ __forceinline__ float amax_sweep(const Src& src, uint32_t i0, uint32_t end, uint32_t step,
+                                            uint4* keep = nullptr, uint32_t v0 = 0)
+{
+    constexpr int V = InTraits<T>::kPerThread;
+    constexpr int U = kUnroll;
+    float m = 0.0f;
+    for (; i0 < end; i0 += U * step) {
+        uint4 w[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t i = i0 + u * step;
+            w[u] = i < end ? src(i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t i = i0 + u * step;
+            if (keep != nullptr && i < end) keep[i - v0] = w[u];
+            float v[V];
+            InTraits<T>::decode(w[u], v);
+#pragma unroll
+            for (int k = 0; k < V; ++k) m = fmaxf(m, fabsf(v[k]));
+        }
+    }
+    return m;
+}
+
+// Quantise vectors [.., end): this warp takes the 32 consecutive vectors w0 + lane, then
+// w0 + step + lane, ... (w0 warp-uniform and a multiple of 32). The TPB lanes that share a
+// 16-element block are consecutive lanes of the warp (a block never straddles a row since
+// vpr % TPB == 0); the first of them computes the block scale and shares it.
+// Per block, in fp32 with explicit rounding and in this order:
+//   amax -> s = e4m3(amax / 6 * gs) -> r = s ? gs / s : 0 -> codes e2m1(x * r).
+// rcp_tab[c] = gs / e4m3(c) (0 where e4m3(c) is zero) for all 256 scale codes: every block
+// scale of the tensor shares gs, so the division is done once per code (by the first 256
+// threads), not once per 16-element block. Same operands, same rounding: the same values.
+__device__ __forceinline__ void build_rcp_table(float gs, float* rcp_tab)
+{
+    if (threadIdx.x < 256) {
+        const float sfd = e4m3_to_f32(threadIdx.x);
+        rcp_tab[threadIdx.x] = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
+    }
+    __syncthreads();
+}
+
+template <typename T, typename Src>
+__device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint32_t end, uint32_t step,
+                                               float gs, const float* rcp_tab, uint8_t* __restrict__ q,
+                                               uint8_t* __restrict__ sf)
+{
+    constexpr int V = InTraits<T>::kPerThread;   // elements per thread
+    constexpr int TPB = 16 / V;                  // threads per 16-element block
+    constexpr int U = kUnroll;
+    const uint32_t lane = threadIdx.x & 31;
+    for (; w0 < end; w0 += U * step) {           // warp-uniform
+        float v[U][V];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t i = w0 + u * step + lane;
+            InTraits<T>::decode(i < end ? src(i) : make_uint4(0u, 0u, 0u, 0u), v[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t ibase = w0 + u * step;
+            if (ibase >= end) break;                 // warp-uniform
+            const uint32_t i = ibase + lane;
+            float amax = 0.0f;
+#pragma unroll
+            for (int k = 0; k < V; ++k) amax = fmaxf(amax, fabsf(v[u][k]));
+#pragma unroll
+            for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+
+            uint32_t sfq = 0;
+            float rcp = 0.0f;
+            if ((lane & (TPB - 1)) == 0) {
+                const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+                sfq = f32_to_e4m3(sf32);
+                rcp = rcp_tab[sfq];
+            }
+            const uint32_t leader = lane & ~static_cast<uint32_t>(TPB - 1);
+            rcp = __shfl_sync(0xffffffffu, rcp, leader);
+
+            uint32_t packed = 0;
+#pragma unroll
+            for (int k = 0; k < V; k += 2)
+                packed |= f32x2_to_e2m1x2(__fmul_rn(v[u][k], rcp), __fmul_rn(v[u][k + 1], rcp)) << (4 * k);
+            if (i < end) {
+                uint8_t* dst = q + static_cast<int64_t>(i) * (V / 2);
+                if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+                else *reinterpret_cast<uint32_t*>(dst) = packed;
+                if ((lane & (TPB - 1)) == 0) sf[i / TPB] = static_cast<uint8_t>(sfq);
+            }
+        }
+    }
+}
+
+// This block's contiguous share of nv vectors when they are split into blocks of `chunk`
+// (a multiple of 32): [v0, v1).
+__device__ __forceinline__ void block_range(uint32_t nv, uint32_t chunk, uint32_t bid, uint32_t& v0,
+                                            uint32_t& v1)
+{
+    const uint64_t a = static_cast<uint64_t>(bid) * chunk;
+    v0 = static_cast<uint32_t>(a < nv ? a : nv);
+    v1 = static_cast<uint32_t>(a + chunk < nv ? a + chunk : nv);
+}
+
+}  // namespace nvfp4
