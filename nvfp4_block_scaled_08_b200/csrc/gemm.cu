@@ -276,8 +276,8 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         const uint64_t rows = static_cast<uint64_t>(L.total_rows);
         ok &= get_map(&tp, L.B, 3, kb, L.N, E, kb, kb * L.N, 128, 128, true);
         ok &= get_map(&tsp, L.sfB, 3, ks, L.N, E, ks, ks * L.N, 16, 128, false);
-        ok &= get_map(&tq, L.A, 2, kb, rows, 1, kb, 0, 128, BN, true);
-        ok &= get_map(&tsq, L.sfA, 2, ks, rows, 1, ks, 0, 16, BN, false);
+        ok &= get_map(&tq, L.A, 2, kb, rows, 1, kb, 0, 128, Cfg::QBOX, true);
+        ok &= get_map(&tsq, L.sfA, 2, ks, rows, 1, ks, 0, 16, Cfg::QBOX, false);
         a.p_rows = a.N;
         a.q_rows = static_cast<int32_t>(L.total_rows);
         a.splits = 1;

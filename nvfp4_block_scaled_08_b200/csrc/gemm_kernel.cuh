@@ -94,6 +94,9 @@ struct GemmCfg {
     static constexpr int SF_TMA_P = BM * 16;       // bytes the scale TMA writes
     static constexpr int SF_TMA_Q = BN * 16;
     static constexpr uint32_t TX_BYTES = P_BYTES + Q_BYTES + SF_TMA_P + SF_TMA_Q;
+    // Grouped: the token tile is loaded in boxes of QBOX rows, only as many as the expert's
+    // rows in the tile need (a tile of a 256-wide plan often holds ~128 rows of one expert).
+    static constexpr int QBOX = BN < 64 ? BN : 64;
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
 
     // TMEM columns: two accumulators, then the scale factors: SFA (4 k-blocks x 4 columns),
@@ -650,7 +653,6 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                 if (!ok) break;
                 if (elect_one()) {
                     uint64_t* fb = &full_bar[stage];
-                    mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
                     const int32_t kx = (ti.k0 + ks) * Cfg::BK_BYTES;   // byte offset along K
                     const int32_t sx = (ti.k0 + ks) * 16;              // scale byte offset
                     uint8_t* pbuf = smem + Cfg::OFF_P + stage * Cfg::P_BYTES;
@@ -658,14 +660,27 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     uint8_t* sfpb = smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES;
                     uint8_t* sfqb = smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES;
                     if constexpr (Cfg::GROUPED) {
+                        // boxes of QBOX token rows covering the tile's MMA N (its rows rounded
+                        // up to 16); the 8-row swizzle atoms of the boxes line up as in one box
+                        const int n_mma = min(BN, (ti.q_valid + 15) & ~15);
+                        const int boxes = (n_mma + Cfg::QBOX - 1) / Cfg::QBOX;
+                        mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::SF_TMA_P +
+                                                  static_cast<uint32_t>(boxes * Cfg::QBOX * (Cfg::BK_BYTES + 16)));
                         tma_load_3d(pbuf, &tm_p, fb, kx, ti.p0, ti.expert, pol_p);
                         tma_load_3d(sfpb, &tm_sfp, fb, sx, ti.p0, ti.expert, pol_p);
+                        for (int b = 0; b < boxes; ++b) {
+                            tma_load_2d(qbuf + b * Cfg::QBOX * Cfg::BK_BYTES, &tm_q, fb, kx,
+                                        ti.q0 + b * Cfg::QBOX, pol_q);
+                            tma_load_2d(sfqb + b * Cfg::QBOX * 16, &tm_sfq, fb, sx, ti.q0 + b * Cfg::QBOX,
+                                        pol_q);
+                        }
                     } else {
+                        mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
                         tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
                         tma_load_2d(sfpb, &tm_sfp, fb, sx, ti.p0, pol_p);
+                        tma_load_2d(qbuf, &tm_q, fb, kx, ti.q0, pol_q);
+                        tma_load_2d(sfqb, &tm_sfq, fb, sx, ti.q0, pol_q);
                     }
-                    tma_load_2d(qbuf, &tm_q, fb, kx, ti.q0, pol_q);
-                    tma_load_2d(sfqb, &tm_sfq, fb, sx, ti.q0, pol_q);
                 }
                 __syncwarp();
                 ++issued;
