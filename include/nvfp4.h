@@ -184,6 +184,15 @@ nvfp4_status nvfp4_round_e4m3(const float* x, int64_t n, uint8_t* out, cudaStrea
 nvfp4_status nvfp4_round_e2m1(const float* x, int64_t n, uint8_t* out, cudaStream_t stream);
 
 /*
+ * Diagnostic of the failure path: launches one CTA that waits, with the same bounded-wait
+ * routine every kernel uses, on an mbarrier that nothing ever completes. After timeout_us
+ * microseconds (1 ... 1000000) the wait gives up and the kernel records code 0x1FF in the
+ * device error word and returns normally: the next nvfp4_last_device_error reports
+ * NVFP4_ERR_TIMEOUT with that code, and the CUDA context stays usable. No fault, no hang.
+ */
+nvfp4_status nvfp4_check_bounded_wait(uint32_t timeout_us, cudaStream_t stream);
+
+/*
  * Reads and clears the current device's error word. Synchronises `stream` first.
  * Returns NVFP4_OK if no kernel recorded an error since the last call, NVFP4_ERR_TIMEOUT
  * if one gave up on a bounded wait, NVFP4_ERR_CUDA if the read itself failed.

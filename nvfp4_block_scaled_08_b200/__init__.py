@@ -58,6 +58,7 @@ SIGNATURES = {
     "nvfp4_gemm_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "nvfp4_gemm_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "nvfp4_check_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _P]),
     "nvfp4_grouped_gemm_workspace_size": (_SZ, [_I32, _I64, _I64, _I64]),
     "nvfp4_grouped_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
                                           _SZ, _P]),
@@ -263,6 +264,11 @@ def round_e2m1(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) ->
     _check("nvfp4_round_e2m1", load().nvfp4_round_e2m1(_ptr(x), x.numel(), _ptr(out),
                                                        _stream(stream)))
     return out
+
+
+def check_bounded_wait(timeout_us: int, stream=None) -> None:
+    """Launch the bounded-wait check (a wait that must give up after timeout_us)."""
+    _check("nvfp4_check_bounded_wait", load().nvfp4_check_bounded_wait(timeout_us, _stream(stream)))
 
 
 def last_device_error(stream=None) -> tuple[int, int]:

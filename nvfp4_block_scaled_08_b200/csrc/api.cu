@@ -16,10 +16,32 @@
 
 #include "../../include/nvfp4.h"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace {
 
 __device__ unsigned g_nvfp4_error_word;
+
+// Code the bounded-wait check records in the device error word.
+constexpr unsigned kErrWaitCheck = 0x1FF;
+
+// One CTA waits, with the kernels' bounded-wait routine and the given limit, on an mbarrier
+// that nothing ever arrives at: the wait gives up, raises the CTA's abort flag, records
+// kErrWaitCheck in the device error word, and the kernel returns normally.
+__global__ void bounded_wait_check_kernel(unsigned* err_word, uint64_t timeout_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        nvfp4::mbar_init(&bar, 1);
+        abort_flag = 0;
+        nvfp4::fence_mbarrier_init();
+    }
+    __syncthreads();
+    const nvfp4::AbortState ab{&abort_flag, err_word};
+    if (threadIdx.x == 0) nvfp4::mbar_wait(&bar, 0, ab, kErrWaitCheck, timeout_ns);
+    __syncthreads();
+}
 
 struct DeviceInfo {
     bool init = false;
@@ -283,6 +305,16 @@ nvfp4_status nvfp4_round_e2m1(const float* x, int64_t n, uint8_t* out, cudaStrea
     nvfp4_status st = current_device(&d);
     if (st != NVFP4_OK) return st;
     return from_cuda(nvfp4::launch_round(x, n, out, true, stream, d.num_sms));
+}
+
+nvfp4_status nvfp4_check_bounded_wait(uint32_t timeout_us, cudaStream_t stream)
+{
+    if (timeout_us == 0 || timeout_us > 1000000u) return NVFP4_ERR_INVALID_ARG;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    bounded_wait_check_kernel<<<1, 32, 0, stream>>>(d.err_word, 1000ull * timeout_us);
+    return from_cuda(cudaGetLastError());
 }
 
 nvfp4_status nvfp4_last_device_error(cudaStream_t stream, uint32_t* where_out)

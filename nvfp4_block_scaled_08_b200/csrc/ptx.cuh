@@ -82,9 +82,10 @@ struct AbortState {
 
 // Wait until the phase with the given parity has completed. Returns false (and raises
 // the CTA's abort flag, recording `where` in the device error word) if the wait exceeds
-// kWaitTimeoutNs, or if another role of the CTA has already aborted.
+// timeout_ns (kWaitTimeoutNs in the kernels), or if another role of the CTA has already
+// aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const AbortState& ab,
-                                          uint32_t where)
+                                          uint32_t where, uint64_t timeout_ns = kWaitTimeoutNs)
 {
     if (mbar_test_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -92,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0) {
             if (*ab.flag) return false;
-            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            if (globaltimer_ns() - t0 > timeout_ns) {
                 *ab.flag = 1;
                 atomicCAS(ab.err_word, 0u, where);
                 return false;

@@ -111,6 +111,11 @@ def test_quantize_dynamic_host_validation(lib):
     assert f(0x1004, 0, 4, 64, 64, 0x2000, 0x3000, 0x4000, None, 0, None, None) == 3
 
 
+def test_bounded_wait_check_host_validation(lib):
+    assert lib.nvfp4_check_bounded_wait(0, None) == 1
+    assert lib.nvfp4_check_bounded_wait(1000001, None) == 1
+
+
 def test_round_and_alpha_host_validation(lib):
     assert lib.nvfp4_round_e4m3(None, 4, 0x1000, None) == 1
     assert lib.nvfp4_round_e2m1(0x1000, -1, 0x1000, None) == 1
