@@ -9,6 +9,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -86,8 +87,8 @@ __global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, 
 constexpr uint32_t kFlagRead = 0x52454144u;
 constexpr uint32_t kErrQuantFlags = 0x201;
 
-template <typename T, bool RESIDENT>
-__global__ void __launch_bounds__(512) quantize_dynamic_kernel(
+template <typename T, bool RESIDENT, int THREADS>
+__global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
     const T* __restrict__ x, const VecIndex ix, uint32_t nv, uint32_t chunk,
     float* __restrict__ gs_out, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
     const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out,
@@ -357,75 +358,46 @@ static int quantize_cluster_size()
 // Tensors up to this size are quantised by one cluster; larger ones by a cooperative grid
 // (measured on B200: one 16-CTA cluster wins at 393 KB, loses from 1.5 MB up).
 constexpr int64_t kClusterQuantizeMaxBytes = int64_t(512) << 10;
-// Largest shared-memory share per block for the resident cooperative quantiser (two blocks
-// per SM); larger tensors are swept twice instead.
-constexpr int64_t kResidentMaxBytes = int64_t(100) << 10;
+// Shared-memory share per cluster CTA the launcher allows (the input is kept on chip).
+constexpr int64_t kClusterStashMaxBytes = int64_t(200) << 10;
+// Tensors up to this size use one 1024-thread block per SM (half the grid-barrier
+// participants), larger ones two 512-thread blocks (measured on B200: 1024 wins at 1.5 and
+// 6.3 MB, loses at 25 MB).
+constexpr int64_t kCoopSmallBytes = int64_t(8) << 20;
 
 static inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
-template <typename T>
-static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64_t ldx, int64_t K,
-                                    float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
-                                    int32_t n_alpha, float* alpha_out, int64_t q_bytes,
-                                    unsigned* err_word, cudaStream_t stream, int num_sms)
+// Cooperative grid: BPS blocks of THREADS per SM at most (co-resident), at least two vectors
+// per thread, and room for the parked maxima and flags (8 bytes per block) in q. Each block
+// keeps its share in shared memory when it fits (about 200 KB per SM); otherwise the tensor
+// is swept twice.
+template <typename T, int THREADS, int BPS>
+static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float* gs_out, uint8_t* q,
+                               uint8_t* sf, const float* gs_other, int32_t n_alpha, float* alpha_out,
+                               int64_t q_bytes, unsigned* err_word, cudaStream_t stream, int num_sms)
 {
-    const int64_t bytes = rows * K * static_cast<int64_t>(sizeof(T));
-    const int64_t nv = rows * vpr;                       // < 2^31 (checked by the caller)
-    const VecIndex ix = make_vec_index(vpr, ldx, K);
-    const int ccs = bytes <= kClusterQuantizeMaxBytes ? quantize_cluster_size<T>() : 0;
-    if (ccs > 0) {
-        const int cs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ccs, (nv + 511) / 512)));
-        const int64_t chunk = round_up((nv + cs - 1) / cs, 32);
-        auto kern = quantize_dynamic_cluster_kernel<T>;
-        static std::once_flag once;
-        std::call_once(once, [&] {
-            // a cluster of >= 8 CTAs: at most 512 KB / 8 of vectors per CTA
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kClusterQuantizeMaxBytes / 8 + 512 * 16));
-        });
-        cudaLaunchConfig_t cfg;
-        std::memset(&cfg, 0, sizeof(cfg));
-        cfg.gridDim = dim3(1, static_cast<unsigned>(cs), 1);
-        cfg.blockDim = dim3(512, 1, 1);
-        cfg.dynamicSmemBytes = static_cast<size_t>(chunk) * 16;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[2];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 1;
-        attr[0].val.clusterDim.y = static_cast<unsigned>(cs);
-        attr[0].val.clusterDim.z = 1;
-        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[1].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 2;
-        return cudaLaunchKernelEx(&cfg, kern, x, ix, static_cast<uint32_t>(nv), static_cast<uint32_t>(chunk),
-                                  gs_out, q, sf, gs_other, n_alpha, alpha_out);
-    }
-
-    // Cooperative grid: two 512-thread blocks per SM at most (enough warps to hide the
-    // arithmetic, few grid-barrier participants), at least two vectors per thread, and room
-    // for the parked maxima and flags (8 bytes per block) in q.
-    int64_t blocks = std::min<int64_t>(2 * static_cast<int64_t>(num_sms), (nv + 1023) / 1024);
+    constexpr int64_t kResidentMaxBytes = (int64_t(200) << 10) / BPS;
+    int64_t blocks = std::min<int64_t>(BPS * static_cast<int64_t>(num_sms), (nv + 2 * THREADS - 1) / (2 * THREADS));
     blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, q_bytes / 8));
     int64_t chunk = round_up((nv + blocks - 1) / blocks, 32);
-    bool resident = chunk * 16 <= kResidentMaxBytes;
+    const bool resident = chunk * 16 <= kResidentMaxBytes;
     void (*kern)(const T*, const VecIndex, uint32_t, uint32_t, float*, uint8_t*, uint8_t*, const float*,
                  int32_t, float*, unsigned*) =
-        resident ? quantize_dynamic_kernel<T, true> : quantize_dynamic_kernel<T, false>;
+        resident ? quantize_dynamic_kernel<T, true, THREADS> : quantize_dynamic_kernel<T, false, THREADS>;
     size_t smem = 0;
     if (resident) {
         static std::once_flag once;
         std::call_once(once, [] {
-            cudaFuncSetAttribute(quantize_dynamic_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kResidentMaxBytes));
+            cudaFuncSetAttribute(quantize_dynamic_kernel<T, true, THREADS>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kResidentMaxBytes));
         });
         smem = static_cast<size_t>(chunk) * 16;
     }
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 512, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const int64_t fit = static_cast<int64_t>(std::min(per_sm, 2)) * num_sms;   // co-resident blocks
+    const int64_t fit = static_cast<int64_t>(std::min(per_sm, BPS)) * num_sms;   // co-resident blocks
     if (resident) {
         if (blocks > fit) {        // fewer blocks than planned: larger shares (same smem bound)
             blocks = fit;
@@ -439,7 +411,7 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
-    cfg.blockDim = dim3(512, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -460,6 +432,54 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
                                 err_word);
     }
     return le;
+}
+
+template <typename T>
+static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64_t ldx, int64_t K,
+                                    float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
+                                    int32_t n_alpha, float* alpha_out, int64_t q_bytes,
+                                    unsigned* err_word, cudaStream_t stream, int num_sms)
+{
+    const int64_t bytes = rows * K * static_cast<int64_t>(sizeof(T));
+    const int64_t nv = rows * vpr;                       // < 2^31 (checked by the caller)
+    const VecIndex ix = make_vec_index(vpr, ldx, K);
+    int64_t cluster_max = kClusterQuantizeMaxBytes;
+    if (const char* v = std::getenv("NVFP4_QCLUSTER_MAX_KB")) cluster_max = std::atoll(v) << 10;  // tuning only
+    const int ccs = bytes <= cluster_max ? quantize_cluster_size<T>() : 0;
+    if (ccs > 0) {
+        const int cs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ccs, (nv + 511) / 512)));
+        const int64_t chunk = round_up((nv + cs - 1) / cs, 32);
+        if (chunk * 16 > kClusterStashMaxBytes) return cudaErrorInvalidValue;
+        auto kern = quantize_dynamic_cluster_kernel<T>;
+        static std::once_flag once;
+        std::call_once(once, [&] {
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kClusterStashMaxBytes));
+        });
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(1, static_cast<unsigned>(cs), 1);
+        cfg.blockDim = dim3(512, 1, 1);
+        cfg.dynamicSmemBytes = static_cast<size_t>(chunk) * 16;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = static_cast<unsigned>(cs);
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        return cudaLaunchKernelEx(&cfg, kern, x, ix, static_cast<uint32_t>(nv), static_cast<uint32_t>(chunk),
+                                  gs_out, q, sf, gs_other, n_alpha, alpha_out);
+    }
+
+    if (bytes <= kCoopSmallBytes)
+        return launch_coop<T, 1024, 1>(x, ix, nv, gs_out, q, sf, gs_other, n_alpha, alpha_out, q_bytes, err_word,
+                                       stream, num_sms);
+    return launch_coop<T, 512, 2>(x, ix, nv, gs_out, q, sf, gs_other, n_alpha, alpha_out, q_bytes, err_word,
+                                  stream, num_sms);
 }
 
 cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
