@@ -8,16 +8,19 @@ once to NVFP4 outside the timed region. One step = for every M: per-tensor globa
 of A, alpha = 1/(gsA gsB), NVFP4 quantisation of A, block-scaled GEMM -> bf16.
 
 Timing: the step is captured as a CUDA graph of its eight kernels, nothing else, so each
-GEMM launches early behind its quantiser (programmatic dependent launch). A second graph
-with event-record nodes between the kernels is replayed afterwards, untimed, for the
-per-shape breakdown (`per_shape`; the event nodes cost each GEMM its early launch). Inputs are larger than L2: 8 independent input sets of the sweep (activations,
-weights, outputs; about 37 MiB each, 300 MiB in all, "layers" with different seeds) are
-replayed in rotation, so each step's data was last touched 7 steps (about 260 MiB) earlier
-and comes from HBM. --flush instead flushes L2 before every step (a 512 MB write, then a
-256 MB read), which also evicts kernel code and tensor maps. W warm-up replays, then exactly
-K timed replays bracketed by a barrier and a device synchronise; step time = sum of the
-per-replay CUDA-event durations, max over ranks. SM clocks and throttle reasons are polled
-through NVML during the timed bracket.
+kernel launches early behind the one before it (programmatic dependent launch). A second
+graph with event-record nodes between the kernels is replayed afterwards, untimed, for the
+per-shape breakdown (`per_shape`; the event nodes cost each kernel its early launch).
+Inputs are larger than L2: 8 independent input sets of the sweep (activations, weights,
+outputs; 41 MiB each, 327 MiB in all, "layers" with different seeds) are replayed in
+rotation, so each step's data was last touched 7 steps (about 286 MiB) earlier and comes
+from HBM. W warm-up replays, then exactly K steps back to back between one pair of CUDA
+events (whole rotations from one graph of all 8 sets, the remainder from single-set
+graphs), bracketed by a barrier and a device synchronise; step time = event time / K, max
+over ranks. --flush instead flushes L2 before every step (a 512 MB write, then a 256 MB
+read, which also evicts kernel code and tensor maps) and brackets each replay on its own,
+the flush outside. SM clocks and throttle reasons are polled through NVML during the timed
+bracket.
 
 e2e: the same metric through the public Python API called eagerly per step, with the
 activations copied from pinned host memory and the outputs copied back inside the timed
@@ -261,6 +264,11 @@ class AttnSweep:
         self.flops = sum(2 * it["M"] * N_ATTN * K_ATTN for it in self.items)
         self.launches_per_step = 2 * len(self.items)   # fused quantize, gemm
 
+    def step_one(self, it, stream=None):
+        """One M of the step: activations (fp32, resident) -> codes, scales, alpha -> bf16 out."""
+        self.run_one(it, stream)
+        self.gemm_one(it, stream)
+
     def run_one(self, it, stream=None):
         # global scale + alpha + NVFP4 quantisation of the activations: one launch
         self.nv.quantize_dynamic(it["a"], gs_other=self.gsB, gs=it["gs"], q=it["q"], sf=it["sf"],
@@ -379,6 +387,13 @@ def run_ours(args, world, rank, local):
     sets = [AttnSweep(dev, rank, i) for i in range(nsets)]
     graphs = [sw.capture() for sw in sets]
     sweep = sets[0]
+    # one graph of a whole rotation (every set once, in order: eight "layers"), so that
+    # consecutive steps are not separated by graph launches; single-set graphs cover the rest
+    rotation = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(rotation):
+        for sw in sets:
+            for it in sw.items:
+                sw.step_one(it)
     stream = torch.cuda.current_stream()
     if args.flush:
         flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -393,9 +408,15 @@ def run_ours(args, world, rank, local):
 
     clocks = ClockSampler(local)
     clocks.start()
-    for i in range(args.warmup):
-        before_step()
-        graphs[i % nsets].replay()
+    if args.flush:
+        for i in range(args.warmup):
+            before_step()
+            graphs[i % nsets].replay()
+    else:                                  # W steps, from the same graphs as the timed ones
+        for _ in range(args.warmup // nsets):
+            rotation.replay()
+        for i in range(args.warmup % nsets):
+            graphs[i].replay()
     torch.cuda.synchronize()
 
     start = torch.cuda.Event(enable_timing=True)
@@ -405,14 +426,26 @@ def run_ours(args, world, rank, local):
     total_ms = 0.0
     barrier(world)
     clocks.mark()
-    for i in range(args.steps):
-        k = i % nsets                      # each set was last touched nsets - 1 steps ago
-        before_step()
+    if args.flush:
+        # the flush before each step stays outside the timing: one bracket per step
+        for i in range(args.steps):
+            before_step()
+            start.record(stream)
+            graphs[i % nsets].replay()
+            end.record(stream)
+            end.synchronize()
+            total_ms += start.elapsed_time(end)
+    else:
+        # K steps back to back (each set was last touched nsets - 1 steps earlier), one
+        # bracket around all of them: whole rotations, then single sets
         start.record(stream)
-        graphs[k].replay()
+        for _ in range(args.steps // nsets):
+            rotation.replay()
+        for i in range(args.steps % nsets):
+            graphs[i].replay()
         end.record(stream)
         end.synchronize()
-        total_ms += start.elapsed_time(end)
+        total_ms = start.elapsed_time(end)
     barrier(world)
     clocks.mark()
     clocks.stop()
@@ -489,6 +522,9 @@ def run_ours(args, world, rank, local):
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
         "config": {"workload": "attn_proj_sweep N=768 K=6144 M={16,64,256,1024}",
                    "step": "per M: quantize_dynamic(A fp32: global scale, alpha, codes) + gemm; one CUDA graph",
+                   "timing": ("one event pair per step, L2 flush before each (outside the pair)" if args.flush
+                              else f"{args.steps} steps back to back between one event pair (graphs of "
+                                   f"{nsets}-set rotations, then single sets)"),
                    "l2": ("flushed before every timed step (512 MB write, then 256 MB read)" if args.flush else
                           f"inputs larger than L2: {nsets} independent input sets of {set_bytes / 2**20:.0f} MiB "
                           f"(activations, weights, outputs) in rotation, {nsets * set_bytes / 2**20:.0f} MiB "
@@ -510,52 +546,63 @@ def run_ours(args, world, rank, local):
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     for sw in sets:
         sw.graph = sw.graph_ev = None
+    del rotation
     del graphs
     return line
 
 
 # ------------------------------------------------------------------ the oracle (CPU)
 
-def oracle_sweep_sample(budget_s: float):
-    """Time the oracle on a bounded sample of the sweep: for every M, the first r rows of A
-    (global scale over the full A), repeated until about budget_s has passed. r is the full
-    M when one pass over the whole sweep fits in the budget, else a proportional share."""
-    import oracle
-    from nvfp4_block_scaled_08_b200 import workloads
-    cases = workloads.attn_proj_cases()
-    b = cases[0].b().numpy()
-    gb = oracle.global_scale(b)
-    qb, sb = oracle.quantize(b, gb)               # weights: once, outside the timing
-    a_all = [c.a().numpy() for c in cases]
-    threads = os.cpu_count() or 1
+class OracleSweep:
+    """The oracle on a bounded sample of the sweep: for every M, the first r rows of A (global
+    scale over the full A). Inputs, the weights' quantisation and a calibration pass are
+    prepared once, outside any timing."""
 
-    def one_pass(rows):
+    def __init__(self):
+        import oracle
+        from nvfp4_block_scaled_08_b200 import workloads
+        self.oracle = oracle
+        cases = workloads.attn_proj_cases()
+        self.Ms = [c.M for c in cases]
+        b = cases[0].b().numpy()
+        self.gb = oracle.global_scale(b)
+        self.qb, self.sb = oracle.quantize(b, self.gb)
+        self.a_all = [c.a().numpy() for c in cases]
+        self.threads = os.cpu_count() or 1
+        t0 = time.perf_counter()
+        self.one_pass([min(64, m) for m in self.Ms])
+        self.per_row = (time.perf_counter() - t0) / sum(min(64, m) for m in self.Ms)
+
+    def one_pass(self, rows):
+        o = self.oracle
         f = 0.0
-        for a, r in zip(a_all, rows):
-            ga = oracle.global_scale(a)
-            qa, sa = oracle.quantize(a[:r], ga)
-            oracle.gemm(qa, sa, qb, sb, oracle.alpha(ga, gb), threads=threads)
+        for a, r in zip(self.a_all, rows):
+            ga = o.global_scale(a)
+            qa, sa = o.quantize(a[:r], ga)
+            o.gemm(qa, sa, self.qb, self.sb, o.alpha(ga, self.gb), threads=self.threads)
             f += 2.0 * r * N_ATTN * K_ATTN
         return f
 
-    # calibration: one pass over 64 rows of every M
-    t0 = time.perf_counter()
-    one_pass([min(64, c.M) for c in cases])
-    per_row = (time.perf_counter() - t0) / sum(min(64, c.M) for c in cases)
-    total_rows = sum(c.M for c in cases)
-    frac = min(1.0, budget_s / max(per_row * total_rows, 1e-9))
-    rows = [max(1, int(round(c.M * frac))) for c in cases]
-    flops, passes = 0.0, 0
-    t0 = time.perf_counter()
-    while True:
-        flops += one_pass(rows)
-        passes += 1
-        if time.perf_counter() - t0 >= 0.8 * budget_s:
-            break
-    dt = time.perf_counter() - t0
-    sample = (f"attn_proj sweep, first {rows} rows of M={list(M_SWEEP)} (global scale over the "
-              f"full A), N=768, K=6144, {passes} pass(es); weights quantised outside timing")
-    return flops, dt, threads, sample
+    def run(self, budget_s: float):
+        """Passes over a row sample sized so that they take about budget_s (at least one
+        pass). Returns (flops, seconds, threads, description)."""
+        frac = min(1.0, budget_s / max(self.per_row * sum(self.Ms), 1e-9))
+        rows = [max(1, int(round(m * frac))) for m in self.Ms]
+        flops, passes = 0.0, 0
+        t0 = time.perf_counter()
+        while True:
+            flops += self.one_pass(rows)
+            passes += 1
+            if time.perf_counter() - t0 >= 0.8 * budget_s:
+                break
+        dt = time.perf_counter() - t0
+        sample = (f"attn_proj sweep, first {rows} rows of M={list(M_SWEEP)} (global scale over the "
+                  f"full A), N=768, K=6144, {passes} pass(es); weights quantised outside timing")
+        return flops, dt, self.threads, sample
+
+
+def oracle_sweep_sample(budget_s: float):
+    return OracleSweep().run(budget_s)
 
 
 def cpu_baseline(budget_s: float):
@@ -567,13 +614,15 @@ def cpu_baseline(budget_s: float):
 def run_reference(args, world, rank):
     if rank != 0:
         return None
-    per_step = max(0.2, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    # every step a bounded sample, so that warm-up + K steps take about two minutes
+    per_step = max(0.02, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    sweep = OracleSweep()
     for _ in range(args.warmup):
-        oracle_sweep_sample(per_step)
+        sweep.run(per_step)
     tot_f = tot_t = 0.0
     info = None
     for _ in range(args.steps):
-        f, t, th, sample = oracle_sweep_sample(per_step)
+        f, t, th, sample = sweep.run(per_step)
         tot_f += f
         tot_t += t
         info = (th, sample)
@@ -597,7 +646,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
