@@ -59,6 +59,22 @@ typedef enum {
     NVFP4_IN_BF16 = 1
 } nvfp4_in_dtype;
 
+/*
+ * Layout of a scale matrix (one e4m3 byte per 16 K-elements of each row).
+ *   NVFP4_SF_LINEAR: row-major [rows][K/16] bytes.
+ *   NVFP4_SF_TILED:  512-byte blocks of 128 rows x 4 scales (64 K-elements): the scale of row r,
+ *                    column c (c = k / 16) is at byte
+ *                        ((r / 128) * (K / 64) + c / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4,
+ *                    rows padded to a multiple of 128 (the padding is never read into an output).
+ *                    Each block's 16-byte row i holds the scales of rows i, i + 32, i + 64, i + 96:
+ *                    the operand layout of the tensor cores' scale copies, so the GEMM fetches a
+ *                    stage's scales with one bulk copy per 128 rows. Requires K % 64 == 0.
+ */
+typedef enum {
+    NVFP4_SF_LINEAR = 0,
+    NVFP4_SF_TILED = 1
+} nvfp4_sf_layout;
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* nvfp4_status_string(nvfp4_status s);
 
@@ -104,6 +120,28 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, nvfp4_in_dtype dtype, int64_t
                                     cudaStream_t stream);
 
 /*
+ * nvfp4_quantize_dynamic with the scales written in the given layout (the same values; for
+ * NVFP4_SF_TILED, sf holds nvfp4_sf_bytes(rows, K, NVFP4_SF_TILED) bytes and K % 64 == 0).
+ * nvfp4_quantize_dynamic is this call with NVFP4_SF_LINEAR.
+ */
+nvfp4_status nvfp4_quantize_dynamic_ex(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
+                                       int64_t ld_x, float* gs_out, uint8_t* q, uint8_t* sf,
+                                       const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                       nvfp4_sf_layout sf_layout, cudaStream_t stream);
+
+/* Bytes of a scale matrix of `rows` rows and K elements per row in the given layout (0 for an
+ * invalid layout or K). */
+size_t nvfp4_sf_bytes(int64_t rows, int64_t K, nvfp4_sf_layout sf_layout);
+
+/*
+ * Re-lays row-major scales sf[rows][K/16] (device) out as NVFP4_SF_TILED into sf_tiled (device,
+ * nvfp4_sf_bytes(rows, K, NVFP4_SF_TILED) bytes; padding rows become 0). K % 64 == 0. For
+ * weights, once, before the GEMMs that use them.
+ */
+nvfp4_status nvfp4_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* sf_tiled,
+                           cudaStream_t stream);
+
+/*
  * GEMM scale from the two global scales: alpha[i] = 1 / (gs_a[0] * gs_b[i]) in fp32,
  * for i < n (n = 1 for a single GEMM, n = experts for the grouped GEMM). All device.
  */
@@ -130,6 +168,19 @@ nvfp4_status nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
                         const uint8_t* sfB, const float* alpha, void* out,
                         int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
                         cudaStream_t stream);
+
+/*
+ * nvfp4_gemm with both scale matrices in the given layout: sfA of nvfp4_sf_bytes(M, K, layout)
+ * and sfB of nvfp4_sf_bytes(N, K, layout) bytes (device). The results are bit for bit those of
+ * nvfp4_gemm on the same scales in the linear layout. NVFP4_SF_TILED skips the
+ * kernel's scale re-layout step (one bulk copy per stage and 128 rows) and is the faster
+ * layout. With tuning overrides that place token tiles off 128-row tile boundaries it returns
+ * NVFP4_ERR_UNSUPPORTED_SHAPE. nvfp4_gemm is this call with NVFP4_SF_LINEAR.
+ */
+nvfp4_status nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                           const uint8_t* sfB, const float* alpha, void* out,
+                           int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
+                           nvfp4_sf_layout sf_layout, cudaStream_t stream);
 
 /*
  * Grouped (mixture-of-experts) NVFP4 GEMM ("When a Benchmark Crashes", section "Why This

@@ -59,6 +59,11 @@ SIGNATURES = {
     "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "nvfp4_gemm_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_check_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _P]),
+    "nvfp4_quantize_dynamic_ex": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _P, _P,
+                                                 ctypes.c_int32, _P, ctypes.c_int, _P]),
+    "nvfp4_sf_bytes": (_SZ, [_I64, _I64, ctypes.c_int]),
+    "nvfp4_sf_tile": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "nvfp4_gemm_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int, _P]),
     "nvfp4_grouped_gemm_workspace_size": (_SZ, [_I32, _I64, _I64, _I64]),
     "nvfp4_grouped_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
                                           _SZ, _P]),
@@ -152,11 +157,28 @@ def quantize(x: torch.Tensor, gs: torch.Tensor, q: torch.Tensor | None = None,
     return q, sf
 
 
+SF_LINEAR, SF_TILED = 0, 1
+
+
+def sf_bytes(rows: int, K: int, tiled: bool = False) -> int:
+    return int(load().nvfp4_sf_bytes(rows, K, SF_TILED if tiled else SF_LINEAR))
+
+
+def sf_tile(sf: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Row-major scales [rows, K/16] -> the tiled layout (flat uint8 tensor)."""
+    rows, K = sf.shape[0], sf.shape[1] * 16
+    if out is None:
+        out = torch.empty(sf_bytes(rows, K, True), dtype=torch.uint8, device=sf.device)
+    _check("nvfp4_sf_tile", load().nvfp4_sf_tile(_ptr(sf), rows, K, _ptr(out), _stream(stream)))
+    return out
+
+
 def quantize_dynamic(x: torch.Tensor, gs_other: torch.Tensor | None = None,
                      gs: torch.Tensor | None = None, q: torch.Tensor | None = None,
                      sf: torch.Tensor | None = None, alpha_out: torch.Tensor | None = None,
-                     stream=None):
-    """Global scale + quantisation (+ alpha against gs_other) in one launch.
+                     stream=None, tiled: bool = False):
+    """Global scale + quantisation (+ alpha against gs_other) in one launch; tiled: scales in
+    the tiled layout (a flat uint8 tensor of sf_bytes(rows, K, True) bytes).
 
     Returns (q, sf, gs, alpha) where alpha is None when gs_other is None."""
     _dev(x, "x")
@@ -166,15 +188,17 @@ def quantize_dynamic(x: torch.Tensor, gs_other: torch.Tensor | None = None,
     if q is None:
         q = torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device)
     if sf is None:
-        sf = torch.empty(rows, K // 16, dtype=torch.uint8, device=x.device)
+        sf = (torch.empty(sf_bytes(rows, K, True), dtype=torch.uint8, device=x.device) if tiled
+              else torch.empty(rows, K // 16, dtype=torch.uint8, device=x.device))
     if gs is None:
         gs = torch.empty(1, dtype=torch.float32, device=x.device)
     n = 0 if gs_other is None else gs_other.numel()
     if n and alpha_out is None:
         alpha_out = torch.empty(n, dtype=torch.float32, device=x.device)
-    _check("nvfp4_quantize_dynamic", load().nvfp4_quantize_dynamic(
+    _check("nvfp4_quantize_dynamic_ex", load().nvfp4_quantize_dynamic_ex(
         _ptr(x), _dtype_code(x), rows, K, x.stride(0), _ptr(gs), _ptr(q), _ptr(sf),
-        _ptr(gs_other), n, _ptr(alpha_out) if n else None, _stream(stream)))
+        _ptr(gs_other), n, _ptr(alpha_out) if n else None, SF_TILED if tiled else SF_LINEAR,
+        _stream(stream)))
     return q, sf, gs, (alpha_out if n else None)
 
 
@@ -203,20 +227,21 @@ def make_workspace(M: int, N: int, K: int, device="cuda") -> torch.Tensor | None
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None) -> torch.Tensor:
+def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None, tiled=False) -> torch.Tensor:
     """out[M, N] = bf16(alpha * sum_k deq(A)[m,k] deq(B)[n,k]).
 
     Aq [M, K/2] uint8, sfA [M, K/16] uint8, Bq [N, K/2], sfB [N, K/16], alpha_t fp32 [1];
     out bf16 [M, N] (allocated if None); workspace: zero-filled uint8 tensor of
-    gemm_workspace_size(M, N, K) bytes or None (no split-K)."""
+    gemm_workspace_size(M, N, K) bytes or None (no split-K). tiled: sfA and sfB in the tiled
+    layout (flat uint8 tensors from sf_tile or quantize_dynamic(tiled=True))."""
     M, K = Aq.shape[0], Aq.shape[1] * 2
     N = Bq.shape[0]
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=Aq.device)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
-    _check("nvfp4_gemm", load().nvfp4_gemm(
+    _check("nvfp4_gemm_ex", load().nvfp4_gemm_ex(
         _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alpha_t), _ptr(out), M, N, K,
-        ws_ptr, ws_bytes, _stream(stream)))
+        ws_ptr, ws_bytes, SF_TILED if tiled else SF_LINEAR, _stream(stream)))
     return out
 
 

@@ -182,18 +182,20 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t rows, i
                                             stream, d.num_sms));
 }
 
-nvfp4_status nvfp4_quantize_dynamic(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
-                                    int64_t ld_x, float* gs_out, uint8_t* q, uint8_t* sf,
-                                    const float* gs_other, int32_t n_alpha, float* alpha_out,
-                                    cudaStream_t stream)
+nvfp4_status nvfp4_quantize_dynamic_ex(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
+                                       int64_t ld_x, float* gs_out, uint8_t* q, uint8_t* sf,
+                                       const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                       nvfp4_sf_layout sf_layout, cudaStream_t stream)
 {
     if (rows < 0 || K < 0 || n_alpha < 0) return NVFP4_ERR_INVALID_ARG;
     if (dtype != NVFP4_IN_F32 && dtype != NVFP4_IN_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (sf_layout != NVFP4_SF_LINEAR && sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_INVALID_ARG;
     if (!gs_out) return NVFP4_ERR_INVALID_ARG;
     if (n_alpha > 0 && (!gs_other || !alpha_out)) return NVFP4_ERR_INVALID_ARG;
     if (rows == 0 || K == 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;   // no tensor to take a scale of
     if (!x || !q || !sf) return NVFP4_ERR_INVALID_ARG;
     if (K % 16 != 0 || K > kMaxDim || rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (sf_layout == NVFP4_SF_TILED && K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (ld_x < K) return NVFP4_ERR_INVALID_ARG;
     const int64_t esz = dtype == NVFP4_IN_BF16 ? 2 : 4;
     if (rows * (K * esz / 16) >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -203,9 +205,39 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, nvfp4_in_dtype dtype, int64_t
     DeviceInfo d;
     nvfp4_status st = current_device(&d);
     if (st != NVFP4_OK) return st;
-    return from_cuda(nvfp4::launch_quantize_dynamic(x, dtype == NVFP4_IN_BF16, rows, K, ld_x, gs_out,
-                                                    q, sf, gs_other, n_alpha, alpha_out, d.err_word,
-                                                    stream, d.num_sms));
+    return from_cuda(nvfp4::launch_quantize_dynamic(x, dtype == NVFP4_IN_BF16, rows, K, ld_x, gs_out, q, sf,
+                                                    sf_layout == NVFP4_SF_TILED, gs_other, n_alpha,
+                                                    alpha_out, d.err_word, stream, d.num_sms));
+}
+
+nvfp4_status nvfp4_quantize_dynamic(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
+                                    int64_t ld_x, float* gs_out, uint8_t* q, uint8_t* sf,
+                                    const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                    cudaStream_t stream)
+{
+    return nvfp4_quantize_dynamic_ex(x, dtype, rows, K, ld_x, gs_out, q, sf, gs_other, n_alpha, alpha_out,
+                                     NVFP4_SF_LINEAR, stream);
+}
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t K, nvfp4_sf_layout sf_layout)
+{
+    if (rows < 0 || K <= 0 || K % 16 != 0) return 0;
+    if (sf_layout == NVFP4_SF_LINEAR) return static_cast<size_t>(rows) * static_cast<size_t>(K / 16);
+    if (sf_layout == NVFP4_SF_TILED && K % 64 == 0)
+        return static_cast<size_t>((rows + 127) / 128 * 128) * static_cast<size_t>(K / 16);
+    return 0;
+}
+
+nvfp4_status nvfp4_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* sf_tiled, cudaStream_t stream)
+{
+    if (rows < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0 || K == 0) return NVFP4_OK;
+    if (!sf || !sf_tiled) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0 || K > kMaxDim || rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_sf_tile(sf, rows, K, sf_tiled, stream, d.num_sms));
 }
 
 nvfp4_status nvfp4_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
@@ -229,11 +261,12 @@ size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K)
     return nvfp4::plan_gemm(M, N, K, true, d.num_sms).ws_bytes;
 }
 
-nvfp4_status nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
-                        const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
-                        size_t ws_bytes, cudaStream_t stream)
+nvfp4_status nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                           const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
+                           size_t ws_bytes, nvfp4_sf_layout sf_layout, cudaStream_t stream)
 {
     if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (sf_layout != NVFP4_SF_LINEAR && sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return NVFP4_OK;
     if (M > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     nvfp4_status st = check_gemm_common(A, sfA, B, sfB, alpha, out, N, K);
@@ -244,11 +277,22 @@ nvfp4_status nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, 
     if (st != NVFP4_OK) return st;
     nvfp4::GemmPlan plan = nvfp4::plan_gemm(M, N, K, ws != nullptr, d.num_sms);
     if (plan.ws_bytes > 0 && ws_bytes < plan.ws_bytes) return NVFP4_ERR_WORKSPACE;
-    nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0, ws, d.err_word};
+    const bool tiled = sf_layout == NVFP4_SF_TILED;
+    // tiled scales: Q tiles start on 128-row tile boundaries (tuning overrides can break it)
+    if (tiled && (plan.swap ? plan.q_tiles != 1 : (plan.bn % 128 != 0)))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0, ws, d.err_word, tiled};
     bool enc_failed = false;
     cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
     if (enc_failed) return NVFP4_ERR_CUDA;
     return from_cuda(e);
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                        const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
+                        size_t ws_bytes, cudaStream_t stream)
+{
+    return nvfp4_gemm_ex(A, sfA, B, sfB, alpha, out, M, N, K, ws, ws_bytes, NVFP4_SF_LINEAR, stream);
 }
 
 size_t nvfp4_grouped_gemm_workspace_size(int32_t E, int64_t total_rows, int64_t N, int64_t K)

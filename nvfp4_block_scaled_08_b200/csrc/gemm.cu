@@ -236,11 +236,11 @@ static int max_active_clusters(int cs)
     return cache[dev][cs] > 0 ? cache[dev][cs] : 0;
 }
 
-template <int BN, bool SWAP, bool GROUPED>
+template <int BN, bool SWAP, bool GROUPED, bool SFT = false>
 static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
                        bool* encode_failed)
 {
-    using Cfg = GemmCfg<BN, SWAP, GROUPED>;
+    using Cfg = GemmCfg<BN, SWAP, GROUPED, SFT>;
     auto kern = nvfp4_gemm_kernel<Cfg>;
     // Opt in to the large dynamic shared memory once per device (not a stream operation,
     // so a later launch may be captured into a CUDA graph).
@@ -292,9 +292,17 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         const uint64_t p_rows = static_cast<uint64_t>(SWAP ? L.N : L.M);
         const uint64_t q_rows = static_cast<uint64_t>(SWAP ? L.M : L.N);
         ok &= get_map(&tp, P, 2, kb, p_rows, 1, kb, 0, 128, 128, true);
-        ok &= get_map(&tsp, sP, 2, ks, p_rows, 1, ks, 0, 16, 128, false);
         ok &= get_map(&tq, Q, 2, kb, q_rows, 1, kb, 0, 128, BN, true);
-        ok &= get_map(&tsq, sQ, 2, ks, q_rows, 1, ks, 0, 16, BN, false);
+        if constexpr (SFT) {
+            tsp = tp;                       // unused: the scales come by bulk copy
+            tsq = tq;
+            a.sf_p = sP;
+            a.sf_q = sQ;
+            a.sf_kb4 = static_cast<int32_t>(L.K / 64);
+        } else {
+            ok &= get_map(&tsp, sP, 2, ks, p_rows, 1, ks, 0, 16, 128, false);
+            ok &= get_map(&tsq, sQ, 2, ks, q_rows, 1, ks, 0, 16, BN, false);
+        }
         a.p_rows = static_cast<int32_t>(p_rows);
         a.q_rows = static_cast<int32_t>(q_rows);
         a.num_q_tiles = plan.q_tiles;
@@ -336,6 +344,23 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
 {
     *encode_failed = false;
     if (plan.grid <= 0) return cudaSuccess;
+    if (L.sf_tiled) {
+        if (plan.grouped) return cudaErrorInvalidValue;
+        if (plan.swap) {
+            if (plan.q_tiles != 1) return cudaErrorInvalidValue;   // Q tile at row 0
+            switch (plan.bn) {
+                case 16: return run<16, true, false, true>(plan, L, stream, encode_failed);
+                case 32: return run<32, true, false, true>(plan, L, stream, encode_failed);
+                case 64: return run<64, true, false, true>(plan, L, stream, encode_failed);
+                default: return cudaErrorInvalidValue;
+            }
+        }
+        switch (plan.bn) {
+            case 128: return run<128, false, false, true>(plan, L, stream, encode_failed);
+            case 256: return run<256, false, false, true>(plan, L, stream, encode_failed);
+            default: return cudaErrorInvalidValue;      // 192 / 224 tiles: linear scales only
+        }
+    }
     if (plan.grouped) {
         switch (plan.bn) {
             case 32: return run<32, true, true>(plan, L, stream, encode_failed);

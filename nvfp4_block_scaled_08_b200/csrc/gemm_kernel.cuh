@@ -71,16 +71,26 @@ struct GemmArgs {
     float* ws_partial;        // split-K fp32 partial tiles
     uint32_t* ws_counters;    // split-K per-tile arrival counters
     unsigned* err_word;
+    const uint8_t* sf_p;      // SFT: tiled scales of the P / Q operands
+    const uint8_t* sf_q;
+    int32_t sf_kb4;           // SFT: 512-byte scale blocks per 128-row tile (K / 64)
     const int32_t* expert_offsets;  // grouped: [E + 1]
     int32_t num_experts;
     int32_t total_rows;       // grouped: rows of A / out
 };
 
-template <int BN_, bool SWAP_, bool GROUPED_>
+template <int BN_, bool SWAP_, bool GROUPED_, bool SFT_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;
     static constexpr bool SWAP = SWAP_;
     static constexpr bool GROUPED = GROUPED_;
+    // SFT: both operands' scales in the tiled layout (include/nvfp4.h, NVFP4_SF_TILED): a
+    // stage's scales of 128 rows are one contiguous 2 KB run already in the tcgen05.cp source
+    // layout, fetched by a bulk copy (no re-layout step). Q tiles then start on a 128-row
+    // tile boundary: BN >= 128 a multiple of 128, or a single Q tile (few-token swap).
+    static constexpr bool SFT = SFT_;
+    static_assert(!SFT || !GROUPED, "tiled scales serve the dense GEMM");
+    static_assert(!SFT || BN % 128 == 0 || (SWAP && BN <= 64), "Q tiles on 128-row tile boundaries");
     static_assert(!GROUPED || SWAP, "grouped GEMM runs with weights as the MMA M operand");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
 
@@ -566,8 +576,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tm_p);
         prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_sfp);
-        prefetch_tensormap(&tm_sfq);
+        if constexpr (!Cfg::SFT) {
+            prefetch_tensormap(&tm_sfp);
+            prefetch_tensormap(&tm_sfq);
+        }
     }
     if (warp == 1) {
         tmem_alloc(s_tmem_base, Cfg::TMEM_COLS);
@@ -674,6 +686,21 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                             tma_load_2d(sfqb + b * Cfg::QBOX * 16, &tm_sfq, fb, sx, ti.q0 + b * Cfg::QBOX,
                                         pol_q);
                         }
+                    } else if constexpr (Cfg::SFT) {
+                        // the stage's 4 scale blocks of each 128-row tile: one 2 KB run; only
+                        // the Q row tiles that exist (the last Q tile may end past the rows)
+                        const int ng = min(QG, (args.q_rows - ti.q0 + 127) >> 7);
+                        mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::Q_BYTES + Cfg::SFP_BYTES +
+                                                  2048u * static_cast<uint32_t>(ng));
+                        tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
+                        tma_load_2d(qbuf, &tm_q, fb, kx, ti.q0, pol_q);
+                        const int64_t kb = 4 * static_cast<int64_t>(ti.k0 + ks);
+                        bulk_load(sfpb, args.sf_p + ((ti.p0 >> 7) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
+                                  2048, fb, pol_p);
+                        for (int g = 0; g < ng; ++g)
+                            bulk_load(sfqb + 2048 * g,
+                                      args.sf_q + (((ti.q0 >> 7) + g) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
+                                      2048, fb, pol_q);
                     } else {
                         mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
                         tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
@@ -722,7 +749,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             const uint32_t d_tmem = tmem_base + acc * BN;
             for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
                 bool got = mbar_wait(&full_bar[stage], phase, ab, kErrMmaFull);
-                got = got && mbar_wait(&sfready_bar[stage], phase, ab, kErrMmaSf);
+                if constexpr (!Cfg::SFT) got = got && mbar_wait(&sfready_bar[stage], phase, ab, kErrMmaSf);
                 ok = __all_sync(0xffffffffu, got);
                 if (!ok) break;
                 if (elect_one()) {
@@ -759,7 +786,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         // Arrives once every tcgen05 operation issued above has completed.
         if (elect_one()) mma_commit(mma_done_bar);
         __syncwarp();
-    } else if (warp == 2 || warp == 3) {
+    } else if (!Cfg::SFT && (warp == 2 || warp == 3)) {
         // -------------------------------------------------------------- scale re-layout
         // The TMA wrote row r's 16 scale bytes (k-blocks 0..15 of the stage) at r * 16.
         // The MMA for k-step j (k-blocks 4j..4j+3) needs, per 128-row group, a 512-byte

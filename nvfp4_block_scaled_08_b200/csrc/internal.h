@@ -17,9 +17,11 @@ cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, i
                             const float* gs, uint8_t* q, uint8_t* sf, cudaStream_t stream,
                             int num_sms);
 cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
-                                    float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
-                                    int32_t n_alpha, float* alpha_out, unsigned* err_word,
-                                    cudaStream_t stream, int num_sms);
+                                    float* gs_out, uint8_t* q, uint8_t* sf, bool sf_tiled,
+                                    const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                    unsigned* err_word, cudaStream_t stream, int num_sms);
+cudaError_t launch_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* out, cudaStream_t stream,
+                           int num_sms);
 cudaError_t launch_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
                          cudaStream_t stream);
 cudaError_t launch_round(const float* x, int64_t n, uint8_t* out, bool e2m1, cudaStream_t stream,
@@ -54,6 +56,7 @@ struct GemmLaunch {
     const int32_t* offsets; int32_t E; int64_t total_rows;
     void* ws;
     unsigned* err_word;
+    bool sf_tiled = false;      // sfA and sfB in the tiled layout (dense GEMM only)
 };
 
 // api.cu: nvfp4_status of the current device's checks; fills the SM count and the device

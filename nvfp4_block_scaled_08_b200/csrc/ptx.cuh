@@ -313,6 +313,17 @@ __device__ __forceinline__ void cluster_wait()
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Bulk (1-D) copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
+// to this CTA's shared memory, completion counted (bytes) on the local mbarrier `bar`.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
 // Asynchronous 16-byte store into another cluster CTA's shared memory; its completion is
 // counted (bytes) on that CTA's mbarrier `remote_bar`. Both addresses come from mapa.
 __device__ __forceinline__ void st_async_f4(uint32_t remote_addr, float a, float b, float c, float d,

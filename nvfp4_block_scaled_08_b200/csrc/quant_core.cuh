@@ -111,6 +111,40 @@ __device__ __forceinline__ int64_t vec_offset(const VecIndex& ix, uint32_t i)
     return static_cast<int64_t>(r) * ix.ld + static_cast<int64_t>(c) * V;
 }
 
+// Where the block scales go: row-major [rows][K/16] bytes, or the tiled layout of
+// include/nvfp4.h (NVFP4_SF_TILED): for row r and scale column c (16-element block),
+//     ((r / 128) * (K / 64) + c / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4,
+// i.e. 512-byte blocks of 128 rows x 4 scales, each holding, in its 16-byte row i, the scales
+// of rows i, i + 32, i + 64, i + 96: the source layout of tcgen05.cp ... 32x128b.warpx4.
+struct SfOut {
+    uint8_t* sf;
+    int32_t tiled;
+    uint32_t kb4;            // K / 64: 512-byte blocks per 128-row tile
+    uint32_t vpr, mul, shift;  // vector -> row, as in VecIndex
+
+    template <int TPB>
+    __device__ __forceinline__ uint8_t* at(uint32_t i) const   // scale of vector i's block
+    {
+        if (!tiled) return sf + i / TPB;
+        const uint32_t r = static_cast<uint32_t>((static_cast<uint64_t>(__umulhi(i, mul)) + i) >> shift);
+        const uint32_t c = (i - r * vpr) / TPB;
+        return sf + (static_cast<uint64_t>(r >> 7) * kb4 + (c >> 2)) * 512 + (r & 31u) * 16 + ((r >> 5) & 3u) * 4 +
+               (c & 3u);
+    }
+};
+
+inline SfOut make_sf_out(uint8_t* sf, bool tiled, const VecIndex& ix, int64_t K)
+{
+    SfOut o;
+    o.sf = sf;
+    o.tiled = tiled ? 1 : 0;
+    o.kb4 = static_cast<uint32_t>(K / 64);
+    o.vpr = ix.vpr;
+    o.mul = ix.mul;
+    o.shift = ix.shift;
+    return o;
+}
+
 // Loads in flight per thread in the sweeps below.
 constexpr int kUnroll = 4;
 
@@ -199,7 +233,7 @@ __device__ __forceinline__ void build_rcp_table(float gs, float* rcp_tab)
 template <typename T, typename Src>
 __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint32_t end, uint32_t step,
                                                float gs, const float* rcp_tab, uint8_t* __restrict__ q,
-                                               uint8_t* __restrict__ sf)
+                                               const SfOut& sfo)
 {
     constexpr int V = InTraits<T>::kPerThread;   // elements per thread
     constexpr int TPB = 16 / V;                  // threads per 16-element block
@@ -241,7 +275,7 @@ __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint
                 uint8_t* dst = q + static_cast<int64_t>(i) * (V / 2);
                 if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
                 else *reinterpret_cast<uint32_t*>(dst) = packed;
-                if ((lane & (TPB - 1)) == 0) sf[i / TPB] = static_cast<uint8_t>(sfq);
+                if ((lane & (TPB - 1)) == 0) *sfo.at<TPB>(i) = static_cast<uint8_t>(sfq);
             }
         }
     }

@@ -65,13 +65,13 @@ __global__ void alpha_kernel(const float* __restrict__ gs_a, const float* __rest
 template <typename T>
 __global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, const VecIndex ix, uint32_t nv,
                                                        const float* __restrict__ gs_ptr,
-                                                       uint8_t* __restrict__ q, uint8_t* __restrict__ sf)
+                                                       uint8_t* __restrict__ q, const SfOut sfo)
 {
     __shared__ float rcp_tab[256];
     const float gs = __ldg(gs_ptr);
     build_rcp_table(gs, rcp_tab);
     quantize_sweep<T>(GlobalVecs<T>{x, ix}, blockIdx.x * blockDim.x + (threadIdx.x & ~31u), nv,
-                      gridDim.x * blockDim.x, gs, rcp_tab, q, sf);
+                      gridDim.x * blockDim.x, gs, rcp_tab, q, sfo);
 }
 
 // One cooperative launch: amax of the whole tensor -> grid barrier -> global scale (and the
@@ -90,7 +90,7 @@ constexpr uint32_t kErrQuantFlags = 0x201;
 template <typename T, bool RESIDENT, int THREADS>
 __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
     const T* __restrict__ x, const VecIndex ix, uint32_t nv, uint32_t chunk,
-    float* __restrict__ gs_out, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+    float* __restrict__ gs_out, uint8_t* __restrict__ q, const SfOut sfo,
     const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out,
     unsigned* __restrict__ err_word)
 {
@@ -155,10 +155,10 @@ __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
     __shared__ float rcp_tab[256];
     build_rcp_table(gs, rcp_tab);
     if constexpr (RESIDENT) {
-        quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sf);
+        quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sfo);
     } else {
         quantize_sweep<T>(GlobalVecs<T>{x, ix}, bid * blockDim.x + (threadIdx.x & ~31u), nv,
-                          nblocks * blockDim.x, gs, rcp_tab, q, sf);
+                          nblocks * blockDim.x, gs, rcp_tab, q, sfo);
     }
 }
 
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
 template <typename T>
 __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
     const T* __restrict__ x, const VecIndex ix, uint32_t nv, uint32_t chunk,
-    float* __restrict__ gs_out, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+    float* __restrict__ gs_out, uint8_t* __restrict__ q, const SfOut sfo,
     const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out)
 {
     extern __shared__ uint4 stash[];
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
     cudaTriggerProgrammaticLaunchCompletion();
     __shared__ float rcp_tab[256];
     build_rcp_table(gs, rcp_tab);
-    quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sf);
+    quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sfo);
     cluster_wait();                                   // no CTA leaves while a peer may read it
 }
 
@@ -308,7 +308,7 @@ cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, i
         const int grid = grid_1d(nv, static_cast<int64_t>(num_sms) * 4);
         const void* xp = static_cast<const uint8_t*>(x) + static_cast<size_t>(r0 * ldx) * esz;
         uint8_t* qp = q + r0 * (K / 2);
-        uint8_t* sp = sf + r0 * (K / 16);
+        const SfOut sp = make_sf_out(sf + r0 * (K / 16), false, ix, K);
         if (bf16)
             quantize_kernel<__nv_bfloat16><<<grid, 512, 0, stream>>>(
                 static_cast<const __nv_bfloat16*>(xp), ix, static_cast<uint32_t>(nv), gs, qp, sp);
@@ -373,7 +373,7 @@ static inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * 
 // is swept twice.
 template <typename T, int THREADS, int BPS>
 static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float* gs_out, uint8_t* q,
-                               uint8_t* sf, const float* gs_other, int32_t n_alpha, float* alpha_out,
+                               const SfOut& sf, const float* gs_other, int32_t n_alpha, float* alpha_out,
                                int64_t q_bytes, unsigned* err_word, cudaStream_t stream, int num_sms)
 {
     constexpr int64_t kResidentMaxBytes = (int64_t(200) << 10) / BPS;
@@ -381,7 +381,7 @@ static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float
     blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, q_bytes / 8));
     int64_t chunk = round_up((nv + blocks - 1) / blocks, 32);
     const bool resident = chunk * 16 <= kResidentMaxBytes;
-    void (*kern)(const T*, const VecIndex, uint32_t, uint32_t, float*, uint8_t*, uint8_t*, const float*,
+    void (*kern)(const T*, const VecIndex, uint32_t, uint32_t, float*, uint8_t*, const SfOut, const float*,
                  int32_t, float*, unsigned*) =
         resident ? quantize_dynamic_kernel<T, true, THREADS> : quantize_dynamic_kernel<T, false, THREADS>;
     size_t smem = 0;
@@ -436,13 +436,14 @@ static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float
 
 template <typename T>
 static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64_t ldx, int64_t K,
-                                    float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
-                                    int32_t n_alpha, float* alpha_out, int64_t q_bytes,
-                                    unsigned* err_word, cudaStream_t stream, int num_sms)
+                                    float* gs_out, uint8_t* q, uint8_t* sf_ptr, bool sf_tiled,
+                                    const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                    int64_t q_bytes, unsigned* err_word, cudaStream_t stream, int num_sms)
 {
     const int64_t bytes = rows * K * static_cast<int64_t>(sizeof(T));
     const int64_t nv = rows * vpr;                       // < 2^31 (checked by the caller)
     const VecIndex ix = make_vec_index(vpr, ldx, K);
+    const SfOut sf = make_sf_out(sf_ptr, sf_tiled, ix, K);
     int64_t cluster_max = kClusterQuantizeMaxBytes;
     if (const char* v = std::getenv("NVFP4_QCLUSTER_MAX_KB")) cluster_max = std::atoll(v) << 10;  // tuning only
     const int ccs = bytes <= cluster_max ? quantize_cluster_size<T>() : 0;
@@ -483,17 +484,17 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
 }
 
 cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
-                                    float* gs_out, uint8_t* q, uint8_t* sf, const float* gs_other,
-                                    int32_t n_alpha, float* alpha_out, unsigned* err_word,
-                                    cudaStream_t stream, int num_sms)
+                                    float* gs_out, uint8_t* q, uint8_t* sf, bool sf_tiled,
+                                    const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                    unsigned* err_word, cudaStream_t stream, int num_sms)
 {
     const int V = bf16 ? 8 : 4;
     const int64_t vpr = K / V;
     const int64_t q_bytes = rows * (K / 2);
     if (bf16)
-        return launch_dynamic_t(static_cast<const __nv_bfloat16*>(x), rows, vpr, ldx, K, gs_out, q, sf,
+        return launch_dynamic_t(static_cast<const __nv_bfloat16*>(x), rows, vpr, ldx, K, gs_out, q, sf, sf_tiled,
                                 gs_other, n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
-    return launch_dynamic_t(static_cast<const float*>(x), rows, vpr, ldx, K, gs_out, q, sf, gs_other,
+    return launch_dynamic_t(static_cast<const float*>(x), rows, vpr, ldx, K, gs_out, q, sf, sf_tiled, gs_other,
                             n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
 }
 
@@ -512,6 +513,33 @@ cudaError_t launch_round(const float* x, int64_t n, uint8_t* out, bool e2m1, cud
     const int grid = grid_for(n, num_sms);
     if (e2m1) round_e2m1_kernel<<<grid, 256, 0, stream>>>(x, n, out);
     else round_e4m3_kernel<<<grid, 256, 0, stream>>>(x, n, out);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ scale layout
+
+// Row-major scales [rows][K/16] -> the tiled layout (quant_core.cuh, SfOut), one output byte
+// per thread; rows past `rows` in the last 128-row tile are zero.
+__global__ void sf_tile_kernel(const uint8_t* __restrict__ sf, int64_t rows, int64_t kb, int64_t kb4,
+                               uint8_t* __restrict__ out, int64_t out_bytes)
+{
+    for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < out_bytes;
+         o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t block = o >> 9, within = o & 511;
+        const int64_t rt = block / kb4, kt = block - rt * kb4;
+        const int64_t r = rt * 128 + ((within >> 2) & 3) * 32 + (within >> 4);
+        const int64_t c = kt * 4 + (within & 3);
+        out[o] = r < rows ? sf[r * kb + c] : 0;
+    }
+}
+
+cudaError_t launch_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* out, cudaStream_t stream,
+                           int num_sms)
+{
+    const int64_t out_bytes = (rows + 127) / 128 * 128 * (K / 16);
+    if (out_bytes == 0) return cudaSuccess;
+    const int grid = grid_for(out_bytes, num_sms);
+    sf_tile_kernel<<<grid, 256, 0, stream>>>(sf, rows, K / 16, K / 64, out, out_bytes);
     return cudaGetLastError();
 }
 

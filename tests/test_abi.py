@@ -111,6 +111,21 @@ def test_quantize_dynamic_host_validation(lib):
     assert f(0x1004, 0, 4, 64, 64, 0x2000, 0x3000, 0x4000, None, 0, None, None) == 3
 
 
+def test_tiled_scale_host_validation(lib):
+    assert lib.nvfp4_sf_bytes(300, 512, 0) == 300 * 32
+    assert lib.nvfp4_sf_bytes(300, 512, 1) == 384 * 32
+    assert lib.nvfp4_sf_bytes(300, 48, 1) == 0          # tiled needs K % 64 == 0
+    assert lib.nvfp4_sf_bytes(300, 512, 5) == 0
+    assert lib.nvfp4_sf_tile(0x1000, 4, 48, 0x2000, None) == 2
+    assert lib.nvfp4_sf_tile(None, 4, 64, 0x2000, None) == 1
+    assert lib.nvfp4_sf_tile(0x1000, 0, 64, 0x2000, None) == 0
+    g = lib.nvfp4_gemm_ex
+    assert g(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 16, 768, 6144, None, 0, 7, None) == 1
+    q = lib.nvfp4_quantize_dynamic_ex
+    assert q(0x1000, 0, 4, 64, 64, 0x2000, 0x3000, 0x4000, None, 0, None, 3, None) == 1
+    assert q(0x1000, 0, 4, 48, 48, 0x2000, 0x3000, 0x4000, None, 0, None, 1, None) == 2
+
+
 def test_bounded_wait_check_host_validation(lib):
     assert lib.nvfp4_check_bounded_wait(0, None) == 1
     assert lib.nvfp4_check_bounded_wait(1000001, None) == 1
