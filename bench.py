@@ -233,7 +233,7 @@ def roofline_us(flops, nbytes, peaks):
 class AttnSweep:
     """Resident inputs, outputs and workspaces of the attention-projection sweep."""
 
-    def __init__(self, dev, rank, set_index=0, tiled=False):
+    def __init__(self, dev, rank, set_index=0, tiled=True):
         import nvfp4_block_scaled_08_b200 as nv
         from nvfp4_block_scaled_08_b200 import workloads
         self.nv = nv
@@ -657,10 +657,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sf-layout", choices=["tiled", "linear"], default="linear",
-                    help="scale layout of both GEMM operands in the sweep (measured on B200: linear "
-                         "189.1 vs tiled 186.4 TFLOP/s here, where the quantiser's tiled scale stores "
-                         "cost more than the GEMM saves; the compute-bound context GEMMs use tiled)")
+    ap.add_argument("--sf-layout", choices=["tiled", "linear"], default="tiled",
+                    help="scale layout of both GEMM operands in the sweep (tiled: the layout the "
+                         "tensor cores read, fetched without a re-layout step)")
     ap.add_argument("--no-context", action="store_true",
                     help="skip the compute-bound context GEMMs reported after the timed step")
     ap.add_argument("--sets", type=int, default=8,

@@ -47,18 +47,35 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi)
     return r;
 }
 
+// Every lane handles a "vector" of 8 consecutive elements (two lanes per 16-element block):
+// 32 bytes of fp32 (two 16-byte loads) or 16 bytes of bf16.
+struct Raw32 {
+    uint4 lo, hi;
+};
+
 template <typename T> struct InTraits;
 template <> struct InTraits<float> {
-    static constexpr int kPerThread = 4;   // 16 bytes
-    __device__ static void decode(const uint4 u, float (&v)[4])
+    static constexpr int kPerThread = 8;
+    using Raw = Raw32;
+    __device__ static Raw load(const float* p)
     {
-        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
-        v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+        return Raw32{__ldg(reinterpret_cast<const uint4*>(p)), __ldg(reinterpret_cast<const uint4*>(p + 4))};
+    }
+    __device__ static Raw zero() { return Raw32{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)}; }
+    __device__ static void decode(const Raw& u, float (&v)[8])
+    {
+        v[0] = __uint_as_float(u.lo.x); v[1] = __uint_as_float(u.lo.y);
+        v[2] = __uint_as_float(u.lo.z); v[3] = __uint_as_float(u.lo.w);
+        v[4] = __uint_as_float(u.hi.x); v[5] = __uint_as_float(u.hi.y);
+        v[6] = __uint_as_float(u.hi.z); v[7] = __uint_as_float(u.hi.w);
     }
 };
 template <> struct InTraits<__nv_bfloat16> {
-    static constexpr int kPerThread = 8;   // 16 bytes
-    __device__ static void decode(const uint4 u, float (&v)[8])
+    static constexpr int kPerThread = 8;
+    using Raw = uint4;
+    __device__ static Raw load(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+    __device__ static Raw zero() { return make_uint4(0u, 0u, 0u, 0u); }
+    __device__ static void decode(const Raw& u, float (&v)[8])
     {
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -172,32 +189,33 @@ template <typename T>
 struct GlobalVecs {
     const T* x;
     VecIndex ix;
-    __device__ uint4 operator()(uint32_t i) const
+    __device__ typename InTraits<T>::Raw operator()(uint32_t i) const
     {
-        return __ldg(reinterpret_cast<const uint4*>(x + vec_offset<InTraits<T>::kPerThread>(ix, i)));
+        return InTraits<T>::load(x + vec_offset<InTraits<T>::kPerThread>(ix, i));
     }
 };
+template <typename T>
 struct StashVecs {
-    const uint4* stash;
+    const typename InTraits<T>::Raw* stash;
     uint32_t v0;
-    __device__ uint4 operator()(uint32_t i) const { return stash[i - v0]; }
+    __device__ typename InTraits<T>::Raw operator()(uint32_t i) const { return stash[i - v0]; }
 };
 
 // max |x| over vectors i0, i0 + step, ... < end of this thread, kUnroll loads in flight. With
 // `keep`, every loaded vector is also copied to stash[i - v0] (the block's own range).
 template <typename T, typename Src>
 __device__ __forceinline__ float amax_sweep(const Src& src, uint32_t i0, uint32_t end, uint32_t step,
-                                            uint4* keep = nullptr, uint32_t v0 = 0)
+                                            typename InTraits<T>::Raw* keep = nullptr, uint32_t v0 = 0)
 {
     constexpr int V = InTraits<T>::kPerThread;
     constexpr int U = kUnroll;
     float m = 0.0f;
     for (; i0 < end; i0 += U * step) {
-        uint4 w[U];
+        typename InTraits<T>::Raw w[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const uint32_t i = i0 + u * step;
-            w[u] = i < end ? src(i) : make_uint4(0u, 0u, 0u, 0u);
+            w[u] = i < end ? src(i) : InTraits<T>::zero();
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -235,7 +253,8 @@ __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint
                                                float gs, const float* rcp_tab, uint8_t* __restrict__ q,
                                                const SfOut& sfo)
 {
-    constexpr int V = InTraits<T>::kPerThread;   // elements per thread
+    constexpr int V = InTraits<T>::kPerThread;   // elements per thread (8)
+    static_assert(V == 8, "8 elements per lane: 4 bytes of codes");
     constexpr int TPB = 16 / V;                  // threads per 16-element block
     constexpr int U = kUnroll;
     const uint32_t lane = threadIdx.x & 31;
@@ -244,7 +263,7 @@ __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const uint32_t i = w0 + u * step + lane;
-            InTraits<T>::decode(i < end ? src(i) : make_uint4(0u, 0u, 0u, 0u), v[u]);
+            InTraits<T>::decode(i < end ? src(i) : InTraits<T>::zero(), v[u]);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -273,8 +292,7 @@ __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint
                 packed |= f32x2_to_e2m1x2(__fmul_rn(v[u][k], rcp), __fmul_rn(v[u][k + 1], rcp)) << (4 * k);
             if (i < end) {
                 uint8_t* dst = q + static_cast<int64_t>(i) * (V / 2);
-                if constexpr (V == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
-                else *reinterpret_cast<uint32_t*>(dst) = packed;
+                *reinterpret_cast<uint32_t*>(dst) = packed;        // V == 8: 4 bytes of codes
                 if ((lane & (TPB - 1)) == 0) *sfo.at<TPB>(i) = static_cast<uint8_t>(sfq);
             }
         }

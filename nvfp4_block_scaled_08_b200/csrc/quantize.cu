@@ -97,7 +97,8 @@ __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
     namespace cg = cooperative_groups;
     constexpr int V = InTraits<T>::kPerThread;
     cg::grid_group grid = cg::this_grid();
-    extern __shared__ uint4 stash[];
+    extern __shared__ uint4 stash_raw[];
+    typename InTraits<T>::Raw* stash = reinterpret_cast<typename InTraits<T>::Raw*>(stash_raw);
     __shared__ float red[32];
     float* partial = reinterpret_cast<float*>(q);
     volatile uint32_t* read_flag = reinterpret_cast<volatile uint32_t*>(q) + gridDim.x;
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
     __shared__ float rcp_tab[256];
     build_rcp_table(gs, rcp_tab);
     if constexpr (RESIDENT) {
-        quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sfo);
+        quantize_sweep<T>(StashVecs<T>{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sfo);
     } else {
         quantize_sweep<T>(GlobalVecs<T>{x, ix}, bid * blockDim.x + (threadIdx.x & ~31u), nv,
                           nblocks * blockDim.x, gs, rcp_tab, q, sfo);
@@ -173,7 +174,8 @@ __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
     float* __restrict__ gs_out, uint8_t* __restrict__ q, const SfOut sfo,
     const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out)
 {
-    extern __shared__ uint4 stash[];
+    extern __shared__ uint4 stash_raw[];
+    typename InTraits<T>::Raw* stash = reinterpret_cast<typename InTraits<T>::Raw*>(stash_raw);
     __shared__ float red[32];
     __shared__ float cta_max;
     grid_dependency_wait();      // launched early behind the previous kernel: wait for its data
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
     cudaTriggerProgrammaticLaunchCompletion();
     __shared__ float rcp_tab[256];
     build_rcp_table(gs, rcp_tab);
-    quantize_sweep<T>(StashVecs{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sfo);
+    quantize_sweep<T>(StashVecs<T>{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sfo);
     cluster_wait();                                   // no CTA leaves while a peer may read it
 }
 
@@ -252,7 +254,7 @@ cudaError_t launch_global_scale(const void* x, bool bf16, int64_t numel, float* 
     if (e != cudaSuccess) return e;
     if (numel > 0) {
         // numel elements viewed as one row of 16-byte vectors, plus a scalar tail
-        const int V = bf16 ? 8 : 4;
+        const int V = 8;                       // elements per vector (quant_core.cuh)
         const int64_t nvec = numel / V;
         if (nvec > 0) {
             // pieces of fewer than 2^31 vectors; the maxima meet in one atomicMax word
@@ -295,7 +297,7 @@ cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, i
                             const float* gs, uint8_t* q, uint8_t* sf, cudaStream_t stream,
                             int num_sms)
 {
-    const int V = bf16 ? 8 : 4;
+    const int V = 8;                       // elements per vector (quant_core.cuh)
     const int64_t vpr = K / V;
     if (rows == 0 || vpr == 0) return cudaSuccess;
     const VecIndex ix = make_vec_index(vpr, ldx, K);
@@ -377,10 +379,13 @@ static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float
                                int64_t q_bytes, unsigned* err_word, cudaStream_t stream, int num_sms)
 {
     constexpr int64_t kResidentMaxBytes = (int64_t(200) << 10) / BPS;
-    int64_t blocks = std::min<int64_t>(BPS * static_cast<int64_t>(num_sms), (nv + 2 * THREADS - 1) / (2 * THREADS));
+    // at least 32 bytes of input per thread
+    const int64_t per_block = 32 * static_cast<int64_t>(THREADS) / static_cast<int64_t>(sizeof(typename InTraits<T>::Raw));
+    int64_t blocks = std::min<int64_t>(BPS * static_cast<int64_t>(num_sms), (nv + per_block - 1) / per_block);
     blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, q_bytes / 8));
     int64_t chunk = round_up((nv + blocks - 1) / blocks, 32);
-    const bool resident = chunk * 16 <= kResidentMaxBytes;
+    constexpr int64_t kVecBytes = sizeof(typename InTraits<T>::Raw);
+    const bool resident = chunk * kVecBytes <= kResidentMaxBytes;
     void (*kern)(const T*, const VecIndex, uint32_t, uint32_t, float*, uint8_t*, const SfOut, const float*,
                  int32_t, float*, unsigned*) =
         resident ? quantize_dynamic_kernel<T, true, THREADS> : quantize_dynamic_kernel<T, false, THREADS>;
@@ -391,7 +396,7 @@ static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float
             cudaFuncSetAttribute(quantize_dynamic_kernel<T, true, THREADS>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kResidentMaxBytes));
         });
-        smem = static_cast<size_t>(chunk) * 16;
+        smem = static_cast<size_t>(chunk) * kVecBytes;
     }
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, smem);
@@ -402,7 +407,7 @@ static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float
         if (blocks > fit) {        // fewer blocks than planned: larger shares (same smem bound)
             blocks = fit;
             chunk = round_up((nv + blocks - 1) / blocks, 32);
-            if (chunk * 16 > static_cast<int64_t>(smem)) return cudaErrorInvalidConfiguration;
+            if (chunk * kVecBytes > static_cast<int64_t>(smem)) return cudaErrorInvalidConfiguration;
         }
         blocks = (nv + chunk - 1) / chunk;       // no empty block
     } else {
@@ -450,7 +455,8 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
     if (ccs > 0) {
         const int cs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ccs, (nv + 511) / 512)));
         const int64_t chunk = round_up((nv + cs - 1) / cs, 32);
-        if (chunk * 16 > kClusterStashMaxBytes) return cudaErrorInvalidValue;
+        if (chunk * static_cast<int64_t>(sizeof(typename InTraits<T>::Raw)) > kClusterStashMaxBytes)
+            return cudaErrorInvalidValue;
         auto kern = quantize_dynamic_cluster_kernel<T>;
         static std::once_flag once;
         std::call_once(once, [&] {
@@ -461,7 +467,7 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
         std::memset(&cfg, 0, sizeof(cfg));
         cfg.gridDim = dim3(1, static_cast<unsigned>(cs), 1);
         cfg.blockDim = dim3(512, 1, 1);
-        cfg.dynamicSmemBytes = static_cast<size_t>(chunk) * 16;
+        cfg.dynamicSmemBytes = static_cast<size_t>(chunk) * sizeof(typename InTraits<T>::Raw);
         cfg.stream = stream;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -488,7 +494,7 @@ cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int6
                                     const float* gs_other, int32_t n_alpha, float* alpha_out,
                                     unsigned* err_word, cudaStream_t stream, int num_sms)
 {
-    const int V = bf16 ? 8 : 4;
+    const int V = 8;                       // elements per vector (quant_core.cuh)
     const int64_t vpr = K / V;
     const int64_t q_bytes = rows * (K / 2);
     if (bf16)
