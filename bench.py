@@ -99,12 +99,12 @@ def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> fl
     return flops_per_rank * world / (step_ms_max * 1e-3) / 1e12
 
 
-# DRAM traffic of the GEMM launches of one sweep (M = 16, 64, 256, 1024), from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum, cold L2; the bf16 outputs stay in L2 within a
-# launch): 2764800 + 2935040 + 3601664 + 6255872 bytes; the capture command and its table are
+# DRAM traffic of the GEMM launches of one sweep (M = 16, 64, 256, 1024; tiled scales), from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, cold L2; the bf16 outputs stay in
+# L2 within a launch): 2802432 + 2954240 + 3596544 + 6251008 bytes; the capture command and its table are
 # in the committed ncu summary of these launches under profiles/. Valid only for the kernel
 # sources it was taken on (hash below); reported as null otherwise.
-GEMM_TRAFFIC_BYTES = 2764800 + 2935040 + 3601664 + 6255872
+GEMM_TRAFFIC_BYTES = 2802432 + 2954240 + 3596544 + 6251008
 GEMM_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "gemm.cu", "ptx.cuh", "internal.h")
 GEMM_TRAFFIC_SHA = "38bbc7cceb6df712"
 
