@@ -106,17 +106,27 @@ def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> fl
 # sources it was taken on (hash below); reported as null otherwise.
 GEMM_TRAFFIC_BYTES = 2802432 + 2954240 + 3596544 + 6251008
 GEMM_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "gemm.cu", "ptx.cuh", "internal.h")
-GEMM_TRAFFIC_SHA = "38bbc7cceb6df712"
+GEMM_TRAFFIC_SHA = "9dbe30d4e3215f45"
+
+
+def _code_hash(files) -> str:
+    """sha256 (16 hex digits) of the sources with their comments removed: it changes when
+    the code the counters were taken on changes, not when a comment does."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "nvfp4_block_scaled_08_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(" ".join(src.split()).encode())
+    return h.hexdigest()[:16]
 
 
 def gemm_traffic():
-    """The captured traffic, or None once the GEMM sources differ from the captured ones."""
-    import hashlib
-    h = hashlib.sha256()
-    for f in GEMM_TRAFFIC_SOURCES:
-        with open(os.path.join(ROOT, "nvfp4_block_scaled_08_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    return GEMM_TRAFFIC_BYTES if h.hexdigest()[:16] == GEMM_TRAFFIC_SHA else None
+    """The captured traffic, or None once the GEMM code differs from the captured one."""
+    return GEMM_TRAFFIC_BYTES if _code_hash(GEMM_TRAFFIC_SOURCES) == GEMM_TRAFFIC_SHA else None
 
 
 def measured_peaks():

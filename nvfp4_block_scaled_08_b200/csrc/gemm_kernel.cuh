@@ -14,11 +14,13 @@
 //   * GROUPED     : SWAP with per-expert weights B[e] and token rows [off[e], off[e+1]).
 //
 // Roles (384 threads, one CTA per SM, persistent over tiles):
-//   warp 0      TMA producer: A/B tiles (128-byte swizzle) and linear scale tiles.
+//   warp 0      TMA producer: A/B tiles (128-byte swizzle) and the scales: with tiled
+//               scales (SFT) one 2 KB bulk copy per 128 rows and stage, already in the form
+//               tcgen05.cp reads; with linear scales, linear [rows][16 B] tiles.
 //   warp 1      TMEM allocator and single-thread MMA issuer (tcgen05.cp of scales, then
 //               four 128 x BN x 64 block-scaled MMAs per 256-element K stage).
-//   warps 2-3   scale re-layout, alternate stages: turn the TMA'd [rows][16 B] scale tile
-//               into the 32-row x 16-byte blocks that tcgen05.cp ... 32x128b.warpx4
+//   warps 2-3   linear scales only: re-layout, alternate stages: turn the TMA'd [rows][16 B]
+//               scale tile into the 32-row x 16-byte blocks that tcgen05.cp ... 32x128b.warpx4
 //               replicates into the TMEM layout the MMA reads (row r at column base + r/32,
 //               byte = k-block). Warp 3 first builds the per-expert tile prefix (grouped).
 //   warps 4-11  epilogue, two warpgroups (one per half of the tile's columns; warp w reads
