@@ -42,6 +42,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import platform
 import statistics
 import sys
 import threading
@@ -589,13 +590,20 @@ class OracleSweep:
         self.one_pass([min(64, m) for m in self.Ms])
         self.per_row = (time.perf_counter() - t0) / sum(min(64, m) for m in self.Ms)
 
-    def one_pass(self, rows):
+    def one_pass(self, rows, split=None):
+        """One pass over the row sample; adds the quantise and GEMM seconds to split[0], [1]."""
         o = self.oracle
         f = 0.0
         for a, r in zip(self.a_all, rows):
+            t0 = time.perf_counter()
             ga = o.global_scale(a)
             qa, sa = o.quantize(a[:r], ga)
+            t1 = time.perf_counter()
             o.gemm(qa, sa, self.qb, self.sb, o.alpha(ga, self.gb), threads=self.threads)
+            t2 = time.perf_counter()
+            if split is not None:
+                split[0] += t1 - t0
+                split[1] += t2 - t1
             f += 2.0 * r * N_ATTN * K_ATTN
         return f
 
@@ -605,26 +613,38 @@ class OracleSweep:
         frac = min(1.0, budget_s / max(self.per_row * sum(self.Ms), 1e-9))
         rows = [max(1, int(round(m * frac))) for m in self.Ms]
         flops, passes = 0.0, 0
+        self.split = [0.0, 0.0]
         t0 = time.perf_counter()
         while True:
-            flops += self.one_pass(rows)
+            flops += self.one_pass(rows, self.split)
             passes += 1
             if time.perf_counter() - t0 >= 0.8 * budget_s:
                 break
         dt = time.perf_counter() - t0
         sample = (f"attn_proj sweep, first {rows} rows of M={list(M_SWEEP)} (global scale over the "
-                  f"full A), N=768, K=6144, {passes} pass(es); weights quantised outside timing")
+                  f"full A), N=768, K=6144, {passes} pass(es); weights quantised outside timing; "
+                  f"GEMM on {self.threads} threads, quantisation on one")
         return flops, dt, self.threads, sample
 
 
-def oracle_sweep_sample(budget_s: float):
-    return OracleSweep().run(budget_s)
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
 
 
 def cpu_baseline(budget_s: float):
-    flops, dt, threads, sample = oracle_sweep_sample(budget_s)
+    sweep = OracleSweep()
+    flops, dt, threads, sample = sweep.run(budget_s)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
-            "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+            "kind": "oracle", "sample": sample, "seconds": round(dt, 2),
+            "quantize_seconds": round(sweep.split[0], 3), "gemm_seconds": round(sweep.split[1], 3),
+            "cpu_model": cpu_model()}
 
 
 def run_reference(args, world, rank):
@@ -635,12 +655,14 @@ def run_reference(args, world, rank):
     sweep = OracleSweep()
     for _ in range(args.warmup):
         sweep.run(per_step)
-    tot_f = tot_t = 0.0
+    tot_f = tot_t = tot_q = tot_g = 0.0
     info = None
     for _ in range(args.steps):
         f, t, th, sample = sweep.run(per_step)
         tot_f += f
         tot_t += t
+        tot_q += sweep.split[0]
+        tot_g += sweep.split[1]
         info = (th, sample)
     value = tot_f / tot_t / 1e12
     return {
@@ -653,7 +675,8 @@ def run_reference(args, world, rank):
         "config": {"workload": "attn_proj_sweep N=768 K=6144 M={16,64,256,1024}",
                    "note": "CPU oracle (test infrastructure) on a bounded row sample per step"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": info[0],
-                         "kind": "oracle", "sample": info[1]},
+                         "kind": "oracle", "sample": info[1], "quantize_seconds": round(tot_q, 3),
+                         "gemm_seconds": round(tot_g, 3), "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
