@@ -3,7 +3,8 @@
 * Format tables and encoders: the ml_dtypes library (float4_e2m1fn, float8_e4m3fn),
   torch's float8_e4m3fn conversion, and brute-force nearest-value search.
 * Quantisation: closed forms (the amax block gets scale 448 and code 6.0, constant blocks,
-  zero blocks, sign symmetry, nibble order) and the NVFP4 reconstruction-error bound.
+  constant tensors that dequantise back to themselves, zero blocks, sign symmetry, nibble
+  order) and the NVFP4 reconstruction-error bound.
 * Products: exact rational arithmetic (fractions.Fraction) on small random cases with the
   operand values decoded by ml_dtypes, all-zero scales, one-hot rows, transposition,
   linearity in alpha, and the grouped form against per-expert products.
@@ -173,6 +174,24 @@ def test_quantize_constant_zero_and_sign():
     np.testing.assert_array_equal(sfn, sf)
     codes_n = np.stack([qn & 0xF, qn >> 4], axis=-1).reshape(2, 64)
     np.testing.assert_array_equal(codes_n, codes | 8)
+
+
+@pytest.mark.parametrize("c", [1.0, 0.25, 1024.0, -8.0, 0.1, 3.7e-5, -12345.678, 448.0 * 6])
+def test_constant_tensor_reproduces_itself(c):
+    """A constant tensor: gs = 2688 / |c|, every block scale rounds to 448 (0x7E) and every
+    code to 6.0, so the dequantised value over gs is 2688 / fl(2688 / |c|), within one fp32
+    rounding of c, and exactly c when |c| is a power of two."""
+    x = np.full((3, 48), c, np.float32)
+    gs = oracle.global_scale(x)
+    q, sf = oracle.quantize(x, gs)
+    assert (sf == 0x7E).all()
+    code = 7 | (8 if c < 0 else 0)
+    assert (q == (code | code << 4)).all()
+    back = oracle.dequantize(q, sf) / np.float64(gs)
+    cf = np.float64(np.float32(c))
+    assert np.all(np.abs(back - cf) <= 2.0 ** -23 * abs(cf))
+    if math.frexp(abs(cf))[0] == 0.5:
+        assert np.all(back == cf)
 
 
 def test_quantize_nibble_order():
