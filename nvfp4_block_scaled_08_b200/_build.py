@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libnvfp4.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
 SOURCES = ["api.cu", "gemm.cu", "quantize.cu", "noalloc.cu"]
-HEADERS = ["ptx.cuh", "gemm_kernel.cuh", "internal.h"]
+HEADERS = ["ptx.cuh", "gemm_kernel.cuh", "internal.h", "quant_core.cuh"]
 
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",

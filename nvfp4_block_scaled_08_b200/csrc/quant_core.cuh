@@ -47,6 +47,40 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi)
     return r;
 }
 
+// Eight fp32 values times r, each product rounded to nearest even (four packed two-lane
+// multiplies, mul.rn.f32x2), then e2m1-coded and packed into 32 bits: value 2i in the low
+// nibble of byte i, as f32x2_to_e2m1x2 does for one pair.
+__device__ __forceinline__ uint32_t scale_to_e2m1x8(const float (&v)[8], float r)
+{
+    uint32_t out;
+    asm("{\n\t"
+        ".reg .b64 s, p0, p1, p2, p3;\n\t"
+        ".reg .f32 y0, y1, y2, y3, y4, y5, y6, y7;\n\t"
+        ".reg .b8 c0, c1, c2, c3;\n\t"
+        "mov.b64 s, {%9, %9};\n\t"
+        "mov.b64 p0, {%1, %2};\n\t"
+        "mov.b64 p1, {%3, %4};\n\t"
+        "mov.b64 p2, {%5, %6};\n\t"
+        "mov.b64 p3, {%7, %8};\n\t"
+        "mul.rn.f32x2 p0, p0, s;\n\t"
+        "mul.rn.f32x2 p1, p1, s;\n\t"
+        "mul.rn.f32x2 p2, p2, s;\n\t"
+        "mul.rn.f32x2 p3, p3, s;\n\t"
+        "mov.b64 {y0, y1}, p0;\n\t"
+        "mov.b64 {y2, y3}, p1;\n\t"
+        "mov.b64 {y4, y5}, p2;\n\t"
+        "mov.b64 {y6, y7}, p3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c0, y1, y0;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c1, y3, y2;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c2, y5, y4;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c3, y7, y6;\n\t"
+        "mov.b32 %0, {c0, c1, c2, c3};\n\t"
+        "}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(r));
+    return out;
+}
+
 // Every lane handles a "vector" of 8 consecutive elements (two lanes per 16-element block):
 // 32 bytes of fp32 (two 16-byte loads) or 16 bytes of bf16.
 struct Raw32 {
@@ -139,14 +173,15 @@ struct SfOut {
     uint32_t kb4;            // K / 64: 512-byte blocks per 128-row tile
     uint32_t vpr, mul, shift;  // vector -> row, as in VecIndex
 
+    // Scale of vector i's block. Offsets fit in 32 bits: there are fewer than 2^31 vectors,
+    // so fewer than 2^30 scales, and the tiled layout pads the rows to 128 at most.
     template <int TPB>
-    __device__ __forceinline__ uint8_t* at(uint32_t i) const   // scale of vector i's block
+    __device__ __forceinline__ uint8_t* at(uint32_t i) const
     {
         if (!tiled) return sf + i / TPB;
         const uint32_t r = static_cast<uint32_t>((static_cast<uint64_t>(__umulhi(i, mul)) + i) >> shift);
         const uint32_t c = (i - r * vpr) / TPB;
-        return sf + (static_cast<uint64_t>(r >> 7) * kb4 + (c >> 2)) * 512 + (r & 31u) * 16 + ((r >> 5) & 3u) * 4 +
-               (c & 3u);
+        return sf + (((r >> 7) * kb4 + (c >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (c & 3u));
     }
 };
 
@@ -233,7 +268,8 @@ __device__ __forceinline__ float amax_sweep(const Src& src, uint32_t i0, uint32_
 // Quantise vectors [.., end): this warp takes the 32 consecutive vectors w0 + lane, then
 // w0 + step + lane, ... (w0 warp-uniform and a multiple of 32). The TPB lanes that share a
 // 16-element block are consecutive lanes of the warp (a block never straddles a row since
-// vpr % TPB == 0); the first of them computes the block scale and shares it.
+// vpr % TPB == 0); after a butterfly exchange each of them holds the block maximum and
+// computes the same scale (no divergent branch), and the first of them stores it.
 // Per block, in fp32 with explicit rounding and in this order:
 //   amax -> s = e4m3(amax / 6 * gs) -> r = s ? gs / s : 0 -> codes e2m1(x * r).
 // rcp_tab[c] = gs / e4m3(c) (0 where e4m3(c) is zero) for all 256 scale codes: every block
@@ -276,20 +312,10 @@ __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint
 #pragma unroll
             for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
 
-            uint32_t sfq = 0;
-            float rcp = 0.0f;
-            if ((lane & (TPB - 1)) == 0) {
-                const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
-                sfq = f32_to_e4m3(sf32);
-                rcp = rcp_tab[sfq];
-            }
-            const uint32_t leader = lane & ~static_cast<uint32_t>(TPB - 1);
-            rcp = __shfl_sync(0xffffffffu, rcp, leader);
-
-            uint32_t packed = 0;
-#pragma unroll
-            for (int k = 0; k < V; k += 2)
-                packed |= f32x2_to_e2m1x2(__fmul_rn(v[u][k], rcp), __fmul_rn(v[u][k + 1], rcp)) << (4 * k);
+            const float sf32 = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+            const uint32_t sfq = f32_to_e4m3(sf32);
+            const float rcp = rcp_tab[sfq];
+            const uint32_t packed = scale_to_e2m1x8(v[u], rcp);
             if (i < end) {
                 uint8_t* dst = q + static_cast<int64_t>(i) * (V / 2);
                 *reinterpret_cast<uint32_t*>(dst) = packed;        // V == 8: 4 bytes of codes
