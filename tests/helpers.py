@@ -46,3 +46,17 @@ def check_within_tolerance(out_gpu: torch.Tensor, v: np.ndarray, S: np.ndarray, 
 
 def bf16_bits_of(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def tile_np(sf: np.ndarray, K: int) -> np.ndarray:
+    """The tiled layout: row r, scale column c at ((r // 128) * (K // 64) + c // 4) * 512
+    + (r % 32) * 16 + ((r // 32) % 4) * 4 + c % 4; rows padded to 128 with zeros."""
+    rows, kb = sf.shape
+    assert kb == K // 16
+    R = (rows + 127) // 128 * 128
+    out = np.zeros(R * kb, dtype=np.uint8)
+    r = np.arange(rows)[:, None]
+    c = np.arange(kb)[None, :]
+    off = ((r // 128) * (K // 64) + c // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + c % 4
+    out[off] = sf
+    return out

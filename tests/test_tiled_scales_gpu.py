@@ -16,23 +16,9 @@ import torch
 import nvfp4_block_scaled_08_b200 as nv
 from nvfp4_block_scaled_08_b200 import workloads
 import oracle
-from helpers import bf16_bits_of, check_within_tolerance, gpu_quantize
+from helpers import bf16_bits_of, check_within_tolerance, gpu_quantize, tile_np
 
 pytestmark = pytest.mark.gpu
-
-
-def tile_np(sf: np.ndarray, K: int) -> np.ndarray:
-    """The tiled layout: row r, scale column c at ((r // 128) * (K // 64) + c // 4) * 512
-    + (r % 32) * 16 + ((r // 32) % 4) * 4 + c % 4; rows padded to 128 with zeros."""
-    rows, kb = sf.shape
-    assert kb == K // 16
-    R = (rows + 127) // 128 * 128
-    out = np.zeros(R * kb, dtype=np.uint8)
-    r = np.arange(rows)[:, None]
-    c = np.arange(kb)[None, :]
-    off = ((r // 128) * (K // 64) + c // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + c % 4
-    out[off] = sf
-    return out
 
 
 @pytest.mark.parametrize("rows,K", [(1, 64), (128, 256), (300, 512), (1024, 6144)])
