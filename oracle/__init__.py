@@ -17,8 +17,14 @@ follows; readings of points the pages leave open are listed in the design notes:
   ("The Moment the Zeros Disappeared", section "The Subject Message"); the grouped form
   is the per-expert product of a 256-expert, top-8 MoE layer ("When a Benchmark
   Crashes", section "Why This Message Was Written").
+* ``mx_quantize`` / ``mx_dequantize`` / ``mx_gemm``: the MXFP4 variant that the mm_fp4
+  signature selects with ``use_nvfp4=False`` ("The Art of Reading the Manual", section "The
+  Message"); the pages do not define it, so it follows the OCP MX v1.0 FP4 format (E8M0
+  power-of-two scale per 32 elements, no per-tensor scale). Not implemented by the CUDA
+  library.
 
-Parity pins: ``tests/test_oracle.py`` (all functions pinned; none is "parity unpinned").
+Parity pins: ``tests/test_oracle.py`` and ``tests/test_oracle_mx.py`` (all functions
+pinned; none is "parity unpinned").
 """
 from __future__ import annotations
 
@@ -74,6 +80,10 @@ def _load():
         "oracle_gemm_dequantized": (cint, [P, P, f64, i64, i64, i64, P, P, cint]),
         "oracle_gemm": (cint, [P, P, P, P, f32, i64, i64, i64, P, P, cint]),
         "oracle_grouped_gemm": (cint, [P, P, P, P, P, P, i32, i64, i64, P, P, cint]),
+        "oracle_e8m0_decode": (f64, [cint]),
+        "oracle_mx_quantize": (None, [P, i64, i64, i64, P, P]),
+        "oracle_mx_dequantize": (None, [P, P, i64, i64, P]),
+        "oracle_mx_gemm": (cint, [P, P, P, P, f32, i64, i64, i64, P, P, cint]),
         "oracle_bf16_bits": (ctypes.c_uint16, [f64]),
         "oracle_bf16_bits_array": (None, [P, i64, P]),
     }
@@ -202,6 +212,59 @@ def grouped_gemm(Aq, sfA, Bq, sfB, alphas, offsets, threads=None):
                                      _threads(threads))
     if ex < 0:
         raise MemoryError("oracle_grouped_gemm: allocation failed")
+    return v, S, bool(ex)
+
+
+# ---- MXFP4 (use_nvfp4=False): OCP MX e2m1 with an E8M0 scale per 32 elements ------------
+
+def e8m0_decode(byte: int) -> float:
+    """Value of an E8M0 scale byte: 2^(byte - 127); 255 is NaN."""
+    return _load().oracle_e8m0_decode(int(byte))
+
+
+def mx_quantize(x) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP4 quantisation of a row-major fp32 [rows, K] tensor (K % 32 == 0): per 32-element
+    block, shared_exp = floor(log2(amax)) - 2 clamped to [-127, 127] (all-zero block: -127),
+    codes e2m1_rn_satfinite(x / 2^shared_exp). Returns (q uint8 [rows, K/2], sf uint8
+    [rows, K/32] E8M0 bytes = shared_exp + 127)."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    rows, K = x.shape
+    assert K % 32 == 0
+    q = np.empty((rows, K // 2), dtype=np.uint8)
+    sf = np.empty((rows, K // 32), dtype=np.uint8)
+    _load().oracle_mx_quantize(_ptr(x), rows, K, K, _ptr(q), _ptr(sf))
+    return q, sf
+
+
+def mx_dequantize(q, sf) -> np.ndarray:
+    """deq[r, k] = e2m1(q[r, k]) * 2^(sf[r, k // 32] - 127) as float64."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    rows, K = q.shape[0], q.shape[1] * 2
+    out = np.empty((rows, K), dtype=np.float64)
+    _load().oracle_mx_dequantize(_ptr(q), _ptr(sf), rows, K, _ptr(out))
+    return out
+
+
+def mx_gemm(Aq, sfA, Bq, sfB, alpha_value=1.0, threads=None):
+    """The MXFP4 product: v = alpha * sum_k deq(A)[m,k] deq(B)[n,k] with E8M0 scales per 32
+    K elements (fp64, ascending k, one rounding of the exact sum), S = sum_k |a b|.
+    Returns (v, S, exact)."""
+    Aq = np.ascontiguousarray(Aq, dtype=np.uint8)
+    Bq = np.ascontiguousarray(Bq, dtype=np.uint8)
+    sfA = np.ascontiguousarray(sfA, dtype=np.uint8)
+    sfB = np.ascontiguousarray(sfB, dtype=np.uint8)
+    M, K = Aq.shape[0], Aq.shape[1] * 2
+    N = Bq.shape[0]
+    assert Bq.shape[1] * 2 == K and K % 32 == 0
+    assert sfA.shape == (M, K // 32) and sfB.shape == (N, K // 32)
+    v = np.empty((M, N), dtype=np.float64)
+    S = np.empty((M, N), dtype=np.float64)
+    ex = _load().oracle_mx_gemm(_ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB),
+                                float(np.float32(alpha_value)), M, N, K, _ptr(v), _ptr(S),
+                                _threads(threads))
+    if ex < 0:
+        raise MemoryError("oracle_mx_gemm: allocation failed")
     return v, S, bool(ex)
 
 

@@ -22,9 +22,12 @@
  *     amax_block/6*gs rounded to e4m3, and e2m1 codes of x*gs/scale. The order of the
  *     fp32 operations, the tie rule and the sign of zero codes are readings of this
  *     build, listed in the design notes; each function below states the one it uses.
+ *   - MXFP4 (use_nvfp4=False): OCP MX e2m1 elements with an E8M0 power-of-two scale per
+ *     32 elements (the MXFP4 section below). The CUDA library does not implement it; the
+ *     functions are here so that a kernel can be checked against them.
  *
- * Parity pins (tests/test_oracle.py) check every function here against something other
- * than itself: torch's float8_e4m3fn conversion, brute-force nearest-value search, exact
+ * Parity pins (tests/test_oracle.py, tests/test_oracle_mx.py) check every function here
+ * against something other than itself: torch's float8_e4m3fn conversion, brute-force nearest-value search, exact
  * rational arithmetic on small products, closed forms and invariants.
  *
  * Floating point: compile with -ffp-contract=off and without -ffast-math; every fp32
@@ -345,6 +348,116 @@ int oracle_grouped_gemm(const uint8_t* Aq, const uint8_t* sfA, const uint8_t* Bq
         if (ex < 0) return -1;
         if (!ex) exact = 0;
     }
+    return exact;
+}
+
+/* ------------------------------------------------------------------------------------
+ * MXFP4: the variant the pages select with use_nvfp4=False ("The Art of Reading the
+ * Manual", section "The Message", the mm_fp4 signature). The pages name the flag but do not
+ * define the format; this is the OCP Microscaling (MX) v1.0 FP4 format: e2m1 elements, one
+ * E8M0 scale (a bare power of two, 2^(byte - 127); byte 255 is NaN) per block of 32
+ * consecutive K elements, no per-tensor scale. Quantisation follows the MX conversion
+ * rule: shared_exp = floor(log2(amax_block)) - 2 (2 = the largest e2m1 exponent), clamped
+ * to the E8M0 range [-127, 127], and codes = e2m1_rn_satfinite(x / 2^shared_exp). A block
+ * of zeros gets byte 0 (the spec leaves log2(0) open; the smallest scale is the plainest
+ * choice, and its codes are 0 whatever the scale).
+ * ---------------------------------------------------------------------------------- */
+
+/* E8M0 byte -> scale (exact). */
+double oracle_e8m0_decode(int byte)
+{
+    if (byte == 255) return NAN;
+    return ldexp(1.0, byte - 127);
+}
+
+/* x[rows, K] (row stride ld) -> q[rows, K/2] codes (element 2i in the low nibble of byte
+ * i) and sf[rows, K/32] E8M0 bytes. */
+void oracle_mx_quantize(const float* x, int64_t rows, int64_t K, int64_t ld, uint8_t* q,
+                        uint8_t* sf)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* xr = x + r * ld;
+        for (int64_t b = 0; b < K / 32; ++b) {
+            float amax = 0.0f;
+            for (int k = 0; k < 32; ++k) {
+                float a = fabsf(xr[b * 32 + k]);
+                if (a > amax) amax = a;
+            }
+            int shared_exp = -127;
+            if (amax > 0.0f) {
+                int e;
+                frexp((double)amax, &e);             /* amax = f * 2^e, f in [0.5, 1) */
+                shared_exp = (e - 1) - 2;            /* floor(log2(amax)) - 2 */
+                if (shared_exp < -127) shared_exp = -127;
+                if (shared_exp > 127) shared_exp = 127;
+            }
+            sf[r * (K / 32) + b] = (uint8_t)(shared_exp + 127);
+            for (int k = 0; k < 32; k += 2) {
+                /* x / 2^shared_exp is exact in double; below 2^-126 it is far under the
+                 * smallest e2m1 step, so the conversion to float changes no code */
+                float y0 = (float)ldexp((double)xr[b * 32 + k], -shared_exp);
+                float y1 = (float)ldexp((double)xr[b * 32 + k + 1], -shared_exp);
+                q[r * (K / 2) + (b * 32 + k) / 2] =
+                    (uint8_t)(oracle_e2m1_encode(y0) | (oracle_e2m1_encode(y1) << 4));
+            }
+        }
+    }
+}
+
+/* deq[r, k] = e2m1(q[r, k]) * 2^(sf[r, k/32] - 127) as doubles (exact). */
+void oracle_mx_dequantize(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t K,
+                          double* deq)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = q[r * (K / 2) + k / 2];
+            int code = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+            deq[r * K + k] = oracle_e2m1_decode(code) * oracle_e8m0_decode(sf[r * (K / 32) + k / 32]);
+        }
+    }
+}
+
+/* Exponent of the smallest nonzero unit of a dequantised operand: every nonzero element is
+ * a multiple of 2^lsb (e2m1 values are multiples of 0.5). Returns 1 << 20 if all are zero. */
+static int min_unit_exponent(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t K)
+{
+    int lsb = 1 << 20;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < K / 32; ++b) {
+            int any = 0;
+            for (int k = 0; k < 16; ++k)
+                if (q[r * (K / 2) + b * 16 + k] & 0x77) any = 1;
+            int e = (int)sf[r * (K / 32) + b] - 127 - 1;
+            if (any && e < lsb) lsb = e;
+        }
+    return lsb;
+}
+
+/* v[m, n] = alpha * sum_k deqA[m, k] * deqB[n, k] with 32-element E8M0 blocks; S as for
+ * NVFP4. Every product is a multiple of 2^(lsbA + lsbB), so the fp64 sum is exact while
+ * sum |a*b| < 2^(53 + lsbA + lsbB). Returns 1 if every sum was exact, 0 otherwise, -1 on
+ * allocation failure. */
+int oracle_mx_gemm(const uint8_t* Aq, const uint8_t* sfA, const uint8_t* Bq, const uint8_t* sfB,
+                   float alpha, int64_t M, int64_t N, int64_t K, double* v, double* S,
+                   int nthreads)
+{
+    double* da = (double*)malloc(sizeof(double) * (size_t)(M > 0 ? M : 1) * (size_t)K);
+    double* db = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1) * (size_t)K);
+    double* s = S ? S : (double*)malloc(sizeof(double) * (size_t)(M > 0 ? M : 1) * (size_t)(N > 0 ? N : 1));
+    if (!da || !db || !s) { free(da); free(db); if (!S) free(s); return -1; }
+    oracle_mx_dequantize(Aq, sfA, M, K, da);
+    oracle_mx_dequantize(Bq, sfB, N, K, db);
+    oracle_gemm_dequantized(da, db, (double)alpha, M, N, K, v, s, nthreads);
+    int lsb = min_unit_exponent(Aq, sfA, M, K) + min_unit_exponent(Bq, sfB, N, K);
+    int exact = 1;
+    if (lsb < (1 << 19)) {
+        double limit = ldexp(1.0, 53 + lsb);
+        for (int64_t i = 0; i < M * N; ++i)
+            if (s[i] >= limit) exact = 0;
+    }
+    free(da);
+    free(db);
+    if (!S) free(s);
     return exact;
 }
 
