@@ -17,14 +17,18 @@ follows; readings of points the pages leave open are listed in the design notes:
   ("The Moment the Zeros Disappeared", section "The Subject Message"); the grouped form
   is the per-expert product of a 256-expert, top-8 MoE layer ("When a Benchmark
   Crashes", section "Why This Message Was Written").
+* ``silu`` / ``swiglu`` / ``swiglu_quantize``: the gate_up -> down step of the MoE expert
+  MLP (intermediate 2048, "When a Benchmark Crashes", section "Why This Message Was
+  Written"), SwiGLU then NVFP4 with a fixed global scale; readings at the function. Not
+  implemented by the CUDA library.
 * ``mx_quantize`` / ``mx_dequantize`` / ``mx_gemm``: the MXFP4 variant that the mm_fp4
   signature selects with ``use_nvfp4=False`` ("The Art of Reading the Manual", section "The
   Message"); the pages do not define it, so it follows the OCP MX v1.0 FP4 format (E8M0
   power-of-two scale per 32 elements, no per-tensor scale). Not implemented by the CUDA
   library.
 
-Parity pins: ``tests/test_oracle.py`` and ``tests/test_oracle_mx.py`` (all functions
-pinned; none is "parity unpinned").
+Parity pins: ``tests/test_oracle.py``, ``tests/test_oracle_mx.py`` and
+``tests/test_oracle_swiglu.py`` (all functions pinned; none is "parity unpinned").
 """
 from __future__ import annotations
 
@@ -213,6 +217,39 @@ def grouped_gemm(Aq, sfA, Bq, sfB, alphas, offsets, threads=None):
     if ex < 0:
         raise MemoryError("oracle_grouped_gemm: allocation failed")
     return v, S, bool(ex)
+
+
+# ---- gate_up epilogue: SwiGLU, then NVFP4 requantisation for the down projection ----------
+# The MoE layer's expert MLP ("When a Benchmark Crashes", section "Why This Message Was
+# Written": intermediate size 2048) multiplies by a gate_up weight of 2 * 2048 rows and feeds
+# down_proj. The pages do not spell out the activation between them; the readings here:
+# columns [0, I) of the gate_up output are the gate g, columns [I, 2I) the up projection u,
+# h = silu(g) * u with silu(g) = g / (1 + exp(-g)), evaluated in fp64 from the product's
+# exact value, rounded once to fp32, and quantised to NVFP4 with a global scale fixed in
+# advance (gs_h) rather than one taken from max|h|, which a GEMM epilogue cannot know.
+
+def silu(g) -> np.ndarray:
+    """silu(g) = g * sigmoid(g) = g / (1 + exp(-g)) in fp64 (exp(-g) overflows to inf for
+    g < -709, giving -0.0 or 0.0, the limit)."""
+    g = np.asarray(g, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g))
+
+
+def swiglu(v) -> np.ndarray:
+    """h = silu(g) * u for the gate_up output v [rows, 2I] (fp64): g = v[:, :I], u = v[:, I:]."""
+    v = np.asarray(v, dtype=np.float64)
+    I = v.shape[1] // 2
+    assert v.shape[1] == 2 * I
+    return silu(v[:, :I]) * v[:, I:]
+
+
+def swiglu_quantize(v, gs_h) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """The gate_up epilogue: h = swiglu(v) rounded to fp32, then the NVFP4 steps of
+    ``quantize`` with the fixed global scale gs_h. Returns (q, sf, h_fp32)."""
+    h = swiglu(v).astype(np.float32)
+    q, sf = quantize(h, gs_h)
+    return q, sf, h
 
 
 # ---- MXFP4 (use_nvfp4=False): OCP MX e2m1 with an E8M0 scale per 32 elements ------------
