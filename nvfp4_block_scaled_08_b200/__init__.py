@@ -11,6 +11,11 @@ loaded, or the device is not sm_100, calls raise.
     al  = alpha(gs_a, gs_b)               # 1 / (gs_a * gs_b)
     gemm(Aq, sfA, Bq, sfB, al, out)       # out[M, N] bf16
     grouped_gemm(Aq, sfA, Bq, sfB, al_e, offsets, out)   # per-expert products
+
+    # activations in one launch (global scale, alpha against the weights' scale, codes),
+    # with the scales in the layout the tensor cores read; weights' scales re-laid out once
+    q, sf, gs, al = quantize_dynamic(x, gs_other=gs_w, tiled=True)
+    gemm(q, sf, Wq, sf_tile(sf_w), al, out, workspace=make_workspace(M, N, K), tiled=True)
 """
 from __future__ import annotations
 
