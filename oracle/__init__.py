@@ -17,6 +17,10 @@ follows; readings of points the pages leave open are listed in the design notes:
   ("The Moment the Zeros Disappeared", section "The Subject Message"); the grouped form
   is the per-expert product of a 256-expert, top-8 MoE layer ("When a Benchmark
   Crashes", section "Why This Message Was Written").
+* ``route_topk`` / ``permute_by_expert`` / ``gather_quantize`` / ``combine``: the MoE
+  layer's top-8-of-256 routing around the grouped product ("When a Benchmark Crashes",
+  section "Why This Message Was Written"); readings at the functions. Not implemented by
+  the CUDA library (the grouped product takes the sorted rows and offsets as inputs).
 * ``silu`` / ``swiglu`` / ``swiglu_quantize``: the gate_up -> down step of the MoE expert
   MLP (intermediate 2048, "When a Benchmark Crashes", section "Why This Message Was
   Written"), SwiGLU then NVFP4 with a fixed global scale; readings at the function. Not
@@ -27,8 +31,9 @@ follows; readings of points the pages leave open are listed in the design notes:
   power-of-two scale per 32 elements, no per-tensor scale). Not implemented by the CUDA
   library.
 
-Parity pins: ``tests/test_oracle.py``, ``tests/test_oracle_mx.py`` and
-``tests/test_oracle_swiglu.py`` (all functions pinned; none is "parity unpinned").
+Parity pins: ``tests/test_oracle.py``, ``tests/test_oracle_mx.py``,
+``tests/test_oracle_swiglu.py`` and ``tests/test_oracle_routing.py`` (all functions pinned;
+none is "parity unpinned").
 """
 from __future__ import annotations
 
@@ -217,6 +222,61 @@ def grouped_gemm(Aq, sfA, Bq, sfB, alphas, offsets, threads=None):
     if ex < 0:
         raise MemoryError("oracle_grouped_gemm: allocation failed")
     return v, S, bool(ex)
+
+
+# ---- MoE routing: top-k selection, expert-sorted permutation, combine ---------------------
+# The layer routes every token to 8 of 256 experts ("When a Benchmark Crashes", section "Why
+# This Message Was Written"); the pages do not give the router. Readings: probabilities are a
+# softmax over the expert logits; a token takes the k largest, ties going to the lower expert
+# index; its k weights are those probabilities renormalised to sum to 1; the expert-sorted
+# order lists each expert's (token, slot) pairs in ascending token order; the combine after
+# the down projection sums each token's k output rows weighted by its k weights.
+
+def route_topk(logits, k: int):
+    """logits fp32 [T, E] -> (experts int32 [T, k] by descending probability, probs fp64 [T, k],
+    weights fp64 [T, k] = probs / probs.sum(row))."""
+    z = np.asarray(logits, dtype=np.float64)
+    z = z - z.max(axis=1, keepdims=True)
+    p = np.exp(z)
+    p = p / p.sum(axis=1, keepdims=True)
+    order = np.argsort(-p, axis=1, kind="stable")[:, :k]     # stable: ties keep index order
+    probs = np.take_along_axis(p, order, axis=1)
+    return order.astype(np.int32), probs, probs / probs.sum(axis=1, keepdims=True)
+
+
+def permute_by_expert(experts, num_experts: int):
+    """experts int32 [T, k] -> (token_of_row int64 [T*k], slot_of_row int64 [T*k],
+    offsets int32 [E + 1], row_of int64 [T, k]): rows of expert e are
+    [offsets[e], offsets[e+1]), in ascending (token, slot) order; row_of[t, s] is the row
+    that holds token t's slot s."""
+    experts = np.asarray(experts)
+    T, k = experts.shape
+    flat = experts.reshape(-1).astype(np.int64)
+    order = np.argsort(flat, kind="stable")                   # pair i = t * k + s
+    counts = np.bincount(flat, minlength=num_experts)
+    offsets = np.zeros(num_experts + 1, dtype=np.int32)
+    offsets[1:] = np.cumsum(counts)
+    row_of = np.empty(T * k, dtype=np.int64)
+    row_of[order] = np.arange(T * k)
+    return order // k, order % k, offsets, row_of.reshape(T, k)
+
+
+def gather_quantize(x, token_of_row, gs):
+    """The expert-sorted NVFP4 activations: the rows token_of_row of x, quantised with the
+    tensor's global scale gs (rows are independent once gs is fixed)."""
+    x = np.asarray(x, dtype=np.float32)
+    return quantize(x[np.asarray(token_of_row)], gs)
+
+
+def combine(y, weights, row_of):
+    """out[t] = sum_s weights[t, s] * y[row_of[t, s]] in fp64, ascending s."""
+    y = np.asarray(y, dtype=np.float64)
+    weights = np.asarray(weights, dtype=np.float64)
+    T, k = weights.shape
+    out = np.zeros((T, y.shape[1]), dtype=np.float64)
+    for s in range(k):
+        out += weights[:, s:s + 1] * y[row_of[:, s]]
+    return out
 
 
 # ---- gate_up epilogue: SwiGLU, then NVFP4 requantisation for the down projection ----------
