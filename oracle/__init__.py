@@ -95,6 +95,7 @@ def _load():
         "oracle_mx_gemm": (cint, [P, P, P, P, f32, i64, i64, i64, P, P, cint]),
         "oracle_bf16_bits": (ctypes.c_uint16, [f64]),
         "oracle_bf16_bits_array": (None, [P, i64, P]),
+        "oracle_fp16_bits_array": (None, [P, i64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -370,6 +371,15 @@ def bf16_bits(v) -> np.ndarray:
     v = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
     out = np.empty(v.shape, dtype=np.uint16)
     _load().oracle_bf16_bits_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def fp16_bits(v) -> np.ndarray:
+    """Round float64 values to fp16 (nearest even, one rounding, inf above the range); raw
+    uint16 bits. For the float16 output option of the product."""
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    out = np.empty(v.shape, dtype=np.uint16)
+    _load().oracle_fp16_bits_array(_ptr(v), v.size, _ptr(out))
     return out
 
 

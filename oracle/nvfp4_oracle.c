@@ -489,3 +489,33 @@ void oracle_bf16_bits_array(const double* v, int64_t n, uint16_t* out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_bits(v[i]);
 }
+
+/* ------------------------------------------------------------------------------------
+ * fp16 rounding of a double (the out_dtype=float16 option of the mm_fp4 signature, "The Art
+ * of Reading the Manual", section "The Message"), one rounding, nearest-even, as raw bits.
+ * fp16: sign | 5-bit exponent (bias 15) | 10-bit mantissa, subnormals, inf above 65504.
+ * ---------------------------------------------------------------------------------- */
+uint16_t oracle_fp16_bits(double v)
+{
+    if (isnan(v)) return 0x7E00;
+    uint16_t s = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0) return s;
+    int e2;
+    frexp(a, &e2);
+    int E = e2 - 1;                                  /* a in [2^E, 2^(E+1)) */
+    if (E < -14) {
+        /* subnormal: multiples of 2^-24; n = 1024 is the smallest normal (exponent 1) */
+        double n = round_half_even(ldexp(a, 24));
+        return (uint16_t)(s | (uint16_t)n);
+    }
+    double n = round_half_even(ldexp(a, 10 - E));    /* 1024 <= n <= 2048 */
+    if (n == 2048.0) { n = 1024.0; E += 1; }
+    if (E > 15) return (uint16_t)(s | 0x7C00);      /* overflow to infinity */
+    return (uint16_t)(s | ((E + 15) << 10) | ((int)n - 1024));
+}
+
+void oracle_fp16_bits_array(const double* v, int64_t n, uint16_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_fp16_bits(v[i]);
+}

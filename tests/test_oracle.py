@@ -8,7 +8,8 @@
 * Products: exact rational arithmetic (fractions.Fraction) on small random cases with the
   operand values decoded by ml_dtypes, all-zero scales, one-hot rows, transposition,
   linearity in alpha, and the grouped form against per-expert products.
-* bf16 output rounding: brute-force nearest bf16 with ties to even.
+* bf16 output rounding: brute-force nearest bf16 with ties to even; fp16 output
+  rounding: numpy's conversion and a nearest-value search.
 """
 import math
 from fractions import Fraction
@@ -387,6 +388,33 @@ def test_bf16_rounding_brute_force():
     for vi, gi in zip(v, got):
         want = _bf16_brute(float(abs(vi))) | (0x8000 if vi < 0 else 0)
         assert gi == want, (vi, hex(gi), hex(want))
+
+
+def test_fp16_rounding_matches_libraries_and_brute_force():
+    """fp16 output option: one direct rounding of the fp64 value, against numpy's float64 ->
+    float16 conversion and a nearest-value search over all finite fp16 values. (torch's
+    conversion goes through fp32 first, two roundings, and differs near midpoints.)"""
+    rng = np.random.default_rng(12)
+    halves = np.arange(0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)   # +finite
+    mids = (halves[:-1] + halves[1:]) / 2
+    v = np.concatenate([rng.standard_normal(20000) * np.exp2(rng.integers(-26, 17, 20000)),
+                        mids[::37], np.nextafter(mids[::41], 0), np.nextafter(mids[::43], np.inf),
+                        [65504.0, 65519.99, 65520.0, 1e6, 2.0 ** -24, 2.0 ** -25, 2.0 ** -26,
+                         3 * 2.0 ** -26, 0.0, -0.0]])
+    v = np.concatenate([v, -v])
+    got = oracle.fp16_bits(v)
+    with np.errstate(over="ignore"):          # 1e6 and 65520 overflow to inf, as intended
+        np.testing.assert_array_equal(got, v.astype(np.float16).view(np.uint16))
+    for vi in v[:400]:
+        a = abs(float(vi))
+        if a >= 65520.0:
+            want = 0x7C00
+        else:
+            d = np.abs(halves - a)
+            best = np.flatnonzero(d == d.min())
+            want = int(best[0] if best.size == 1 else best[best % 2 == 0][0])
+        want |= 0x8000 if np.signbit(vi) else 0
+        assert oracle.fp16_bits(np.array([vi]))[0] == want, vi
 
 
 # ---------------------------------------------------------------- frozen regression fixture
