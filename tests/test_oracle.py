@@ -429,3 +429,23 @@ def test_oracle_regression_fixture():
     with open(os.path.join(here, "oracle_regression.json")) as f:
         stored = json.load(f)
     assert make_oracle_regression.compute() == stored
+
+
+def test_oracle_next_regression_fixture():
+    """The frozen results of the oracle's MXFP4, fp16, SwiGLU and routing functions; values
+    that pass through exp are compared with a tolerance (libm implementations may differ in
+    the last bit)."""
+    import json
+    import os
+    import sys
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    sys.path.insert(0, here)
+    import make_oracle_next_regression
+    with open(os.path.join(here, "oracle_next_regression.json")) as f:
+        stored = json.load(f)
+    got = make_oracle_next_regression.compute()
+    for section in ("swiglu", "routing"):
+        for key in ("h_samples", "weights_samples"):
+            if key in stored[section]:
+                np.testing.assert_allclose(got[section].pop(key), stored[section].pop(key), rtol=1e-14)
+    assert got == stored
