@@ -144,3 +144,15 @@ def test_binding_is_argument_marshalling_only():
     src = open(os.path.join(ROOT, "nvfp4_block_scaled_08_b200", "__init__.py")).read()
     assert "oracle" not in src.replace("no CPU or alternative-backend path", "")
     assert "import numpy" not in src
+
+
+def test_build_tracks_every_source_and_header():
+    """The library is rebuilt when any of its inputs is newer than it: every .cu file under
+    csrc/ must be compiled and every header must be among the tracked inputs."""
+    import os
+    from nvfp4_block_scaled_08_b200 import _build
+    files = set(os.listdir(_build.CSRC))
+    assert {f for f in files if f.endswith(".cu")} == set(_build.SOURCES)
+    assert {f for f in files if f.endswith((".cuh", ".h"))} == set(_build.HEADERS)
+    tracked = {os.path.basename(p) for p in _build._inputs()}
+    assert "nvfp4.h" in tracked and set(_build.SOURCES) | set(_build.HEADERS) <= tracked
