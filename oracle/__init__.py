@@ -202,6 +202,21 @@ def gemm(Aq, sfA, Bq, sfB, alpha_value, threads=None):
     return v, S, bool(ex)
 
 
+def gemm_dequantized(deqA, deqB, alpha_value, threads=None):
+    """The sum of ``gemm`` on operands already dequantised (float64 [M, K] and [N, K]):
+    ``gemm`` is dequantise-both then this. Returns (v, S, exact)."""
+    deqA = np.ascontiguousarray(deqA, dtype=np.float64)
+    deqB = np.ascontiguousarray(deqB, dtype=np.float64)
+    M, K = deqA.shape
+    N = deqB.shape[0]
+    assert deqB.shape[1] == K
+    v = np.empty((M, N), dtype=np.float64)
+    S = np.empty((M, N), dtype=np.float64)
+    ex = _load().oracle_gemm_dequantized(_ptr(deqA), _ptr(deqB), float(np.float32(alpha_value)), M, N, K,
+                                         _ptr(v), _ptr(S), _threads(threads))
+    return v, S, bool(ex)
+
+
 def grouped_gemm(Aq, sfA, Bq, sfB, alphas, offsets, threads=None):
     """Per expert e: rows [off[e], off[e+1]) of A times B[e]^T, scaled by alpha[e].
 

@@ -390,6 +390,23 @@ def test_bf16_rounding_brute_force():
         assert gi == want, (vi, hex(gi), hex(want))
 
 
+def test_gemm_equals_gemm_of_dequantised_operands():
+    # the benchmark's oracle leg dequantises the static weights once and calls
+    # gemm_dequantized per step; gemm is defined as exactly that composition
+    rng = np.random.default_rng(13)
+    a = rng.standard_normal((9, 256)).astype(np.float32)
+    b = rng.standard_normal((7, 256)).astype(np.float32)
+    ga, gb = oracle.global_scale(a), oracle.global_scale(b)
+    qa, sa = oracle.quantize(a, ga)
+    qb, sb = oracle.quantize(b, gb)
+    al = oracle.alpha(ga, gb)
+    v, S, ex = oracle.gemm(qa, sa, qb, sb, al, threads=3)
+    v2, S2, ex2 = oracle.gemm_dequantized(oracle.dequantize(qa, sa), oracle.dequantize(qb, sb), al, threads=2)
+    np.testing.assert_array_equal(v, v2)
+    np.testing.assert_array_equal(S, S2)
+    assert ex and ex2
+
+
 def test_fp16_rounding_matches_libraries_and_brute_force():
     """fp16 output option: one direct rounding of the fp64 value, against numpy's float64 ->
     float16 conversion and a nearest-value search over all finite fp16 values. (torch's
