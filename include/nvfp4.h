@@ -25,7 +25,8 @@
  *   - Calls are asynchronous on the given stream (0 = legacy default stream). The returned
  *     status covers argument checks and launch errors only. A kernel that gives up on a
  *     bounded internal wait records NVFP4_ERR_TIMEOUT in a device error word that
- *     nvfp4_last_device_error() reads.
+ *     nvfp4_last_device_error() reads; the outputs of the call whose kernel recorded it are
+ *     undefined (the kernel stops early, or goes on after a wait that did not complete).
  *   - No fallback: on a device other than compute capability 10.0 every compute call
  *     returns NVFP4_ERR_ARCH; there is no CPU or alternative-backend path.
  *   - Shapes: K % 256 == 0, N % 8 == 0, M >= 0 arbitrary (M == 0 is a no-op), all sizes
@@ -81,6 +82,10 @@ const char* nvfp4_status_string(nvfp4_status s);
 /*
  * Per-tensor global scale: gs_out[0] = 2688 / max|x| in fp32 (2688 = 448 * 6, so the
  * largest block scale of the tensor lands on e4m3's maximum 448), or 1 if x is all zero.
+ * The pages name the NVFP4 format (e2m1 values, one e4m3 scale per 16 elements: "When a
+ * Benchmark Crashes", section "Input Knowledge Required", item 3) but give no quantisation
+ * recipe; this two-level recipe (a per-tensor fp32 scale, then per-block scales) is the
+ * library's reading of them, and nvfp4_quantize below follows it.
  * x: device, numel elements of the given dtype, 16-byte aligned. gs_out: device, one
  * float, used as the reduction accumulator while the call runs (its old value is
  * ignored). Three stream operations (clear, reduce, finalise). numel == 0 gives 1.
@@ -215,7 +220,9 @@ nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint
  * that every GPU which loads the library holds until the process exits. A shape whose
  * split-K scratch would exceed that size returns NVFP4_ERR_WORKSPACE (nothing launched).
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress
- * with that device current); make that first call before any stream capture. All calls on
+ * with that device current), and so does the first call after the device's CUDA context was
+ * created anew or from a host thread with no context bound yet; make that first call before
+ * any stream capture. All calls on
  * a device share the array and it keeps the last call's contents: each call clears the part
  * that must start at zero, and calls whose kernels overlap on the GPU (other streams,
  * other host threads) race on it, so serialise them. Calls no cudaMalloc / cudaFree.
@@ -225,6 +232,21 @@ nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint
 nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
                                 const uint8_t* sfB, const float* alpha, void* out,
                                 int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+
+/*
+ * Tuning and test hook: forces parts of the GEMM launch plan for every later call in the
+ * process, from any thread (0 = the planner's own choice for that part):
+ *   bn          dense tile width along the weights: 128, 192, 224 or 256 (linear scales;
+ *               NVFP4_SF_TILED accepts 128 and 256), other values ignored;
+ *   cluster     split-K CTAs per thread-block cluster, 1 ... 8;
+ *   groups      split-K clusters per output tile, reduced through the workspace (needs one);
+ *   band        output P tiles per rasterisation band;
+ *   grouped_bn  token tile width of the grouped GEMM: 32, 64, 128 or 256.
+ * The planner's choices need no override; results stay within the GEMM tolerance under any
+ * of them, and every override layout is deterministic. Negative values: NVFP4_ERR_INVALID_ARG.
+ */
+nvfp4_status nvfp4_set_plan_override(int32_t bn, int32_t cluster, int32_t groups, int32_t band,
+                                     int32_t grouped_bn);
 
 /*
  * Elementwise conversions used by the quantiser, exposed so that they can be checked

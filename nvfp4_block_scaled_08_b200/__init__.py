@@ -29,7 +29,7 @@ from . import _build
 
 __all__ = [
     "Nvfp4Error", "load", "global_scale", "quantize", "quantize_dynamic", "alpha", "gemm", "gemm_workspace_size",
-    "gemm_noalloc",
+    "gemm_noalloc", "plan_override",
     "make_workspace", "grouped_gemm", "round_e4m3", "round_e2m1", "last_device_error",
     "STATUS",
 ]
@@ -72,6 +72,7 @@ SIGNATURES = {
     "nvfp4_grouped_gemm_workspace_size": (_SZ, [_I32, _I64, _I64, _I64]),
     "nvfp4_grouped_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
                                           _SZ, _P]),
+    "nvfp4_set_plan_override": (ctypes.c_int, [_I32, _I32, _I32, _I32, _I32]),
     "nvfp4_round_e4m3": (ctypes.c_int, [_P, _I64, _P, _P]),
     "nvfp4_round_e2m1": (ctypes.c_int, [_P, _I64, _P, _P]),
     "nvfp4_last_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -276,6 +277,22 @@ def grouped_gemm(Aq, sfA, Bq, sfB, alphas, offsets, out=None, stream=None) -> to
         _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alphas), _ptr(offsets), E, rows, N, K,
         _ptr(out), None, 0, _stream(stream)))
     return out
+
+
+class plan_override:
+    """Context manager forcing parts of the GEMM launch plan (tuning and tests only):
+    ``with plan_override(cluster=2, groups=3): ...``; the planner's choices return on exit."""
+
+    def __init__(self, bn=0, cluster=0, groups=0, band=0, grouped_bn=0):
+        self.values = (bn, cluster, groups, band, grouped_bn)
+
+    def __enter__(self):
+        _check("nvfp4_set_plan_override", load().nvfp4_set_plan_override(*self.values))
+        return self
+
+    def __exit__(self, *exc):
+        _check("nvfp4_set_plan_override", load().nvfp4_set_plan_override(0, 0, 0, 0, 0))
+        return False
 
 
 # ------------------------------------------------------------------ conversions and errors

@@ -100,9 +100,20 @@ nvfp4_status from_cuda(cudaError_t e)
     return NVFP4_ERR_CUDA;
 }
 
-// Shape and pointer checks shared by the GEMMs; no CUDA call.
 nvfp4_status check_gemm_common(const void* A, const void* sfA, const void* B, const void* sfB,
                                const void* alpha, const void* out, int64_t N, int64_t K)
+{
+    return static_cast<nvfp4_status>(nvfp4::check_gemm_args(A, sfA, B, sfB, alpha, out, N, K));
+}
+
+}  // namespace
+
+namespace nvfp4 {
+
+// Shape and pointer checks shared by every GEMM entry point (also nvfp4_gemm_noalloc); no
+// CUDA call.
+int check_gemm_args(const void* A, const void* sfA, const void* B, const void* sfB,
+                    const void* alpha, const void* out, int64_t N, int64_t K)
 {
     if (!A || !sfA || !B || !sfB || !alpha || !out) return NVFP4_ERR_INVALID_ARG;
     if (K <= 0 || K % 256 != 0 || K > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -113,7 +124,7 @@ nvfp4_status check_gemm_common(const void* A, const void* sfA, const void* B, co
     return NVFP4_OK;
 }
 
-}  // namespace
+}  // namespace nvfp4
 
 namespace nvfp4 {
 
@@ -327,6 +338,14 @@ nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint
     cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
     if (enc_failed) return NVFP4_ERR_CUDA;
     return from_cuda(e);
+}
+
+nvfp4_status nvfp4_set_plan_override(int32_t bn, int32_t cluster, int32_t groups, int32_t band,
+                                     int32_t grouped_bn)
+{
+    if (bn < 0 || cluster < 0 || groups < 0 || band < 0 || grouped_bn < 0) return NVFP4_ERR_INVALID_ARG;
+    nvfp4::set_plan_override(bn, cluster, groups, band, grouped_bn);
+    return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_round_e4m3(const float* x, int64_t n, uint8_t* out, cudaStream_t stream)

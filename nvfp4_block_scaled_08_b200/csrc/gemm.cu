@@ -6,8 +6,7 @@
 
 #include <algorithm>
 #include <array>
-#include <cstdio>
-#include <cstdlib>
+#include <atomic>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -19,11 +18,18 @@ namespace nvfp4 {
 
 // ------------------------------------------------------------------ planning
 
-static int env_int(const char* name, int dflt)
+// Process-wide overrides of the planner's choices (nvfp4_set_plan_override; 0 = planner).
+// Plain atomics: a GEMM call reads them without a lock or a string look-up.
+static std::atomic<int> g_force_bn{0}, g_force_cluster{0}, g_force_groups{0}, g_force_band{0},
+    g_force_grouped_bn{0};
+
+void set_plan_override(int bn, int cluster, int groups, int band, int grouped_bn)
 {
-    const char* v = std::getenv(name);
-    if (!v || !*v) return dflt;
-    return std::atoi(v);
+    g_force_bn.store(bn, std::memory_order_relaxed);
+    g_force_cluster.store(cluster, std::memory_order_relaxed);
+    g_force_groups.store(groups, std::memory_order_relaxed);
+    g_force_band.store(band, std::memory_order_relaxed);
+    g_force_grouped_bn.store(grouped_bn, std::memory_order_relaxed);
 }
 
 static int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
@@ -42,7 +48,8 @@ static int max_active_clusters(int cs);
 //    over distributed shared memory; the largest cluster whose clusters all run in one
 //    wave is taken. Layouts with `groups` > 1 clusters per tile, which meet in the
 //    workspace, are available through the overrides (and nvfp4_gemm_noalloc's scratch).
-// NVFP4_BN, NVFP4_CLUSTER and NVFP4_GROUPS override the choice (tuning only).
+// nvfp4_set_plan_override can force the tile width, cluster size, groups and band (tuning
+// and tests only).
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int num_sms)
 {
     GemmPlan p;
@@ -63,7 +70,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
         // too few 256-wide tiles to fill the GPU: split-K follows, and 128-wide tiles halve
         // the partial tile each CTA hands over (and the splits needed)
         if (p.bn == 256 && t256 * 4 < num_sms * 3 && nk >= 2) p.bn = 128;
-        const int force = env_int("NVFP4_BN", 0);
+        const int force = g_force_bn.load(std::memory_order_relaxed);
         if (force == 128 || force == 192 || force == 224 || force == 256) p.bn = force;
         p.q_tiles = ceil_div(N, p.bn);
     }
@@ -77,7 +84,8 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
             if (tiles <= max_active_clusters(c)) { cs = c; break; }
         }
     }
-    const int fc = env_int("NVFP4_CLUSTER", 0), fg = env_int("NVFP4_GROUPS", 0);
+    const int fc = g_force_cluster.load(std::memory_order_relaxed);
+    const int fg = g_force_groups.load(std::memory_order_relaxed);
     if (fc > 0 || fg > 0) {
         cs = std::max(1, std::min(fc > 0 ? fc : cs, 8));
         g = std::max(1, fg > 0 ? fg : g);
@@ -92,7 +100,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
     const double packed_bytes = static_cast<double>(M + N) * static_cast<double>(K) * 0.5;
     p.band = packed_bytes <= 80e6 ? p.p_tiles : std::max(1, std::min(p.p_tiles, 16));
     {
-        const int fb = env_int("NVFP4_BAND", 0);
+        const int fb = g_force_band.load(std::memory_order_relaxed);
         if (fb > 0) p.band = std::min(p.p_tiles, fb);
     }
     p.cluster = cs;
@@ -105,11 +113,6 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
         p.ws_counter_bytes = ((static_cast<size_t>(tiles) * cs * 4 + 255) / 256) * 256;
         p.ws_bytes = p.ws_counter_bytes + static_cast<size_t>(tiles) * g * 128 * p.bn * sizeof(float);
     }
-    if (env_int("NVFP4_DEBUG", 0))
-        std::fprintf(stderr, "nvfp4 plan M=%lld N=%lld K=%lld: bn=%d swap=%d tiles=%d cluster=%d groups=%d "
-                     "grid=%d ws=%zu (max active clusters: 2:%d 4:%d 8:%d)\n",
-                     (long long)M, (long long)N, (long long)K, p.bn, (int)p.swap, tiles, cs, g, p.grid,
-                     p.ws_bytes, max_active_clusters(2), max_active_clusters(4), max_active_clusters(8));
     return p;
 }
 
@@ -123,7 +126,7 @@ GemmPlan plan_grouped(int32_t E, int64_t total_rows, int64_t N, int64_t K, int n
     p.swap = true;
     const int64_t avg = E > 0 ? total_rows / E : 0;
     p.bn = avg <= 24 ? 32 : avg <= 48 ? 64 : avg <= 96 ? 128 : 256;
-    const int force = env_int("NVFP4_GROUPED_BN", 0);
+    const int force = g_force_grouped_bn.load(std::memory_order_relaxed);
     if (force == 32 || force == 64 || force == 128 || force == 256) p.bn = force;
     p.p_tiles = ceil_div(N, 128);
     p.splits = 1;

@@ -48,6 +48,8 @@ struct GemmPlan {
 // needs none.
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int num_sms);
 GemmPlan plan_grouped(int32_t E, int64_t total_rows, int64_t N, int64_t K, int num_sms);
+// Forces planner choices for later calls (0 = the planner's own); nvfp4_set_plan_override.
+void set_plan_override(int bn, int cluster, int groups, int band, int grouped_bn);
 
 struct GemmLaunch {
     const uint8_t* A; const uint8_t* sfA; const uint8_t* B; const uint8_t* sfB;
@@ -62,6 +64,11 @@ struct GemmLaunch {
 // api.cu: nvfp4_status of the current device's checks; fills the SM count and the device
 // error word on success.
 int query_current_device(int* num_sms, unsigned** err_word);
+
+// api.cu: nvfp4_status of the pointer and shape checks every GEMM entry point applies (null
+// pointers, K % 256, N % 8, sizes below 2^31, 16-byte alignment, alpha 4-byte aligned).
+int check_gemm_args(const void* A, const void* sfA, const void* B, const void* sfB,
+                    const void* alpha, const void* out, int64_t N, int64_t K);
 
 // Returns cudaSuccess or the first CUDA error; *encode_failed is set if a TMA descriptor
 // could not be encoded.

@@ -26,27 +26,56 @@ static __device__ __align__(256) uint8_t g_nvfp4_noalloc_scratch[kNoallocScratch
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices];   // device address of the array, per device (set-up once)
+// Device address of the array per device, and the CUDA context it was looked up in. The
+// module (and with it the array) is loaded once per context: after the primary context is
+// released and created again it may sit at another address, so a change of context repeats
+// the look-up.
+void* g_scratch_ptr[kMaxDevices];
+void* g_scratch_ctx[kMaxDevices];
+
+using CtxGetCurrentFn = int (*)(void**);   // cuCtxGetCurrent(CUcontext*) -> CUresult
+
+CtxGetCurrentFn ctx_get_current()
+{
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
 
 // In host code `g_nvfp4_noalloc_scratch` names a host-side stand-in, not device memory;
 // the device address must come from cudaGetSymbolAddress, taken with the device current.
+// Set-up: the first call on a device (and the first after its context changed) looks it up.
+// A host thread that has made no CUDA call yet has no context bound; the look-up binds the
+// device's primary context to it, and the context is read again afterwards.
 nvfp4_status scratch_address(int dev, void** out)
 {
+    CtxGetCurrentFn get = ctx_get_current();
+    if (!get) return NVFP4_ERR_CUDA;
+    void* ctx = nullptr;
+    if (get(&ctx) != 0) return NVFP4_ERR_CUDA;
     std::lock_guard<std::mutex> g(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (ctx == nullptr || !g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_nvfp4_noalloc_scratch);
         if (e != cudaSuccess || p == nullptr) {
             cudaGetLastError();
             return NVFP4_ERR_CUDA;
         }
+        if (get(&ctx) != 0 || ctx == nullptr) return NVFP4_ERR_CUDA;
         g_scratch_ptr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_ptr[dev];
     return NVFP4_OK;
 }
-
-inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -58,13 +87,11 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint
 {
     if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return NVFP4_OK;
-    if (!A || !sfA || !B || !sfB || !alpha || !out) return NVFP4_ERR_INVALID_ARG;
     constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
-    if (K % 256 != 0 || N % 8 != 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
-        return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(A) || !aligned16(sfA) || !aligned16(B) || !aligned16(sfB) || !aligned16(out) ||
-        (reinterpret_cast<uintptr_t>(alpha) & 3u) != 0)
-        return NVFP4_ERR_MISALIGNED;
+    if (M > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    // the same pointer, shape and alignment checks as nvfp4_gemm
+    const int chk = nvfp4::check_gemm_args(A, sfA, B, sfB, alpha, out, N, K);
+    if (chk != NVFP4_OK) return static_cast<nvfp4_status>(chk);
 
     int num_sms = 0;
     unsigned* err_word = nullptr;

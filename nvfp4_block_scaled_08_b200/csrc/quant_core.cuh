@@ -1,6 +1,6 @@
-// quant_core.cuh -- the NVFP4 quantisation arithmetic shared by the quantiser kernels and the
-// GEMM's fused activation-quantisation phase: format conversions, the flat vector view of a
-// [rows, K] tensor, the amax and quantisation sweeps and the block reductions.
+// quant_core.cuh -- the NVFP4 quantisation arithmetic of the quantiser kernels: format
+// conversions, the flat vector view of a [rows, K] tensor, the amax and quantisation sweeps
+// and the block reductions.
 //
 // Format: packed e2m1 values two per byte with one float8_e4m3fn scale per 16 K-elements
 // ("When a Benchmark Crashes", section "Input Knowledge Required", item 3; block_size=16

@@ -1,7 +1,7 @@
 // quantize.cu -- NVFP4 two-level quantisation kernels for sm_100a: per-tensor global scale
 // (amax reduction), per-16-element block scale (e4m3) and element codes (e2m1), plus the
 // GEMM alpha and the elementwise conversions exposed for exhaustive checking. The
-// arithmetic itself lives in quant_core.cuh (shared with the GEMM's fused phase).
+// arithmetic itself lives in quant_core.cuh.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -9,7 +9,6 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -449,9 +448,7 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
     const int64_t nv = rows * vpr;                       // < 2^31 (checked by the caller)
     const VecIndex ix = make_vec_index(vpr, ldx, K);
     const SfOut sf = make_sf_out(sf_ptr, sf_tiled, ix, K);
-    int64_t cluster_max = kClusterQuantizeMaxBytes;
-    if (const char* v = std::getenv("NVFP4_QCLUSTER_MAX_KB")) cluster_max = std::atoll(v) << 10;  // tuning only
-    const int ccs = bytes <= cluster_max ? quantize_cluster_size<T>() : 0;
+    const int ccs = bytes <= kClusterQuantizeMaxBytes ? quantize_cluster_size<T>() : 0;
     if (ccs > 0) {
         const int cs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ccs, (nv + 511) / 512)));
         const int64_t chunk = round_up((nv + cs - 1) / cs, 32);

@@ -66,6 +66,31 @@ def test_gemm_host_validation(lib):
     assert _gemm(lib, ws=0x7010, ws_bytes=1 << 20) == 3   # workspace needs 256-byte alignment
 
 
+def _noalloc(lib, A=0x1000, sfA=0x2000, B=0x3000, sfB=0x4000, alpha=0x5000, out=0x6000,
+             M=16, N=768, K=6144):
+    return lib.nvfp4_gemm_noalloc(A, sfA, B, sfB, alpha, out, M, N, K, None)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(M=0), dict(N=0), dict(M=-1), dict(K=-256), dict(A=None), dict(sfA=None), dict(B=None),
+    dict(sfB=None), dict(alpha=None), dict(out=None), dict(K=100), dict(K=0), dict(N=12),
+    dict(M=1 << 31), dict(N=1 << 31), dict(A=0x1001), dict(sfA=0x2004), dict(B=0x3008),
+    dict(sfB=0x4008), dict(out=0x6002), dict(alpha=0x5002),
+], ids=lambda d: ",".join(f"{k}={v}" for k, v in d.items()))
+def test_noalloc_host_validation_matches_gemm(lib, bad):
+    """The allocation-free entry point rejects every bad argument with the same status as
+    nvfp4_gemm, before any CUDA call."""
+    assert _noalloc(lib, **bad) == _gemm(lib, **bad)
+
+
+def test_plan_override_validation(lib):
+    assert lib.nvfp4_set_plan_override(-1, 0, 0, 0, 0) == 1
+    assert lib.nvfp4_set_plan_override(0, 0, -2, 0, 0) == 1
+    assert lib.nvfp4_set_plan_override(0, 0, 0, 0, 0) == 0
+    with nv.plan_override(cluster=2, groups=3):
+        pass
+
+
 def test_grouped_host_validation(lib):
     f = lib.nvfp4_grouped_gemm
     args = dict(A=0x1000, sfA=0x2000, B=0x3000, sfB=0x4000, alpha=0x5000, off=0x8000,

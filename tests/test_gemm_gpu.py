@@ -145,10 +145,13 @@ def test_one_hot_rows_bit_exact(cuda_device, M, N, K):
 
 
 @pytest.mark.parametrize("cluster,groups", [(1, 1), (8, 1), (2, 6), (1, 12)])
-def test_split_k_deterministic_and_within_tolerance(cuda_device, monkeypatch, cluster, groups):
+def test_split_k_deterministic_and_within_tolerance(cuda_device, cluster, groups):
     c = workloads.attn_proj_cases()[0]          # M = 16: the most split-heavy shape
-    monkeypatch.setenv("NVFP4_CLUSTER", str(cluster))
-    monkeypatch.setenv("NVFP4_GROUPS", str(groups))
+    with nv.plan_override(cluster=cluster, groups=groups):
+        _split_k_deterministic(cuda_device, c, cluster, groups)
+
+
+def _split_k_deterministic(cuda_device, c, cluster, groups):
     a, b = c.a(), c.b()
     d = cuda_device
     Aq, sfA, gsA = gpu_quantize(a, d)
@@ -167,14 +170,13 @@ def test_split_k_deterministic_and_within_tolerance(cuda_device, monkeypatch, cl
 @pytest.mark.parametrize("cluster,groups", [(2, 1), (3, 1), (4, 1), (8, 1), (2, 3), (3, 2), (1, 5)])
 @pytest.mark.parametrize("M,N,K", [(16, 768, 6144), (256, 768, 6144), (130, 776, 2560),
                                    (40, 264, 4096)])
-def test_split_k_layouts(cuda_device, monkeypatch, cluster, groups, M, N, K):
+def test_split_k_layouts(cuda_device, cluster, groups, M, N, K):
     """Every cluster / group layout of split-K (distributed-shared-memory reduction inside
     a cluster, workspace reduction across clusters) against the oracle."""
-    monkeypatch.setenv("NVFP4_CLUSTER", str(cluster))
-    monkeypatch.setenv("NVFP4_GROUPS", str(groups))
     a = workloads.normal(M, K, 1.0, M + 3 * N)
     b = workloads.normal(N, K, 0.02, N + 5 * K)
-    run_case(cuda_device, a, b, use_ws=True)
+    with nv.plan_override(cluster=cluster, groups=groups):
+        run_case(cuda_device, a, b, use_ws=True)
 
 
 def bf16_bits_tensor(t):
@@ -196,9 +198,12 @@ def test_transposed_product_agrees(cuda_device):
     check_within_tolerance(o2.t().contiguous(), v, S, alo, "(B A^T)^T")
 
 
-def test_workspace_too_small_is_rejected(cuda_device, monkeypatch):
-    monkeypatch.setenv("NVFP4_CLUSTER", "2")
-    monkeypatch.setenv("NVFP4_GROUPS", "4")
+def test_workspace_too_small_is_rejected(cuda_device):
+    with nv.plan_override(cluster=2, groups=4):
+        _workspace_too_small(cuda_device)
+
+
+def _workspace_too_small(cuda_device):
     n = nv.gemm_workspace_size(16, 768, 6144)
     assert n > 0
     d = cuda_device

@@ -6,11 +6,14 @@ that hand a kernel no workspace argument, and latency-critical paths that cannot
 cudaMalloc / cudaFree that may synchronise the device. The entry point takes its split-K
 scratch from a fixed array inside the library instead of a workspace.
 
-Checked here, through the C ABI: on shapes that use split-K scratch, two calls in a row
-give the same output as nvfp4_gemm within the GEMM tolerance (2^-7 |alpha| sum|a b| +
-1e-6 against the CPU oracle), and a shape whose scratch would exceed the fixed array is
-rejected with NVFP4_ERR_WORKSPACE. This file is collected last so that a failure here
-cannot hide a failure elsewhere; it also passes when run on its own in a fresh process.
+Checked here, through the C ABI: two calls in a row give the same output as nvfp4_gemm
+within the GEMM tolerance (2^-7 |alpha| sum|a b| + 1e-6 against the CPU oracle), both with
+the default plan (which splits K inside one thread-block cluster and needs no scratch) and
+with a plan forced to reduce split-K partials across several clusters, which goes through
+the fixed scratch array and its tile counters; and a shape whose scratch would exceed the
+fixed array is rejected with NVFP4_ERR_WORKSPACE. This file is collected last so that a
+failure here cannot hide a failure elsewhere; it also passes when run on its own in a fresh
+process.
 """
 import numpy as np
 import pytest
@@ -35,14 +38,21 @@ def _call_noalloc(lib, Aq, sfA, Bq, sfB, al, out, M, N, K):
 @pytest.mark.parametrize("case", workloads.attn_proj_cases()[:3] + workloads.moe_expert_cases()[1:2],
                          ids=lambda c: c.name)
 @pytest.mark.parametrize("layout", ["planned", "workspace"])
-def test_noalloc_matches_gemm_on_two_calls(cuda_device, case, layout, monkeypatch):
-    d = cuda_device
-    M, N, K = case.M, case.N, case.K
+def test_noalloc_matches_gemm_on_two_calls(cuda_device, case, layout):
     if layout == "workspace":
         # split-K across several clusters per tile, so the partials go through the scratch
-        monkeypatch.setenv("NVFP4_CLUSTER", "2")
-        monkeypatch.setenv("NVFP4_GROUPS", "3")
-        assert nv.gemm_workspace_size(M, N, K) > 0, "shape must exercise the split-K scratch"
+        with nv.plan_override(cluster=2, groups=3):
+            assert nv.gemm_workspace_size(case.M, case.N, case.K) > 0, "must use the scratch"
+            _two_calls(cuda_device, case)
+    else:
+        # the default plan: no scratch (nothing for the fixed array to hold)
+        assert nv.gemm_workspace_size(case.M, case.N, case.K) == 0
+        _two_calls(cuda_device, case)
+
+
+def _two_calls(cuda_device, case):
+    d = cuda_device
+    M, N, K = case.M, case.N, case.K
     a, b = case.a(), case.b()
     Aq, sfA, gsA = gpu_quantize(a, d)
     Bq, sfB, gsB = gpu_quantize(b, d)
@@ -69,11 +79,14 @@ def test_noalloc_matches_gemm_on_two_calls(cuda_device, case, layout, monkeypatc
         check_within_tolerance(out, v, S, alo, f"{case.name} call {call}")
 
 
-def test_noalloc_rejects_scratch_beyond_the_fixed_array(cuda_device, monkeypatch):
-    d = cuda_device
+def test_noalloc_rejects_scratch_beyond_the_fixed_array(cuda_device):
     # force 24 cluster groups per tile on 1024 x 768 x 6144: 48 tiles x 24 x 64 KB > 16 MiB
-    monkeypatch.setenv("NVFP4_CLUSTER", "1")
-    monkeypatch.setenv("NVFP4_GROUPS", "24")
+    with nv.plan_override(cluster=1, groups=24):
+        _rejects(cuda_device)
+
+
+def _rejects(cuda_device):
+    d = cuda_device
     M, N, K = 1024, 768, 6144
     Aq = torch.zeros(M, K // 2, dtype=torch.uint8, device=d)
     sfA = torch.zeros(M, K // 16, dtype=torch.uint8, device=d)
