@@ -1,47 +1,54 @@
 #!/usr/bin/env python
 """Benchmark of the NVFP4 block-scaled GEMM hot path on B200.
 
-Metric: NVFP4 GEMM TFLOP/s (whole step) and the fraction of the B200 roofline per
-M x N x K. Workload (default): the attention-projection sweep N=768, K=6144,
-M in {16, 64, 256, 1024}, A ~ N(0,1) fp32 activations, B ~ N(0,0.02) weights quantised
-once to NVFP4 outside the timed region. One step = for every M: per-tensor global scale
-of A, alpha = 1/(gsA gsB), NVFP4 quantisation of A, block-scaled GEMM -> bf16.
+Metric: NVFP4 GEMM TFLOP/s and the fraction of the B200 roofline per M x N x K.
 
-Timing: the step is captured as a CUDA graph of its eight kernels, nothing else, so each
-kernel launches early behind the one before it (programmatic dependent launch). A second
-graph with event-record nodes between the kernels is replayed afterwards, untimed, for the
-per-shape breakdown (`per_shape`; the event nodes cost each kernel its early launch).
-Inputs are larger than L2: 8 independent input sets of the sweep (activations, weights,
-outputs; 41 MiB each, 327 MiB in all, "layers" with different seeds) are replayed in
-rotation, so each step's data was last touched 7 steps (about 286 MiB) earlier and comes
-from HBM. W warm-up replays, then exactly K steps back to back between one pair of CUDA
-events (whole rotations from one graph of all 8 sets, the remainder from single-set
-graphs), bracketed by a barrier and a device synchronise; step time = event time / K, max
-over ranks. --flush instead flushes L2 before every step (a 512 MB write, then a 256 MB
-read, which also evicts kernel code and tensor maps) and brackets each replay on its own,
-the flush outside. SM clocks and throttle reasons are polled through NVML during the timed
-bracket.
+Headline workload (the largest single-GPU configuration): the compute-bound plateau
+M = N = K = 16384, A and B ~ U(-1, 1) fp32. The weights B are quantised to NVFP4 once,
+outside the timed region (scales re-laid out in the tiled layout the tensor cores read).
+One step = quantise the fp32 activations A (global scale, alpha = 1 / (gsA gsB), e4m3
+block scales, e2m1 codes: one launch) and the block-scaled GEMM -> bf16 out [16384, 16384]:
+two kernels, captured once as a CUDA graph with an event node between them, so that the
+GEMM's own duration is measured inside the timed region. Inputs are larger than L2 (A alone
+is 1 GiB of fp32), so every step reads them from HBM. W warm-up replays, then exactly K
+steps back to back between one pair of CUDA events, bracketed by a barrier and a device
+synchronise; step time = event time / K, max over ranks. SM clocks and throttle reasons are
+polled through NVML during the timed bracket.
 
-e2e: the same metric through the public Python API called eagerly per step, with the
-activations copied from pinned host memory and the outputs copied back inside the timed
-region. The input copies run on a second stream into two alternating device buffers, so a
-step's copy overlaps the previous step's kernels; the outputs are checked against the graph's.
+e2e: the same step through the public Python API, with A copied in from pinned host memory
+and the bf16 output copied back inside the timed region every step; the input copies run on
+a second stream into two alternating device buffers (so a step's copy overlaps the previous
+step's kernels), and the outputs are checked bit for bit against the graph's.
 
-context (rank 0, after the timed step, --no-context skips it): the compute-bound 8192^3 GEMM
-against the FP4 tensor peak, and 512 x 2048 x 6144 beside a bf16 torch matmul of that shape,
-both with the tiled scale layout.
+per_config (rank 0, after the timed step; --no-per-config skips it): every workload of the
+five configurations -- 128 x 256 x 512; the attention-projection sweep N=768, K=6144,
+M in {16, 64, 256, 1024}; the MoE expert shapes (up N=2048 K=6144, down N=6144 K=2048,
+M in {16 .. 1024}); the grouped MoE GEMM (256 experts, top-8 of T in {512, 4096} tokens,
+gate_up N=4096 K=6144 and down N=6144 K=2048); and the plateau 4096^3 / 8192^3 / 16384^3 plus
+512 x 2048 x 6144 beside a bf16 torch matmul. Each shape is timed from CUDA graphs of
+back-to-back launches (median of 5 replays): the GEMM alone, the activation quantiser alone
+and the two as one step. Shapes whose data is smaller than L2 rotate through enough
+independent copies (at least 4 x L2 in all) that every launch reads from HBM.
 
---impl reference: the CPU oracle as it stands (test infrastructure), on a bounded sample
-of the same workload per step, on this machine's host cores.
+Rooflines: time = max(flops / P_fp4, bytes / BW), against two denominators: the B200
+specification (9 PFLOP/s dense FP4, 8 TB/s HBM3e; the targets are stated against these) and
+the peaks measured on this machine (MEASURED_PEAKS.json: HBM copy bandwidth; dense FP4 = the
+measured cuBLAS bf16 rate x 4, the nominal FP4 / BF16 ratio of B200).
 
-Multi-GPU (torchrun, --gpus N): independent replicas, one per GPU ("weak" scaling); the
-path has no exchange step on one GPU's worth of work, so no collective is used on the
-data path.
+cpu_baseline: the CPU oracle as it stands (test infrastructure), timed on this machine's
+host cores on a bounded row sample of the headline workload; per_config entries carry their
+own sample, extrapolated to the full shape and labelled so.
+
+--impl reference: the CPU oracle on a bounded sample of the headline workload per step.
+
+Multi-GPU (torchrun, --gpus N): independent replicas, one per GPU ("weak" scaling); the path
+has no exchange step on one GPU's worth of work, so no collective is used on the data path.
 """
 from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import platform
 import statistics
@@ -55,10 +62,12 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-N_ATTN, K_ATTN, M_SWEEP = 768, 6144, (16, 64, 256, 1024)
-FLUSH_BYTES = 512 << 20
-CLEAN_BYTES = 256 << 20
-FP4_PER_BF16 = 4.0     # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PF)
+METRIC = "NVFP4 GEMM TFLOPS and % of B200 FP4/HBM roofline per M x N x K"
+HEADLINE = "plateau M=N=K=16384"
+FP4_PER_BF16 = 4.0       # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PF)
+SPEC_FP4_TFLOPS = 9000.0  # B200 specification, dense FP4
+SPEC_HBM_GBS = 8000.0     # B200 specification, HBM3e
+ROTATE_L2_MULT = 4       # rotated copies span at least this many L2 sizes
 
 
 # ------------------------------------------------------------------ environment
@@ -101,14 +110,13 @@ def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> fl
     return flops_per_rank * world / (step_ms_max * 1e-3) / 1e12
 
 
-# DRAM traffic of the GEMM launches of one sweep (M = 16, 64, 256, 1024; tiled scales), from one
-# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, cold L2; the bf16 outputs stay in
-# L2 within a launch): 2802432 + 2954240 + 3596544 + 6251008 bytes; the capture command and its table are
-# in the committed ncu summary of these launches under profiles/. Valid only for the kernel
-# sources it was taken on (hash below); reported as null otherwise.
-GEMM_TRAFFIC_BYTES = 2802432 + 2954240 + 3596544 + 6251008
+# DRAM traffic of one 16384^3 GEMM launch (tiled scales): dram__bytes_read.sum +
+# dram__bytes_write.sum from one ncu capture of the full-size launch (one pass); the command
+# and the figures are in the committed ncu summary of the plateau under profiles/. Valid only
+# for the kernel sources it was taken on (hash below); reported as null otherwise.
+GEMM_TRAFFIC_BYTES = None
 GEMM_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "gemm.cu", "ptx.cuh", "internal.h")
-GEMM_TRAFFIC_SHA = "9dbe30d4e3215f45"
+GEMM_TRAFFIC_SHA = ""
 
 
 def _code_hash(files) -> str:
@@ -128,6 +136,8 @@ def _code_hash(files) -> str:
 
 def gemm_traffic():
     """The captured traffic, or None once the GEMM code differs from the captured one."""
+    if GEMM_TRAFFIC_BYTES is None:
+        return None
     return GEMM_TRAFFIC_BYTES if _code_hash(GEMM_TRAFFIC_SOURCES) == GEMM_TRAFFIC_SHA else None
 
 
@@ -223,447 +233,447 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ roofline model
 
-def gemm_bytes(M, N, K):
-    """Algorithmic HBM bytes of one GEMM: packed operands + scales once, bf16 out once."""
-    return (M + N) * K * (0.5 + 1.0 / 16.0) + 2.0 * M * N
+def gemm_bytes(M, N, K, experts=1):
+    """Algorithmic HBM bytes of one GEMM: packed operands + scales once (weights once per
+    expert touched), bf16 out once."""
+    return M * K * (0.5 + 1.0 / 16.0) + experts * N * K * (0.5 + 1.0 / 16.0) + 2.0 * M * N
 
 
-def quant_bytes(M, K):
-    """Algorithmic HBM bytes of quantising an fp32 [M, K]: read once, codes + scales out."""
-    return M * K * (4.0 + 0.5 + 1.0 / 16.0)
+def quant_bytes(M, K, in_bytes=4):
+    """Algorithmic HBM bytes of quantising an [M, K] tensor: read once, codes + scales out."""
+    return M * K * (in_bytes + 0.5 + 1.0 / 16.0)
 
 
-def roofline_us(flops, nbytes, peaks):
-    p_fp4 = peaks["bf16_tflops"] * FP4_PER_BF16 * 1e12
-    bw = peaks["hbm_gbs"] * 1e9
-    t_tc, t_mem = flops / p_fp4, nbytes / bw
-    return max(t_tc, t_mem) * 1e6, ("tensor" if t_tc >= t_mem else "hbm")
+def roofline(flops, nbytes, peaks):
+    """Roofline time (us) and bound, against the B200 specification and the measured peaks."""
+    out = {}
+    for tag, p_tf, bw in (("spec", SPEC_FP4_TFLOPS, SPEC_HBM_GBS),
+                          ("measured", peaks["bf16_tflops"] * FP4_PER_BF16, peaks["hbm_gbs"])):
+        t_tc, t_mem = flops / (p_tf * 1e12), nbytes / (bw * 1e9)
+        out[tag] = (max(t_tc, t_mem) * 1e6, "tensor" if t_tc >= t_mem else "hbm")
+    return out
 
 
-# ------------------------------------------------------------------ our implementation
-
-class AttnSweep:
-    """Resident inputs, outputs and workspaces of the attention-projection sweep."""
-
-    def __init__(self, dev, rank, set_index=0, tiled=True):
-        import nvfp4_block_scaled_08_b200 as nv
-        from nvfp4_block_scaled_08_b200 import workloads
-        self.nv = nv
-        self.dev = dev
-        cases = workloads.attn_proj_cases()
-        # set 0 is the canonical seeded case; the other sets (other "layers") differ only in
-        # their seeds
-        b = cases[0].b() if set_index == 0 else workloads.normal(
-            N_ATTN, K_ATTN, 0.02, cases[0].seed + 1 + 7919 * set_index)   # same weights for every M
-        bd = b.to(dev)
-        self.gsB = nv.global_scale(bd)
-        self.Bq, self.sfB = nv.quantize(bd, self.gsB)
-        self.tiled = tiled
-        if tiled:                   # weights' scales re-laid out once, outside any timing
-            self.sfB = nv.sf_tile(self.sfB)
-        del bd
-        self.items = []
-        for c in cases:
-            a_cpu = c.a() if set_index == 0 else workloads.normal(c.M, K_ATTN, 1.0, c.seed + 7919 * set_index)
-            it = {
-                "M": c.M, "a_cpu": a_cpu.pin_memory(),
-                "a": a_cpu.to(dev),
-                "gs": torch.empty(1, dtype=torch.float32, device=dev),
-                "alpha": torch.empty(1, dtype=torch.float32, device=dev),
-                "q": torch.empty(c.M, K_ATTN // 2, dtype=torch.uint8, device=dev),
-                "sf": torch.empty(nv.sf_bytes(c.M, K_ATTN, tiled), dtype=torch.uint8, device=dev),
-                "out": torch.empty(c.M, N_ATTN, dtype=torch.bfloat16, device=dev),
-                "out_host": torch.empty(c.M, N_ATTN, dtype=torch.bfloat16).pin_memory(),
-                "ws": nv.make_workspace(c.M, N_ATTN, K_ATTN, dev),
-            }
-            self.items.append(it)
-        self.flops = sum(2 * it["M"] * N_ATTN * K_ATTN for it in self.items)
-        self.launches_per_step = 2 * len(self.items)   # fused quantize, gemm
-
-    def step_one(self, it, stream=None):
-        """One M of the step: activations (fp32, resident) -> codes, scales, alpha -> bf16 out."""
-        self.run_one(it, stream)
-        self.gemm_one(it, stream)
-
-    def run_one(self, it, stream=None, a=None):
-        # global scale + alpha + NVFP4 quantisation of the activations: one launch
-        self.nv.quantize_dynamic(it["a"] if a is None else a, gs_other=self.gsB, gs=it["gs"], q=it["q"],
-                                 sf=it["sf"], alpha_out=it["alpha"], stream=stream, tiled=self.tiled)
-
-    def gemm_one(self, it, stream=None):
-        self.nv.gemm(it["q"], it["sf"], self.Bq, self.sfB, it["alpha"], out=it["out"],
-                     workspace=it["ws"], stream=stream, tiled=self.tiled)
-
-    def capture(self):
-        """Two CUDA graphs of the whole step: `graph`, the timed one, holds only the kernels
-        (so each GEMM keeps its programmatic dependency on the quantiser before it); `graph_ev`
-        adds event nodes around each kernel for the per-shape breakdown."""
-        self.ev = []
-        for it in self.items:
-            self.ev.append([torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)])
-        # run once eagerly so every lazily-initialised resource exists before capture
-        for it in self.items:
-            self.run_one(it)
-            self.gemm_one(it)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for it in self.items:
-                self.run_one(it)
-                self.gemm_one(it)
-        ge = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(ge):
-            for it, ev in zip(self.items, self.ev):
-                ev[0].record()
-                self.run_one(it)
-                ev[1].record()
-                self.gemm_one(it)
-                ev[2].record()
-        self.graph, self.graph_ev = g, ge
-        return g
-
-    def setup_e2e(self):
-        """A second device buffer for every activation tensor, and the events that order the
-        host copies (on their own stream) against the quantiser that reads them."""
-        for it in self.items:
-            it["a_dev"] = [it["a"], torch.empty_like(it["a"])]
-            it["ready"] = [torch.cuda.Event(), torch.cuda.Event()]
-            it["consumed"] = [torch.cuda.Event(), torch.cuda.Event()]
-
-    def e2e_step(self, step, stream, copy_stream):
-        """One step through the public API with host buffers. Every M's fp32 activations are
-        copied from pinned host memory on `copy_stream` into one of two device buffers
-        (alternating by step, so that the copy overlaps the previous step's kernels), then
-        quantised and multiplied on `stream`, and the bf16 output is copied back to pinned
-        host memory on `stream`."""
-        b = step & 1
-        for it in self.items:
-            with torch.cuda.stream(copy_stream):
-                copy_stream.wait_event(it["consumed"][b])     # step - 2 has read this buffer
-                it["a_dev"][b].copy_(it["a_cpu"], non_blocking=True)
-                it["ready"][b].record(copy_stream)
-            stream.wait_event(it["ready"][b])
-            self.run_one(it, stream, a=it["a_dev"][b])
-            it["consumed"][b].record(stream)
-            self.gemm_one(it, stream)
-            it["out_host"].copy_(it["out"], non_blocking=True)
-
-    @property
-    def h2d_bytes(self):
-        return sum(it["a_cpu"].numel() * 4 for it in self.items)
-
-    @property
-    def d2h_bytes(self):
-        return sum(it["out"].numel() * 2 for it in self.items)
+def frac_fields(flops, nbytes, us, peaks):
+    r = roofline(flops, nbytes, peaks)
+    return {"roofline_us_spec": round(r["spec"][0], 3), "bound": r["spec"][1],
+            "frac_of_spec": round(r["spec"][0] / us, 4),
+            "roofline_us_measured": round(r["measured"][0], 3),
+            "frac_of_measured": round(r["measured"][0] / us, 4)}
 
 
-def graph_time_us(fn, reps: int, iters: int = 5) -> float:
-    """Median device time of one call, from CUDA graphs of `reps` back-to-back calls."""
-    fn()
+# ------------------------------------------------------------------ timing helpers
+
+def l2_bytes(dev) -> int:
+    try:
+        return int(torch.cuda.get_device_properties(dev).L2_cache_size)
+    except Exception:
+        return 126 << 20
+
+
+def graph_time_us(calls, iters: int = 5, min_ms: float = 2.0) -> float:
+    """Median device time of one call from a CUDA graph of `calls` back to back (each a
+    zero-argument function launching on the current stream), repeated within the graph
+    until one replay takes at least min_ms."""
+    for c in calls:
+        c()
     torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for c in calls:
+        c()
+    e.record()
+    e.synchronize()
+    est_ms = max(s.elapsed_time(e), 1e-3)
+    reps = max(1, min(200, int(math.ceil(min_ms / est_ms))))
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for _ in range(reps):
-            fn()
+            for c in calls:
+                c()
+    g.replay()
+    torch.cuda.synchronize()
     ts = []
     for _ in range(iters):
-        s = torch.cuda.Event(enable_timing=True)
-        e = torch.cuda.Event(enable_timing=True)
         s.record()
         g.replay()
         e.record()
         e.synchronize()
-        ts.append(s.elapsed_time(e) * 1e3 / reps)
+        ts.append(s.elapsed_time(e) * 1e3 / (reps * len(calls)))
     del g
     return statistics.median(ts)
 
 
-def context_gemms(dev, peaks):
-    """Context outside the timed step, from the compute-bound configurations: the 8192^3
-    NVFP4 GEMM (uniform(-1, 1) inputs, quantised on the device) against the FP4 tensor peak,
-    and the 512 x 2048 x 6144 NVFP4 GEMM beside a bf16 torch matmul of the same shape."""
+def n_copies(set_bytes: float, dev, cap: int = 256) -> int:
+    """Independent copies to rotate so that together they span ROTATE_L2_MULT x L2."""
+    need = ROTATE_L2_MULT * l2_bytes(dev)
+    return max(1, min(cap, int(math.ceil(need / max(set_bytes, 1.0)))))
+
+
+# ------------------------------------------------------------------ our implementation
+
+class DenseStep:
+    """One dense workload on the device: fp32 activations A [M, K] and weights B [N, K]
+    quantised once (tiled scales). step = quantize_dynamic(A) (global scale, alpha, codes,
+    tiled scales) + gemm -> bf16 out. `copies` independent copies of everything (distinct
+    memory, same values) are rotated so that the data of each launch comes from HBM."""
+
+    def __init__(self, nv, M, N, K, a_cpu, b_cpu, dev, copies=None):
+        self.nv, self.M, self.N, self.K = nv, M, N, K
+        bd = b_cpu.to(dev)
+        gsB = nv.global_scale(bd)
+        Bq, sfB = nv.quantize(bd, gsB)
+        sfB = nv.sf_tile(sfB)
+        del bd
+        ad = a_cpu.to(dev)
+        self.set_bytes = (ad.numel() * 4 + M * K // 2 + nv.sf_bytes(M, K, True) + Bq.numel()
+                          + sfB.numel() + 2 * M * N)
+        n = copies if copies is not None else n_copies(self.set_bytes, dev)
+        self.sets = []
+        for i in range(n):
+            self.sets.append({
+                "a": ad if i == 0 else ad.clone(),
+                "Bq": Bq if i == 0 else Bq.clone(), "sfB": sfB if i == 0 else sfB.clone(),
+                "gsB": gsB, "gs": torch.empty(1, dtype=torch.float32, device=dev),
+                "alpha": torch.empty(1, dtype=torch.float32, device=dev),
+                "q": torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+                "sf": torch.empty(nv.sf_bytes(M, K, True), dtype=torch.uint8, device=dev),
+                "out": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                "ws": nv.make_workspace(M, N, K, dev),
+            })
+        self.flops = 2.0 * M * N * K
+
+    def quant(self, s, stream=None, a=None):
+        self.nv.quantize_dynamic(s["a"] if a is None else a, gs_other=s["gsB"], gs=s["gs"], q=s["q"],
+                                 sf=s["sf"], alpha_out=s["alpha"], stream=stream, tiled=True)
+
+    def gemm(self, s, stream=None):
+        self.nv.gemm(s["q"], s["sf"], s["Bq"], s["sfB"], s["alpha"], out=s["out"], workspace=s["ws"],
+                     stream=stream, tiled=True)
+
+    def step(self, s, stream=None):
+        self.quant(s, stream)
+        self.gemm(s, stream)
+
+    def time_all(self):
+        """(gemm_us, quant_us, step_us) per launch / step, each from its own graph."""
+        self.step(self.sets[0])
+        g = graph_time_us([lambda s=s: self.gemm(s) for s in self.sets])
+        q = graph_time_us([lambda s=s: self.quant(s) for s in self.sets])
+        st = graph_time_us([lambda s=s: self.step(s) for s in self.sets])
+        return g, q, st
+
+
+class GroupedStep:
+    """The grouped MoE GEMM: E experts' weights [E, N, K] drawn on the device and quantised
+    once per expert (linear scales), expert-sorted fp32 activations [rows, K];
+    step = quantize_dynamic(A) (one global scale, alpha[e] against every expert's scale) +
+    grouped_gemm -> bf16 out. The weights (1.8 - 3.6 GB) are far larger than L2."""
+
+    _weights = {}     # (N, K, weight seed) -> quantised weights, shared by both token counts
+
+    @classmethod
+    def weights(cls, nv, case, dev):
+        key = (case.N, case.K, case.weight_seed)
+        if key not in cls._weights:
+            E, N, K = case.num_experts, case.N, case.K
+            Bq = torch.empty(E, N, K // 2, dtype=torch.uint8, device=dev)
+            sfB = torch.empty(E, N, K // 16, dtype=torch.uint8, device=dev)
+            gsB = torch.empty(E, dtype=torch.float32, device=dev)
+            for e in range(E):
+                w = case.b(e, device=dev)
+                nv.global_scale(w, out=gsB[e:e + 1])
+                nv.quantize(w, gsB[e:e + 1], q=Bq[e], sf=sfB[e])
+                del w
+            cls._weights = {key: (Bq, sfB, gsB)}      # keep one projection's weights at a time
+        return cls._weights[key]
+
+    def __init__(self, nv, case, dev):
+        self.nv, self.case = nv, case
+        r = case.route()
+        self.rows, E, N, K = r.rows, case.num_experts, case.N, case.K
+        self.E, self.N, self.K = E, N, K
+        self.offsets = r.offsets.to(dev)
+        self.a = case.a(self.rows).to(dev)
+        self.Bq, self.sfB, self.gsB = self.weights(nv, case, dev)
+        self.gs = torch.empty(1, dtype=torch.float32, device=dev)
+        self.alpha = torch.empty(E, dtype=torch.float32, device=dev)
+        self.q = torch.empty(self.rows, K // 2, dtype=torch.uint8, device=dev)
+        self.sf = torch.empty(self.rows, K // 16, dtype=torch.uint8, device=dev)
+        self.out = torch.empty(self.rows, N, dtype=torch.bfloat16, device=dev)
+        self.flops = 2.0 * self.rows * N * K
+        counts = (r.offsets[1:] - r.offsets[:-1])
+        self.touched = int((counts > 0).sum())
+        self.rows_per_expert = (int(counts.min()), int(counts.max()))
+
+    def quant(self):
+        self.nv.quantize_dynamic(self.a, gs_other=self.gsB, gs=self.gs, q=self.q, sf=self.sf,
+                                 alpha_out=self.alpha)
+
+    def gemm(self):
+        self.nv.grouped_gemm(self.q, self.sf, self.Bq, self.sfB, self.alpha, self.offsets, out=self.out)
+
+    def time_all(self):
+        self.quant()
+        g = graph_time_us([self.gemm])
+        q = graph_time_us([self.quant])
+        st = graph_time_us([lambda: (self.quant(), self.gemm())])
+        return g, q, st
+
+
+def dense_entry(name, M, N, K, g_us, q_us, st_us, copies, set_bytes, peaks):
+    fl = 2.0 * M * N * K
+    by = gemm_bytes(M, N, K)
+    e = {"name": name, "M": M, "N": N, "K": K, "gemm_us": round(g_us, 3),
+         "gemm_tflops": round(fl / (g_us * 1e-6) / 1e12, 1)}
+    e.update(frac_fields(fl, by, g_us, peaks))
+    e.update({"quantize_us": round(q_us, 3),
+              "quantize_gbs": round(quant_bytes(M, K) / (q_us * 1e-6) / 1e9, 1),
+              "quantize_frac_of_spec_hbm": round(quant_bytes(M, K) / (q_us * 1e-6) / 1e9 / SPEC_HBM_GBS, 4),
+              "step_us": round(st_us, 3), "step_tflops": round(fl / (st_us * 1e-6) / 1e12, 1),
+              "l2": f"{copies} rotated copies of {set_bytes / 2**20:.1f} MiB"})
+    return e
+
+
+def per_config(dev, peaks, log):
+    """Every workload of the five configurations, each shape timed on its own."""
     import nvfp4_block_scaled_08_b200 as nv
     from nvfp4_block_scaled_08_b200 import workloads
-    p_fp4 = peaks["bf16_tflops"] * FP4_PER_BF16
-    out = {}
-    for c in workloads.plateau_cases():
-        if c.name not in ("square_8192", "ratio_512x2048x6144"):
-            continue
-        a, b = c.a().to(dev), c.b().to(dev)
-        gsa, gsb = nv.global_scale(a), nv.global_scale(b)
-        qa, sa = nv.quantize(a, gsa)
-        qb, sb = nv.quantize(b, gsb)
-        sa, sb = nv.sf_tile(sa), nv.sf_tile(sb)
-        al = nv.alpha(gsa, gsb)
-        o = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
-        ws = nv.make_workspace(c.M, c.N, c.K, dev)
-        us = graph_time_us(lambda: nv.gemm(qa, sa, qb, sb, al, out=o, workspace=ws, tiled=True),
-                           reps=5 if c.M >= 8192 else 20)
-        tf = c.flops / (us * 1e-6) / 1e12
-        item = {"M": c.M, "N": c.N, "K": c.K, "us": round(us, 2), "tflops": round(tf, 1),
-                "frac_of_fp4_peak": round(tf / p_fp4, 4),
-                "fp4_peak_tflops": round(p_fp4, 1), "peak_source": "measured bf16 burst x 4"}
-        if c.name.startswith("ratio"):
-            ab, bb = a.to(torch.bfloat16), b.to(torch.bfloat16)
-            ub = graph_time_us(lambda: torch.matmul(ab, bb.t()), reps=20)
-            item["bf16_torch_us"] = round(ub, 2)
-            item["fp4_over_bf16"] = round(ub / us, 3)
-            del ab, bb
-        out[c.name] = item
-        del a, b, qa, sa, qb, sb, o, ws
+    out = []
+
+    def dense(config, cases, extra=None):
+        items = []
+        for c in cases:
+            t0 = time.perf_counter()
+            ds = DenseStep(nv, c.M, c.N, c.K, c.a(), c.b(), dev)
+            g, q, st = ds.time_all()
+            it = dense_entry(c.name, c.M, c.N, c.K, g, q, st, len(ds.sets), ds.set_bytes, peaks)
+            if extra is not None:
+                extra(c, ds, it)
+            items.append(it)
+            del ds
+            torch.cuda.empty_cache()
+            log(f"  {c.name}: gemm {g:.2f} us, quant {q:.2f} us, step {st:.2f} us "
+                f"({time.perf_counter() - t0:.1f} s)")
+        tot_fl = sum(2.0 * i["M"] * i["N"] * i["K"] for i in items)
+        tot_g = sum(i["gemm_us"] for i in items)
+        tot_st = sum(i["step_us"] for i in items)
+        out.append({"config": config, "shapes": items,
+                    "gemm_tflops_all": round(tot_fl / (tot_g * 1e-6) / 1e12, 1),
+                    "step_tflops_all": round(tot_fl / (tot_st * 1e-6) / 1e12, 1)})
+
+    dense("single 128x256x512, A,B ~ N(0,1)", [workloads.single_case()])
+    dense("attention projection N=768 K=6144 M={16,64,256,1024}", workloads.attn_proj_cases())
+    dense("MoE expert shapes: up N=2048 K=6144, down N=6144 K=2048, M={16,32,64,128,512,1024}",
+          workloads.moe_expert_cases())
+
+    # grouped MoE
+    items = []
+    for c in sorted(workloads.grouped_cases(), key=lambda c: (c.N, c.T)):
+        t0 = time.perf_counter()
+        gs = GroupedStep(nv, c, dev)
+        g, q, st = gs.time_all()
+        fl = gs.flops
+        by = gemm_bytes(gs.rows, gs.N, gs.K, experts=gs.touched)
+        it = {"name": c.name, "T": c.T, "experts": gs.E, "rows": gs.rows, "N": gs.N, "K": gs.K,
+              "rows_per_expert_min_max": list(gs.rows_per_expert),
+              "gemm_us": round(g, 2), "gemm_tflops": round(fl / (g * 1e-6) / 1e12, 1)}
+        it.update(frac_fields(fl, by, g, peaks))
+        it.update({"quantize_us": round(q, 3),
+                   "quantize_gbs": round(quant_bytes(gs.rows, gs.K) / (q * 1e-6) / 1e9, 1),
+                   "step_us": round(st, 2),
+                   "l2": f"weights {gs.Bq.numel() / 2**30:.2f} GiB packed, larger than L2"})
+        items.append(it)
+        log(f"  {c.name}: gemm {g:.1f} us, quant {q:.1f} us ({time.perf_counter() - t0:.1f} s)")
+        del gs
+        torch.cuda.empty_cache()
+    GroupedStep._weights = {}
     torch.cuda.empty_cache()
+    out.append({"config": "grouped MoE: 256 experts, top-8 of T={512,4096}; gate_up N=4096 K=6144, "
+                          "down N=6144 K=2048", "shapes": items})
+
+    # plateau (+ the bf16 ratio context)
+    def bf16_ratio(c, ds, it):
+        if not c.name.startswith("ratio"):
+            return
+        a = c.a().to(dev, torch.bfloat16)
+        b = c.b().to(dev, torch.bfloat16)
+        copies = n_copies((a.numel() + b.numel()) * 2 + c.M * c.N * 2, dev)
+        pairs = [(a.clone(), b.clone()) for _ in range(copies)]
+        ub = graph_time_us([lambda p=p: torch.matmul(p[0], p[1].t()) for p in pairs])
+        it["bf16_torch_us"] = round(ub, 3)
+        it["fp4_over_bf16"] = round(ub / it["gemm_us"], 3)
+        del pairs, a, b
+
+    dense("plateau M=N=K in {4096,8192,16384}, U(-1,1); 512x2048x6144 beside bf16 torch matmul",
+          workloads.plateau_cases(), extra=bf16_ratio)
     return out
 
 
+class HeadlineStep(DenseStep):
+    """The headline step. `timed` holds K steps in one graph, each with its own event pair
+    around the GEMM, so that every GEMM launch of the timed region has its own duration;
+    `single` is one step without events (warm-up)."""
+
+    def capture(self, steps):
+        s = self.sets[0]
+        self.step(s)
+        torch.cuda.synchronize()
+        single = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(single):
+            self.step(s)
+        self.ev = [(torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) for _ in range(steps)]
+        timed = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(timed):
+            for e0, e1 in self.ev:
+                self.quant(s)
+                e0.record()
+                self.gemm(s)
+                e1.record()
+        self.single, self.timed = single, timed
+
+    def gemm_ms(self):
+        return [e0.elapsed_time(e1) for e0, e1 in self.ev]
+
+
 def run_ours(args, world, rank, local):
+    from nvfp4_block_scaled_08_b200 import workloads
+    import nvfp4_block_scaled_08_b200 as nv
     dev = torch.device("cuda", local)
     peaks = measured_peaks()
-    nsets = 1 if args.flush else args.sets
-    sets = [AttnSweep(dev, rank, i, args.sf_layout == "tiled") for i in range(nsets)]
-    graphs = [sw.capture() for sw in sets]
-    sweep = sets[0]
-    # one graph of a whole rotation (every set once, in order: eight "layers"), so that
-    # consecutive steps are not separated by graph launches; single-set graphs cover the rest
-    rotation = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(rotation):
-        for sw in sets:
-            for it in sw.items:
-                sw.step_one(it)
-    stream = torch.cuda.current_stream()
-    if args.flush:
-        flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-        clean = torch.ones(CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
 
-    def before_step():
-        if args.flush:
-            # write a buffer 4x the L2, then read another 2x the L2: the step starts with
-            # nothing cached (data, kernel code and tensor maps alike) and no dirty lines
-            flush.zero_()
-            torch.sum(clean)
+    def log(msg):
+        if rank == 0 and args.verbose:
+            print(msg, file=sys.stderr, flush=True)
+
+    case = [c for c in workloads.plateau_cases() if c.name == args.workload][0]
+    t0 = time.perf_counter()
+    hs = HeadlineStep(nv, case.M, case.N, case.K, case.a(), case.b(), dev, copies=1)
+    log(f"headline inputs ready ({time.perf_counter() - t0:.1f} s)")
+    hs.capture(args.steps)
+    stream = torch.cuda.current_stream()
 
     clocks = ClockSampler(local)
     clocks.start()
-    if args.flush:
-        for i in range(args.warmup):
-            before_step()
-            graphs[i % nsets].replay()
-    else:                                  # W steps, from the same graphs as the timed ones
-        for _ in range(args.warmup // nsets):
-            rotation.replay()
-        for i in range(args.warmup % nsets):
-            graphs[i].replay()
+    for _ in range(args.warmup):
+        hs.single.replay()
+    hs.timed.replay()                 # the timed graph once untimed: its first launch uploads it
     torch.cuda.synchronize()
-
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    quant_ms = [0.0] * len(sweep.items)
-    gemm_ms = [0.0] * len(sweep.items)
-    total_ms = 0.0
     barrier(world)
     clocks.mark()
-    if args.flush:
-        # the flush before each step stays outside the timing: one bracket per step
-        for i in range(args.steps):
-            before_step()
-            start.record(stream)
-            graphs[i % nsets].replay()
-            end.record(stream)
-            end.synchronize()
-            total_ms += start.elapsed_time(end)
-    else:
-        # K steps back to back (each set was last touched nsets - 1 steps earlier), one
-        # bracket around all of them: whole rotations, then single sets
-        start.record(stream)
-        for _ in range(args.steps // nsets):
-            rotation.replay()
-        for i in range(args.steps % nsets):
-            graphs[i].replay()
-        end.record(stream)
-        end.synchronize()
-        total_ms = start.elapsed_time(end)
+    start.record(stream)
+    hs.timed.replay()
+    end.record(stream)
+    end.synchronize()
+    total_ms = start.elapsed_time(end)
     barrier(world)
     clocks.mark()
     clocks.stop()
-    # per-shape breakdown, untimed pass: the same step with event nodes between the kernels
-    # (they cost each GEMM its early launch, so this pass runs slower than the timed one)
-    nbreak = min(args.steps, 100)
-    for i in range(nbreak):
-        k = i % nsets
-        before_step()
-        sets[k].graph_ev.replay()
-        torch.cuda.synchronize()
-        for j, ev in enumerate(sets[k].ev):
-            quant_ms[j] += ev[0].elapsed_time(ev[1]) / nbreak
-            gemm_ms[j] += ev[1].elapsed_time(ev[2]) / nbreak
-    step_ms = total_ms / args.steps
-    set_bytes = sum(it["a"].numel() * 4 + it["q"].numel() + it["sf"].numel() + it["out"].numel() * 2
-                    for it in sweep.items) + sweep.Bq.numel() + sweep.sfB.numel()
+    g_ms = hs.gemm_ms()               # every GEMM launch of the timed region
+    gemm_us = statistics.fmean(g_ms) * 1e3
+    step_ms = max_over_ranks(total_ms / args.steps, world)
+    value = whole_job_value(hs.flops, step_ms, world)
 
-    step_ms = max_over_ranks(step_ms, world)
-    value = whole_job_value(sweep.flops, step_ms, world)
-
-    # e2e through the public API with host buffers; its outputs must equal the graph's
-    golden = [it["out"].cpu() for it in sweep.items]    # set 0's outputs from its last replay
-    sweep.setup_e2e()
+    # e2e through the public API with host buffers; its output must equal the graph's
+    s0 = hs.sets[0]
+    golden = s0["out"].cpu()
+    a_host = s0["a"].cpu().pin_memory()
+    out_host = torch.empty(case.M, case.N, dtype=torch.bfloat16).pin_memory()
+    a_dev = [s0["a"], torch.empty_like(s0["a"])]
+    ready = [torch.cuda.Event(), torch.cuda.Event()]
+    consumed = [torch.cuda.Event(), torch.cuda.Event()]
     copy_stream = torch.cuda.Stream(device=dev)
+
+    def e2e_step(i):
+        b = i & 1
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(consumed[b])          # step i - 2 has read this buffer
+            a_dev[b].copy_(a_host, non_blocking=True)
+            ready[b].record(copy_stream)
+        stream.wait_event(ready[b])
+        hs.quant(s0, stream, a=a_dev[b])
+        consumed[b].record(stream)
+        hs.gemm(s0, stream)
+        out_host.copy_(s0["out"], non_blocking=True)
+
+    nwarm = 2
+    for i in range(nwarm):
+        e2e_step(i)
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    barrier(world)
     e2e_start = torch.cuda.Event(enable_timing=True)
     e2e_end = torch.cuda.Event(enable_timing=True)
-    nwarm = max(2, min(args.warmup, 4))
-    for i in range(nwarm):
-        sweep.e2e_step(i, stream, copy_stream)
-    barrier(world)
     e2e_start.record(stream)
-    copy_stream.wait_event(e2e_start)       # no timed copy starts before the bracket
-    for i in range(args.steps):
-        sweep.e2e_step(nwarm + i, stream, copy_stream)
+    copy_stream.wait_event(e2e_start)                    # no timed copy starts before the bracket
+    for i in range(e2e_steps):
+        e2e_step(nwarm + i)
     e2e_end.record(stream)
     barrier(world)
     torch.cuda.synchronize()
-    e2e_match = all(torch.equal(it["out_host"], g) for it, g in zip(sweep.items, golden))
-    e2e_ms = max_over_ranks(e2e_start.elapsed_time(e2e_end) / args.steps, world)
-    e2e_value = whole_job_value(sweep.flops, e2e_ms, world)
+    e2e_match = torch.equal(out_host, golden)
+    e2e_ms = max_over_ranks(e2e_start.elapsed_time(e2e_end) / e2e_steps, world)
+    e2e_value = whole_job_value(hs.flops, e2e_ms, world)
 
-    # roofline: per shape, and for the dominant kernel family
-    per_shape = []
-    tot_gemm_us = tot_quant_us = tot_gemm_bytes = tot_quant_bytes = 0.0
-    for it, qm, gm in zip(sweep.items, quant_ms, gemm_ms):
-        M = it["M"]
-        fl = 2.0 * M * N_ATTN * K_ATTN
-        by = gemm_bytes(M, N_ATTN, K_ATTN)
-        r_us, bound = roofline_us(fl, by, peaks)
-        per_shape.append({
-            "M": M, "N": N_ATTN, "K": K_ATTN, "gemm_us": round(gm * 1e3, 3),
-            "gemm_tflops": round(fl / (gm * 1e-3) / 1e12, 1),
-            "roofline_us": round(r_us, 3), "bound": bound, "frac": round(r_us / (gm * 1e3), 4),
-            "quantize_us": round(qm * 1e3, 3),
-            "quantize_gbs": round(quant_bytes(M, K_ATTN) / (qm * 1e-3) / 1e9, 1),
-        })
-        tot_gemm_us += gm * 1e3
-        tot_quant_us += qm * 1e3
-        tot_gemm_bytes += by
-        tot_quant_bytes += quant_bytes(M, K_ATTN)
-    gemm_dominant = tot_gemm_us >= tot_quant_us
-    if gemm_dominant:
-        achieved = tot_gemm_bytes / (tot_gemm_us * 1e-6) / 1e9
-        kernel = "nvfp4_gemm_kernel (all M of the sweep)"
-        units = f"{tot_gemm_bytes:.0f} algorithmic bytes per sweep of 4 launches"
-    else:
-        achieved = tot_quant_bytes / (tot_quant_us * 1e-6) / 1e9
-        kernel = "quantize_dynamic_kernel (all M of the sweep)"
-        units = f"{tot_quant_bytes:.0f} algorithmic bytes per sweep"
-    roof = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1),
-            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": gemm_traffic() if gemm_dominant else None, "per": units,
-            "peak_source": f"{peaks['source']} hbm_gbs (burst copy)"}
-
+    peak_meas = peaks["bf16_tflops"] * FP4_PER_BF16
+    achieved = hs.flops / (gemm_us * 1e-6) / 1e12
+    roof = {"kernel": "nvfp4_gemm_kernel<256, non-swap, tiled scales> (one 16384^3 launch)",
+            "bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_meas, 1),
+            "unit": "TFLOP/s", "frac": round(achieved / peak_meas, 4), "traffic": gemm_traffic(),
+            "per": f"{hs.flops:.4g} algorithmic flops per launch (2 M N K)",
+            "peak_source": (f"{peaks['source']} bf16_tflops (burst) x {FP4_PER_BF16:g}, the nominal "
+                            "FP4/BF16 ratio"),
+            "peak_spec": SPEC_FP4_TFLOPS, "frac_of_spec": round(achieved / SPEC_FP4_TFLOPS, 4),
+            "gemm_us": round(gemm_us, 2), "gemm_us_min_max": [round(min(g_ms) * 1e3, 2),
+                                                              round(max(g_ms) * 1e3, 2)],
+            "traffic_algorithmic_bytes": gemm_bytes(case.M, case.N, case.K)}
+    quant_us = step_ms * 1e3 - gemm_us
     line = {
-        "metric": "NVFP4 GEMM TFLOPS and % of B200 FP4/HBM roofline per M x N x K",
+        "metric": METRIC,
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) -> fp32 acc -> bf16",
-        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
-        "config": {"workload": "attn_proj_sweep N=768 K=6144 M={16,64,256,1024}",
-                   "scales": f"{args.sf_layout} layout (both operands)",
-                   "step": "per M: quantize_dynamic(A fp32: global scale, alpha, codes) + gemm; one CUDA graph",
-                   "timing": ("one event pair per step, L2 flush before each (outside the pair)" if args.flush
-                              else f"{args.steps} steps back to back between one event pair (graphs of "
-                                   f"{nsets}-set rotations, then single sets)"),
-                   "l2": ("flushed before every timed step (512 MB write, then 256 MB read)" if args.flush else
-                          f"inputs larger than L2: {nsets} independent input sets of {set_bytes / 2**20:.0f} MiB "
-                          f"(activations, weights, outputs) in rotation, {nsets * set_bytes / 2**20:.0f} MiB "
-                          "in all, so each set was last touched nsets-1 steps ago"),
+        "data": "synthetic (seeded U(-1,1) fp32 activations and weights)",
+        "config": {"workload": HEADLINE if args.workload == "square_16384" else args.workload,
+                   "M": case.M, "N": case.N, "K": case.K,
+                   "scales": "tiled layout (both operands)",
+                   "step": ("quantize_dynamic(A fp32 [M,K]: global scale, alpha, codes, tiled scales) + "
+                            "gemm -> bf16 [M,N]; weights quantised once outside timing; one CUDA graph"),
+                   "timing": f"{args.steps} steps back to back between one event pair",
+                   "l2": (f"inputs larger than L2: A is {case.M * case.K * 4 / 2**30:.2f} GiB of fp32 "
+                          "read from HBM every step"),
                    "parallelism": f"replicas x{world}"},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": sweep.h2d_bytes, "d2h_bytes_per_step": sweep.d2h_bytes,
-                "ms_per_step": round(e2e_ms, 5),
+                "h2d_bytes_per_step": a_host.numel() * 4, "d2h_bytes_per_step": out_host.numel() * 2,
+                "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,
                 "how": ("eager public-API calls per step; pinned host A copied in on a second stream "
                         "into double-buffered device inputs (overlapping the previous step's kernels), "
                         "bf16 out copied back every step"),
                 "outputs_match_graph": e2e_match},
-        "gpu_launches": sweep.launches_per_step * args.steps,
+        "gpu_launches": 2 * args.steps,
         "roofline": roof,
-        "per_shape": per_shape,
-        "gemm_only_tflops": round(sweep.flops / (tot_gemm_us * 1e-6) / 1e12, 1),
+        "step_breakdown_us": {"gemm": round(gemm_us, 2), "quantize_and_gaps": round(quant_us, 2),
+                              "note": "an event node between the two kernels of every timed step"},
         "clocks": clocks.summary(),
     }
-    if rank == 0 and not args.no_context:
-        line["context"] = context_gemms(dev, peaks)
+    hs.single = hs.timed = None
+    del hs, a_dev, a_host, out_host, golden
+    torch.cuda.empty_cache()
+    if rank == 0 and not args.no_per_config:
+        t0 = time.perf_counter()
+        line["per_config"] = per_config(dev, peaks, log)
+        line["per_config_seconds"] = round(time.perf_counter() - t0, 1)
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
-    for sw in sets:
-        sw.graph = sw.graph_ev = None
-    del rotation
-    del graphs
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds, case)
+        if "per_config" in line:
+            add_cpu_per_config(line["per_config"], args.cpu_seconds_per_config)
     return line
 
 
 # ------------------------------------------------------------------ the oracle (CPU)
-
-class OracleSweep:
-    """The oracle on a bounded sample of the sweep: for every M, the first r rows of A (global
-    scale over the full A). Inputs, the weights' quantisation and dequantisation (the weights
-    are static, as in the GPU step) and a calibration pass are prepared once, outside any
-    timing. Each pass runs the oracle's quantisation of the A sample, its dequantisation and
-    the oracle's product of the dequantised operands (oracle.gemm is exactly that composition;
-    calling it would dequantise the 768 x 6144 weights again on every call, a fixed cost that
-    would swamp small samples)."""
-
-    def __init__(self):
-        import oracle
-        from nvfp4_block_scaled_08_b200 import workloads
-        self.oracle = oracle
-        cases = workloads.attn_proj_cases()
-        self.Ms = [c.M for c in cases]
-        b = cases[0].b().numpy()
-        self.gb = oracle.global_scale(b)
-        qb, sb = oracle.quantize(b, self.gb)
-        self.deq_b = oracle.dequantize(qb, sb)
-        self.a_all = [c.a().numpy() for c in cases]
-        self.threads = os.cpu_count() or 1
-        self.used_threads = 1
-        t0 = time.perf_counter()
-        self.one_pass([min(64, m) for m in self.Ms])
-        self.per_row = (time.perf_counter() - t0) / sum(min(64, m) for m in self.Ms)
-
-    def one_pass(self, rows, split=None):
-        """One pass over the row sample; adds the quantise and GEMM seconds to split[0], [1]."""
-        o = self.oracle
-        f = 0.0
-        for a, r in zip(self.a_all, rows):
-            t0 = time.perf_counter()
-            ga = o.global_scale(a)
-            qa, sa = o.quantize(a[:r], ga)
-            t1 = time.perf_counter()
-            o.gemm_dequantized(o.dequantize(qa, sa), self.deq_b, o.alpha(ga, self.gb), threads=self.threads)
-            t2 = time.perf_counter()
-            self.used_threads = max(self.used_threads, min(r, self.threads))   # rows split over threads
-            if split is not None:
-                split[0] += t1 - t0
-                split[1] += t2 - t1
-            f += 2.0 * r * N_ATTN * K_ATTN
-        return f
-
-    def run(self, budget_s: float):
-        """Passes over a row sample sized so that they take about budget_s (at least one
-        pass). Returns (flops, seconds, threads, description)."""
-        frac = min(1.0, budget_s / max(self.per_row * sum(self.Ms), 1e-9))
-        rows = [max(1, int(round(m * frac))) for m in self.Ms]
-        flops, passes = 0.0, 0
-        self.split = [0.0, 0.0]
-        self.used_threads = 1
-        t0 = time.perf_counter()
-        while True:
-            flops += self.one_pass(rows, self.split)
-            passes += 1
-            if time.perf_counter() - t0 >= 0.8 * budget_s:
-                break
-        dt = time.perf_counter() - t0
-        sample = (f"attn_proj sweep, first {rows} rows of M={list(M_SWEEP)} (global scale over the "
-                  f"full A), N=768, K=6144, {passes} pass(es); weights quantised and dequantised "
-                  f"outside timing; GEMM on up to {self.used_threads} threads (one per row), "
-                  f"quantisation on one")
-        return flops, dt, self.used_threads, sample
-
 
 def cpu_model() -> str:
     try:
@@ -676,44 +686,154 @@ def cpu_model() -> str:
     return platform.processor() or "unknown"
 
 
-def cpu_baseline(budget_s: float):
-    sweep = OracleSweep()
-    flops, dt, threads, sample = sweep.run(budget_s)
-    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
-            "kind": "oracle", "sample": sample, "seconds": round(dt, 2),
-            "quantize_seconds": round(sweep.split[0], 3), "gemm_seconds": round(sweep.split[1], 3),
-            "cpu_model": cpu_model()}
+class OracleDense:
+    """The oracle on a bounded sample of one dense shape: the first r rows of A against the
+    first c rows of B, full K. The global scales (over the full tensors) and the weights'
+    quantisation and dequantisation (static weights, as in the GPU step) are prepared once,
+    outside any timing. A pass runs the oracle's quantisation of the A rows, their
+    dequantisation and the oracle's product of the dequantised operands (oracle.gemm is that
+    composition; calling it would dequantise the weights again on every call)."""
+
+    def __init__(self, a, b, K, r, c):
+        import oracle
+        self.o = oracle
+        self.K = K
+        self.ga = oracle.global_scale(a)
+        self.gb = oracle.global_scale(b)
+        qb, sb = oracle.quantize(b[:c], self.gb)
+        self.deq_b = oracle.dequantize(qb, sb)
+        self.alpha = oracle.alpha(self.ga, self.gb)
+        self.a = a[:r]
+        self.r, self.c = r, c
+        self.threads = os.cpu_count() or 1
+
+    def one_pass(self, split):
+        o = self.o
+        t0 = time.perf_counter()
+        qa, sa = o.quantize(self.a, self.ga)
+        deq_a = o.dequantize(qa, sa)
+        t1 = time.perf_counter()
+        o.gemm_dequantized(deq_a, self.deq_b, self.alpha, threads=self.threads)
+        t2 = time.perf_counter()
+        split[0] += t1 - t0
+        split[1] += t2 - t1
+        return 2.0 * self.r * self.c * self.K
+
+    @property
+    def used_threads(self):
+        return min(self.r, self.threads)      # the product splits its rows over threads
+
+
+def oracle_sample_for(a, b, M, N, K, budget_s):
+    """An OracleDense whose pass takes about budget_s, from a small calibration pass."""
+    threads = os.cpu_count() or 1
+    r0, c0 = min(M, threads), min(N, 64)
+    probe = OracleDense(a, b, K, r0, c0)
+    split = [0.0, 0.0]
+    t0 = time.perf_counter()
+    probe.one_pass(split)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    scale = budget_s / dt
+    c = int(min(N, 2048, max(c0, c0 * min(scale, 64.0))))
+    scale_r = max(1.0, budget_s / max(dt * c / c0, 1e-4))
+    r = int(min(M, max(r0, r0 * scale_r)))
+    return OracleDense(a, b, K, r, c)
+
+
+def run_oracle(sample: OracleDense, budget_s: float):
+    split = [0.0, 0.0]
+    flops, passes = 0.0, 0
+    t0 = time.perf_counter()
+    while True:
+        flops += sample.one_pass(split)
+        passes += 1
+        if time.perf_counter() - t0 >= 0.8 * budget_s:
+            break
+    return flops, time.perf_counter() - t0, passes, split
+
+
+def cpu_baseline(budget_s: float, case):
+    a, b = case.a().numpy(), case.b().numpy()
+    s = oracle_sample_for(a, b, case.M, case.N, case.K, budget_s)
+    flops, dt, passes, split = run_oracle(s, budget_s)
+    rate = flops / dt
+    return {"value": round(rate / 1e12, 6), "unit": "TFLOP/s", "cores": s.used_threads,
+            "kind": "oracle",
+            "sample": (f"{case.name}: first {s.r} rows of A x first {s.c} rows of B, K={case.K}, "
+                       f"{passes} pass(es); global scales over the full tensors and the weights' "
+                       "quantisation outside timing; GEMM rows split over threads"),
+            "seconds": round(dt, 2), "quantize_seconds": round(split[0], 3),
+            "gemm_seconds": round(split[1], 3),
+            "extrapolated_full_step_seconds": round(2.0 * case.M * case.N * case.K / rate, 1),
+            "cpu_model": cpu_model(), "host_threads": os.cpu_count()}
+
+
+def add_cpu_per_config(entries, budget_s):
+    """One oracle sample per configuration (its largest dense shape, or an expert slice of the
+    grouped one), extrapolated to the configuration's shapes at the sampled rate."""
+    from nvfp4_block_scaled_08_b200 import workloads
+    picks = {0: workloads.single_case(), 1: workloads.attn_proj_cases()[-1],
+             2: workloads.moe_expert_cases()[-2], 4: workloads.plateau_cases()[1]}
+    for i, entry in enumerate(entries):
+        if i == 3:
+            c = workloads.grouped_cases()[0]
+            r = c.route()
+            rows = int(r.offsets[2])                      # the first two experts' rows
+            a = c.a(r.rows).numpy()
+            b = c.b(0).numpy()
+            s = OracleDense(a, b, c.K, rows, min(c.N, 512))
+            label = f"{c.name}: the first 2 experts' {rows} rows x {s.c} weight rows, K={c.K}"
+        else:
+            c = picks[i]
+            a, b = c.a().numpy(), c.b().numpy()
+            s = oracle_sample_for(a, b, c.M, c.N, c.K, budget_s)
+            label = f"{c.name}: first {s.r} rows of A x first {s.c} rows of B, K={c.K}"
+        flops, dt, passes, _ = run_oracle(s, budget_s)
+        rate = flops / dt
+        total = sum(2.0 * sh.get("rows", sh.get("M", 0)) * sh["N"] * sh["K"] for sh in entry["shapes"])
+        entry["cpu_baseline"] = {"value": round(rate / 1e12, 6), "unit": "TFLOP/s",
+                                 "cores": s.used_threads, "kind": "oracle",
+                                 "sample": label + f", {passes} pass(es)",
+                                 "extrapolated_seconds_for_all_shapes": round(total / rate, 2),
+                                 "label": "extrapolated from the sample's rate"}
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return None
+    from nvfp4_block_scaled_08_b200 import workloads
+    case = [c for c in workloads.plateau_cases() if c.name == args.workload][0]
     # every step a bounded sample, so that warm-up + K steps take about two minutes
-    per_step = max(0.02, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
-    sweep = OracleSweep()
+    per_step = max(0.05, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    a, b = case.a().numpy(), case.b().numpy()
+    s = oracle_sample_for(a, b, case.M, case.N, case.K, per_step)
     for _ in range(args.warmup):
-        sweep.run(per_step)
+        run_oracle(s, per_step)
     tot_f = tot_t = tot_q = tot_g = 0.0
-    info = None
+    passes = 0
     for _ in range(args.steps):
-        f, t, th, sample = sweep.run(per_step)
+        f, t, p, split = run_oracle(s, per_step)
         tot_f += f
         tot_t += t
-        tot_q += sweep.split[0]
-        tot_g += sweep.split[1]
-        info = (th, sample)
+        tot_q += split[0]
+        tot_g += split[1]
+        passes += p
     value = tot_f / tot_t / 1e12
+    sample = (f"{case.name}: first {s.r} rows of A x first {s.c} rows of B, K={case.K}, {passes} "
+              f"pass(es) over {args.steps} steps; global scales and the weights' quantisation "
+              "outside timing; GEMM rows split over threads")
     return {
         "impl": "reference",
-        "metric": "NVFP4 GEMM TFLOPS and % of B200 FP4/HBM roofline per M x N x K",
+        "metric": METRIC,
         "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
         "data": "synthetic (seeded)",
-        "config": {"workload": "attn_proj_sweep N=768 K=6144 M={16,64,256,1024}",
+        "config": {"workload": HEADLINE if args.workload == "square_16384" else args.workload,
+                   "M": case.M, "N": case.N, "K": case.K,
                    "note": "CPU oracle (test infrastructure) on a bounded row sample per step"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": info[0],
-                         "kind": "oracle", "sample": info[1], "quantize_seconds": round(tot_q, 3),
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": s.used_threads,
+                         "kind": "oracle", "sample": sample, "quantize_seconds": round(tot_q, 3),
                          "gemm_seconds": round(tot_g, 3), "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -723,20 +843,18 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--workload", default="square_16384",
+                    choices=["square_16384", "square_8192", "square_4096", "ratio_512x2048x6144"],
+                    help="headline workload (a plateau shape)")
+    ap.add_argument("--e2e-steps", type=int, default=20, help="steps of the host-buffer e2e run (<= steps)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds-per-config", type=float, default=2.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sf-layout", choices=["tiled", "linear"], default="tiled",
-                    help="scale layout of both GEMM operands in the sweep (tiled: the layout the "
-                         "tensor cores read, fetched without a re-layout step)")
-    ap.add_argument("--no-context", action="store_true",
-                    help="skip the compute-bound context GEMMs reported after the timed step")
-    ap.add_argument("--sets", type=int, default=8,
-                    help="independent input sets rotated between steps (together larger than L2)")
-    ap.add_argument("--flush", action="store_true",
-                    help="flush L2 before every step instead of rotating input sets")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--verbose", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
