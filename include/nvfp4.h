@@ -76,6 +76,18 @@ typedef enum {
     NVFP4_SF_TILED = 1
 } nvfp4_sf_layout;
 
+/*
+ * Element type of a GEMM output (the mm_fp4 signature's out_dtype: "The Art of Reading the
+ * Manual", section "The Message"). The value alpha * acc is computed in fp32 from the fp32
+ * accumulator and rounded once to the output type, to nearest even; fp16 values beyond its
+ * range become +-infinity. NVFP4_OUT_F32 stores alpha * acc itself (4 bytes per element).
+ */
+typedef enum {
+    NVFP4_OUT_BF16 = 0,
+    NVFP4_OUT_F16 = 1,
+    NVFP4_OUT_F32 = 2
+} nvfp4_out_dtype;
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* nvfp4_status_string(nvfp4_status s);
 
@@ -188,6 +200,16 @@ nvfp4_status nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* 
                            nvfp4_sf_layout sf_layout, cudaStream_t stream);
 
 /*
+ * nvfp4_gemm_ex with the output element type chosen: out[M, N] holds elements of out_dtype
+ * (2 or 4 bytes each, row-major, 16-byte aligned). Same operation, checks and split-K rules;
+ * nvfp4_gemm_ex is this call with NVFP4_OUT_BF16. A bad out_dtype: NVFP4_ERR_INVALID_ARG.
+ */
+nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                            const uint8_t* sfB, const float* alpha, void* out,
+                            int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
+                            nvfp4_sf_layout sf_layout, nvfp4_out_dtype out_dtype, cudaStream_t stream);
+
+/*
  * Grouped (mixture-of-experts) NVFP4 GEMM ("When a Benchmark Crashes", section "Why This
  * Message Was Written": 256 experts, 8 active per token). Rows of A are sorted by expert;
  * expert e owns rows [expert_offsets[e], expert_offsets[e+1]) and computes
@@ -205,6 +227,90 @@ nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint
                                 const int32_t* expert_offsets, int32_t E, int64_t total_rows,
                                 int64_t N, int64_t K, void* out, void* ws, size_t ws_bytes,
                                 cudaStream_t stream);
+
+/*
+ * nvfp4_grouped_gemm with the output element type chosen (out[total_rows, N] of out_dtype;
+ * no workspace). nvfp4_grouped_gemm is this call with NVFP4_OUT_BF16.
+ */
+nvfp4_status nvfp4_grouped_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                                   const uint8_t* sfB, const float* alpha,
+                                   const int32_t* expert_offsets, int32_t E, int64_t total_rows,
+                                   int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
+                                   cudaStream_t stream);
+
+/*
+ * Grouped gate_up GEMM of a mixture-of-experts MLP with the SwiGLU activation and the NVFP4
+ * requantisation for the down projection fused into its epilogue (the layer of "When a
+ * Benchmark Crashes", section "Why This Message Was Written": 256 experts, MoE intermediate
+ * size I = 2048, gate_up N = 2 I). Per expert e and row r in [expert_offsets[e],
+ * expert_offsets[e+1]), with v = alpha[e] * sum_k deq(A)[r, k] deq(B[e])[n, k] in fp32:
+ *     g = v[n = j], u = v[n = I + j],  h[r, j] = (g / (1 + exp(-g))) * u     (j < I, fp32)
+ * and h is quantised exactly as nvfp4_quantize does, with the fixed global scale gs_h
+ * (device, one float, chosen in advance: an epilogue cannot know max|h|):
+ *     h_q[total_rows, I/2] (e2m1 codes) and h_sf[total_rows, I/16] (e4m3, linear layout),
+ * ready to be the A operand of the down projection (nvfp4_grouped_gemm with
+ * alpha_down[e] = 1 / (gs_h * gsB_down[e])). B[E, 2I, K/2] holds the gate rows [0, I) then
+ * the up rows [I, 2I) of each expert, sfB[E, 2I, K/16] likewise. The gate / up split of the
+ * gate_up output and this order are the library's reading (the pages name the layer, not its
+ * activation). Requires I % 64 == 0 and the nvfp4_grouped_gemm conditions; h_q 16-byte
+ * aligned. Rows past expert_offsets[E] are not written. h is computed in fp32 with CUDA's
+ * expf, so a code can differ from a correctly rounded fp64 evaluation where h lies next to a
+ * rounding boundary.
+ */
+nvfp4_status nvfp4_grouped_gemm_swiglu(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                                       const uint8_t* sfB, const float* alpha,
+                                       const int32_t* expert_offsets, int32_t E, int64_t total_rows,
+                                       int64_t I, int64_t K, const float* gs_h, uint8_t* h_q,
+                                       uint8_t* h_sf, cudaStream_t stream);
+
+/*
+ * The mixture-of-experts layer around the grouped GEMMs ("When a Benchmark Crashes", section
+ * "Why This Message Was Written": every token is routed to 8 of 256 experts). The pages name
+ * the layer, not its router; the readings: probabilities are a softmax over the expert logits;
+ * a token takes its k largest, ties going to the lower expert index, in descending order; its
+ * k weights are those probabilities renormalised to sum to 1; the expert-sorted order lists
+ * each expert's (token, slot) pairs in ascending token order.
+ *
+ * nvfp4_moe_route: logits[T, E] (fp32, device) ->
+ *   experts[T, k] (int32): slot s = the s-th largest logit (exact: the selection compares the
+ *                          logits themselves, which order like the probabilities);
+ *   weights[T, k] (fp32):  exp(l_s - l_0) / sum_j exp(l_j - l_0) over the k winners (fp32,
+ *                          CUDA's expf; within a few ulp of the exact renormalised softmax);
+ *   expert_offsets[E + 1]: expert e owns rows [offsets[e], offsets[e+1]) of the sorted order;
+ *   row_of[T, k]:          the sorted row that holds token t's slot s;
+ *   token_of_row[T k]:     the token of every sorted row.
+ * All device, int32 / fp32, 4-byte aligned. E <= 1024, k <= min(E, 32). Three launches; no
+ * scratch (row_of and expert_offsets hold intermediate counts until the last one). Results are
+ * deterministic (no atomics). T == 0 writes expert_offsets as all zero.
+ */
+nvfp4_status nvfp4_moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t* experts,
+                             float* weights, int32_t* expert_offsets, int32_t* row_of,
+                             int32_t* token_of_row, cudaStream_t stream);
+
+/*
+ * Quantises the tokens x[T, H] (fp32 or bf16, row stride ld_x elements) once, exactly as
+ * nvfp4_quantize_dynamic does (global scale of all of x written to gs_out[0], alpha_out[i] =
+ * 1 / (gs_out[0] * gs_other[i]) for i < n_alpha, e.g. against every expert's weight scale), and
+ * writes token t's codes and scales to each of its k expert-sorted rows row_of[t, s]:
+ * q[T k, H/2] and sf[T k, H/16] (linear layout), the A operand of the grouped GEMM. Quantising
+ * then gathering equals gathering then quantising, as rows are independent once the global
+ * scale is known. One launch. Requires H % 16 == 0, k <= 32; x, q 16-byte aligned; every row
+ * index in row_of below T k (as nvfp4_moe_route writes them).
+ */
+nvfp4_status nvfp4_moe_gather_quantize(const void* x, nvfp4_in_dtype dtype, int32_t T, int64_t H,
+                                       int64_t ld_x, int32_t k, const int32_t* row_of, float* gs_out,
+                                       uint8_t* q, uint8_t* sf, const float* gs_other, int32_t n_alpha,
+                                       float* alpha_out, cudaStream_t stream);
+
+/*
+ * The weighted combine after the down projection: out[t, :] = sum_s weights[t, s] *
+ * y[row_of[t, s], :] for t < T, accumulated in fp32 in ascending slot order (deterministic) and
+ * rounded once to out_dtype. y[T k, H] holds y_dtype elements (the down GEMM's output), out
+ * [T, H] out_dtype; both 16-byte aligned, H % 8 == 0, k <= 32. All device.
+ */
+nvfp4_status nvfp4_moe_combine(const void* y, nvfp4_out_dtype y_dtype, const float* weights,
+                               const int32_t* row_of, int32_t T, int64_t H, int32_t k, void* out,
+                               nvfp4_out_dtype out_dtype, cudaStream_t stream);
 
 /*
  * nvfp4_gemm without a workspace argument and without any device allocation. The reference

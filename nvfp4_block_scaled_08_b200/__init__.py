@@ -30,7 +30,8 @@ from . import _build
 __all__ = [
     "Nvfp4Error", "load", "global_scale", "quantize", "quantize_dynamic", "alpha", "gemm", "gemm_workspace_size",
     "gemm_noalloc", "plan_override",
-    "make_workspace", "grouped_gemm", "round_e4m3", "round_e2m1", "last_device_error",
+    "make_workspace", "grouped_gemm", "grouped_gemm_swiglu", "moe_route", "moe_gather_quantize",
+    "moe_combine", "round_e4m3", "round_e2m1", "last_device_error",
     "STATUS",
 ]
 
@@ -69,6 +70,16 @@ SIGNATURES = {
     "nvfp4_sf_bytes": (_SZ, [_I64, _I64, ctypes.c_int]),
     "nvfp4_sf_tile": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "nvfp4_gemm_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int, _P]),
+    "nvfp4_gemm_ex2": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int,
+                                      ctypes.c_int, _P]),
+    "nvfp4_grouped_gemm_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P,
+                                             ctypes.c_int, _P]),
+    "nvfp4_grouped_gemm_swiglu": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
+                                                 _P, _P]),
+    "nvfp4_moe_route": (ctypes.c_int, [_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_moe_gather_quantize": (ctypes.c_int, [_P, ctypes.c_int, _I32, _I64, _I64, _I32, _P, _P, _P, _P, _P,
+                                                 _I32, _P, _P]),
+    "nvfp4_moe_combine": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _I32, _I64, _I32, _P, ctypes.c_int, _P]),
     "nvfp4_grouped_gemm_workspace_size": (_SZ, [_I32, _I64, _I64, _I64]),
     "nvfp4_grouped_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
                                           _SZ, _P]),
@@ -233,21 +244,32 @@ def make_workspace(M: int, N: int, K: int, device="cuda") -> torch.Tensor | None
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None, tiled=False) -> torch.Tensor:
-    """out[M, N] = bf16(alpha * sum_k deq(A)[m,k] deq(B)[n,k]).
+OUT_DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
+
+
+def _out_code(out: torch.Tensor) -> int:
+    if out.dtype not in OUT_DTYPES:
+        raise ValueError("out must be bfloat16, float16 or float32")
+    return OUT_DTYPES[out.dtype]
+
+
+def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None, tiled=False,
+         out_dtype=torch.bfloat16) -> torch.Tensor:
+    """out[M, N] = alpha * sum_k deq(A)[m,k] deq(B)[n,k] in bf16, fp16 or fp32.
 
     Aq [M, K/2] uint8, sfA [M, K/16] uint8, Bq [N, K/2], sfB [N, K/16], alpha_t fp32 [1];
-    out bf16 [M, N] (allocated if None); workspace: zero-filled uint8 tensor of
-    gemm_workspace_size(M, N, K) bytes or None (no split-K). tiled: sfA and sfB in the tiled
-    layout (flat uint8 tensors from sf_tile or quantize_dynamic(tiled=True))."""
+    out [M, N] (allocated with out_dtype if None; otherwise its dtype decides); workspace:
+    zero-filled uint8 tensor of gemm_workspace_size(M, N, K) bytes or None (no split-K).
+    tiled: sfA and sfB in the tiled layout (flat uint8 tensors from sf_tile or
+    quantize_dynamic(tiled=True))."""
     M, K = Aq.shape[0], Aq.shape[1] * 2
     N = Bq.shape[0]
     if out is None:
-        out = torch.empty(M, N, dtype=torch.bfloat16, device=Aq.device)
+        out = torch.empty(M, N, dtype=out_dtype, device=Aq.device)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
-    _check("nvfp4_gemm_ex", load().nvfp4_gemm_ex(
+    _check("nvfp4_gemm_ex2", load().nvfp4_gemm_ex2(
         _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alpha_t), _ptr(out), M, N, K,
-        ws_ptr, ws_bytes, SF_TILED if tiled else SF_LINEAR, _stream(stream)))
+        ws_ptr, ws_bytes, SF_TILED if tiled else SF_LINEAR, _out_code(out), _stream(stream)))
     return out
 
 
@@ -266,16 +288,18 @@ def gemm_noalloc(Aq, sfA, Bq, sfB, alpha_t, out=None, stream=None) -> torch.Tens
     return out
 
 
-def grouped_gemm(Aq, sfA, Bq, sfB, alphas, offsets, out=None, stream=None) -> torch.Tensor:
-    """Per expert e: out[r] = bf16(alpha[e] * deq(A)[r] . deq(B[e])^T) for rows r in
-    [offsets[e], offsets[e+1]). Bq [E, N, K/2], sfB [E, N, K/16], offsets int32 [E+1]."""
+def grouped_gemm(Aq, sfA, Bq, sfB, alphas, offsets, out=None, stream=None,
+                 out_dtype=torch.bfloat16) -> torch.Tensor:
+    """Per expert e: out[r] = alpha[e] * deq(A)[r] . deq(B[e])^T for rows r in
+    [offsets[e], offsets[e+1]) (bf16, fp16 or fp32). Bq [E, N, K/2], sfB [E, N, K/16],
+    offsets int32 [E+1]."""
     rows, K = Aq.shape[0], Aq.shape[1] * 2
     E, N = Bq.shape[0], Bq.shape[1]
     if out is None:
-        out = torch.empty(rows, N, dtype=torch.bfloat16, device=Aq.device)
-    _check("nvfp4_grouped_gemm", load().nvfp4_grouped_gemm(
+        out = torch.empty(rows, N, dtype=out_dtype, device=Aq.device)
+    _check("nvfp4_grouped_gemm_ex", load().nvfp4_grouped_gemm_ex(
         _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alphas), _ptr(offsets), E, rows, N, K,
-        _ptr(out), None, 0, _stream(stream)))
+        _ptr(out), _out_code(out), _stream(stream)))
     return out
 
 
@@ -293,6 +317,89 @@ class plan_override:
     def __exit__(self, *exc):
         _check("nvfp4_set_plan_override", load().nvfp4_set_plan_override(0, 0, 0, 0, 0))
         return False
+
+
+def grouped_gemm_swiglu(Aq, sfA, Bq, sfB, alphas, offsets, gs_h, h_q=None, h_sf=None, stream=None):
+    """Grouped gate_up GEMM with SwiGLU and NVFP4 requantisation fused into the epilogue.
+
+    Bq [E, 2I, K/2] (gate rows [0, I), up rows [I, 2I) per expert), sfB [E, 2I, K/16];
+    gs_h fp32 [1] (device): the fixed global scale of h = silu(gate) * up.
+    Returns (h_q uint8 [rows, I/2], h_sf uint8 [rows, I/16]), the down projection's A."""
+    rows, K = Aq.shape[0], Aq.shape[1] * 2
+    E, N = Bq.shape[0], Bq.shape[1]
+    I = N // 2
+    if h_q is None:
+        h_q = torch.empty(rows, I // 2, dtype=torch.uint8, device=Aq.device)
+    if h_sf is None:
+        h_sf = torch.empty(rows, I // 16, dtype=torch.uint8, device=Aq.device)
+    _check("nvfp4_grouped_gemm_swiglu", load().nvfp4_grouped_gemm_swiglu(
+        _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alphas), _ptr(offsets), E, rows, I, K,
+        _ptr(gs_h), _ptr(h_q), _ptr(h_sf), _stream(stream)))
+    return h_q, h_sf
+
+
+# ------------------------------------------------------------------ mixture-of-experts layer
+
+def moe_route(logits: torch.Tensor, k: int, stream=None):
+    """Top-k routing of router logits [T, E] (fp32) and the expert-sorted permutation.
+
+    Returns (experts int32 [T, k], weights fp32 [T, k], offsets int32 [E+1],
+    row_of int32 [T, k], token_of_row int32 [T*k])."""
+    _dev(logits, "logits")
+    if logits.dtype != torch.float32 or not logits.is_contiguous():
+        raise ValueError("logits must be contiguous float32")
+    T, E = logits.shape
+    dev = logits.device
+    experts = torch.empty(T, k, dtype=torch.int32, device=dev)
+    weights = torch.empty(T, k, dtype=torch.float32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty(T, k, dtype=torch.int32, device=dev)
+    token_of_row = torch.empty(T * k, dtype=torch.int32, device=dev)
+    _check("nvfp4_moe_route", load().nvfp4_moe_route(
+        _ptr(logits), T, E, k, _ptr(experts), _ptr(weights), _ptr(offsets), _ptr(row_of),
+        _ptr(token_of_row), _stream(stream)))
+    return experts, weights, offsets, row_of, token_of_row
+
+
+def moe_gather_quantize(x: torch.Tensor, row_of: torch.Tensor, gs_other: torch.Tensor | None = None,
+                        gs=None, q=None, sf=None, alpha_out=None, stream=None):
+    """Quantise tokens x [T, H] once (global scale over x) into their k expert-sorted rows.
+
+    Returns (q uint8 [T*k, H/2], sf uint8 [T*k, H/16], gs, alpha or None)."""
+    _dev(x, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    T, H = x.shape
+    k = row_of.shape[1]
+    dev = x.device
+    if q is None:
+        q = torch.empty(T * k, H // 2, dtype=torch.uint8, device=dev)
+    if sf is None:
+        sf = torch.empty(T * k, H // 16, dtype=torch.uint8, device=dev)
+    if gs is None:
+        gs = torch.empty(1, dtype=torch.float32, device=dev)
+    n = 0 if gs_other is None else gs_other.numel()
+    if n and alpha_out is None:
+        alpha_out = torch.empty(n, dtype=torch.float32, device=dev)
+    _check("nvfp4_moe_gather_quantize", load().nvfp4_moe_gather_quantize(
+        _ptr(x), _dtype_code(x), T, H, x.stride(0), k, _ptr(row_of), _ptr(gs), _ptr(q), _ptr(sf),
+        _ptr(gs_other), n, _ptr(alpha_out) if n else None, _stream(stream)))
+    return q, sf, gs, (alpha_out if n else None)
+
+
+def moe_combine(y: torch.Tensor, weights: torch.Tensor, row_of: torch.Tensor, out=None,
+                out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    """out[t] = sum_s weights[t, s] * y[row_of[t, s]] (fp32 accumulation, slot order)."""
+    T, k = weights.shape
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty(T, H, dtype=out_dtype, device=y.device)
+    if y.dtype not in OUT_DTYPES:
+        raise ValueError("y must be bfloat16, float16 or float32")
+    _check("nvfp4_moe_combine", load().nvfp4_moe_combine(
+        _ptr(y), OUT_DTYPES[y.dtype], _ptr(weights), _ptr(row_of), T, H, k, _ptr(out), _out_code(out),
+        _stream(stream)))
+    return out
 
 
 # ------------------------------------------------------------------ conversions and errors

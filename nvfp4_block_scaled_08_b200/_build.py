@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libnvfp4.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["api.cu", "gemm.cu", "quantize.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "gemm.cu", "quantize.cu", "moe.cu", "noalloc.cu"]
 HEADERS = ["ptx.cuh", "gemm_kernel.cuh", "internal.h", "quant_core.cuh"]
 
 NVCC_FLAGS = [

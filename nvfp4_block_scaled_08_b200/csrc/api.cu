@@ -272,12 +272,15 @@ size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K)
     return nvfp4::plan_gemm(M, N, K, true, d.num_sms).ws_bytes;
 }
 
-nvfp4_status nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
-                           const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
-                           size_t ws_bytes, nvfp4_sf_layout sf_layout, cudaStream_t stream)
+nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                            const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
+                            size_t ws_bytes, nvfp4_sf_layout sf_layout, nvfp4_out_dtype out_dtype,
+                            cudaStream_t stream)
 {
     if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
     if (sf_layout != NVFP4_SF_LINEAR && sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F16 && out_dtype != NVFP4_OUT_F32)
+        return NVFP4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return NVFP4_OK;
     if (M > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     nvfp4_status st = check_gemm_common(A, sfA, B, sfB, alpha, out, N, K);
@@ -292,18 +295,28 @@ nvfp4_status nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* 
     // tiled scales: Q tiles start on 128-row tile boundaries (tuning overrides can break it)
     if (tiled && (plan.swap ? plan.q_tiles != 1 : (plan.bn % 128 != 0)))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0, ws, d.err_word, tiled};
+    nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0, ws, d.err_word, tiled,
+                        static_cast<int32_t>(out_dtype)};
     bool enc_failed = false;
     cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
     if (enc_failed) return NVFP4_ERR_CUDA;
     return from_cuda(e);
 }
 
+nvfp4_status nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                           const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
+                           size_t ws_bytes, nvfp4_sf_layout sf_layout, cudaStream_t stream)
+{
+    return nvfp4_gemm_ex2(A, sfA, B, sfB, alpha, out, M, N, K, ws, ws_bytes, sf_layout, NVFP4_OUT_BF16,
+                          stream);
+}
+
 nvfp4_status nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                         const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
                         size_t ws_bytes, cudaStream_t stream)
 {
-    return nvfp4_gemm_ex(A, sfA, B, sfB, alpha, out, M, N, K, ws, ws_bytes, NVFP4_SF_LINEAR, stream);
+    return nvfp4_gemm_ex2(A, sfA, B, sfB, alpha, out, M, N, K, ws, ws_bytes, NVFP4_SF_LINEAR, NVFP4_OUT_BF16,
+                          stream);
 }
 
 size_t nvfp4_grouped_gemm_workspace_size(int32_t E, int64_t total_rows, int64_t N, int64_t K)
@@ -312,14 +325,15 @@ size_t nvfp4_grouped_gemm_workspace_size(int32_t E, int64_t total_rows, int64_t 
     return 0;
 }
 
-nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
-                                const uint8_t* sfB, const float* alpha,
-                                const int32_t* expert_offsets, int32_t E, int64_t total_rows,
-                                int64_t N, int64_t K, void* out, void* ws, size_t ws_bytes,
-                                cudaStream_t stream)
+nvfp4_status nvfp4_grouped_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                                   const uint8_t* sfB, const float* alpha,
+                                   const int32_t* expert_offsets, int32_t E, int64_t total_rows,
+                                   int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
+                                   cudaStream_t stream)
 {
-    (void)ws; (void)ws_bytes;
     if (E < 0 || total_rows < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F16 && out_dtype != NVFP4_OUT_F32)
+        return NVFP4_ERR_INVALID_ARG;
     if (E == 0 || total_rows == 0 || N == 0) return NVFP4_OK;
     if (E > nvfp4::kMaxExperts) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (total_rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -333,11 +347,114 @@ nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint
     if (st != NVFP4_OK) return st;
     nvfp4::GemmPlan plan = nvfp4::plan_grouped(E, total_rows, N, K, d.num_sms);
     nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, 0, N, K, expert_offsets, E, total_rows,
-                        nullptr, d.err_word};
+                        nullptr, d.err_word, false, static_cast<int32_t>(out_dtype)};
     bool enc_failed = false;
     cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
     if (enc_failed) return NVFP4_ERR_CUDA;
     return from_cuda(e);
+}
+
+nvfp4_status nvfp4_grouped_gemm_swiglu(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                                       const uint8_t* sfB, const float* alpha,
+                                       const int32_t* expert_offsets, int32_t E, int64_t total_rows,
+                                       int64_t I, int64_t K, const float* gs_h, uint8_t* h_q,
+                                       uint8_t* h_sf, cudaStream_t stream)
+{
+    if (E < 0 || total_rows < 0 || I < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (E == 0 || total_rows == 0 || I == 0) return NVFP4_OK;
+    if (!expert_offsets || !gs_h || !h_sf) return NVFP4_ERR_INVALID_ARG;
+    if (E > nvfp4::kMaxExperts || total_rows > kMaxDim || I % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    nvfp4_status st = check_gemm_common(A, sfA, B, sfB, alpha, h_q, 2 * I, K);
+    if (st != NVFP4_OK) return st;
+    if (!aligned4(expert_offsets) || !aligned4(gs_h)) return NVFP4_ERR_MISALIGNED;
+    if (static_cast<int64_t>(E) * 2 * I > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    DeviceInfo d;
+    st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    nvfp4::GemmPlan plan = nvfp4::plan_grouped(E, total_rows, 2 * I, K, d.num_sms);
+    nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, nullptr, 0, 2 * I, K, expert_offsets, E, total_rows,
+                        nullptr, d.err_word, false, 0, h_q, h_sf, gs_h};
+    bool enc_failed = false;
+    cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
+    if (enc_failed) return NVFP4_ERR_CUDA;
+    return from_cuda(e);
+}
+
+nvfp4_status nvfp4_grouped_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                                const uint8_t* sfB, const float* alpha,
+                                const int32_t* expert_offsets, int32_t E, int64_t total_rows,
+                                int64_t N, int64_t K, void* out, void* ws, size_t ws_bytes,
+                                cudaStream_t stream)
+{
+    (void)ws; (void)ws_bytes;
+    return nvfp4_grouped_gemm_ex(A, sfA, B, sfB, alpha, expert_offsets, E, total_rows, N, K, out,
+                                 NVFP4_OUT_BF16, stream);
+}
+
+nvfp4_status nvfp4_moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t* experts,
+                             float* weights, int32_t* expert_offsets, int32_t* row_of, int32_t* token_of_row,
+                             cudaStream_t stream)
+{
+    if (T < 0 || E <= 0 || k <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (E > 1024 || k > 32 || k > E) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!expert_offsets) return NVFP4_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !experts || !weights || !row_of || !token_of_row)) return NVFP4_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(T) * k > kMaxDim || static_cast<int64_t>(T) * E > (int64_t(1) << 40))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned4(logits) || !aligned4(experts) || !aligned4(weights) || !aligned4(expert_offsets) ||
+        !aligned4(row_of) || !aligned4(token_of_row))
+        return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_moe_route(logits, T, E, k, experts, weights, expert_offsets, row_of,
+                                             token_of_row, stream));
+}
+
+nvfp4_status nvfp4_moe_gather_quantize(const void* x, nvfp4_in_dtype dtype, int32_t T, int64_t H, int64_t ld_x,
+                                       int32_t k, const int32_t* row_of, float* gs_out, uint8_t* q, uint8_t* sf,
+                                       const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                       cudaStream_t stream)
+{
+    if (T < 0 || H < 0 || k <= 0 || n_alpha < 0) return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_F32 && dtype != NVFP4_IN_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (!gs_out || (n_alpha > 0 && (!gs_other || !alpha_out))) return NVFP4_ERR_INVALID_ARG;
+    if (T == 0 || H == 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;     // no tensor to take a scale of
+    if (!x || !row_of || !q || !sf) return NVFP4_ERR_INVALID_ARG;
+    if (H % 16 != 0 || H > kMaxDim || k > 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld_x < H) return NVFP4_ERR_INVALID_ARG;
+    const int64_t esz = dtype == NVFP4_IN_BF16 ? 2 : 4;
+    if (static_cast<int64_t>(T) * (H * esz / 16) >= (int64_t(1) << 31) ||
+        static_cast<int64_t>(T) * k * (H / 2) >= (int64_t(1) << 40))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || (ld_x * esz) % 16 != 0 || !aligned16(q) || !aligned4(gs_out) || !aligned4(row_of) ||
+        (n_alpha > 0 && (!aligned4(gs_other) || !aligned4(alpha_out))))
+        return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_gather_quantize(x, dtype == NVFP4_IN_BF16, T, H, ld_x, k, row_of, gs_out, q,
+                                                   sf, gs_other, n_alpha, alpha_out, d.err_word, stream,
+                                                   d.num_sms));
+}
+
+nvfp4_status nvfp4_moe_combine(const void* y, nvfp4_out_dtype y_dtype, const float* weights,
+                               const int32_t* row_of, int32_t T, int64_t H, int32_t k, void* out,
+                               nvfp4_out_dtype out_dtype, cudaStream_t stream)
+{
+    if (T < 0 || H < 0 || k <= 0) return NVFP4_ERR_INVALID_ARG;
+    if ((y_dtype != NVFP4_OUT_BF16 && y_dtype != NVFP4_OUT_F16 && y_dtype != NVFP4_OUT_F32) ||
+        (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F16 && out_dtype != NVFP4_OUT_F32))
+        return NVFP4_ERR_INVALID_ARG;
+    if (T == 0 || H == 0) return NVFP4_OK;
+    if (!y || !weights || !row_of || !out) return NVFP4_ERR_INVALID_ARG;
+    if (H % 8 != 0 || H > kMaxDim || k > 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(y) || !aligned16(out) || !aligned4(weights) || !aligned4(row_of)) return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_moe_combine(y, static_cast<int32_t>(y_dtype), weights, row_of, T, H, k, out,
+                                               static_cast<int32_t>(out_dtype), stream, d.num_sms));
 }
 
 nvfp4_status nvfp4_set_plan_override(int32_t bn, int32_t cluster, int32_t groups, int32_t band,

@@ -151,23 +151,29 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 }
 
 struct MapKey {
-    std::array<uint64_t, 11> v;
+    std::array<uint64_t, 18> v;
     bool operator<(const MapKey& o) const { return v < o.v; }
 };
 
 static std::mutex g_map_mu;
 static std::map<MapKey, CUtensorMap> g_map_cache;
 
-// uint8 tensor of `rank` (2 or 3) dims {inner bytes, rows[, depth]} with row stride
-// `stride1` and depth stride `stride2` (bytes); box {box0, box1[, 1]}.
-static bool get_map(CUtensorMap* out, const void* ptr, int rank, uint64_t d0, uint64_t d1,
-                    uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0, uint32_t box1,
-                    bool swizzle128)
+// uint8 tensor of `rank` (2 ... 5) dims (innermost first: dims[0] bytes per row), strides of
+// dims 1 .. rank-1 in bytes, box extents per dim; cached per (pointer, geometry, device).
+static bool get_map_nd(CUtensorMap* out, const void* ptr, int rank, const uint64_t* dims,
+                       const uint64_t* strides, const uint32_t* box, bool swizzle128)
 {
     int dev = 0;
     cudaGetDevice(&dev);
-    MapKey key{{reinterpret_cast<uint64_t>(ptr), static_cast<uint64_t>(rank), d0, d1, d2, stride1,
-                stride2, box0, box1, swizzle128 ? 1ull : 0ull, static_cast<uint64_t>(dev)}};
+    MapKey key;
+    key.v.fill(0);
+    key.v[0] = reinterpret_cast<uint64_t>(ptr);
+    key.v[1] = static_cast<uint64_t>(rank) | (swizzle128 ? 0x100ull : 0ull) | (static_cast<uint64_t>(dev) << 16);
+    for (int i = 0; i < rank; ++i) {
+        key.v[2 + i] = dims[i];
+        key.v[7 + i] = box[i];
+        if (i + 1 < rank) key.v[12 + i] = strides[i];
+    }
     {
         std::lock_guard<std::mutex> g(g_map_mu);
         auto it = g_map_cache.find(key);
@@ -178,14 +184,19 @@ static bool get_map(CUtensorMap* out, const void* ptr, int rank, uint64_t d0, ui
     }
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[3] = {d0, d1, d2};
-    cuuint64_t strides[2] = {stride1, stride2};
-    cuuint32_t box[3] = {box0, box1, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
+    cuuint64_t d[5];
+    cuuint64_t st[4];
+    cuuint32_t bx[5];
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        if (i + 1 < rank) st[i] = strides[i];
+    }
     CUtensorMap m;
     std::memset(&m, 0, sizeof(m));
-    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank),
-                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank), const_cast<void*>(ptr), d,
+                    st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
@@ -196,6 +207,31 @@ static bool get_map(CUtensorMap* out, const void* ptr, int rank, uint64_t d0, ui
     }
     *out = m;
     return true;
+}
+
+// uint8 tensor of `rank` (2 or 3) dims {inner bytes, rows[, depth]} with row stride
+// `stride1` and depth stride `stride2` (bytes); box {box0, box1[, 1]}.
+static bool get_map(CUtensorMap* out, const void* ptr, int rank, uint64_t d0, uint64_t d1,
+                    uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0, uint32_t box1,
+                    bool swizzle128)
+{
+    const uint64_t dims[3] = {d0, d1, d2};
+    const uint64_t strides[2] = {stride1, stride2};
+    const uint32_t box[3] = {box0, box1, 1};
+    return get_map_nd(out, ptr, rank, dims, strides, box, swizzle128);
+}
+
+// The gate_up weights [E, 2I, row_bytes] viewed so that one box of 128 rows holds four groups of
+// [16 gate rows j .. j + 15, the 16 up rows I + j .. I + j + 15]: dims (innermost first)
+// {row_bytes, 16 rows, gate/up, I / 16 groups, E}, strides {row_bytes, I rows, 16 rows,
+// 2I rows}, box {box0, 16, 2, 4, 1}.
+static bool get_map_swiglu(CUtensorMap* out, const void* ptr, uint64_t row_bytes, uint64_t I, uint64_t E,
+                           uint32_t box0, bool swizzle128)
+{
+    const uint64_t dims[5] = {row_bytes, 16, 2, I / 16, E};
+    const uint64_t strides[4] = {row_bytes, I * row_bytes, 16 * row_bytes, 2 * I * row_bytes};
+    const uint32_t box[5] = {box0, 16, 2, 4, 1};
+    return get_map_nd(out, ptr, 5, dims, strides, box, swizzle128);
 }
 
 // ------------------------------------------------------------------ launch
@@ -239,11 +275,11 @@ static int max_active_clusters(int cs)
     return cache[dev][cs] > 0 ? cache[dev][cs] : 0;
 }
 
-template <int BN, bool SWAP, bool GROUPED, bool SFT = false>
+template <int BN, bool SWAP, bool GROUPED, bool SFT = false, bool SWIGLU = false>
 static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
                        bool* encode_failed)
 {
-    using Cfg = GemmCfg<BN, SWAP, GROUPED, SFT>;
+    using Cfg = GemmCfg<BN, SWAP, GROUPED, SFT, SWIGLU>;
     auto kern = nvfp4_gemm_kernel<Cfg>;
     // Opt in to the large dynamic shared memory once per device (not a stream operation,
     // so a later launch may be captured into a CUDA graph).
@@ -271,14 +307,25 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
     a.N = static_cast<int32_t>(L.N);
     a.num_kstages = static_cast<int32_t>(L.K / 256);
     a.num_p_tiles = plan.p_tiles;
-    a.out = static_cast<__nv_bfloat16*>(L.out);
+    a.out = L.out;
+    a.out_dtype = L.out_dtype;
     a.alpha = L.alpha;
     a.err_word = L.err_word;
     if constexpr (GROUPED) {
         const uint64_t E = static_cast<uint64_t>(L.E);
         const uint64_t rows = static_cast<uint64_t>(L.total_rows);
-        ok &= get_map(&tp, L.B, 3, kb, L.N, E, kb, kb * L.N, 128, 128, true);
-        ok &= get_map(&tsp, L.sfB, 3, ks, L.N, E, ks, ks * L.N, 16, 128, false);
+        if constexpr (SWIGLU) {
+            const uint64_t I = static_cast<uint64_t>(L.N / 2);
+            ok &= get_map_swiglu(&tp, L.B, kb, I, E, 128, true);
+            ok &= get_map_swiglu(&tsp, L.sfB, ks, I, E, 16, false);
+            a.h_q = L.h_q;
+            a.h_sf = L.h_sf;
+            a.gs_h = L.gs_h;
+            a.inter = static_cast<int32_t>(I);
+        } else {
+            ok &= get_map(&tp, L.B, 3, kb, L.N, E, kb, kb * L.N, 128, 128, true);
+            ok &= get_map(&tsp, L.sfB, 3, ks, L.N, E, ks, ks * L.N, 16, 128, false);
+        }
         ok &= get_map(&tq, L.A, 2, kb, rows, 1, kb, 0, 128, Cfg::QBOX, true);
         ok &= get_map(&tsq, L.sfA, 2, ks, rows, 1, ks, 0, 16, Cfg::QBOX, false);
         a.p_rows = a.N;
@@ -362,6 +409,15 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
             case 128: return run<128, false, false, true>(plan, L, stream, encode_failed);
             case 256: return run<256, false, false, true>(plan, L, stream, encode_failed);
             default: return cudaErrorInvalidValue;      // 192 / 224 tiles: linear scales only
+        }
+    }
+    if (plan.grouped && L.h_q != nullptr) {
+        switch (plan.bn) {
+            case 32: return run<32, true, true, false, true>(plan, L, stream, encode_failed);
+            case 64: return run<64, true, true, false, true>(plan, L, stream, encode_failed);
+            case 128: return run<128, true, true, false, true>(plan, L, stream, encode_failed);
+            case 256: return run<256, true, true, false, true>(plan, L, stream, encode_failed);
+            default: return cudaErrorInvalidValue;
         }
     }
     if (plan.grouped) {

@@ -24,7 +24,8 @@
 //               replicates into the TMEM layout the MMA reads (row r at column base + r/32,
 //               byte = k-block). Warp 3 first builds the per-expert tile prefix (grouped).
 //   warps 4-11  epilogue, two warpgroups (one per half of the tile's columns; warp w reads
-//               TMEM lane quadrant w % 4): TMEM -> registers -> alpha -> bf16 -> global; with split-K,
+//               TMEM lane quadrant w % 4): TMEM -> registers -> alpha -> bf16 (or fp16, fp32)
+//               -> global; with split-K,
 //               the cluster's fp32 partials meet in shared memory (st.async over DSMEM)
 //               and are summed in a fixed rank order (deterministic); with several
 //               clusters per tile, through the workspace in a fixed group order.
@@ -35,6 +36,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -57,6 +59,9 @@ enum : uint32_t {
 constexpr int kEpilogueWarps = 8;
 constexpr int kGemmThreads = 32 * (4 + kEpilogueWarps);
 
+// Output element types (include/nvfp4.h, nvfp4_out_dtype).
+enum : int32_t { kOutBF16 = 0, kOutF16 = 1, kOutF32 = 2 };
+
 struct GemmArgs {
     int32_t M, N;             // output is out[M][N] (row-major, leading dimension N)
     int32_t p_rows, q_rows;   // rows of the P and Q operands (non-grouped)
@@ -68,7 +73,8 @@ struct GemmArgs {
     int32_t groups;           // clusters per output tile (reduced through the workspace)
     int32_t num_tiles;        // non-grouped: p_tiles * q_tiles * splits
     int32_t band;             // non-grouped: P tiles per rasterisation band (>= 1)
-    __nv_bfloat16* out;
+    void* out;                // out_dtype elements
+    int32_t out_dtype;        // kOutBF16, kOutF16 or kOutF32
     const float* alpha;       // [1] or [E]
     float* ws_partial;        // split-K fp32 partial tiles
     uint32_t* ws_counters;    // split-K per-tile arrival counters
@@ -79,13 +85,22 @@ struct GemmArgs {
     const int32_t* expert_offsets;  // grouped: [E + 1]
     int32_t num_experts;
     int32_t total_rows;       // grouped: rows of A / out
+    uint8_t* h_q;             // SWIGLU: NVFP4 codes of h [total_rows, I/2]
+    uint8_t* h_sf;            // SWIGLU: e4m3 scales of h [total_rows, I/16]
+    const float* gs_h;        // SWIGLU: global scale of h (device, 1)
+    int32_t inter;            // SWIGLU: I (gate rows = up rows), N = 2 I
 };
 
-template <int BN_, bool SWAP_, bool GROUPED_, bool SFT_ = false>
+template <int BN_, bool SWAP_, bool GROUPED_, bool SFT_ = false, bool SWIGLU_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;
     static constexpr bool SWAP = SWAP_;
     static constexpr bool GROUPED = GROUPED_;
+    // SWIGLU (grouped gate_up only): a P tile holds 64 gate rows and the 64 matching up rows,
+    // as four groups of [16 gate rows, 16 up rows] (one 5-D TMA view of the weights), and the
+    // epilogue writes h = silu(gate) * up quantised to NVFP4 instead of the product itself.
+    static constexpr bool SWIGLU = SWIGLU_;
+    static_assert(!SWIGLU || GROUPED, "the fused SwiGLU epilogue serves the grouped gate_up GEMM");
     // SFT: both operands' scales in the tiled layout (include/nvfp4.h, NVFP4_SF_TILED): a
     // stage's scales of 128 rows are one contiguous 2 KB run already in the tcgen05.cp source
     // layout, fetched by a bulk copy (no re-layout step). Q tiles then start on a 128-row
@@ -130,7 +145,10 @@ struct GemmCfg {
     static_assert(TMEM_USED <= 512, "TMEM budget");
 
     static constexpr int SMEM_LIMIT = 232448;      // max dynamic shared memory per block
-    static constexpr int MISC_BYTES = 1024 + (GROUPED ? 4 * (kMaxExperts + 1) : 0);
+    // SWIGLU: gs_h / e4m3 table (256 floats), per epilogue warp a 16-token x 8-byte code stage
+    // and a 16-byte scale stage
+    static constexpr int SWIGLU_BYTES = SWIGLU ? 1024 + kEpilogueWarps * (128 + 16) : 0;
+    static constexpr int MISC_BYTES = 1024 + (GROUPED ? 4 * (kMaxExperts + 1) : 0) + SWIGLU_BYTES;
     static constexpr int ALIGN_SLACK = 1024;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - MISC_BYTES - ALIGN_SLACK) / STAGE_BYTES;
     // Few-token (swap, non-grouped) launches split K finely and run a handful of stages per
@@ -150,8 +168,8 @@ struct GemmCfg {
     static constexpr int NUM_BARS = 3 * STAGES + 8;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;     // tmem base, flags
     static constexpr int OFF_PREFIX = OFF_MISC + 64;
-    static constexpr int SMEM_BYTES = OFF_PREFIX + (GROUPED ? 4 * (kMaxExperts + 1) : 0)
-                                    + ALIGN_SLACK;
+    static constexpr int OFF_SWIGLU = OFF_PREFIX + (GROUPED ? ((4 * (kMaxExperts + 1) + 15) & ~15) : 0);
+    static constexpr int SMEM_BYTES = OFF_SWIGLU + SWIGLU_BYTES + ALIGN_SLACK;
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     // split-K partial tile in shared memory: [128 rows][BN + 4 floats]
     static constexpr int PSTRIDE = BN + 4;
@@ -248,7 +266,42 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
     return r != 0;
 }
 
-// Store 16 consecutive accumulator columns (c .. c + 15) of P row `p` as bf16(alpha * v).
+// Two fp32 values -> one 32-bit word of the 16-bit output type (round to nearest even),
+// `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_out16x2(float lo, float hi, int32_t dt)
+{
+    return dt == kOutF16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+}
+
+// out[idx] = alpha * v in the output type (one element).
+__device__ __forceinline__ void store_out1(const GemmArgs& a, size_t idx, float v)
+{
+    if (a.out_dtype == kOutF32) static_cast<float*>(a.out)[idx] = v;
+    else if (a.out_dtype == kOutF16) static_cast<__half*>(a.out)[idx] = __float2half_rn(v);
+    else static_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(v);
+}
+
+// Eight consecutive output elements out[idx .. idx + 7] = v[0..7] (idx % 8 == 0): one 16-byte
+// store for 16-bit types, two for fp32.
+__device__ __forceinline__ void store_out8(const GemmArgs& a, size_t idx, const float (&v)[8])
+{
+    if (a.out_dtype == kOutF32) {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + idx);
+        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+        const int32_t dt = a.out_dtype;
+        uint4 w;
+        w.x = pack_out16x2(v[0], v[1], dt);
+        w.y = pack_out16x2(v[2], v[3], dt);
+        w.z = pack_out16x2(v[4], v[5], dt);
+        w.w = pack_out16x2(v[6], v[7], dt);
+        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + idx) = w;
+    }
+}
+
+// Store 16 consecutive accumulator columns (c .. c + 15) of P row `p` as alpha * v in the
+// output type.
 template <class Cfg>
 __device__ __forceinline__ void store_out16(const GemmArgs& a, const Tile& ti, int p, int c,
                                             const uint32_t (&r)[16], float alpha)
@@ -257,18 +310,12 @@ __device__ __forceinline__ void store_out16(const GemmArgs& a, const Tile& ti, i
         // thread owns output row m = p, columns n = q0 + c .. + 15 (N % 8 == 0)
         const int n0 = ti.q0 + c;
         if (p < a.M) {
-            __nv_bfloat16* dst = a.out + static_cast<size_t>(p) * a.N + n0;
-            uint4 w0, w1;
-            w0.x = pack_bf16x2(alpha * __uint_as_float(r[0]), alpha * __uint_as_float(r[1]));
-            w0.y = pack_bf16x2(alpha * __uint_as_float(r[2]), alpha * __uint_as_float(r[3]));
-            w0.z = pack_bf16x2(alpha * __uint_as_float(r[4]), alpha * __uint_as_float(r[5]));
-            w0.w = pack_bf16x2(alpha * __uint_as_float(r[6]), alpha * __uint_as_float(r[7]));
-            w1.x = pack_bf16x2(alpha * __uint_as_float(r[8]), alpha * __uint_as_float(r[9]));
-            w1.y = pack_bf16x2(alpha * __uint_as_float(r[10]), alpha * __uint_as_float(r[11]));
-            w1.z = pack_bf16x2(alpha * __uint_as_float(r[12]), alpha * __uint_as_float(r[13]));
-            w1.w = pack_bf16x2(alpha * __uint_as_float(r[14]), alpha * __uint_as_float(r[15]));
-            if (n0 < a.N) *reinterpret_cast<uint4*>(dst) = w0;
-            if (n0 + 8 < a.N) *reinterpret_cast<uint4*>(dst + 8) = w1;
+            const size_t idx = static_cast<size_t>(p) * a.N + n0;
+            float v[2][8];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j >> 3][j & 7] = alpha * __uint_as_float(r[j]);
+            if (n0 < a.N) store_out8(a, idx, v[0]);
+            if (n0 + 8 < a.N) store_out8(a, idx + 8, v[1]);
         }
     } else {
         // thread owns output column n = p; accumulator columns are output rows
@@ -281,31 +328,18 @@ __device__ __forceinline__ void store_out16(const GemmArgs& a, const Tile& ti, i
                 if constexpr (Cfg::GROUPED) valid = qi < ti.q_valid;
                 else valid = ti.q0 + qi < a.M;
                 if (valid)
-                    a.out[static_cast<size_t>(ti.q0 + qi) * a.N + n] =
-                        __float2bfloat16_rn(alpha * __uint_as_float(r[j]));
+                    store_out1(a, static_cast<size_t>(ti.q0 + qi) * a.N + n, alpha * __uint_as_float(r[j]));
             }
         }
     }
 }
 
-// Stores 64 accumulator columns (c0 .. c0 + 63) of the 32 rows a warp holds (lane = row,
-// non-swap tiles) as bf16(alpha * v), four rows x 128 contiguous bytes per store instruction.
-// A lane's row is eight 16-byte chunks (8 columns each); an 8 x 8 transpose of chunks within
-// each group of 8 lanes (three butterfly stages of shuffles: at stage m the lanes whose bit m
-// differs from the chunk index's swap those chunks) leaves lane 8 g + j holding chunk j of
-// rows 8 g .. 8 g + 7, so that lanes 8 g .. 8 g + 7 write one 128-byte row segment together.
-// (Stores straight from the row-per-lane layout would touch 32 lines per instruction.)
-template <class Cfg>
-__device__ __forceinline__ void store_rows64(const GemmArgs& a, const Tile& ti, int quad, int lane, int c0,
-                                             const uint32_t (&r)[4][16], float alpha)
+// An 8 x 8 transpose of 16-byte chunks within each group of 8 lanes (three butterfly stages of
+// shuffles: at stage m the lanes whose bit m differs from the chunk index's swap those
+// chunks): lane 8 g + j enters with chunks 0..7 of its own row and leaves with chunk j of
+// rows 8 g .. 8 g + 7 (w[t] = row 8 g + t).
+__device__ __forceinline__ void transpose_chunks8(uint32_t (&w)[8][4], int lane)
 {
-    uint32_t w[8][4];
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            w[e][k] = pack_bf16x2(alpha * __uint_as_float(r[e >> 1][(e & 1) * 8 + 2 * k]),
-                                  alpha * __uint_as_float(r[e >> 1][(e & 1) * 8 + 2 * k + 1]));
     const int j = lane & 7;
 #pragma unroll
     for (int m = 4; m >= 1; m >>= 1) {
@@ -322,14 +356,58 @@ __device__ __forceinline__ void store_rows64(const GemmArgs& a, const Tile& ti, 
             }
         }
     }
-    const int n = ti.q0 + c0 + 8 * j;
+}
+
+// Stores 64 accumulator columns (c0 .. c0 + 63) of the 32 rows a warp holds (lane = row,
+// non-swap tiles) as alpha * v in the output type, each store instruction writing 4 rows x 128
+// contiguous bytes. A lane's row is cut into 16-byte chunks (8 columns of a 16-bit type, 4 of
+// fp32); after transpose_chunks8, lanes 8 g .. 8 g + 7 write one 128-byte row segment together.
+// (Stores straight from the row-per-lane layout would touch 32 lines per instruction.)
+template <class Cfg>
+__device__ __forceinline__ void store_rows64(const GemmArgs& a, const Tile& ti, int quad, int lane, int c0,
+                                             const uint32_t (&r)[4][16], float alpha)
+{
+    const int j = lane & 7;
     const int m0 = ti.p0 + 32 * quad + (lane & ~7);
+    uint32_t w[8][4];
+    if (a.out_dtype == kOutF32) {
+        // two halves of 32 columns, 8 chunks of 4 fp32 each
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    w[e][k] = __float_as_uint(alpha * __uint_as_float(r[2 * h + (e >> 2)][(e & 3) * 4 + k]));
+            transpose_chunks8(w, lane);
+            const int n = ti.q0 + c0 + 32 * h + 4 * j;
+            if (n < a.N) {
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const int m = m0 + t;
+                    if (m < a.M)
+                        *reinterpret_cast<uint4*>(static_cast<float*>(a.out) + static_cast<size_t>(m) * a.N + n) =
+                            make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
+                }
+            }
+        }
+        return;
+    }
+    const int32_t dt = a.out_dtype;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[e][k] = pack_out16x2(alpha * __uint_as_float(r[e >> 1][(e & 1) * 8 + 2 * k]),
+                                   alpha * __uint_as_float(r[e >> 1][(e & 1) * 8 + 2 * k + 1]), dt);
+    transpose_chunks8(w, lane);
+    const int n = ti.q0 + c0 + 8 * j;
     if (n < a.N) {
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
             const int m = m0 + t;
             if (m < a.M)
-                *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(m) * a.N + n) =
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + static_cast<size_t>(m) * a.N + n) =
                     make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
         }
     }
@@ -343,9 +421,9 @@ __device__ __forceinline__ int chunk_owner(int row, int cs) { return ((row >> 3)
 
 // Writes a reduced chunk of a tile: rows [r0, r0 + rows) of the 128 x BN accumulator tile,
 // each the in-order sum of `nsrc` fp32 copies in shared memory (copy j, chunk row lr, column
-// c at src[(j * rows + lr) * PSTRIDE + c]), times alpha, as bf16. All 128 epilogue threads
-// (tid) take part; every store is 16 bytes (8 bf16) and consecutive threads write
-// consecutive addresses.
+// c at src[(j * rows + lr) * PSTRIDE + c]), times alpha, in the output type. All 128 epilogue
+// threads (tid) take part; each writes 8 consecutive outputs (16 bytes, or 32 for fp32) and
+// consecutive threads write consecutive addresses.
 template <class Cfg>
 __device__ __forceinline__ void store_chunk(const GemmArgs& a, const Tile& ti, const float* src, int nsrc,
                                             int r0, int rows, int tid, float alpha)
@@ -371,12 +449,9 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& a, const Tile& ti, c
             const int m = ti.p0 + r0 + lr;
             const int n0 = ti.q0 + c;
             if (m < a.M && n0 < a.N) {
-                uint4 w;
-                w.x = pack_bf16x2(alpha * v[0], alpha * v[1]);
-                w.y = pack_bf16x2(alpha * v[2], alpha * v[3]);
-                w.z = pack_bf16x2(alpha * v[4], alpha * v[5]);
-                w.w = pack_bf16x2(alpha * v[6], alpha * v[7]);
-                *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(m) * a.N + n0) = w;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) v[t] *= alpha;
+                store_out8(a, static_cast<size_t>(m) * a.N + n0, v);
             }
         }
     } else {
@@ -397,15 +472,96 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& a, const Tile& ti, c
             const int m = ti.q0 + c;
             const int n0 = ti.p0 + r0 + lr;
             if (m < a.M && n0 < a.N) {
-                uint4 w;
-                w.x = pack_bf16x2(alpha * v[0], alpha * v[1]);
-                w.y = pack_bf16x2(alpha * v[2], alpha * v[3]);
-                w.z = pack_bf16x2(alpha * v[4], alpha * v[5]);
-                w.w = pack_bf16x2(alpha * v[6], alpha * v[7]);
-                *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(m) * a.N + n0) = w;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) v[t] *= alpha;
+                store_out8(a, static_cast<size_t>(m) * a.N + n0, v);
             }
         }
     }
+}
+
+// fp32 -> e4m3fn byte, round to nearest even, finite values saturate to +-448.
+__device__ __forceinline__ uint32_t f32_to_e4m3_byte(float v)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(v), "f"(v));
+    return r & 0xFFu;
+}
+
+// e4m3fn byte -> fp32 (exact).
+__device__ __forceinline__ float e4m3_byte_to_f32(uint32_t byte)
+{
+    const uint16_t pair = static_cast<uint16_t>(byte | (byte << 8));
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// fp32 -> e2m1 code (round to nearest even, saturating at +-6, sign kept) in bits 0..3.
+__device__ __forceinline__ uint32_t f32_to_e2m1_code(float v)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\t"
+        "mov.b32 %0, {t, 0, 0, 0};\n\t}"
+        : "=r"(r)
+        : "f"(v));
+    return r & 0xFu;
+}
+
+// SwiGLU + NVFP4 epilogue of 16 accumulator columns (tokens c .. c + 15 of the tile) in one
+// warp of TMEM lane quadrant `quad`: P rows 32 quad + i (i < 16) are gate row j0 + 16 quad + i
+// and P rows 32 quad + 16 + i the up row of the same index (j0 = p0 / 2), so that lane i and
+// lane 16 + i hold g and u of intermediate index j = j0 + 16 quad + i, and each half-warp's 16
+// indices are one NVFP4 block of h. After one exchange lane i (i < 16) holds (g, u) of tokens
+// c .. c + 7 and lane 16 + i those of tokens c + 8 .. c + 15:
+//     g, u = alpha * acc;   h = (g / (1 + exp(-g))) * u     (fp32, CUDA's expf)
+// then the quantiser's steps for the 16 values of a token (a half-warp), with the fixed
+// global scale gs_h, in fp32 with explicit rounding and in this order:
+//     amax -> s = e4m3(amax / 6 * gs_h) -> r = s ? gs_h / s : 0 -> codes e2m1(h * r)
+// (rcp_tab[s] = gs_h / e4m3(s), as the quantiser builds it). Codes go through the warp's
+// stage (16 tokens x 8 bytes) and leave as one 8-byte store per token; the scale as one byte.
+template <class Cfg>
+__device__ __forceinline__ void swiglu_chunk16(const GemmArgs& a, const Tile& ti, int quad, int lane, int c,
+                                               const uint32_t (&r)[16], float alpha, float gsh,
+                                               const float* rcp_tab, uint8_t* stage, uint8_t* sstage)
+{
+    const bool up = lane >= 16;
+    const int i = lane & 15;
+    float h[8];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        const float lo = alpha * __uint_as_float(r[cc]);        // token c + cc
+        const float hi = alpha * __uint_as_float(r[cc + 8]);    // token c + 8 + cc
+        const float other = __shfl_xor_sync(0xffffffffu, up ? lo : hi, 16);
+        const float g = up ? other : lo;
+        const float u = up ? hi : other;
+        h[cc] = (g / (1.0f + expf(-g))) * u;
+    }
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        float amax = fabsf(h[cc]);
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const uint32_t sfq = f32_to_e4m3_byte(__fmul_rn(__fdiv_rn(amax, 6.0f), gsh));
+        const uint32_t code = f32_to_e2m1_code(__fmul_rn(h[cc], rcp_tab[sfq]));
+        const uint32_t hi_code = __shfl_xor_sync(0xffffffffu, code, 1);
+        const int tok = cc + (up ? 8 : 0);
+        if ((i & 1) == 0) stage[tok * 8 + (i >> 1)] = static_cast<uint8_t>(code | (hi_code << 4));
+        if (i == 0) sstage[tok] = static_cast<uint8_t>(sfq);
+    }
+    __syncwarp();
+    if (lane < 16) {
+        const int tok = c + lane;
+        if (tok < ti.q_valid) {
+            const size_t row = static_cast<size_t>(ti.q0 + tok);
+            const int blk = (ti.p0 >> 5) + quad;          // 16-element block of h: j0 / 16 + quad
+            *reinterpret_cast<uint2*>(a.h_q + row * (a.inter >> 1) + blk * 8) =
+                *reinterpret_cast<const uint2*>(stage + lane * 8);
+            a.h_sf[row * (a.inter >> 4) + blk] = sstage[lane];
+        }
+    }
+    __syncwarp();
 }
 
 // Split-K epilogue of one CTA, run by the 128 threads of the first epilogue warpgroup
@@ -680,8 +836,15 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                         const int boxes = (n_mma + Cfg::QBOX - 1) / Cfg::QBOX;
                         mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::SF_TMA_P +
                                                   static_cast<uint32_t>(boxes * Cfg::QBOX * (Cfg::BK_BYTES + 16)));
-                        tma_load_3d(pbuf, &tm_p, fb, kx, ti.p0, ti.expert, pol_p);
-                        tma_load_3d(sfpb, &tm_sfp, fb, sx, ti.p0, ti.expert, pol_p);
+                        if constexpr (Cfg::SWIGLU) {
+                            // 4 groups x [16 gate rows, 16 up rows] of intermediate indices
+                            // [p0 / 2, p0 / 2 + 64): group coordinate (p0 / 2) / 16
+                            tma_load_5d(pbuf, &tm_p, fb, kx, 0, 0, ti.p0 >> 5, ti.expert, pol_p);
+                            tma_load_5d(sfpb, &tm_sfp, fb, sx, 0, 0, ti.p0 >> 5, ti.expert, pol_p);
+                        } else {
+                            tma_load_3d(pbuf, &tm_p, fb, kx, ti.p0, ti.expert, pol_p);
+                            tma_load_3d(sfpb, &tm_sfp, fb, sx, ti.p0, ti.expert, pol_p);
+                        }
                         for (int b = 0; b < boxes; ++b) {
                             tma_load_2d(qbuf + b * Cfg::QBOX * Cfg::BK_BYTES, &tm_q, fb, kx,
                                         ti.q0 + b * Cfg::QBOX, pol_q);
@@ -847,6 +1010,18 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
         const int half = (warp - 4) >> 2;
         const int row = 32 * quad + lane;          // accumulator row (P row within the tile)
+        float gsh = 0.0f;
+        float* rcp_tab = reinterpret_cast<float*>(smem + Cfg::OFF_SWIGLU);
+        uint8_t* stage_w = smem + Cfg::OFF_SWIGLU + 1024 + (warp - 4) * 128;
+        uint8_t* sstage_w = smem + Cfg::OFF_SWIGLU + 1024 + kEpilogueWarps * 128 + (warp - 4) * 16;
+        if constexpr (Cfg::SWIGLU) {
+            // gs_h / e4m3(s) for all 256 scale codes, once per CTA (one entry per epilogue thread)
+            gsh = __ldg(args.gs_h);
+            const uint32_t code = threadIdx.x - 128;
+            const float sfd = e4m3_byte_to_f32(code);
+            rcp_tab[code] = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gsh, sfd);
+            named_bar_sync(1, 32 * kEpilogueWarps);
+        }
         uint32_t acc = 0, acc_phase = 0;
         for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
@@ -893,6 +1068,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     if (need) {
                         if constexpr (!Cfg::SWAP && !Cfg::GROUPED) {
                             store_rows64<Cfg>(args, ti, quad, lane, BN - 64, r, alpha);
+                        } else if constexpr (Cfg::SWIGLU) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                if (BN - 64 + 16 * i < n_cols)
+                                    swiglu_chunk16<Cfg>(args, ti, quad, lane, BN - 64 + 16 * i, r[i], alpha, gsh,
+                                                        rcp_tab, stage_w, sstage_w);
                         } else {
 #pragma unroll
                             for (int i = 0; i < 4; ++i)
@@ -932,7 +1113,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     for (int h = 0; h < 2; ++h) {
                         if (h == 1 && !two) break;
                         const int c = c0 + 16 * h;
-                        store_out16<Cfg>(args, ti, p, c, r[h], alpha);
+                        if constexpr (Cfg::SWIGLU)
+                            swiglu_chunk16<Cfg>(args, ti, quad, lane, c, r[h], alpha, gsh, rcp_tab, stage_w, sstage_w);
+                        else
+                            store_out16<Cfg>(args, ti, p, c, r[h], alpha);
                     }
                 }
             }

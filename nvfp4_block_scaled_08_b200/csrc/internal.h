@@ -20,6 +20,19 @@ cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int6
                                     float* gs_out, uint8_t* q, uint8_t* sf, bool sf_tiled,
                                     const float* gs_other, int32_t n_alpha, float* alpha_out,
                                     unsigned* err_word, cudaStream_t stream, int num_sms);
+// Dynamic quantisation of x[T, H] (global scale over all of x) with every row t's codes and
+// scales written to the k rows row_of[t k + s] of q[T k, H/2] and sf[T k, H/16] (linear).
+cudaError_t launch_gather_quantize(const void* x, bool bf16, int64_t T, int64_t H, int64_t ldx, int32_t k,
+                                   const int32_t* row_of, float* gs_out, uint8_t* q, uint8_t* sf,
+                                   const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                   unsigned* err_word, cudaStream_t stream, int num_sms);
+// moe.cu: top-k routing and the expert-sorted permutation (three launches), the combine.
+cudaError_t launch_moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t* experts,
+                             float* weights, int32_t* offsets, int32_t* row_of, int32_t* token_of_row,
+                             cudaStream_t stream);
+cudaError_t launch_moe_combine(const void* y, int32_t y_dt, const float* weights, const int32_t* row_of,
+                               int32_t T, int64_t H, int32_t k, void* out, int32_t out_dt, cudaStream_t stream,
+                               int num_sms);
 cudaError_t launch_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* out, cudaStream_t stream,
                            int num_sms);
 cudaError_t launch_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
@@ -59,6 +72,13 @@ struct GemmLaunch {
     void* ws;
     unsigned* err_word;
     bool sf_tiled = false;      // sfA and sfB in the tiled layout (dense GEMM only)
+    int32_t out_dtype = 0;      // nvfp4_out_dtype of out
+    // grouped gate_up with the fused SwiGLU + NVFP4 epilogue (h_q != nullptr): B holds gate rows
+    // [0, N/2) and up rows [N/2, N) per expert; h = silu(gate) * up is written as codes h_q
+    // [total_rows, N/4] and e4m3 scales h_sf [total_rows, N/32] with the global scale gs_h
+    uint8_t* h_q = nullptr;
+    uint8_t* h_sf = nullptr;
+    const float* gs_h = nullptr;
 };
 
 // api.cu: nvfp4_status of the current device's checks; fills the SM count and the device

@@ -284,10 +284,46 @@ __device__ __forceinline__ void build_rcp_table(float gs, float* rcp_tab)
     __syncthreads();
 }
 
-template <typename T, typename Src>
+// Where the codes and scale of vector i go.
+// DenseDst: the codes of vector i at q + 4 i, its block scale through SfOut (row-major order).
+struct DenseDst {
+    uint8_t* q;
+    SfOut sfo;
+    static constexpr bool kContiguous = true;   // codes of vector i at q + 4 i
+    template <int TPB>
+    __device__ __forceinline__ void store(uint32_t i, uint32_t packed, uint32_t sfq, bool leader) const
+    {
+        *reinterpret_cast<uint32_t*>(q + static_cast<int64_t>(i) * 4) = packed;
+        if (leader) *sfo.at<TPB>(i) = static_cast<uint8_t>(sfq);
+    }
+};
+
+// ScatterDst: row t of the input goes to the k rows row_of[t k + s] (s < k) of the output
+// (codes [rows_out][vpr * 4] bytes, linear scales [rows_out][vpr / 2]): the expert-sorted
+// activations of a mixture-of-experts layer, quantised once per token.
+struct ScatterDst {
+    uint8_t* q;
+    uint8_t* sf;
+    const int32_t* row_of;
+    int32_t k;
+    uint32_t vpr, mul, shift;    // vector -> input row, as in VecIndex
+    static constexpr bool kContiguous = false;
+    template <int TPB>
+    __device__ __forceinline__ void store(uint32_t i, uint32_t packed, uint32_t sfq, bool leader) const
+    {
+        const uint32_t t = static_cast<uint32_t>((static_cast<uint64_t>(__umulhi(i, mul)) + i) >> shift);
+        const uint32_t c = i - t * vpr;
+        for (int s = 0; s < k; ++s) {
+            const int64_t row = __ldg(row_of + static_cast<int64_t>(t) * k + s);
+            *reinterpret_cast<uint32_t*>(q + row * (static_cast<int64_t>(vpr) * 4) + c * 4) = packed;
+            if (leader) sf[row * (static_cast<int64_t>(vpr) / TPB) + c / TPB] = static_cast<uint8_t>(sfq);
+        }
+    }
+};
+
+template <typename T, typename Src, typename Dst>
 __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint32_t end, uint32_t step,
-                                               float gs, const float* rcp_tab, uint8_t* __restrict__ q,
-                                               const SfOut& sfo)
+                                               float gs, const float* rcp_tab, const Dst& dst)
 {
     constexpr int V = InTraits<T>::kPerThread;   // elements per thread (8)
     static_assert(V == 8, "8 elements per lane: 4 bytes of codes");
@@ -316,11 +352,7 @@ __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint
             const uint32_t sfq = f32_to_e4m3(sf32);
             const float rcp = rcp_tab[sfq];
             const uint32_t packed = scale_to_e2m1x8(v[u], rcp);
-            if (i < end) {
-                uint8_t* dst = q + static_cast<int64_t>(i) * (V / 2);
-                *reinterpret_cast<uint32_t*>(dst) = packed;        // V == 8: 4 bytes of codes
-                if ((lane & (TPB - 1)) == 0) *sfo.at<TPB>(i) = static_cast<uint8_t>(sfq);
-            }
+            if (i < end) dst.template store<TPB>(i, packed, sfq, (lane & (TPB - 1)) == 0);
         }
     }
 }

@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, 
     const float gs = __ldg(gs_ptr);
     build_rcp_table(gs, rcp_tab);
     quantize_sweep<T>(GlobalVecs<T>{x, ix}, blockIdx.x * blockDim.x + (threadIdx.x & ~31u), nv,
-                      gridDim.x * blockDim.x, gs, rcp_tab, q, sfo);
+                      gridDim.x * blockDim.x, gs, rcp_tab, DenseDst{q, sfo});
 }
 
 // One cooperative launch: amax of the whole tensor -> grid barrier -> global scale (and the
@@ -80,16 +80,17 @@ __global__ void __launch_bounds__(512) quantize_kernel(const T* __restrict__ x, 
 // the tensor grid-strided twice (the second time mostly from L2).
 // The per-block maxima are parked in the first 4 * gridDim.x bytes of q, followed by one
 // "read" flag per block (cleared before the barrier, set once the block has read every
-// maximum). Only the blocks whose codes overwrite that area wait for all flags; the launcher
-// keeps gridDim.x * 8 <= rows * K / 2. The wait is bounded; on a timeout the kernel records
-// kErrQuantFlags in err_word and goes on.
+// maximum). Only the blocks whose codes overwrite that area wait for all flags (every block,
+// when the codes are scattered); the launcher keeps gridDim.x * 8 <= the bytes of q. The wait
+// is bounded; on a timeout the kernel records kErrQuantFlags in err_word and goes on (the
+// codes of that call are then undefined).
 constexpr uint32_t kFlagRead = 0x52454144u;
 constexpr uint32_t kErrQuantFlags = 0x201;
 
-template <typename T, bool RESIDENT, int THREADS>
+template <typename T, bool RESIDENT, int THREADS, class Dst>
 __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
     const T* __restrict__ x, const VecIndex ix, uint32_t nv, uint32_t chunk,
-    float* __restrict__ gs_out, uint8_t* __restrict__ q, const SfOut sfo,
+    float* __restrict__ gs_out, uint8_t* __restrict__ q, const Dst dst,
     const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out,
     unsigned* __restrict__ err_word)
 {
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
 
     // this block's first code byte; the parked area is q[0, 8 * nblocks)
     const uint32_t first_vec = RESIDENT ? v0 : bid * blockDim.x;
-    if (static_cast<uint64_t>(first_vec) * (V / 2) < 8ull * nblocks) {
+    if (!Dst::kContiguous || static_cast<uint64_t>(first_vec) * (V / 2) < 8ull * nblocks) {
         // every thread watches its own flags (one L2 round trip, not one per block)
         const uint64_t t0 = globaltimer_ns();
         bool late = false;
@@ -155,10 +156,10 @@ __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
     __shared__ float rcp_tab[256];
     build_rcp_table(gs, rcp_tab);
     if constexpr (RESIDENT) {
-        quantize_sweep<T>(StashVecs<T>{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sfo);
+        quantize_sweep<T>(StashVecs<T>{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, dst);
     } else {
         quantize_sweep<T>(GlobalVecs<T>{x, ix}, bid * blockDim.x + (threadIdx.x & ~31u), nv,
-                          nblocks * blockDim.x, gs, rcp_tab, q, sfo);
+                          nblocks * blockDim.x, gs, rcp_tab, dst);
     }
 }
 
@@ -167,10 +168,10 @@ __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
 // memory and reduces its maximum, the cluster exchanges the per-CTA maxima through
 // distributed shared memory, and every CTA quantises its share from shared memory.
 // gridDim = (1, cluster size, 1).
-template <typename T>
+template <typename T, class Dst>
 __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
     const T* __restrict__ x, const VecIndex ix, uint32_t nv, uint32_t chunk,
-    float* __restrict__ gs_out, uint8_t* __restrict__ q, const SfOut sfo,
+    float* __restrict__ gs_out, const Dst dst,
     const float* __restrict__ gs_other, int32_t n_alpha, float* __restrict__ alpha_out)
 {
     extern __shared__ uint4 stash_raw[];
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
     cudaTriggerProgrammaticLaunchCompletion();
     __shared__ float rcp_tab[256];
     build_rcp_table(gs, rcp_tab);
-    quantize_sweep<T>(StashVecs<T>{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, q, sfo);
+    quantize_sweep<T>(StashVecs<T>{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, dst);
     cluster_wait();                                   // no CTA leaves while a peer may read it
 }
 
@@ -323,7 +324,7 @@ cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, i
 }
 
 // Largest cluster (16, else 8) of 512-thread quantiser CTAs the device runs; cached.
-template <typename T>
+template <typename T, class Dst>
 static int quantize_cluster_size()
 {
     static int cached[64];
@@ -332,7 +333,7 @@ static int quantize_cluster_size()
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return 0; }
     std::lock_guard<std::mutex> g(mu);
     if (cached[dev] == 0) {
-        auto kern = quantize_dynamic_cluster_kernel<T>;
+        auto kern = quantize_dynamic_cluster_kernel<T, Dst>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         int best = -1;
         for (int cs : {16, 8}) {
@@ -372,9 +373,9 @@ static inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * 
 // per thread, and room for the parked maxima and flags (8 bytes per block) in q. Each block
 // keeps its share in shared memory when it fits (about 200 KB per SM); otherwise the tensor
 // is swept twice.
-template <typename T, int THREADS, int BPS>
+template <typename T, int THREADS, int BPS, class Dst>
 static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float* gs_out, uint8_t* q,
-                               const SfOut& sf, const float* gs_other, int32_t n_alpha, float* alpha_out,
+                               const Dst& sf, const float* gs_other, int32_t n_alpha, float* alpha_out,
                                int64_t q_bytes, unsigned* err_word, cudaStream_t stream, int num_sms)
 {
     constexpr int64_t kResidentMaxBytes = (int64_t(200) << 10) / BPS;
@@ -385,14 +386,14 @@ static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float
     int64_t chunk = round_up((nv + blocks - 1) / blocks, 32);
     constexpr int64_t kVecBytes = sizeof(typename InTraits<T>::Raw);
     const bool resident = chunk * kVecBytes <= kResidentMaxBytes;
-    void (*kern)(const T*, const VecIndex, uint32_t, uint32_t, float*, uint8_t*, const SfOut, const float*,
+    void (*kern)(const T*, const VecIndex, uint32_t, uint32_t, float*, uint8_t*, const Dst, const float*,
                  int32_t, float*, unsigned*) =
-        resident ? quantize_dynamic_kernel<T, true, THREADS> : quantize_dynamic_kernel<T, false, THREADS>;
+        resident ? quantize_dynamic_kernel<T, true, THREADS, Dst> : quantize_dynamic_kernel<T, false, THREADS, Dst>;
     size_t smem = 0;
     if (resident) {
         static std::once_flag once;
         std::call_once(once, [] {
-            cudaFuncSetAttribute(quantize_dynamic_kernel<T, true, THREADS>,
+            cudaFuncSetAttribute(quantize_dynamic_kernel<T, true, THREADS, Dst>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kResidentMaxBytes));
         });
         smem = static_cast<size_t>(chunk) * kVecBytes;
@@ -438,23 +439,21 @@ static cudaError_t launch_coop(const T* x, const VecIndex& ix, int64_t nv, float
     return le;
 }
 
-template <typename T>
-static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64_t ldx, int64_t K,
-                                    float* gs_out, uint8_t* q, uint8_t* sf_ptr, bool sf_tiled,
+template <typename T, class Dst>
+static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, const VecIndex& ix, int64_t K,
+                                    float* gs_out, uint8_t* q, const Dst& sf,
                                     const float* gs_other, int32_t n_alpha, float* alpha_out,
                                     int64_t q_bytes, unsigned* err_word, cudaStream_t stream, int num_sms)
 {
     const int64_t bytes = rows * K * static_cast<int64_t>(sizeof(T));
     const int64_t nv = rows * vpr;                       // < 2^31 (checked by the caller)
-    const VecIndex ix = make_vec_index(vpr, ldx, K);
-    const SfOut sf = make_sf_out(sf_ptr, sf_tiled, ix, K);
-    const int ccs = bytes <= kClusterQuantizeMaxBytes ? quantize_cluster_size<T>() : 0;
+    const int ccs = bytes <= kClusterQuantizeMaxBytes ? quantize_cluster_size<T, Dst>() : 0;
     if (ccs > 0) {
         const int cs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ccs, (nv + 511) / 512)));
         const int64_t chunk = round_up((nv + cs - 1) / cs, 32);
         if (chunk * static_cast<int64_t>(sizeof(typename InTraits<T>::Raw)) > kClusterStashMaxBytes)
             return cudaErrorInvalidValue;
-        auto kern = quantize_dynamic_cluster_kernel<T>;
+        auto kern = quantize_dynamic_cluster_kernel<T, Dst>;
         static std::once_flag once;
         std::call_once(once, [&] {
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -476,7 +475,7 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, int64
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         return cudaLaunchKernelEx(&cfg, kern, x, ix, static_cast<uint32_t>(nv), static_cast<uint32_t>(chunk),
-                                  gs_out, q, sf, gs_other, n_alpha, alpha_out);
+                                  gs_out, sf, gs_other, n_alpha, alpha_out);
     }
 
     if (bytes <= kCoopSmallBytes)
@@ -494,10 +493,29 @@ cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int6
     const int V = 8;                       // elements per vector (quant_core.cuh)
     const int64_t vpr = K / V;
     const int64_t q_bytes = rows * (K / 2);
+    const VecIndex ix = make_vec_index(vpr, ldx, K);
+    const DenseDst dst{q, make_sf_out(sf, sf_tiled, ix, K)};
     if (bf16)
-        return launch_dynamic_t(static_cast<const __nv_bfloat16*>(x), rows, vpr, ldx, K, gs_out, q, sf, sf_tiled,
+        return launch_dynamic_t(static_cast<const __nv_bfloat16*>(x), rows, vpr, ix, K, gs_out, q, dst,
                                 gs_other, n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
-    return launch_dynamic_t(static_cast<const float*>(x), rows, vpr, ldx, K, gs_out, q, sf, sf_tiled, gs_other,
+    return launch_dynamic_t(static_cast<const float*>(x), rows, vpr, ix, K, gs_out, q, dst, gs_other,
+                            n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
+}
+
+cudaError_t launch_gather_quantize(const void* x, bool bf16, int64_t T, int64_t H, int64_t ldx, int32_t k,
+                                   const int32_t* row_of, float* gs_out, uint8_t* q, uint8_t* sf,
+                                   const float* gs_other, int32_t n_alpha, float* alpha_out,
+                                   unsigned* err_word, cudaStream_t stream, int num_sms)
+{
+    const int V = 8;                       // elements per vector (quant_core.cuh)
+    const int64_t vpr = H / V;
+    const int64_t q_bytes = T * k * (H / 2);
+    const VecIndex ix = make_vec_index(vpr, ldx, H);
+    const ScatterDst dst{q, sf, row_of, k, ix.vpr, ix.mul, ix.shift};
+    if (bf16)
+        return launch_dynamic_t(static_cast<const __nv_bfloat16*>(x), T, vpr, ix, H, gs_out, q, dst,
+                                gs_other, n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
+    return launch_dynamic_t(static_cast<const float*>(x), T, vpr, ix, H, gs_out, q, dst, gs_other,
                             n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
 }
 

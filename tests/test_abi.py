@@ -83,6 +83,18 @@ def test_noalloc_host_validation_matches_gemm(lib, bad):
     assert _noalloc(lib, **bad) == _gemm(lib, **bad)
 
 
+def test_out_dtype_host_validation(lib):
+    g = lib.nvfp4_gemm_ex2
+    base = (0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 16, 768, 6144, None, 0, 0)
+    assert g(*base, 3, None) == 1                    # bad out_dtype
+    assert g(*base, -1, None) == 1
+    assert g(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6008, 16, 768, 6144, None, 0, 0, 2, None) == 3
+    gg = lib.nvfp4_grouped_gemm_ex
+    args = (0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x8000, 256, 4096, 4096, 6144, 0x6000)
+    assert gg(*args, 3, None) == 1
+    assert gg(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x8000, 256, 4096, 4096, 6000, 0x6000, 1, None) == 2
+
+
 def test_plan_override_validation(lib):
     assert lib.nvfp4_set_plan_override(-1, 0, 0, 0, 0) == 1
     assert lib.nvfp4_set_plan_override(0, 0, -2, 0, 0) == 1
