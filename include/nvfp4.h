@@ -210,6 +210,44 @@ nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t*
                             nvfp4_sf_layout sf_layout, nvfp4_out_dtype out_dtype, cudaStream_t stream);
 
 /*
+ * MXFP4: the mm_fp4 variant that use_nvfp4=False selects ("The Art of Reading the Manual",
+ * section "The Message"; the pages name it without defining it). The library's reading is
+ * OCP Microscaling v1.0 FP4: e2m1 elements as above, one E8M0 scale byte per 32 consecutive K
+ * elements (value 2^(byte - 127); 255 is NaN and never written) and no per-tensor scale.
+ *
+ * nvfp4_mx_quantize: for every row and 32-element block, with amax = max|x| (fp32):
+ *     shared_exp = floor(log2(amax)) - 2, clamped to [-127, 127] (all-zero block: -127),
+ *     byte = shared_exp + 127,  code_k = e2m1_rn_satfinite(x_k * 2^-shared_exp)
+ * (elements in (6, 8) * 2^shared_exp saturate to 6). x[rows, K] fp32 or bf16 (row stride
+ * ld_x), q[rows, K/2] as for NVFP4, sf: E8M0 bytes in the given layout: NVFP4_SF_LINEAR
+ * [rows][K/32], or NVFP4_SF_TILED: the NVFP4 tiled layout with K/32 scale columns (512-byte
+ * blocks of 128 rows x 4 scales; row r, column c = k / 32 at
+ * ((r / 128) * (K / 128) + c / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4, rows padded
+ * to 128; K % 128 == 0). One launch, no reduction across blocks. K % 32 == 0.
+ */
+nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
+                               int64_t ld_x, uint8_t* q, uint8_t* sf, nvfp4_sf_layout sf_layout,
+                               cudaStream_t stream);
+
+/* Bytes of an MXFP4 scale matrix of `rows` rows and K elements per row in the given layout. */
+size_t nvfp4_mx_sf_bytes(int64_t rows, int64_t K, nvfp4_sf_layout sf_layout);
+
+/* Re-lays row-major MXFP4 scales [rows][K/32] out as NVFP4_SF_TILED (K % 128 == 0). */
+nvfp4_status nvfp4_mx_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* sf_tiled,
+                              cudaStream_t stream);
+
+/*
+ * MXFP4 GEMM: out[M, N] = alpha[0] * sum_k deq(A)[m, k] deq(B)[n, k] in out_dtype, with
+ * deq(X)[r, k] = e2m1(X[r, k]) * 2^(sfX[r, k / 32] - 127). A, B as for nvfp4_gemm; sfA, sfB:
+ * E8M0 scales in the tiled layout (nvfp4_mx_sf_bytes(rows, K, NVFP4_SF_TILED) bytes each, from
+ * nvfp4_mx_quantize or nvfp4_mx_sf_tile). alpha is a required device scalar (1 for plain MX).
+ * Same shape rules, split-K workspace rules and determinism as nvfp4_gemm.
+ */
+nvfp4_status nvfp4_mx_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                           const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
+                           size_t ws_bytes, nvfp4_out_dtype out_dtype, cudaStream_t stream);
+
+/*
  * Grouped (mixture-of-experts) NVFP4 GEMM ("When a Benchmark Crashes", section "Why This
  * Message Was Written": 256 experts, 8 active per token). Rows of A are sorted by expert;
  * expert e owns rows [expert_offsets[e], expert_offsets[e+1]) and computes

@@ -31,7 +31,7 @@ __all__ = [
     "Nvfp4Error", "load", "global_scale", "quantize", "quantize_dynamic", "alpha", "gemm", "gemm_workspace_size",
     "gemm_noalloc", "plan_override",
     "make_workspace", "grouped_gemm", "grouped_gemm_swiglu", "moe_route", "moe_gather_quantize",
-    "moe_combine", "round_e4m3", "round_e2m1", "last_device_error",
+    "moe_combine", "mx_quantize", "mx_sf_tile", "mx_sf_bytes", "mx_gemm", "round_e4m3", "round_e2m1", "last_device_error",
     "STATUS",
 ]
 
@@ -80,6 +80,10 @@ SIGNATURES = {
     "nvfp4_moe_gather_quantize": (ctypes.c_int, [_P, ctypes.c_int, _I32, _I64, _I64, _I32, _P, _P, _P, _P, _P,
                                                  _I32, _P, _P]),
     "nvfp4_moe_combine": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _I32, _I64, _I32, _P, ctypes.c_int, _P]),
+    "nvfp4_mx_quantize": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P, ctypes.c_int, _P]),
+    "nvfp4_mx_sf_bytes": (_SZ, [_I64, _I64, ctypes.c_int]),
+    "nvfp4_mx_sf_tile": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "nvfp4_mx_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int, _P]),
     "nvfp4_grouped_gemm_workspace_size": (_SZ, [_I32, _I64, _I64, _I64]),
     "nvfp4_grouped_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
                                           _SZ, _P]),
@@ -336,6 +340,53 @@ def grouped_gemm_swiglu(Aq, sfA, Bq, sfB, alphas, offsets, gs_h, h_q=None, h_sf=
         _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alphas), _ptr(offsets), E, rows, I, K,
         _ptr(gs_h), _ptr(h_q), _ptr(h_sf), _stream(stream)))
     return h_q, h_sf
+
+
+# ------------------------------------------------------------------ MXFP4 (use_nvfp4=False)
+
+def mx_sf_bytes(rows: int, K: int, tiled: bool = True) -> int:
+    return int(load().nvfp4_mx_sf_bytes(rows, K, SF_TILED if tiled else SF_LINEAR))
+
+
+def mx_quantize(x: torch.Tensor, q=None, sf=None, tiled: bool = True, stream=None):
+    """MXFP4 quantisation of x[rows, K] (E8M0 scale per 32 elements, no per-tensor scale).
+    Returns (q uint8 [rows, K/2], sf uint8: flat tiled scales, or [rows, K/32] if not tiled)."""
+    _dev(x, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    rows, K = x.shape
+    if q is None:
+        q = torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = (torch.empty(mx_sf_bytes(rows, K, True), dtype=torch.uint8, device=x.device) if tiled
+              else torch.empty(rows, K // 32, dtype=torch.uint8, device=x.device))
+    _check("nvfp4_mx_quantize", load().nvfp4_mx_quantize(
+        _ptr(x), _dtype_code(x), rows, K, x.stride(0), _ptr(q), _ptr(sf), SF_TILED if tiled else SF_LINEAR,
+        _stream(stream)))
+    return q, sf
+
+
+def mx_sf_tile(sf: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Row-major MXFP4 scales [rows, K/32] -> the tiled layout (flat uint8 tensor)."""
+    rows, K = sf.shape[0], sf.shape[1] * 32
+    if out is None:
+        out = torch.empty(mx_sf_bytes(rows, K, True), dtype=torch.uint8, device=sf.device)
+    _check("nvfp4_mx_sf_tile", load().nvfp4_mx_sf_tile(_ptr(sf), rows, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def mx_gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None,
+            out_dtype=torch.bfloat16) -> torch.Tensor:
+    """MXFP4 product out[M, N] = alpha * sum_k deq(A) deq(B); sfA, sfB tiled E8M0 scales."""
+    M, K = Aq.shape[0], Aq.shape[1] * 2
+    N = Bq.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=Aq.device)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    _check("nvfp4_mx_gemm", load().nvfp4_mx_gemm(
+        _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alpha_t), _ptr(out), M, N, K, ws_ptr, ws_bytes,
+        _out_code(out), _stream(stream)))
+    return out
 
 
 # ------------------------------------------------------------------ mixture-of-experts layer

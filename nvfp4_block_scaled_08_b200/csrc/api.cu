@@ -303,6 +303,76 @@ nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t*
     return from_cuda(e);
 }
 
+nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K, int64_t ld_x,
+                               uint8_t* q, uint8_t* sf, nvfp4_sf_layout sf_layout, cudaStream_t stream)
+{
+    if (rows < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_F32 && dtype != NVFP4_IN_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (sf_layout != NVFP4_SF_LINEAR && sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0 || K == 0) return NVFP4_OK;
+    if (!x || !q || !sf) return NVFP4_ERR_INVALID_ARG;
+    if (K % 32 != 0 || K > kMaxDim || rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (sf_layout == NVFP4_SF_TILED && K % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld_x < K) return NVFP4_ERR_INVALID_ARG;
+    const int64_t esz = dtype == NVFP4_IN_BF16 ? 2 : 4;
+    if (rows * (K / 8) >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || (ld_x * esz) % 16 != 0 || !aligned16(q)) return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_mx_quantize(x, dtype == NVFP4_IN_BF16, rows, K, ld_x, q, sf,
+                                               sf_layout == NVFP4_SF_TILED, stream, d.num_sms));
+}
+
+size_t nvfp4_mx_sf_bytes(int64_t rows, int64_t K, nvfp4_sf_layout sf_layout)
+{
+    if (rows < 0 || K <= 0 || K % 32 != 0) return 0;
+    if (sf_layout == NVFP4_SF_LINEAR) return static_cast<size_t>(rows) * static_cast<size_t>(K / 32);
+    if (sf_layout == NVFP4_SF_TILED && K % 128 == 0)
+        return static_cast<size_t>((rows + 127) / 128 * 128) * static_cast<size_t>(K / 32);
+    return 0;
+}
+
+nvfp4_status nvfp4_mx_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* sf_tiled, cudaStream_t stream)
+{
+    if (rows < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0 || K == 0) return NVFP4_OK;
+    if (!sf || !sf_tiled) return NVFP4_ERR_INVALID_ARG;
+    if (K % 128 != 0 || K > kMaxDim || rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_sf_tile(sf, rows, K, sf_tiled, stream, d.num_sms, 32));
+}
+
+nvfp4_status nvfp4_mx_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                           const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
+                           size_t ws_bytes, nvfp4_out_dtype out_dtype, cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F16 && out_dtype != NVFP4_OUT_F32)
+        return NVFP4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (M > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    nvfp4_status st = check_gemm_common(A, sfA, B, sfB, alpha, out, N, K);
+    if (st != NVFP4_OK) return st;
+    if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    nvfp4::GemmPlan plan = nvfp4::plan_gemm(M, N, K, ws != nullptr, d.num_sms);
+    if (plan.ws_bytes > 0 && ws_bytes < plan.ws_bytes) return NVFP4_ERR_WORKSPACE;
+    // tiled scales: Q tiles start on 128-row tile boundaries (tuning overrides can break it)
+    if (plan.swap ? plan.q_tiles != 1 : (plan.bn % 128 != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0, ws, d.err_word, true,
+                        static_cast<int32_t>(out_dtype)};
+    L.mx = true;
+    bool enc_failed = false;
+    cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
+    if (enc_failed) return NVFP4_ERR_CUDA;
+    return from_cuda(e);
+}
+
 nvfp4_status nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                            const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
                            size_t ws_bytes, nvfp4_sf_layout sf_layout, cudaStream_t stream)

@@ -275,11 +275,11 @@ static int max_active_clusters(int cs)
     return cache[dev][cs] > 0 ? cache[dev][cs] : 0;
 }
 
-template <int BN, bool SWAP, bool GROUPED, bool SFT = false, bool SWIGLU = false>
+template <int BN, bool SWAP, bool GROUPED, bool SFT = false, bool SWIGLU = false, bool MX = false>
 static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
                        bool* encode_failed)
 {
-    using Cfg = GemmCfg<BN, SWAP, GROUPED, SFT, SWIGLU>;
+    using Cfg = GemmCfg<BN, SWAP, GROUPED, SFT, SWIGLU, MX>;
     auto kern = nvfp4_gemm_kernel<Cfg>;
     // Opt in to the large dynamic shared memory once per device (not a stream operation,
     // so a later launch may be captured into a CUDA graph).
@@ -348,7 +348,7 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
             tsq = tq;
             a.sf_p = sP;
             a.sf_q = sQ;
-            a.sf_kb4 = static_cast<int32_t>(L.K / 64);
+            a.sf_kb4 = static_cast<int32_t>(L.K / (MX ? 128 : 64));   // 512-byte blocks per 128 rows
         } else {
             ok &= get_map(&tsp, sP, 2, ks, p_rows, 1, ks, 0, 16, 128, false);
             ok &= get_map(&tsq, sQ, 2, ks, q_rows, 1, ks, 0, 16, BN, false);
@@ -394,6 +394,23 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
 {
     *encode_failed = false;
     if (plan.grid <= 0) return cudaSuccess;
+    if (L.mx) {
+        if (plan.grouped || !L.sf_tiled) return cudaErrorInvalidValue;
+        if (plan.swap) {
+            if (plan.q_tiles != 1) return cudaErrorInvalidValue;   // Q tile at row 0
+            switch (plan.bn) {
+                case 16: return run<16, true, false, true, false, true>(plan, L, stream, encode_failed);
+                case 32: return run<32, true, false, true, false, true>(plan, L, stream, encode_failed);
+                case 64: return run<64, true, false, true, false, true>(plan, L, stream, encode_failed);
+                default: return cudaErrorInvalidValue;
+            }
+        }
+        switch (plan.bn) {
+            case 128: return run<128, false, false, true, false, true>(plan, L, stream, encode_failed);
+            case 256: return run<256, false, false, true, false, true>(plan, L, stream, encode_failed);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     if (L.sf_tiled) {
         if (plan.grouped) return cudaErrorInvalidValue;
         if (plan.swap) {

@@ -91,7 +91,7 @@ struct GemmArgs {
     int32_t inter;            // SWIGLU: I (gate rows = up rows), N = 2 I
 };
 
-template <int BN_, bool SWAP_, bool GROUPED_, bool SFT_ = false, bool SWIGLU_ = false>
+template <int BN_, bool SWAP_, bool GROUPED_, bool SFT_ = false, bool SWIGLU_ = false, bool MX_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;
     static constexpr bool SWAP = SWAP_;
@@ -101,12 +101,19 @@ struct GemmCfg {
     // epilogue writes h = silu(gate) * up quantised to NVFP4 instead of the product itself.
     static constexpr bool SWIGLU = SWIGLU_;
     static_assert(!SWIGLU || GROUPED, "the fused SwiGLU epilogue serves the grouped gate_up GEMM");
+    // MX: MXFP4 operands (one E8M0 scale per 32 K elements, "use_nvfp4=False"), scales in the
+    // tiled layout: a stage's 8 scale bytes per row are two 512-byte blocks per 128 rows, each
+    // covering 128 K elements; the MMA is the block32 form with UE8M0 scales, and the two
+    // 64-wide MMAs of a block read its scale column at byte 0 and byte 2.
+    static constexpr bool MX = MX_;
+    static constexpr int SF_BLOCKS = MX ? 2 : 4;   // 512-byte scale blocks per stage and 128 rows
     // SFT: both operands' scales in the tiled layout (include/nvfp4.h, NVFP4_SF_TILED): a
     // stage's scales of 128 rows are one contiguous 2 KB run already in the tcgen05.cp source
     // layout, fetched by a bulk copy (no re-layout step). Q tiles then start on a 128-row
     // tile boundary: BN >= 128 a multiple of 128, or a single Q tile (few-token swap).
     static constexpr bool SFT = SFT_;
     static_assert(!SFT || !GROUPED, "tiled scales serve the dense GEMM");
+    static_assert(!MX || (SFT && !GROUPED), "MXFP4 serves the dense GEMM with tiled scales");
     static_assert(!SFT || BN % 128 == 0 || (SWAP && BN <= 64), "Q tiles on 128-row tile boundaries");
     static_assert(!GROUPED || SWAP, "grouped GEMM runs with weights as the MMA M operand");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
@@ -116,8 +123,8 @@ struct GemmCfg {
     static constexpr int P_BYTES = BM * BK_BYTES;  // 16 KB
     static constexpr int Q_BYTES = BN * BK_BYTES;
     static constexpr int QG = (BN + 127) / 128;    // 128-row scale groups of the Q tile
-    static constexpr int SFP_BYTES = 2048;         // 128 rows x 16 B (= 4 k-blocks x 512 B)
-    static constexpr int SFQ_BYTES = 2048 * QG;
+    static constexpr int SFP_BYTES = 512 * SF_BLOCKS;   // 128 rows x 16 B (NVFP4) or 8 B (MX)
+    static constexpr int SFQ_BYTES = SFP_BYTES * QG;
     static constexpr int SF_TMA_P = BM * 16;       // bytes the scale TMA writes
     static constexpr int SF_TMA_Q = BN * 16;
     static constexpr uint32_t TX_BYTES = P_BYTES + Q_BYTES + SF_TMA_P + SF_TMA_Q;
@@ -133,7 +140,7 @@ struct GemmCfg {
     // first and signals sf_free, and the MMA warp waits for that before the tile's first
     // tcgen05.cp (by then the previous tile's MMAs have completed, so the copies cannot
     // overwrite scales still being read, and the epilogue overlaps the next tile's MMAs).
-    static constexpr int SF_COLS = 16 + 16 * QG;
+    static constexpr int SF_COLS = 4 * SF_BLOCKS * (1 + QG);
     static constexpr int ACC_STAGES = 2;
     static constexpr bool SF_IN_ACC = 2 * BN + SF_COLS > 512;
     static_assert(!SF_IN_ACC || SF_COLS <= 64, "scale columns fit the last 64-column chunk");
@@ -852,20 +859,21 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                                         pol_q);
                         }
                     } else if constexpr (Cfg::SFT) {
-                        // the stage's 4 scale blocks of each 128-row tile: one 2 KB run; only
-                        // the Q row tiles that exist (the last Q tile may end past the rows)
+                        // the stage's scale blocks of each 128-row tile: one contiguous run (2 KB,
+                        // MX 1 KB); only the Q row tiles that exist (the last Q tile may end past
+                        // the rows)
                         const int ng = min(QG, (args.q_rows - ti.q0 + 127) >> 7);
                         mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::Q_BYTES + Cfg::SFP_BYTES +
-                                                  2048u * static_cast<uint32_t>(ng));
+                                                  static_cast<uint32_t>(Cfg::SFP_BYTES * ng));
                         tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
                         tma_load_2d(qbuf, &tm_q, fb, kx, ti.q0, pol_q);
-                        const int64_t kb = 4 * static_cast<int64_t>(ti.k0 + ks);
+                        const int64_t kb = Cfg::SF_BLOCKS * static_cast<int64_t>(ti.k0 + ks);
                         bulk_load(sfpb, args.sf_p + ((ti.p0 >> 7) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
-                                  2048, fb, pol_p);
+                                  Cfg::SFP_BYTES, fb, pol_p);
                         for (int g = 0; g < ng; ++g)
-                            bulk_load(sfqb + 2048 * g,
+                            bulk_load(sfqb + Cfg::SFP_BYTES * g,
                                       args.sf_q + (((ti.q0 >> 7) + g) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
-                                      2048, fb, pol_q);
+                                      Cfg::SFP_BYTES, fb, pol_q);
                     } else {
                         mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
                         tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
@@ -910,7 +918,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             const uint32_t sf_b = sf_a + 16;
             uint32_t n_mma = BN;
             if constexpr (Cfg::GROUPED) n_mma = min(BN, (ti.q_valid + 15) & ~15);
-            const uint32_t idesc = idesc_mxf4nvf4(128, n_mma);
+            const uint32_t idesc = Cfg::MX ? idesc_mxf4_ue8m0(128, n_mma) : idesc_mxf4nvf4(128, n_mma);
             const uint32_t d_tmem = tmem_base + acc * BN;
             for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
                 bool got = mbar_wait(&full_bar[stage], phase, ab, kErrMmaFull);
@@ -921,12 +929,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     const uint32_t sfp = smem_u32(smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES);
                     const uint32_t sfq = smem_u32(smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
+                    for (int j = 0; j < Cfg::SF_BLOCKS; ++j) {
                         tmem_cp_32x128b_warpx4(sf_a + 4 * j, sdesc_sf_32x16(sfp + 512 * j));
 #pragma unroll
                         for (int g = 0; g < QG; ++g)
                             tmem_cp_32x128b_warpx4(sf_b + 4 * QG * j + 4 * g,
-                                                   sdesc_sf_32x16(sfq + 2048 * g + 512 * j));
+                                                   sdesc_sf_32x16(sfq + Cfg::SFP_BYTES * g + 512 * j));
                     }
                     const uint64_t pdesc =
                         sdesc_kmajor_sw128(smem_u32(smem + Cfg::OFF_P + stage * Cfg::P_BYTES));
@@ -935,8 +943,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         // advance 32 bytes (64 fp4 values) along K inside the swizzled rows
-                        mma_mxf4nvf4(d_tmem, pdesc + 2u * j, qdesc + 2u * j, idesc, sf_a + 4 * j,
-                                     sf_b + 4 * QG * j, (ks > 0 || j > 0) ? 1u : 0u);
+                        if constexpr (Cfg::MX) {
+                            // block j / 2; its scale column holds 4 E8M0 bytes per row (K 128):
+                            // bytes 0-1 for the first 64, 2-3 for the second
+                            mma_mxf4_block32(d_tmem, pdesc + 2u * j, qdesc + 2u * j,
+                                             idesc_sf_id(idesc, 2u * (j & 1)), sf_a + 4 * (j >> 1),
+                                             sf_b + 4 * QG * (j >> 1), (ks > 0 || j > 0) ? 1u : 0u);
+                        } else {
+                            mma_mxf4nvf4(d_tmem, pdesc + 2u * j, qdesc + 2u * j, idesc, sf_a + 4 * j,
+                                         sf_b + 4 * QG * j, (ks > 0 || j > 0) ? 1u : 0u);
+                        }
                     }
                     mma_commit(&empty_bar[stage]);
                 }

@@ -33,8 +33,12 @@ cudaError_t launch_moe_route(const float* logits, int32_t T, int32_t E, int32_t 
 cudaError_t launch_moe_combine(const void* y, int32_t y_dt, const float* weights, const int32_t* row_of,
                                int32_t T, int64_t H, int32_t k, void* out, int32_t out_dt, cudaStream_t stream,
                                int num_sms);
+// Row-major scales [rows][K / block] -> the tiled layout (block = 16: NVFP4, 32: MXFP4).
 cudaError_t launch_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* out, cudaStream_t stream,
-                           int num_sms);
+                           int num_sms, int block = 16);
+// MXFP4 quantisation (E8M0 scale per 32 elements, no per-tensor scale), linear or tiled scales.
+cudaError_t launch_mx_quantize(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx, uint8_t* q,
+                               uint8_t* sf, bool sf_tiled, cudaStream_t stream, int num_sms);
 cudaError_t launch_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
                          cudaStream_t stream);
 cudaError_t launch_round(const float* x, int64_t n, uint8_t* out, bool e2m1, cudaStream_t stream,
@@ -79,6 +83,7 @@ struct GemmLaunch {
     uint8_t* h_q = nullptr;
     uint8_t* h_sf = nullptr;
     const float* gs_h = nullptr;
+    bool mx = false;            // MXFP4 operands (E8M0 scale per 32 elements, tiled scales)
 };
 
 // api.cu: nvfp4_status of the current device's checks; fills the SM count and the device

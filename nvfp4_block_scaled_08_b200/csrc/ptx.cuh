@@ -257,6 +257,20 @@ __host__ __device__ constexpr uint32_t idesc_mxf4nvf4(uint32_t M, uint32_t N)
     return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// The same descriptor for 32-element blocks with UE8M0 (power-of-two) scales: scale type bit
+// 23 = 1 (UE8M0).
+__host__ __device__ constexpr uint32_t idesc_mxf4_ue8m0(uint32_t M, uint32_t N)
+{
+    return idesc_mxf4nvf4(M, N) | (1u << 23);
+}
+
+// Selects the byte of the 32-bit TMEM scale column an MMA reads its scales from: A scale
+// factor id at bits [29, 31), B at [4, 6) (with two scales per row and MMA, byte 0 or 2).
+__host__ __device__ constexpr uint32_t idesc_sf_id(uint32_t idesc, uint32_t byte)
+{
+    return idesc | (byte << 29) | (byte << 4);
+}
+
 // D[tmem] (+)= A[smem] x B[smem]^T with per-16-element e4m3 scales read from TMEM.
 // One 128 x N x 64 block-scaled FP4 MMA; issued by a single thread.
 __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -267,6 +281,20 @@ __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t adesc, ui
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+          "r"(sfb_tmem)
+        : "memory");
+}
+
+// One 128 x N x 64 block-scaled FP4 MMA with one UE8M0 scale per 32 K elements (MXFP4).
+__device__ __forceinline__ void mma_mxf4_block32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t sfa_tmem,
+                                                 uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
           "r"(sfb_tmem)
         : "memory");

@@ -185,12 +185,14 @@ struct SfOut {
     }
 };
 
-inline SfOut make_sf_out(uint8_t* sf, bool tiled, const VecIndex& ix, int64_t K)
+// block: elements per scale (16 for NVFP4, 32 for MXFP4); the tiled layout holds 4 scale
+// columns per 512-byte block, so a 128-row tile spans K / (4 block) blocks.
+inline SfOut make_sf_out(uint8_t* sf, bool tiled, const VecIndex& ix, int64_t K, int block = 16)
 {
     SfOut o;
     o.sf = sf;
     o.tiled = tiled ? 1 : 0;
-    o.kb4 = static_cast<uint32_t>(K / 64);
+    o.kb4 = static_cast<uint32_t>(K / (4 * block));
     o.vpr = ix.vpr;
     o.mul = ix.mul;
     o.shift = ix.shift;
@@ -353,6 +355,44 @@ __device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint
             const float rcp = rcp_tab[sfq];
             const uint32_t packed = scale_to_e2m1x8(v[u], rcp);
             if (i < end) dst.template store<TPB>(i, packed, sfq, (lane & (TPB - 1)) == 0);
+        }
+    }
+}
+
+// MXFP4 (OCP MX v1.0 FP4: e2m1 elements, one E8M0 scale 2^(byte - 127) per 32 elements, no
+// per-tensor scale; "The Art of Reading the Manual", section "The Message": use_nvfp4=False).
+// Per block: shared_exp = floor(log2(amax)) - 2, clamped to [-127, 127] (an all-zero block:
+// -127); byte = shared_exp + 127; codes e2m1_rn_satfinite(x * 2^-shared_exp). For finite
+// amax >= 0 with biased exponent field E (0 for zero and subnormals), floor(log2(amax)) =
+// E - 127 when E > 0, so byte = max(E - 2, 0) (E = 1 and subnormals clamp to byte 0), and
+// 2^-shared_exp is the normal float with biased exponent 254 - byte (byte <= 252). x times a
+// power of two is exact unless the product is below 2^-126, where no e2m1 code depends on
+// the rounding (only the sign, which the product keeps).
+// Four lanes (32 elements, 8 each) per block, warp-aligned vectors [w0 + lane, ...).
+template <typename T, typename Src>
+__device__ __forceinline__ void mx_quantize_sweep(const Src& src, uint32_t w0, uint32_t end, uint32_t step,
+                                                  uint8_t* __restrict__ q, const SfOut& sfo)
+{
+    constexpr int V = InTraits<T>::kPerThread;
+    static_assert(V == 8, "8 elements per lane");
+    constexpr int TPB = 32 / V;                  // lanes per 32-element block
+    const uint32_t lane = threadIdx.x & 31;
+    for (; w0 < end; w0 += step) {               // warp-uniform
+        const uint32_t i = w0 + lane;
+        float v[V];
+        InTraits<T>::decode(i < end ? src(i) : InTraits<T>::zero(), v);
+        float amax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < V; ++k) amax = fmaxf(amax, fabsf(v[k]));
+#pragma unroll
+        for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const int e = static_cast<int>(__float_as_uint(amax) >> 23);   // amax >= 0: no sign bit
+        const uint32_t byte = static_cast<uint32_t>(e > 2 ? e - 2 : 0);
+        const float scale = __uint_as_float((254u - byte) << 23);
+        const uint32_t packed = scale_to_e2m1x8(v, scale);
+        if (i < end) {
+            *reinterpret_cast<uint32_t*>(q + static_cast<int64_t>(i) * 4) = packed;
+            if ((lane & (TPB - 1)) == 0) *sfo.at<TPB>(i) = static_cast<uint8_t>(byte);
         }
     }
 }

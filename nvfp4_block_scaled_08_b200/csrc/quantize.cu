@@ -210,6 +210,17 @@ __global__ void __launch_bounds__(512) quantize_dynamic_cluster_kernel(
     cluster_wait();                                   // no CTA leaves while a peer may read it
 }
 
+// ------------------------------------------------------------------ MXFP4
+
+template <typename T>
+__global__ void __launch_bounds__(512) mx_quantize_kernel(const T* __restrict__ x, const VecIndex ix, uint32_t nv,
+                                                          uint8_t* __restrict__ q, const SfOut sfo)
+{
+    grid_dependency_wait();      // launched early behind the previous kernel: wait for its data
+    mx_quantize_sweep<T>(GlobalVecs<T>{x, ix}, blockIdx.x * blockDim.x + (threadIdx.x & ~31u), nv,
+                         gridDim.x * blockDim.x, q, sfo);
+}
+
 // ------------------------------------------------------------------ elementwise conversions
 
 __global__ void round_e4m3_kernel(const float* __restrict__ x, int64_t n, uint8_t* __restrict__ out)
@@ -519,6 +530,36 @@ cudaError_t launch_gather_quantize(const void* x, bool bf16, int64_t T, int64_t 
                             n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
 }
 
+cudaError_t launch_mx_quantize(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx, uint8_t* q,
+                               uint8_t* sf, bool sf_tiled, cudaStream_t stream, int num_sms)
+{
+    const int V = 8;                       // elements per vector (quant_core.cuh)
+    const int64_t vpr = K / V;
+    if (rows == 0 || vpr == 0) return cudaSuccess;
+    const VecIndex ix = make_vec_index(vpr, ldx, K);
+    const int64_t nv = rows * vpr;         // < 2^31 (checked by the caller)
+    const SfOut sfo = make_sf_out(sf, sf_tiled, ix, K, 32);
+    // one vector per thread per pass: enough warps to cover the tensor, at most 8 per SM
+    int64_t grid = (nv + 511) / 512;
+    if (grid > static_cast<int64_t>(num_sms) * 4) grid = static_cast<int64_t>(num_sms) * 4;
+    if (grid < 1) grid = 1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(512, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (bf16)
+        return cudaLaunchKernelEx(&cfg, mx_quantize_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(x),
+                                  ix, static_cast<uint32_t>(nv), q, sfo);
+    return cudaLaunchKernelEx(&cfg, mx_quantize_kernel<float>, static_cast<const float*>(x), ix,
+                              static_cast<uint32_t>(nv), q, sfo);
+}
+
 cudaError_t launch_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
                          cudaStream_t stream)
 {
@@ -555,12 +596,13 @@ __global__ void sf_tile_kernel(const uint8_t* __restrict__ sf, int64_t rows, int
 }
 
 cudaError_t launch_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* out, cudaStream_t stream,
-                           int num_sms)
+                           int num_sms, int block)
 {
-    const int64_t out_bytes = (rows + 127) / 128 * 128 * (K / 16);
+    const int64_t kb = K / block;          // scale columns per row
+    const int64_t out_bytes = (rows + 127) / 128 * 128 * kb;
     if (out_bytes == 0) return cudaSuccess;
     const int grid = grid_for(out_bytes, num_sms);
-    sf_tile_kernel<<<grid, 256, 0, stream>>>(sf, rows, K / 16, K / 64, out, out_bytes);
+    sf_tile_kernel<<<grid, 256, 0, stream>>>(sf, rows, kb, kb / 4, out, out_bytes);
     return cudaGetLastError();
 }
 

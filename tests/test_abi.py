@@ -95,6 +95,40 @@ def test_out_dtype_host_validation(lib):
     assert gg(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x8000, 256, 4096, 4096, 6000, 0x6000, 1, None) == 2
 
 
+def test_mx_host_validation(lib):
+    q = lib.nvfp4_mx_quantize
+    assert q(0x1000, 0, 0, 512, 512, 0x2000, 0x3000, 0, None) == 0             # no rows
+    assert q(0x1000, 0, 4, 48, 48, 0x2000, 0x3000, 0, None) == 2               # K % 32
+    assert q(0x1000, 0, 4, 96, 96, 0x2000, 0x3000, 1, None) == 2               # tiled needs K % 128
+    assert q(0x1000, 0, 4, 128, 128, 0x2000, 0x3000, 2, None) == 1             # bad layout
+    assert q(0x1008, 0, 4, 128, 128, 0x2000, 0x3000, 0, None) == 3
+    assert lib.nvfp4_mx_sf_bytes(300, 512, 0) == 300 * 16
+    assert lib.nvfp4_mx_sf_bytes(300, 512, 1) == 384 * 16
+    assert lib.nvfp4_mx_sf_bytes(300, 96, 1) == 0
+    assert lib.nvfp4_mx_sf_tile(0x1000, 4, 96, 0x2000, None) == 2
+    g = lib.nvfp4_mx_gemm
+    assert g(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 16, 768, 6000, None, 0, 0, None) == 2
+    assert g(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 16, 768, 6144, None, 0, 5, None) == 1
+    assert g(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 0, 768, 6144, None, 0, 0, None) == 0
+
+
+def test_moe_host_validation(lib):
+    r = lib.nvfp4_moe_route
+    assert r(0x1000, 4, 256, 8, 0x2000, 0x3000, None, 0x5000, 0x6000, None) == 1      # offsets
+    assert r(0x1000, 4, 2048, 8, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == 2  # E > 1024
+    assert r(0x1000, 4, 256, 33, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == 2  # k > 32
+    assert r(0x1000, 4, 4, 8, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == 2     # k > E
+    assert r(0x1002, 4, 256, 8, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == 3
+    gq = lib.nvfp4_moe_gather_quantize
+    assert gq(0x1000, 0, 0, 6144, 6144, 8, 0x2000, 0x3000, 0x4000, 0x5000, None, 0, None, None) == 2
+    assert gq(0x1000, 0, 4, 6008, 6008, 8, 0x2000, 0x3000, 0x4000, 0x5000, None, 0, None, None) == 2
+    assert gq(0x1008, 0, 4, 6144, 6144, 8, 0x2000, 0x3000, 0x4000, 0x5000, None, 0, None, None) == 3
+    c = lib.nvfp4_moe_combine
+    assert c(0x1000, 0, 0x2000, 0x3000, 4, 6144, 8, 0x4000, 3, None) == 1               # out dtype
+    assert c(0x1000, 0, 0x2000, 0x3000, 4, 6148, 8, 0x4000, 0, None) == 2               # H % 8
+    assert c(0x1000, 0, 0x2000, 0x3000, 0, 6144, 8, 0x4000, 0, None) == 0
+
+
 def test_plan_override_validation(lib):
     assert lib.nvfp4_set_plan_override(-1, 0, 0, 0, 0) == 1
     assert lib.nvfp4_set_plan_override(0, 0, -2, 0, 0) == 1
