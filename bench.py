@@ -386,7 +386,9 @@ class GroupedStep:
                 nv.global_scale(w, out=gsB[e:e + 1])
                 nv.quantize(w, gsB[e:e + 1], q=Bq[e], sf=sfB[e])
                 del w
-            cls._weights = {key: (Bq, sfB, gsB)}      # keep one projection's weights at a time
+            if len(cls._weights) >= 2:                 # keep two projections' weights at a time
+                cls._weights.pop(next(iter(cls._weights)))
+            cls._weights[key] = (Bq, sfB, gsB)
         return cls._weights[key]
 
     def __init__(self, nv, case, dev):
@@ -422,6 +424,99 @@ class GroupedStep:
         return g, q, st
 
 
+class MoeLayer:
+    """The MoE layer around the grouped GEMMs: top-8 routing of T tokens over 256 experts,
+    one quantisation of the tokens into their expert-sorted rows, the gate_up GEMM with the
+    fused SwiGLU + NVFP4 epilogue, the down GEMM and the weighted combine; seven launches.
+    h's global scale is fixed in advance (2688 / 256: |h| of these inputs stays below 256)."""
+
+    GS_H = 2688.0 / 256.0
+
+    def __init__(self, nv, T, dev):
+        from nvfp4_block_scaled_08_b200 import workloads
+        self.nv, self.T = nv, T
+        up = [c for c in workloads.grouped_cases() if c.name == f"moe_gate_up_T{T}"][0]
+        down = [c for c in workloads.grouped_cases() if c.name == f"moe_down_T{T}"][0]
+        self.E, self.k, self.H, self.I = up.num_experts, workloads.TOP_K, up.K, up.N // 2
+        g = torch.Generator().manual_seed(up.route_seed)
+        self.logits = torch.randn(T, self.E, generator=g).to(dev)
+        self.x = workloads.normal(T, self.H, 1.0, up.route_seed + 1).to(dev)
+        self.Bu, self.sfBu, self.gsBu = GroupedStep.weights(nv, up, dev)
+        self.Bu, self.sfBu, self.gsBu = self.Bu.clone(), self.sfBu.clone(), self.gsBu.clone()
+        self.Bd, self.sfBd, self.gsBd = GroupedStep.weights(nv, down, dev)
+        self.gs_h = torch.tensor([self.GS_H], dtype=torch.float32, device=dev)
+        self.alpha_d = nv.alpha(self.gs_h, self.gsBd)
+        R = T * self.k
+        self.rows = R
+        e = lambda *shape, dt=torch.uint8: torch.empty(*shape, dtype=dt, device=dev)
+        self.experts, self.w = e(T, self.k, dt=torch.int32), e(T, self.k, dt=torch.float32)
+        self.off, self.row_of = e(self.E + 1, dt=torch.int32), e(T, self.k, dt=torch.int32)
+        self.tok = e(R, dt=torch.int32)
+        self.qx, self.sfx = e(R, self.H // 2), e(R, self.H // 16)
+        self.gsx, self.alpha_u = e(1, dt=torch.float32), e(self.E, dt=torch.float32)
+        self.hq, self.hsf = e(R, self.I // 2), e(R, self.I // 16)
+        self.y = e(R, self.H, dt=torch.bfloat16)
+        self.out = e(T, self.H, dt=torch.bfloat16)
+        self.route()
+        torch.cuda.synchronize()
+        counts = (self.off[1:] - self.off[:-1]).cpu()
+        self.touched = int((counts > 0).sum())
+
+    def route(self):
+        self.nv.moe_route(self.logits, self.k, experts=self.experts, weights=self.w, offsets=self.off,
+                          row_of=self.row_of, token_of_row=self.tok)
+
+    def gather(self):
+        self.nv.moe_gather_quantize(self.x, self.row_of, gs_other=self.gsBu, gs=self.gsx, q=self.qx, sf=self.sfx,
+                                    alpha_out=self.alpha_u)
+
+    def gate_up(self):
+        self.nv.grouped_gemm_swiglu(self.qx, self.sfx, self.Bu, self.sfBu, self.alpha_u, self.off, self.gs_h,
+                                    h_q=self.hq, h_sf=self.hsf)
+
+    def down(self):
+        self.nv.grouped_gemm(self.hq, self.hsf, self.Bd, self.sfBd, self.alpha_d, self.off, out=self.y)
+
+    def combine(self):
+        self.nv.moe_combine(self.y, self.w, self.row_of, out=self.out)
+
+    def layer(self):
+        self.route()
+        self.gather()
+        self.gate_up()
+        self.down()
+        self.combine()
+
+
+def moe_layer_entries(nv, dev, peaks, log):
+    items = []
+    for T in (512, 4096):
+        t0 = time.perf_counter()
+        L = MoeLayer(nv, T, dev)
+        parts = {n: graph_time_us([getattr(L, n)]) for n in ("route", "gather", "gate_up", "down", "combine")}
+        layer = graph_time_us([L.layer])
+        R, H, I, E = L.rows, L.H, L.I, L.E
+        fl = 2.0 * R * (2 * I) * H + 2.0 * R * H * I
+        w_bytes = L.touched * ((2 * I) * H + H * I) * (0.5 + 1.0 / 16.0)
+        by = (w_bytes + T * H * 4 + R * H * (0.5 + 1 / 16) * 2 + R * I * (0.5 + 1 / 16) * 2
+              + R * H * 2 * 2 + T * H * 2)
+        it = {"name": f"moe_layer_T{T}", "T": T, "experts": E, "top_k": L.k, "hidden": H, "inter": I,
+              "experts_touched": L.touched, "layer_us": round(layer, 2),
+              "layer_tflops": round(fl / (layer * 1e-6) / 1e12, 1),
+              "parts_us": {k: round(v, 2) for k, v in parts.items()},
+              "launches": 7, "gs_h": MoeLayer.GS_H}
+        r = roofline(fl, by, peaks)
+        it.update({"roofline_us_spec": round(r["spec"][0], 2), "bound": r["spec"][1],
+                   "frac_of_spec": round(r["spec"][0] / layer, 4),
+                   "frac_of_measured": round(r["measured"][0] / layer, 4),
+                   "algorithmic_bytes": by})
+        items.append(it)
+        log(f"  moe_layer_T{T}: layer {layer:.1f} us, parts {parts} ({time.perf_counter() - t0:.1f} s)")
+        del L
+        torch.cuda.empty_cache()
+    return items
+
+
 def dense_entry(name, M, N, K, g_us, q_us, st_us, copies, set_bytes, peaks):
     fl = 2.0 * M * N * K
     by = gemm_bytes(M, N, K)
@@ -442,7 +537,7 @@ def per_config(dev, peaks, log):
     from nvfp4_block_scaled_08_b200 import workloads
     out = []
 
-    def dense(config, cases, extra=None):
+    def dense(key, config, cases, extra=None):
         items = []
         for c in cases:
             t0 = time.perf_counter()
@@ -459,13 +554,13 @@ def per_config(dev, peaks, log):
         tot_fl = sum(2.0 * i["M"] * i["N"] * i["K"] for i in items)
         tot_g = sum(i["gemm_us"] for i in items)
         tot_st = sum(i["step_us"] for i in items)
-        out.append({"config": config, "shapes": items,
+        out.append({"key": key, "config": config, "shapes": items,
                     "gemm_tflops_all": round(tot_fl / (tot_g * 1e-6) / 1e12, 1),
                     "step_tflops_all": round(tot_fl / (tot_st * 1e-6) / 1e12, 1)})
 
-    dense("single 128x256x512, A,B ~ N(0,1)", [workloads.single_case()])
-    dense("attention projection N=768 K=6144 M={16,64,256,1024}", workloads.attn_proj_cases())
-    dense("MoE expert shapes: up N=2048 K=6144, down N=6144 K=2048, M={16,32,64,128,512,1024}",
+    dense("single", "single 128x256x512, A,B ~ N(0,1)", [workloads.single_case()])
+    dense("attn", "attention projection N=768 K=6144 M={16,64,256,1024}", workloads.attn_proj_cases())
+    dense("moe_expert", "MoE expert shapes: up N=2048 K=6144, down N=6144 K=2048, M={16,32,64,128,512,1024}",
           workloads.moe_expert_cases())
 
     # grouped MoE
@@ -488,10 +583,13 @@ def per_config(dev, peaks, log):
         log(f"  {c.name}: gemm {g:.1f} us, quant {q:.1f} us ({time.perf_counter() - t0:.1f} s)")
         del gs
         torch.cuda.empty_cache()
+    out.append({"key": "grouped", "config": "grouped MoE: 256 experts, top-8 of T={512,4096}; gate_up N=4096 K=6144, "
+                          "down N=6144 K=2048", "shapes": items})
+    out.append({"key": "moe_layer", "config": "MoE layer: routing + gather-quantise + gate_up with fused SwiGLU/NVFP4 + down + "
+                          "combine, 256 experts, top-8, hidden 6144, intermediate 2048",
+                "shapes": moe_layer_entries(nv, dev, peaks, log)})
     GroupedStep._weights = {}
     torch.cuda.empty_cache()
-    out.append({"config": "grouped MoE: 256 experts, top-8 of T={512,4096}; gate_up N=4096 K=6144, "
-                          "down N=6144 K=2048", "shapes": items})
 
     # plateau (+ the bf16 ratio context)
     def bf16_ratio(c, ds, it):
@@ -506,7 +604,7 @@ def per_config(dev, peaks, log):
         it["fp4_over_bf16"] = round(ub / it["gemm_us"], 3)
         del pairs, a, b
 
-    dense("plateau M=N=K in {4096,8192,16384}, U(-1,1); 512x2048x6144 beside bf16 torch matmul",
+    dense("plateau", "plateau M=N=K in {4096,8192,16384}, U(-1,1); 512x2048x6144 beside bf16 torch matmul",
           workloads.plateau_cases(), extra=bf16_ratio)
     return out
 
@@ -772,10 +870,11 @@ def add_cpu_per_config(entries, budget_s):
     """One oracle sample per configuration (its largest dense shape, or an expert slice of the
     grouped one), extrapolated to the configuration's shapes at the sampled rate."""
     from nvfp4_block_scaled_08_b200 import workloads
-    picks = {0: workloads.single_case(), 1: workloads.attn_proj_cases()[-1],
-             2: workloads.moe_expert_cases()[-2], 4: workloads.plateau_cases()[1]}
-    for i, entry in enumerate(entries):
-        if i == 3:
+    picks = {"single": workloads.single_case(), "attn": workloads.attn_proj_cases()[-1],
+             "moe_expert": workloads.moe_expert_cases()[-2], "plateau": workloads.plateau_cases()[1]}
+    for entry in entries:
+        key = entry.get("key")
+        if key == "grouped":
             c = workloads.grouped_cases()[0]
             r = c.route()
             rows = int(r.offsets[2])                      # the first two experts' rows
@@ -783,11 +882,13 @@ def add_cpu_per_config(entries, budget_s):
             b = c.b(0).numpy()
             s = OracleDense(a, b, c.K, rows, min(c.N, 512))
             label = f"{c.name}: the first 2 experts' {rows} rows x {s.c} weight rows, K={c.K}"
-        else:
-            c = picks[i]
+        elif key in picks:
+            c = picks[key]
             a, b = c.a().numpy(), c.b().numpy()
             s = oracle_sample_for(a, b, c.M, c.N, c.K, budget_s)
             label = f"{c.name}: first {s.r} rows of A x first {s.c} rows of B, K={c.K}"
+        else:
+            continue                                      # the MoE layer chain: no oracle sample
         flops, dt, passes, _ = run_oracle(s, budget_s)
         rate = flops / dt
         total = sum(2.0 * sh.get("rows", sh.get("M", 0)) * sh["N"] * sh["K"] for sh in entry["shapes"])
@@ -840,6 +941,54 @@ def run_reference(args, world, rank):
     }
 
 
+def run_profile(args):
+    """A few untimed passes over one configuration's kernels, for ncu (the launch list and
+    counters of profiles/ come from this mode): `--profile KEY` with KEY one of single, attn,
+    moe_expert, grouped, moe_layer, plateau (all its shapes, or --shape NAME for one)."""
+    import nvfp4_block_scaled_08_b200 as nv
+    from nvfp4_block_scaled_08_b200 import workloads
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    key = args.profile
+    reps = args.steps
+    if key in ("single", "attn", "moe_expert", "plateau"):
+        cases = {"single": [workloads.single_case()], "attn": workloads.attn_proj_cases(),
+                 "moe_expert": workloads.moe_expert_cases(), "plateau": workloads.plateau_cases()}[key]
+        for c in cases:
+            if args.shape and c.name != args.shape:
+                continue
+            ds = DenseStep(nv, c.M, c.N, c.K, c.a(), c.b(), dev, copies=1)
+            for _ in range(reps):
+                ds.step(ds.sets[0])
+            torch.cuda.synchronize()
+            del ds
+    elif key == "grouped":
+        for c in sorted(workloads.grouped_cases(), key=lambda c: (c.N, c.T)):
+            if args.shape and c.name != args.shape:
+                continue
+            gs = GroupedStep(nv, c, dev)
+            for _ in range(reps):
+                gs.quant()
+                gs.gemm()
+            torch.cuda.synchronize()
+            del gs
+    elif key == "moe_layer":
+        for T in (512, 4096):
+            if args.shape and args.shape != f"moe_layer_T{T}":
+                continue
+            L = MoeLayer(nv, T, dev)
+            for _ in range(reps):
+                L.layer()
+            torch.cuda.synchronize()
+            del L
+    else:
+        raise SystemExit(f"unknown --profile {key}")
+    st, code = nv.last_device_error()
+    if st != 0:
+        raise SystemExit(f"device error word {code:#x}")
+    print(json.dumps({"profile": key, "shape": args.shape, "passes": reps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -855,7 +1004,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--profile", default=None,
+                    help="untimed passes over one configuration's kernels for ncu (see run_profile)")
+    ap.add_argument("--shape", default=None, help="with --profile: one shape of the configuration")
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

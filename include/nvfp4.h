@@ -385,12 +385,15 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint
  *   cluster     split-K CTAs per thread-block cluster, 1 ... 8;
  *   groups      split-K clusters per output tile, reduced through the workspace (needs one);
  *   band        output P tiles per rasterisation band;
- *   grouped_bn  token tile width of the grouped GEMM: 32, 64, 128 or 256.
+ *   grouped_bn  token tile width of the grouped GEMM: 32, 64, 128 or 256;
+ *   pair        CTA pairs that share 256-row weight tiles (128 x 256 tiles with tiled scales and
+ *               no split-K): 1 = never, 2 = wherever possible (0 = the planner: wherever possible).
  * The planner's choices need no override; results stay within the GEMM tolerance under any
- * of them, and every override layout is deterministic. Negative values: NVFP4_ERR_INVALID_ARG.
+ * of them, and every override layout is deterministic. Negative values (pair above 2):
+ * NVFP4_ERR_INVALID_ARG.
  */
 nvfp4_status nvfp4_set_plan_override(int32_t bn, int32_t cluster, int32_t groups, int32_t band,
-                                     int32_t grouped_bn);
+                                     int32_t grouped_bn, int32_t pair);
 
 /*
  * Elementwise conversions used by the quantiser, exposed so that they can be checked

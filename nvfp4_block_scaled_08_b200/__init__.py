@@ -87,7 +87,7 @@ SIGNATURES = {
     "nvfp4_grouped_gemm_workspace_size": (_SZ, [_I32, _I64, _I64, _I64]),
     "nvfp4_grouped_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
                                           _SZ, _P]),
-    "nvfp4_set_plan_override": (ctypes.c_int, [_I32, _I32, _I32, _I32, _I32]),
+    "nvfp4_set_plan_override": (ctypes.c_int, [_I32, _I32, _I32, _I32, _I32, _I32]),
     "nvfp4_round_e4m3": (ctypes.c_int, [_P, _I64, _P, _P]),
     "nvfp4_round_e2m1": (ctypes.c_int, [_P, _I64, _P, _P]),
     "nvfp4_last_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -311,15 +311,15 @@ class plan_override:
     """Context manager forcing parts of the GEMM launch plan (tuning and tests only):
     ``with plan_override(cluster=2, groups=3): ...``; the planner's choices return on exit."""
 
-    def __init__(self, bn=0, cluster=0, groups=0, band=0, grouped_bn=0):
-        self.values = (bn, cluster, groups, band, grouped_bn)
+    def __init__(self, bn=0, cluster=0, groups=0, band=0, grouped_bn=0, pair=0):
+        self.values = (bn, cluster, groups, band, grouped_bn, pair)
 
     def __enter__(self):
         _check("nvfp4_set_plan_override", load().nvfp4_set_plan_override(*self.values))
         return self
 
     def __exit__(self, *exc):
-        _check("nvfp4_set_plan_override", load().nvfp4_set_plan_override(0, 0, 0, 0, 0))
+        _check("nvfp4_set_plan_override", load().nvfp4_set_plan_override(0, 0, 0, 0, 0, 0))
         return False
 
 
@@ -391,21 +391,27 @@ def mx_gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None,
 
 # ------------------------------------------------------------------ mixture-of-experts layer
 
-def moe_route(logits: torch.Tensor, k: int, stream=None):
+def moe_route(logits: torch.Tensor, k: int, experts=None, weights=None, offsets=None, row_of=None,
+              token_of_row=None, stream=None):
     """Top-k routing of router logits [T, E] (fp32) and the expert-sorted permutation.
 
     Returns (experts int32 [T, k], weights fp32 [T, k], offsets int32 [E+1],
-    row_of int32 [T, k], token_of_row int32 [T*k])."""
+    row_of int32 [T, k], token_of_row int32 [T*k]) (allocated where not given)."""
     _dev(logits, "logits")
     if logits.dtype != torch.float32 or not logits.is_contiguous():
         raise ValueError("logits must be contiguous float32")
     T, E = logits.shape
     dev = logits.device
-    experts = torch.empty(T, k, dtype=torch.int32, device=dev)
-    weights = torch.empty(T, k, dtype=torch.float32, device=dev)
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    row_of = torch.empty(T, k, dtype=torch.int32, device=dev)
-    token_of_row = torch.empty(T * k, dtype=torch.int32, device=dev)
+    if experts is None:
+        experts = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if weights is None:
+        weights = torch.empty(T, k, dtype=torch.float32, device=dev)
+    if offsets is None:
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    if row_of is None:
+        row_of = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if token_of_row is None:
+        token_of_row = torch.empty(T * k, dtype=torch.int32, device=dev)
     _check("nvfp4_moe_route", load().nvfp4_moe_route(
         _ptr(logits), T, E, k, _ptr(experts), _ptr(weights), _ptr(offsets), _ptr(row_of),
         _ptr(token_of_row), _stream(stream)))

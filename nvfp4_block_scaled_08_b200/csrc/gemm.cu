@@ -21,15 +21,16 @@ namespace nvfp4 {
 // Process-wide overrides of the planner's choices (nvfp4_set_plan_override; 0 = planner).
 // Plain atomics: a GEMM call reads them without a lock or a string look-up.
 static std::atomic<int> g_force_bn{0}, g_force_cluster{0}, g_force_groups{0}, g_force_band{0},
-    g_force_grouped_bn{0};
+    g_force_grouped_bn{0}, g_force_pair{0};
 
-void set_plan_override(int bn, int cluster, int groups, int band, int grouped_bn)
+void set_plan_override(int bn, int cluster, int groups, int band, int grouped_bn, int pair)
 {
     g_force_bn.store(bn, std::memory_order_relaxed);
     g_force_cluster.store(cluster, std::memory_order_relaxed);
     g_force_groups.store(groups, std::memory_order_relaxed);
     g_force_band.store(band, std::memory_order_relaxed);
     g_force_grouped_bn.store(grouped_bn, std::memory_order_relaxed);
+    g_force_pair.store(pair, std::memory_order_relaxed);
 }
 
 static int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
@@ -112,6 +113,16 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
     if (g > 1) {
         p.ws_counter_bytes = ((static_cast<size_t>(tiles) * cs * 4 + 255) / 256) * 256;
         p.ws_bytes = p.ws_counter_bytes + static_cast<size_t>(tiles) * g * 128 * p.bn * sizeof(float);
+    }
+    // CTA pairs sharing 256-row Q tiles (used with tiled scales): 128 x 256 tiles without
+    // split-K and at least one pair of P tiles. The pair's work items are P tile pairs.
+    const int fp = g_force_pair.load(std::memory_order_relaxed);     // 1: off, 2: on where possible
+    p.pair = !p.swap && p.bn == 256 && p.splits == 1 && p.p_tiles >= 2 && fp != 1;
+    if (p.pair) {
+        const int pairs = ((p.p_tiles + 1) / 2) * p.q_tiles;
+        const int clusters = std::max(1, std::min(pairs, max_active_clusters(2)));
+        p.pair_grid = 2 * clusters;
+        p.pair_band = std::max(1, p.band / 2);
     }
     return p;
 }
@@ -275,11 +286,12 @@ static int max_active_clusters(int cs)
     return cache[dev][cs] > 0 ? cache[dev][cs] : 0;
 }
 
-template <int BN, bool SWAP, bool GROUPED, bool SFT = false, bool SWIGLU = false, bool MX = false>
+template <int BN, bool SWAP, bool GROUPED, bool SFT = false, bool SWIGLU = false, bool MX = false,
+          bool PAIR = false>
 static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
                        bool* encode_failed)
 {
-    using Cfg = GemmCfg<BN, SWAP, GROUPED, SFT, SWIGLU, MX>;
+    using Cfg = GemmCfg<BN, SWAP, GROUPED, SFT, SWIGLU, MX, PAIR>;
     auto kern = nvfp4_gemm_kernel<Cfg>;
     // Opt in to the large dynamic shared memory once per device (not a stream operation,
     // so a later launch may be captured into a CUDA graph).
@@ -342,7 +354,7 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         const uint64_t p_rows = static_cast<uint64_t>(SWAP ? L.N : L.M);
         const uint64_t q_rows = static_cast<uint64_t>(SWAP ? L.M : L.N);
         ok &= get_map(&tp, P, 2, kb, p_rows, 1, kb, 0, 128, 128, true);
-        ok &= get_map(&tq, Q, 2, kb, q_rows, 1, kb, 0, 128, BN, true);
+        ok &= get_map(&tq, Q, 2, kb, q_rows, 1, kb, 0, 128, PAIR ? BN / 2 : BN, true);   // PAIR: half tiles
         if constexpr (SFT) {
             tsp = tp;                       // unused: the scales come by bulk copy
             tsq = tq;
@@ -356,6 +368,7 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         a.p_rows = static_cast<int32_t>(p_rows);
         a.q_rows = static_cast<int32_t>(q_rows);
         a.num_q_tiles = plan.q_tiles;
+        if constexpr (PAIR) a.num_p_tiles = (plan.p_tiles + 1) / 2;   // work items are P tile pairs
         a.splits = plan.splits;
         a.cluster_size = plan.cluster;
         a.groups = plan.groups;
@@ -370,9 +383,13 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         *encode_failed = true;
         return cudaSuccess;
     }
+    if constexpr (PAIR) {
+        a.band = plan.pair_band;
+        a.num_tiles = a.num_p_tiles * plan.q_tiles;
+    }
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>(plan.grid), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(PAIR ? plan.pair_grid : plan.grid), 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cfg.stream = stream;
@@ -384,8 +401,9 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
     attrs[1].val.clusterDim.x = static_cast<unsigned>(plan.cluster);
     attrs[1].val.clusterDim.y = 1;
     attrs[1].val.clusterDim.z = 1;
+    if constexpr (PAIR) attrs[1].val.clusterDim.x = 2;
     cfg.attrs = attrs;
-    cfg.numAttrs = (!GROUPED && plan.cluster > 1) ? 2 : 1;
+    cfg.numAttrs = (!GROUPED && (plan.cluster > 1 || PAIR)) ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, kern, tp, tq, tsp, tsq, a);
 }
 
@@ -405,6 +423,8 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
                 default: return cudaErrorInvalidValue;
             }
         }
+        if (plan.pair && plan.bn == 256)
+            return run<256, false, false, true, false, true, true>(plan, L, stream, encode_failed);
         switch (plan.bn) {
             case 128: return run<128, false, false, true, false, true>(plan, L, stream, encode_failed);
             case 256: return run<256, false, false, true, false, true>(plan, L, stream, encode_failed);
@@ -422,6 +442,8 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
                 default: return cudaErrorInvalidValue;
             }
         }
+        if (plan.pair && plan.bn == 256)
+            return run<256, false, false, true, false, false, true>(plan, L, stream, encode_failed);
         switch (plan.bn) {
             case 128: return run<128, false, false, true>(plan, L, stream, encode_failed);
             case 256: return run<256, false, false, true>(plan, L, stream, encode_failed);

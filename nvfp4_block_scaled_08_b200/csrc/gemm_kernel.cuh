@@ -53,6 +53,8 @@ enum : uint32_t {
     kErrEpiAccFull = 0x106,
     kErrSplitRx = 0x107,
     kErrMmaSfFree = 0x108,
+    kErrMmaHalf = 0x109,
+    kErrForward = 0x10A,
 };
 
 // Threads per CTA: warps 0-3 (producer, MMA, scale re-layout) and two epilogue warpgroups.
@@ -91,7 +93,8 @@ struct GemmArgs {
     int32_t inter;            // SWIGLU: I (gate rows = up rows), N = 2 I
 };
 
-template <int BN_, bool SWAP_, bool GROUPED_, bool SFT_ = false, bool SWIGLU_ = false, bool MX_ = false>
+template <int BN_, bool SWAP_, bool GROUPED_, bool SFT_ = false, bool SWIGLU_ = false, bool MX_ = false,
+          bool PAIR_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;
     static constexpr bool SWAP = SWAP_;
@@ -114,6 +117,15 @@ struct GemmCfg {
     static constexpr bool SFT = SFT_;
     static_assert(!SFT || !GROUPED, "tiled scales serve the dense GEMM");
     static_assert(!MX || (SFT && !GROUPED), "MXFP4 serves the dense GEMM with tiled scales");
+    // PAIR: the two CTAs of a 2-CTA cluster take adjacent 128-row P tiles of the same 256-row Q
+    // tile. Each loads its own P tile and only its half of the Q tile (rows 128 rank ..) and
+    // forwards that half to the peer's stage buffer with a shared-to-shared bulk copy over
+    // distributed shared memory, so each SM pulls 2/3 of the bytes a lone 128 x 256 tile needs
+    // from L2. The MMA itself is the single-CTA 128 x 256 MMA on the whole Q tile; a stage is
+    // released when both CTAs' MMAs are done with it (the commit arrives on both).
+    static constexpr bool PAIR = PAIR_;
+    static_assert(!PAIR || (SFT && !SWAP && !GROUPED && BN == 256), "CTA pairs share 256-row Q tiles");
+    static constexpr int QH_BYTES = 128 * 128;     // PAIR: one half of the Q tile per stage
     static_assert(!SFT || BN % 128 == 0 || (SWAP && BN <= 64), "Q tiles on 128-row tile boundaries");
     static_assert(!GROUPED || SWAP, "grouped GEMM runs with weights as the MMA M operand");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
@@ -171,8 +183,8 @@ struct GemmCfg {
     static constexpr int OFF_SFQ = OFF_SFP + STAGES * SFP_BYTES;
     static constexpr int OFF_BAR = OFF_SFQ + STAGES * SFQ_BYTES;
     // barriers: full, sfready, empty [STAGES]; acc_full, acc_empty [2]; mma_done; split-K rx;
-    // sf_free [2]
-    static constexpr int NUM_BARS = 3 * STAGES + 8;
+    // sf_free [2]; own Q half landed (PAIR) [STAGES]
+    static constexpr int NUM_BARS = 4 * STAGES + 8;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;     // tmem base, flags
     static constexpr int OFF_PREFIX = OFF_MISC + 64;
     static constexpr int OFF_SWIGLU = OFF_PREFIX + (GROUPED ? ((4 * (kMaxExperts + 1) + 15) & ~15) : 0);
@@ -247,7 +259,8 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, int32_t t, const 
         const int32_t pt = b * a.band + (in_band - qt * width);
         const int32_t base = a.num_kstages / a.splits;
         const int32_t rem = a.num_kstages % a.splits;
-        ti.p0 = pt * Cfg::BM;
+        if constexpr (Cfg::PAIR) ti.p0 = (2 * pt + static_cast<int32_t>(cluster_ctarank())) * Cfg::BM;
+        else ti.p0 = pt * Cfg::BM;
         ti.q0 = qt * Cfg::BN;
         ti.k0 = split * base + min(split, rem);
         ti.kcnt = base + (split < rem ? 1 : 0);
@@ -711,6 +724,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     uint64_t* mma_done_bar = bars + 3 * STAGES + 4;
     uint64_t* rx_bar = bars + 3 * STAGES + 5;       // split-K: partial rows received from peers
     uint64_t* sf_free_bar = bars + 3 * STAGES + 6;  // SF_IN_ACC: scale columns drained
+    uint64_t* half_bar = bars + 3 * STAGES + 8;     // PAIR: this CTA's Q half landed
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
     volatile int* s_is_last = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 8);
@@ -725,7 +739,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&sfready_bar[s], 1);
-            mbar_init(&empty_bar[s], 1);
+            mbar_init(&empty_bar[s], Cfg::PAIR ? 2 : 1);   // PAIR: both CTAs' MMAs
+            mbar_init(&half_bar[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full_bar[s], 1);
@@ -791,12 +806,18 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // PAIR: the peer forwards into this CTA's stages and arrives on its barriers; both CTAs'
+    // barriers are initialised before either touches the other's
+    if constexpr (Cfg::PAIR) cluster_sync();
     // Every CTA of this grid is resident: the next kernel in the stream may be scheduled
     // (it waits for this grid's completion before touching memory).
     grid_launch_dependents();
 
     const uint32_t tmem_base = *s_tmem_base;
     const int32_t num_tiles = Cfg::GROUPED ? s_prefix[args.num_experts] : args.num_tiles;
+    // persistent work loop: CTA pairs (PAIR) walk the work items as one
+    const int32_t tile_start = static_cast<int32_t>(Cfg::PAIR ? blockIdx.x >> 1 : blockIdx.x);
+    const int32_t tile_step = static_cast<int32_t>(Cfg::PAIR ? gridDim.x >> 1 : gridDim.x);
 
     if (warp == 0) {
         // -------------------------------------------------------------- TMA producer
@@ -809,8 +830,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         if constexpr (!Cfg::GROUPED) {
             // Warm L2 with this CTA's first weight tiles while the previous kernel finishes
             // (a prefetch only fills L2, the coherence point, so it cannot see stale data).
-            if (blockIdx.x < num_tiles && elect_one()) {
-                const Tile ti = decode_tile<Cfg>(args, blockIdx.x, s_prefix);
+            if (tile_start < num_tiles && elect_one()) {
+                const Tile ti = decode_tile<Cfg>(args, tile_start, s_prefix);
                 const int n = ti.kcnt < STAGES ? ti.kcnt : STAGES;
                 for (int ks = 0; ks < n; ++ks) {
                     const int32_t kx = (ti.k0 + ks) * Cfg::BK_BYTES;
@@ -823,7 +844,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         grid_dependency_wait();
         uint32_t stage = 0, phase = 0, issued = 0;
         bool ok = true;
-        for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int32_t t = tile_start; t < num_tiles && ok; t += tile_step) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
             for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, ab, kErrProducerEmpty));
@@ -857,6 +878,30 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                                         ti.q0 + b * Cfg::QBOX, pol_q);
                             tma_load_2d(sfqb + b * Cfg::QBOX * 16, &tm_sfq, fb, sx, ti.q0 + b * Cfg::QBOX,
                                         pol_q);
+                        }
+                    } else if constexpr (Cfg::PAIR) {
+                        // own P tile and scales on full[stage], together with the peer's half of
+                        // the Q tile (forwarded); own half of the Q tile and its scales on
+                        // half[stage] (the forwarder sends them on once they have landed). A half
+                        // past the Q rows is neither loaded nor forwarded, by either CTA.
+                        const int rank = static_cast<int>(cluster_ctarank());
+                        const bool peer_half = ti.q0 + 128 * (rank ^ 1) < args.q_rows;
+                        const bool own_half = ti.q0 + 128 * rank < args.q_rows;
+                        const int64_t kb = Cfg::SF_BLOCKS * static_cast<int64_t>(ti.k0 + ks);
+                        mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::SFP_BYTES +
+                                                  (peer_half ? Cfg::QH_BYTES + Cfg::SFP_BYTES : 0u));
+                        tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
+                        bulk_load(sfpb, args.sf_p + ((ti.p0 >> 7) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
+                                  Cfg::SFP_BYTES, fb, pol_p);
+                        uint64_t* hb = &half_bar[stage];
+                        if (own_half) {
+                            mbar_arrive_expect_tx(hb, Cfg::QH_BYTES + Cfg::SFP_BYTES);
+                            tma_load_2d(qbuf + rank * Cfg::QH_BYTES, &tm_q, hb, kx, ti.q0 + 128 * rank, pol_q);
+                            bulk_load(sfqb + rank * Cfg::SFP_BYTES,
+                                      args.sf_q + (((ti.q0 >> 7) + rank) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
+                                      Cfg::SFP_BYTES, hb, pol_q);
+                        } else {
+                            mbar_arrive(hb);
                         }
                     } else if constexpr (Cfg::SFT) {
                         // the stage's scale blocks of each 128-row tile: one contiguous run (2 KB,
@@ -900,12 +945,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
         uint32_t sf_phases = 0;                    // bit b: parity of the next sf_free[b] wait
         bool ok = true;
-        for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int32_t t = tile_start; t < num_tiles && ok; t += tile_step) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
             ok = __all_sync(0xffffffffu, mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, ab, kErrMmaAccEmpty));
             if (!ok) break;
             if constexpr (Cfg::SF_IN_ACC) {
-                if (t != static_cast<int32_t>(blockIdx.x)) {   // the previous tile's scale columns
+                if (t != tile_start) {                         // the previous tile's scale columns
                     const uint32_t o = acc ^ 1u;
                     ok = __all_sync(0xffffffffu,
                                     mbar_wait(&sf_free_bar[o], (sf_phases >> o) & 1u, ab, kErrMmaSfFree));
@@ -923,6 +968,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
                 bool got = mbar_wait(&full_bar[stage], phase, ab, kErrMmaFull);
                 if constexpr (!Cfg::SFT) got = got && mbar_wait(&sfready_bar[stage], phase, ab, kErrMmaSf);
+                if constexpr (Cfg::PAIR) got = got && mbar_wait(&half_bar[stage], phase, ab, kErrMmaHalf);
                 ok = __all_sync(0xffffffffu, got);
                 if (!ok) break;
                 if (elect_one()) {
@@ -954,7 +1000,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                                          sf_b + 4 * QG * j, (ks > 0 || j > 0) ? 1u : 0u);
                         }
                     }
-                    mma_commit(&empty_bar[stage]);
+                    if constexpr (Cfg::PAIR) mma_commit_pair(&empty_bar[stage]);   // both CTAs' stage
+                    else mma_commit(&empty_bar[stage]);
                 }
                 __syncwarp();
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -967,6 +1014,43 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         // Arrives once every tcgen05 operation issued above has completed.
         if (elect_one()) mma_commit(mma_done_bar);
         __syncwarp();
+    } else if (Cfg::PAIR && warp == 2) {
+        // -------------------------------------------------------------- Q-half forwarder
+        // Sends this CTA's half of every stage's Q tile and its scales into the same place of
+        // the peer's stage, completion counted on the peer's full barrier. The stage is free in
+        // the peer too: the producer loaded this half only after both CTAs' MMAs released the
+        // stage (the empty barrier counts both commits).
+        const int rank = static_cast<int>(cluster_ctarank());
+        const uint32_t peer = static_cast<uint32_t>(rank ^ 1);
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        for (int32_t t = tile_start; t < num_tiles && ok; t += tile_step) {
+            const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
+            const bool own_half = ti.q0 + 128 * rank < args.q_rows;
+            if (!own_half) {
+                // nothing to send (and nothing to wait for: without a forward from here the
+                // producer may run rounds ahead on these stages)
+                for (int32_t ks = 0; ks < ti.kcnt; ++ks)
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                continue;
+            }
+            for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&half_bar[stage], phase, ab, kErrForward));
+                if (!ok) break;
+                if (elect_one()) {
+                    uint8_t* qh = smem + Cfg::OFF_Q + stage * Cfg::Q_BYTES + rank * Cfg::QH_BYTES;
+                    uint8_t* sh = smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES + rank * Cfg::SFP_BYTES;
+                    const uint32_t rbar = mapa_shared(smem_u32(&full_bar[stage]), peer);
+                    bulk_copy_s2peer(mapa_shared(smem_u32(qh), peer), smem_u32(qh), Cfg::QH_BYTES, rbar);
+                    bulk_copy_s2peer(mapa_shared(smem_u32(sh), peer), smem_u32(sh), Cfg::SFP_BYTES, rbar);
+                    bulk_commit_group();
+                }
+                __syncwarp();
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        if (elect_one()) bulk_wait_group_read0();        // sources read before teardown
+        __syncwarp();
     } else if (!Cfg::SFT && (warp == 2 || warp == 3)) {
         // -------------------------------------------------------------- scale re-layout
         // The TMA wrote row r's 16 scale bytes (k-blocks 0..15 of the stage) at r * 16.
@@ -977,7 +1061,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         // Warps 2 and 3 take alternate stages.
         const uint32_t sf_warp = static_cast<uint32_t>(warp - 2);
         uint32_t stage = 0, phase = 0, seq = 0;
-        for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        for (int32_t t = tile_start; t < num_tiles; t += tile_step) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
             bool ok = true;
             for (int32_t ks = 0; ks < ti.kcnt; ++ks, ++seq) {
@@ -1039,7 +1123,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             named_bar_sync(1, 32 * kEpilogueWarps);
         }
         uint32_t acc = 0, acc_phase = 0;
-        for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        for (int32_t t = tile_start; t < num_tiles; t += tile_step) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
             bool ok = mbar_wait(&acc_full_bar[acc], acc_phase, ab, kErrEpiAccFull);
             ok = named_bar_and(1, 32 * kEpilogueWarps, ok);
@@ -1159,6 +1243,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     if (warp == 1) {
         if (lane == 0) mbar_wait_drain(mma_done_bar, 0);
         __syncwarp();
+    }
+    if constexpr (Cfg::PAIR) {
+        // neither CTA leaves while the peer's forwards or MMA commits may still reach it: every
+        // thread of both arrives once, after its own roles (and this MMA warp's commits) are done
+        __syncthreads();
+        cluster_sync();
+    }
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }

@@ -56,6 +56,9 @@ struct GemmPlan {
     int num_tiles = 0;     // work items (non-grouped)
     int band = 1;          // P tiles per rasterisation band (non-grouped)
     int grid = 0;          // persistent CTAs
+    bool pair = false;     // 2-CTA clusters sharing 256-row Q tiles (tiled scales, no split-K)
+    int pair_grid = 0;     // CTAs of the pair launch (2 per cluster)
+    int pair_band = 1;     // rasterisation band of the pair launch, in P tile pairs
     size_t ws_bytes = 0;   // workspace needed (split-K)
     size_t ws_counter_bytes = 0;
 };
@@ -66,7 +69,7 @@ struct GemmPlan {
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int num_sms);
 GemmPlan plan_grouped(int32_t E, int64_t total_rows, int64_t N, int64_t K, int num_sms);
 // Forces planner choices for later calls (0 = the planner's own); nvfp4_set_plan_override.
-void set_plan_override(int bn, int cluster, int groups, int band, int grouped_bn);
+void set_plan_override(int bn, int cluster, int groups, int band, int grouped_bn, int pair);
 
 struct GemmLaunch {
     const uint8_t* A; const uint8_t* sfA; const uint8_t* B; const uint8_t* sfB;

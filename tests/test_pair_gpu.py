@@ -1,0 +1,84 @@
+"""GPU checks of the CTA-pair launch of the dense GEMM: the two CTAs of a 2-CTA cluster take
+adjacent 128-row tiles that share one 256-row weight tile, each loads half of that tile and
+forwards it to the other over distributed shared memory.
+
+Every output tile is computed by the same MMAs in the same order with or without pairs, so
+the two launches must agree bit for bit; both must be within the GEMM tolerance of the CPU
+oracle (2^-7 |alpha| sum|a b| + 1e-6). Shapes cover an odd number of row tiles (the last
+pair's second CTA has no rows), weight rows that end inside a tile's second half (that half
+is neither loaded nor forwarded), NVFP4 and MXFP4, and the plateau shapes the planner pairs."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_08_b200 as nv
+from nvfp4_block_scaled_08_b200 import workloads
+import oracle
+from helpers import check_within_tolerance, gpu_quantize
+
+pytestmark = pytest.mark.gpu
+
+
+def _operands(dev, a, b):
+    Aq, sfA, gsA = gpu_quantize(a, dev)
+    Bq, sfB, gsB = gpu_quantize(b, dev)
+    return Aq, nv.sf_tile(sfA), Bq, nv.sf_tile(sfB), nv.alpha(gsA, gsB)
+
+
+def _gemm(Aq, sA, Bq, sB, al, M, N, pair):
+    out = torch.full((M + 2, N), -12352.0, dtype=torch.bfloat16, device=Aq.device)
+    with nv.plan_override(bn=256, cluster=1, groups=1, pair=pair):
+        nv.gemm(Aq, sA, Bq, sB, al, out=out[:M], tiled=True)
+    st, code = nv.last_device_error()
+    assert st == 0, hex(code)
+    assert (out[M:].float() == -12352.0).all(), "write past the last output row"
+    return out[:M]
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 776, 1024), (512, 1024, 2048), (1000, 264, 512),
+                                   (129, 520, 768), (256, 256, 256), (640, 2048, 6144)])
+def test_pair_matches_single_cta_and_oracle(cuda_device, M, N, K):
+    d = cuda_device
+    a = workloads.normal(M, K, 1.0, 3 * M + N)
+    b = workloads.normal(N, K, 0.02, 5 * N + K)
+    ops = _operands(d, a, b)
+    o_pair = _gemm(*ops, M, N, pair=2)
+    o_single = _gemm(*ops, M, N, pair=1)
+    assert torch.equal(o_pair.view(torch.int16), o_single.view(torch.int16)), "pair != single-CTA tiles"
+    ga, gb = oracle.global_scale(a.numpy()), oracle.global_scale(b.numpy())
+    rows = np.r_[0:min(M, 40), max(0, M - 40):M]
+    qa, sa = oracle.quantize(a[rows].contiguous().numpy(), ga)
+    qb, sb = oracle.quantize(b.numpy(), gb)
+    alo = oracle.alpha(ga, gb)
+    v, S, _ = oracle.gemm(qa, sa, qb, sb, alo)
+    check_within_tolerance(o_pair[torch.as_tensor(rows, device=d)], v, S, alo, f"pair {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 776, 1024), (512, 1024, 2048)])
+def test_pair_mx(cuda_device, M, N, K):
+    d = cuda_device
+    a = workloads.normal(M, K, 1.0, 7 * M + N)
+    b = workloads.normal(N, K, 0.02, 9 * N + K)
+    qa, sa = nv.mx_quantize(a.to(d), tiled=True)
+    qb, sb = nv.mx_quantize(b.to(d), tiled=True)
+    al = torch.ones(1, device=d)
+    outs = []
+    for pair in (2, 1):
+        with nv.plan_override(bn=256, cluster=1, groups=1, pair=pair):
+            outs.append(nv.mx_gemm(qa, sa, qb, sb, al))
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    qa_o, sa_o = oracle.mx_quantize(a.numpy())
+    qb_o, sb_o = oracle.mx_quantize(b.numpy())
+    v, S, _ = oracle.mx_gemm(qa_o, sa_o, qb_o, sb_o, 1.0)
+    check_within_tolerance(outs[0], v, S, 1.0, f"mx pair {M}x{N}x{K}")
+
+
+def test_planner_pairs_the_plateau(cuda_device):
+    """The default plan of 4096^3 and 8192^3 with tiled scales uses pairs; same bits as without."""
+    d = cuda_device
+    for c in workloads.plateau_cases()[:2]:
+        ops = _operands(d, c.a(), c.b())
+        o_default = nv.gemm(*ops, tiled=True)
+        with nv.plan_override(pair=1):
+            o_single = nv.gemm(*ops, tiled=True)
+        assert torch.equal(o_default.view(torch.int16), o_single.view(torch.int16)), c.name
