@@ -167,7 +167,14 @@ struct GemmCfg {
     // SWIGLU: gs_h / e4m3 table (256 floats), per epilogue warp a 16-token x 8-byte code stage
     // and a 16-byte scale stage
     static constexpr int SWIGLU_BYTES = SWIGLU ? 1024 + kEpilogueWarps * (128 + 16) : 0;
-    static constexpr int MISC_BYTES = 1024 + (GROUPED ? 4 * (kMaxExperts + 1) : 0) + SWIGLU_BYTES;
+    // split-K receive buffer: this rank's chunk (at most ceil(16 / cs) * 8 rows) from each of
+    // cs <= 8 ranks, cs * ceil(16 / cs) * 8 <= 168 rows of [BN + 4] floats. Few-token (swap)
+    // launches give it a region of its own (RX_OWN), so that the cluster barrier before the
+    // exchange moves into the prologue; other split-K launches reuse the drained stage ring.
+    static constexpr int PSTRIDE = BN + 4;
+    static constexpr bool RX_OWN = SWAP && !GROUPED;
+    static constexpr int RX_BYTES = RX_OWN ? ((168 * PSTRIDE * 4 + 1023) & ~1023) : 0;
+    static constexpr int MISC_BYTES = 1024 + (GROUPED ? 4 * (kMaxExperts + 1) : 0) + SWIGLU_BYTES + RX_BYTES;
     static constexpr int ALIGN_SLACK = 1024;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - MISC_BYTES - ALIGN_SLACK) / STAGE_BYTES;
     // Few-token (swap, non-grouped) launches split K finely and run a handful of stages per
@@ -188,13 +195,10 @@ struct GemmCfg {
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;     // tmem base, flags
     static constexpr int OFF_PREFIX = OFF_MISC + 64;
     static constexpr int OFF_SWIGLU = OFF_PREFIX + (GROUPED ? ((4 * (kMaxExperts + 1) + 15) & ~15) : 0);
-    static constexpr int SMEM_BYTES = OFF_SWIGLU + SWIGLU_BYTES + ALIGN_SLACK;
+    static constexpr int OFF_RX = (OFF_SWIGLU + SWIGLU_BYTES + 1023) & ~1023;
+    static constexpr int SMEM_BYTES = OFF_RX + RX_BYTES + ALIGN_SLACK;
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
-    // split-K partial tile in shared memory: [128 rows][BN + 4 floats]
-    static constexpr int PSTRIDE = BN + 4;
-    // split-K receive buffer in the pipeline memory: this rank's chunk (at most
-    // ceil(16 / cs) * 8 rows) from each of cs <= 8 ranks, cs * ceil(16 / cs) * 8 <= 168 rows
-    static_assert(168 * PSTRIDE * 4 <= STAGES * STAGE_BYTES, "split-K receive buffer fits the pipeline buffers");
+    static_assert(RX_OWN || 168 * PSTRIDE * 4 <= STAGES * STAGE_BYTES, "split-K receive buffer fits the pipeline buffers");
     static_assert(OFF_Q % 1024 == 0 && OFF_SFP % 1024 == 0, "swizzle atoms need 1 KB alignment");
 };
 
@@ -588,8 +592,9 @@ __device__ __forceinline__ void swiglu_chunk16(const GemmArgs& a, const Tile& ti
 // (thread = accumulator row; named barrier 2);
 // every CTA of a split-K launch owns exactly one tile. The `cluster_size` CTAs of a cluster
 // hold consecutive K slices of the same output tile, and row chunk k is reduced by cluster
-// rank k. After the cluster barrier (every CTA of the cluster has drained its main loop, so
-// its pipeline shared memory is free) each thread copies its accumulator row, straight from
+// rank k. Once the receive buffers may be written (a region of their own: since the
+// prologue's cluster barrier; otherwise after a cluster barrier here, when every CTA of the
+// cluster has drained its main loop) each thread copies its accumulator row, straight from
 // TMEM through registers, into slot `rank` of the owning rank's receive buffer
 // [cs][my_rows][PSTRIDE]: st.async to a peer (completion counted in bytes on the peer's rx
 // barrier), a plain store for its own chunk. Once the peers' bytes have landed all 128
@@ -609,8 +614,10 @@ __device__ __forceinline__ void split_k_epilogue(const GemmArgs& a, const Tile& 
     const int g = a.groups;
     const int rank = cs > 1 ? static_cast<int>(cluster_ctarank()) : 0;
     const int owner = chunk_owner(row, cs);
-    float* rx = reinterpret_cast<float*>(smem + Cfg::OFF_P);
-    if (cs > 1) { cluster_arrive(); cluster_wait(); }
+    float* rx = reinterpret_cast<float*>(smem + (Cfg::RX_OWN ? Cfg::OFF_RX : Cfg::OFF_P));
+    // the receive buffer aliases the stage ring: wait until every CTA of the cluster has drained
+    // its main loop (with a region of its own, the prologue's cluster barrier covered it)
+    if (!Cfg::RX_OWN && cs > 1) { cluster_arrive(); cluster_wait(); }
 
     const int my0 = chunk_begin(rank, cs);
     const int my_rows = chunk_begin(rank + 1, cs) - my0;
@@ -806,9 +813,13 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // PAIR: the peer forwards into this CTA's stages and arrives on its barriers; both CTAs'
-    // barriers are initialised before either touches the other's
+    // PAIR: the peer forwards into this CTA's stages and arrives on its barriers; split-K with
+    // a receive region of its own: peers send into it as soon as their rows are done. Either
+    // way both CTAs' barriers are initialised before either touches the other's.
     if constexpr (Cfg::PAIR) cluster_sync();
+    if constexpr (Cfg::RX_OWN) {
+        if (args.splits > 1 && args.cluster_size > 1) cluster_sync();
+    }
     // Every CTA of this grid is resident: the next kernel in the stream may be scheduled
     // (it waits for this grid's completion before touching memory).
     grid_launch_dependents();
@@ -1131,7 +1142,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                 if constexpr (!Cfg::GROUPED) {
                     // cluster peers wait for this CTA on the cluster barrier: arrive anyway (the
                     // second warpgroup arrives in the teardown)
-                    if (half == 0 && args.splits > 1 && args.cluster_size > 1) { cluster_arrive(); cluster_wait(); }
+                    if (!Cfg::RX_OWN && half == 0 && args.splits > 1 && args.cluster_size > 1) {
+                        cluster_arrive();
+                        cluster_wait();
+                    }
                 }
                 break;
             }
@@ -1236,7 +1250,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         // the pipeline; together with the first epilogue warpgroup's arrival (after its
         // accumulator is complete) this tells the cluster peers that this CTA's shared memory
         // may receive their partial rows
-        if ((warp < 4 || warp >= 8) && args.splits > 1 && args.cluster_size > 1) { cluster_arrive(); cluster_wait(); }
+        // (with a receive region of its own the first warpgroup has not arrived yet either: no
+        // CTA leaves while a peer's rows may still be on their way to it)
+        if ((Cfg::RX_OWN || warp < 4 || warp >= 8) && args.splits > 1 && args.cluster_size > 1) {
+            cluster_arrive();
+            cluster_wait();
+        }
     }
     tc_fence_before();
     __syncthreads();
