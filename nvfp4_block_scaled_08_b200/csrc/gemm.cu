@@ -114,10 +114,12 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
         p.ws_counter_bytes = ((static_cast<size_t>(tiles) * cs * 4 + 255) / 256) * 256;
         p.ws_bytes = p.ws_counter_bytes + static_cast<size_t>(tiles) * g * 128 * p.bn * sizeof(float);
     }
-    // CTA pairs sharing 256-row Q tiles (used with tiled scales): 128 x 256 tiles without
-    // split-K and at least one pair of P tiles. The pair's work items are P tile pairs.
+    // CTA pairs sharing 256-row Q tiles (tiled scales): 128 x 256 tiles without split-K and at
+    // least one pair of P tiles; the pair's work items are P tile pairs. Only on request: with
+    // a 4-deep stage ring the forward's extra hop leaves the MMA waiting (measured on B200:
+    // 8192^3 in 371 us with pairs against 209 us without).
     const int fp = g_force_pair.load(std::memory_order_relaxed);     // 1: off, 2: on where possible
-    p.pair = !p.swap && p.bn == 256 && p.splits == 1 && p.p_tiles >= 2 && fp != 1;
+    p.pair = !p.swap && p.bn == 256 && p.splits == 1 && p.p_tiles >= 2 && fp == 2;
     if (p.pair) {
         const int pairs = ((p.p_tiles + 1) / 2) * p.q_tiles;
         const int clusters = std::max(1, std::min(pairs, max_active_clusters(2)));

@@ -971,7 +971,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             }
             tc_fence_after();
             const uint32_t sf_a = tmem_base + Cfg::TMEM_SFA + (Cfg::SF_IN_ACC ? (acc ^ 1u) * BN : 0u);
-            const uint32_t sf_b = sf_a + 16;
+            const uint32_t sf_b = sf_a + 4 * Cfg::SF_BLOCKS;    // after the SFA columns
             uint32_t n_mma = BN;
             if constexpr (Cfg::GROUPED) n_mma = min(BN, (ti.q_valid + 15) & ~15);
             const uint32_t idesc = Cfg::MX ? idesc_mxf4_ue8m0(128, n_mma) : idesc_mxf4nvf4(128, n_mma);
