@@ -944,7 +944,8 @@ def run_reference(args, world, rank):
 def run_profile(args):
     """A few untimed passes over one configuration's kernels, for ncu (the launch list and
     counters of profiles/ come from this mode): `--profile KEY` with KEY one of single, attn,
-    moe_expert, grouped, moe_layer, plateau (all its shapes, or --shape NAME for one)."""
+    moe_expert, grouped, grouped_small (the T = 4096 density on 32 experts), moe_layer, plateau
+    (all its shapes, or --shape NAME for one)."""
     import nvfp4_block_scaled_08_b200 as nv
     from nvfp4_block_scaled_08_b200 import workloads
     dev = torch.device("cuda", 0)
@@ -972,6 +973,21 @@ def run_profile(args):
                 gs.gemm()
             torch.cuda.synchronize()
             del gs
+    elif key == "grouped_small":
+        # the T = 4096 token density (~128 rows per expert) on 32 experts: a small case of the
+        # grouped launch for full ncu captures (weights 200 MB / 100 MB)
+        from dataclasses import replace
+        for c in sorted(workloads.grouped_cases(), key=lambda c: (c.N, c.T)):
+            if c.T != 4096 or (args.shape and c.name != args.shape):
+                continue
+            small = replace(c, T=512, num_experts=32)
+            gs = GroupedStep(nv, small, dev)
+            for _ in range(reps):
+                gs.quant()
+                gs.gemm()
+            torch.cuda.synchronize()
+            del gs
+            GroupedStep._weights = {}
     elif key == "moe_layer":
         for T in (512, 4096):
             if args.shape and args.shape != f"moe_layer_T{T}":

@@ -248,6 +248,24 @@ nvfp4_status nvfp4_mx_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* 
                            size_t ws_bytes, nvfp4_out_dtype out_dtype, cudaStream_t stream);
 
 /*
+ * Few-token GEMM on unquantised activations: the quantisation of x and the product in one
+ * launch. Computes exactly what nvfp4_quantize_dynamic_ex(x, gs_other = gs_b) followed by
+ * nvfp4_gemm_ex2 compute (the same codes, scales, alpha and MMAs, so the same output bits):
+ * out[M, N] = alpha * sum_k deq(Q(x))[m, k] deq(B)[n, k], alpha = 1 / (gs_x * gs_b[0]), gs_x =
+ * 2688 / max|x| (1 if x is all zero). x[M, K]: fp32 or bf16 (device, row stride ld_x elements,
+ * 16-byte aligned rows), gs_b: the weights' global scale (device, 1 float), B[N, K/2] and
+ * sfB in NVFP4_SF_TILED (device), out[M, N] of out_dtype. gs_out / alpha_out (device, 1 float
+ * each, optional): receive gs_x and alpha. M <= 64 (decode shapes); the planned split-K
+ * cluster must give every CTA at most its stage ring's depth of 256-element K stages (K <=
+ * 1024 per CTA at 64 tokens), else NVFP4_ERR_UNSUPPORTED_SHAPE (the two-call path serves
+ * those shapes). Each CTA of the cluster reads its own K slice of x and the slices' maxima meet
+ * in distributed shared memory, so the global scale needs no grid-wide barrier.
+ */
+nvfp4_status nvfp4_gemm_act(const void* x, nvfp4_in_dtype dtype, int64_t ld_x, const float* gs_b,
+                            const uint8_t* B, const uint8_t* sfB, void* out, int64_t M, int64_t N, int64_t K,
+                            float* gs_out, float* alpha_out, nvfp4_out_dtype out_dtype, cudaStream_t stream);
+
+/*
  * Grouped (mixture-of-experts) NVFP4 GEMM ("When a Benchmark Crashes", section "Why This
  * Message Was Written": 256 experts, 8 active per token). Rows of A are sorted by expert;
  * expert e owns rows [expert_offsets[e], expert_offsets[e+1]) and computes
@@ -317,9 +335,9 @@ nvfp4_status nvfp4_grouped_gemm_swiglu(const uint8_t* A, const uint8_t* sfA, con
  *   expert_offsets[E + 1]: expert e owns rows [offsets[e], offsets[e+1]) of the sorted order;
  *   row_of[T, k]:          the sorted row that holds token t's slot s;
  *   token_of_row[T k]:     the token of every sorted row.
- * All device, int32 / fp32, 4-byte aligned. E <= 1024, k <= min(E, 32). Three launches; no
- * scratch (row_of and expert_offsets hold intermediate counts until the last one). Results are
- * deterministic (no atomics). T == 0 writes expert_offsets as all zero.
+ * All device, int32 / fp32, 4-byte aligned. E <= 1024, k <= min(E, 32). Four launches; no
+ * scratch (row_of and expert_offsets hold the ranks and counts until the last ones). Results
+ * are deterministic (no atomics). T == 0 writes expert_offsets as all zero.
  */
 nvfp4_status nvfp4_moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t* experts,
                              float* weights, int32_t* expert_offsets, int32_t* row_of,

@@ -29,7 +29,7 @@ from . import _build
 
 __all__ = [
     "Nvfp4Error", "load", "global_scale", "quantize", "quantize_dynamic", "alpha", "gemm", "gemm_workspace_size",
-    "gemm_noalloc", "plan_override",
+    "gemm_noalloc", "gemm_act", "plan_override",
     "make_workspace", "grouped_gemm", "grouped_gemm_swiglu", "moe_route", "moe_gather_quantize",
     "moe_combine", "mx_quantize", "mx_sf_tile", "mx_sf_bytes", "mx_gemm", "round_e4m3", "round_e2m1", "last_device_error",
     "STATUS",
@@ -84,6 +84,8 @@ SIGNATURES = {
     "nvfp4_mx_sf_bytes": (_SZ, [_I64, _I64, ctypes.c_int]),
     "nvfp4_mx_sf_tile": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "nvfp4_mx_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int, _P]),
+    "nvfp4_gemm_act": (ctypes.c_int, [_P, ctypes.c_int, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P,
+                                      ctypes.c_int, _P]),
     "nvfp4_grouped_gemm_workspace_size": (_SZ, [_I32, _I64, _I64, _I64]),
     "nvfp4_grouped_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
                                           _SZ, _P]),
@@ -274,6 +276,24 @@ def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None, tiled
     _check("nvfp4_gemm_ex2", load().nvfp4_gemm_ex2(
         _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alpha_t), _ptr(out), M, N, K,
         ws_ptr, ws_bytes, SF_TILED if tiled else SF_LINEAR, _out_code(out), _stream(stream)))
+    return out
+
+
+def gemm_act(x, gs_b, Bq, sfB_tiled, out=None, gs_out=None, alpha_out=None, stream=None,
+             out_dtype=torch.bfloat16) -> torch.Tensor:
+    """Few-token GEMM on unquantised activations x [M <= 64, K] (fp32 or bf16): the dynamic
+    NVFP4 quantisation of x and the product in one launch (same bits as quantize_dynamic +
+    gemm). Bq [N, K/2], sfB_tiled (tiled layout), gs_b fp32 [1] (the weights' global scale)."""
+    _dev(x, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    M, K = x.shape
+    N = Bq.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=x.device)
+    _check("nvfp4_gemm_act", load().nvfp4_gemm_act(
+        _ptr(x), _dtype_code(x), x.stride(0), _ptr(gs_b), _ptr(Bq), _ptr(sfB_tiled), _ptr(out), M, N, K,
+        _ptr(gs_out), _ptr(alpha_out), _out_code(out), _stream(stream)))
     return out
 
 

@@ -373,6 +373,50 @@ nvfp4_status nvfp4_mx_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* 
     return from_cuda(e);
 }
 
+nvfp4_status nvfp4_gemm_act(const void* x, nvfp4_in_dtype dtype, int64_t ld_x, const float* gs_b,
+                            const uint8_t* B, const uint8_t* sfB, void* out, int64_t M, int64_t N, int64_t K,
+                            float* gs_out, float* alpha_out, nvfp4_out_dtype out_dtype, cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_F32 && dtype != NVFP4_IN_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F16 && out_dtype != NVFP4_OUT_F32)
+        return NVFP4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (!gs_b) return NVFP4_ERR_INVALID_ARG;
+    // the shared checks with x in A's place (its scales come from the kernel: sfA is not read)
+    nvfp4_status st = check_gemm_common(x, B, B, sfB, gs_b, out, N, K);
+    if (st != NVFP4_OK) return st;
+    if (M > 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld_x < K) return NVFP4_ERR_INVALID_ARG;
+    const int64_t esz = dtype == NVFP4_IN_BF16 ? 2 : 4;
+    if ((ld_x * esz) % 16 != 0 || (gs_out && !aligned4(gs_out)) || (alpha_out && !aligned4(alpha_out)))
+        return NVFP4_ERR_MISALIGNED;
+    DeviceInfo d;
+    st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    nvfp4::GemmPlan plan = nvfp4::plan_gemm(M, N, K, false, d.num_sms);
+    // every CTA's K slice must fit its stage ring; the cluster's slices together cover K
+    const int nk = static_cast<int>(K / 256);
+    const int stages = nvfp4::act_gemm_stages(plan.bn);
+    if (!plan.swap || plan.q_tiles != 1 || plan.groups != 1 || stages == 0 ||
+        (nk + plan.splits - 1) / plan.splits > stages)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    nvfp4::GemmLaunch L{nullptr, nullptr, B, sfB, gs_b, out, M, N, K, nullptr, 0, 0, nullptr, d.err_word, true,
+                        static_cast<int32_t>(out_dtype)};
+    L.A = static_cast<const uint8_t*>(x);
+    L.sfA = B;
+    L.act = x;
+    L.act_ld = ld_x;
+    L.act_bf16 = dtype == NVFP4_IN_BF16;
+    L.gs_b = gs_b;
+    L.gs_out = gs_out;
+    L.alpha_out = alpha_out;
+    bool enc_failed = false;
+    cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
+    if (enc_failed) return NVFP4_ERR_CUDA;
+    return from_cuda(e);
+}
+
 nvfp4_status nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                            const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
                            size_t ws_bytes, nvfp4_sf_layout sf_layout, cudaStream_t stream)

@@ -289,11 +289,11 @@ static int max_active_clusters(int cs)
 }
 
 template <int BN, bool SWAP, bool GROUPED, bool SFT = false, bool SWIGLU = false, bool MX = false,
-          bool PAIR = false>
+          bool PAIR = false, bool ACTQ = false>
 static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
                        bool* encode_failed)
 {
-    using Cfg = GemmCfg<BN, SWAP, GROUPED, SFT, SWIGLU, MX, PAIR>;
+    using Cfg = GemmCfg<BN, SWAP, GROUPED, SFT, SWIGLU, MX, PAIR, ACTQ>;
     auto kern = nvfp4_gemm_kernel<Cfg>;
     // Opt in to the large dynamic shared memory once per device (not a stream operation,
     // so a later launch may be captured into a CUDA graph).
@@ -356,7 +356,8 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         const uint64_t p_rows = static_cast<uint64_t>(SWAP ? L.N : L.M);
         const uint64_t q_rows = static_cast<uint64_t>(SWAP ? L.M : L.N);
         ok &= get_map(&tp, P, 2, kb, p_rows, 1, kb, 0, 128, 128, true);
-        ok &= get_map(&tq, Q, 2, kb, q_rows, 1, kb, 0, 128, PAIR ? BN / 2 : BN, true);   // PAIR: half tiles
+        if constexpr (ACTQ) tq = tp;          // unused: the kernel quantises the activations itself
+        else ok &= get_map(&tq, Q, 2, kb, q_rows, 1, kb, 0, 128, PAIR ? BN / 2 : BN, true);   // PAIR: half tiles
         if constexpr (SFT) {
             tsp = tp;                       // unused: the scales come by bulk copy
             tsq = tq;
@@ -369,6 +370,14 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         }
         a.p_rows = static_cast<int32_t>(p_rows);
         a.q_rows = static_cast<int32_t>(q_rows);
+        if constexpr (ACTQ) {
+            a.act = L.act;
+            a.act_ld = L.act_ld;
+            a.act_bf16 = L.act_bf16 ? 1 : 0;
+            a.gs_b = L.gs_b;
+            a.gs_out = L.gs_out;
+            a.alpha_out = L.alpha_out;
+        }
         a.num_q_tiles = plan.q_tiles;
         if constexpr (PAIR) a.num_p_tiles = (plan.p_tiles + 1) / 2;   // work items are P tile pairs
         a.splits = plan.splits;
@@ -409,11 +418,30 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
     return cudaLaunchKernelEx(&cfg, kern, tp, tq, tsp, tsq, a);
 }
 
+int act_gemm_stages(int bn)
+{
+    switch (bn) {
+        case 16: return GemmCfg<16, true, false, true, false, false, false, true>::STAGES;
+        case 32: return GemmCfg<32, true, false, true, false, false, false, true>::STAGES;
+        case 64: return GemmCfg<64, true, false, true, false, false, false, true>::STAGES;
+        default: return 0;
+    }
+}
+
 cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t stream,
                         bool* encode_failed)
 {
     *encode_failed = false;
     if (plan.grid <= 0) return cudaSuccess;
+    if (L.act) {
+        if (!plan.swap || plan.q_tiles != 1 || plan.groups != 1 || !L.sf_tiled || L.mx) return cudaErrorInvalidValue;
+        switch (plan.bn) {
+            case 16: return run<16, true, false, true, false, false, false, true>(plan, L, stream, encode_failed);
+            case 32: return run<32, true, false, true, false, false, false, true>(plan, L, stream, encode_failed);
+            case 64: return run<64, true, false, true, false, false, false, true>(plan, L, stream, encode_failed);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     if (L.mx) {
         if (plan.grouped || !L.sf_tiled) return cudaErrorInvalidValue;
         if (plan.swap) {

@@ -40,6 +40,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_core.cuh"
 
 namespace nvfp4 {
 
@@ -55,6 +56,8 @@ enum : uint32_t {
     kErrMmaSfFree = 0x108,
     kErrMmaHalf = 0x109,
     kErrForward = 0x10A,
+    kErrActqMax = 0x10B,
+    kErrMmaActq = 0x10C,
 };
 
 // Threads per CTA: warps 0-3 (producer, MMA, scale re-layout) and two epilogue warpgroups.
@@ -87,6 +90,12 @@ struct GemmArgs {
     const int32_t* expert_offsets;  // grouped: [E + 1]
     int32_t num_experts;
     int32_t total_rows;       // grouped: rows of A / out
+    const void* act;          // ACTQ: activations A [M, K] (fp32 or bf16), row stride act_ld elements
+    int64_t act_ld;
+    int32_t act_bf16;
+    const float* gs_b;        // ACTQ: the weights' global scale (device, 1)
+    float* gs_out;            // ACTQ: optional outputs: A's global scale and alpha (device, 1 each)
+    float* alpha_out;
     uint8_t* h_q;             // SWIGLU: NVFP4 codes of h [total_rows, I/2]
     uint8_t* h_sf;            // SWIGLU: e4m3 scales of h [total_rows, I/16]
     const float* gs_h;        // SWIGLU: global scale of h (device, 1)
@@ -94,7 +103,7 @@ struct GemmArgs {
 };
 
 template <int BN_, bool SWAP_, bool GROUPED_, bool SFT_ = false, bool SWIGLU_ = false, bool MX_ = false,
-          bool PAIR_ = false>
+          bool PAIR_ = false, bool ACTQ_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;
     static constexpr bool SWAP = SWAP_;
@@ -126,6 +135,18 @@ struct GemmCfg {
     static constexpr bool PAIR = PAIR_;
     static_assert(!PAIR || (SFT && !SWAP && !GROUPED && BN == 256), "CTA pairs share 256-row Q tiles");
     static constexpr int QH_BYTES = 128 * 128;     // PAIR: one half of the Q tile per stage
+    // ACTQ (few-token launches with tiled weight scales): the activations come in as fp32 or
+    // bf16 and are quantised inside the kernel. Every CTA of a split-K cluster reads its own K
+    // slice of them, the slices' maxima meet over distributed shared memory (the cluster's
+    // slices cover all of A: the tensor's global scale without a grid barrier), and each CTA
+    // quantises its slice straight into the Q stages in the MMA's swizzled operand layout,
+    // with its scales in the tcgen05.cp block layout; the epilogue warps do this before they
+    // wait for the accumulator. The CTA's whole K slice fits in the stage ring (kcnt <=
+    // STAGES): Q stage ks holds K stage ks for the whole launch.
+    static constexpr bool ACTQ = ACTQ_;
+    static_assert(!ACTQ || (SWAP && !GROUPED && SFT && !MX && !PAIR && BN <= 64),
+                  "in-kernel activation quantisation serves the few-token NVFP4 launches");
+    static constexpr int ACTQ_BYTES = ACTQ ? 1024 + 64 + 64 : 0;   // gs / e4m3 table, maxima slots, reduction
     static_assert(!SFT || BN % 128 == 0 || (SWAP && BN <= 64), "Q tiles on 128-row tile boundaries");
     static_assert(!GROUPED || SWAP, "grouped GEMM runs with weights as the MMA M operand");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
@@ -174,7 +195,8 @@ struct GemmCfg {
     static constexpr int PSTRIDE = BN + 4;
     static constexpr bool RX_OWN = SWAP && !GROUPED;
     static constexpr int RX_BYTES = RX_OWN ? ((168 * PSTRIDE * 4 + 1023) & ~1023) : 0;
-    static constexpr int MISC_BYTES = 1024 + (GROUPED ? 4 * (kMaxExperts + 1) : 0) + SWIGLU_BYTES + RX_BYTES;
+    static constexpr int MISC_BYTES = 1024 + (GROUPED ? 4 * (kMaxExperts + 1) : 0) + SWIGLU_BYTES + RX_BYTES +
+                                      ACTQ_BYTES;
     static constexpr int ALIGN_SLACK = 1024;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - MISC_BYTES - ALIGN_SLACK) / STAGE_BYTES;
     // Few-token (swap, non-grouped) launches split K finely and run a handful of stages per
@@ -190,13 +212,15 @@ struct GemmCfg {
     static constexpr int OFF_SFQ = OFF_SFP + STAGES * SFP_BYTES;
     static constexpr int OFF_BAR = OFF_SFQ + STAGES * SFQ_BYTES;
     // barriers: full, sfready, empty [STAGES]; acc_full, acc_empty [2]; mma_done; split-K rx;
-    // sf_free [2]; own Q half landed (PAIR) [STAGES]
-    static constexpr int NUM_BARS = 4 * STAGES + 8;
+    // sf_free [2]; own Q half landed (PAIR) [STAGES]; activations quantised, slice maxima
+    // received (ACTQ)
+    static constexpr int NUM_BARS = 4 * STAGES + 10;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;     // tmem base, flags
     static constexpr int OFF_PREFIX = OFF_MISC + 64;
     static constexpr int OFF_SWIGLU = OFF_PREFIX + (GROUPED ? ((4 * (kMaxExperts + 1) + 15) & ~15) : 0);
     static constexpr int OFF_RX = (OFF_SWIGLU + SWIGLU_BYTES + 1023) & ~1023;
-    static constexpr int SMEM_BYTES = OFF_RX + RX_BYTES + ALIGN_SLACK;
+    static constexpr int OFF_ACTQ = OFF_RX + RX_BYTES;
+    static constexpr int SMEM_BYTES = OFF_ACTQ + ACTQ_BYTES + ALIGN_SLACK;
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(RX_OWN || 168 * PSTRIDE * 4 <= STAGES * STAGE_BYTES, "split-K receive buffer fits the pipeline buffers");
     static_assert(OFF_Q % 1024 == 0 && OFF_SFP % 1024 == 0, "swizzle atoms need 1 KB alignment");
@@ -504,35 +528,6 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& a, const Tile& ti, c
     }
 }
 
-// fp32 -> e4m3fn byte, round to nearest even, finite values saturate to +-448.
-__device__ __forceinline__ uint32_t f32_to_e4m3_byte(float v)
-{
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(v), "f"(v));
-    return r & 0xFFu;
-}
-
-// e4m3fn byte -> fp32 (exact).
-__device__ __forceinline__ float e4m3_byte_to_f32(uint32_t byte)
-{
-    const uint16_t pair = static_cast<uint16_t>(byte | (byte << 8));
-    uint32_t h2;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
-}
-
-// fp32 -> e2m1 code (round to nearest even, saturating at +-6, sign kept) in bits 0..3.
-__device__ __forceinline__ uint32_t f32_to_e2m1_code(float v)
-{
-    uint32_t r;
-    asm("{\n\t.reg .b8 t;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\t"
-        "mov.b32 %0, {t, 0, 0, 0};\n\t}"
-        : "=r"(r)
-        : "f"(v));
-    return r & 0xFu;
-}
-
 // SwiGLU + NVFP4 epilogue of 16 accumulator columns (tokens c .. c + 15 of the tile) in one
 // warp of TMEM lane quadrant `quad`: P rows 32 quad + i (i < 16) are gate row j0 + 16 quad + i
 // and P rows 32 quad + 16 + i the up row of the same index (j0 = p0 / 2), so that lane i and
@@ -567,8 +562,8 @@ __device__ __forceinline__ void swiglu_chunk16(const GemmArgs& a, const Tile& ti
         float amax = fabsf(h[cc]);
 #pragma unroll
         for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const uint32_t sfq = f32_to_e4m3_byte(__fmul_rn(__fdiv_rn(amax, 6.0f), gsh));
-        const uint32_t code = f32_to_e2m1_code(__fmul_rn(h[cc], rcp_tab[sfq]));
+        const uint32_t sfq = f32_to_e4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gsh));
+        const uint32_t code = f32x2_to_e2m1x2(__fmul_rn(h[cc], rcp_tab[sfq]), 0.0f) & 0xFu;
         const uint32_t hi_code = __shfl_xor_sync(0xffffffffu, code, 1);
         const int tok = cc + (up ? 8 : 0);
         if ((i & 1) == 0) stage[tok * 8 + (i >> 1)] = static_cast<uint8_t>(code | (hi_code << 4));
@@ -586,6 +581,121 @@ __device__ __forceinline__ void swiglu_chunk16(const GemmArgs& a, const Tile& ti
         }
     }
     __syncwarp();
+}
+
+// 32-bit asynchronous store into a cluster peer's shared memory, completion counted (bytes) on
+// the peer's mbarrier; both addresses from mapa.
+__device__ __forceinline__ void st_async_u32(uint32_t remote_addr, uint32_t v, uint32_t remote_bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 ::"r"(remote_addr), "r"(v), "r"(remote_bar)
+                 : "memory");
+}
+
+// ACTQ: quantises this CTA's K slice of the activations into its Q stages (run by the 256
+// epilogue threads, e = 0 .. 255, before the epilogue proper). Returns alpha = 1 / (gs_A gs_B),
+// or a negative value if a wait gave up. The steps and fp32 operations are the quantiser's
+// (nvfp4_quantize_dynamic): the global scale from the maximum over all of A, then per 16-element
+// block amax -> s = e4m3(amax / 6 * gs) -> r = gs / e4m3(s) (table) -> codes e2m1(x * r).
+// Vector v (8 elements) of the slice: token row v / (kcnt 32), K stage (v / 32) % kcnt, element
+// 8 (v % 32) of the stage; lanes 2j, 2j + 1 hold one 16-element block.
+template <class Cfg, typename T>
+__device__ __forceinline__ float actq_quantize_t(const GemmArgs& a, uint8_t* smem, int k0, int kcnt, int e,
+                                                 uint64_t* amax_bar, const AbortState& ab)
+{
+    constexpr int V = InTraits<T>::kPerThread;
+    const T* x = static_cast<const T*>(a.act);
+    const int M = a.M;
+    const uint32_t per_row = static_cast<uint32_t>(kcnt) * 32u;
+    const uint32_t nvec = static_cast<uint32_t>(M) * per_row;
+    float* rcp_tab = reinterpret_cast<float*>(smem + Cfg::OFF_ACTQ);
+    float* slots = reinterpret_cast<float*>(smem + Cfg::OFF_ACTQ + 1024);
+    float* red = reinterpret_cast<float*>(smem + Cfg::OFF_ACTQ + 1024 + 64);
+    auto load = [&](uint32_t v, float (&vals)[8]) {
+        const uint32_t r = v / per_row, w = v - r * per_row;
+        const int64_t k = (static_cast<int64_t>(k0) + (w >> 5)) * 256 + (w & 31) * 8;
+        InTraits<T>::decode(InTraits<T>::load(x + static_cast<int64_t>(r) * a.act_ld + k), vals);
+    };
+
+    // zero the slice's Q stages (padding token rows stay zero) while the first loads fly
+    {
+        uint4* q = reinterpret_cast<uint4*>(smem + Cfg::OFF_Q);
+        for (int i = e; i < kcnt * Cfg::Q_BYTES / 16; i += 256) q[i] = make_uint4(0u, 0u, 0u, 0u);
+        uint4* sq = reinterpret_cast<uint4*>(smem + Cfg::OFF_SFQ);
+        for (int i = e; i < kcnt * Cfg::SFQ_BYTES / 16; i += 256) sq[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // 1. the slice's maximum
+    float m = 0.0f;
+    for (uint32_t v = e; v < nvec; v += 256) {
+        float vals[8];
+        load(v, vals);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(vals[k]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((e & 31) == 0) red[e >> 5] = m;
+    named_bar_sync(1, 256);
+    // 2. the cluster's maxima: every CTA's slice together is all of A
+    const int cs = a.cluster_size;
+    bool ok = true;
+    if (e == 0) {
+        float cm = 0.0f;
+        for (int w = 0; w < 8; ++w) cm = fmaxf(cm, red[w]);
+        const uint32_t rank = cs > 1 ? cluster_ctarank() : 0u;
+        slots[rank] = cm;
+        if (cs > 1) {
+            for (int pr = 0; pr < cs; ++pr) {
+                if (pr == static_cast<int>(rank)) continue;
+                st_async_u32(mapa_shared(smem_u32(&slots[rank]), static_cast<uint32_t>(pr)), __float_as_uint(cm),
+                             mapa_shared(smem_u32(amax_bar), static_cast<uint32_t>(pr)));
+            }
+            mbar_arrive_expect_tx(amax_bar, static_cast<uint32_t>((cs - 1) * 4));
+            ok = mbar_wait(amax_bar, 0, ab, kErrActqMax);
+        }
+    }
+    ok = named_bar_and(1, 256, ok);
+    if (!ok) return -1.0f;
+    float amax = 0.0f;
+    for (int r = 0; r < cs; ++r) amax = fmaxf(amax, slots[r]);
+    const float gs = (amax == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, amax);
+    const float alpha = __fdiv_rn(1.0f, __fmul_rn(gs, __ldg(a.gs_b)));
+    {
+        const float sfd = e4m3_to_f32(static_cast<uint32_t>(e));
+        rcp_tab[e] = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gs, sfd);
+    }
+    if (blockIdx.x == 0 && e == 0) {
+        if (a.gs_out) *a.gs_out = gs;
+        if (a.alpha_out) *a.alpha_out = alpha;
+    }
+    named_bar_sync(1, 256);
+    // 3. codes and block scales into the Q stages
+    const int lane = e & 31;
+    for (uint32_t v0 = e & ~31; v0 < nvec; v0 += 256) {     // warp-uniform (nvec % 32 == 0)
+        const uint32_t v = v0 + lane;
+        float vals[8];
+        load(v, vals);
+        float bm = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) bm = fmaxf(bm, fabsf(vals[k]));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+        const uint32_t sfq = f32_to_e4m3(__fmul_rn(__fdiv_rn(bm, 6.0f), gs));
+        const uint32_t packed = scale_to_e2m1x8(vals, rcp_tab[sfq]);
+        const uint32_t r = v / per_row, w = v - r * per_row;
+        const uint32_t st = w >> 5, u = w & 31;
+        const uint32_t kbyte = u * 4;                          // 4 code bytes per vector
+        uint8_t* qs = smem + Cfg::OFF_Q + st * Cfg::Q_BYTES + r * 128;
+        *reinterpret_cast<uint32_t*>(qs + ((((kbyte >> 4) ^ (r & 7u)) << 4) | (kbyte & 15u))) = packed;
+        if ((u & 1u) == 0) {
+            const uint32_t kb = u >> 1;                        // 16-element block of the stage
+            smem[Cfg::OFF_SFQ + st * Cfg::SFQ_BYTES + (kb >> 2) * 512 + (r & 31u) * 16 + ((r >> 5) & 3u) * 4 +
+                 (kb & 3u)] = static_cast<uint8_t>(sfq);
+        }
+    }
+    (void)V;
+    fence_proxy_async_smem();                                  // generic writes -> tensor core reads
+    named_bar_sync(1, 256);
+    return alpha;
 }
 
 // Split-K epilogue of one CTA, run by the 128 threads of the first epilogue warpgroup
@@ -732,6 +842,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     uint64_t* rx_bar = bars + 3 * STAGES + 5;       // split-K: partial rows received from peers
     uint64_t* sf_free_bar = bars + 3 * STAGES + 6;  // SF_IN_ACC: scale columns drained
     uint64_t* half_bar = bars + 3 * STAGES + 8;     // PAIR: this CTA's Q half landed
+    uint64_t* actq_bar = bars + 4 * STAGES + 8;     // ACTQ: the Q stages hold the activations
+    uint64_t* amax_bar = bars + 4 * STAGES + 9;     // ACTQ: the peers' slice maxima arrived
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
     volatile int* s_is_last = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 8);
@@ -756,6 +868,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         }
         mbar_init(mma_done_bar, 1);
         mbar_init(rx_bar, 1);
+        mbar_init(actq_bar, 1);
+        mbar_init(amax_bar, 1);
         *s_abort = 0;
         *s_is_last = 0;
         fence_mbarrier_init();
@@ -869,6 +983,18 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     uint8_t* sfpb = smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES;
                     uint8_t* sfqb = smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES;
                     if constexpr (Cfg::GROUPED) {
+                        // Weight tiles are streamed from HBM once: besides the STAGES in the
+                        // ring, keep the next STAGES of this tile requested into L2 (a prefetch
+                        // needs no shared memory), doubling the weight bytes in flight per SM.
+                        auto prefetch_w = [&](int32_t kk) {
+                            if constexpr (Cfg::SWIGLU)
+                                tma_prefetch_5d(&tm_p, kk * Cfg::BK_BYTES, 0, 0, ti.p0 >> 5, ti.expert);
+                            else
+                                tma_prefetch_3d(&tm_p, kk * Cfg::BK_BYTES, ti.p0, ti.expert);
+                        };
+                        if (ks == 0)
+                            for (int32_t j = STAGES; j < 2 * STAGES - 1 && j < ti.kcnt; ++j) prefetch_w(ti.k0 + j);
+                        if (ks + 2 * STAGES - 1 < ti.kcnt) prefetch_w(ti.k0 + ks + 2 * STAGES - 1);
                         // boxes of QBOX token rows covering the tile's MMA N (its rows rounded
                         // up to 16); the 8-row swizzle atoms of the boxes line up as in one box
                         const int n_mma = min(BN, (ti.q_valid + 15) & ~15);
@@ -914,6 +1040,13 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                         } else {
                             mbar_arrive(hb);
                         }
+                    } else if constexpr (Cfg::ACTQ) {
+                        // weights and their scales only: the epilogue warps fill the Q stages
+                        mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::SFP_BYTES);
+                        tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
+                        const int64_t kb = Cfg::SF_BLOCKS * static_cast<int64_t>(ti.k0 + ks);
+                        bulk_load(sfpb, args.sf_p + ((ti.p0 >> 7) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
+                                  Cfg::SFP_BYTES, fb, pol_p);
                     } else if constexpr (Cfg::SFT) {
                         // the stage's scale blocks of each 128-row tile: one contiguous run (2 KB,
                         // MX 1 KB); only the Q row tiles that exist (the last Q tile may end past
@@ -956,6 +1089,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
         uint32_t sf_phases = 0;                    // bit b: parity of the next sf_free[b] wait
         bool ok = true;
+        if constexpr (Cfg::ACTQ) ok = __all_sync(0xffffffffu, mbar_wait(actq_bar, 0, ab, kErrMmaActq));
         for (int32_t t = tile_start; t < num_tiles && ok; t += tile_step) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
             ok = __all_sync(0xffffffffu, mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, ab, kErrMmaAccEmpty));
@@ -982,9 +1116,11 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                 if constexpr (Cfg::PAIR) got = got && mbar_wait(&half_bar[stage], phase, ab, kErrMmaHalf);
                 ok = __all_sync(0xffffffffu, got);
                 if (!ok) break;
+                // ACTQ: the activations' K stage ks stays in Q stage ks for the whole launch
+                const uint32_t qslot = Cfg::ACTQ ? static_cast<uint32_t>(ks) : stage;
                 if (elect_one()) {
                     const uint32_t sfp = smem_u32(smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES);
-                    const uint32_t sfq = smem_u32(smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES);
+                    const uint32_t sfq = smem_u32(smem + Cfg::OFF_SFQ + qslot * Cfg::SFQ_BYTES);
 #pragma unroll
                     for (int j = 0; j < Cfg::SF_BLOCKS; ++j) {
                         tmem_cp_32x128b_warpx4(sf_a + 4 * j, sdesc_sf_32x16(sfp + 512 * j));
@@ -996,7 +1132,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     const uint64_t pdesc =
                         sdesc_kmajor_sw128(smem_u32(smem + Cfg::OFF_P + stage * Cfg::P_BYTES));
                     const uint64_t qdesc =
-                        sdesc_kmajor_sw128(smem_u32(smem + Cfg::OFF_Q + stage * Cfg::Q_BYTES));
+                        sdesc_kmajor_sw128(smem_u32(smem + Cfg::OFF_Q + qslot * Cfg::Q_BYTES));
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         // advance 32 bytes (64 fp4 values) along K inside the swizzled rows
@@ -1125,11 +1261,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         float* rcp_tab = reinterpret_cast<float*>(smem + Cfg::OFF_SWIGLU);
         uint8_t* stage_w = smem + Cfg::OFF_SWIGLU + 1024 + (warp - 4) * 128;
         uint8_t* sstage_w = smem + Cfg::OFF_SWIGLU + 1024 + kEpilogueWarps * 128 + (warp - 4) * 16;
+        float actq_alpha = 0.0f;
+        if constexpr (Cfg::ACTQ) {
+            const Tile t0 = decode_tile<Cfg>(args, tile_start, s_prefix);
+            actq_alpha = args.act_bf16
+                ? actq_quantize_t<Cfg, __nv_bfloat16>(args, smem, t0.k0, t0.kcnt, threadIdx.x - 128, amax_bar, ab)
+                : actq_quantize_t<Cfg, float>(args, smem, t0.k0, t0.kcnt, threadIdx.x - 128, amax_bar, ab);
+            if (actq_alpha >= 0.0f && threadIdx.x == 128) mbar_arrive(actq_bar);
+        }
         if constexpr (Cfg::SWIGLU) {
             // gs_h / e4m3(s) for all 256 scale codes, once per CTA (one entry per epilogue thread)
             gsh = __ldg(args.gs_h);
             const uint32_t code = threadIdx.x - 128;
-            const float sfd = e4m3_byte_to_f32(code);
+            const float sfd = e4m3_to_f32(code);
             rcp_tab[code] = (sfd == 0.0f) ? 0.0f : __fdiv_rn(gsh, sfd);
             named_bar_sync(1, 32 * kEpilogueWarps);
         }
@@ -1151,7 +1295,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             }
             tc_fence_after();
 
-            const float alpha = Cfg::GROUPED ? __ldg(args.alpha + ti.expert) : __ldg(args.alpha);
+            const float alpha = Cfg::ACTQ ? actq_alpha
+                              : Cfg::GROUPED ? __ldg(args.alpha + ti.expert) : __ldg(args.alpha);
             const uint32_t tacc = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) + acc * BN;
             const int p = ti.p0 + row;             // P row this thread owns
             const bool split_k = !Cfg::GROUPED && args.splits > 1;

@@ -87,6 +87,13 @@ struct GemmLaunch {
     uint8_t* h_sf = nullptr;
     const float* gs_h = nullptr;
     bool mx = false;            // MXFP4 operands (E8M0 scale per 32 elements, tiled scales)
+    // activations quantised inside the GEMM (few tokens): A is act [M, K] (fp32 or bf16)
+    const void* act = nullptr;
+    int64_t act_ld = 0;
+    bool act_bf16 = false;
+    const float* gs_b = nullptr;
+    float* gs_out = nullptr;
+    float* alpha_out = nullptr;
 };
 
 // api.cu: nvfp4_status of the current device's checks; fills the SM count and the device
@@ -97,6 +104,10 @@ int query_current_device(int* num_sms, unsigned** err_word);
 // pointers, K % 256, N % 8, sizes below 2^31, 16-byte alignment, alpha 4-byte aligned).
 int check_gemm_args(const void* A, const void* sfA, const void* B, const void* sfB,
                     const void* alpha, const void* out, int64_t N, int64_t K);
+
+// Stage ring depth of the activation-quantising few-token GEMM with token tile width bn (the
+// most K stages one CTA can hold); 0 for other widths.
+int act_gemm_stages(int bn);
 
 // Returns cudaSuccess or the first CUDA error; *encode_failed is set if a TMA descriptor
 // could not be encoded.

@@ -85,22 +85,29 @@ __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__
 
 // ------------------------------------------------------------------ expert-sorted permutation
 
-// Block e: the (token, slot) pairs routed to expert e, in ascending token order. Each thread
-// takes a contiguous range of tokens; a block scan of the per-thread hit counts gives each
-// hit its rank among expert e's pairs, written to rank_out[t k + s] (each pair has exactly one
-// expert, so exactly one block writes it). The expert's count goes to count_out[e].
-__global__ void __launch_bounds__(256) moe_rank_kernel(const int32_t* __restrict__ experts, int32_t T,
-                                                       int32_t k, int32_t* __restrict__ rank_out,
-                                                       int32_t* __restrict__ count_out)
+// Block e (1024 threads): the (token, slot) pairs routed to expert e, in ascending token
+// order. Each thread takes a contiguous range of at most ceil(T / 1024) tokens; a block scan
+// of the per-thread hit counts gives each hit its rank among expert e's pairs, written to
+// rank_out[t k + s] (each pair has exactly one expert, so exactly one block writes it). The
+// expert's count goes to count_out[e]. A token's k slots are read as one unrolled run of
+// independent loads (the second pass finds them in L1).
+constexpr int kRankThreads = 1024;
+
+__global__ void __launch_bounds__(kRankThreads) moe_rank_kernel(const int32_t* __restrict__ experts, int32_t T,
+                                                                int32_t k, int32_t* __restrict__ rank_out,
+                                                                int32_t* __restrict__ count_out)
 {
-    __shared__ int32_t warp_tot[8];
+    __shared__ int32_t warp_tot[kRankThreads / 32];
     const int e = blockIdx.x;
     const int tid = threadIdx.x;
-    const int chunk = (T + blockDim.x - 1) / blockDim.x;
+    const int chunk = (T + kRankThreads - 1) / kRankThreads;
     const int t0 = min(T, tid * chunk), t1 = min(T, t0 + chunk);
     int c = 0;
-    for (int t = t0; t < t1; ++t)
-        for (int s = 0; s < k; ++s) c += (__ldg(experts + static_cast<int64_t>(t) * k + s) == e);
+    for (int t = t0; t < t1; ++t) {
+        const int32_t* row = experts + static_cast<int64_t>(t) * k;
+#pragma unroll 8
+        for (int s = 0; s < k; ++s) c += (__ldg(row + s) == e);
+    }
     // exclusive scan over the block (thread order = token order)
     const int lane = tid & 31, warp = tid >> 5;
     int incl = c;
@@ -114,25 +121,23 @@ __global__ void __launch_bounds__(256) moe_rank_kernel(const int32_t* __restrict
     int base = 0;
     for (int w = 0; w < warp; ++w) base += warp_tot[w];
     int r = base + incl - c;
-    for (int t = t0; t < t1; ++t)
-        for (int s = 0; s < k; ++s)
-            if (__ldg(experts + static_cast<int64_t>(t) * k + s) == e) rank_out[static_cast<int64_t>(t) * k + s] = r++;
-    if (tid == blockDim.x - 1) count_out[e] = base + incl;
+    if (c > 0) {
+        for (int t = t0; t < t1; ++t) {
+            const int32_t* row = experts + static_cast<int64_t>(t) * k;
+#pragma unroll 8
+            for (int s = 0; s < k; ++s)
+                if (__ldg(row + s) == e) rank_out[static_cast<int64_t>(t) * k + s] = r++;
+        }
+    }
+    if (tid == kRankThreads - 1) count_out[e] = base + incl;
 }
 
-// One block: offsets[0] = 0, offsets[e + 1] = offsets[e] + count[e] (the counts are read from
-// offsets[1 .. E], where moe_rank_kernel left them); then for every pair p = t k + s:
-// row_of[p] = offsets[expert] + rank (the rank is read from row_of[p], in place) and
-// token_of_row[row_of[p]] = t.
-__global__ void __launch_bounds__(1024) moe_offsets_kernel(const int32_t* __restrict__ experts, int32_t T,
-                                                           int32_t E, int32_t k, int32_t* __restrict__ offsets,
-                                                           int32_t* __restrict__ row_of,
-                                                           int32_t* __restrict__ token_of_row)
+// One block: offsets[0] = 0, offsets[e + 1] = offsets[e] + count[e], in place (the counts are
+// read from offsets[1 .. E], where moe_rank_kernel left them; E <= 1024, one per thread).
+__global__ void __launch_bounds__(1024) moe_scan_kernel(int32_t E, int32_t* __restrict__ offsets)
 {
-    __shared__ int32_t s_off[1025];
     __shared__ int32_t warp_tot[32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // E <= 1024: one count per thread
     const int c = tid < E ? offsets[tid + 1] : 0;
     int incl = c;
 #pragma unroll
@@ -141,15 +146,26 @@ __global__ void __launch_bounds__(1024) moe_offsets_kernel(const int32_t* __rest
         if (lane >= d) incl += y;
     }
     if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
+    __syncthreads();                                   // every count has been read
     int base = 0;
     for (int w = 0; w < warp; ++w) base += warp_tot[w];
-    if (tid < E) s_off[tid + 1] = base + incl;
-    if (tid == 0) s_off[0] = 0;
+    if (tid < E) offsets[tid + 1] = base + incl;
+    if (tid == 0) offsets[0] = 0;
+}
+
+// Every pair p = t k + s: row_of[p] = offsets[expert] + rank (the rank is read from row_of[p],
+// in place) and token_of_row[row_of[p]] = t. Grid-stride; each block keeps the offsets in
+// shared memory.
+__global__ void __launch_bounds__(256) moe_fill_kernel(const int32_t* __restrict__ experts, int64_t pairs,
+                                                       int32_t E, int32_t k, const int32_t* __restrict__ offsets,
+                                                       int32_t* __restrict__ row_of,
+                                                       int32_t* __restrict__ token_of_row)
+{
+    __shared__ int32_t s_off[1025];
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
     __syncthreads();
-    for (int e = tid; e <= E; e += blockDim.x) offsets[e] = s_off[e];
-    const int64_t pairs = static_cast<int64_t>(T) * k;
-    for (int64_t p = tid; p < pairs; p += blockDim.x) {
+    for (int64_t p = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; p < pairs;
+         p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int32_t row = s_off[__ldg(experts + p)] + row_of[p];
         row_of[p] = row;
         token_of_row[row] = static_cast<int32_t>(p / k);
@@ -166,11 +182,21 @@ cudaError_t launch_moe_route(const float* logits, int32_t T, int32_t E, int32_t 
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    moe_rank_kernel<<<E, 256, 0, stream>>>(experts, T, k, row_of, offsets + 1);
+    moe_rank_kernel<<<E, kRankThreads, 0, stream>>>(experts, T, k, row_of, offsets + 1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    moe_offsets_kernel<<<1, 1024, 0, stream>>>(experts, T, E, k, offsets, row_of, token_of_row);
-    return cudaGetLastError();
+    moe_scan_kernel<<<1, 1024, 0, stream>>>(E, offsets);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t pairs = static_cast<int64_t>(T) * k;
+    if (pairs > 0) {
+        int64_t blocks = (pairs + 255) / 256;
+        if (blocks > 1024) blocks = 1024;
+        moe_fill_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(experts, pairs, E, k, offsets, row_of,
+                                                                          token_of_row);
+        e = cudaGetLastError();
+    }
+    return e;
 }
 
 // ------------------------------------------------------------------ combine
