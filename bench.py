@@ -356,13 +356,26 @@ class DenseStep:
         self.quant(s, stream)
         self.gemm(s, stream)
 
+    def act(self, s, stream=None):
+        """The same step as one launch: the few-token GEMM that quantises A itself."""
+        self.nv.gemm_act(s["a"], s["gsB"], s["Bq"], s["sfB"], out=s["out"], gs_out=s["gs"],
+                         alpha_out=s["alpha"], stream=stream)
+
     def time_all(self):
-        """(gemm_us, quant_us, step_us) per launch / step, each from its own graph."""
+        """(gemm_us, quant_us, step_us, act_us) per launch / step, each from its own graph
+        (act_us: the one-launch step of nvfp4_gemm_act, None where it does not apply)."""
         self.step(self.sets[0])
         g = graph_time_us([lambda s=s: self.gemm(s) for s in self.sets])
         q = graph_time_us([lambda s=s: self.quant(s) for s in self.sets])
         st = graph_time_us([lambda s=s: self.step(s) for s in self.sets])
-        return g, q, st
+        act = None
+        if self.M <= 64:
+            try:
+                self.act(self.sets[0])
+                act = graph_time_us([lambda s=s: self.act(s) for s in self.sets])
+            except self.nv.Nvfp4Error:
+                act = None
+        return g, q, st, act
 
 
 class GroupedStep:
@@ -542,14 +555,19 @@ def per_config(dev, peaks, log):
         for c in cases:
             t0 = time.perf_counter()
             ds = DenseStep(nv, c.M, c.N, c.K, c.a(), c.b(), dev)
-            g, q, st = ds.time_all()
+            g, q, st, act = ds.time_all()
             it = dense_entry(c.name, c.M, c.N, c.K, g, q, st, len(ds.sets), ds.set_bytes, peaks)
+            if act is not None:
+                fl = 2.0 * c.M * c.N * c.K
+                it["act_step_us"] = round(act, 3)
+                it["act_step_tflops"] = round(fl / (act * 1e-6) / 1e12, 1)
+                it["act_step_note"] = "nvfp4_gemm_act: quantisation of A and the GEMM in one launch"
             if extra is not None:
                 extra(c, ds, it)
             items.append(it)
             del ds
             torch.cuda.empty_cache()
-            log(f"  {c.name}: gemm {g:.2f} us, quant {q:.2f} us, step {st:.2f} us "
+            log(f"  {c.name}: gemm {g:.2f} us, quant {q:.2f} us, step {st:.2f} us, act step {act} us "
                 f"({time.perf_counter() - t0:.1f} s)")
         tot_fl = sum(2.0 * i["M"] * i["N"] * i["K"] for i in items)
         tot_g = sum(i["gemm_us"] for i in items)

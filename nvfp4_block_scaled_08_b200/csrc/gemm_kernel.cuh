@@ -983,18 +983,6 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     uint8_t* sfpb = smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES;
                     uint8_t* sfqb = smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES;
                     if constexpr (Cfg::GROUPED) {
-                        // Weight tiles are streamed from HBM once: besides the STAGES in the
-                        // ring, keep the next STAGES of this tile requested into L2 (a prefetch
-                        // needs no shared memory), doubling the weight bytes in flight per SM.
-                        auto prefetch_w = [&](int32_t kk) {
-                            if constexpr (Cfg::SWIGLU)
-                                tma_prefetch_5d(&tm_p, kk * Cfg::BK_BYTES, 0, 0, ti.p0 >> 5, ti.expert);
-                            else
-                                tma_prefetch_3d(&tm_p, kk * Cfg::BK_BYTES, ti.p0, ti.expert);
-                        };
-                        if (ks == 0)
-                            for (int32_t j = STAGES; j < 2 * STAGES - 1 && j < ti.kcnt; ++j) prefetch_w(ti.k0 + j);
-                        if (ks + 2 * STAGES - 1 < ti.kcnt) prefetch_w(ti.k0 + ks + 2 * STAGES - 1);
                         // boxes of QBOX token rows covering the tile's MMA N (its rows rounded
                         // up to 16); the 8-row swizzle atoms of the boxes line up as in one box
                         const int n_mma = min(BN, (ti.q_valid + 15) & ~15);

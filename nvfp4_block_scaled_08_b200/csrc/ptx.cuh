@@ -147,14 +147,6 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int32_t 
                  ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z) : "memory");
 }
 
-__device__ __forceinline__ void tma_prefetch_5d(const CUtensorMap* map, int32_t c0, int32_t c1, int32_t c2,
-                                                int32_t c3, int32_t c4)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];"
-                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-                 : "memory");
-}
-
 // 2-D tile load global -> shared, completion counted on `bar` (bytes).
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x, int32_t y, uint64_t policy)
