@@ -403,7 +403,7 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint
  *   cluster     split-K CTAs per thread-block cluster, 1 ... 8;
  *   groups      split-K clusters per output tile, reduced through the workspace (needs one);
  *   band        output P tiles per rasterisation band;
- *   grouped_bn  token tile width of the grouped GEMM: 32, 64, 128 or 256;
+ *   grouped_bn  token tile width of the grouped GEMM: 32, 64, 128, 176 or 256;
  *   pair        CTA pairs that share 256-row weight tiles (128 x 256 tiles with tiled scales and
  *               no split-K): 2 = wherever possible, 0 or 1 = never (the planner does not use them).
  * The planner's choices need no override; results stay within the GEMM tolerance under any

@@ -137,10 +137,12 @@ GemmPlan plan_grouped(int32_t E, int64_t total_rows, int64_t N, int64_t K, int n
     GemmPlan p;
     p.grouped = true;
     p.swap = true;
+    // 176-row tiles cover experts of up to 176 rows in one tile with a 44 KB stage (5 deep)
+    // where 256-row tiles need 54 KB (4 deep): more weight bytes in flight per SM
     const int64_t avg = E > 0 ? total_rows / E : 0;
-    p.bn = avg <= 24 ? 32 : avg <= 48 ? 64 : avg <= 96 ? 128 : 256;
+    p.bn = avg <= 24 ? 32 : avg <= 48 ? 64 : avg <= 96 ? 128 : avg <= 140 ? 176 : 256;
     const int force = g_force_grouped_bn.load(std::memory_order_relaxed);
-    if (force == 32 || force == 64 || force == 128 || force == 256) p.bn = force;
+    if (force == 32 || force == 64 || force == 128 || force == 176 || force == 256) p.bn = force;
     p.p_tiles = ceil_div(N, 128);
     p.splits = 1;
     p.grid = num_sms;
@@ -485,6 +487,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
             case 32: return run<32, true, true, false, true>(plan, L, stream, encode_failed);
             case 64: return run<64, true, true, false, true>(plan, L, stream, encode_failed);
             case 128: return run<128, true, true, false, true>(plan, L, stream, encode_failed);
+            case 176: return run<176, true, true, false, true>(plan, L, stream, encode_failed);
             case 256: return run<256, true, true, false, true>(plan, L, stream, encode_failed);
             default: return cudaErrorInvalidValue;
         }
@@ -494,6 +497,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
             case 32: return run<32, true, true>(plan, L, stream, encode_failed);
             case 64: return run<64, true, true>(plan, L, stream, encode_failed);
             case 128: return run<128, true, true>(plan, L, stream, encode_failed);
+            case 176: return run<176, true, true>(plan, L, stream, encode_failed);
             case 256: return run<256, true, true>(plan, L, stream, encode_failed);
             default: return cudaErrorInvalidValue;
         }

@@ -163,7 +163,9 @@ struct GemmCfg {
     static constexpr uint32_t TX_BYTES = P_BYTES + Q_BYTES + SF_TMA_P + SF_TMA_Q;
     // Grouped: the token tile is loaded in boxes of QBOX rows, only as many as the expert's
     // rows in the tile need (a tile of a 256-wide plan often holds ~128 rows of one expert).
-    static constexpr int QBOX = BN < 64 ? BN : 64;
+    // (176-row tiles: two boxes of 88, which end exactly at the tile)
+    static constexpr int QBOX = BN < 64 ? BN : (BN == 176 ? 88 : 64);
+    static_assert(!GROUPED || BN % QBOX == 0, "token boxes tile the token buffer");
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
 
     // TMEM columns: two accumulators, then the scale factors: SFA (4 k-blocks x 4 columns),
@@ -603,7 +605,8 @@ template <class Cfg, typename T>
 __device__ __forceinline__ float actq_quantize_t(const GemmArgs& a, uint8_t* smem, int k0, int kcnt, int e,
                                                  uint64_t* amax_bar, const AbortState& ab)
 {
-    constexpr int V = InTraits<T>::kPerThread;
+    using Raw = typename InTraits<T>::Raw;
+    constexpr int U = 4;                                       // loads in flight per thread
     const T* x = static_cast<const T*>(a.act);
     const int M = a.M;
     const uint32_t per_row = static_cast<uint32_t>(kcnt) * 32u;
@@ -611,10 +614,11 @@ __device__ __forceinline__ float actq_quantize_t(const GemmArgs& a, uint8_t* sme
     float* rcp_tab = reinterpret_cast<float*>(smem + Cfg::OFF_ACTQ);
     float* slots = reinterpret_cast<float*>(smem + Cfg::OFF_ACTQ + 1024);
     float* red = reinterpret_cast<float*>(smem + Cfg::OFF_ACTQ + 1024 + 64);
-    auto load = [&](uint32_t v, float (&vals)[8]) {
+    auto load = [&](uint32_t v) -> Raw {
+        if (v >= nvec) return InTraits<T>::zero();
         const uint32_t r = v / per_row, w = v - r * per_row;
         const int64_t k = (static_cast<int64_t>(k0) + (w >> 5)) * 256 + (w & 31) * 8;
-        InTraits<T>::decode(InTraits<T>::load(x + static_cast<int64_t>(r) * a.act_ld + k), vals);
+        return InTraits<T>::load(x + static_cast<int64_t>(r) * a.act_ld + k);
     };
 
     // zero the slice's Q stages (padding token rows stay zero) while the first loads fly
@@ -626,11 +630,17 @@ __device__ __forceinline__ float actq_quantize_t(const GemmArgs& a, uint8_t* sme
     }
     // 1. the slice's maximum
     float m = 0.0f;
-    for (uint32_t v = e; v < nvec; v += 256) {
-        float vals[8];
-        load(v, vals);
+    for (uint32_t v0 = e; v0 < nvec; v0 += 256 * U) {
+        Raw raw[U];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(vals[k]));
+        for (int u = 0; u < U; ++u) raw[u] = load(v0 + 256 * u);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float vals[8];
+            InTraits<T>::decode(raw[u], vals);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(vals[k]));
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -669,30 +679,38 @@ __device__ __forceinline__ float actq_quantize_t(const GemmArgs& a, uint8_t* sme
         if (a.alpha_out) *a.alpha_out = alpha;
     }
     named_bar_sync(1, 256);
-    // 3. codes and block scales into the Q stages
+    // 3. codes and block scales into the Q stages: the warp takes 32 consecutive vectors
+    //    (lanes 2j, 2j + 1 share a 16-element block), U groups of them per round
     const int lane = e & 31;
-    for (uint32_t v0 = e & ~31; v0 < nvec; v0 += 256) {     // warp-uniform (nvec % 32 == 0)
-        const uint32_t v = v0 + lane;
-        float vals[8];
-        load(v, vals);
-        float bm = 0.0f;
+    for (uint32_t w0 = static_cast<uint32_t>(e & ~31); w0 < nvec; w0 += 256 * U) {   // warp-uniform
+        Raw raw[U];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) bm = fmaxf(bm, fabsf(vals[k]));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-        const uint32_t sfq = f32_to_e4m3(__fmul_rn(__fdiv_rn(bm, 6.0f), gs));
-        const uint32_t packed = scale_to_e2m1x8(vals, rcp_tab[sfq]);
-        const uint32_t r = v / per_row, w = v - r * per_row;
-        const uint32_t st = w >> 5, u = w & 31;
-        const uint32_t kbyte = u * 4;                          // 4 code bytes per vector
-        uint8_t* qs = smem + Cfg::OFF_Q + st * Cfg::Q_BYTES + r * 128;
-        *reinterpret_cast<uint32_t*>(qs + ((((kbyte >> 4) ^ (r & 7u)) << 4) | (kbyte & 15u))) = packed;
-        if ((u & 1u) == 0) {
-            const uint32_t kb = u >> 1;                        // 16-element block of the stage
-            smem[Cfg::OFF_SFQ + st * Cfg::SFQ_BYTES + (kb >> 2) * 512 + (r & 31u) * 16 + ((r >> 5) & 3u) * 4 +
-                 (kb & 3u)] = static_cast<uint8_t>(sfq);
+        for (int u = 0; u < U; ++u) raw[u] = load(w0 + 256 * u + lane);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t vb = w0 + 256 * u;
+            if (vb >= nvec) break;                             // warp-uniform (nvec % 32 == 0)
+            const uint32_t v = vb + lane;
+            float vals[8];
+            InTraits<T>::decode(raw[u], vals);
+            float bm = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) bm = fmaxf(bm, fabsf(vals[k]));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+            const uint32_t sfq = f32_to_e4m3(__fmul_rn(__fdiv_rn(bm, 6.0f), gs));
+            const uint32_t packed = scale_to_e2m1x8(vals, rcp_tab[sfq]);
+            const uint32_t r = v / per_row, w = v - r * per_row;
+            const uint32_t st = w >> 5, uu = w & 31;
+            const uint32_t kbyte = uu * 4;                     // 4 code bytes per vector
+            uint8_t* qs = smem + Cfg::OFF_Q + st * Cfg::Q_BYTES + r * 128;
+            *reinterpret_cast<uint32_t*>(qs + ((((kbyte >> 4) ^ (r & 7u)) << 4) | (kbyte & 15u))) = packed;
+            if ((uu & 1u) == 0) {
+                const uint32_t kb = uu >> 1;                   // 16-element block of the stage
+                smem[Cfg::OFF_SFQ + st * Cfg::SFQ_BYTES + (kb >> 2) * 512 + (r & 31u) * 16 + ((r >> 5) & 3u) * 4 +
+                     (kb & 3u)] = static_cast<uint8_t>(sfq);
+            }
         }
     }
-    (void)V;
     fence_proxy_async_smem();                                  // generic writes -> tensor core reads
     named_bar_sync(1, 256);
     return alpha;

@@ -66,11 +66,19 @@ def test_grouped_single_expert_and_all_empty_but_one(cuda_device):
     _small_case(cuda_device, [300], 128, 768, 13)
 
 
-@pytest.mark.parametrize("rows_each", [16, 128, 200])
+@pytest.mark.parametrize("rows_each", [16, 128, 160, 200])
 def test_grouped_token_tile_widths(cuda_device, rows_each):
-    # mean rows per expert drives the token-tile width (32, 64, 128 or 256)
+    # mean rows per expert drives the token-tile width (32, 64, 128, 176 or 256); at 160 the
+    # 176-row tiles (two 88-row boxes) hold 157..165 rows
     _small_case(cuda_device, [rows_each - 3, rows_each, rows_each + 5, rows_each - 1], 384, 1024,
                 rows_each)
+
+
+@pytest.mark.parametrize("grouped_bn", [32, 64, 128, 176, 256])
+def test_grouped_every_forced_tile_width(cuda_device, grouped_bn):
+    # ragged experts (empty, 1 row, a tile and a bit, several tiles) in every token-tile width
+    with nv.plan_override(grouped_bn=grouped_bn):
+        _small_case(cuda_device, [0, 1, 177, 90, 3, 400, 0, 33], 264, 512, 40 + grouped_bn, pad_rows=3)
 
 
 def _full_config(dev, case: workloads.GroupedCase, n_experts_checked=5, n_cols=192):

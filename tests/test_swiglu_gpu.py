@@ -59,7 +59,7 @@ def _run_gpu(dev, Aq, sfA, Bq, sfB, alphas, off, gs_h, rows_total, pad=3):
     return hq[:rows_total].cpu().numpy(), hsf[:rows_total].cpu().numpy()
 
 
-@pytest.mark.parametrize("grouped_bn", [32, 64, 128, 256])
+@pytest.mark.parametrize("grouped_bn", [32, 64, 128, 176, 256])
 def test_swiglu_bit_exact_on_exact_products(cuda_device, grouped_bn):
     d = cuda_device
     rng = np.random.default_rng(7 + grouped_bn)
