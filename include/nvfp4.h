@@ -70,10 +70,21 @@ typedef enum {
  *                    Each block's 16-byte row i holds the scales of rows i, i + 32, i + 64, i + 96:
  *                    the operand layout of the tensor cores' scale copies, so the GEMM fetches a
  *                    stage's scales with one bulk copy per 128 rows. Requires K % 64 == 0.
+ *   NVFP4_SF_8X4:    32-byte blocks of 8 rows x 4 scales, row-major inside the block, a row group's
+ *                    blocks consecutive along K: the scale of row r, column c is at byte
+ *                        ((r / 8) * (K / 64) + c / 4) * 32 + (r % 8) * 4 + c % 4,
+ *                    rows padded to a multiple of 8 (the padding is never read into an output).
+ *                    The mm_fp4 signature's use_8x4_sf_layout ("The Art of Reading the Manual",
+ *                    section "The Message") names an 8 x 4 scale layout without defining it; this
+ *                    is the library's reading: the tiled layout's 4-scale columns with 8-row
+ *                    instead of 128-row groups, so that a few-token scale matrix is padded to 8
+ *                    rows, not 128. The dense NVFP4 GEMM reads it directly (one 2D copy per stage
+ *                    and operand, re-laid in shared memory). Requires K % 64 == 0.
  */
 typedef enum {
     NVFP4_SF_LINEAR = 0,
-    NVFP4_SF_TILED = 1
+    NVFP4_SF_TILED = 1,
+    NVFP4_SF_8X4 = 2
 } nvfp4_sf_layout;
 
 /*
@@ -138,7 +149,8 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, nvfp4_in_dtype dtype, int64_t
 
 /*
  * nvfp4_quantize_dynamic with the scales written in the given layout (the same values; for
- * NVFP4_SF_TILED, sf holds nvfp4_sf_bytes(rows, K, NVFP4_SF_TILED) bytes and K % 64 == 0).
+ * NVFP4_SF_TILED and NVFP4_SF_8X4, sf holds nvfp4_sf_bytes(rows, K, sf_layout) bytes and
+ * K % 64 == 0; the padding rows' bytes are left as they are).
  * nvfp4_quantize_dynamic is this call with NVFP4_SF_LINEAR.
  */
 nvfp4_status nvfp4_quantize_dynamic_ex(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K,
@@ -157,6 +169,13 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t K, nvfp4_sf_layout sf_layout);
  */
 nvfp4_status nvfp4_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* sf_tiled,
                            cudaStream_t stream);
+
+/*
+ * Re-lays row-major scales sf[rows][K/16] (device) out as NVFP4_SF_8X4 into sf_8x4 (device,
+ * nvfp4_sf_bytes(rows, K, NVFP4_SF_8X4) bytes; padding rows become 0). K % 64 == 0. One launch.
+ */
+nvfp4_status nvfp4_sf_8x4(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* sf_8x4,
+                          cudaStream_t stream);
 
 /*
  * GEMM scale from the two global scales: alpha[i] = 1 / (gs_a[0] * gs_b[i]) in fp32,
@@ -192,7 +211,8 @@ nvfp4_status nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
  * nvfp4_gemm on the same scales in the linear layout. NVFP4_SF_TILED skips the
  * kernel's scale re-layout step (one bulk copy per stage and 128 rows) and is the faster
  * layout. With tuning overrides that place token tiles off 128-row tile boundaries it returns
- * NVFP4_ERR_UNSUPPORTED_SHAPE. nvfp4_gemm is this call with NVFP4_SF_LINEAR.
+ * NVFP4_ERR_UNSUPPORTED_SHAPE. NVFP4_SF_8X4 runs every tiling the linear layout runs (tiles
+ * start on 8-row boundaries). nvfp4_gemm is this call with NVFP4_SF_LINEAR.
  */
 nvfp4_status nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
                            const uint8_t* sfB, const float* alpha, void* out,

@@ -69,6 +69,7 @@ SIGNATURES = {
                                                  ctypes.c_int32, _P, ctypes.c_int, _P]),
     "nvfp4_sf_bytes": (_SZ, [_I64, _I64, ctypes.c_int]),
     "nvfp4_sf_tile": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "nvfp4_sf_8x4": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "nvfp4_gemm_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int, _P]),
     "nvfp4_gemm_ex2": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int,
                                       ctypes.c_int, _P]),
@@ -180,11 +181,20 @@ def quantize(x: torch.Tensor, gs: torch.Tensor, q: torch.Tensor | None = None,
     return q, sf
 
 
-SF_LINEAR, SF_TILED = 0, 1
+SF_LINEAR, SF_TILED, SF_8X4 = 0, 1, 2
 
 
-def sf_bytes(rows: int, K: int, tiled: bool = False) -> int:
-    return int(load().nvfp4_sf_bytes(rows, K, SF_TILED if tiled else SF_LINEAR))
+def _layout(tiled: bool, layout: int | None) -> int:
+    """Scale layout code from the `tiled` flag or an explicit SF_* `layout` (which wins)."""
+    if layout is None:
+        return SF_TILED if tiled else SF_LINEAR
+    if layout not in (SF_LINEAR, SF_TILED, SF_8X4):
+        raise ValueError("layout must be SF_LINEAR, SF_TILED or SF_8X4")
+    return layout
+
+
+def sf_bytes(rows: int, K: int, tiled: bool = False, layout: int | None = None) -> int:
+    return int(load().nvfp4_sf_bytes(rows, K, _layout(tiled, layout)))
 
 
 def sf_tile(sf: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -196,12 +206,22 @@ def sf_tile(sf: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> t
     return out
 
 
+def sf_8x4(sf: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Row-major scales [rows, K/16] -> the 8 x 4 layout (flat uint8 tensor)."""
+    rows, K = sf.shape[0], sf.shape[1] * 16
+    if out is None:
+        out = torch.empty(sf_bytes(rows, K, layout=SF_8X4), dtype=torch.uint8, device=sf.device)
+    _check("nvfp4_sf_8x4", load().nvfp4_sf_8x4(_ptr(sf), rows, K, _ptr(out), _stream(stream)))
+    return out
+
+
 def quantize_dynamic(x: torch.Tensor, gs_other: torch.Tensor | None = None,
                      gs: torch.Tensor | None = None, q: torch.Tensor | None = None,
                      sf: torch.Tensor | None = None, alpha_out: torch.Tensor | None = None,
-                     stream=None, tiled: bool = False):
+                     stream=None, tiled: bool = False, layout: int | None = None):
     """Global scale + quantisation (+ alpha against gs_other) in one launch; tiled: scales in
-    the tiled layout (a flat uint8 tensor of sf_bytes(rows, K, True) bytes).
+    the tiled layout (a flat uint8 tensor of sf_bytes(rows, K, True) bytes); layout: any SF_*
+    layout (overrides tiled; SF_8X4 gives a flat tensor of sf_bytes(rows, K, layout=SF_8X4)).
 
     Returns (q, sf, gs, alpha) where alpha is None when gs_other is None."""
     _dev(x, "x")
@@ -210,8 +230,9 @@ def quantize_dynamic(x: torch.Tensor, gs_other: torch.Tensor | None = None,
     rows, K = x.shape
     if q is None:
         q = torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device)
+    lay = _layout(tiled, layout)
     if sf is None:
-        sf = (torch.empty(sf_bytes(rows, K, True), dtype=torch.uint8, device=x.device) if tiled
+        sf = (torch.empty(sf_bytes(rows, K, layout=lay), dtype=torch.uint8, device=x.device) if lay != SF_LINEAR
               else torch.empty(rows, K // 16, dtype=torch.uint8, device=x.device))
     if gs is None:
         gs = torch.empty(1, dtype=torch.float32, device=x.device)
@@ -220,8 +241,7 @@ def quantize_dynamic(x: torch.Tensor, gs_other: torch.Tensor | None = None,
         alpha_out = torch.empty(n, dtype=torch.float32, device=x.device)
     _check("nvfp4_quantize_dynamic_ex", load().nvfp4_quantize_dynamic_ex(
         _ptr(x), _dtype_code(x), rows, K, x.stride(0), _ptr(gs), _ptr(q), _ptr(sf),
-        _ptr(gs_other), n, _ptr(alpha_out) if n else None, SF_TILED if tiled else SF_LINEAR,
-        _stream(stream)))
+        _ptr(gs_other), n, _ptr(alpha_out) if n else None, lay, _stream(stream)))
     return q, sf, gs, (alpha_out if n else None)
 
 
@@ -260,14 +280,14 @@ def _out_code(out: torch.Tensor) -> int:
 
 
 def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None, tiled=False,
-         out_dtype=torch.bfloat16) -> torch.Tensor:
+         out_dtype=torch.bfloat16, layout: int | None = None) -> torch.Tensor:
     """out[M, N] = alpha * sum_k deq(A)[m,k] deq(B)[n,k] in bf16, fp16 or fp32.
 
     Aq [M, K/2] uint8, sfA [M, K/16] uint8, Bq [N, K/2], sfB [N, K/16], alpha_t fp32 [1];
     out [M, N] (allocated with out_dtype if None; otherwise its dtype decides); workspace:
     zero-filled uint8 tensor of gemm_workspace_size(M, N, K) bytes or None (no split-K).
     tiled: sfA and sfB in the tiled layout (flat uint8 tensors from sf_tile or
-    quantize_dynamic(tiled=True))."""
+    quantize_dynamic(tiled=True)); layout: any SF_* layout of both (overrides tiled)."""
     M, K = Aq.shape[0], Aq.shape[1] * 2
     N = Bq.shape[0]
     if out is None:
@@ -275,7 +295,7 @@ def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None, tiled
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
     _check("nvfp4_gemm_ex2", load().nvfp4_gemm_ex2(
         _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alpha_t), _ptr(out), M, N, K,
-        ws_ptr, ws_bytes, SF_TILED if tiled else SF_LINEAR, _out_code(out), _stream(stream)))
+        ws_ptr, ws_bytes, _layout(tiled, layout), _out_code(out), _stream(stream)))
     return out
 
 

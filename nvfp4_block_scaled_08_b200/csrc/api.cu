@@ -200,13 +200,14 @@ nvfp4_status nvfp4_quantize_dynamic_ex(const void* x, nvfp4_in_dtype dtype, int6
 {
     if (rows < 0 || K < 0 || n_alpha < 0) return NVFP4_ERR_INVALID_ARG;
     if (dtype != NVFP4_IN_F32 && dtype != NVFP4_IN_BF16) return NVFP4_ERR_INVALID_ARG;
-    if (sf_layout != NVFP4_SF_LINEAR && sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_INVALID_ARG;
+    if (sf_layout != NVFP4_SF_LINEAR && sf_layout != NVFP4_SF_TILED && sf_layout != NVFP4_SF_8X4)
+        return NVFP4_ERR_INVALID_ARG;
     if (!gs_out) return NVFP4_ERR_INVALID_ARG;
     if (n_alpha > 0 && (!gs_other || !alpha_out)) return NVFP4_ERR_INVALID_ARG;
     if (rows == 0 || K == 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;   // no tensor to take a scale of
     if (!x || !q || !sf) return NVFP4_ERR_INVALID_ARG;
     if (K % 16 != 0 || K > kMaxDim || rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (sf_layout == NVFP4_SF_TILED && K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (sf_layout != NVFP4_SF_LINEAR && K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (ld_x < K) return NVFP4_ERR_INVALID_ARG;
     const int64_t esz = dtype == NVFP4_IN_BF16 ? 2 : 4;
     if (rows * (K * esz / 16) >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -217,7 +218,7 @@ nvfp4_status nvfp4_quantize_dynamic_ex(const void* x, nvfp4_in_dtype dtype, int6
     nvfp4_status st = current_device(&d);
     if (st != NVFP4_OK) return st;
     return from_cuda(nvfp4::launch_quantize_dynamic(x, dtype == NVFP4_IN_BF16, rows, K, ld_x, gs_out, q, sf,
-                                                    sf_layout == NVFP4_SF_TILED, gs_other, n_alpha,
+                                                    static_cast<int>(sf_layout), gs_other, n_alpha,
                                                     alpha_out, d.err_word, stream, d.num_sms));
 }
 
@@ -236,6 +237,8 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t K, nvfp4_sf_layout sf_layout)
     if (sf_layout == NVFP4_SF_LINEAR) return static_cast<size_t>(rows) * static_cast<size_t>(K / 16);
     if (sf_layout == NVFP4_SF_TILED && K % 64 == 0)
         return static_cast<size_t>((rows + 127) / 128 * 128) * static_cast<size_t>(K / 16);
+    if (sf_layout == NVFP4_SF_8X4 && K % 64 == 0)
+        return static_cast<size_t>((rows + 7) / 8 * 8) * static_cast<size_t>(K / 16);
     return 0;
 }
 
@@ -249,6 +252,18 @@ nvfp4_status nvfp4_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* 
     nvfp4_status st = current_device(&d);
     if (st != NVFP4_OK) return st;
     return from_cuda(nvfp4::launch_sf_tile(sf, rows, K, sf_tiled, stream, d.num_sms));
+}
+
+nvfp4_status nvfp4_sf_8x4(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* sf_8x4, cudaStream_t stream)
+{
+    if (rows < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0 || K == 0) return NVFP4_OK;
+    if (!sf || !sf_8x4) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0 || K > kMaxDim || rows > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    DeviceInfo d;
+    nvfp4_status st = current_device(&d);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_sf_8x4(sf, rows, K, sf_8x4, stream, d.num_sms));
 }
 
 nvfp4_status nvfp4_alpha(const float* gs_a, const float* gs_b, int32_t n, float* alpha,
@@ -278,7 +293,8 @@ nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t*
                             cudaStream_t stream)
 {
     if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
-    if (sf_layout != NVFP4_SF_LINEAR && sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_INVALID_ARG;
+    if (sf_layout != NVFP4_SF_LINEAR && sf_layout != NVFP4_SF_TILED && sf_layout != NVFP4_SF_8X4)
+        return NVFP4_ERR_INVALID_ARG;
     if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F16 && out_dtype != NVFP4_OUT_F32)
         return NVFP4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return NVFP4_OK;
@@ -297,6 +313,7 @@ nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t*
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0, ws, d.err_word, tiled,
                         static_cast<int32_t>(out_dtype)};
+    L.sf_8x4 = sf_layout == NVFP4_SF_8X4;
     bool enc_failed = false;
     cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
     if (enc_failed) return NVFP4_ERR_CUDA;

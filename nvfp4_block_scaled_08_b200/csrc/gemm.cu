@@ -366,6 +366,13 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
             a.sf_p = sP;
             a.sf_q = sQ;
             a.sf_kb4 = static_cast<int32_t>(L.K / (MX ? 128 : 64));   // 512-byte blocks per 128 rows
+        } else if (L.sf_8x4) {
+            // rows of the map: 8-row groups of K / 2 bytes; a stage's box: 128 bytes of 128 / 8
+            // (P) or BN / 8 (Q) groups, the same bytes as the row-major box
+            const uint64_t gb = static_cast<uint64_t>(L.K / 2);
+            ok &= get_map(&tsp, sP, 2, gb, (p_rows + 7) / 8, 1, gb, 0, 128, 128 / 8, false);
+            ok &= get_map(&tsq, sQ, 2, gb, (q_rows + 7) / 8, 1, gb, 0, 128, BN / 8, false);
+            a.sf_8x4 = 1;
         } else {
             ok &= get_map(&tsp, sP, 2, ks, p_rows, 1, ks, 0, 16, 128, false);
             ok &= get_map(&tsq, sQ, 2, ks, q_rows, 1, ks, 0, 16, BN, false);
@@ -463,6 +470,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
             default: return cudaErrorInvalidValue;
         }
     }
+    if (L.sf_8x4 && (plan.grouped || L.sf_tiled || L.h_q != nullptr)) return cudaErrorInvalidValue;
     if (L.sf_tiled) {
         if (plan.grouped) return cudaErrorInvalidValue;
         if (plan.swap) {

@@ -87,6 +87,7 @@ struct GemmArgs {
     const uint8_t* sf_p;      // SFT: tiled scales of the P / Q operands
     const uint8_t* sf_q;
     int32_t sf_kb4;           // SFT: 512-byte scale blocks per 128-row tile (K / 64)
+    int32_t sf_8x4;           // linear-path scales in the 8 x 4 layout (1) or row-major (0)
     const int32_t* expert_offsets;  // grouped: [E + 1]
     int32_t num_experts;
     int32_t total_rows;       // grouped: rows of A / out
@@ -1070,11 +1071,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                                       args.sf_q + (((ti.q0 >> 7) + g) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
                                       Cfg::SFP_BYTES, fb, pol_q);
                     } else {
+                        // row-major scales: [rows][16 B] per stage; 8 x 4 scales: the scale map's
+                        // rows are 8-row groups, a stage's 4 blocks of one group 128 contiguous
+                        // bytes at byte 128 * stage (tiles start on 8-row boundaries)
+                        const int32_t sfx = args.sf_8x4 ? kx : sx;
+                        const int32_t sfr = args.sf_8x4 ? 3 : 0;
                         mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
                         tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
-                        tma_load_2d(sfpb, &tm_sfp, fb, sx, ti.p0, pol_p);
+                        tma_load_2d(sfpb, &tm_sfp, fb, sfx, ti.p0 >> sfr, pol_p);
                         tma_load_2d(qbuf, &tm_q, fb, kx, ti.q0, pol_q);
-                        tma_load_2d(sfqb, &tm_sfq, fb, sx, ti.q0, pol_q);
+                        tma_load_2d(sfqb, &tm_sfq, fb, sfx, ti.q0 >> sfr, pol_q);
                     }
                 }
                 __syncwarp();
@@ -1206,12 +1212,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         __syncwarp();
     } else if (!Cfg::SFT && (warp == 2 || warp == 3)) {
         // -------------------------------------------------------------- scale re-layout
-        // The TMA wrote row r's 16 scale bytes (k-blocks 0..15 of the stage) at r * 16.
+        // The TMA wrote row r's 16 scale bytes (k-blocks 0..15 of the stage) at r * 16
+        // (8 x 4 layout: row r's k-step j word at (r / 8) * 128 + j * 32 + (r % 8) * 4).
         // The MMA for k-step j (k-blocks 4j..4j+3) needs, per 128-row group, a 512-byte
         // block whose 16-byte row i holds the 4 scale bytes of rows i, i+32, i+64, i+96.
         // Each lane owns row i = lane: it reads its 4 rows (16 B each), transposes the
         // 4 x 4 words in registers and writes 4 blocks (one per k-step), in place.
         // Warps 2 and 3 take alternate stages.
+        const bool in_8x4 = args.sf_8x4 != 0;
         const uint32_t sf_warp = static_cast<uint32_t>(warp - 2);
         uint32_t stage = 0, phase = 0, seq = 0;
         for (int32_t t = tile_start; t < num_tiles; t += tile_step) {
@@ -1235,8 +1243,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int r = 32 * q + lane;
-                        v[q] = (r < rows_here) ? *reinterpret_cast<const uint4*>(base + 16 * r)
-                                               : make_uint4(0u, 0u, 0u, 0u);
+                        if (r >= rows_here) {
+                            v[q] = make_uint4(0u, 0u, 0u, 0u);
+                        } else if (in_8x4) {
+                            const uint32_t* w = reinterpret_cast<const uint32_t*>(base + (r >> 3) * 128 + (r & 7) * 4);
+                            v[q] = make_uint4(w[0], w[8], w[16], w[24]);
+                        } else {
+                            v[q] = *reinterpret_cast<const uint4*>(base + 16 * r);
+                        }
                     }
                     __syncwarp();
                     uint4 o0 = make_uint4(v[0].x, v[1].x, v[2].x, v[3].x);

@@ -16,8 +16,9 @@ cudaError_t launch_global_scale(const void* x, bool bf16, int64_t numel, float* 
 cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
                             const float* gs, uint8_t* q, uint8_t* sf, cudaStream_t stream,
                             int num_sms);
+// sf_layout: 0 linear, 1 tiled (128 x 4), 2 8 x 4 (nvfp4_sf_layout)
 cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
-                                    float* gs_out, uint8_t* q, uint8_t* sf, bool sf_tiled,
+                                    float* gs_out, uint8_t* q, uint8_t* sf, int sf_layout,
                                     const float* gs_other, int32_t n_alpha, float* alpha_out,
                                     unsigned* err_word, cudaStream_t stream, int num_sms);
 // Dynamic quantisation of x[T, H] (global scale over all of x) with every row t's codes and
@@ -33,6 +34,9 @@ cudaError_t launch_moe_route(const float* logits, int32_t T, int32_t E, int32_t 
 cudaError_t launch_moe_combine(const void* y, int32_t y_dt, const float* weights, const int32_t* row_of,
                                int32_t T, int64_t H, int32_t k, void* out, int32_t out_dt, cudaStream_t stream,
                                int num_sms);
+// Row-major NVFP4 scales [rows][K / 16] -> the 8 x 4 layout.
+cudaError_t launch_sf_8x4(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* out, cudaStream_t stream,
+                          int num_sms);
 // Row-major scales [rows][K / block] -> the tiled layout (block = 16: NVFP4, 32: MXFP4).
 cudaError_t launch_sf_tile(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* out, cudaStream_t stream,
                            int num_sms, int block = 16);
@@ -94,6 +98,7 @@ struct GemmLaunch {
     const float* gs_b = nullptr;
     float* gs_out = nullptr;
     float* alpha_out = nullptr;
+    bool sf_8x4 = false;        // sfA and sfB in the 8 x 4 layout (dense NVFP4 GEMM only)
 };
 
 // api.cu: nvfp4_status of the current device's checks; fills the SM count and the device

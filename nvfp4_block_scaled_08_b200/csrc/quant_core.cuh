@@ -167,31 +167,37 @@ __device__ __forceinline__ int64_t vec_offset(const VecIndex& ix, uint32_t i)
 //     ((r / 128) * (K / 64) + c / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4,
 // i.e. 512-byte blocks of 128 rows x 4 scales, each holding, in its 16-byte row i, the scales
 // of rows i, i + 32, i + 64, i + 96: the source layout of tcgen05.cp ... 32x128b.warpx4.
+// Or the 8 x 4 layout (NVFP4_SF_8X4): 32-byte blocks of 8 rows x 4 scales, row-major inside
+// the block, the blocks of a row group consecutive along K:
+//     ((r / 8) * (K / 64) + c / 4) * 32 + (r % 8) * 4 + c % 4.
+enum : int32_t { kSfLinear = 0, kSfTiled = 1, kSf8x4 = 2 };
+
 struct SfOut {
     uint8_t* sf;
-    int32_t tiled;
-    uint32_t kb4;            // K / 64: 512-byte blocks per 128-row tile
+    int32_t layout;          // kSfLinear, kSfTiled or kSf8x4
+    uint32_t kb4;            // 4-scale column groups per row: K / 64 (NVFP4), K / 128 (MXFP4)
     uint32_t vpr, mul, shift;  // vector -> row, as in VecIndex
 
     // Scale of vector i's block. Offsets fit in 32 bits: there are fewer than 2^31 vectors,
-    // so fewer than 2^30 scales, and the tiled layout pads the rows to 128 at most.
+    // so fewer than 2^30 scales, and the non-linear layouts pad the rows to 128 at most.
     template <int TPB>
     __device__ __forceinline__ uint8_t* at(uint32_t i) const
     {
-        if (!tiled) return sf + i / TPB;
+        if (layout == kSfLinear) return sf + i / TPB;
         const uint32_t r = static_cast<uint32_t>((static_cast<uint64_t>(__umulhi(i, mul)) + i) >> shift);
         const uint32_t c = (i - r * vpr) / TPB;
+        if (layout == kSf8x4) return sf + (((r >> 3) * kb4 + (c >> 2)) * 32u + (r & 7u) * 4u + (c & 3u));
         return sf + (((r >> 7) * kb4 + (c >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (c & 3u));
     }
 };
 
-// block: elements per scale (16 for NVFP4, 32 for MXFP4); the tiled layout holds 4 scale
-// columns per 512-byte block, so a 128-row tile spans K / (4 block) blocks.
-inline SfOut make_sf_out(uint8_t* sf, bool tiled, const VecIndex& ix, int64_t K, int block = 16)
+// block: elements per scale (16 for NVFP4, 32 for MXFP4); the non-linear layouts hold 4 scale
+// columns per block, so a row group spans K / (4 block) blocks.
+inline SfOut make_sf_out(uint8_t* sf, int layout, const VecIndex& ix, int64_t K, int block = 16)
 {
     SfOut o;
     o.sf = sf;
-    o.tiled = tiled ? 1 : 0;
+    o.layout = layout;
     o.kb4 = static_cast<uint32_t>(K / (4 * block));
     o.vpr = ix.vpr;
     o.mul = ix.mul;

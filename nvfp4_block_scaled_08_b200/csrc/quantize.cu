@@ -321,7 +321,7 @@ cudaError_t launch_quantize(const void* x, bool bf16, int64_t rows, int64_t K, i
         const int grid = grid_1d(nv, static_cast<int64_t>(num_sms) * 4);
         const void* xp = static_cast<const uint8_t*>(x) + static_cast<size_t>(r0 * ldx) * esz;
         uint8_t* qp = q + r0 * (K / 2);
-        const SfOut sp = make_sf_out(sf + r0 * (K / 16), false, ix, K);
+        const SfOut sp = make_sf_out(sf + r0 * (K / 16), kSfLinear, ix, K);
         if (bf16)
             quantize_kernel<__nv_bfloat16><<<grid, 512, 0, stream>>>(
                 static_cast<const __nv_bfloat16*>(xp), ix, static_cast<uint32_t>(nv), gs, qp, sp);
@@ -497,7 +497,7 @@ static cudaError_t launch_dynamic_t(const T* x, int64_t rows, int64_t vpr, const
 }
 
 cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx,
-                                    float* gs_out, uint8_t* q, uint8_t* sf, bool sf_tiled,
+                                    float* gs_out, uint8_t* q, uint8_t* sf, int sf_layout,
                                     const float* gs_other, int32_t n_alpha, float* alpha_out,
                                     unsigned* err_word, cudaStream_t stream, int num_sms)
 {
@@ -505,7 +505,7 @@ cudaError_t launch_quantize_dynamic(const void* x, bool bf16, int64_t rows, int6
     const int64_t vpr = K / V;
     const int64_t q_bytes = rows * (K / 2);
     const VecIndex ix = make_vec_index(vpr, ldx, K);
-    const DenseDst dst{q, make_sf_out(sf, sf_tiled, ix, K)};
+    const DenseDst dst{q, make_sf_out(sf, sf_layout, ix, K)};
     if (bf16)
         return launch_dynamic_t(static_cast<const __nv_bfloat16*>(x), rows, vpr, ix, K, gs_out, q, dst,
                                 gs_other, n_alpha, alpha_out, q_bytes, err_word, stream, num_sms);
@@ -538,7 +538,7 @@ cudaError_t launch_mx_quantize(const void* x, bool bf16, int64_t rows, int64_t K
     if (rows == 0 || vpr == 0) return cudaSuccess;
     const VecIndex ix = make_vec_index(vpr, ldx, K);
     const int64_t nv = rows * vpr;         // < 2^31 (checked by the caller)
-    const SfOut sfo = make_sf_out(sf, sf_tiled, ix, K, 32);
+    const SfOut sfo = make_sf_out(sf, sf_tiled ? kSfTiled : kSfLinear, ix, K, 32);
     // one vector per thread per pass: enough warps to cover the tensor, at most 8 per SM
     int64_t grid = (nv + 511) / 512;
     if (grid > static_cast<int64_t>(num_sms) * 4) grid = static_cast<int64_t>(num_sms) * 4;
@@ -579,6 +579,32 @@ cudaError_t launch_round(const float* x, int64_t n, uint8_t* out, bool e2m1, cud
 }
 
 // ------------------------------------------------------------------ scale layout
+
+// Row-major scales [rows][kb] -> the 8 x 4 layout (quant_core.cuh, SfOut), one output byte per
+// thread; rows past `rows` in the last 8-row group are zero.
+__global__ void sf_8x4_kernel(const uint8_t* __restrict__ sf, int64_t rows, int64_t kb, int64_t kb4,
+                              uint8_t* __restrict__ out, int64_t out_bytes)
+{
+    for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < out_bytes;
+         o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t block = o >> 5, within = o & 31;
+        const int64_t rg = block / kb4, cg = block - rg * kb4;
+        const int64_t r = rg * 8 + (within >> 2);
+        const int64_t c = cg * 4 + (within & 3);
+        out[o] = r < rows ? sf[r * kb + c] : 0;
+    }
+}
+
+cudaError_t launch_sf_8x4(const uint8_t* sf, int64_t rows, int64_t K, uint8_t* out, cudaStream_t stream,
+                          int num_sms)
+{
+    const int64_t kb = K / 16;
+    const int64_t out_bytes = (rows + 7) / 8 * 8 * kb;
+    if (out_bytes == 0) return cudaSuccess;
+    const int grid = grid_for(out_bytes, num_sms);
+    sf_8x4_kernel<<<grid, 256, 0, stream>>>(sf, rows, kb, kb / 4, out, out_bytes);
+    return cudaGetLastError();
+}
 
 // Row-major scales [rows][K/16] -> the tiled layout (quant_core.cuh, SfOut), one output byte
 // per thread; rows past `rows` in the last 128-row tile are zero.

@@ -60,3 +60,17 @@ def tile_np(sf: np.ndarray, K: int) -> np.ndarray:
     off = ((r // 128) * (K // 64) + c // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + c % 4
     out[off] = sf
     return out
+
+
+def layout_8x4_np(sf: np.ndarray, K: int) -> np.ndarray:
+    """The 8 x 4 layout: row r, scale column c at ((r // 8) * (K // 64) + c // 4) * 32
+    + (r % 8) * 4 + c % 4; rows padded to 8 with zeros."""
+    rows, kb = sf.shape
+    assert kb == K // 16
+    R = (rows + 7) // 8 * 8
+    out = np.zeros(R * kb, dtype=np.uint8)
+    r = np.arange(rows)[:, None]
+    c = np.arange(kb)[None, :]
+    off = ((r // 8) * (K // 64) + c // 4) * 32 + (r % 8) * 4 + c % 4
+    out[off] = sf
+    return out

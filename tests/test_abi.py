@@ -196,6 +196,22 @@ def test_tiled_scale_host_validation(lib):
     q = lib.nvfp4_quantize_dynamic_ex
     assert q(0x1000, 0, 4, 64, 64, 0x2000, 0x3000, 0x4000, None, 0, None, 3, None) == 1
     assert q(0x1000, 0, 4, 48, 48, 0x2000, 0x3000, 0x4000, None, 0, None, 1, None) == 2
+    assert q(0x1000, 0, 4, 48, 48, 0x2000, 0x3000, 0x4000, None, 0, None, 2, None) == 2
+
+
+def test_8x4_scale_host_validation(lib):
+    assert lib.nvfp4_sf_bytes(300, 512, 2) == 304 * 32      # rows padded to 8
+    assert lib.nvfp4_sf_bytes(8, 512, 2) == 8 * 32
+    assert lib.nvfp4_sf_bytes(1, 64, 2) == 8 * 4
+    assert lib.nvfp4_sf_bytes(300, 48, 2) == 0             # K % 64 == 0
+    assert lib.nvfp4_sf_8x4(0x1000, 4, 48, 0x2000, None) == 2
+    assert lib.nvfp4_sf_8x4(None, 4, 64, 0x2000, None) == 1
+    assert lib.nvfp4_sf_8x4(0x1000, 4, 64, None, None) == 1
+    assert lib.nvfp4_sf_8x4(0x1000, 0, 64, 0x2000, None) == 0
+    assert lib.nvfp4_sf_8x4(0x1000, -1, 64, 0x2000, None) == 1
+    g = lib.nvfp4_gemm_ex
+    assert g(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 16, 768, 6000, None, 0, 2, None) == 2   # K % 256
+    assert g(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 16, 768, 6144, None, 0, 3, None) == 1
 
 
 def test_bounded_wait_check_host_validation(lib):
