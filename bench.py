@@ -110,7 +110,7 @@ def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> fl
     return flops_per_rank * world / (step_ms_max * 1e-3) / 1e12
 
 
-# DRAM traffic of one 16384^3 GEMM launch (tiled scales): dram__bytes_read.sum +
+# DRAM traffic of one 16384^3 GEMM launch (tiled scales, CTA pairs): dram__bytes_read.sum +
 # dram__bytes_write.sum from one ncu capture of the full-size launch (one pass); the command
 # and the figures are in the committed ncu summary of the plateau under profiles/. Valid only
 # for the kernel sources it was taken on (hash below); reported as null otherwise.
@@ -736,7 +736,7 @@ def run_ours(args, world, rank, local):
 
     peak_meas = peaks["bf16_tflops"] * FP4_PER_BF16
     achieved = hs.flops / (gemm_us * 1e-6) / 1e12
-    roof = {"kernel": "nvfp4_gemm_kernel<256, non-swap, tiled scales> (one 16384^3 launch)",
+    roof = {"kernel": "nvfp4_gemm_kernel<256, non-swap, tiled scales, CTA pair: 2-SM MMA> (one 16384^3 launch)",
             "bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_meas, 1),
             "unit": "TFLOP/s", "frac": round(achieved / peak_meas, 4), "traffic": gemm_traffic(),
             "per": f"{hs.flops:.4g} algorithmic flops per launch (2 M N K)",

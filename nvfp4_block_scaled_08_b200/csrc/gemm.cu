@@ -114,12 +114,13 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
         p.ws_counter_bytes = ((static_cast<size_t>(tiles) * cs * 4 + 255) / 256) * 256;
         p.ws_bytes = p.ws_counter_bytes + static_cast<size_t>(tiles) * g * 128 * p.bn * sizeof(float);
     }
-    // CTA pairs sharing 256-row Q tiles (tiled scales): 128 x 256 tiles without split-K and at
-    // least one pair of P tiles; the pair's work items are P tile pairs. Only on request: with
-    // a 4-deep stage ring the forward's extra hop leaves the MMA waiting (measured on B200:
-    // 8192^3 in 371 us with pairs against 209 us without).
-    const int fp = g_force_pair.load(std::memory_order_relaxed);     // 1: off, 2: on where possible
-    p.pair = !p.swap && p.bn == 256 && p.splits == 1 && p.p_tiles >= 2 && fp == 2;
+    // CTA pairs computing 256 x 256 tiles with the 2-SM MMA (tiled scales): 256-wide Q tiles
+    // without split-K and at least one pair of P tiles; the pair's work items are P tile
+    // pairs. Each SM then stages 38 KB per K step instead of 54 KB for the same MMA work
+    // (measured on B200: 16384^3 in 1543-1644 us against 1790-1867 us, 8192^3 in 192-203 us
+    // against 216-222 us, 4096^3 in 30.1 us against 32-33 us).
+    const int fp = g_force_pair.load(std::memory_order_relaxed);     // 1: off, 0 / 2: where possible
+    p.pair = !p.swap && p.bn == 256 && p.splits == 1 && p.p_tiles >= 2 && fp != 1;
     if (p.pair) {
         const int pairs = ((p.p_tiles + 1) / 2) * p.q_tiles;
         const int clusters = std::max(1, std::min(pairs, max_active_clusters(2)));
@@ -360,7 +361,17 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         ok &= get_map(&tp, P, 2, kb, p_rows, 1, kb, 0, 128, 128, true);
         if constexpr (ACTQ) tq = tp;          // unused: the kernel quantises the activations itself
         else ok &= get_map(&tq, Q, 2, kb, q_rows, 1, kb, 0, 128, PAIR ? BN / 2 : BN, true);   // PAIR: half tiles
-        if constexpr (SFT) {
+        if constexpr (PAIR) {
+            // the tiled scales as rows of 256 bytes: a stage's run of one 128-row tile is
+            // SFP_BYTES / 256 rows (past the last tile: zero fill)
+            const uint64_t sp_rows = (p_rows + 127) / 128 * (L.K / (MX ? 64 : 32));
+            const uint64_t sq_rows = (q_rows + 127) / 128 * (L.K / (MX ? 64 : 32));
+            ok &= get_map(&tsp, sP, 2, 256, sp_rows, 1, 256, 0, 256, Cfg::SF_ROWS256, false);
+            ok &= get_map(&tsq, sQ, 2, 256, sq_rows, 1, 256, 0, 256, Cfg::SF_ROWS256, false);
+            a.sf_p = sP;
+            a.sf_q = sQ;
+            a.sf_kb4 = static_cast<int32_t>(L.K / (MX ? 128 : 64));
+        } else if constexpr (SFT) {
             tsp = tp;                       // unused: the scales come by bulk copy
             tsq = tq;
             a.sf_p = sP;

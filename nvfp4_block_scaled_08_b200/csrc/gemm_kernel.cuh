@@ -54,8 +54,6 @@ enum : uint32_t {
     kErrEpiAccFull = 0x106,
     kErrSplitRx = 0x107,
     kErrMmaSfFree = 0x108,
-    kErrMmaHalf = 0x109,
-    kErrForward = 0x10A,
     kErrActqMax = 0x10B,
     kErrMmaActq = 0x10C,
 };
@@ -127,15 +125,15 @@ struct GemmCfg {
     static constexpr bool SFT = SFT_;
     static_assert(!SFT || !GROUPED, "tiled scales serve the dense GEMM");
     static_assert(!MX || (SFT && !GROUPED), "MXFP4 serves the dense GEMM with tiled scales");
-    // PAIR: the two CTAs of a 2-CTA cluster take adjacent 128-row P tiles of the same 256-row Q
-    // tile. Each loads its own P tile and only its half of the Q tile (rows 128 rank ..) and
-    // forwards that half to the peer's stage buffer with a shared-to-shared bulk copy over
-    // distributed shared memory, so each SM pulls 2/3 of the bytes a lone 128 x 256 tile needs
-    // from L2. The MMA itself is the single-CTA 128 x 256 MMA on the whole Q tile; a stage is
-    // released when both CTAs' MMAs are done with it (the commit arrives on both).
+    // PAIR: the two CTAs of a 2-CTA cluster compute one 256 x 256 tile with the 2-SM MMA
+    // (cta_group::2, M = 256): CTA r loads P rows [p0 + 128 r, + 128), Q rows [q0 + 128 r, + 128)
+    // and the scales of its P rows and of all 256 Q rows; the even CTA issues the MMAs, which
+    // read both CTAs' stages, and each CTA's TMEM receives its own 128 rows of the tile. Per
+    // SM a stage is 38 KB instead of 54 KB for the same MMA work, so the ring is 5 deep and
+    // L2 serves a third fewer bytes. Every copy's completion is counted on the even CTA's
+    // full barrier; its commits release both CTAs' stages and accumulators.
     static constexpr bool PAIR = PAIR_;
-    static_assert(!PAIR || (SFT && !SWAP && !GROUPED && BN == 256), "CTA pairs share 256-row Q tiles");
-    static constexpr int QH_BYTES = 128 * 128;     // PAIR: one half of the Q tile per stage
+    static_assert(!PAIR || (SFT && !SWAP && !GROUPED && BN == 256), "CTA pairs compute 256-row Q tiles");
     // ACTQ (few-token launches with tiled weight scales): the activations come in as fp32 or
     // bf16 and are quantised inside the kernel. Every CTA of a split-K cluster reads its own K
     // slice of them, the slices' maxima meet over distributed shared memory (the cluster's
@@ -155,13 +153,15 @@ struct GemmCfg {
     static constexpr int BM = 128;                 // MMA M
     static constexpr int BK_BYTES = 128;           // 256 fp4 values per K stage
     static constexpr int P_BYTES = BM * BK_BYTES;  // 16 KB
-    static constexpr int Q_BYTES = BN * BK_BYTES;
+    static constexpr int Q_BYTES = (PAIR ? BN / 2 : BN) * BK_BYTES;   // this CTA's rows of the Q tile
     static constexpr int QG = (BN + 127) / 128;    // 128-row scale groups of the Q tile
     static constexpr int SFP_BYTES = 512 * SF_BLOCKS;   // 128 rows x 16 B (NVFP4) or 8 B (MX)
     static constexpr int SFQ_BYTES = SFP_BYTES * QG;
     static constexpr int SF_TMA_P = BM * 16;       // bytes the scale TMA writes
     static constexpr int SF_TMA_Q = BN * 16;
     static constexpr uint32_t TX_BYTES = P_BYTES + Q_BYTES + SF_TMA_P + SF_TMA_Q;
+    static constexpr uint32_t PAIR_TX_BYTES = 2u * (P_BYTES + Q_BYTES + SFP_BYTES + SFP_BYTES * QG);  // both CTAs'
+    static constexpr int SF_ROWS256 = SFP_BYTES / 256;   // PAIR: a stage's scale run as rows of 256 bytes
     // Grouped: the token tile is loaded in boxes of QBOX rows, only as many as the expert's
     // rows in the tile need (a tile of a 256-wide plan often holds ~128 rows of one expert).
     // (176-row tiles: two boxes of 88, which end exactly at the tile)
@@ -860,7 +860,6 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     uint64_t* mma_done_bar = bars + 3 * STAGES + 4;
     uint64_t* rx_bar = bars + 3 * STAGES + 5;       // split-K: partial rows received from peers
     uint64_t* sf_free_bar = bars + 3 * STAGES + 6;  // SF_IN_ACC: scale columns drained
-    uint64_t* half_bar = bars + 3 * STAGES + 8;     // PAIR: this CTA's Q half landed
     uint64_t* actq_bar = bars + 4 * STAGES + 8;     // ACTQ: the Q stages hold the activations
     uint64_t* amax_bar = bars + 4 * STAGES + 9;     // ACTQ: the peers' slice maxima arrived
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
@@ -877,13 +876,13 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&sfready_bar[s], 1);
-            mbar_init(&empty_bar[s], Cfg::PAIR ? 2 : 1);   // PAIR: both CTAs' MMAs
-            mbar_init(&half_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full_bar[s], 1);
-            mbar_init(&acc_empty_bar[s], kEpilogueWarps);
-            mbar_init(&sf_free_bar[s], 4);            // the second epilogue warpgroup
+            // PAIR: the even CTA's barriers count both CTAs' epilogue warps
+            mbar_init(&acc_empty_bar[s], Cfg::PAIR ? 2 * kEpilogueWarps : kEpilogueWarps);
+            mbar_init(&sf_free_bar[s], Cfg::PAIR ? 8 : 4);   // the second epilogue warpgroup(s)
         }
         mbar_init(mma_done_bar, 1);
         mbar_init(rx_bar, 1);
@@ -896,14 +895,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tm_p);
         prefetch_tensormap(&tm_q);
-        if constexpr (!Cfg::SFT) {
+        if constexpr (!Cfg::SFT || Cfg::PAIR) {
             prefetch_tensormap(&tm_sfp);
             prefetch_tensormap(&tm_sfq);
         }
     }
     if (warp == 1) {
-        tmem_alloc(s_tmem_base, Cfg::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (Cfg::PAIR) {
+            tmem_alloc_pair(s_tmem_base, Cfg::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(s_tmem_base, Cfg::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     // Everything above touches only this CTA's resources and the kernel parameters. Reads of
     // data the previous kernel in the stream may write come after grid_dependency_wait():
@@ -946,9 +950,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // PAIR: the peer forwards into this CTA's stages and arrives on its barriers; split-K with
-    // a receive region of its own: peers send into it as soon as their rows are done. Either
-    // way both CTAs' barriers are initialised before either touches the other's.
+    // PAIR: the odd CTA's copies and epilogue arrive on the even CTA's barriers and the even
+    // CTA's commits on the odd CTA's; split-K with a receive region of its own: peers send into
+    // it as soon as their rows are done. Either way both CTAs' barriers are initialised before
+    // either touches the other's.
     if constexpr (Cfg::PAIR) cluster_sync();
     if constexpr (Cfg::RX_OWN) {
         if (args.splits > 1 && args.cluster_size > 1) cluster_sync();
@@ -980,6 +985,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                 for (int ks = 0; ks < n; ++ks) {
                     const int32_t kx = (ti.k0 + ks) * Cfg::BK_BYTES;
                     if constexpr (Cfg::SWAP) tma_prefetch_2d(&tm_p, kx, ti.p0);
+                    else if constexpr (Cfg::PAIR) tma_prefetch_2d(&tm_q, kx, ti.q0 + 128 * static_cast<int32_t>(cluster_ctarank()));
                     else tma_prefetch_2d(&tm_q, kx, ti.q0);
                 }
             }
@@ -1024,29 +1030,23 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                                         pol_q);
                         }
                     } else if constexpr (Cfg::PAIR) {
-                        // own P tile and scales on full[stage], together with the peer's half of
-                        // the Q tile (forwarded); own half of the Q tile and its scales on
-                        // half[stage] (the forwarder sends them on once they have landed). A half
-                        // past the Q rows is neither loaded nor forwarded, by either CTA.
-                        const int rank = static_cast<int>(cluster_ctarank());
-                        const bool peer_half = ti.q0 + 128 * (rank ^ 1) < args.q_rows;
-                        const bool own_half = ti.q0 + 128 * rank < args.q_rows;
-                        const int64_t kb = Cfg::SF_BLOCKS * static_cast<int64_t>(ti.k0 + ks);
-                        mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::SFP_BYTES +
-                                                  (peer_half ? Cfg::QH_BYTES + Cfg::SFP_BYTES : 0u));
-                        tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
-                        bulk_load(sfpb, args.sf_p + ((ti.p0 >> 7) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
-                                  Cfg::SFP_BYTES, fb, pol_p);
-                        uint64_t* hb = &half_bar[stage];
-                        if (own_half) {
-                            mbar_arrive_expect_tx(hb, Cfg::QH_BYTES + Cfg::SFP_BYTES);
-                            tma_load_2d(qbuf + rank * Cfg::QH_BYTES, &tm_q, hb, kx, ti.q0 + 128 * rank, pol_q);
-                            bulk_load(sfqb + rank * Cfg::SFP_BYTES,
-                                      args.sf_q + (((ti.q0 >> 7) + rank) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
-                                      Cfg::SFP_BYTES, hb, pol_q);
-                        } else {
-                            mbar_arrive(hb);
-                        }
+                        // this CTA's P rows and Q rows, the scales of its P rows and of the whole
+                        // Q tile; all counted on the even CTA's full barrier, which the even CTA
+                        // arms for both CTAs' bytes (rows past the operands read as zero). The
+                        // scale runs are read through 2-D views of the tiled layout (rows of
+                        // 256 bytes), so that they can complete on the even CTA's barrier too.
+                        const uint32_t rank = cluster_ctarank();
+                        const uint32_t fb0 = mapa_shared(smem_u32(fb), 0);
+                        if (rank == 0) mbar_arrive_expect_tx(fb, Cfg::PAIR_TX_BYTES);
+                        const int32_t kb = Cfg::SF_BLOCKS * (ti.k0 + ks);
+                        const int32_t kb4 = args.sf_kb4;
+                        tma_load_2d_pair(pbuf, &tm_p, fb0, kx, ti.p0, pol_p);
+                        tma_load_2d_pair(qbuf, &tm_q, fb0, kx, ti.q0 + 128 * static_cast<int32_t>(rank), pol_q);
+                        tma_load_2d_pair(sfpb, &tm_sfp, fb0, 0, ((ti.p0 >> 7) * kb4 + kb) * 2, pol_p);
+#pragma unroll
+                        for (int g = 0; g < QG; ++g)
+                            tma_load_2d_pair(sfqb + Cfg::SFP_BYTES * g, &tm_sfq, fb0, 0,
+                                             (((ti.q0 >> 7) + g) * kb4 + kb) * 2, pol_q);
                     } else if constexpr (Cfg::ACTQ) {
                         // weights and their scales only: the epilogue warps fill the Q stages
                         mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::SFP_BYTES);
@@ -1088,19 +1088,23 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
         }
-        // Let every copy still in flight land before shared memory can be released.
+        // Let every copy still in flight land before shared memory can be released (the odd
+        // CTA of a pair cannot wait on the even CTA's full barrier: it waits until the MMAs
+        // that read each stage have released it).
+        const bool on_empty = Cfg::PAIR && cluster_ctarank() != 0;
         const uint32_t inflight = issued < (uint32_t)STAGES ? issued : (uint32_t)STAGES;
         for (uint32_t i = 1; i <= inflight; ++i) {
             const int s = ((int)stage - (int)i + 2 * STAGES) % STAGES;
             const uint32_t ph = ((int)stage - (int)i < 0) ? (phase ^ 1u) : phase;
-            mbar_wait_drain(&full_bar[s], ph);
+            mbar_wait_drain(on_empty ? &empty_bar[s] : &full_bar[s], ph);
         }
     } else if (warp == 1) {
         // -------------------------------------------------------------- MMA issuer
-        // Whole warp in the loop, one elected lane issues tcgen05.cp / tcgen05.mma.
+        // Whole warp in the loop, one elected lane issues tcgen05.cp / tcgen05.mma (PAIR: the
+        // even CTA's warp for both CTAs; the odd CTA's only allocates and frees TMEM).
         uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
         uint32_t sf_phases = 0;                    // bit b: parity of the next sf_free[b] wait
-        bool ok = true;
+        bool ok = !(Cfg::PAIR && cluster_ctarank() != 0);
         if constexpr (Cfg::ACTQ) ok = __all_sync(0xffffffffu, mbar_wait(actq_bar, 0, ab, kErrMmaActq));
         for (int32_t t = tile_start; t < num_tiles && ok; t += tile_step) {
             const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
@@ -1120,12 +1124,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             const uint32_t sf_b = sf_a + 4 * Cfg::SF_BLOCKS;    // after the SFA columns
             uint32_t n_mma = BN;
             if constexpr (Cfg::GROUPED) n_mma = min(BN, (ti.q_valid + 15) & ~15);
-            const uint32_t idesc = Cfg::MX ? idesc_mxf4_ue8m0(128, n_mma) : idesc_mxf4nvf4(128, n_mma);
+            constexpr uint32_t kMmaM = Cfg::PAIR ? 256 : 128;
+            const uint32_t idesc = Cfg::MX ? idesc_mxf4_ue8m0(kMmaM, n_mma) : idesc_mxf4nvf4(kMmaM, n_mma);
             const uint32_t d_tmem = tmem_base + acc * BN;
             for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
                 bool got = mbar_wait(&full_bar[stage], phase, ab, kErrMmaFull);
                 if constexpr (!Cfg::SFT) got = got && mbar_wait(&sfready_bar[stage], phase, ab, kErrMmaSf);
-                if constexpr (Cfg::PAIR) got = got && mbar_wait(&half_bar[stage], phase, ab, kErrMmaHalf);
                 ok = __all_sync(0xffffffffu, got);
                 if (!ok) break;
                 // ACTQ: the activations' K stage ks stays in Q stage ks for the whole launch
@@ -1135,11 +1139,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     const uint32_t sfq = smem_u32(smem + Cfg::OFF_SFQ + qslot * Cfg::SFQ_BYTES);
 #pragma unroll
                     for (int j = 0; j < Cfg::SF_BLOCKS; ++j) {
-                        tmem_cp_32x128b_warpx4(sf_a + 4 * j, sdesc_sf_32x16(sfp + 512 * j));
+                        if constexpr (Cfg::PAIR) {
+                            tmem_cp_32x128b_warpx4_pair(sf_a + 4 * j, sdesc_sf_32x16(sfp + 512 * j));
 #pragma unroll
-                        for (int g = 0; g < QG; ++g)
-                            tmem_cp_32x128b_warpx4(sf_b + 4 * QG * j + 4 * g,
-                                                   sdesc_sf_32x16(sfq + Cfg::SFP_BYTES * g + 512 * j));
+                            for (int g = 0; g < QG; ++g)
+                                tmem_cp_32x128b_warpx4_pair(sf_b + 4 * QG * j + 4 * g,
+                                                            sdesc_sf_32x16(sfq + Cfg::SFP_BYTES * g + 512 * j));
+                        } else {
+                            tmem_cp_32x128b_warpx4(sf_a + 4 * j, sdesc_sf_32x16(sfp + 512 * j));
+#pragma unroll
+                            for (int g = 0; g < QG; ++g)
+                                tmem_cp_32x128b_warpx4(sf_b + 4 * QG * j + 4 * g,
+                                                       sdesc_sf_32x16(sfq + Cfg::SFP_BYTES * g + 512 * j));
+                        }
                     }
                     const uint64_t pdesc =
                         sdesc_kmajor_sw128(smem_u32(smem + Cfg::OFF_P + stage * Cfg::P_BYTES));
@@ -1148,67 +1160,49 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         // advance 32 bytes (64 fp4 values) along K inside the swizzled rows
+                        const uint32_t accum = (ks > 0 || j > 0) ? 1u : 0u;
                         if constexpr (Cfg::MX) {
                             // block j / 2; its scale column holds 4 E8M0 bytes per row (K 128):
                             // bytes 0-1 for the first 64, 2-3 for the second
-                            mma_mxf4_block32(d_tmem, pdesc + 2u * j, qdesc + 2u * j,
-                                             idesc_sf_id(idesc, 2u * (j & 1)), sf_a + 4 * (j >> 1),
-                                             sf_b + 4 * QG * (j >> 1), (ks > 0 || j > 0) ? 1u : 0u);
+                            const uint32_t id = idesc_sf_id(idesc, 2u * (j & 1));
+                            if constexpr (Cfg::PAIR)
+                                mma_mxf4_block32_pair(d_tmem, pdesc + 2u * j, qdesc + 2u * j, id, sf_a + 4 * (j >> 1),
+                                                      sf_b + 4 * QG * (j >> 1), accum);
+                            else
+                                mma_mxf4_block32(d_tmem, pdesc + 2u * j, qdesc + 2u * j, id, sf_a + 4 * (j >> 1),
+                                                 sf_b + 4 * QG * (j >> 1), accum);
                         } else {
-                            mma_mxf4nvf4(d_tmem, pdesc + 2u * j, qdesc + 2u * j, idesc, sf_a + 4 * j,
-                                         sf_b + 4 * QG * j, (ks > 0 || j > 0) ? 1u : 0u);
+                            if constexpr (Cfg::PAIR)
+                                mma_mxf4nvf4_pair(d_tmem, pdesc + 2u * j, qdesc + 2u * j, idesc, sf_a + 4 * j,
+                                                  sf_b + 4 * QG * j, accum);
+                            else
+                                mma_mxf4nvf4(d_tmem, pdesc + 2u * j, qdesc + 2u * j, idesc, sf_a + 4 * j,
+                                             sf_b + 4 * QG * j, accum);
                         }
                     }
-                    if constexpr (Cfg::PAIR) mma_commit_pair(&empty_bar[stage]);   // both CTAs' stage
+                    if constexpr (Cfg::PAIR) mma_commit_both(&empty_bar[stage]);   // both CTAs' stage
                     else mma_commit(&empty_bar[stage]);
                 }
                 __syncwarp();
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
-            if (elect_one()) mma_commit(&acc_full_bar[acc]);
+            if (elect_one()) {
+                if constexpr (Cfg::PAIR) mma_commit_both(&acc_full_bar[acc]);
+                else mma_commit(&acc_full_bar[acc]);
+            }
             __syncwarp();
             if (++acc == Cfg::ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
         }
-        // Arrives once every tcgen05 operation issued above has completed.
-        if (elect_one()) mma_commit(mma_done_bar);
-        __syncwarp();
-    } else if (Cfg::PAIR && warp == 2) {
-        // -------------------------------------------------------------- Q-half forwarder
-        // Sends this CTA's half of every stage's Q tile and its scales into the same place of
-        // the peer's stage, completion counted on the peer's full barrier. The stage is free in
-        // the peer too: the producer loaded this half only after both CTAs' MMAs released the
-        // stage (the empty barrier counts both commits).
-        const int rank = static_cast<int>(cluster_ctarank());
-        const uint32_t peer = static_cast<uint32_t>(rank ^ 1);
-        uint32_t stage = 0, phase = 0;
-        bool ok = true;
-        for (int32_t t = tile_start; t < num_tiles && ok; t += tile_step) {
-            const Tile ti = decode_tile<Cfg>(args, t, s_prefix);
-            const bool own_half = ti.q0 + 128 * rank < args.q_rows;
-            if (!own_half) {
-                // nothing to send (and nothing to wait for: without a forward from here the
-                // producer may run rounds ahead on these stages)
-                for (int32_t ks = 0; ks < ti.kcnt; ++ks)
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                continue;
-            }
-            for (int32_t ks = 0; ks < ti.kcnt; ++ks) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&half_bar[stage], phase, ab, kErrForward));
-                if (!ok) break;
-                if (elect_one()) {
-                    uint8_t* qh = smem + Cfg::OFF_Q + stage * Cfg::Q_BYTES + rank * Cfg::QH_BYTES;
-                    uint8_t* sh = smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES + rank * Cfg::SFP_BYTES;
-                    const uint32_t rbar = mapa_shared(smem_u32(&full_bar[stage]), peer);
-                    bulk_copy_s2peer(mapa_shared(smem_u32(qh), peer), smem_u32(qh), Cfg::QH_BYTES, rbar);
-                    bulk_copy_s2peer(mapa_shared(smem_u32(sh), peer), smem_u32(sh), Cfg::SFP_BYTES, rbar);
-                    bulk_commit_group();
-                }
-                __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        // Arrives once every tcgen05 operation issued above has completed (PAIR: in both CTAs,
+        // from the even CTA's warp).
+        if (elect_one()) {
+            if constexpr (Cfg::PAIR) {
+                if (cluster_ctarank() == 0) mma_commit_both(mma_done_bar);
+            } else {
+                mma_commit(mma_done_bar);
             }
         }
-        if (elect_one()) bulk_wait_group_read0();        // sources read before teardown
         __syncwarp();
     } else if (!Cfg::SFT && (warp == 2 || warp == 3)) {
         // -------------------------------------------------------------- scale re-layout
@@ -1343,7 +1337,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     }
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sf_free_bar[acc]);
+                    if (lane == 0) {
+                        if constexpr (Cfg::PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_free_bar[acc]), 0));
+                        else mbar_arrive(&sf_free_bar[acc]);
+                    }
                     if (need) {
                         if constexpr (!Cfg::SWAP && !Cfg::GROUPED) {
                             store_rows64<Cfg>(args, ti, quad, lane, BN - 64, r, alpha);
@@ -1399,10 +1396,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     }
                 }
             }
-            // Accumulator drained into registers / workspace: hand it back to the MMA warp.
+            // Accumulator drained into registers / workspace: hand it back to the MMA warp (PAIR:
+            // the even CTA's, which writes both CTAs' accumulators).
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty_bar[acc]);
+            if (lane == 0) {
+                if constexpr (Cfg::PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty_bar[acc]), 0));
+                else mbar_arrive(&acc_empty_bar[acc]);
+            }
             if (++acc == Cfg::ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
 
         }
@@ -1429,14 +1430,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         __syncwarp();
     }
     if constexpr (Cfg::PAIR) {
-        // neither CTA leaves while the peer's forwards or MMA commits may still reach it: every
-        // thread of both arrives once, after its own roles (and this MMA warp's commits) are done
+        // neither CTA frees its TMEM or leaves while the other's copies, arrivals or the even
+        // CTA's MMAs may still reach it: every thread of both arrives once, after its own roles
+        // are done and both MMA warps have seen the last commit
         __syncthreads();
         cluster_sync();
     }
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+        if constexpr (Cfg::PAIR) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+        else tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
 }
 

@@ -86,50 +86,89 @@ __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__
 // ------------------------------------------------------------------ expert-sorted permutation
 
 // Block e (1024 threads): the (token, slot) pairs routed to expert e, in ascending token
-// order. Each thread takes a contiguous range of at most ceil(T / 1024) tokens; a block scan
-// of the per-thread hit counts gives each hit its rank among expert e's pairs, written to
-// rank_out[t k + s] (each pair has exactly one expert, so exactly one block writes it). The
-// expert's count goes to count_out[e]. A token's k slots are read as one unrolled run of
-// independent loads (the second pass finds them in L1).
+// order; pair p = t k + s, and ascending p is ascending token order (a token's k experts are
+// distinct). The pairs are read in rounds of 16 per thread: load j of thread i is the 16-byte
+// vector 4 (i + 1024 j) .. + 3 (four 4-byte loads if `experts` is not 16-byte aligned), so every
+// load instruction is coalesced. The four loads' hit
+// counts (each 0..4) travel packed in 16-bit fields of one 64-bit value through one block
+// scan, which gives every hit its rank among expert e's pairs (all of load j's pairs precede
+// load j + 1's); the rank is written to rank_out[p] (each pair has one expert, so exactly one
+// block writes it). The expert's count goes to count_out[e].
 constexpr int kRankThreads = 1024;
+constexpr int kRankLoads = 4;                          // 16-byte loads per thread and round
 
-__global__ void __launch_bounds__(kRankThreads) moe_rank_kernel(const int32_t* __restrict__ experts, int32_t T,
-                                                                int32_t k, int32_t* __restrict__ rank_out,
-                                                                int32_t* __restrict__ count_out)
+__device__ __forceinline__ unsigned long long warp_incl_scan_u64(unsigned long long v, int lane)
 {
-    __shared__ int32_t warp_tot[kRankThreads / 32];
-    const int e = blockIdx.x;
-    const int tid = threadIdx.x;
-    const int chunk = (T + kRankThreads - 1) / kRankThreads;
-    const int t0 = min(T, tid * chunk), t1 = min(T, t0 + chunk);
-    int c = 0;
-    for (int t = t0; t < t1; ++t) {
-        const int32_t* row = experts + static_cast<int64_t>(t) * k;
-#pragma unroll 8
-        for (int s = 0; s < k; ++s) c += (__ldg(row + s) == e);
-    }
-    // exclusive scan over the block (thread order = token order)
-    const int lane = tid & 31, warp = tid >> 5;
-    int incl = c;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += y;
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, v, d);
+        if (lane >= d) v += y;
     }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += warp_tot[w];
-    int r = base + incl - c;
-    if (c > 0) {
-        for (int t = t0; t < t1; ++t) {
-            const int32_t* row = experts + static_cast<int64_t>(t) * k;
-#pragma unroll 8
-            for (int s = 0; s < k; ++s)
-                if (__ldg(row + s) == e) rank_out[static_cast<int64_t>(t) * k + s] = r++;
+    return v;
+}
+
+__global__ void __launch_bounds__(kRankThreads) moe_rank_kernel(const int32_t* __restrict__ experts, int64_t pairs,
+                                                                int32_t* __restrict__ rank_out,
+                                                                int32_t* __restrict__ count_out)
+{
+    __shared__ unsigned long long warp_tot[kRankThreads / 32];
+    __shared__ unsigned long long s_total;
+    const int e = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int64_t kVec = 4;
+    constexpr int64_t kRound = kVec * kRankThreads * kRankLoads;
+    const bool vec_ok = (reinterpret_cast<uintptr_t>(experts) & 15u) == 0;   // else 4-byte loads
+    int32_t run = 0;                                   // expert e's pairs before this round
+    for (int64_t p0 = 0; p0 < pairs; p0 += kRound) {
+        int4 v[kRankLoads];
+        uint32_t hits[kRankLoads];
+        unsigned long long packed = 0;
+#pragma unroll
+        for (int j = 0; j < kRankLoads; ++j) {
+            const int64_t p = p0 + kVec * (tid + static_cast<int64_t>(kRankThreads) * j);
+            if (vec_ok && p + kVec <= pairs) {
+                v[j] = __ldg(reinterpret_cast<const int4*>(experts + p));
+            } else {
+                v[j].x = p < pairs ? __ldg(experts + p) : -1;
+                v[j].y = p + 1 < pairs ? __ldg(experts + p + 1) : -1;
+                v[j].z = p + 2 < pairs ? __ldg(experts + p + 2) : -1;
+                v[j].w = p + 3 < pairs ? __ldg(experts + p + 3) : -1;
+            }
+            hits[j] = (v[j].x == e ? 1u : 0u) | (v[j].y == e ? 2u : 0u) | (v[j].z == e ? 4u : 0u) |
+                      (v[j].w == e ? 8u : 0u);
+            packed |= static_cast<unsigned long long>(__popc(hits[j])) << (16 * j);
         }
+        // exclusive scan of the packed counts over the block (thread order within each load j;
+        // a field never exceeds 4 * 1024, so the fields do not carry into one another)
+        const unsigned long long incl = warp_incl_scan_u64(packed, lane);
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const unsigned long long t = warp_tot[lane];
+            const unsigned long long ti = warp_incl_scan_u64(t, lane);
+            warp_tot[lane] = ti - t;                   // the warps before this one
+            if (lane == 31) s_total = ti;              // the round's count per load
+        }
+        __syncthreads();
+        const unsigned long long excl = warp_tot[warp] + incl - packed;
+        const unsigned long long total = s_total;
+        int32_t base = run;
+#pragma unroll
+        for (int j = 0; j < kRankLoads; ++j) {
+            int32_t r = base + static_cast<int32_t>((excl >> (16 * j)) & 0xFFFFu);
+            if (hits[j]) {
+                const int64_t p = p0 + kVec * (tid + static_cast<int64_t>(kRankThreads) * j);
+                if (hits[j] & 1u) rank_out[p] = r++;
+                if (hits[j] & 2u) rank_out[p + 1] = r++;
+                if (hits[j] & 4u) rank_out[p + 2] = r++;
+                if (hits[j] & 8u) rank_out[p + 3] = r++;
+            }
+            base += static_cast<int32_t>((total >> (16 * j)) & 0xFFFFu);
+        }
+        run = base;
+        __syncthreads();                               // warp_tot and s_total are reused
     }
-    if (tid == kRankThreads - 1) count_out[e] = base + incl;
+    if (tid == 0) count_out[e] = run;
 }
 
 // One block: offsets[0] = 0, offsets[e + 1] = offsets[e] + count[e], in place (the counts are
@@ -182,7 +221,7 @@ cudaError_t launch_moe_route(const float* logits, int32_t T, int32_t E, int32_t 
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    moe_rank_kernel<<<E, kRankThreads, 0, stream>>>(experts, T, k, row_of, offsets + 1);
+    moe_rank_kernel<<<E, kRankThreads, 0, stream>>>(experts, static_cast<int64_t>(T) * k, row_of, offsets + 1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     moe_scan_kernel<<<1, 1024, 0, stream>>>(E, offsets);

@@ -308,20 +308,100 @@ __device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t 
                  : "memory");
 }
 
-// Arrive on the mbarrier at `bar`'s offset in both CTAs of a 2-CTA cluster (CTA mask 0b11)
-// once every tcgen05 operation this thread issued so far has completed.
-__device__ __forceinline__ void mma_commit_pair(uint64_t* bar)
-{
-    const uint16_t mask = 0x3;
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-                 ::"r"(smem_u32(bar)), "h"(mask) : "memory");
-}
-
 // Arrive on `bar` once every tcgen05 operation this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(smem_u32(bar)) : "memory");
+}
+
+// ---------------------------------------------------------------------------- CTA pairs
+// The 2-SM forms (cta_group::2) for the two CTAs of a 2-CTA cluster that compute one tile
+// together: one 256-row MMA whose A operand is split across the pair (rows 0-127 in the
+// even CTA's shared memory, 128-255 in the odd CTA's, at the same offset) and whose B
+// operand is split the same way along N; each CTA's TMEM holds its own 128 rows of D and
+// its own copy of the scales the MMA reads. A kernel that uses these uses cta_group::2 for
+// every tcgen05 allocation, copy, MMA and commit. Allocation and deallocation are issued by
+// the same warp in both CTAs (with the same shared-memory result slot); copies, MMAs and
+// commits by one thread of the even CTA only.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_result, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(smem_result)), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                 ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// tmem_cp_32x128b_warpx4 in both CTAs: each CTA's block at `sdesc` into its own TMEM.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+// One 256 x N x 64 block-scaled FP4 MMA over the pair (idesc with M = 256).
+__device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                  uint32_t idesc, uint32_t sfa_tmem,
+                                                  uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+          "r"(sfb_tmem)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf4_block32_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                      uint32_t idesc, uint32_t sfa_tmem,
+                                                      uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+          "r"(sfb_tmem)
+        : "memory");
+}
+
+// Arrive on the mbarrier at `bar`'s offset in both CTAs of the pair (CTA mask 0b11) once every
+// cta_group::2 tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit_both(uint64_t* bar)
+{
+    const uint16_t mask = 0x3;
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 ::"r"(smem_u32(bar)), "h"(mask) : "memory");
+}
+
+// 2-D tile load into this CTA's shared memory whose completion (bytes) is counted on the
+// mbarrier at `bar_cluster` (a shared::cluster address from mapa: this CTA's or the pair
+// peer's). A plain load (no multicast): the source is this GPU's global memory.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t x, int32_t y, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster),
+          "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+// Arrive (release, cluster scope) on the mbarrier at `bar_cluster` (from mapa).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 // ---------------------------------------------------------------------------- TMEM loads
@@ -371,28 +451,6 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
         ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
-}
-
-// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this CTA's
-// shared memory to a cluster peer's (dst and the peer's mbarrier from mapa); completion is
-// counted in bytes on that mbarrier. Not a multicast: one destination CTA.
-__device__ __forceinline__ void bulk_copy_s2peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
-                                                 uint32_t bar_cluster)
-{
-    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst_cluster), "r"(src_cta), "r"(bytes), "r"(bar_cluster)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit_group()
-{
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until the sources of every committed bulk group of this thread have been read.
-__device__ __forceinline__ void bulk_wait_group_read0()
-{
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // Asynchronous 16-byte store into another cluster CTA's shared memory; its completion is

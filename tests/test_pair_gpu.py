@@ -1,13 +1,13 @@
-"""GPU checks of the CTA-pair launch of the dense GEMM: the two CTAs of a 2-CTA cluster take
-adjacent 128-row tiles that share one 256-row weight tile, each loads half of that tile and
-forwards it to the other over distributed shared memory.
+"""GPU checks of the CTA-pair launch of the dense GEMM: the two CTAs of a 2-CTA cluster compute
+one 256 x 256 tile with the 2-SM MMA (tcgen05.mma.cta_group::2): each loads its own 128 rows of
+the token tile and of the weight tile, and the even CTA's MMAs read both CTAs' shared memory.
 
-Every output tile is computed by the same MMAs in the same order with or without pairs, so
-the two launches must agree bit for bit; both must be within the GEMM tolerance of the CPU
-oracle (2^-7 |alpha| sum|a b| + 1e-6). Shapes cover an odd number of row tiles (the last
-pair's second CTA has no rows), weight rows that end inside a tile's second half (that half
-is neither loaded nor forwarded), NVFP4 and MXFP4, and the plateau shapes. (The planner does
-not use pairs; they are reached through the plan override.)"""
+Every output element is the same sequence of 64-wide block-scaled products with or without
+pairs, so the two launches must agree bit for bit; both must be within the GEMM tolerance of
+the CPU oracle (2^-7 |alpha| sum|a b| + 1e-6). Shapes cover an odd number of row tiles (the
+last pair's second CTA has no rows), weight rows that end inside a tile's second half (that
+half reads as zero), NVFP4 and MXFP4, and the plateau shapes. (The planner uses pairs wherever
+they apply; the plan override switches them off for the comparison.)"""
 import numpy as np
 import pytest
 import torch
@@ -75,11 +75,12 @@ def test_pair_mx(cuda_device, M, N, K):
 
 
 def test_pairs_on_the_plateau(cuda_device):
-    """4096^3 and 8192^3 with tiled scales, pairs on request: same bits as the default plan."""
+    """4096^3 and 8192^3 with tiled scales: the default plan (pairs) gives the same bits as
+    single-CTA tiles."""
     d = cuda_device
     for c in workloads.plateau_cases()[:2]:
         ops = _operands(d, c.a(), c.b())
         o_default = nv.gemm(*ops, tiled=True)
-        with nv.plan_override(pair=2):
-            o_pair = nv.gemm(*ops, tiled=True)
-        assert torch.equal(o_default.view(torch.int16), o_pair.view(torch.int16)), c.name
+        with nv.plan_override(pair=1):
+            o_single = nv.gemm(*ops, tiled=True)
+        assert torch.equal(o_default.view(torch.int16), o_single.view(torch.int16)), c.name
