@@ -424,9 +424,9 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint
  *   groups      split-K clusters per output tile, reduced through the workspace (needs one);
  *   band        output P tiles per rasterisation band;
  *   grouped_bn  token tile width of the grouped GEMM: 32, 64, 128, 176 or 256;
- *   pair        CTA pairs computing 256 x 256 tiles with the 2-SM MMA (256-wide weight tiles
- *               with tiled scales and no split-K): 0 = the planner (pairs wherever they apply),
- *               1 = never, 2 = wherever they apply.
+ *   pair        CTA pairs computing 256-row tiles with the 2-SM MMA (tiled scales, no split-K):
+ *               0 = the planner (pairs for 256-wide tiles with K >= 3072), 1 = never,
+ *               2 = for every 256- or 128-wide tile.
  * The planner's choices need no override; results stay within the GEMM tolerance under any
  * of them, and every override layout is deterministic. Negative values (pair above 2):
  * NVFP4_ERR_INVALID_ARG.

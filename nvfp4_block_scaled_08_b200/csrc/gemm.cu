@@ -115,12 +115,16 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
         p.ws_bytes = p.ws_counter_bytes + static_cast<size_t>(tiles) * g * 128 * p.bn * sizeof(float);
     }
     // CTA pairs computing 256 x 256 tiles with the 2-SM MMA (tiled scales): 256-wide Q tiles
-    // without split-K and at least one pair of P tiles; the pair's work items are P tile
-    // pairs. Each SM then stages 38 KB per K step instead of 54 KB for the same MMA work
-    // (measured on B200: 16384^3 in 1543-1644 us against 1790-1867 us, 8192^3 in 192-203 us
-    // against 216-222 us, 4096^3 in 30.1 us against 32-33 us).
-    const int fp = g_force_pair.load(std::memory_order_relaxed);     // 1: off, 0 / 2: where possible
-    p.pair = !p.swap && p.bn == 256 && p.splits == 1 && p.p_tiles >= 2 && fp != 1;
+    // without split-K, at least one pair of P tiles and at least 12 K stages; the pair's work
+    // items are P tile pairs. Each SM then stages 38 KB per K step instead of 54 KB for the
+    // same MMA work. Measured on B200: 16384^3 in 1528-1577 us against 1771-1850 us, 8192^3 in
+    // 193-194 us against 215-224 us, 4096^3 in 30.3 us against 32.7 us, 8192 x 4096 x 6144 in
+    // 77.6 us against 84.5 us; with 8 K stages (4096 x 6144 x 2048) single CTAs win, 28.8
+    // against 30.8 us. 256 x 128 pair tiles (the override with bn = 128) lost to 256 x 256
+    // ones on every shape measured.
+    const int fp = g_force_pair.load(std::memory_order_relaxed);     // 1: off, 2: wherever possible
+    const bool pair_shape = !p.swap && p.splits == 1 && p.p_tiles >= 2;
+    p.pair = pair_shape && ((fp == 0 && p.bn == 256 && nk >= 12) || (fp == 2 && (p.bn == 256 || p.bn == 128)));
     if (p.pair) {
         const int pairs = ((p.p_tiles + 1) / 2) * p.q_tiles;
         const int clusters = std::max(1, std::min(pairs, max_active_clusters(2)));
@@ -475,6 +479,8 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
         }
         if (plan.pair && plan.bn == 256)
             return run<256, false, false, true, false, true, true>(plan, L, stream, encode_failed);
+        if (plan.pair && plan.bn == 128)
+            return run<128, false, false, true, false, true, true>(plan, L, stream, encode_failed);
         switch (plan.bn) {
             case 128: return run<128, false, false, true, false, true>(plan, L, stream, encode_failed);
             case 256: return run<256, false, false, true, false, true>(plan, L, stream, encode_failed);
@@ -495,6 +501,8 @@ cudaError_t launch_gemm(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t 
         }
         if (plan.pair && plan.bn == 256)
             return run<256, false, false, true, false, false, true>(plan, L, stream, encode_failed);
+        if (plan.pair && plan.bn == 128)
+            return run<128, false, false, true, false, false, true>(plan, L, stream, encode_failed);
         switch (plan.bn) {
             case 128: return run<128, false, false, true>(plan, L, stream, encode_failed);
             case 256: return run<256, false, false, true>(plan, L, stream, encode_failed);

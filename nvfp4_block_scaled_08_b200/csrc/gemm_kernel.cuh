@@ -125,15 +125,17 @@ struct GemmCfg {
     static constexpr bool SFT = SFT_;
     static_assert(!SFT || !GROUPED, "tiled scales serve the dense GEMM");
     static_assert(!MX || (SFT && !GROUPED), "MXFP4 serves the dense GEMM with tiled scales");
-    // PAIR: the two CTAs of a 2-CTA cluster compute one 256 x 256 tile with the 2-SM MMA
-    // (cta_group::2, M = 256): CTA r loads P rows [p0 + 128 r, + 128), Q rows [q0 + 128 r, + 128)
-    // and the scales of its P rows and of all 256 Q rows; the even CTA issues the MMAs, which
-    // read both CTAs' stages, and each CTA's TMEM receives its own 128 rows of the tile. Per
-    // SM a stage is 38 KB instead of 54 KB for the same MMA work, so the ring is 5 deep and
-    // L2 serves a third fewer bytes. Every copy's completion is counted on the even CTA's
-    // full barrier; its commits release both CTAs' stages and accumulators.
+    // PAIR: the two CTAs of a 2-CTA cluster compute one 256 x BN tile with the 2-SM MMA
+    // (cta_group::2, M = 256): CTA r loads P rows [p0 + 128 r, + 128), Q rows
+    // [q0 + BN/2 r, + BN/2) and the scales of its P rows and of all BN Q rows; the even CTA
+    // issues the MMAs, which read both CTAs' stages, and each CTA's TMEM receives its own 128
+    // rows of the tile. For BN = 256 a stage is 38 KB per SM instead of 54 KB for the same MMA
+    // work (5 deep); BN = 128 gives 28 KB stages (7 deep) and twice the work items. Every
+    // copy's completion is counted on the even CTA's full barrier; its commits release both
+    // CTAs' stages and accumulators.
     static constexpr bool PAIR = PAIR_;
-    static_assert(!PAIR || (SFT && !SWAP && !GROUPED && BN == 256), "CTA pairs compute 256-row Q tiles");
+    static_assert(!PAIR || (SFT && !SWAP && !GROUPED && (BN == 256 || BN == 128)),
+                  "CTA pairs compute 256 x 256 or 256 x 128 tiles");
     // ACTQ (few-token launches with tiled weight scales): the activations come in as fp32 or
     // bf16 and are quantised inside the kernel. Every CTA of a split-K cluster reads its own K
     // slice of them, the slices' maxima meet over distributed shared memory (the cluster's
@@ -985,7 +987,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                 for (int ks = 0; ks < n; ++ks) {
                     const int32_t kx = (ti.k0 + ks) * Cfg::BK_BYTES;
                     if constexpr (Cfg::SWAP) tma_prefetch_2d(&tm_p, kx, ti.p0);
-                    else if constexpr (Cfg::PAIR) tma_prefetch_2d(&tm_q, kx, ti.q0 + 128 * static_cast<int32_t>(cluster_ctarank()));
+                    else if constexpr (Cfg::PAIR) tma_prefetch_2d(&tm_q, kx, ti.q0 + (BN / 2) * static_cast<int32_t>(cluster_ctarank()));
                     else tma_prefetch_2d(&tm_q, kx, ti.q0);
                 }
             }
@@ -1041,7 +1043,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                         const int32_t kb = Cfg::SF_BLOCKS * (ti.k0 + ks);
                         const int32_t kb4 = args.sf_kb4;
                         tma_load_2d_pair(pbuf, &tm_p, fb0, kx, ti.p0, pol_p);
-                        tma_load_2d_pair(qbuf, &tm_q, fb0, kx, ti.q0 + 128 * static_cast<int32_t>(rank), pol_q);
+                        tma_load_2d_pair(qbuf, &tm_q, fb0, kx, ti.q0 + (BN / 2) * static_cast<int32_t>(rank), pol_q);
                         tma_load_2d_pair(sfpb, &tm_sfp, fb0, 0, ((ti.p0 >> 7) * kb4 + kb) * 2, pol_p);
 #pragma unroll
                         for (int g = 0; g < QG; ++g)

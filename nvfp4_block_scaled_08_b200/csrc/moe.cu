@@ -20,12 +20,29 @@ namespace nvfp4 {
 
 // ------------------------------------------------------------------ top-k routing
 
-// One warp per token. Lane l holds logits l, l + 32, ... of its token (at most 32 each, E <=
-// 1024). k rounds of a warp arg-max (larger logit first, ties to the lower expert index; the
-// softmax is monotonic, so this is the order of the probabilities), each removing its winner.
+// One warp per token. Lane l holds logits l, l + 32, ... of its token (PER of them, E <= 32
+// PER; entries past E count as taken) and keeps its best untaken entry (larger logit first,
+// then the lower expert index). k rounds of a warp arg-max over the lanes' bests (ties to the
+// lower expert index; the softmax is monotonic, so this is the order of the probabilities);
+// only the winning lane marks its entry taken and looks for its next best.
 // Weights: w_s = exp(l_s - l_0) / sum_j exp(l_j - l_0) over the k winners (l_0 the largest):
 // the softmax probabilities renormalised over the winners (the full softmax's denominator
 // cancels), in fp32 with CUDA's expf, summed in slot order.
+template <int PER>
+__device__ __forceinline__ void lane_best(const float (&v)[PER], uint32_t taken, int lane, float& bv, int& bi)
+{
+    bv = -INFINITY;
+    bi = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        if (!(taken & (1u << i)) && (v[i] > bv || bi == 0x7FFFFFFF)) {
+            bv = v[i];
+            bi = lane + 32 * i;
+        }
+    }
+}
+
+template <int PER>
 __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__ logits, int32_t T, int32_t E,
                                                        int32_t k, int32_t* __restrict__ experts,
                                                        float* __restrict__ weights)
@@ -34,43 +51,40 @@ __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__
     const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;                                   // warp-uniform
     const float* row = logits + t * E;
-    const int per = (E + 31) >> 5;
-    float v[32];
+    float v[PER];
     uint32_t taken = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < PER; ++i) {
         const int e = lane + 32 * i;
-        v[i] = (i < per && e < E) ? __ldg(row + e) : -INFINITY;
-        if (!(i < per && e < E)) taken |= 1u << i;
+        v[i] = e < E ? __ldg(row + e) : -INFINITY;
+        if (e >= E) taken |= 1u << i;
     }
+    float bv;
+    int bi;
+    lane_best<PER>(v, taken, lane, bv, bi);
     float my_val = 0.0f, top = 0.0f;
     int my_idx = 0;
     for (int s = 0; s < k; ++s) {
-        // this lane's best untaken entry
-        float bv = -INFINITY;
-        int bi = 0x7FFFFFFF;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            if (!(taken & (1u << i)) && (v[i] > bv || bi == 0x7FFFFFFF)) {
-                bv = v[i];
-                bi = lane + 32 * i;
-            }
-        }
-        // warp arg-max: larger value, then lower index
+        // warp arg-max of the lanes' bests: larger value, then lower index
+        float wv = bv;
+        int wi = bi;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) {
-                bv = ov;
-                bi = oi;
+            const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, wi, o);
+            if (ov > wv || (ov == wv && oi < wi)) {
+                wv = ov;
+                wi = oi;
             }
         }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (s == 0) top = bv;
+        if ((wi & 31) == lane) {
+            taken |= 1u << (wi >> 5);
+            lane_best<PER>(v, taken, lane, bv, bi);
+        }
+        if (s == 0) top = wv;
         if (lane == s) {
-            my_val = bv;
-            my_idx = bi;
+            my_val = wv;
+            my_idx = wi;
         }
     }
     // weights of the k winners: lane s holds winner s
@@ -217,7 +231,15 @@ cudaError_t launch_moe_route(const float* logits, int32_t T, int32_t E, int32_t 
 {
     cudaError_t e;
     if (T > 0) {
-        moe_topk_kernel<<<(T + 7) / 8, 256, 0, stream>>>(logits, T, E, k, experts, weights);
+        // entries per lane: the power of two at or above ceil(E / 32)
+        const int per = (E + 31) / 32;
+        const unsigned grid = static_cast<unsigned>((T + 7) / 8);
+        if (per <= 1) moe_topk_kernel<1><<<grid, 256, 0, stream>>>(logits, T, E, k, experts, weights);
+        else if (per <= 2) moe_topk_kernel<2><<<grid, 256, 0, stream>>>(logits, T, E, k, experts, weights);
+        else if (per <= 4) moe_topk_kernel<4><<<grid, 256, 0, stream>>>(logits, T, E, k, experts, weights);
+        else if (per <= 8) moe_topk_kernel<8><<<grid, 256, 0, stream>>>(logits, T, E, k, experts, weights);
+        else if (per <= 16) moe_topk_kernel<16><<<grid, 256, 0, stream>>>(logits, T, E, k, experts, weights);
+        else moe_topk_kernel<32><<<grid, 256, 0, stream>>>(logits, T, E, k, experts, weights);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

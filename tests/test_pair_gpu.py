@@ -1,6 +1,7 @@
 """GPU checks of the CTA-pair launch of the dense GEMM: the two CTAs of a 2-CTA cluster compute
-one 256 x 256 tile with the 2-SM MMA (tcgen05.mma.cta_group::2): each loads its own 128 rows of
-the token tile and of the weight tile, and the even CTA's MMAs read both CTAs' shared memory.
+one 256 x 256 (or, on request, 256 x 128) tile with the 2-SM MMA (tcgen05.mma.cta_group::2): each
+loads its own 128 rows of the token tile and its half of the weight tile, and the even CTA's MMAs
+read both CTAs' shared memory.
 
 Every output element is the same sequence of 64-wide block-scaled products with or without
 pairs, so the two launches must agree bit for bit; both must be within the GEMM tolerance of
@@ -26,9 +27,9 @@ def _operands(dev, a, b):
     return Aq, nv.sf_tile(sfA), Bq, nv.sf_tile(sfB), nv.alpha(gsA, gsB)
 
 
-def _gemm(Aq, sA, Bq, sB, al, M, N, pair):
+def _gemm(Aq, sA, Bq, sB, al, M, N, pair, bn=256):
     out = torch.full((M + 2, N), -12352.0, dtype=torch.bfloat16, device=Aq.device)
-    with nv.plan_override(bn=256, cluster=1, groups=1, pair=pair):
+    with nv.plan_override(bn=bn, cluster=1, groups=1, pair=pair):
         nv.gemm(Aq, sA, Bq, sB, al, out=out[:M], tiled=True)
     st, code = nv.last_device_error()
     assert st == 0, hex(code)
@@ -36,15 +37,16 @@ def _gemm(Aq, sA, Bq, sB, al, M, N, pair):
     return out[:M]
 
 
+@pytest.mark.parametrize("bn", [256, 128])
 @pytest.mark.parametrize("M,N,K", [(300, 776, 1024), (512, 1024, 2048), (1000, 264, 512),
                                    (129, 520, 768), (256, 256, 256), (640, 2048, 6144)])
-def test_pair_matches_single_cta_and_oracle(cuda_device, M, N, K):
+def test_pair_matches_single_cta_and_oracle(cuda_device, M, N, K, bn):
     d = cuda_device
     a = workloads.normal(M, K, 1.0, 3 * M + N)
     b = workloads.normal(N, K, 0.02, 5 * N + K)
     ops = _operands(d, a, b)
-    o_pair = _gemm(*ops, M, N, pair=2)
-    o_single = _gemm(*ops, M, N, pair=1)
+    o_pair = _gemm(*ops, M, N, pair=2, bn=bn)
+    o_single = _gemm(*ops, M, N, pair=1, bn=bn)
     assert torch.equal(o_pair.view(torch.int16), o_single.view(torch.int16)), "pair != single-CTA tiles"
     ga, gb = oracle.global_scale(a.numpy()), oracle.global_scale(b.numpy())
     rows = np.r_[0:min(M, 40), max(0, M - 40):M]
@@ -55,8 +57,9 @@ def test_pair_matches_single_cta_and_oracle(cuda_device, M, N, K):
     check_within_tolerance(o_pair[torch.as_tensor(rows, device=d)], v, S, alo, f"pair {M}x{N}x{K}")
 
 
+@pytest.mark.parametrize("bn", [256, 128])
 @pytest.mark.parametrize("M,N,K", [(300, 776, 1024), (512, 1024, 2048)])
-def test_pair_mx(cuda_device, M, N, K):
+def test_pair_mx(cuda_device, M, N, K, bn):
     d = cuda_device
     a = workloads.normal(M, K, 1.0, 7 * M + N)
     b = workloads.normal(N, K, 0.02, 9 * N + K)
@@ -65,7 +68,7 @@ def test_pair_mx(cuda_device, M, N, K):
     al = torch.ones(1, device=d)
     outs = []
     for pair in (2, 1):
-        with nv.plan_override(bn=256, cluster=1, groups=1, pair=pair):
+        with nv.plan_override(bn=bn, cluster=1, groups=1, pair=pair):
             outs.append(nv.mx_gemm(qa, sa, qb, sb, al))
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
     qa_o, sa_o = oracle.mx_quantize(a.numpy())
