@@ -114,7 +114,7 @@ def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> fl
 # dram__bytes_write.sum from one ncu capture of the full-size launch (one pass); the command
 # and the figures are in the committed ncu summary of the plateau under profiles/. Valid only
 # for the kernel sources it was taken on (hash below); reported as null otherwise.
-GEMM_TRAFFIC_BYTES = 1806304768 + 488804096
+GEMM_TRAFFIC_BYTES = 2594956032 + 490243840
 GEMM_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "gemm.cu", "ptx.cuh", "internal.h", "quant_core.cuh")
 GEMM_TRAFFIC_SHA = "e50f3e6377c80c14"
 
