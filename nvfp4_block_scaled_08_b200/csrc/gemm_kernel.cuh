@@ -387,6 +387,78 @@ __device__ __forceinline__ void store_out16(const GemmArgs& a, const Tile& ti, i
     }
 }
 
+// An 8 x 8 transpose of 16-bit elements within each group of 8 lanes: lane 8 g + j enters
+// with elements 0..7 of row j (w[k] = elements 2k, 2k+1, the lower one in the low half) and
+// leaves with element j of rows 0..7 in the same packing. Three butterfly stages (lane bit m =
+// 4, 2, 1): each lane hands its partner (lane ^ m) the four elements it is about to replace
+// and puts the four it receives at their index ^ m.
+__device__ __forceinline__ void transpose8x8_b16(uint32_t (&w)[4], int lane)
+{
+    const int j = lane & 7;
+    {   // m = 4: whole words 2, 3 <-> 0, 1
+        const bool hb = (j & 4) != 0;
+        const uint32_t s0 = hb ? w[0] : w[2], s1 = hb ? w[1] : w[3];
+        const uint32_t r0 = __shfl_xor_sync(0xffffffffu, s0, 4), r1 = __shfl_xor_sync(0xffffffffu, s1, 4);
+        if (hb) { w[0] = r0; w[1] = r1; } else { w[2] = r0; w[3] = r1; }
+    }
+    {   // m = 2: words 1, 3 <-> 0, 2
+        const bool hb = (j & 2) != 0;
+        const uint32_t s0 = hb ? w[0] : w[1], s1 = hb ? w[2] : w[3];
+        const uint32_t r0 = __shfl_xor_sync(0xffffffffu, s0, 2), r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
+        if (hb) { w[0] = r0; w[2] = r1; } else { w[1] = r0; w[3] = r1; }
+    }
+    {   // m = 1: high halves (odd elements) <-> low halves (even elements)
+        const bool hb = (j & 1) != 0;
+        const uint32_t sel = hb ? 0x5410u : 0x7632u;
+        const uint32_t s0 = __byte_perm(w[0], w[1], sel), s1 = __byte_perm(w[2], w[3], sel);
+        const uint32_t r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+        if (hb) {
+            w[0] = __byte_perm(w[0], r0, 0x3254u);
+            w[1] = __byte_perm(w[1], r0, 0x3276u);
+            w[2] = __byte_perm(w[2], r1, 0x3254u);
+            w[3] = __byte_perm(w[3], r1, 0x3276u);
+        } else {
+            w[0] = __byte_perm(w[0], r0, 0x5410u);
+            w[1] = __byte_perm(w[1], r0, 0x7610u);
+            w[2] = __byte_perm(w[2], r1, 0x5410u);
+            w[3] = __byte_perm(w[3], r1, 0x7610u);
+        }
+    }
+}
+
+// Weights-as-M (swap, grouped) epilogue for 16-bit outputs: the warp holds 32 P rows (its lanes:
+// output columns p0 + 32 quad + lane) x 16 accumulator columns c .. c + 15 (output rows, one per
+// token). Scaled, rounded and packed, each 8 x 8 block is transposed within its group of 8
+// lanes, so that lane 8 g + i holds token c + 8 b + i's output columns p0 + 32 quad + 8 g .. + 7:
+// one 16-byte store per lane and block, 64 contiguous bytes per token row and warp.
+template <class Cfg>
+__device__ __forceinline__ void store_tok16(const GemmArgs& a, const Tile& ti, int quad, int lane, int c,
+                                            const uint32_t (&r)[16], float alpha)
+{
+    const int32_t dt = a.out_dtype;
+    uint32_t w[2][4];
+#pragma unroll
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[b][k] = pack_out16x2(alpha * __uint_as_float(r[8 * b + 2 * k]),
+                                   alpha * __uint_as_float(r[8 * b + 2 * k + 1]), dt);
+    transpose8x8_b16(w[0], lane);
+    transpose8x8_b16(w[1], lane);
+    const int n = ti.p0 + 32 * quad + 8 * (lane >> 3);      // 8 output columns; N % 8 == 0
+    if (n >= a.N) return;
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+        const int qi = c + 8 * b + (lane & 7);
+        bool valid;
+        if constexpr (Cfg::GROUPED) valid = qi < ti.q_valid;
+        else valid = ti.q0 + qi < a.M;
+        if (valid)
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + static_cast<size_t>(ti.q0 + qi) * a.N + n) =
+                make_uint4(w[b][0], w[b][1], w[b][2], w[b][3]);
+    }
+}
+
 // An 8 x 8 transpose of 16-byte chunks within each group of 8 lanes (three butterfly stages of
 // shuffles: at stage m the lanes whose bit m differs from the chunk index's swap those
 // chunks): lane 8 g + j enters with chunks 0..7 of its own row and leaves with chunk j of
@@ -1355,7 +1427,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                         } else {
 #pragma unroll
                             for (int i = 0; i < 4; ++i)
-                                if (BN - 64 + 16 * i < n_cols) store_out16<Cfg>(args, ti, p, BN - 64 + 16 * i, r[i], alpha);
+                                if (BN - 64 + 16 * i < n_cols) {
+                                    if (args.out_dtype != kOutF32)
+                                        store_tok16<Cfg>(args, ti, quad, lane, BN - 64 + 16 * i, r[i], alpha);
+                                    else
+                                        store_out16<Cfg>(args, ti, p, BN - 64 + 16 * i, r[i], alpha);
+                                }
                         }
                     }
                     c_hi = min(c_hi, BN - 64);
@@ -1393,6 +1470,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                         const int c = c0 + 16 * h;
                         if constexpr (Cfg::SWIGLU)
                             swiglu_chunk16<Cfg>(args, ti, quad, lane, c, r[h], alpha, gsh, rcp_tab, stage_w, sstage_w);
+                        else if (args.out_dtype != kOutF32)
+                            store_tok16<Cfg>(args, ti, quad, lane, c, r[h], alpha);
                         else
                             store_out16<Cfg>(args, ti, p, c, r[h], alpha);
                     }
