@@ -329,16 +329,23 @@ struct ScatterDst {
     }
 };
 
+// reverse: walk the warp's chunks last to first (a second sweep over a tensor larger than
+// the first sweep could leave in L2 then starts on what the first sweep read last). Each
+// vector is quantised on its own, so the order does not change any output.
 template <typename T, typename Src, typename Dst>
-__device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w0, uint32_t end, uint32_t step,
-                                               float gs, const float* rcp_tab, const Dst& dst)
+__device__ __forceinline__ void quantize_sweep(const Src& src, uint32_t w_first, uint32_t end, uint32_t step,
+                                               float gs, const float* rcp_tab, const Dst& dst,
+                                               bool reverse = false)
 {
     constexpr int V = InTraits<T>::kPerThread;   // elements per thread (8)
     static_assert(V == 8, "8 elements per lane: 4 bytes of codes");
     constexpr int TPB = 16 / V;                  // threads per 16-element block
     constexpr int U = kUnroll;
     const uint32_t lane = threadIdx.x & 31;
-    for (; w0 < end; w0 += U * step) {           // warp-uniform
+    const uint32_t stride = U * step;
+    const uint32_t chunks = w_first < end ? (end - w_first + stride - 1) / stride : 0u;
+    for (uint32_t n = 0; n < chunks; ++n) {      // warp-uniform
+        const uint32_t w0 = w_first + (reverse ? chunks - 1u - n : n) * stride;
         float v[U][V];
 #pragma unroll
         for (int u = 0; u < U; ++u) {

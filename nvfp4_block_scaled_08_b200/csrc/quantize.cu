@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(THREADS) quantize_dynamic_kernel(
         quantize_sweep<T>(StashVecs<T>{stash, v0}, v0 + (threadIdx.x & ~31u), v1, blockDim.x, gs, rcp_tab, dst);
     } else {
         quantize_sweep<T>(GlobalVecs<T>{x, ix}, bid * blockDim.x + (threadIdx.x & ~31u), nv,
-                          nblocks * blockDim.x, gs, rcp_tab, dst);
+                          nblocks * blockDim.x, gs, rcp_tab, dst, true);
     }
 }
 
