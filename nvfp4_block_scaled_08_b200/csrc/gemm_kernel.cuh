@@ -217,9 +217,8 @@ struct GemmCfg {
     static constexpr int OFF_SFQ = OFF_SFP + STAGES * SFP_BYTES;
     static constexpr int OFF_BAR = OFF_SFQ + STAGES * SFQ_BYTES;
     // barriers: full, sfready, empty [STAGES]; acc_full, acc_empty [2]; mma_done; split-K rx;
-    // sf_free [2]; own Q half landed (PAIR) [STAGES]; activations quantised, slice maxima
-    // received (ACTQ)
-    static constexpr int NUM_BARS = 4 * STAGES + 10;
+    // sf_free [2]; activations quantised, slice maxima received (ACTQ)
+    static constexpr int NUM_BARS = 3 * STAGES + 10;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;     // tmem base, flags
     static constexpr int OFF_PREFIX = OFF_MISC + 64;
     static constexpr int OFF_SWIGLU = OFF_PREFIX + (GROUPED ? ((4 * (kMaxExperts + 1) + 15) & ~15) : 0);
@@ -934,8 +933,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     uint64_t* mma_done_bar = bars + 3 * STAGES + 4;
     uint64_t* rx_bar = bars + 3 * STAGES + 5;       // split-K: partial rows received from peers
     uint64_t* sf_free_bar = bars + 3 * STAGES + 6;  // SF_IN_ACC: scale columns drained
-    uint64_t* actq_bar = bars + 4 * STAGES + 8;     // ACTQ: the Q stages hold the activations
-    uint64_t* amax_bar = bars + 4 * STAGES + 9;     // ACTQ: the peers' slice maxima arrived
+    uint64_t* actq_bar = bars + 3 * STAGES + 8;     // ACTQ: the Q stages hold the activations
+    uint64_t* amax_bar = bars + 3 * STAGES + 9;     // ACTQ: the peers' slice maxima arrived
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
     volatile int* s_is_last = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 8);
