@@ -114,9 +114,9 @@ def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> fl
 # dram__bytes_write.sum from one ncu capture of the full-size launch (one pass); the command
 # and the figures are in the committed ncu summary of the plateau under profiles/. Valid only
 # for the kernel sources it was taken on (hash below); reported as null otherwise.
-GEMM_TRAFFIC_BYTES = 3445722368 + 491428352
+GEMM_TRAFFIC_BYTES = 3503670016 + 491254016
 GEMM_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "gemm.cu", "ptx.cuh", "internal.h", "quant_core.cuh")
-GEMM_TRAFFIC_SHA = "0987976bfc0f5f71"
+GEMM_TRAFFIC_SHA = "552f8b41302d6b49"
 
 
 def _code_hash(files) -> str:
