@@ -32,7 +32,7 @@ independent copies (at least 4 x L2 in all) that every launch reads from HBM.
 
 Rooflines: time = max(flops / P_fp4, bytes / BW), against two denominators: the B200
 specification (9 PFLOP/s dense FP4, 8 TB/s HBM3e; the targets are stated against these) and
-the peaks measured on this machine (MEASURED_PEAKS.json: HBM copy bandwidth; dense FP4 = the
+the peaks measured on the B200s in use (MEASURED_PEAKS.json: HBM copy bandwidth; dense FP4 = the
 measured cuBLAS bf16 rate x 4, the nominal FP4 / BF16 ratio of B200).
 
 cpu_baseline: the CPU oracle as it stands (test infrastructure), timed on this machine's
@@ -114,9 +114,9 @@ def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> fl
 # dram__bytes_write.sum from one ncu capture of the full-size launch (one pass); the command
 # and the figures are in the committed ncu summary of the plateau under profiles/. Valid only
 # for the kernel sources it was taken on (hash below); reported as null otherwise.
-GEMM_TRAFFIC_BYTES = 3503670016 + 491254016
+GEMM_TRAFFIC_BYTES = 2204735744 + 512013056
 GEMM_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "gemm.cu", "ptx.cuh", "internal.h", "quant_core.cuh")
-GEMM_TRAFFIC_SHA = "552f8b41302d6b49"
+GEMM_TRAFFIC_SHA = "b7eaedb97e4fc82a"
 
 
 def _code_hash(files) -> str:
@@ -963,8 +963,18 @@ def run_profile(args):
     """A few untimed passes over one configuration's kernels, for ncu (the launch list and
     counters of profiles/ come from this mode): `--profile KEY` with KEY one of single, attn,
     moe_expert, grouped, grouped_small (the T = 4096 density on 32 experts), moe_layer, plateau
-    (all its shapes, or --shape NAME for one)."""
+    (all its shapes, or --shape NAME for one). `--plan band=32,pair=1` runs it under a tile
+    plan override (the fields of nvfp4_set_plan_override), for comparing plans under ncu."""
     import nvfp4_block_scaled_08_b200 as nv
+    kw = {}
+    for item in filter(None, (args.plan or "").split(",")):
+        name, _, val = item.partition("=")
+        kw[name.strip()] = int(val)
+    with nv.plan_override(**kw):
+        _profile_passes(args, nv)
+
+
+def _profile_passes(args, nv):
     from nvfp4_block_scaled_08_b200 import workloads
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -1020,7 +1030,7 @@ def run_profile(args):
     st, code = nv.last_device_error()
     if st != 0:
         raise SystemExit(f"device error word {code:#x}")
-    print(json.dumps({"profile": key, "shape": args.shape, "passes": reps}), flush=True)
+    print(json.dumps({"profile": key, "shape": args.shape, "passes": reps, "plan": args.plan}), flush=True)
 
 
 def main():
@@ -1041,6 +1051,9 @@ def main():
     ap.add_argument("--profile", default=None,
                     help="untimed passes over one configuration's kernels for ncu (see run_profile)")
     ap.add_argument("--shape", default=None, help="with --profile: one shape of the configuration")
+    ap.add_argument("--plan", default=None,
+                    help="with --profile: tile plan override, e.g. band=32 or pair=1 (fields: bn, "
+                         "cluster, groups, band, grouped_bn, pair)")
     args = ap.parse_args()
     if args.profile:
         run_profile(args)

@@ -95,11 +95,15 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
         while (cs * g > nk && cs > 1) --cs;
     }
     // Rasterisation band. While both packed operands fit in L2 together, P-fastest order
-    // over the whole grid (one band); beyond that, bands of 16 P tiles, so that one wave of
-    // tiles spans similar shares of A rows and B columns (16 P x ~9 Q tiles of 256 on 148
-    // SMs). Measured on B200: 8192^3 runs best in one band, 16384^3 with bands of 16.
+    // over the whole grid (one band); beyond that, bands of 32 P tiles (4096 rows of A): all
+    // of B streams through L2 once per band while the band's rows of A stay there. DRAM
+    // bytes read by one launch on B200 (ncu), bands of 16 / 32 / 64 P tiles: 16384^3 with
+    // CTA pairs 3.31 / 2.23 / 4.65 GB in 1579 / 1509 / 1663 us, single CTAs 1.57 / 1.13 GB
+    // (16 / 32); 32768 x 8192 x 8192 1.36 / 0.68 / 0.69 GB in 846 / 798 / 817 us;
+    // 65536 x 16384 x 4096 1.54 / 0.91 / 0.61 GB in 1861 / 1815 / 1799 us;
+    // 16384 x 16384 x 32768 9.87 / 9.62 / 14.8 GB in 3401 / 3386 / 3698 us.
     const double packed_bytes = static_cast<double>(M + N) * static_cast<double>(K) * 0.5;
-    p.band = packed_bytes <= 80e6 ? p.p_tiles : std::max(1, std::min(p.p_tiles, 16));
+    p.band = packed_bytes <= 80e6 ? p.p_tiles : std::max(1, std::min(p.p_tiles, 32));
     {
         const int fb = g_force_band.load(std::memory_order_relaxed);
         if (fb > 0) p.band = std::min(p.p_tiles, fb);
