@@ -1411,8 +1411,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
-                        if constexpr (Cfg::PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_free_bar[acc]), 0));
-                        else mbar_arrive(&sf_free_bar[acc]);
+                        if constexpr (Cfg::PAIR) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&sf_free_bar[acc]), 0));
+                        else mbar_arrive_relaxed(&sf_free_bar[acc]);
                     }
                     if (need) {
                         if constexpr (!Cfg::SWAP && !Cfg::GROUPED) {
@@ -1481,8 +1481,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if constexpr (Cfg::PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty_bar[acc]), 0));
-                else mbar_arrive(&acc_empty_bar[acc]);
+                if constexpr (Cfg::PAIR) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&acc_empty_bar[acc]), 0));
+                else mbar_arrive_relaxed(&acc_empty_bar[acc]);
             }
             if (++acc == Cfg::ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
 

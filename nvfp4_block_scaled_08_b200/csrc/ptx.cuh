@@ -398,10 +398,20 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         : "memory");
 }
 
-// Arrive (release, cluster scope) on the mbarrier at `bar_cluster` (from mapa).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster)
+// Relaxed arrivals: they order no memory. For signals whose only content is "this thread's
+// tcgen05.ld reads have completed" (tcgen05.wait::ld, then tcgen05.fence::before_thread_sync):
+// the waiting side's tcgen05 writes are issued only after it observes the arrival. A release
+// arrival would first wait until the thread's earlier global stores are visible at its scope,
+// which at cluster scope cost ~0.6 us per tile in the epilogue of the CTA-pair GEMM.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t* bar)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// On the mbarrier at `bar_cluster` (from mapa), possibly another CTA's.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_cluster)
+{
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 // ---------------------------------------------------------------------------- TMEM loads
