@@ -425,10 +425,12 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint
  *   band        output P tiles per rasterisation band;
  *   grouped_bn  token tile width of the grouped GEMM: 32, 64, 128, 176 or 256;
  *   pair        CTA pairs computing 256-row tiles with the 2-SM MMA (tiled scales, no split-K):
- *               0 = the planner (pairs for 256-wide tiles with K >= 3072), 1 = never,
- *               2 = for every 256- or 128-wide tile.
+ *               0 = the planner (pairs for 256-wide tiles with K >= 3072; a last round of
+ *               256 x 256 tiles that fills at most half of the pairs runs as 256 x 128
+ *               halves), 1 = never, 2 = for every 256- or 128-wide tile, 3 = as 0 but
+ *               without the halves.
  * The planner's choices need no override; results stay within the GEMM tolerance under any
- * of them, and every override layout is deterministic. Negative values (pair above 2):
+ * of them, and every override layout is deterministic. Negative values (pair above 3):
  * NVFP4_ERR_INVALID_ARG.
  */
 nvfp4_status nvfp4_set_plan_override(int32_t bn, int32_t cluster, int32_t groups, int32_t band,

@@ -591,7 +591,7 @@ nvfp4_status nvfp4_moe_combine(const void* y, nvfp4_out_dtype y_dtype, const flo
 nvfp4_status nvfp4_set_plan_override(int32_t bn, int32_t cluster, int32_t groups, int32_t band,
                                      int32_t grouped_bn, int32_t pair)
 {
-    if (bn < 0 || cluster < 0 || groups < 0 || band < 0 || grouped_bn < 0 || pair < 0 || pair > 2)
+    if (bn < 0 || cluster < 0 || groups < 0 || band < 0 || grouped_bn < 0 || pair < 0 || pair > 3)
         return NVFP4_ERR_INVALID_ARG;
     nvfp4::set_plan_override(bn, cluster, groups, band, grouped_bn, pair);
     return NVFP4_OK;

@@ -126,14 +126,25 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
     // 77.6 us against 84.5 us; with 8 K stages (4096 x 6144 x 2048) single CTAs win, 28.8
     // against 30.8 us. 256 x 128 pair tiles (the override with bn = 128) lost to 256 x 256
     // ones on every shape measured.
-    const int fp = g_force_pair.load(std::memory_order_relaxed);     // 1: off, 2: wherever possible
+    // 1: off, 2: wherever possible, 3: the planner's pairs without half tiles
+    const int fp = g_force_pair.load(std::memory_order_relaxed);
     const bool pair_shape = !p.swap && p.splits == 1 && p.p_tiles >= 2;
-    p.pair = pair_shape && ((fp == 0 && p.bn == 256 && nk >= 12) || (fp == 2 && (p.bn == 256 || p.bn == 128)));
+    p.pair = pair_shape && (((fp == 0 || fp == 3) && p.bn == 256 && nk >= 12) || (fp == 2 && (p.bn == 256 || p.bn == 128)));
     if (p.pair) {
         const int pairs = ((p.p_tiles + 1) / 2) * p.q_tiles;
         const int clusters = std::max(1, std::min(pairs, max_active_clusters(2)));
         p.pair_grid = 2 * clusters;
         p.pair_band = std::max(1, p.band / 2);
+        // A last round of 256 x 256 tiles that fills at most half of the pairs runs as twice
+        // as many 256 x 128 halves, in about half the time (4096^3: 256 tiles on 74 pairs,
+        // 3.46 rounds).
+        const int tail = pairs % clusters;
+        p.pair_items = pairs;
+        p.narrow_from = pairs;
+        if (p.bn == 256 && tail > 0 && 2 * tail <= clusters && fp != 3) {
+            p.narrow_from = pairs - tail;
+            p.pair_items = pairs + tail;
+        }
     }
     return p;
 }
@@ -322,7 +333,7 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
 
     const uint64_t kb = static_cast<uint64_t>(L.K / 2);    // packed bytes per row
     const uint64_t ks = static_cast<uint64_t>(L.K / 16);   // scale bytes per row
-    CUtensorMap tp, tq, tsp, tsq;
+    CUtensorMap tp, tq, tsp, tsq, tq_half;
     bool ok = true;
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -369,6 +380,8 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
         ok &= get_map(&tp, P, 2, kb, p_rows, 1, kb, 0, 128, 128, true);
         if constexpr (ACTQ) tq = tp;          // unused: the kernel quantises the activations itself
         else ok &= get_map(&tq, Q, 2, kb, q_rows, 1, kb, 0, 128, PAIR ? BN / 2 : BN, true);   // PAIR: half tiles
+        // PAIR, BN = 256: each CTA's 64 rows of a 256 x 128 half tile
+        if constexpr (Cfg::NARROW) ok &= get_map(&tq_half, Q, 2, kb, q_rows, 1, kb, 0, 128, BN / 4, true);
         if constexpr (PAIR) {
             // the tiled scales as rows of 256 bytes: a stage's run of one 128-row tile is
             // SFP_BYTES / 256 rows (past the last tile: zero fill)
@@ -418,13 +431,15 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
             a.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(L.ws) + plan.ws_counter_bytes);
         }
     }
+    if constexpr (!Cfg::NARROW) tq_half = tq;   // unused
     if (!ok) {
         *encode_failed = true;
         return cudaSuccess;
     }
     if constexpr (PAIR) {
         a.band = plan.pair_band;
-        a.num_tiles = a.num_p_tiles * plan.q_tiles;
+        a.num_tiles = plan.pair_items;
+        a.narrow_from = plan.narrow_from;
     }
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
@@ -443,7 +458,7 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
     if constexpr (PAIR) attrs[1].val.clusterDim.x = 2;
     cfg.attrs = attrs;
     cfg.numAttrs = (!GROUPED && (plan.cluster > 1 || PAIR)) ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, kern, tp, tq, tsp, tsq, a);
+    return cudaLaunchKernelEx(&cfg, kern, tp, tq, tsp, tsq, tq_half, a);
 }
 
 int act_gemm_stages(int bn)

@@ -76,6 +76,7 @@ struct GemmArgs {
     int32_t groups;           // clusters per output tile (reduced through the workspace)
     int32_t num_tiles;        // non-grouped: p_tiles * q_tiles * splits
     int32_t band;             // non-grouped: P tiles per rasterisation band (>= 1)
+    int32_t narrow_from;      // PAIR, BN = 256: work items from here on are half tiles (see decode_tile)
     void* out;                // out_dtype elements
     int32_t out_dtype;        // kOutBF16, kOutF16 or kOutF32
     const float* alpha;       // [1] or [E]
@@ -163,6 +164,9 @@ struct GemmCfg {
     static constexpr int SF_TMA_Q = BN * 16;
     static constexpr uint32_t TX_BYTES = P_BYTES + Q_BYTES + SF_TMA_P + SF_TMA_Q;
     static constexpr uint32_t PAIR_TX_BYTES = 2u * (P_BYTES + Q_BYTES + SFP_BYTES + SFP_BYTES * QG);  // both CTAs'
+    // PAIR, BN = 256: a half tile (256 x 128) loads half the Q rows and one Q scale group
+    static constexpr bool NARROW = PAIR && BN == 256;
+    static constexpr uint32_t PAIR_TX_NARROW = 2u * (P_BYTES + Q_BYTES / 2 + SFP_BYTES + SFP_BYTES);
     static constexpr int SF_ROWS256 = SFP_BYTES / 256;   // PAIR: a stage's scale run as rows of 256 bytes
     // Grouped: the token tile is loaded in boxes of QBOX rows, only as many as the expert's
     // rows in the tile need (a tile of a 256-wide plan often holds ~128 rows of one expert).
@@ -240,6 +244,7 @@ struct Tile {
     int32_t split;     // split index
     int32_t expert;    // grouped: expert id
     int32_t q_valid;   // grouped: valid Q rows in this tile (<= BN)
+    int32_t q_span;    // Q rows (MMA N) of the tile: BN, or BN / 2 for a half tile
 };
 
 // Row range of expert e, clamped to [0, total_rows] and made non-decreasing, so that
@@ -273,12 +278,23 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, int32_t t, const 
         ti.p0 = pt * Cfg::BM;
         ti.q0 = r0 + qt * Cfg::BN;
         ti.q_valid = min(Cfg::BN, rows - qt * Cfg::BN);
+        ti.q_span = Cfg::BN;
         ti.k0 = 0;
         ti.kcnt = a.num_kstages;
         ti.pq = 0;
         ti.split = 0;
         ti.expert = e;
     } else {
+        // PAIR, BN = 256: items from narrow_from on split the last output tiles in two halves
+        // of 128 columns each (a last round of tiles shorter than a full one fills twice as
+        // many SMs for half as long): item narrow_from + 2 j + h is half h of tile narrow_from + j.
+        int32_t half = -1;
+        if constexpr (Cfg::NARROW) {
+            if (t >= a.narrow_from) {
+                half = (t - a.narrow_from) & 1;
+                t = a.narrow_from + ((t - a.narrow_from) >> 1);
+            }
+        }
         const int32_t split = t % a.splits;
         const int32_t pq = t / a.splits;
         // Output tiles in bands of `band` P tiles: column by column (Q tile) within a band, P
@@ -293,13 +309,14 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, int32_t t, const 
         const int32_t rem = a.num_kstages % a.splits;
         if constexpr (Cfg::PAIR) ti.p0 = (2 * pt + static_cast<int32_t>(cluster_ctarank())) * Cfg::BM;
         else ti.p0 = pt * Cfg::BM;
-        ti.q0 = qt * Cfg::BN;
+        ti.q0 = qt * Cfg::BN + (half > 0 ? Cfg::BN / 2 : 0);
+        ti.q_span = half >= 0 ? Cfg::BN / 2 : Cfg::BN;
         ti.k0 = split * base + min(split, rem);
         ti.kcnt = base + (split < rem ? 1 : 0);
         ti.pq = pq;
         ti.split = split;
         ti.expert = 0;
-        ti.q_valid = min(Cfg::BN, a.q_rows - ti.q0);
+        ti.q_valid = min(ti.q_span, a.q_rows - ti.q0);
     }
     return ti;
 }
@@ -914,7 +931,7 @@ template <class Cfg>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_sfp, const __grid_constant__ CUtensorMap tm_sfq,
-                  const GemmArgs args)
+                  const __grid_constant__ CUtensorMap tm_q_half, const GemmArgs args)
 {
     constexpr int BN = Cfg::BN;
     constexpr int STAGES = Cfg::STAGES;
@@ -972,6 +989,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             prefetch_tensormap(&tm_sfp);
             prefetch_tensormap(&tm_sfq);
         }
+        if constexpr (Cfg::NARROW) prefetch_tensormap(&tm_q_half);
     }
     if (warp == 1) {
         if constexpr (Cfg::PAIR) {
@@ -1058,7 +1076,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                 for (int ks = 0; ks < n; ++ks) {
                     const int32_t kx = (ti.k0 + ks) * Cfg::BK_BYTES;
                     if constexpr (Cfg::SWAP) tma_prefetch_2d(&tm_p, kx, ti.p0);
-                    else if constexpr (Cfg::PAIR) tma_prefetch_2d(&tm_q, kx, ti.q0 + (BN / 2) * static_cast<int32_t>(cluster_ctarank()));
+                    else if constexpr (Cfg::PAIR) tma_prefetch_2d(&tm_q, kx, ti.q0 + (ti.q_span / 2) * static_cast<int32_t>(cluster_ctarank()));
                     else tma_prefetch_2d(&tm_q, kx, ti.q0);
                 }
             }
@@ -1108,18 +1126,23 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                         // arms for both CTAs' bytes (rows past the operands read as zero). The
                         // scale runs are read through 2-D views of the tiled layout (rows of
                         // 256 bytes), so that they can complete on the even CTA's barrier too.
+                        // (a half tile: 64 Q rows per CTA through the half-height map, and the
+                        // scales of its 128 Q rows only)
                         const uint32_t rank = cluster_ctarank();
                         const uint32_t fb0 = mapa_shared(smem_u32(fb), 0);
-                        if (rank == 0) mbar_arrive_expect_tx(fb, Cfg::PAIR_TX_BYTES);
+                        const bool narrow = Cfg::NARROW && ti.q_span < BN;
+                        if (rank == 0) mbar_arrive_expect_tx(fb, narrow ? Cfg::PAIR_TX_NARROW : Cfg::PAIR_TX_BYTES);
                         const int32_t kb = Cfg::SF_BLOCKS * (ti.k0 + ks);
                         const int32_t kb4 = args.sf_kb4;
                         tma_load_2d_pair(pbuf, &tm_p, fb0, kx, ti.p0, pol_p);
-                        tma_load_2d_pair(qbuf, &tm_q, fb0, kx, ti.q0 + (BN / 2) * static_cast<int32_t>(rank), pol_q);
+                        tma_load_2d_pair(qbuf, narrow ? &tm_q_half : &tm_q, fb0, kx,
+                                         ti.q0 + (ti.q_span / 2) * static_cast<int32_t>(rank), pol_q);
                         tma_load_2d_pair(sfpb, &tm_sfp, fb0, 0, ((ti.p0 >> 7) * kb4 + kb) * 2, pol_p);
 #pragma unroll
                         for (int g = 0; g < QG; ++g)
-                            tma_load_2d_pair(sfqb + Cfg::SFP_BYTES * g, &tm_sfq, fb0, 0,
-                                             (((ti.q0 >> 7) + g) * kb4 + kb) * 2, pol_q);
+                            if (g == 0 || !narrow)
+                                tma_load_2d_pair(sfqb + Cfg::SFP_BYTES * g, &tm_sfq, fb0, 0,
+                                                 (((ti.q0 >> 7) + g) * kb4 + kb) * 2, pol_q);
                     } else if constexpr (Cfg::ACTQ) {
                         // weights and their scales only: the epilogue warps fill the Q stages
                         mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::SFP_BYTES);
@@ -1197,6 +1220,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             const uint32_t sf_b = sf_a + 4 * Cfg::SF_BLOCKS;    // after the SFA columns
             uint32_t n_mma = BN;
             if constexpr (Cfg::GROUPED) n_mma = min(BN, (ti.q_valid + 15) & ~15);
+            if constexpr (Cfg::NARROW) n_mma = static_cast<uint32_t>(ti.q_span);
             constexpr uint32_t kMmaM = Cfg::PAIR ? 256 : 128;
             const uint32_t idesc = Cfg::MX ? idesc_mxf4_ue8m0(kMmaM, n_mma) : idesc_mxf4nvf4(kMmaM, n_mma);
             const uint32_t d_tmem = tmem_base + acc * BN;
@@ -1216,8 +1240,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                             tmem_cp_32x128b_warpx4_pair(sf_a + 4 * j, sdesc_sf_32x16(sfp + 512 * j));
 #pragma unroll
                             for (int g = 0; g < QG; ++g)
-                                tmem_cp_32x128b_warpx4_pair(sf_b + 4 * QG * j + 4 * g,
-                                                            sdesc_sf_32x16(sfq + Cfg::SFP_BYTES * g + 512 * j));
+                                if (128 * g < static_cast<int>(n_mma))
+                                    tmem_cp_32x128b_warpx4_pair(sf_b + 4 * QG * j + 4 * g,
+                                                                sdesc_sf_32x16(sfq + Cfg::SFP_BYTES * g + 512 * j));
                         } else {
                             tmem_cp_32x128b_warpx4(sf_a + 4 * j, sdesc_sf_32x16(sfp + 512 * j));
 #pragma unroll
@@ -1389,6 +1414,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             const bool split_k = !Cfg::GROUPED && args.splits > 1;
             int n_cols = BN;
             if constexpr (Cfg::GROUPED) n_cols = min(BN, (ti.q_valid + 15) & ~15);
+            if constexpr (Cfg::NARROW) n_cols = ti.q_span;
             if constexpr (!Cfg::GROUPED) {
                 if (split_k && half == 0)
                     split_k_epilogue<Cfg>(args, ti, smem, rx_bar, s_is_last, tacc, row, alpha, ab);

@@ -63,6 +63,8 @@ struct GemmPlan {
     bool pair = false;     // 2-CTA clusters sharing 256-row Q tiles (tiled scales, no split-K)
     int pair_grid = 0;     // CTAs of the pair launch (2 per cluster)
     int pair_band = 1;     // rasterisation band of the pair launch, in P tile pairs
+    int pair_items = 0;    // work items of the pair launch (tiles, the last ones split in halves)
+    int narrow_from = 0;   // first half-tile item of the pair launch (= pair_items: none)
     size_t ws_bytes = 0;   // workspace needed (split-K)
     size_t ws_counter_bytes = 0;
 };

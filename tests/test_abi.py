@@ -132,7 +132,7 @@ def test_moe_host_validation(lib):
 def test_plan_override_validation(lib):
     assert lib.nvfp4_set_plan_override(-1, 0, 0, 0, 0, 0) == 1
     assert lib.nvfp4_set_plan_override(0, 0, -2, 0, 0, 0) == 1
-    assert lib.nvfp4_set_plan_override(0, 0, 0, 0, 0, 3) == 1
+    assert lib.nvfp4_set_plan_override(0, 0, 0, 0, 0, 4) == 1
     assert lib.nvfp4_set_plan_override(0, 0, 0, 0, 0, 0) == 0
     with nv.plan_override(cluster=2, groups=3):
         pass

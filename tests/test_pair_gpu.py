@@ -87,3 +87,49 @@ def test_pairs_on_the_plateau(cuda_device):
         with nv.plan_override(pair=1):
             o_single = nv.gemm(*ops, tiled=True)
         assert torch.equal(o_default.view(torch.int16), o_single.view(torch.int16)), c.name
+
+
+@pytest.mark.parametrize("M,N,K", [(2500, 2056, 1024), (4096, 4096, 3072)])
+def test_pair_half_tiles(cuda_device, M, N, K):
+    """A last round of 256 x 256 pair tiles that fills at most half of the pairs runs as
+    256 x 128 halves. On 148 SMs (74 pairs): 2500 x 2056 has 10 x 9 = 90 tiles, the last 16
+    split in halves, the last Q tile 8 columns wide (its second half starts past N) and the
+    last P tile 68 rows; 4096 x 4096 has 256 tiles, the last 34 split. Same bits as the
+    single-CTA tiles and as pairs without halves, within tolerance of the oracle."""
+    d = cuda_device
+    a = workloads.normal(M, K, 1.0, 11 * M + N)
+    b = workloads.normal(N, K, 0.02, 13 * N + K)
+    ops = _operands(d, a, b)
+    o_half = _gemm(*ops, M, N, pair=2)
+    o_whole = _gemm(*ops, M, N, pair=3) if K >= 3072 else None
+    o_single = _gemm(*ops, M, N, pair=1)
+    assert torch.equal(o_half.view(torch.int16), o_single.view(torch.int16)), "half tiles != single-CTA tiles"
+    if o_whole is not None:
+        assert torch.equal(o_half.view(torch.int16), o_whole.view(torch.int16)), "half tiles != whole pair tiles"
+    ga, gb = oracle.global_scale(a.numpy()), oracle.global_scale(b.numpy())
+    rows = np.r_[0:24, M - 72:M]
+    qa, sa = oracle.quantize(a[rows].contiguous().numpy(), ga)
+    qb, sb = oracle.quantize(b.numpy(), gb)
+    alo = oracle.alpha(ga, gb)
+    v, S, _ = oracle.gemm(qa, sa, qb, sb, alo)
+    check_within_tolerance(o_half[torch.as_tensor(rows, device=d)], v, S, alo, f"half tiles {M}x{N}x{K}")
+
+
+def test_pair_half_tiles_mx(cuda_device):
+    d = cuda_device
+    M, N, K = 2500, 2056, 1024
+    a = workloads.normal(M, K, 1.0, 17 * M + N)
+    b = workloads.normal(N, K, 0.02, 19 * N + K)
+    qa, sa = nv.mx_quantize(a.to(d), tiled=True)
+    qb, sb = nv.mx_quantize(b.to(d), tiled=True)
+    al = torch.ones(1, device=d)
+    outs = []
+    for pair in (2, 1):
+        with nv.plan_override(bn=256, cluster=1, groups=1, pair=pair):
+            outs.append(nv.mx_gemm(qa, sa, qb, sb, al))
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    rows = np.r_[0:16, M - 48:M]
+    qa_o, sa_o = oracle.mx_quantize(a[rows].contiguous().numpy())
+    qb_o, sb_o = oracle.mx_quantize(b.numpy())
+    v, S, _ = oracle.mx_gemm(qa_o, sa_o, qb_o, sb_o, 1.0)
+    check_within_tolerance(outs[0][torch.as_tensor(rows, device=d)], v, S, 1.0, f"mx half tiles {M}x{N}x{K}")
