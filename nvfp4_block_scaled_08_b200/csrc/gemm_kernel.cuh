@@ -1517,16 +1517,27 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
 
     // ------------------------------------------------------------------ teardown
     __syncwarp();
-    if constexpr (!Cfg::GROUPED) {
+    if constexpr (!Cfg::GROUPED && !Cfg::RX_OWN) {
         // split-K: the non-epilogue warps (and the second epilogue warpgroup) are done with
         // the pipeline; together with the first epilogue warpgroup's arrival (after its
         // accumulator is complete) this tells the cluster peers that this CTA's shared memory
         // may receive their partial rows
-        // (with a receive region of its own the first warpgroup has not arrived yet either: no
-        // CTA leaves while a peer's rows may still be on their way to it)
-        if ((Cfg::RX_OWN || warp < 4 || warp >= 8) && args.splits > 1 && args.cluster_size > 1) {
+        if ((warp < 4 || warp >= 8) && args.splits > 1 && args.cluster_size > 1) {
             cluster_arrive();
             cluster_wait();
+        }
+    }
+    if constexpr (Cfg::RX_OWN) {
+        // split-K with a receive region of its own: no cluster barrier. Every byte a peer sends
+        // to this CTA (partial rows; ACTQ: slice maxima) is counted on this CTA's own rx (amax)
+        // barrier, which its epilogue has waited for, so nothing is still on its way here when
+        // it leaves. After an abort those waits may not have completed: wait for them once more,
+        // bounded, so that no peer's rows land in the shared memory of a CTA that has left.
+        if (warp == 4 && lane == 0 && args.splits > 1 && args.cluster_size > 1) {
+            if (!mbar_test_wait(rx_bar, 0)) mbar_wait_drain(rx_bar, 0);
+            if constexpr (Cfg::ACTQ) {
+                if (!mbar_test_wait(amax_bar, 0)) mbar_wait_drain(amax_bar, 0);
+            }
         }
     }
     tc_fence_before();
