@@ -428,7 +428,8 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint
  *               0 = the planner (pairs for 256-wide tiles with K >= 3072; a last round of
  *               256 x 256 tiles that fills at most half of the pairs runs as 256 x 128
  *               halves), 1 = never, 2 = for every 256- or 128-wide tile, 3 = as 0 but
- *               without the halves.
+ *               without the halves; the grouped GEMM runs pairs for 128- and 176-row token
+ *               tiles unless this is 1.
  * The planner's choices need no override; results stay within the GEMM tolerance under any
  * of them, and every override layout is deterministic. Negative values (pair above 3):
  * NVFP4_ERR_INVALID_ARG.

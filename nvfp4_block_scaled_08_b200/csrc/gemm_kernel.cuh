@@ -135,8 +135,14 @@ struct GemmCfg {
     // copy's completion is counted on the even CTA's full barrier; its commits release both
     // CTAs' stages and accumulators.
     static constexpr bool PAIR = PAIR_;
-    static_assert(!PAIR || (SFT && !SWAP && !GROUPED && (BN == 256 || BN == 128)),
-                  "CTA pairs compute 256 x 256 or 256 x 128 tiles");
+    // Grouped pairs (GPAIR): the two CTAs hold 128 weight rows each of a 256-row weight tile
+    // pair of one expert and half of its token tile (each CTA loads all the tile's token
+    // scales); their linear scales are re-laid out in each CTA, which then signals the even
+    // CTA's sfready barrier before the MMA may copy them.
+    static constexpr bool GPAIR = PAIR && GROUPED;
+    static_assert(!PAIR || (SFT && !SWAP && !GROUPED && (BN == 256 || BN == 128)) ||
+                  (GROUPED && SWAP && !SFT && (BN == 128 || BN == 176)),
+                  "CTA pairs compute 256 x 256 or 256 x 128 dense tiles, or grouped 256 x 128 / 176 tiles");
     // ACTQ (few-token launches with tiled weight scales): the activations come in as fp32 or
     // bf16 and are quantised inside the kernel. Every CTA of a split-K cluster reads its own K
     // slice of them, the slices' maxima meet over distributed shared memory (the cluster's
@@ -165,7 +171,7 @@ struct GemmCfg {
     static constexpr uint32_t TX_BYTES = P_BYTES + Q_BYTES + SF_TMA_P + SF_TMA_Q;
     static constexpr uint32_t PAIR_TX_BYTES = 2u * (P_BYTES + Q_BYTES + SFP_BYTES + SFP_BYTES * QG);  // both CTAs'
     // PAIR, BN = 256: a half tile (256 x 128) loads half the Q rows and one Q scale group
-    static constexpr bool NARROW = PAIR && BN == 256;
+    static constexpr bool NARROW = PAIR && BN == 256 && !GROUPED;
     static constexpr uint32_t PAIR_TX_NARROW = 2u * (P_BYTES + Q_BYTES / 2 + SFP_BYTES + SFP_BYTES);
     static constexpr int SF_ROWS256 = SFP_BYTES / 256;   // PAIR: a stage's scale run as rows of 256 bytes
     // Grouped: the token tile is loaded in boxes of QBOX rows, only as many as the expert's
@@ -221,8 +227,9 @@ struct GemmCfg {
     static constexpr int OFF_SFQ = OFF_SFP + STAGES * SFP_BYTES;
     static constexpr int OFF_BAR = OFF_SFQ + STAGES * SFQ_BYTES;
     // barriers: full, sfready, empty [STAGES]; acc_full, acc_empty [2]; mma_done; split-K rx;
-    // sf_free [2]; activations quantised, slice maxima received (ACTQ)
-    static constexpr int NUM_BARS = 3 * STAGES + 10;
+    // sf_free [2]; activations quantised, slice maxima received (ACTQ); GPAIR: this CTA's
+    // scales landed [STAGES]
+    static constexpr int NUM_BARS = 4 * STAGES + 10;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;     // tmem base, flags
     static constexpr int OFF_PREFIX = OFF_MISC + 64;
     static constexpr int OFF_SWIGLU = OFF_PREFIX + (GROUPED ? ((4 * (kMaxExperts + 1) + 15) & ~15) : 0);
@@ -275,7 +282,9 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, int32_t t, const 
         const int32_t local = t - prefix[e];
         const int32_t pt = local / qt_count;
         const int32_t qt = local - pt * qt_count;
-        ti.p0 = pt * Cfg::BM;
+        // GPAIR: pt counts 256-row weight tile pairs; this CTA's half
+        if constexpr (Cfg::PAIR) ti.p0 = (2 * pt + static_cast<int32_t>(cluster_ctarank())) * Cfg::BM;
+        else ti.p0 = pt * Cfg::BM;
         ti.q0 = r0 + qt * Cfg::BN;
         ti.q_valid = min(Cfg::BN, rows - qt * Cfg::BN);
         ti.q_span = Cfg::BN;
@@ -952,6 +961,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     uint64_t* sf_free_bar = bars + 3 * STAGES + 6;  // SF_IN_ACC: scale columns drained
     uint64_t* actq_bar = bars + 3 * STAGES + 8;     // ACTQ: the Q stages hold the activations
     uint64_t* amax_bar = bars + 3 * STAGES + 9;     // ACTQ: the peers' slice maxima arrived
+    uint64_t* sf_full_bar = bars + 3 * STAGES + 10; // GPAIR: this CTA's scales of stage s landed
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
     volatile int* s_is_last = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 8);
@@ -965,8 +975,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&sfready_bar[s], 1);
+            // GPAIR: the even CTA's counts one re-layout arrival from each CTA
+            mbar_init(&sfready_bar[s], Cfg::GPAIR ? 2 : 1);
             mbar_init(&empty_bar[s], 1);
+            mbar_init(&sf_full_bar[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full_bar[s], 1);
@@ -1098,7 +1110,35 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     uint8_t* qbuf = smem + Cfg::OFF_Q + stage * Cfg::Q_BYTES;
                     uint8_t* sfpb = smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES;
                     uint8_t* sfqb = smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES;
-                    if constexpr (Cfg::GROUPED) {
+                    if constexpr (Cfg::GPAIR) {
+                        // this CTA's 128 weight rows and half of the token tile's MMA N (its
+                        // rows rounded up to 16), both counted on the even CTA's full barrier,
+                        // which the even CTA arms for both CTAs' bytes; the scales of its weight
+                        // rows and of all the tile's token rows on its own sf_full barrier (its
+                        // re-layout warps wait there)
+                        const uint32_t rank = cluster_ctarank();
+                        const uint32_t fb0 = mapa_shared(smem_u32(fb), 0);
+                        const int n_mma = min(BN, (ti.q_valid + 15) & ~15);
+                        const int half = n_mma / 2;
+                        const int qb = (half + Cfg::QBOX - 1) / Cfg::QBOX;
+                        const int sb = (n_mma + Cfg::QBOX - 1) / Cfg::QBOX;
+                        uint64_t* sfb = &sf_full_bar[stage];
+                        if (rank == 0)
+                            mbar_arrive_expect_tx(fb, 2u * static_cast<uint32_t>(Cfg::P_BYTES + qb * Cfg::QBOX * Cfg::BK_BYTES));
+                        mbar_arrive_expect_tx(sfb, static_cast<uint32_t>(Cfg::SF_TMA_P + sb * Cfg::QBOX * 16));
+                        if constexpr (Cfg::SWIGLU) {
+                            tma_load_5d_pair(pbuf, &tm_p, fb0, kx, 0, 0, ti.p0 >> 5, ti.expert, pol_p);
+                            tma_load_5d(sfpb, &tm_sfp, sfb, sx, 0, 0, ti.p0 >> 5, ti.expert, pol_p);
+                        } else {
+                            tma_load_3d_pair(pbuf, &tm_p, fb0, kx, ti.p0, ti.expert, pol_p);
+                            tma_load_3d(sfpb, &tm_sfp, sfb, sx, ti.p0, ti.expert, pol_p);
+                        }
+                        for (int b = 0; b < qb; ++b)
+                            tma_load_2d_pair(qbuf + b * Cfg::QBOX * Cfg::BK_BYTES, &tm_q, fb0, kx,
+                                             ti.q0 + half * static_cast<int32_t>(rank) + b * Cfg::QBOX, pol_q);
+                        for (int b = 0; b < sb; ++b)
+                            tma_load_2d(sfqb + b * Cfg::QBOX * 16, &tm_sfq, sfb, sx, ti.q0 + b * Cfg::QBOX, pol_q);
+                    } else if constexpr (Cfg::GROUPED) {
                         // boxes of QBOX token rows covering the tile's MMA N (its rows rounded
                         // up to 16); the 8-row swizzle atoms of the boxes line up as in one box
                         const int n_mma = min(BN, (ti.q_valid + 15) & ~15);
@@ -1193,6 +1233,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
             const int s = ((int)stage - (int)i + 2 * STAGES) % STAGES;
             const uint32_t ph = ((int)stage - (int)i < 0) ? (phase ^ 1u) : phase;
             mbar_wait_drain(on_empty ? &empty_bar[s] : &full_bar[s], ph);
+            if constexpr (Cfg::GPAIR) mbar_wait_drain(&sf_full_bar[s], ph);   // this CTA's scale copies
         }
     } else if (warp == 1) {
         // -------------------------------------------------------------- MMA issuer
@@ -1322,7 +1363,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     continue;
                 }
-                ok = mbar_wait(&full_bar[stage], phase, ab, kErrSfFull);
+                ok = mbar_wait(Cfg::GPAIR ? &sf_full_bar[stage] : &full_bar[stage], phase, ab, kErrSfFull);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 uint8_t* sfpb = smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES;
@@ -1356,7 +1397,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sfready_bar[stage]);
+                if (lane == 0) {
+                    // GPAIR: the even CTA's MMA warp copies both CTAs' scales, each from the
+                    // shared memory of the CTA that wrote them
+                    if constexpr (Cfg::GPAIR) mbar_arrive_remote(mapa_shared(smem_u32(&sfready_bar[stage]), 0));
+                    else mbar_arrive(&sfready_bar[stage]);
+                }
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;

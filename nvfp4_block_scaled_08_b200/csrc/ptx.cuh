@@ -398,6 +398,42 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         : "memory");
 }
 
+// 5-D form of tma_load_2d_pair (the grouped gate_up weights in gate / up row groups).
+__device__ __forceinline__ void tma_load_5d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t c0, int32_t c1, int32_t c2, int32_t c3, int32_t c4,
+                                                 uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster),
+          "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "l"(policy)
+        : "memory");
+}
+
+// 3-D form of tma_load_2d_pair (the grouped weights [E][N][K/2]).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t x, int32_t y, int32_t z, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster),
+          "r"(x), "r"(y), "r"(z), "l"(policy)
+        : "memory");
+}
+
+// Arrive on the mbarrier at `bar_cluster` (from mapa, possibly another CTA's) with release at
+// CTA scope: this thread's earlier writes to its own CTA's shared memory (after
+// fence.proxy.async, for the tensor core's reads of it) are complete before the arrival. A
+// release at cluster scope waits for every earlier memory operation to be visible to the
+// whole cluster, outstanding global stores included: on B200 about 1 us per arrival while
+// other warps of the SM stream their output.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
 // Relaxed arrivals: they order no memory. For signals whose only content is "this thread's
 // tcgen05.ld reads have completed" (tcgen05.wait::ld, then tcgen05.fence::before_thread_sync):
 // the waiting side's tcgen05 writes are issued only after it observes the arrival. A release
