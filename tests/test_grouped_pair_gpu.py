@@ -132,3 +132,20 @@ def test_grouped_pair_swiglu_matches_single_cta(cuda_device, grouped_bn):
         res.append((hq[:rows].clone(), hsf[:rows].clone()))
     assert torch.equal(res[0][0], res[1][0]), "h codes differ with pairs"
     assert torch.equal(res[0][1], res[1][1]), "h scales differ with pairs"
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float16, torch.float32])
+def test_grouped_pair_output_dtypes(cuda_device, out_dtype):
+    """fp16 and fp32 outputs of the grouped pairs: the same bits as the single-CTA launch."""
+    d = cuda_device
+    counts = [140, 3, 0, 176, 99]
+    _, _, off, ops = _operands(d, counts, 384, 512, 130)
+    Aq, sfA, Bq, sfB, al, offd = ops
+    outs = []
+    for pair in (2, 1):
+        with nv.plan_override(grouped_bn=176, pair=pair):
+            outs.append(nv.grouped_gemm(Aq, sfA, Bq, sfB, al, offd, out_dtype=out_dtype))
+        st, code = nv.last_device_error()
+        assert st == 0, hex(code)
+    view = torch.int16 if out_dtype == torch.float16 else torch.int32
+    assert torch.equal(outs[0].view(view), outs[1].view(view))
