@@ -349,8 +349,10 @@ class DenseStep:
                                  sf=s["sf"], alpha_out=s["alpha"], stream=stream, tiled=True)
 
     def gemm(self, s, stream=None):
+        # the weights are quantised once, before any timing, and never rewritten: the GEMM may
+        # load its first stages of B before waiting for the kernel ahead of it (B_READY)
         self.nv.gemm(s["q"], s["sf"], s["Bq"], s["sfB"], s["alpha"], out=s["out"], workspace=s["ws"],
-                     stream=stream, tiled=True)
+                     stream=stream, tiled=True, b_ready=True)
 
     def step(self, s, stream=None):
         self.quant(s, stream)

@@ -229,6 +229,27 @@ nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t*
                             int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
                             nvfp4_sf_layout sf_layout, nvfp4_out_dtype out_dtype, cudaStream_t stream);
 
+/* Flags of nvfp4_gemm_ex3. */
+enum { NVFP4_GEMM_B_READY = 1 };
+
+/*
+ * nvfp4_gemm_ex2 with flags (nvfp4_gemm_ex2 is this call with flags = 0); other bits:
+ * NVFP4_ERR_INVALID_ARG. Same operation, output bits, checks and split-K rules.
+ *   NVFP4_GEMM_B_READY: the caller guarantees that B and sfB are not written by any kernel
+ *     that may still be running when this call's kernel starts (for example weights quantised
+ *     earlier and not rewritten since). The kernel is launched early behind the previous
+ *     kernel in the stream (programmatic dependent launch); with this flag it also loads its
+ *     first K stages of B into shared memory before waiting for that kernel, instead of only
+ *     requesting them into L2. Applies to NVFP4_SF_TILED launches on one CTA per tile (few-token
+ *     and mid-size products); the others ignore it. Without the guarantee the result may read
+ *     stale B.
+ */
+nvfp4_status nvfp4_gemm_ex3(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                            const uint8_t* sfB, const float* alpha, void* out,
+                            int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
+                            nvfp4_sf_layout sf_layout, nvfp4_out_dtype out_dtype, uint32_t flags,
+                            cudaStream_t stream);
+
 /*
  * MXFP4: the mm_fp4 variant that use_nvfp4=False selects ("The Art of Reading the Manual",
  * section "The Message"; the pages name it without defining it). The library's reading is

@@ -73,6 +73,8 @@ SIGNATURES = {
     "nvfp4_gemm_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int, _P]),
     "nvfp4_gemm_ex2": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int,
                                       ctypes.c_int, _P]),
+    "nvfp4_gemm_ex3": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_uint32, _P]),
     "nvfp4_grouped_gemm_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P,
                                              ctypes.c_int, _P]),
     "nvfp4_grouped_gemm_swiglu": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
@@ -280,22 +282,25 @@ def _out_code(out: torch.Tensor) -> int:
 
 
 def gemm(Aq, sfA, Bq, sfB, alpha_t, out=None, workspace=None, stream=None, tiled=False,
-         out_dtype=torch.bfloat16, layout: int | None = None) -> torch.Tensor:
+         out_dtype=torch.bfloat16, layout: int | None = None, b_ready: bool = False) -> torch.Tensor:
     """out[M, N] = alpha * sum_k deq(A)[m,k] deq(B)[n,k] in bf16, fp16 or fp32.
 
     Aq [M, K/2] uint8, sfA [M, K/16] uint8, Bq [N, K/2], sfB [N, K/16], alpha_t fp32 [1];
     out [M, N] (allocated with out_dtype if None; otherwise its dtype decides); workspace:
     zero-filled uint8 tensor of gemm_workspace_size(M, N, K) bytes or None (no split-K).
     tiled: sfA and sfB in the tiled layout (flat uint8 tensors from sf_tile or
-    quantize_dynamic(tiled=True)); layout: any SF_* layout of both (overrides tiled)."""
+    quantize_dynamic(tiled=True)); layout: any SF_* layout of both (overrides tiled).
+    b_ready: NVFP4_GEMM_B_READY, a promise that no kernel that may still run writes Bq / sfB
+    (weights quantised earlier): the kernel then loads its first stages of B before waiting
+    for the previous kernel in the stream."""
     M, K = Aq.shape[0], Aq.shape[1] * 2
     N = Bq.shape[0]
     if out is None:
         out = torch.empty(M, N, dtype=out_dtype, device=Aq.device)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
-    _check("nvfp4_gemm_ex2", load().nvfp4_gemm_ex2(
+    _check("nvfp4_gemm_ex3", load().nvfp4_gemm_ex3(
         _ptr(Aq), _ptr(sfA), _ptr(Bq), _ptr(sfB), _ptr(alpha_t), _ptr(out), M, N, K,
-        ws_ptr, ws_bytes, _layout(tiled, layout), _out_code(out), _stream(stream)))
+        ws_ptr, ws_bytes, _layout(tiled, layout), _out_code(out), 1 if b_ready else 0, _stream(stream)))
     return out
 
 

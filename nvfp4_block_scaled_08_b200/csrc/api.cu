@@ -287,12 +287,13 @@ size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K)
     return nvfp4::plan_gemm(M, N, K, true, d.num_sms).ws_bytes;
 }
 
-nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+nvfp4_status nvfp4_gemm_ex3(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                             const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
                             size_t ws_bytes, nvfp4_sf_layout sf_layout, nvfp4_out_dtype out_dtype,
-                            cudaStream_t stream)
+                            uint32_t flags, cudaStream_t stream)
 {
     if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARG;
+    if ((flags & ~static_cast<uint32_t>(NVFP4_GEMM_B_READY)) != 0) return NVFP4_ERR_INVALID_ARG;
     if (sf_layout != NVFP4_SF_LINEAR && sf_layout != NVFP4_SF_TILED && sf_layout != NVFP4_SF_8X4)
         return NVFP4_ERR_INVALID_ARG;
     if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F16 && out_dtype != NVFP4_OUT_F32)
@@ -314,10 +315,19 @@ nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t*
     nvfp4::GemmLaunch L{A, sfA, B, sfB, alpha, out, M, N, K, nullptr, 0, 0, ws, d.err_word, tiled,
                         static_cast<int32_t>(out_dtype)};
     L.sf_8x4 = sf_layout == NVFP4_SF_8X4;
+    L.b_ready = (flags & NVFP4_GEMM_B_READY) != 0;
     bool enc_failed = false;
     cudaError_t e = nvfp4::launch_gemm(plan, L, stream, &enc_failed);
     if (enc_failed) return NVFP4_ERR_CUDA;
     return from_cuda(e);
+}
+
+nvfp4_status nvfp4_gemm_ex2(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                            const float* alpha, void* out, int64_t M, int64_t N, int64_t K, void* ws,
+                            size_t ws_bytes, nvfp4_sf_layout sf_layout, nvfp4_out_dtype out_dtype,
+                            cudaStream_t stream)
+{
+    return nvfp4_gemm_ex3(A, sfA, B, sfB, alpha, out, M, N, K, ws, ws_bytes, sf_layout, out_dtype, 0u, stream);
 }
 
 nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_in_dtype dtype, int64_t rows, int64_t K, int64_t ld_x,

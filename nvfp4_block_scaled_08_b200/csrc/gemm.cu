@@ -355,6 +355,7 @@ static cudaError_t run(const GemmPlan& plan, const GemmLaunch& L, cudaStream_t s
     a.out_dtype = L.out_dtype;
     a.alpha = L.alpha;
     a.err_word = L.err_word;
+    a.b_ready = L.b_ready ? 1 : 0;
     if constexpr (GROUPED) {
         const uint64_t E = static_cast<uint64_t>(L.E);
         const uint64_t rows = static_cast<uint64_t>(L.total_rows);

@@ -87,6 +87,7 @@ struct GemmArgs {
     const uint8_t* sf_q;
     int32_t sf_kb4;           // SFT: 512-byte scale blocks per 128-row tile (K / 64)
     int32_t sf_8x4;           // linear-path scales in the 8 x 4 layout (1) or row-major (0)
+    int32_t b_ready;          // B and its scales are not written by a kernel that may still run
     const int32_t* expert_offsets;  // grouped: [E + 1]
     int32_t num_experts;
     int32_t total_rows;       // grouped: rows of A / out
@@ -936,6 +937,52 @@ __device__ __forceinline__ void split_k_epilogue(const GemmArgs& a, const Tile& 
     if (row == 0) *counter = 0u;             // re-arm for the next call
 }
 
+// Copies of one stage of a dense tiled-scale tile (SFT, single CTA) into ring slot `stage`,
+// all completing on that slot's full barrier: part 1 = the weight operand (B: Q, or P when the
+// weights are the MMA M operand) and its scales, after arming the barrier for the whole
+// stage; part 2 = the activation operand (A) and its scales; part 3 = both. The stage's scale
+// blocks of each 128-row tile are one contiguous run (2 KB, MX 1 KB); only the Q row tiles that
+// exist are fetched (the last Q tile may end past the rows). ACTQ: the weights only (the
+// epilogue warps fill the Q stages).
+template <class Cfg>
+__device__ __forceinline__ void sft_stage_copies(const GemmArgs& a, const Tile& ti, int32_t ks, uint32_t stage,
+                                                 uint8_t* smem, const CUtensorMap* tm_p, const CUtensorMap* tm_q,
+                                                 uint64_t* full_bar, int part)
+{
+    constexpr int QG = Cfg::QG;
+    const uint64_t pol_stream = l2_policy_evict_first();  // weights: read once
+    const uint64_t pol_keep = l2_policy_evict_last();     // activations: re-read
+    const uint64_t pol_p = Cfg::SWAP ? pol_stream : pol_keep;
+    const uint64_t pol_q = Cfg::SWAP ? pol_keep : pol_stream;
+    uint64_t* fb = &full_bar[stage];
+    const int32_t kx = (ti.k0 + ks) * Cfg::BK_BYTES;
+    uint8_t* pbuf = smem + Cfg::OFF_P + stage * Cfg::P_BYTES;
+    uint8_t* qbuf = smem + Cfg::OFF_Q + stage * Cfg::Q_BYTES;
+    uint8_t* sfpb = smem + Cfg::OFF_SFP + stage * Cfg::SFP_BYTES;
+    uint8_t* sfqb = smem + Cfg::OFF_SFQ + stage * Cfg::SFQ_BYTES;
+    const int64_t kb = Cfg::SF_BLOCKS * static_cast<int64_t>(ti.k0 + ks);
+    const int ng = Cfg::ACTQ ? 0 : min(QG, (a.q_rows - ti.q0 + 127) >> 7);
+    const bool weights = (part & 1) != 0, acts = (part & 2) != 0;
+    const bool do_p = Cfg::SWAP ? weights : acts;          // P is the weights when swapped
+    const bool do_q = !Cfg::ACTQ && (Cfg::SWAP ? acts : weights);
+    if (weights) {
+        const uint32_t q_bytes = Cfg::ACTQ ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES + Cfg::SFP_BYTES * ng);
+        mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::SFP_BYTES + q_bytes);
+    }
+    if (do_p) {
+        tma_load_2d(pbuf, tm_p, fb, kx, ti.p0, pol_p);
+        bulk_load(sfpb, a.sf_p + ((ti.p0 >> 7) * static_cast<int64_t>(a.sf_kb4) + kb) * 512, Cfg::SFP_BYTES, fb,
+                  pol_p);
+    }
+    if (do_q) {
+        tma_load_2d(qbuf, tm_q, fb, kx, ti.q0, pol_q);
+        for (int g = 0; g < ng; ++g)
+            bulk_load(sfqb + Cfg::SFP_BYTES * g,
+                      a.sf_q + (((ti.q0 >> 7) + g) * static_cast<int64_t>(a.sf_kb4) + kb) * 512, Cfg::SFP_BYTES,
+                      fb, pol_q);
+    }
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
@@ -1079,10 +1126,26 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         const uint64_t pol_keep = l2_policy_evict_last();     // activations: re-read
         const uint64_t pol_p = Cfg::SWAP ? pol_stream : pol_keep;
         const uint64_t pol_q = Cfg::SWAP ? pol_keep : pol_stream;
+        // The first tile's stages whose weight tiles (and scales) were requested before the
+        // wait for the previous kernel in the stream (b_ready: the caller guarantees that no
+        // kernel that may still run writes B); their full barriers are armed for the whole
+        // stage, and the activations follow after the wait.
+        int32_t early = 0;
+        if constexpr (Cfg::SFT && !Cfg::PAIR && !Cfg::GROUPED) {
+            if (args.b_ready && tile_start < num_tiles) {
+                const Tile ti = decode_tile<Cfg>(args, tile_start, s_prefix);
+                early = ti.kcnt < STAGES ? ti.kcnt : STAGES;
+                if (elect_one()) {
+                    for (int32_t ks = 0; ks < early; ++ks) sft_stage_copies<Cfg>(args, ti, ks, ks, smem, &tm_p, &tm_q,
+                                                                                 full_bar, 1);
+                }
+                __syncwarp();
+            }
+        }
         if constexpr (!Cfg::GROUPED) {
             // Warm L2 with this CTA's first weight tiles while the previous kernel finishes
             // (a prefetch only fills L2, the coherence point, so it cannot see stale data).
-            if (tile_start < num_tiles && elect_one()) {
+            if (early == 0 && tile_start < num_tiles && elect_one()) {
                 const Tile ti = decode_tile<Cfg>(args, tile_start, s_prefix);
                 const int n = ti.kcnt < STAGES ? ti.kcnt : STAGES;
                 for (int ks = 0; ks < n; ++ks) {
@@ -1183,29 +1246,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
                             if (g == 0 || !narrow)
                                 tma_load_2d_pair(sfqb + Cfg::SFP_BYTES * g, &tm_sfq, fb0, 0,
                                                  (((ti.q0 >> 7) + g) * kb4 + kb) * 2, pol_q);
-                    } else if constexpr (Cfg::ACTQ) {
-                        // weights and their scales only: the epilogue warps fill the Q stages
-                        mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::SFP_BYTES);
-                        tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
-                        const int64_t kb = Cfg::SF_BLOCKS * static_cast<int64_t>(ti.k0 + ks);
-                        bulk_load(sfpb, args.sf_p + ((ti.p0 >> 7) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
-                                  Cfg::SFP_BYTES, fb, pol_p);
                     } else if constexpr (Cfg::SFT) {
-                        // the stage's scale blocks of each 128-row tile: one contiguous run (2 KB,
-                        // MX 1 KB); only the Q row tiles that exist (the last Q tile may end past
-                        // the rows)
-                        const int ng = min(QG, (args.q_rows - ti.q0 + 127) >> 7);
-                        mbar_arrive_expect_tx(fb, Cfg::P_BYTES + Cfg::Q_BYTES + Cfg::SFP_BYTES +
-                                                  static_cast<uint32_t>(Cfg::SFP_BYTES * ng));
-                        tma_load_2d(pbuf, &tm_p, fb, kx, ti.p0, pol_p);
-                        tma_load_2d(qbuf, &tm_q, fb, kx, ti.q0, pol_q);
-                        const int64_t kb = Cfg::SF_BLOCKS * static_cast<int64_t>(ti.k0 + ks);
-                        bulk_load(sfpb, args.sf_p + ((ti.p0 >> 7) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
-                                  Cfg::SFP_BYTES, fb, pol_p);
-                        for (int g = 0; g < ng; ++g)
-                            bulk_load(sfqb + Cfg::SFP_BYTES * g,
-                                      args.sf_q + (((ti.q0 >> 7) + g) * static_cast<int64_t>(args.sf_kb4) + kb) * 512,
-                                      Cfg::SFP_BYTES, fb, pol_q);
+                        // (the first tile's `early` stages: their weight copies are in flight)
+                        const bool first = t == tile_start && ks < early;
+                        sft_stage_copies<Cfg>(args, ti, ks, stage, smem, &tm_p, &tm_q, full_bar, first ? 2 : 3);
                     } else {
                         // row-major scales: [rows][16 B] per stage; 8 x 4 scales: the scale map's
                         // rows are 8-row groups, a stage's 4 blocks of one group 128 contiguous

@@ -101,6 +101,8 @@ struct GemmLaunch {
     float* gs_out = nullptr;
     float* alpha_out = nullptr;
     bool sf_8x4 = false;        // sfA and sfB in the 8 x 4 layout (dense NVFP4 GEMM only)
+    bool b_ready = false;       // NVFP4_GEMM_B_READY: B's first stages may load before the
+                                // wait for the previous kernel in the stream
 };
 
 // api.cu: nvfp4_status of the current device's checks; fills the SM count and the device

@@ -95,6 +95,14 @@ def test_out_dtype_host_validation(lib):
     assert gg(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x8000, 256, 4096, 4096, 6000, 0x6000, 1, None) == 2
 
 
+def test_gemm_flags_host_validation(lib):
+    g = lib.nvfp4_gemm_ex3
+    base = (0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 16, 768, 6144, None, 0, 1, 0)
+    assert g(*base, 2, None) == 1                    # unknown flag bit
+    assert g(*base, 0x80000000, None) == 1
+    assert g(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 16, 768, 6000, None, 0, 1, 0, 1, None) == 2
+
+
 def test_mx_host_validation(lib):
     q = lib.nvfp4_mx_quantize
     assert q(0x1000, 0, 0, 512, 512, 0x2000, 0x3000, 0, None) == 0             # no rows
