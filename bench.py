@@ -114,9 +114,9 @@ def whole_job_value(flops_per_rank: float, step_ms_max: float, world: int) -> fl
 # dram__bytes_write.sum from one ncu capture of the full-size launch (one pass); the command
 # and the figures are in the committed ncu summary of the plateau under profiles/. Valid only
 # for the kernel sources it was taken on (hash below); reported as null otherwise.
-GEMM_TRAFFIC_BYTES = 2222823680 + 511686144
+GEMM_TRAFFIC_BYTES = 2301937152 + 509914624
 GEMM_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "gemm.cu", "ptx.cuh", "internal.h", "quant_core.cuh")
-GEMM_TRAFFIC_SHA = "7fdcea98290d783c"
+GEMM_TRAFFIC_SHA = "e000b73d3155a97d"
 
 
 def _code_hash(files) -> str:
