@@ -1270,7 +1270,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constan
         }
         // Let every copy still in flight land before shared memory can be released (the odd
         // CTA of a pair cannot wait on the even CTA's full barrier: it waits until the MMAs
-        // that read each stage have released it).
+        // that read each stage have released it). The `early` weight copies of the first tile
+        // are among the issued stages once the loop has reached them; the loop can stop before
+        // that only after some role waited 1 s in vain, long after those copies landed.
         const bool on_empty = Cfg::PAIR && cluster_ctarank() != 0;
         const uint32_t inflight = issued < (uint32_t)STAGES ? issued : (uint32_t)STAGES;
         for (uint32_t i = 1; i <= inflight; ++i) {
