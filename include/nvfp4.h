@@ -446,7 +446,7 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* A, const uint8_t* sfA, const uint
  *   band        output P tiles per rasterisation band;
  *   grouped_bn  token tile width of the grouped GEMM: 32, 64, 128, 176 or 256;
  *   pair        CTA pairs computing 256-row tiles with the 2-SM MMA (tiled scales, no split-K):
- *               0 = the planner (pairs for 256-wide tiles with K >= 3072; a last round of
+ *               0 = the planner (pairs for 256-wide tiles with K >= 3072; a last wave of
  *               256 x 256 tiles that fills at most half of the pairs runs as 256 x 128
  *               halves), 1 = never, 2 = for every 256- or 128-wide tile, 3 = as 0 but
  *               without the halves; the grouped GEMM runs pairs for 128- and 176-row token

@@ -135,7 +135,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool allow_workspace, int nu
         const int clusters = std::max(1, std::min(pairs, max_active_clusters(2)));
         p.pair_grid = 2 * clusters;
         p.pair_band = std::max(1, p.band / 2);
-        // A last round of 256 x 256 tiles that fills at most half of the pairs runs as twice
+        // A last wave of 256 x 256 tiles that fills at most half of the pairs runs as twice
         // as many 256 x 128 halves, in about half the time (4096^3: 256 tiles on 74 pairs,
         // 3.46 rounds).
         const int tail = pairs % clusters;

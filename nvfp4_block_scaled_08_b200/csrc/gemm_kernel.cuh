@@ -296,7 +296,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, int32_t t, const 
         ti.expert = e;
     } else {
         // PAIR, BN = 256: items from narrow_from on split the last output tiles in two halves
-        // of 128 columns each (a last round of tiles shorter than a full one fills twice as
+        // of 128 columns each (a last wave of tiles shorter than a full one fills twice as
         // many SMs for half as long): item narrow_from + 2 j + h is half h of tile narrow_from + j.
         int32_t half = -1;
         if constexpr (Cfg::NARROW) {

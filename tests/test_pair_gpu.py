@@ -91,7 +91,7 @@ def test_pairs_on_the_plateau(cuda_device):
 
 @pytest.mark.parametrize("M,N,K", [(2500, 2056, 1024), (4096, 4096, 3072)])
 def test_pair_half_tiles(cuda_device, M, N, K):
-    """A last round of 256 x 256 pair tiles that fills at most half of the pairs runs as
+    """A last wave of 256 x 256 pair tiles that fills at most half of the pairs runs as
     256 x 128 halves. On 148 SMs (74 pairs): 2500 x 2056 has 10 x 9 = 90 tiles, the last 16
     split in halves, the last Q tile 8 columns wide (its second half starts past N) and the
     last P tile 68 rows; 4096 x 4096 has 256 tiles, the last 34 split. Same bits as the
