@@ -133,3 +133,23 @@ def test_pair_half_tiles_mx(cuda_device):
     qb_o, sb_o = oracle.mx_quantize(b.numpy())
     v, S, _ = oracle.mx_gemm(qa_o, sa_o, qb_o, sb_o, 1.0)
     check_within_tolerance(outs[0][torch.as_tensor(rows, device=d)], v, S, 1.0, f"mx half tiles {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float16, torch.float32])
+def test_pair_half_tiles_output_dtypes(cuda_device, out_dtype):
+    """fp16 and fp32 outputs of pair tiles and of the half tiles of a short last wave
+    (4096 x 4096 x 3072: 256 pair tiles on 74 pairs, the last 34 split): the same bits as
+    single-CTA tiles."""
+    d = cuda_device
+    M, N, K = 4096, 4096, 3072
+    a = workloads.normal(M, K, 1.0, 41)
+    b = workloads.normal(N, K, 0.02, 43)
+    Aq, sA, Bq, sB, al = _operands(d, a, b)
+    outs = []
+    for pair in (0, 1):
+        with nv.plan_override(pair=pair):
+            outs.append(nv.gemm(Aq, sA, Bq, sB, al, tiled=True, out_dtype=out_dtype))
+        st, code = nv.last_device_error()
+        assert st == 0, hex(code)
+    view = torch.int16 if out_dtype == torch.float16 else torch.int32
+    assert torch.equal(outs[0].view(view), outs[1].view(view))
